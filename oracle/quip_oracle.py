@@ -1,0 +1,419 @@
+"""Plain FP64 oracle of the QuIP pipeline for one linear layer.
+
+TEST INFRASTRUCTURE: imported only by tests/, __graft_entry__.smoke() and the
+CPU legs of bench.py.  Nothing here is on the product path.
+
+Sources (page title, then the section / equation each step follows):
+
+[QuIP]  "QuIP: 2-Bit Quantization of Large Language Models With Guarantees"
+        (Chee, Cai, Kuleshov, De Sa; arXiv 2307.13304), HTML body.
+          - Introduction: proxy objective l(W^) = tr((W^ - W) H (W^ - W)^T)
+            and the Kronecker product of random orthogonal matrices.
+          - Adaptive-rounding section (Eq. (1), display lost in the page):
+            H is the second moment of the calibration inputs; rows of W are
+            independent ("run in parallel across neurons").
+          - "OPTQ (Formerly known as GPTQ)." paragraph: nearest rounding,
+            scaled error update of the remaining columns, repeat.
+          - Incoherence-processing section: H~ <- V H V^T, W~ <- U W V^T and
+            the trace identity tr(W~ H~ W~^T) = tr(W H W^T).
+          - Experiments, "Methods.": damping H <- H + alpha*mean(diag(H)) I;
+            nearest rounding and LDLQ as rounding methods; LDLQ = OPTQ.
+[QuIP#] "QuIP#: Even Better LLM Quantization with Hadamard Incoherence and
+        Lattice Codebooks" (arXiv 2402.04396), abstract: incoherence by the
+        randomized Hadamard transform.
+
+The LDLQ display and its LDL factorisation were lost from the QuIP page; the
+reading used here (and by the CUDA path) is the one the rest of the text
+supports: H = (I + U)(D)(I + U)^T with U strictly upper triangular, and
+W^_k = Q(W_k + (W - W^) U_k), column k using only columns j < k.
+
+Readings where the pages are silent (each one is listed in the design doc):
+  * grid: per-row asymmetric min/max grid of 2^b levels over the whole
+    incoherent row, fixed before rounding; s = (hi - lo) / (2^b - 1); a
+    constant row uses s = 1;
+  * Q: round half to even (numpy.rint), then clamp to [0, 2^b - 1];
+  * Hadamard: Sylvester order, V = H_n diag(s) / sqrt(n), s_i = +-1;
+  * Kronecker: V = A (x) B with A, B Haar-distributed (QR of a Gaussian
+    matrix with the sign of diag(R) folded into Q);
+  * the random signs and Gaussians come from SplitMix64, counter-based (see
+    ``splitmix64``); the CUDA library implements the same published
+    generator independently.
+
+Pinned by tests/test_oracle_*.py (CPU).  Functions with no pin: none.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+from typing import Optional, Tuple
+
+import numpy as np
+
+__all__ = [
+    "hessian", "damp", "splitmix64", "uniform53", "random_signs", "gaussian_matrix",
+    "haar_orthogonal", "sylvester_hadamard", "hadamard_row", "SideTransform", "make_side",
+    "incoherence_forward", "incoherence_inverse", "udu", "row_grid", "quantize",
+    "ldlq", "ldlq_blocked", "nearest", "optq", "dequantize", "proxy_loss", "Pipeline",
+    "run_pipeline", "STREAM_M_SIGNS", "STREAM_N_SIGNS", "STREAM_M_A", "STREAM_M_B",
+    "STREAM_N_A", "STREAM_N_B",
+]
+
+# ----------------------------------------------------------------------------
+# O1/O2  Proxy Hessian and damping
+# ----------------------------------------------------------------------------
+
+
+def hessian(X: np.ndarray) -> np.ndarray:
+    """H = X^T X / N: second moment of the calibration inputs x in R^n.
+
+    [QuIP] adaptive-rounding section: "H is the second moment matrix of these
+    vectors, interpreted as a proxy Hessian".  X is N x n (one token per row).
+    """
+    X = np.asarray(X, dtype=np.float64)
+    return X.T @ X / X.shape[0]
+
+
+def damp(H: np.ndarray, alpha: float) -> np.ndarray:
+    """H + alpha * mean(diag(H)) * I  ([QuIP] Experiments, "Methods.")."""
+    H = np.array(H, dtype=np.float64, copy=True)
+    mu = float(np.mean(np.diag(H)))
+    H[np.diag_indices_from(H)] += alpha * mu
+    return H
+
+
+# ----------------------------------------------------------------------------
+# O3  Random orthogonal transforms
+# ----------------------------------------------------------------------------
+#
+# Counter-based SplitMix64 (Steele, Lea & Flood, "Fast splittable pseudorandom
+# number generators", OOPSLA 2014): the k-th output (k >= 1) from seed s is
+# mix(s + k * gamma) with gamma = 0x9E3779B97F4A7C15 and mix the published
+# 64-bit finaliser below.  Stream t, element i uses k = t * 2^40 + i + 1.
+
+_GAMMA = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+
+STREAM_M_SIGNS, STREAM_N_SIGNS = 0, 1
+STREAM_M_A, STREAM_M_B, STREAM_N_A, STREAM_N_B = 2, 3, 4, 5
+
+
+def splitmix64(seed: int, stream: int, index: np.ndarray) -> np.ndarray:
+    """uint64 outputs of SplitMix64 for the given stream and element indices."""
+    idx = np.asarray(index, dtype=np.uint64)
+    k = np.uint64(stream) * np.uint64(1 << 40) + idx + np.uint64(1)
+    with np.errstate(over="ignore"):
+        z = np.uint64(seed & 0xFFFFFFFFFFFFFFFF) + k * _GAMMA
+        z = (z ^ (z >> np.uint64(30))) * _M1
+        z = (z ^ (z >> np.uint64(27))) * _M2
+        z = z ^ (z >> np.uint64(31))
+    return z
+
+
+def uniform53(r: np.ndarray) -> np.ndarray:
+    """Map uint64 to (0, 1]: ((r >> 11) + 1) * 2^-53."""
+    return ((r >> np.uint64(11)).astype(np.float64) + 1.0) * (2.0 ** -53)
+
+
+def random_signs(seed: int, stream: int, n: int) -> np.ndarray:
+    """s_i = -1 if the top bit of the i-th draw is set, else +1."""
+    r = splitmix64(seed, stream, np.arange(n, dtype=np.uint64))
+    return np.where((r >> np.uint64(63)) == np.uint64(1), -1.0, 1.0)
+
+
+def gaussian_matrix(seed: int, stream: int, p: int) -> np.ndarray:
+    """p x p i.i.d. N(0,1), row-major element e from draws 2e and 2e+1 by
+    Box-Muller: sqrt(-2 ln u1) * cos(2 pi u2)."""
+    e = np.arange(p * p, dtype=np.uint64)
+    u1 = uniform53(splitmix64(seed, stream, 2 * e))
+    u2 = uniform53(splitmix64(seed, stream, 2 * e + np.uint64(1)))
+    g = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * math.pi * u2)
+    return g.reshape(p, p)
+
+
+def haar_orthogonal(G: np.ndarray) -> np.ndarray:
+    """Q of G = QR with diag(R) > 0, i.e. Q <- Q diag(sign(diag R)).
+
+    This is the standard way to draw a uniformly (Haar) distributed orthogonal
+    matrix; [QuIP] Introduction asks for "random orthogonal matrices".
+    """
+    Q, R = np.linalg.qr(np.asarray(G, dtype=np.float64))
+    d = np.sign(np.diag(R))
+    d[d == 0] = 1.0
+    return Q * d[None, :]
+
+
+def sylvester_hadamard(n: int) -> np.ndarray:
+    """H_1 = [1], H_2k = [[H_k, H_k], [H_k, -H_k]] (Sylvester, natural order)."""
+    if n < 1 or n & (n - 1):
+        raise ValueError("Hadamard order must be a power of two")
+    H = np.ones((1, 1))
+    while H.shape[0] < n:
+        H = np.block([[H, H], [H, -H]])
+    return H
+
+
+def hadamard_row(n: int, i: int) -> np.ndarray:
+    """Row i of the Sylvester H_n without forming it: (-1)^popcount(i & j)."""
+    j = np.arange(n, dtype=np.int64)
+    x = j & i
+    par = np.zeros(n, dtype=np.int64)
+    while np.any(x):
+        par ^= x & 1
+        x >>= 1
+    return 1.0 - 2.0 * par
+
+
+@dataclass
+class SideTransform:
+    """One random orthogonal matrix S (m-side U or n-side V).
+
+    kind 'hadamard': S = H_d diag(s) / sqrt(d)          ([QuIP#] abstract)
+    kind 'kronecker': S = A (x) B, A p x p, B q x q     ([QuIP] Introduction)
+    kind 'identity':  S = I
+    """
+    kind: str
+    dim: int
+    signs: Optional[np.ndarray] = None
+    A: Optional[np.ndarray] = None
+    B: Optional[np.ndarray] = None
+
+    def matrix(self) -> np.ndarray:
+        d = self.dim
+        if self.kind == "identity":
+            return np.eye(d)
+        if self.kind == "hadamard":
+            return sylvester_hadamard(d) * self.signs[None, :] / math.sqrt(d)
+        return np.kron(self.A, self.B)
+
+    def row(self, i: int) -> np.ndarray:
+        d = self.dim
+        if self.kind == "identity":
+            r = np.zeros(d)
+            r[i] = 1.0
+            return r
+        if self.kind == "hadamard":
+            return hadamard_row(d, i) * self.signs / math.sqrt(d)
+        q = self.B.shape[0]
+        return np.kron(self.A[i // q], self.B[i % q])
+
+
+def make_side(seed: int, side: str, kind: str, dim: int, p: int = 0, q: int = 0) -> SideTransform:
+    """Draw the transform for side 'm' (rows of W) or 'n' (columns of W)."""
+    if kind == "identity":
+        return SideTransform("identity", dim)
+    if kind == "hadamard":
+        st = STREAM_M_SIGNS if side == "m" else STREAM_N_SIGNS
+        return SideTransform("hadamard", dim, signs=random_signs(seed, st, dim))
+    if kind == "kronecker":
+        if p * q != dim:
+            raise ValueError("Kronecker factors must multiply to the dimension")
+        sa, sb = (STREAM_M_A, STREAM_M_B) if side == "m" else (STREAM_N_A, STREAM_N_B)
+        A = haar_orthogonal(gaussian_matrix(seed, sa, p))
+        B = haar_orthogonal(gaussian_matrix(seed, sb, q))
+        return SideTransform("kronecker", dim, A=A, B=B)
+    raise ValueError(kind)
+
+
+def incoherence_forward(W: np.ndarray, H: np.ndarray, U: SideTransform, V: SideTransform
+                        ) -> Tuple[np.ndarray, np.ndarray]:
+    """W~ = U W V^T and H~ = V H V^T (symmetrised).
+
+    [QuIP] incoherence-processing section ("random orthogonal
+    multiplications H~ <- V H V^T and W~ <- U W V^T").
+    """
+    Um, Vn = U.matrix(), V.matrix()
+    Wt = Um @ np.asarray(W, dtype=np.float64) @ Vn.T
+    Ht = Vn @ np.asarray(H, dtype=np.float64) @ Vn.T
+    return Wt, 0.5 * (Ht + Ht.T)
+
+
+def incoherence_inverse(Wt_hat: np.ndarray, U: SideTransform, V: SideTransform) -> np.ndarray:
+    """W^ = U^T W~^ V: undo the transforms (QuIP post-processing)."""
+    return U.matrix().T @ np.asarray(Wt_hat, dtype=np.float64) @ V.matrix()
+
+
+# ----------------------------------------------------------------------------
+# O4  LDL factorisation H = (I + U) D (I + U)^T, U strictly upper
+# ----------------------------------------------------------------------------
+
+
+def udu(H: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Return (U, D) with H = (I + U) diag(D) (I + U)^T, U strictly upper.
+
+    The factor is unique for positive-definite H.  Written via the Cholesky
+    factorisation of the index-reversed matrix J H J = L L^T (a library
+    routine): R = J L J is upper triangular with H = R R^T, so D_k = R_kk^2
+    and I + U = R diag(R)^-1.
+    """
+    H = np.asarray(H, dtype=np.float64)
+    n = H.shape[0]
+    if n == 0:
+        return np.zeros((0, 0)), np.zeros(0)
+    J = np.arange(n)[::-1]
+    L = np.linalg.cholesky(H[np.ix_(J, J)])   # raises LinAlgError if not PD
+    R = L[np.ix_(J, J)]
+    d = np.diag(R).copy()
+    Ufull = R / d[None, :]
+    return np.triu(Ufull, 1), d * d
+
+
+# ----------------------------------------------------------------------------
+# O5/O6  Grid, rounding, LDLQ
+# ----------------------------------------------------------------------------
+
+
+def row_grid(Wt: np.ndarray, bits: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Per-row asymmetric 2^b-level grid: lo = min, s = (max - min)/(2^b - 1).
+
+    A constant row (max == min) gets s = 1 so every code is 0.
+    """
+    Wt = np.asarray(Wt, dtype=np.float64)
+    lo = Wt.min(axis=1)
+    hi = Wt.max(axis=1)
+    s = (hi - lo) / (2 ** bits - 1)
+    s = np.where(hi > lo, s, 1.0)
+    return lo, s
+
+
+def quantize(a: np.ndarray, lo: np.ndarray, s: np.ndarray, bits: int) -> np.ndarray:
+    """Q(a): nearest grid level, ties to even, clamped to [0, 2^b - 1]."""
+    return np.clip(np.rint((a - lo) / s), 0, 2 ** bits - 1)
+
+
+def ldlq(Wt: np.ndarray, U: np.ndarray, lo: np.ndarray, s: np.ndarray, bits: int
+         ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """LDLQ, unblocked: for k = 0..n-1
+         a_k  = W_k + sum_{j<k} (W_j - W^_j) U_jk
+         c_k  = Q(a_k),   W^_k = lo + s c_k,   eta_k = W^_k - a_k.
+
+    [QuIP] adaptive-rounding section (LDLQ; feedback matrix from the LDL
+    factorisation of H).  Returns integer codes (m x n, int64), W^ and eta.
+    Rows are independent.
+    """
+    Wt = np.asarray(Wt, dtype=np.float64)
+    U = np.asarray(U, dtype=np.float64)
+    m, n = Wt.shape
+    codes = np.zeros((m, n), dtype=np.int64)
+    What = np.zeros((m, n))
+    eta = np.zeros((m, n))
+    errT = np.zeros((n, m))                 # (W - W^)^T, filled column by column
+    for k in range(n):
+        a = Wt[:, k] + U[:k, k] @ errT[:k]
+        c = quantize(a, lo, s, bits)
+        codes[:, k] = c
+        What[:, k] = lo + s * c
+        eta[:, k] = What[:, k] - a
+        errT[k] = Wt[:, k] - What[:, k]
+    return codes, What, eta
+
+
+def ldlq_blocked(Wt: np.ndarray, U: np.ndarray, lo: np.ndarray, s: np.ndarray, bits: int,
+                 block: int) -> Tuple[np.ndarray, np.ndarray]:
+    """LDLQ with the column sum split at block boundaries (lazy batch).
+
+    Inside a block of ``block`` columns the feedback is applied column by
+    column; when the block ends, every later column receives the block's
+    error times the matching rows of U at once.  Same a_k as ``ldlq`` up to
+    the order of additions.
+    """
+    Wt = np.asarray(Wt, dtype=np.float64)
+    m, n = Wt.shape
+    A = Wt.copy()
+    codes = np.zeros((m, n), dtype=np.int64)
+    What = np.zeros((m, n))
+    for k0 in range(0, n, block):
+        k1 = min(n, k0 + block)
+        for k in range(k0, k1):
+            c = quantize(A[:, k], lo, s, bits)
+            codes[:, k] = c
+            What[:, k] = lo + s * c
+            A[:, k + 1:k1] += np.outer(Wt[:, k] - What[:, k], U[k, k + 1:k1])
+        A[:, k1:] += (Wt[:, k0:k1] - What[:, k0:k1]) @ U[k0:k1, k1:]
+    return codes, What
+
+
+def nearest(Wt: np.ndarray, lo: np.ndarray, s: np.ndarray, bits: int) -> np.ndarray:
+    """Nearest rounding ([QuIP] Experiments, "Methods."); lo, s are per row."""
+    lo = np.asarray(lo, dtype=np.float64)[:, None]
+    s = np.asarray(s, dtype=np.float64)[:, None]
+    return quantize(np.asarray(Wt, dtype=np.float64), lo, s, bits).astype(np.int64)
+
+
+def optq(Wt: np.ndarray, H: np.ndarray, lo: np.ndarray, s: np.ndarray, bits: int) -> np.ndarray:
+    """OPTQ's update order ([QuIP] "OPTQ (Formerly known as GPTQ)."):
+    quantize column k by nearest rounding, compute its error scaled by the
+    pivot of the upper Cholesky factor R of H^-1 (H^-1 = R^T R), subtract it
+    from the remaining columns along row k of R, repeat.  Returns codes."""
+    w = np.array(Wt, dtype=np.float64, copy=True)
+    Hinv = np.linalg.inv(np.asarray(H, dtype=np.float64))
+    R = np.linalg.cholesky(Hinv).T              # upper, Hinv = R^T R
+    m, n = w.shape
+    codes = np.zeros((m, n), dtype=np.int64)
+    for k in range(n):
+        c = quantize(w[:, k], lo, s, bits)
+        codes[:, k] = c
+        e = (w[:, k] - (lo + s * c)) / R[k, k]
+        w[:, k + 1:] -= np.outer(e, R[k, k + 1:])
+    return codes
+
+
+# ----------------------------------------------------------------------------
+# O7/O8  Dequantisation, loss
+# ----------------------------------------------------------------------------
+
+
+def dequantize(codes: np.ndarray, lo: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """W~^ = lo + s * code, per row."""
+    return np.asarray(lo, dtype=np.float64)[:, None] + np.asarray(s, dtype=np.float64)[:, None] * codes
+
+
+def proxy_loss(What: np.ndarray, W: np.ndarray, H: np.ndarray) -> float:
+    """l(W^) = tr((W^ - W) H (W^ - W)^T)  ([QuIP] Introduction)."""
+    E = np.asarray(What, dtype=np.float64) - np.asarray(W, dtype=np.float64)
+    return float(np.einsum("ij,ij->", E @ np.asarray(H, dtype=np.float64), E))
+
+
+# ----------------------------------------------------------------------------
+# The whole layer
+# ----------------------------------------------------------------------------
+
+
+@dataclass
+class Pipeline:
+    H: np.ndarray           # damped proxy Hessian
+    U: SideTransform
+    V: SideTransform
+    Wt: np.ndarray          # incoherent weights
+    Ht: np.ndarray          # incoherent damped Hessian
+    Uf: np.ndarray          # strictly upper LDL factor of Ht
+    D: np.ndarray
+    lo: np.ndarray
+    s: np.ndarray
+    codes: np.ndarray
+    Wt_hat: np.ndarray      # dequantised, incoherent domain
+    W_hat: np.ndarray       # dequantised, original domain
+    loss: float             # tr((Wt_hat - Wt) Ht (Wt_hat - Wt)^T)
+
+
+def run_pipeline(W: np.ndarray, X: np.ndarray, seed: int, m_side, n_side, bits: int,
+                 alpha: float = 0.01, block: Optional[int] = None) -> Pipeline:
+    """Hessian -> damping -> incoherence -> LDL -> grid -> LDLQ -> dequant -> inverse.
+
+    ``m_side`` / ``n_side`` are objects with attributes kind, p, q.
+    """
+    W = np.asarray(W, dtype=np.float64)
+    m, n = W.shape
+    H = damp(hessian(X), alpha)
+    U = make_side(seed, "m", m_side.kind, m, m_side.p, m_side.q)
+    V = make_side(seed, "n", n_side.kind, n, n_side.p, n_side.q)
+    Wt, Ht = incoherence_forward(W, H, U, V)
+    Uf, D = udu(Ht)
+    lo, s = row_grid(Wt, bits)
+    if block is None:
+        codes, Wt_hat, _ = ldlq(Wt, Uf, lo, s, bits)
+    else:
+        codes, Wt_hat = ldlq_blocked(Wt, Uf, lo, s, bits, block)
+    W_hat = incoherence_inverse(Wt_hat, U, V)
+    return Pipeline(H, U, V, Wt, Ht, Uf, D, lo, s, codes, Wt_hat, W_hat,
+                    proxy_loss(Wt_hat, Wt, Ht))

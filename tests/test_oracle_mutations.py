@@ -1,0 +1,124 @@
+"""Plant plausible mistakes in the oracle (CPU only) and check that at least
+one pin in test_oracle_pins.py fails for each: a dropped term, a wrong sign,
+a transposed operand, a wrong index or normalisation."""
+import numpy as np
+import pytest
+
+import oracle as O
+import oracle.quip_oracle as Q
+import test_oracle_pins as P
+
+
+def _fails(pins):
+    for pin in pins:
+        try:
+            pin()
+        except (AssertionError, ValueError, IndexError, np.linalg.LinAlgError):
+            return True
+    return False
+
+
+def _ldlq_wrong_sign(Wt, U, lo, s, bits):
+    Wt = np.asarray(Wt, dtype=np.float64)
+    m, n = Wt.shape
+    codes = np.zeros((m, n), dtype=np.int64)
+    What = np.zeros((m, n))
+    eta = np.zeros((m, n))
+    errT = np.zeros((n, m))
+    for k in range(n):
+        a = Wt[:, k] - U[:k, k] @ errT[:k]            # planted: feedback sign
+        c = Q.quantize(a, lo, s, bits)
+        codes[:, k], What[:, k] = c, lo + s * c
+        eta[:, k] = What[:, k] - a
+        errT[k] = Wt[:, k] - What[:, k]
+    return codes, What, eta
+
+
+def _ldlq_transposed(Wt, U, lo, s, bits):
+    return Q.__dict__["_ldlq_orig"](Wt, np.asarray(U).T, lo, s, bits)
+
+
+def _ldlq_drop_feedback(Wt, U, lo, s, bits):
+    return Q.__dict__["_ldlq_orig"](Wt, np.zeros_like(U), lo, s, bits)
+
+
+def _udu_lower(H):
+    U, D = Q.__dict__["_udu_orig"](H)
+    return U.T, D
+
+
+def _udu_no_sqrt(H):
+    U, D = Q.__dict__["_udu_orig"](H)
+    return U, np.sqrt(D)
+
+
+def _hessian_no_norm(X):
+    X = np.asarray(X, dtype=np.float64)
+    return X.T @ X
+
+
+def _damp_trace(H, alpha):
+    H = np.array(H, dtype=np.float64, copy=True)
+    H[np.diag_indices_from(H)] += alpha * float(np.trace(H))     # planted: sum, not mean
+    return H
+
+
+def _grid_bits(Wt, bits):
+    lo, s = Q.__dict__["_row_grid_orig"](Wt, bits)
+    return lo, s * (2 ** bits - 1) / 2 ** bits                   # planted: 2^b not 2^b - 1
+
+
+def _rint_floor(a, lo, s, bits):
+    return np.clip(np.floor((a - lo) / s), 0, 2 ** bits - 1)
+
+
+def _signs_on_output(self):
+    if self.kind == "hadamard":
+        return self.signs[:, None] * O.sylvester_hadamard(self.dim) / np.sqrt(self.dim)
+    return Q.__dict__["_matrix_orig"](self)
+
+
+def _forward_no_transpose(W, H, U, V):
+    Um, Vn = U.matrix(), V.matrix()
+    Wt = Um @ W @ Vn                                              # planted: V not V^T
+    Ht = Vn @ H @ Vn.T
+    return Wt, 0.5 * (Ht + Ht.T)
+
+
+def _box_muller_sin(seed, stream, p):
+    e = np.arange(p * p, dtype=np.uint64)
+    u1 = Q.uniform53(Q.splitmix64(seed, stream, 2 * e))
+    u2 = Q.uniform53(Q.splitmix64(seed, stream, 2 * e + np.uint64(1)))
+    return (np.sqrt(-2.0 * np.log(u1)) * np.sin(2.0 * np.pi * u2)).reshape(p, p)
+
+
+LDLQ_PINS = [P.test_ldlq_worked_examples, lambda: P.test_ldlq_loss_equals_eta_D_eta(2),
+             lambda: P.test_ldlq_equals_optq_order(2)]
+
+MUTANTS = [
+    ("ldlq", _ldlq_wrong_sign, LDLQ_PINS),
+    ("ldlq", _ldlq_transposed, LDLQ_PINS),
+    ("ldlq", _ldlq_drop_feedback, LDLQ_PINS),
+    ("udu", _udu_lower, [P.test_udu_hand_2x2, lambda: P.test_udu_reconstructs(7)]),
+    ("udu", _udu_no_sqrt, [P.test_udu_hand_2x2, lambda: P.test_udu_reconstructs(7)]),
+    ("hessian", _hessian_no_norm, [P.test_hessian_hand_example, P.test_hessian_equals_sum_of_outer_products]),
+    ("damp", _damp_trace, [P.test_damp_adds_alpha_mean_diag]),
+    ("row_grid", _grid_bits, [P.test_grid_and_quantize_basics]),
+    ("quantize", _rint_floor, [P.test_grid_and_quantize_basics, P.test_ldlq_worked_examples]),
+    ("incoherence_forward", _forward_no_transpose, [P.test_incoherence_preserves_proxy_and_inverts]),
+    ("gaussian_matrix", _box_muller_sin, [P.test_signs_and_gaussians_statistics]),
+]
+
+
+@pytest.mark.parametrize("name,mutant,pins", MUTANTS, ids=[f"{m[0]}:{m[1].__name__}" for m in MUTANTS])
+def test_planted_mistake_is_caught(monkeypatch, name, mutant, pins):
+    monkeypatch.setitem(Q.__dict__, f"_{name}_orig", getattr(Q, name))
+    monkeypatch.setattr(Q, name, mutant)
+    monkeypatch.setattr(O, name, mutant)
+    assert _fails(pins), f"no pin caught the planted mistake in {name}"
+
+
+def test_planted_sign_placement_is_caught(monkeypatch):
+    monkeypatch.setitem(Q.__dict__, "_matrix_orig", Q.SideTransform.matrix)
+    monkeypatch.setattr(Q.SideTransform, "matrix", _signs_on_output)
+    assert _fails([P.test_hadamard_sign_placement_hand_example])
