@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Throughput of incoherence-processed LDLQ for one linear layer on B200.
+
+One step = the whole hot path for one layer on device-resident inputs:
+draw (U, V) -> H = X^T X (tensor cores) -> finalise + damp -> W~ = U W V^T,
+H~ = V H V^T -> LDL of H~ -> LDLQ rounding -> dequantise -> inverse transform.
+Metric: quantized weights per second (m * n / step time), whole job.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config attn7b]
+  python bench.py --impl reference ...    # the FP64 CPU oracle, bounded sample
+
+Multi-GPU (torchrun): each rank quantises its own layer of the same shape
+(seed + rank), no data-path collective (weak scaling); the step time is the
+max over ranks.  L2 is flushed (256 MB write) before every timed step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quip_synth import CONFIGS, LayerConfig, make_layer  # noqa: E402
+
+METRIC = "quantized weights/s per layer (Hessian+incoherence+LDLQ)"
+UNIT = "weights/s"
+STAGES = ["transform", "hessian", "finalize", "incoherence_fwd", "ldl", "ldlq", "dequant",
+          "incoherence_inv"]
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# FP32 FFMA peak from unit counts and clock: 148 SMs x 128 FP32 lanes x 2 flop x 1.965 GHz.
+FFMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def stage_work(cfg: LayerConfig):
+    """Algorithmic work per stage: (kind, amount, bound, engine-note)."""
+    m, n, N, b = cfg.m, cfg.n, cfg.N, cfg.block
+    xb = 2 if cfg.dtype == "bf16" else 4
+    return {
+        "transform": ("bytes", 4.0 * (m + n), "hbm"),
+        "hessian": ("flops", float(N) * n * (n + 1), "tensor" if cfg.dtype == "bf16" else "alu"),
+        "finalize": ("bytes", 8.0 * n * n, "hbm"),
+        # W read + W~ write, H read + H~ write (minimum traffic of the transform)
+        "incoherence_fwd": ("bytes", (xb + 4.0) * m * n + 8.0 * n * n, "hbm"),
+        "ldl": ("flops", n ** 3 / 3.0, "alu"),
+        # trailing GEMMs m n (n - b) plus in-block feedback m n b
+        "ldlq": ("flops", float(m) * n * n, "alu"),
+        "dequant": ("bytes", 5.0 * m * n + 8.0 * m, "hbm"),
+        "incoherence_inv": ("bytes", 8.0 * m * n, "hbm"),
+    }
+
+
+def roofline_entry(kind, amount, bound, ms, pk):
+    if kind == "bytes":
+        achieved = amount / (ms * 1e-3) / 1e9
+        peak, unit = pk["hbm_gbs"], "GB/s"
+    else:
+        achieved = amount / (ms * 1e-3) / 1e12
+        peak, unit = (pk["bf16_tflops"], "TFLOP/s") if bound == "tensor" else (FFMA_TFLOPS, "TFLOP/s")
+    return {"bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 1), "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": None}
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle timing
+
+
+def oracle_sample(cfg: LayerConfig, d, rows: int = 64, tokens: int = 1024):
+    """Time the FP64 oracle's own stage functions on a bounded sample of the
+    layer and scale to the whole layer.  Row-separable stages (LDLQ,
+    dequantisation) run on `rows` rows, the Hessian on `tokens` tokens; the
+    n x n and m x n transforms and the LDL run at full size.  Returns
+    (estimated seconds for the whole layer, breakdown, description)."""
+    import oracle as O
+    m, n, N = cfg.m, cfg.n, cfg.N
+    t = {}
+    t0 = time.perf_counter()
+    H = O.hessian(d["X"][:tokens])
+    t["hessian"] = (time.perf_counter() - t0) * (N / min(tokens, N))
+    t0 = time.perf_counter()
+    H = O.damp(H, cfg.damp)
+    t["finalize"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    U = O.make_side(cfg.seed, "m", cfg.m_side.kind, m, cfg.m_side.p, cfg.m_side.q)
+    V = O.make_side(cfg.seed, "n", cfg.n_side.kind, n, cfg.n_side.p, cfg.n_side.q)
+    t["transform"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    Wt, Ht = O.incoherence_forward(d["W"], H, U, V)
+    t["incoherence_fwd"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    Uf, _ = O.udu(Ht)
+    t["ldl"] = time.perf_counter() - t0
+    r = min(rows, m)
+    t0 = time.perf_counter()
+    lo, s = O.row_grid(Wt, cfg.bits)
+    codes, _, _ = O.ldlq(Wt[:r], Uf, lo[:r], s[:r], cfg.bits)
+    t["ldlq"] = (time.perf_counter() - t0) * (m / r)
+    t0 = time.perf_counter()
+    O.dequantize(codes, lo[:r], s[:r])
+    t["dequant"] = (time.perf_counter() - t0) * (m / r)
+    t0 = time.perf_counter()
+    O.incoherence_inverse(Wt, U, V)
+    t["incoherence_inv"] = time.perf_counter() - t0
+    desc = (f"FP64 oracle stages on {cfg.name}: Hessian on {min(tokens, N)} of {N} tokens, LDLQ and "
+            f"dequant on {r} of {m} rows (scaled linearly), transforms, LDL and grid at full size")
+    return sum(t.values()), t, desc
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return sum(i.get("num_threads", 0) for i in info if i.get("user_api") == "blas") or os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+# ----------------------------------------------------------------------------- arms
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args, cfg: LayerConfig):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return
+    d = make_layer(cfg)
+    for _ in range(args.warmup):
+        oracle_sample(cfg, d, rows=32, tokens=512)
+    est, wall = [], 0.0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        e, _, desc = oracle_sample(cfg, d, rows=32, tokens=512)
+        wall += time.perf_counter() - t0
+        est.append(e)
+    sec = statistics.mean(est)
+    value = cfg.m * cfg.n / sec
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_desc(cfg, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc + f"; {args.steps} samples, {wall:.1f} s wall"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_desc(cfg: LayerConfig, args):
+    side = lambda s: s.kind if s.kind != "kronecker" else f"kronecker {s.p}x{s.q}"
+    return {
+        "workload": f"{cfg.name}: W {cfg.m}x{cfg.n} {cfg.dtype}, X {cfg.N}x{cfg.n} {cfg.dtype}, "
+                    f"U {side(cfg.m_side)}, V {side(cfg.n_side)}, LDLQ block {cfg.block}, {cfg.bits}-bit",
+        "m": cfg.m, "n": cfg.n, "tokens": cfg.N, "bits": cfg.bits, "block": cfg.block,
+        "damp": cfg.damp, "l2": "flushed before every timed step (256 MB write)",
+        "parallelism": f"replicas x{args.gpus} (one layer per GPU)",
+    }
+
+
+def run_ours(args, cfg: LayerConfig):
+    import torch
+    import torch.distributed as dist
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    if world > 1 and not dist.is_initialized():
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    import post_weight_quantization_09_b200 as Q
+    from post_weight_quantization_09_b200 import _lib as L
+    lib = Q.load()
+    rcfg = LayerConfig(**{**cfg.__dict__, "seed": cfg.seed + rank})
+    d = make_layer(rcfg)
+    as_t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 \
+        else torch.from_numpy(a)
+    W_h = as_t(d["W_bf16"] if cfg.dtype == "bf16" else d["W"]).pin_memory()
+    X_h = as_t(d["X_bf16"] if cfg.dtype == "bf16" else d["X"]).pin_memory()
+    W = W_h.cuda()
+    X = X_h.cuda()
+    q = Q.LayerQuantizer(cfg.m, cfg.n, cfg.m_side, cfg.n_side, cfg.bits, cfg.block, cfg.damp,
+                         rcfg.seed)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")   # 256 MB > L2
+
+    def step(ev=None):
+        mark = (lambda i: ev[i].record(stream)) if ev else (lambda i: None)
+        mark(0)
+        q.new_transform()
+        mark(1)
+        Q.quip_hessian_accumulate(X, q.H, False)
+        mark(2)
+        Q.quip_hessian_finalize(q.H, cfg.N, cfg.damp)
+        mark(3)
+        Q.quip_incoherence_forward(q.tf, W, q.W_t, q.H, q.ws)
+        mark(4)
+        Q.quip_ldl(q.H, q.D, q.ws)
+        mark(5)
+        Q.quip_ldlq_quantize(q.W_t, q.H, cfg.bits, cfg.block, q.codes, q.lo, q.scale, q.ws)
+        mark(6)
+        Q.quip_dequantize(q.codes, q.lo, q.scale, q.W_hat)
+        mark(7)
+        Q.quip_incoherence_inverse(q.tf, q.W_hat, q.W_hat, q.ws)
+        mark(8)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    st = Q.quip_sync_status()
+    if st != L.QUIP_OK:
+        raise RuntimeError(f"device status after warm-up: {L.status_string(st)}")
+
+    nev = len(STAGES) + 1
+    step_ms, stage_ms = [], [[] for _ in STAGES]
+    launches0 = lib.quip_kernel_launches()
+    with ClockSampler(local) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(nev)]
+            step(ev)
+            torch.cuda.synchronize()
+            step_ms.append(ev[0].elapsed_time(ev[-1]))
+            for i in range(len(STAGES)):
+                stage_ms[i].append(ev[i].elapsed_time(ev[i + 1]))
+            if world > 1:
+                dist.barrier()
+    launches = lib.quip_kernel_launches() - launches0
+    st = Q.quip_sync_status()
+    if st != L.QUIP_OK:
+        raise RuntimeError(f"device status after timing: {L.status_string(st)}")
+
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * cfg.m * cfg.n / (ms_per_step * 1e-3)
+
+    # ---- end to end through the public API: pinned host inputs in, codes + grid out
+    codes_h = torch.empty(cfg.m, cfg.n, dtype=torch.uint8).pin_memory()
+    lo_h = torch.empty(cfg.m, dtype=torch.float32).pin_memory()
+    sc_h = torch.empty(cfg.m, dtype=torch.float32).pin_memory()
+    e2e_ms = []
+    for i in range(args.e2e_steps + 1):
+        flush.zero_()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        q.run_host(W_h, X_h, codes_h, lo_h, sc_h)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i > 0:                      # the first one is a warm-up
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e = statistics.mean(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e = float(t.item())
+    h2d = W_h.numel() * W_h.element_size() + X_h.numel() * X_h.element_size()
+    d2h = codes_h.numel() + 4 * (lo_h.numel() + sc_h.numel())
+
+    if rank != 0:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
+    pk = peaks()
+    work = stage_work(cfg)
+    stages = {}
+    for i, name in enumerate(STAGES):
+        ms = statistics.mean(stage_ms[i])
+        kind, amount, bound = work[name]
+        stages[name] = {"ms": round(ms, 4), **roofline_entry(kind, amount, bound, ms, pk)}
+    dominant = max(stages, key=lambda k: stages[k]["ms"])
+    roof = {k: v for k, v in stages[dominant].items() if k != "ms"}
+    roof["stage"] = dominant
+    roof["peak_source"] = pk["source"]
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded Gaussian W / X with outliers, bf16; no weights or C4 in the box)",
+        "config": config_desc(cfg, args),
+        "roofline": roof,
+        "stages": stages,
+        "e2e": {"value": world * cfg.m * cfg.n / (e2e * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        sec, _, desc = oracle_sample(cfg, d)
+        line["cpu_baseline"] = {"value": cfg.m * cfg.n / sec, "unit": UNIT, "cores": blas_threads(),
+                                "kind": "oracle", "sample": desc}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="attn7b", choices=sorted(CONFIGS))
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,239 @@
+/*
+ * quip.h — C ABI of libquip: incoherence-processed LDLQ for one linear layer
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * The method is QuIP ("QuIP: 2-Bit Quantization of Large Language Models With
+ * Guarantees", arXiv 2307.13304) with the randomized Hadamard incoherence of
+ * QuIP# ("QuIP#: Even Better LLM Quantization with Hadamard Incoherence and
+ * Lattice Codebooks", arXiv 2402.04396, abstract).  For W in R^{m x n} and
+ * calibration activations X in R^{N x n} the library computes, all on the GPU:
+ *
+ *   H   = X^T X / N                           (QuIP, adaptive-rounding section)
+ *   H  += alpha * mean(diag H) * I            (QuIP, Experiments, "Methods.")
+ *   W~  = U W V^T,  H~ = V H V^T              (QuIP, incoherence processing)
+ *   H~  = (I + Ů) D (I + Ů)^T, Ů strictly upper         (LDL factorisation)
+ *   per row: lo = min W~_i,  s = (max W~_i - lo) / (2^b - 1)
+ *   for k:  a_k = W~_k + sum_{j<k} (W~_j - W^_j) Ů_jk,  c_k = Q(a_k),
+ *           W^_k = lo + s c_k                               (LDLQ)
+ *   W^  = U^T W~^ V                           (QuIP, incoherence post-processing)
+ *
+ * with U (m side) and V (n side) each a randomized Hadamard transform
+ * H_d diag(s) / sqrt(d) (d a power of two) or a Kronecker product A (x) B of
+ * two Haar-random orthogonal matrices (QuIP, Introduction).
+ *
+ * Conventions for every entry point
+ *  - Matrices are row-major.  "device" pointers are CUDA global memory of
+ *    the current device; "host" pointers are ordinary CPU memory.
+ *  - The caller owns every buffer it passes; the library never frees or
+ *    keeps a caller pointer after the call returns.  The library owns only
+ *    quip_transform objects (created / destroyed below).
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *    enqueue work on it and return before the work finishes, unless stated.
+ *  - Argument and shape errors are returned synchronously before anything
+ *    is launched.  Errors found on the device (a non-positive LDL pivot, a
+ *    non-finite value, a bounded wait that ran out) set a library status
+ *    word that quip_sync_status() returns.
+ *  - Workspace: entry points that take (ws, ws_bytes) need at least the
+ *    bytes quip_workspace_size() reports for the same arguments, device
+ *    memory, 256-byte aligned; the contents on entry are irrelevant.
+ */
+#ifndef QUIP_H_
+#define QUIP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QUIP_OK = 0,
+  QUIP_ERR_ARG = 1,          /* null pointer, bad enum, bad bit width, ...   */
+  QUIP_ERR_SHAPE = 2,        /* sizes inconsistent or unsupported            */
+  QUIP_ERR_UNSUPPORTED = 3,  /* valid request this build does not implement  */
+  QUIP_ERR_NOT_PD = 4,       /* LDL met a pivot <= 0 (H~ not positive definite) */
+  QUIP_ERR_NONFINITE = 5,    /* NaN or Inf met on the device                 */
+  QUIP_ERR_CUDA = 6,         /* a CUDA runtime / driver call failed          */
+  QUIP_ERR_TIMEOUT = 7,      /* a bounded device-side wait ran out           */
+  QUIP_ERR_WORKSPACE = 8     /* ws too small or misaligned                   */
+} quip_status;
+
+typedef enum { QUIP_F32 = 0, QUIP_BF16 = 1 } quip_dtype;
+
+/* Kind of random orthogonal matrix on one side of W. */
+typedef enum {
+  QUIP_T_IDENTITY = 0,   /* no transform on this side                              */
+  QUIP_T_HADAMARD = 1,   /* H_d diag(s) / sqrt(d), Sylvester order, s_i = +-1;
+                            d a power of two, 2 <= d <= 8192                     */
+  QUIP_T_KRONECKER = 2   /* A (x) B, A p x p, B q x q Haar-random, p * q = d,
+                            1 <= p, q <= 256                                     */
+} quip_tkind;
+
+/* Operations whose workspace quip_workspace_size() reports. */
+typedef enum {
+  QUIP_OP_INCOHERENCE_FORWARD = 0,
+  QUIP_OP_INCOHERENCE_INVERSE = 1,
+  QUIP_OP_LDL = 2,
+  QUIP_OP_LDLQ = 3
+} quip_op;
+
+typedef struct quip_transform quip_transform;   /* opaque, library-owned */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* quip_status_string(int status);
+
+/* Library version string, e.g. "quip-b200 0.1.0 sm_100a". */
+const char* quip_version(void);
+
+/* Number of CUDA kernels this library has enqueued since it was loaded
+ * (all entry points, all streams; host-side counter). */
+uint64_t quip_kernel_launches(void);
+
+/*
+ * Draw the two random orthogonal matrices for an m x n layer from `seed`
+ * (QuIP, incoherence-processing section: U in O(m), V in O(n); QuIP# abstract:
+ * randomized Hadamard).  Randomness: counter-based SplitMix64 (Steele, Lea &
+ * Flood 2014); element i of stream t is output t*2^40 + i + 1 of the
+ * sequence started at `seed`.  Streams: 0 = m-side signs, 1 = n-side signs,
+ * 2 / 3 = m-side A / B Gaussians, 4 / 5 = n-side A / B Gaussians.  A sign is
+ * -1 when the draw's top bit is set.  A Gaussian matrix element e (row-major)
+ * is sqrt(-2 ln u1) cos(2 pi u2) with u = ((draw >> 11) + 1) 2^-53 of draws
+ * 2e and 2e+1; the factor is Q of G = QR with diag(R) > 0.
+ * Signs, factors and the QR are computed on the device on `stream`.
+ *   m_kind / n_kind : quip_tkind for each side; m_p*m_q == m for KRONECKER.
+ *   out             : receives the new object (host pointer to a handle).
+ * Allocates device memory owned by the object (freed by destroy).  The
+ * object may be used on any stream after the creating stream has passed it.
+ */
+quip_status quip_transform_create(uint64_t seed, int64_t m, int64_t n,
+                                  int m_kind, int64_t m_p, int64_t m_q,
+                                  int n_kind, int64_t n_p, int64_t n_q,
+                                  void* stream, quip_transform** out);
+
+/*
+ * Redraw an existing transform's random signs / factors from `seed` in place
+ * (same definition as quip_transform_create, no allocation): kernels only,
+ * enqueued on `stream`.  Work already enqueued that reads the transform must
+ * be ordered before this call by the caller.
+ */
+quip_status quip_transform_draw(quip_transform* tf, uint64_t seed, void* stream);
+
+/* Free a transform (synchronises the device first).  NULL is accepted. */
+quip_status quip_transform_destroy(quip_transform* tf);
+
+/*
+ * Device pointers (library-owned, read-only, fp32) of one side's data:
+ * side 0 = m side (U), 1 = n side (V).  For HADAMARD `signs` has d entries;
+ * for KRONECKER `A` is p x p and `B` is q x q, row-major; pointers that do
+ * not apply are set to NULL.  kind, p, q may be NULL.
+ */
+quip_status quip_transform_info(const quip_transform* tf, int side, int* kind,
+                                int64_t* p, int64_t* q, const float** signs,
+                                const float** A, const float** B);
+
+/*
+ * Proxy Hessian accumulation (QuIP, adaptive-rounding section: H is the
+ * second moment of the calibration inputs): H_acc (+)= X^T X.
+ *   X          : device, N x n, row stride ldx elements, dtype QUIP_BF16 or
+ *                QUIP_F32.  For BF16 the bf16 products are exact and summed
+ *                in fp32 on the tensor cores (tcgen05); ldx*2 must be a
+ *                multiple of 16 bytes and X 16-byte aligned.
+ *   H_acc      : device, n x n fp32, row stride n.  On return its lower
+ *                triangle (i >= j) holds the (accumulated) sum; the strict
+ *                upper triangle is unspecified until quip_hessian_finalize.
+ *   accumulate : 0 = overwrite, 1 = add to the lower triangle already there
+ *                (stream X in token chunks; N may differ per call).
+ * N == 0 with accumulate == 0 writes zeros.
+ */
+quip_status quip_hessian_accumulate(const void* X, int dtype, int64_t N, int64_t n,
+                                    int64_t ldx, float* H_acc, int accumulate,
+                                    void* stream);
+
+/*
+ * H = sym(H_acc) / N_total + damp * mean(diag(H_acc / N_total)) * I, in place
+ * (QuIP, Experiments, "Methods.": H <- H + alpha mean(diag H) I).  Reads the
+ * lower triangle, writes the full symmetric matrix.  N_total >= 1, damp >= 0.
+ */
+quip_status quip_hessian_finalize(float* H, int64_t n, int64_t N_total, float damp,
+                                  void* stream);
+
+/*
+ * Incoherence pre-processing (QuIP, incoherence-processing section):
+ *   W_t = U W V^T   (m x n fp32, row stride n), W: device m x n, row stride
+ *                   ldw, dtype QUIP_BF16 or QUIP_F32; W and W_t must not overlap;
+ *   H   = V H V^T   in place (n x n fp32, full symmetric on entry and exit),
+ *                   skipped when H is NULL.
+ * ws: workspace for QUIP_OP_INCOHERENCE_FORWARD.
+ */
+quip_status quip_incoherence_forward(const quip_transform* tf, const void* W, int w_dtype,
+                                     int64_t ldw, float* W_t, float* H, void* ws,
+                                     size_t ws_bytes, void* stream);
+
+/*
+ * Incoherence post-processing: W_hat = U^T W_hat_t V (m x n fp32, row stride
+ * n).  W_hat may equal W_hat_t (in place).  ws: QUIP_OP_INCOHERENCE_INVERSE.
+ */
+quip_status quip_incoherence_inverse(const quip_transform* tf, const float* W_hat_t,
+                                     float* W_hat, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * LDL factorisation H_t = (I + Ů) diag(D) (I + Ů)^T with Ů strictly upper
+ * triangular (the factorisation that defines LDLQ's feedback; QuIP,
+ * adaptive-rounding section).  In place on H_t (n x n fp32, row stride n,
+ * symmetric positive definite; only the upper triangle is read):
+ * on return the strict upper triangle holds Ů, D (device, n fp32) the
+ * pivots; the diagonal and lower triangle of H_t are unspecified.
+ * A pivot <= 0 or non-finite sets QUIP_ERR_NOT_PD in the status word
+ * (quip_sync_status).  ws: QUIP_OP_LDL.
+ */
+quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/*
+ * LDLQ adaptive rounding of the incoherent weights (QuIP, adaptive-rounding
+ * section; "Methods.": LDLQ = OPTQ), one b-bit per-row min/max grid:
+ *   lo_i = min_j W_t[i,j], s_i = (max_j W_t[i,j] - lo_i) / (2^bits - 1)
+ *   (s_i = 1 for a constant row);
+ *   for k = 0..n-1: a_k = W_t[:,k] + sum_{j<k} (W_t[:,j] - W^[:,j]) Ů[j,k],
+ *   codes[:,k] = clamp(rint((a_k - lo) / s), 0, 2^bits - 1) (ties to even),
+ *   W^[:,k] = lo + s codes[:,k].
+ * Evaluated in fp32, blocked over `block` columns (the result does not
+ * depend on block in exact arithmetic).
+ *   W_t   : device m x n fp32 (row stride n), not modified.
+ *   Uring : device n x n fp32, row stride ldu >= n; only the strict upper
+ *           triangle is read (the H_t buffer quip_ldl returned).
+ *   bits  : 1..8.  block: 32, 64 or 128, with n % block == 0.
+ *   codes : device m x n uint8 (row stride n).  lo, scale: device m fp32.
+ * ws: QUIP_OP_LDLQ.
+ */
+quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu,
+                               int64_t m, int64_t n, int bits, int64_t block,
+                               uint8_t* codes, float* lo, float* scale, void* ws,
+                               size_t ws_bytes, void* stream);
+
+/* W_hat_t[i,j] = lo[i] + scale[i] * codes[i,j]  (device; m x n, row stride n). */
+quip_status quip_dequantize(const uint8_t* codes, const float* lo, const float* scale,
+                            int64_t m, int64_t n, float* W_hat_t, void* stream);
+
+/*
+ * Bytes of workspace `op` needs (quip_op).  tf is required for the
+ * incoherence ops and ignored otherwise; block is used by QUIP_OP_LDLQ.
+ * *bytes may be 0.
+ */
+quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int64_t n,
+                                 int64_t block, size_t* bytes);
+
+/*
+ * Synchronise `stream`, then return and clear the device status word
+ * (QUIP_OK if no device-side error was recorded since the last call), or
+ * QUIP_ERR_CUDA if a CUDA error is pending.  The status word is shared by all
+ * streams of the process on the current device.
+ */
+quip_status quip_sync_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QUIP_H_ */

@@ -1,0 +1,283 @@
+"""Incoherence-processed LDLQ (QuIP / QuIP#) for one linear layer on a B200.
+
+Thin PyTorch-facing binding of libquip (``include/quip.h``).  PyTorch only
+owns device memory and supplies the CUDA stream; every step runs in the
+library's sm_100a kernels.  The functions below carry the C entry points'
+names and take torch tensors; ``LayerQuantizer`` strings them together for
+one layer (Hessian -> damping -> incoherence -> LDL -> LDLQ -> dequantise ->
+inverse transform) with buffers allocated once.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _lib as L
+from ._lib import QuipError, load, status_string  # noqa: F401
+
+__all__ = [
+    "Transform", "quip_hessian_accumulate", "quip_hessian_finalize", "quip_incoherence_forward",
+    "quip_incoherence_inverse", "quip_ldl", "quip_ldlq_quantize", "quip_dequantize",
+    "quip_workspace_size", "quip_sync_status", "LayerQuantizer", "quantize_layer", "QuipError",
+    "KIND",
+]
+
+KIND = {"identity": L.QUIP_T_IDENTITY, "hadamard": L.QUIP_T_HADAMARD, "kronecker": L.QUIP_T_KRONECKER}
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return L.QUIP_BF16
+    if t.dtype == torch.float32:
+        return L.QUIP_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _cuda(t: torch.Tensor, name: str) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+_cudart = None
+
+
+def _memcpy_d2d(dst_ptr: int, src_ptr: int, nbytes: int) -> None:
+    """Device-to-device copy through the CUDA runtime torch already loaded."""
+    global _cudart
+    if _cudart is None:
+        _cudart = ctypes.CDLL("libcudart.so.12")
+        _cudart.cudaMemcpy.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int]
+        _cudart.cudaMemcpy.restype = ctypes.c_int
+    if _cudart.cudaMemcpy(ctypes.c_void_p(dst_ptr), ctypes.c_void_p(src_ptr), nbytes, 3) != 0:
+        raise RuntimeError("cudaMemcpy failed")
+
+
+class Transform:
+    """The pair (U, V) of random orthogonal matrices for an m x n layer."""
+
+    def __init__(self, seed: int, m: int, n: int, m_side, n_side, stream=None):
+        lib = load()
+        self.m, self.n = m, n
+        self.m_side, self.n_side = m_side, n_side
+        h = ctypes.c_void_p()
+        L.check(lib.quip_transform_create(
+            ctypes.c_uint64(seed & 0xFFFFFFFFFFFFFFFF), m, n, KIND[m_side.kind], m_side.p, m_side.q,
+            KIND[n_side.kind], n_side.p, n_side.q, _s(stream), ctypes.byref(h)), "quip_transform_create")
+        self.handle = h
+
+    def draw(self, seed: int, stream=None) -> None:
+        """Redraw the random signs / factors from `seed` in place (no allocation)."""
+        L.check(load().quip_transform_draw(self.handle, ctypes.c_uint64(seed & 0xFFFFFFFFFFFFFFFF),
+                                           _s(stream)), "quip_transform_draw")
+
+    def close(self) -> None:
+        if self.handle:
+            load().quip_transform_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def factors(self, side: int) -> dict:
+        """Copies of one side's data: {'kind', 'signs'} or {'kind', 'A', 'B'} (fp32, cuda)."""
+        kind, p, q = ctypes.c_int(), ctypes.c_int64(), ctypes.c_int64()
+        s, a, b = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_void_p()
+        L.check(load().quip_transform_info(self.handle, side, ctypes.byref(kind), ctypes.byref(p),
+                                           ctypes.byref(q), ctypes.byref(s), ctypes.byref(a),
+                                           ctypes.byref(b)), "quip_transform_info")
+        torch.cuda.synchronize()
+        dim = self.m if side == 0 else self.n
+        out = {"kind": kind.value}
+        if kind.value == L.QUIP_T_HADAMARD:
+            t = torch.empty(dim, dtype=torch.float32, device="cuda")
+            _memcpy_d2d(t.data_ptr(), s.value, dim * 4)
+            out["signs"] = t
+        elif kind.value == L.QUIP_T_KRONECKER:
+            A = torch.empty(p.value, p.value, dtype=torch.float32, device="cuda")
+            B = torch.empty(q.value, q.value, dtype=torch.float32, device="cuda")
+            _memcpy_d2d(A.data_ptr(), a.value, A.numel() * 4)
+            _memcpy_d2d(B.data_ptr(), b.value, B.numel() * 4)
+            out["A"], out["B"] = A, B
+        return out
+
+
+def quip_workspace_size(op: int, tf: Optional[Transform], m: int, n: int, block: int = 0) -> int:
+    nb = ctypes.c_size_t()
+    L.check(load().quip_workspace_size(op, tf.handle if tf else None, m, n, block, ctypes.byref(nb)),
+            "quip_workspace_size")
+    return nb.value
+
+
+def _ws(nbytes: int, device) -> Optional[torch.Tensor]:
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def quip_hessian_accumulate(X: torch.Tensor, H_acc: torch.Tensor, accumulate: bool = False,
+                            stream=None) -> None:
+    _cuda(X, "X"), _cuda(H_acc, "H_acc")
+    N, n = X.shape
+    L.check(load().quip_hessian_accumulate(_p(X), _dtype(X), N, n, X.stride(0), _p(H_acc),
+                                           int(accumulate), _s(stream)), "quip_hessian_accumulate")
+
+
+def quip_hessian_finalize(H: torch.Tensor, N_total: int, damp: float, stream=None) -> None:
+    _cuda(H, "H")
+    L.check(load().quip_hessian_finalize(_p(H), H.shape[0], N_total, damp, _s(stream)),
+            "quip_hessian_finalize")
+
+
+def quip_incoherence_forward(tf: Transform, W: torch.Tensor, W_t: torch.Tensor,
+                             H: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                             stream=None) -> None:
+    _cuda(W, "W"), _cuda(W_t, "W_t")
+    need = quip_workspace_size(L.QUIP_OP_INCOHERENCE_FORWARD, tf, tf.m, tf.n)
+    if ws is None:
+        ws = _ws(need, W.device)
+    L.check(load().quip_incoherence_forward(tf.handle, _p(W), _dtype(W), W.stride(0), _p(W_t), _p(H),
+                                            _p(ws), 0 if ws is None else ws.numel(), _s(stream)),
+            "quip_incoherence_forward")
+
+
+def quip_incoherence_inverse(tf: Transform, W_hat_t: torch.Tensor, W_hat: torch.Tensor,
+                             ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    need = quip_workspace_size(L.QUIP_OP_INCOHERENCE_INVERSE, tf, tf.m, tf.n)
+    if ws is None:
+        ws = _ws(need, W_hat.device)
+    L.check(load().quip_incoherence_inverse(tf.handle, _p(W_hat_t), _p(W_hat), _p(ws),
+                                            0 if ws is None else ws.numel(), _s(stream)),
+            "quip_incoherence_inverse")
+
+
+def quip_ldl(H_t: torch.Tensor, D: torch.Tensor, ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    _cuda(H_t, "H_t")
+    n = H_t.shape[0]
+    need = quip_workspace_size(L.QUIP_OP_LDL, None, n, n)
+    if ws is None:
+        ws = _ws(need, H_t.device)
+    L.check(load().quip_ldl(_p(H_t), _p(D), n, _p(ws), 0 if ws is None else ws.numel(), _s(stream)),
+            "quip_ldl")
+
+
+def quip_ldlq_quantize(W_t: torch.Tensor, Uring: torch.Tensor, bits: int, block: int,
+                       codes: torch.Tensor, lo: torch.Tensor, scale: torch.Tensor,
+                       ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    m, n = W_t.shape
+    need = quip_workspace_size(L.QUIP_OP_LDLQ, None, m, n, block)
+    if ws is None:
+        ws = _ws(need, W_t.device)
+    L.check(load().quip_ldlq_quantize(_p(W_t), _p(Uring), Uring.stride(0), m, n, bits, block, _p(codes),
+                                      _p(lo), _p(scale), _p(ws), 0 if ws is None else ws.numel(),
+                                      _s(stream)), "quip_ldlq_quantize")
+
+
+def quip_dequantize(codes: torch.Tensor, lo: torch.Tensor, scale: torch.Tensor, W_hat_t: torch.Tensor,
+                    stream=None) -> None:
+    m, n = codes.shape
+    L.check(load().quip_dequantize(_p(codes), _p(lo), _p(scale), m, n, _p(W_hat_t), _s(stream)),
+            "quip_dequantize")
+
+
+def quip_sync_status(stream=None) -> int:
+    return load().quip_sync_status(_s(stream))
+
+
+@dataclass
+class LayerResult:
+    codes: torch.Tensor      # m x n uint8
+    lo: torch.Tensor         # m fp32
+    scale: torch.Tensor      # m fp32
+    W_hat: torch.Tensor      # m x n fp32, dequantised in the original basis
+
+
+class LayerQuantizer:
+    """Buffers and transform for quantising one m x n layer; ``run`` issues the
+    whole pipeline on one stream through the C ABI."""
+
+    def __init__(self, m: int, n: int, m_side, n_side, bits: int, block: int, damp: float = 0.01,
+                 seed: int = 0, device: str = "cuda", stream=None):
+        self.m, self.n, self.bits, self.block, self.damp, self.seed = m, n, bits, block, damp, seed
+        self.m_side, self.n_side = m_side, n_side
+        self.stream = stream
+        dev = torch.device(device)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.H = torch.empty(n, n, **f32)
+        self.W_t = torch.empty(m, n, **f32)
+        self.D = torch.empty(n, **f32)
+        self.codes = torch.empty(m, n, dtype=torch.uint8, device=dev)
+        self.lo = torch.empty(m, **f32)
+        self.scale = torch.empty(m, **f32)
+        self.W_hat = torch.empty(m, n, **f32)
+        self.tf: Optional[Transform] = None
+        ws = 0
+        probe = Transform(seed, m, n, m_side, n_side, stream)
+        for op, blk in ((L.QUIP_OP_INCOHERENCE_FORWARD, 0), (L.QUIP_OP_INCOHERENCE_INVERSE, 0),
+                        (L.QUIP_OP_LDL, 0), (L.QUIP_OP_LDLQ, block)):
+            ws = max(ws, quip_workspace_size(op, probe, m, n, blk))
+        self.tf = probe
+        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+
+    def new_transform(self) -> None:
+        """Draw (U, V) again from the seed on the device (part of a full pass)."""
+        self.tf.draw(self.seed, self.stream)
+
+    def run(self, W: torch.Tensor, X: torch.Tensor, redraw_transform: bool = True) -> LayerResult:
+        st = self.stream
+        if redraw_transform:
+            self.new_transform()
+        quip_hessian_accumulate(X, self.H, False, st)
+        quip_hessian_finalize(self.H, X.shape[0], self.damp, st)
+        quip_incoherence_forward(self.tf, W, self.W_t, self.H, self.ws, st)
+        quip_ldl(self.H, self.D, self.ws, st)
+        quip_ldlq_quantize(self.W_t, self.H, self.bits, self.block, self.codes, self.lo, self.scale,
+                           self.ws, st)
+        quip_dequantize(self.codes, self.lo, self.scale, self.W_hat, st)
+        quip_incoherence_inverse(self.tf, self.W_hat, self.W_hat, self.ws, st)
+        return LayerResult(self.codes, self.lo, self.scale, self.W_hat)
+
+    def run_host(self, W_host: torch.Tensor, X_host: torch.Tensor, codes_out: torch.Tensor,
+                 lo_out: torch.Tensor, scale_out: torch.Tensor) -> None:
+        """Host in, host out: copy W and X (pinned host tensors) to the device,
+        run the layer, copy codes / lo / scale back into the pinned outputs.
+        Everything is enqueued on the current stream; synchronise to read."""
+        if getattr(self, "_W_dev", None) is None or self._W_dev.shape != W_host.shape \
+                or self._W_dev.dtype != W_host.dtype:
+            self._W_dev = torch.empty_like(W_host, device="cuda")
+        if getattr(self, "_X_dev", None) is None or self._X_dev.shape != X_host.shape \
+                or self._X_dev.dtype != X_host.dtype:
+            self._X_dev = torch.empty_like(X_host, device="cuda")
+        self._W_dev.copy_(W_host, non_blocking=True)
+        self._X_dev.copy_(X_host, non_blocking=True)
+        r = self.run(self._W_dev, self._X_dev)
+        codes_out.copy_(r.codes, non_blocking=True)
+        lo_out.copy_(r.lo, non_blocking=True)
+        scale_out.copy_(r.scale, non_blocking=True)
+
+
+def quantize_layer(W: torch.Tensor, X: torch.Tensor, m_side, n_side, bits: int, block: int,
+                   damp: float = 0.01, seed: int = 0) -> LayerResult:
+    """Quantise one layer from host (or device) tensors; results come back to the host."""
+    q = LayerQuantizer(W.shape[0], W.shape[1], m_side, n_side, bits, block, damp, seed)
+    Wd = W.to("cuda", non_blocking=True)
+    Xd = X.to("cuda", non_blocking=True)
+    r = q.run(Wd, Xd)
+    st = quip_sync_status()
+    if st != L.QUIP_OK:
+        raise QuipError(st, "quantize_layer")
+    return LayerResult(r.codes.cpu(), r.lo.cpu(), r.scale.cpu(), r.W_hat.cpu())

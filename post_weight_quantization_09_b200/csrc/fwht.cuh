@@ -1,0 +1,245 @@
+// Randomized Hadamard transform (QuIP#, arXiv 2402.04396, abstract; QuIP,
+// incoherence-processing section): y = H_d diag(s) x / sqrt(d) with the
+// Sylvester H_d (H_1 = [1], H_2k = [[H_k, H_k], [H_k, -H_k]]).
+//
+// Two kernels, both HBM-bound (d log d add/sub per vector, one read and one
+// write of every element):
+//  * k_fwht_rows: transforms each contiguous row of a matrix.  A row of
+//    d = 2^L values is held by d/16 threads, 16 values each: the low 4 index
+//    bits are done in registers, the next 5 with warp shuffles, the rest
+//    (L > 9) after one transposition through shared memory, again in
+//    registers.  Loads and stores are 16-byte vectors / full 128-byte lines.
+//  * k_fwht_cols: mixes groups of g = 2^G rows (16 <= g <= 256) at a row
+//    stride, 32 columns per CTA; H_R = H_a (x) H_b lets a column transform of
+//    length R = a*b run as two such passes (inner rows then strided rows).
+// Optional sign vectors: pre (applied to the input index), post (applied to
+// the output index), and a per-row sign for the orthogonal direction.
+#pragma once
+
+#include "common.cuh"
+
+namespace quip {
+
+__device__ __forceinline__ void load16(const float* p, float (&v)[16]) {
+  const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 f = q[i];
+    v[4 * i] = f.x, v[4 * i + 1] = f.y, v[4 * i + 2] = f.z, v[4 * i + 3] = f.w;
+  }
+}
+__device__ __forceinline__ void load16(const __nv_bfloat16* p, float (&v)[16]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint4 u = q[i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
+      v[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+  }
+}
+
+// Butterflies over register index bits given by h = 1, 2, 4, ... < (1 << nbits).
+template <int NB, int N>
+__device__ __forceinline__ void reg_fwht(float (&v)[N]) {
+#pragma unroll
+  for (int h = 1; h < (1 << NB); h <<= 1) {
+#pragma unroll
+    for (int r = 0; r < N; ++r) {
+      if ((r & h) == 0) {
+        const float a = v[r], b = v[r + h];
+        v[r] = a + b;
+        v[r + h] = a - b;
+      }
+    }
+  }
+}
+
+// Padded shared-memory index (one pad word per 32) for the row kernel.
+__device__ __forceinline__ int pidx(int i) { return i + (i >> 5); }
+
+// rows x d matrix, d = 2^LOGN, 16 <= d <= 8192.  CTA = max(256, d/16)
+// threads; each group of d/16 threads owns one row.  In place allowed
+// (in == out with equal strides).
+template <int LOGN, typename TIn>
+__global__ void __launch_bounds__((1 << LOGN) / 16 > 256 ? (1 << LOGN) / 16 : 256)
+    k_fwht_rows(const TIn* in, int64_t ldin, float* out, int64_t ldout, int64_t rows,
+                const float* __restrict__ pre, const float* __restrict__ post,
+                const float* __restrict__ row_sign, float scale) {
+  constexpr int D = 1 << LOGN;
+  constexpr int T = D / 16;                           // threads per row
+  constexpr int NT = T > 256 ? T : 256;               // threads per CTA
+  constexpr int RPC = NT / T;                         // rows per CTA
+  constexpr int LB = (LOGN - 4) < 5 ? (LOGN - 4) : 5; // lane-bit stages
+  constexpr int W = LOGN > 9 ? LOGN - 9 : 0;          // stages after transpose
+  extern __shared__ float smem[];
+  const int t = threadIdx.x % T;
+  const int rl = threadIdx.x / T;
+  const int64_t row = (int64_t)blockIdx.x * RPC + rl;
+  const bool active = row < rows;
+  float v[16];
+  if (active) {
+    load16(in + row * ldin + 16 * t, v);
+    if (pre) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) v[r] *= pre[16 * t + r];
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < 16; ++r) v[r] = 0.f;
+  }
+  reg_fwht<4>(v);
+#pragma unroll
+  for (int b = 0; b < LB; ++b) {
+    const int mask = 1 << b;
+    const bool upper = (t & mask) != 0;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[r], mask);
+      v[r] = upper ? (o - v[r]) : (v[r] + o);
+    }
+  }
+  const float rs = (row_sign && active) ? row_sign[row] * scale : scale;
+  if constexpr (W == 0) {
+    if (active) {
+      float* o = out + row * ldout + 16 * t;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float4 f;
+        f.x = v[4 * q] * rs, f.y = v[4 * q + 1] * rs, f.z = v[4 * q + 2] * rs, f.w = v[4 * q + 3] * rs;
+        if (post) {
+          f.x *= post[16 * t + 4 * q], f.y *= post[16 * t + 4 * q + 1];
+          f.z *= post[16 * t + 4 * q + 2], f.w *= post[16 * t + 4 * q + 3];
+        }
+        reinterpret_cast<float4*>(o)[q] = f;
+      }
+    }
+  } else {
+    // D >= 1024: RPC = NT / T rows per CTA, each with its own padded slice.
+    float* sr = smem + rl * (D + D / 32);
+#pragma unroll
+    for (int r = 0; r < 16; ++r) sr[pidx(16 * t + r)] = v[r];
+    __syncthreads();
+    constexpr int NH = 1 << W;        // values of the high bits
+    constexpr int NK = 16 / NH;       // low-part values per thread
+#pragma unroll
+    for (int k = 0; k < NK; ++k)
+#pragma unroll
+      for (int h = 0; h < NH; ++h) v[k * NH + h] = sr[pidx(t + k * T + (h << 9))];
+    // butterflies over h (register bits 0..W-1 inside each k group)
+#pragma unroll
+    for (int hb = 1; hb < NH; hb <<= 1) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        if ((e & hb) == 0) {
+          const float a = v[e], b = v[e + hb];
+          v[e] = a + b;
+          v[e + hb] = a - b;
+        }
+      }
+    }
+    if (active) {
+      float* o = out + row * ldout;
+#pragma unroll
+      for (int k = 0; k < NK; ++k)
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          const int idx = t + k * T + (h << 9);
+          float x = v[k * NH + h] * rs;
+          if (post) x *= post[idx];
+          o[idx] = x;
+        }
+    }
+  }
+}
+
+// d < 16: one thread per row, everything in registers.
+template <typename TIn>
+__global__ void k_fwht_rows_small(const TIn* in, int64_t ldin, float* out, int64_t ldout,
+                                  int64_t rows, int d, const float* pre, const float* post,
+                                  const float* row_sign, float scale) {
+  const int64_t row = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (row >= rows) return;
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    v[i] = (i < d) ? to_f32<TIn>(in[row * ldin + i]) * (pre ? pre[i] : 1.f) : 0.f;
+  for (int h = 1; h < d; h <<= 1)
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < d && (i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+  const float rs = row_sign ? row_sign[row] * scale : scale;
+  for (int i = 0; i < d; ++i) out[row * ldout + i] = v[i] * rs * (post ? post[i] : 1.f);
+}
+
+// Column pass: for every base row b0 (u in [0, R/g): b0 = (u / gs) * g * gs + u % gs)
+// and every column c, transform the g values A[b0 + k*gs][c], k < g = 2^LOGG.
+// pre / post are indexed by the global row; scale multiplies the output.
+// CTA: 32 columns x (g/16) warps; thread (lane c, warp q) first holds
+// k = q + (g/16) r (high 4 bits in registers), then k = 16 q + r.
+template <int LOGG>
+__global__ void __launch_bounds__(32 * ((1 << LOGG) / 16))
+    k_fwht_cols(float* A, int64_t ld, int64_t ncols, int64_t gs, const float* __restrict__ pre,
+                const float* __restrict__ post, float scale) {
+  constexpr int G = 1 << LOGG;
+  constexpr int NW = G / 16;
+  constexpr int LOW = LOGG - 4;   // bits handled after the transposition
+  __shared__ float s[G][32];
+  const int c = threadIdx.x & 31, q = threadIdx.x >> 5;
+  const int64_t col = (int64_t)blockIdx.x * 32 + c;
+  const int64_t u = blockIdx.y;
+  const int64_t b0 = (u / gs) * (int64_t)G * gs + (u % gs);
+  const bool cok = col < ncols;
+  float v[16];
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    const int k = q + NW * r;
+    const int64_t grow = b0 + (int64_t)k * gs;
+    float x = cok ? A[grow * ld + col] : 0.f;
+    if (pre) x *= pre[grow];
+    v[r] = x;
+  }
+  reg_fwht<4>(v);     // high 4 bits of k
+#pragma unroll
+  for (int r = 0; r < 16; ++r) s[q + NW * r][c] = v[r];
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < 16; ++r) v[r] = s[16 * q + r][c];
+  if constexpr (LOW > 0) reg_fwht<LOW>(v);
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    const int k = 16 * q + r;
+    const int64_t grow = b0 + (int64_t)k * gs;
+    float x = v[r] * scale;
+    if (post) x *= post[grow];
+    if (cok) A[grow * ld + col] = x;
+  }
+}
+
+// R < 16 rows: one thread per column.
+__global__ void k_fwht_cols_small(float* A, int64_t ld, int64_t ncols, int R,
+                                  const float* pre, const float* post, float scale) {
+  const int64_t col = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (col >= ncols) return;
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = (i < R) ? A[i * ld + col] * (pre ? pre[i] : 1.f) : 0.f;
+  for (int h = 1; h < R; h <<= 1)
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < R && (i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+  for (int i = 0; i < R; ++i) A[i * ld + col] = v[i] * scale * (post ? post[i] : 1.f);
+}
+
+}  // namespace quip

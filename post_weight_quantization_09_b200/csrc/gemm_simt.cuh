@@ -1,0 +1,99 @@
+// Strided, batched fp32 FFMA GEMM on the CUDA cores:
+//   C_b[i][j] = alpha * sum_k A_b[i][k] * B_b[k][j] + beta * C_b[i][j]
+// with arbitrary element strides for every operand (so transposes are free).
+// Used where the contraction is small or must stay in fp32: the Kronecker
+// factors of the incoherence transform, the fp32-input Hessian, and the
+// trailing updates of the LDL and LDLQ steps.
+#pragma once
+
+#include "common.cuh"
+
+namespace quip {
+
+struct GemmArgs {
+  int64_t M, N, K;
+  float alpha, beta;              // beta == 0: C is not read
+  const void* A;
+  int64_t sam, sak, sab;          // A[b][i][k] = A[b*sab + i*sam + k*sak]
+  const void* B;
+  int64_t sbk, sbn, sbb;          // B[b][k][j] = B[b*sbb + k*sbk + j*sbn]
+  float* C;
+  int64_t scm, scn, scb;          // C[b][i][j]
+  int tri;                        // 0 all tiles, 1 tiles with ti >= tj, 2 ti <= tj
+};
+
+constexpr int SG_BM = 64, SG_BN = 64, SG_BK = 16;
+
+// 256 threads; each computes a 4 x 4 block of the 64 x 64 tile.
+template <typename TA, typename TB>
+__global__ void __launch_bounds__(256) k_gemm_simt(GemmArgs g) {
+  const int64_t ti = blockIdx.y, tj = blockIdx.x, b = blockIdx.z;
+  if (g.tri == 1 && ti < tj) return;
+  if (g.tri == 2 && ti > tj) return;
+  __shared__ float sA[SG_BK][SG_BM + 4];
+  __shared__ float sB[SG_BK][SG_BN + 4];
+  const TA* A = reinterpret_cast<const TA*>(g.A) + b * g.sab;
+  const TB* B = reinterpret_cast<const TB*>(g.B) + b * g.sbb;
+  float* C = g.C + b * g.scb;
+  const int tid = threadIdx.x;
+  const int tx = tid % 16, ty = tid / 16;
+  const int64_t i0 = ti * SG_BM, j0 = tj * SG_BN;
+  float acc[4][4] = {};
+  for (int64_t k0 = 0; k0 < g.K; k0 += SG_BK) {
+    // A tile 64 x 16 and B tile 16 x 64: 1024 elements each, 4 per thread.
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int idx = tid + e * 256;
+      {  // A: consecutive threads walk k first when A is k-contiguous
+        const int kk = (g.sak == 1) ? (idx % SG_BK) : (idx / SG_BM);
+        const int ii = (g.sak == 1) ? (idx / SG_BK) : (idx % SG_BM);
+        const int64_t gi = i0 + ii, gk = k0 + kk;
+        sA[kk][ii] = (gi < g.M && gk < g.K) ? to_f32<TA>(A[gi * g.sam + gk * g.sak]) : 0.f;
+      }
+      {
+        const int jj = (g.sbn == 1) ? (idx % SG_BN) : (idx / SG_BK);
+        const int kk = (g.sbn == 1) ? (idx / SG_BN) : (idx % SG_BK);
+        const int64_t gj = j0 + jj, gk = k0 + kk;
+        sB[kk][jj] = (gj < g.N && gk < g.K) ? to_f32<TB>(B[gk * g.sbk + gj * g.sbn]) : 0.f;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < SG_BK; ++kk) {
+      float a[4], bb[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) a[r] = sA[kk][ty + 16 * r];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) bb[c] = sB[kk][tx + 16 * c];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(a[r], bb[c], acc[r][c]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int64_t gi = i0 + ty + 16 * r;
+    if (gi >= g.M) continue;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int64_t gj = j0 + tx + 16 * c;
+      if (gj >= g.N) continue;
+      float* p = C + gi * g.scm + gj * g.scn;
+      const float v = g.alpha * acc[r][c];
+      *p = (g.beta == 0.f) ? v : fmaf(g.beta, *p, v);
+    }
+  }
+}
+
+template <typename TA, typename TB>
+inline cudaError_t gemm_simt(const GemmArgs& g, int64_t batch, cudaStream_t st) {
+  if (g.M <= 0 || g.N <= 0 || batch <= 0) return cudaSuccess;
+  dim3 grid((unsigned)((g.N + SG_BN - 1) / SG_BN), (unsigned)((g.M + SG_BM - 1) / SG_BM),
+            (unsigned)batch);
+  k_gemm_simt<TA, TB><<<grid, 256, 0, st>>>(g); count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace quip

@@ -1,0 +1,649 @@
+// libquip: the C ABI declared in include/quip.h, built as one translation
+// unit for sm_100a.  Host code here checks arguments, lays out workspace and
+// enqueues the kernels of the *.cuh files on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "fwht.cuh"
+#include "gemm_simt.cuh"
+#include "hessian.cuh"
+#include "ldl.cuh"
+#include "ldlq.cuh"
+#include "rng.cuh"
+#include "syrk_tc.cuh"
+
+using namespace quip;
+
+namespace {
+
+#define QCHECK(expr)                                 \
+  do {                                               \
+    cudaError_t e_ = (expr);                         \
+    if (e_ != cudaSuccess) return QUIP_ERR_CUDA;     \
+  } while (0)
+
+struct SideData {
+  int kind = QUIP_T_IDENTITY;
+  int64_t dim = 0, p = 0, q = 0;
+  float* signs = nullptr;   // HADAMARD
+  float* A = nullptr;       // KRONECKER p x p
+  float* B = nullptr;       // KRONECKER q x q
+  double* G = nullptr;      // KRONECKER: Gaussian draw scratch, max(p,q)^2
+  double* Qc = nullptr;     // KRONECKER: CGS2 scratch, max(p,q)^2
+};
+
+inline bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+inline int ilog2(int64_t x) {
+  int l = 0;
+  while ((int64_t(1) << l) < x) ++l;
+  return l;
+}
+inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------- TMA descriptors
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map with 64 x 64 boxes and the 128-byte swizzle.
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- Hadamard plans
+
+template <typename TIn>
+cudaError_t fwht_rows(const TIn* in, int64_t ldin, float* out, int64_t ldout, int64_t rows,
+                      int64_t d, const float* pre, const float* post, const float* row_sign,
+                      float scale, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  const int L = ilog2(d);
+  if (L < 4) {
+    k_fwht_rows_small<TIn><<<(unsigned)((rows + 127) / 128), 128, 0, st>>>(
+        in, ldin, out, ldout, rows, (int)d, pre, post, row_sign, scale); count_launch();
+    return cudaGetLastError();
+  }
+  const int T = (int)(d / 16);
+  const int NT = T > 256 ? T : 256;
+  const int RPC = NT / T;
+  const size_t smem = (L > 9) ? (size_t)RPC * (d + d / 32) * sizeof(float) : 0;
+  const unsigned grid = (unsigned)((rows + RPC - 1) / RPC);
+#define QUIP_ROWS_CASE(LL)                                                                    \
+  case LL:                                                                                    \
+    k_fwht_rows<LL, TIn><<<grid, NT, smem, st>>>(in, ldin, out, ldout, rows, pre, post,       \
+                                                 row_sign, scale); count_launch();                           \
+    break;
+  switch (L) {
+    QUIP_ROWS_CASE(4)
+    QUIP_ROWS_CASE(5)
+    QUIP_ROWS_CASE(6)
+    QUIP_ROWS_CASE(7)
+    QUIP_ROWS_CASE(8)
+    QUIP_ROWS_CASE(9)
+    QUIP_ROWS_CASE(10)
+    QUIP_ROWS_CASE(11)
+    QUIP_ROWS_CASE(12)
+    QUIP_ROWS_CASE(13)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef QUIP_ROWS_CASE
+  return cudaGetLastError();
+}
+
+cudaError_t fwht_cols_pass(float* A, int64_t ld, int64_t ncols, int64_t R, int LG, int64_t gs,
+                           const float* pre, const float* post, float scale, cudaStream_t st) {
+  dim3 grid((unsigned)((ncols + 31) / 32), (unsigned)(R >> LG));
+  const int threads = 32 * ((1 << LG) / 16);
+#define QUIP_COLS_CASE(LL)                                                                 \
+  case LL:                                                                                 \
+    k_fwht_cols<LL><<<grid, threads, 0, st>>>(A, ld, ncols, gs, pre, post, scale); count_launch();         \
+    break;
+  switch (LG) {
+    QUIP_COLS_CASE(4)
+    QUIP_COLS_CASE(5)
+    QUIP_COLS_CASE(6)
+    QUIP_COLS_CASE(7)
+    QUIP_COLS_CASE(8)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef QUIP_COLS_CASE
+  return cudaGetLastError();
+}
+
+// Column Hadamard of an R x ncols matrix (R = 2^L): H_R = H_outer (x) H_inner,
+// the inner factor on consecutive rows.  pre-sign on the first pass,
+// post-sign and the 1/sqrt(R) scale on the last.
+cudaError_t fwht_cols(float* A, int64_t ld, int64_t ncols, int64_t R, const float* pre,
+                      const float* post, cudaStream_t st) {
+  const int L = ilog2(R);
+  const float scale = (float)(1.0 / std::sqrt((double)R));
+  if (L < 4) {
+    k_fwht_cols_small<<<(unsigned)((ncols + 127) / 128), 128, 0, st>>>(A, ld, ncols, (int)R,
+                                                                        pre, post, scale); count_launch();
+    return cudaGetLastError();
+  }
+  if (L <= 8) return fwht_cols_pass(A, ld, ncols, R, L, 1, pre, post, scale, st);
+  const int Li = (L + 1) / 2, Lo = L - Li;
+  cudaError_t e = fwht_cols_pass(A, ld, ncols, R, Li, 1, pre, nullptr, 1.0f, st);
+  if (e != cudaSuccess) return e;
+  return fwht_cols_pass(A, ld, ncols, R, Lo, int64_t(1) << Li, nullptr, post, scale, st);
+}
+
+// ---------------------------------------------------------------- Kronecker plans
+
+// Rows: dst[i, :] = vec(A' Xr_i B'^T) for each row Xr_i (p x q view) of src,
+// with A' = A or A^T, B' = B or B^T (transpose = inverse transform).
+template <typename TIn>
+cudaError_t kron_rows(const TIn* src, int64_t ldsrc, float* dst, int64_t rows,
+                      const SideData& sd, bool transpose, float* tmp, cudaStream_t st) {
+  const int64_t p = sd.p, q = sd.q, n = p * q;
+  GemmArgs g{};
+  // tmp_i = Xr_i B'^T : M = p, N = q, K = q, batched over rows
+  g.M = p, g.N = q, g.K = q, g.alpha = 1.f, g.beta = 0.f, g.tri = 0;
+  g.A = src, g.sam = q, g.sak = 1, g.sab = ldsrc;
+  g.B = sd.B;
+  if (!transpose) g.sbk = 1, g.sbn = q;   // B'^T[k][j] = B[j][k]
+  else g.sbk = q, g.sbn = 1;              // (B^T)^T = B
+  g.sbb = 0;
+  g.C = tmp, g.scm = q, g.scn = 1, g.scb = n;
+  cudaError_t e = gemm_simt<TIn, float>(g, rows, st);
+  if (e != cudaSuccess) return e;
+  // dst_i = A' tmp_i : M = p, N = q, K = p
+  GemmArgs h{};
+  h.M = p, h.N = q, h.K = p, h.alpha = 1.f, h.beta = 0.f, h.tri = 0;
+  h.A = sd.A;
+  if (!transpose) h.sam = p, h.sak = 1;
+  else h.sam = 1, h.sak = p;
+  h.sab = 0;
+  h.B = tmp, h.sbk = q, h.sbn = 1, h.sbb = n;
+  h.C = dst, h.scm = q, h.scn = 1, h.scb = n;
+  return gemm_simt<float, float>(h, rows, st);
+}
+
+// Columns: X (R x ncols, R = p q) <- (A' (x) B') X, through tmp.
+cudaError_t kron_cols(float* X, int64_t ncols, const SideData& sd, bool transpose, float* tmp,
+                      cudaStream_t st) {
+  const int64_t p = sd.p, q = sd.q;
+  GemmArgs g{};
+  // tmp[a'] = B' X[a'] : batch p, M = q, N = ncols, K = q
+  g.M = q, g.N = ncols, g.K = q, g.alpha = 1.f, g.beta = 0.f, g.tri = 0;
+  g.A = sd.B;
+  if (!transpose) g.sam = q, g.sak = 1;
+  else g.sam = 1, g.sak = q;
+  g.sab = 0;
+  g.B = X, g.sbk = ncols, g.sbn = 1, g.sbb = q * ncols;
+  g.C = tmp, g.scm = ncols, g.scn = 1, g.scb = q * ncols;
+  cudaError_t e = gemm_simt<float, float>(g, p, st);
+  if (e != cudaSuccess) return e;
+  // X = A' tmp (tmp as p x (q ncols))
+  GemmArgs h{};
+  h.M = p, h.N = q * ncols, h.K = p, h.alpha = 1.f, h.beta = 0.f, h.tri = 0;
+  h.A = sd.A;
+  if (!transpose) h.sam = p, h.sak = 1;
+  else h.sam = 1, h.sak = p;
+  h.B = tmp, h.sbk = q * ncols, h.sbn = 1;
+  h.C = X, h.scm = q * ncols, h.scn = 1;
+  return gemm_simt<float, float>(h, 1, st);
+}
+
+__global__ void k_convert_rows_bf16(const __nv_bfloat16* in, int64_t ld, float* out, int64_t m,
+                                    int64_t n) {
+  const int64_t total = m * n;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x)
+    out[e] = __bfloat162float(in[(e / n) * ld + e % n]);
+}
+__global__ void k_copy_rows_f32(const float* in, int64_t ld, float* out, int64_t m, int64_t n) {
+  const int64_t total = m * n;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x)
+    out[e] = in[(e / n) * ld + e % n];
+}
+
+// n-side (row) transform of an m x n source into dst (row stride n).
+template <typename TIn>
+cudaError_t side_rows(const SideData& sd, bool inverse, const TIn* src, int64_t ldsrc, float* dst,
+                      int64_t rows, float* tmp, cudaStream_t st) {
+  const int64_t n = sd.dim;
+  if (sd.kind == QUIP_T_HADAMARD) {
+    const float scale = (float)(1.0 / std::sqrt((double)n));
+    // forward: y = H (s . x) / sqrt(n); inverse: x = s . (H y) / sqrt(n)
+    return fwht_rows<TIn>(src, ldsrc, dst, n, rows, n, inverse ? nullptr : sd.signs,
+                          inverse ? sd.signs : nullptr, nullptr, scale, st);
+  }
+  if (sd.kind == QUIP_T_KRONECKER) return kron_rows<TIn>(src, ldsrc, dst, rows, sd, inverse, tmp, st);
+  // identity
+  const unsigned grid = (unsigned)std::min<int64_t>((rows * n + 255) / 256, 65535 * 8);
+  if constexpr (std::is_same<TIn, float>::value) {
+    if ((const void*)src == (const void*)dst && ldsrc == n) return cudaSuccess;
+    k_copy_rows_f32<<<grid, 256, 0, st>>>(src, ldsrc, dst, rows, n); count_launch();
+  } else {
+    k_convert_rows_bf16<<<grid, 256, 0, st>>>(src, ldsrc, dst, rows, n); count_launch();
+  }
+  return cudaGetLastError();
+}
+
+// m-side (column) transform in place on X (R x ncols, row stride ncols).
+cudaError_t side_cols(const SideData& sd, bool inverse, float* X, int64_t ncols, float* tmp,
+                      cudaStream_t st) {
+  if (sd.kind == QUIP_T_HADAMARD)
+    return fwht_cols(X, ncols, ncols, sd.dim, inverse ? nullptr : sd.signs,
+                     inverse ? sd.signs : nullptr, st);
+  if (sd.kind == QUIP_T_KRONECKER) return kron_cols(X, ncols, sd, inverse, tmp, st);
+  return cudaSuccess;
+}
+
+}  // namespace
+
+struct quip_transform {
+  int device = 0;
+  int64_t m = 0, n = 0;
+  SideData side[2];
+};
+
+// ============================================================================
+extern "C" {
+
+const char* quip_status_string(int s) {
+  switch (s) {
+    case QUIP_OK: return "ok";
+    case QUIP_ERR_ARG: return "invalid argument";
+    case QUIP_ERR_SHAPE: return "invalid or unsupported shape";
+    case QUIP_ERR_UNSUPPORTED: return "unsupported";
+    case QUIP_ERR_NOT_PD: return "matrix not positive definite (LDL pivot <= 0)";
+    case QUIP_ERR_NONFINITE: return "non-finite value";
+    case QUIP_ERR_CUDA: return "CUDA error";
+    case QUIP_ERR_TIMEOUT: return "device-side wait timed out";
+    case QUIP_ERR_WORKSPACE: return "workspace too small or misaligned";
+    default: return "unknown status";
+  }
+}
+
+const char* quip_version(void) { return "quip-b200 0.1.0 sm_100a"; }
+
+uint64_t quip_kernel_launches(void) { return g_launch_count.load(); }
+
+static quip_status check_side(int kind, int64_t dim, int64_t p, int64_t q) {
+  if (dim <= 0) return QUIP_ERR_SHAPE;
+  if (kind == QUIP_T_IDENTITY) return QUIP_OK;
+  if (kind == QUIP_T_HADAMARD) return (is_pow2(dim) && dim >= 2 && dim <= 8192) ? QUIP_OK : QUIP_ERR_SHAPE;
+  if (kind == QUIP_T_KRONECKER)
+    return (p >= 1 && q >= 1 && p <= 256 && q <= 256 && p * q == dim) ? QUIP_OK : QUIP_ERR_SHAPE;
+  return QUIP_ERR_ARG;
+}
+
+static quip_status alloc_side(SideData& sd, int kind, int64_t dim, int64_t p, int64_t q) {
+  sd.kind = kind, sd.dim = dim, sd.p = p, sd.q = q;
+  if (kind == QUIP_T_HADAMARD) {
+    QCHECK(cudaMalloc(&sd.signs, dim * sizeof(float)));
+  } else if (kind == QUIP_T_KRONECKER) {
+    const int64_t mx = std::max(p, q);
+    QCHECK(cudaMalloc(&sd.A, p * p * sizeof(float)));
+    QCHECK(cudaMalloc(&sd.B, q * q * sizeof(float)));
+    QCHECK(cudaMalloc(&sd.G, mx * mx * sizeof(double)));
+    QCHECK(cudaMalloc(&sd.Qc, mx * mx * sizeof(double)));
+  }
+  return QUIP_OK;
+}
+
+// Draw one side's random data from `seed` into its existing buffers.
+static quip_status draw_side(const SideData& sd, uint64_t seed, int which, cudaStream_t st) {
+  if (sd.kind == QUIP_T_HADAMARD) {
+    k_random_signs<<<(unsigned)((sd.dim + 255) / 256), 256, 0, st>>>(sd.signs, sd.dim, seed,
+                                                                      which == 0 ? 0u : 1u);
+    count_launch();
+  } else if (sd.kind == QUIP_T_KRONECKER) {
+    const uint32_t sa = which == 0 ? 2u : 4u, sb = which == 0 ? 3u : 5u;
+    for (int f = 0; f < 2; ++f) {
+      const int64_t d = f == 0 ? sd.p : sd.q;
+      k_gaussian<<<(unsigned)((d * d + 255) / 256), 256, 0, st>>>(sd.G, d * d, seed, f == 0 ? sa : sb);
+      count_launch();
+      k_haar_cgs2<<<1, 256, 0, st>>>(sd.G, sd.Qc, f == 0 ? sd.A : sd.B, (int)d);
+      count_launch();
+    }
+  }
+  QCHECK(cudaGetLastError());
+  return QUIP_OK;
+}
+
+quip_status quip_transform_create(uint64_t seed, int64_t m, int64_t n, int m_kind, int64_t m_p,
+                                  int64_t m_q, int n_kind, int64_t n_p, int64_t n_q, void* stream,
+                                  quip_transform** out) {
+  if (!out) return QUIP_ERR_ARG;
+  *out = nullptr;
+  quip_status s;
+  if ((s = check_side(m_kind, m, m_p, m_q)) != QUIP_OK) return s;
+  if ((s = check_side(n_kind, n, n_p, n_q)) != QUIP_OK) return s;
+  quip_transform* tf = new quip_transform();
+  cudaGetDevice(&tf->device);
+  tf->m = m, tf->n = n;
+  if ((s = alloc_side(tf->side[0], m_kind, m, m_p, m_q)) != QUIP_OK ||
+      (s = alloc_side(tf->side[1], n_kind, n, n_p, n_q)) != QUIP_OK ||
+      (s = quip_transform_draw(tf, seed, stream)) != QUIP_OK) {
+    quip_transform_destroy(tf);
+    return s;
+  }
+  *out = tf;
+  return QUIP_OK;
+}
+
+quip_status quip_transform_draw(quip_transform* tf, uint64_t seed, void* stream) {
+  if (!tf) return QUIP_ERR_ARG;
+  quip_status s;
+  if ((s = draw_side(tf->side[0], seed, 0, S(stream))) != QUIP_OK) return s;
+  return draw_side(tf->side[1], seed, 1, S(stream));
+}
+
+quip_status quip_transform_destroy(quip_transform* tf) {
+  if (!tf) return QUIP_OK;
+  cudaDeviceSynchronize();
+  for (auto& sd : tf->side) {
+    cudaFree(sd.signs);
+    cudaFree(sd.A);
+    cudaFree(sd.B);
+    cudaFree(sd.G);
+    cudaFree(sd.Qc);
+  }
+  delete tf;
+  return QUIP_OK;
+}
+
+quip_status quip_transform_info(const quip_transform* tf, int side, int* kind, int64_t* p,
+                                int64_t* q, const float** signs, const float** A,
+                                const float** B) {
+  if (!tf || side < 0 || side > 1) return QUIP_ERR_ARG;
+  const SideData& sd = tf->side[side];
+  if (kind) *kind = sd.kind;
+  if (p) *p = sd.p;
+  if (q) *q = sd.q;
+  if (signs) *signs = sd.signs;
+  if (A) *A = sd.A;
+  if (B) *B = sd.B;
+  return QUIP_OK;
+}
+
+quip_status quip_hessian_accumulate(const void* X, int dtype, int64_t N, int64_t n, int64_t ldx,
+                                    float* H_acc, int accumulate, void* stream) {
+  if (!H_acc || (!X && N > 0)) return QUIP_ERR_ARG;
+  if (dtype != QUIP_F32 && dtype != QUIP_BF16) return QUIP_ERR_ARG;
+  if (n <= 0 || N < 0 || ldx < n || n > (int64_t)1 << 16 || N > ((int64_t)1 << 31) - 64)
+    return QUIP_ERR_SHAPE;
+  cudaStream_t st = S(stream);
+  if (N == 0) {
+    if (!accumulate) QCHECK(cudaMemsetAsync(H_acc, 0, n * n * sizeof(float), st));
+    return QUIP_OK;
+  }
+  const bool tma_ok = dtype == QUIP_BF16 && n >= 64 && (ldx % 8) == 0 &&
+                      (reinterpret_cast<uintptr_t>(X) % 16) == 0;
+  if (tma_ok) {
+    CUtensorMap map;
+    if (!make_tmap_bf16_2d(&map, X, (uint64_t)n, (uint64_t)N, (uint64_t)ldx * 2, 64, 64))
+      return QUIP_ERR_CUDA;
+    static bool attr = false;
+    if (!attr) {
+      QCHECK(cudaFuncSetAttribute(syrk::k_syrk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  syrk::SMEM_BYTES));
+      attr = true;
+    }
+    const int T = (int)((n + syrk::BT - 1) / syrk::BT);
+    syrk::k_syrk_tc<<<T * (T + 1) / 2, 256, syrk::SMEM_BYTES, st>>>(map, H_acc, (int)n, (int)N,
+                                                                     accumulate ? 1 : 0); count_launch();
+    QCHECK(cudaGetLastError());
+    return QUIP_OK;
+  }
+  GemmArgs g{};
+  g.M = n, g.N = n, g.K = N, g.alpha = 1.f, g.beta = accumulate ? 1.f : 0.f, g.tri = 1;
+  g.A = X, g.sam = 1, g.sak = ldx;        // A[i][t] = X[t][i]
+  g.B = X, g.sbk = ldx, g.sbn = 1;        // B[t][j] = X[t][j]
+  g.C = H_acc, g.scm = n, g.scn = 1;
+  if (dtype == QUIP_BF16) QCHECK((gemm_simt<__nv_bfloat16, __nv_bfloat16>(g, 1, st)));
+  else QCHECK((gemm_simt<float, float>(g, 1, st)));
+  return QUIP_OK;
+}
+
+quip_status quip_hessian_finalize(float* H, int64_t n, int64_t N_total, float damp, void* stream) {
+  if (!H) return QUIP_ERR_ARG;
+  if (n <= 0 || N_total < 1) return QUIP_ERR_SHAPE;
+  if (!(damp >= 0.f) || !std::isfinite(damp)) return QUIP_ERR_ARG;
+  cudaStream_t st = S(stream);
+  k_finalize_diag<<<1, 1024, 0, st>>>(H, n, 1.0 / (double)N_total, (double)damp); count_launch();
+  const unsigned T = (unsigned)((n + 31) / 32);
+  k_mirror_scale<<<dim3(T, T), 256, 0, st>>>(H, n, (float)(1.0 / (double)N_total)); count_launch();
+  QCHECK(cudaGetLastError());
+  return QUIP_OK;
+}
+
+quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int64_t n,
+                                int64_t block, size_t* bytes) {
+  if (!bytes) return QUIP_ERR_ARG;
+  *bytes = 0;
+  switch (op) {
+    case QUIP_OP_INCOHERENCE_FORWARD:
+    case QUIP_OP_INCOHERENCE_INVERSE: {
+      if (!tf) return QUIP_ERR_ARG;
+      const bool kron = tf->side[0].kind == QUIP_T_KRONECKER || tf->side[1].kind == QUIP_T_KRONECKER;
+      if (kron) {
+        size_t e = (size_t)tf->m * tf->n;
+        if (op == QUIP_OP_INCOHERENCE_FORWARD) e = std::max(e, (size_t)tf->n * tf->n);
+        *bytes = round256(e * sizeof(float));
+      }
+      return QUIP_OK;
+    }
+    case QUIP_OP_LDL:
+      return QUIP_OK;
+    case QUIP_OP_LDLQ:
+      if (m <= 0 || n <= 0 || block <= 0) return QUIP_ERR_SHAPE;
+      *bytes = round256((size_t)m * n * sizeof(float)) + round256((size_t)m * block * sizeof(float));
+      return QUIP_OK;
+    default:
+      return QUIP_ERR_ARG;
+  }
+}
+
+static quip_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (need == 0) return QUIP_OK;
+  if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255)) return QUIP_ERR_WORKSPACE;
+  return QUIP_OK;
+}
+
+quip_status quip_incoherence_forward(const quip_transform* tf, const void* W, int w_dtype,
+                                     int64_t ldw, float* W_t, float* H, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  if (!tf || !W || !W_t) return QUIP_ERR_ARG;
+  if (w_dtype != QUIP_F32 && w_dtype != QUIP_BF16) return QUIP_ERR_ARG;
+  const int64_t m = tf->m, n = tf->n;
+  if (ldw < n) return QUIP_ERR_SHAPE;
+  const SideData &U = tf->side[0], &V = tf->side[1];
+  if (V.kind == QUIP_T_HADAMARD && n >= 16) {   // vector loads in the row kernel
+    const size_t esz = w_dtype == QUIP_BF16 ? 2 : 4;
+    if ((reinterpret_cast<uintptr_t>(W) % 16) || ((ldw * esz) % 16)) return QUIP_ERR_ARG;
+  }
+  size_t need = 0;
+  quip_status s = quip_workspace_size(QUIP_OP_INCOHERENCE_FORWARD, tf, m, n, 0, &need);
+  if (s != QUIP_OK) return s;
+  if ((s = check_ws(ws, ws_bytes, need)) != QUIP_OK) return s;
+  cudaStream_t st = S(stream);
+  float* tmp = static_cast<float*>(ws);
+  if (w_dtype == QUIP_BF16)
+    QCHECK(side_rows<__nv_bfloat16>(V, false, static_cast<const __nv_bfloat16*>(W), ldw, W_t, m, tmp, st));
+  else
+    QCHECK(side_rows<float>(V, false, static_cast<const float*>(W), ldw, W_t, m, tmp, st));
+  QCHECK(side_cols(U, false, W_t, n, tmp, st));
+  if (H) {
+    QCHECK(side_rows<float>(V, false, H, n, H, n, tmp, st));   // H V^T
+    QCHECK(side_cols(V, false, H, n, tmp, st));                // V (H V^T)
+  }
+  return QUIP_OK;
+}
+
+quip_status quip_incoherence_inverse(const quip_transform* tf, const float* W_hat_t, float* W_hat,
+                                     void* ws, size_t ws_bytes, void* stream) {
+  if (!tf || !W_hat_t || !W_hat) return QUIP_ERR_ARG;
+  const int64_t m = tf->m, n = tf->n;
+  size_t need = 0;
+  quip_status s = quip_workspace_size(QUIP_OP_INCOHERENCE_INVERSE, tf, m, n, 0, &need);
+  if (s != QUIP_OK) return s;
+  if ((s = check_ws(ws, ws_bytes, need)) != QUIP_OK) return s;
+  cudaStream_t st = S(stream);
+  float* tmp = static_cast<float*>(ws);
+  QCHECK(side_rows<float>(tf->side[1], true, W_hat_t, n, W_hat, m, tmp, st));
+  QCHECK(side_cols(tf->side[0], true, W_hat, n, tmp, st));
+  return QUIP_OK;
+}
+
+namespace {
+__global__ void k_diag_to(const float* H, int64_t n, float* D) {
+  const int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (k < n) D[k] = H[k * n + k];
+}
+// Ů[j][k] = R[j][k] / R[k][k] for k > j (row j per CTA); D holds R_kk.
+__global__ void k_scale_upper(float* H, int64_t n, const float* D) {
+  const int64_t j = blockIdx.x;
+  for (int64_t k = j + 1 + threadIdx.x; k < n; k += blockDim.x) H[j * n + k] /= D[k];
+}
+__global__ void k_square(float* D, int64_t n) {
+  const int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (k < n) D[k] = D[k] * D[k];
+}
+}  // namespace
+
+quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (!H_t || !D) return QUIP_ERR_ARG;
+  if (n <= 0 || n > ((int64_t)1 << 16)) return QUIP_ERR_SHAPE;
+  cudaStream_t st = S(stream);
+  const int64_t P = (n + LDL_PB - 1) / LDL_PB;
+  for (int64_t p = P - 1; p >= 0; --p) {
+    const int64_t c0 = p * LDL_PB;
+    const int w = (int)std::min<int64_t>(LDL_PB, n - c0);
+    k_ldl_diag<<<1, 256, 0, st>>>(H_t, n, c0, w); count_launch();
+    if (c0 > 0) {
+      k_ldl_trsm<<<(unsigned)((c0 + 63) / 64), 64, 0, st>>>(H_t, n, c0, w); count_launch();
+      GemmArgs g{};
+      g.M = c0, g.N = c0, g.K = w, g.alpha = -1.f, g.beta = 1.f, g.tri = 2;
+      g.A = H_t + c0, g.sam = n, g.sak = 1;          // R[i][c0 + k]
+      g.B = H_t + c0, g.sbk = 1, g.sbn = n;          // R[j][c0 + k]
+      g.C = H_t, g.scm = n, g.scn = 1;
+      QCHECK((gemm_simt<float, float>(g, 1, st)));
+    }
+  }
+  k_diag_to<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(H_t, n, D); count_launch();
+  k_scale_upper<<<(unsigned)n, 256, 0, st>>>(H_t, n, D); count_launch();
+  k_square<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(D, n); count_launch();
+  QCHECK(cudaGetLastError());
+  return QUIP_OK;
+}
+
+quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu, int64_t m,
+                               int64_t n, int bits, int64_t block, uint8_t* codes, float* lo,
+                               float* scale, void* ws, size_t ws_bytes, void* stream) {
+  if (!W_t || !Uring || !codes || !lo || !scale) return QUIP_ERR_ARG;
+  if (bits < 1 || bits > 8) return QUIP_ERR_ARG;
+  if (m <= 0 || n <= 0 || ldu < n) return QUIP_ERR_SHAPE;
+  if (!(block == 32 || block == 64 || block == 128) || n % block) return QUIP_ERR_SHAPE;
+  size_t need = 0;
+  quip_status s = quip_workspace_size(QUIP_OP_LDLQ, nullptr, m, n, block, &need);
+  if (s != QUIP_OK) return s;
+  if ((s = check_ws(ws, ws_bytes, need)) != QUIP_OK) return s;
+  cudaStream_t st = S(stream);
+  float* A = static_cast<float*>(ws);
+  float* E = reinterpret_cast<float*>(static_cast<char*>(ws) + round256((size_t)m * n * sizeof(float)));
+  const int qmax = (1 << bits) - 1;
+  k_row_grid<<<(unsigned)((m + 7) / 8), 256, 0, st>>>(W_t, m, n, qmax, lo, scale); count_launch();
+  QCHECK(cudaMemcpyAsync(A, W_t, (size_t)m * n * sizeof(float), cudaMemcpyDeviceToDevice, st));
+  const size_t smem = (size_t)block * block * 4 + 32 * (block + 4) * 4 + 32 * block;
+  static bool attr[3] = {false, false, false};
+  auto launch = [&](int64_t k0) -> cudaError_t {
+    const unsigned grid = (unsigned)((m + 31) / 32);
+    switch (block) {
+      case 32:
+        k_ldlq_block<32><<<grid, 128, smem, st>>>(W_t, A, m, n, k0, Uring, ldu, lo, scale,
+                                                  (float)qmax, codes, E); count_launch();
+        break;
+      case 64:
+        k_ldlq_block<64><<<grid, 128, smem, st>>>(W_t, A, m, n, k0, Uring, ldu, lo, scale,
+                                                  (float)qmax, codes, E); count_launch();
+        break;
+      default:
+        if (!attr[2]) {
+          cudaFuncSetAttribute(k_ldlq_block<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+          attr[2] = true;
+        }
+        k_ldlq_block<128><<<grid, 128, smem, st>>>(W_t, A, m, n, k0, Uring, ldu, lo, scale,
+                                                   (float)qmax, codes, E); count_launch();
+    }
+    return cudaGetLastError();
+  };
+  for (int64_t k0 = 0; k0 < n; k0 += block) {
+    QCHECK(launch(k0));
+    const int64_t k1 = k0 + block;
+    if (k1 < n) {
+      GemmArgs g{};
+      g.M = m, g.N = n - k1, g.K = block, g.alpha = 1.f, g.beta = 1.f, g.tri = 0;
+      g.A = E, g.sam = block, g.sak = 1;
+      g.B = Uring + k0 * ldu + k1, g.sbk = ldu, g.sbn = 1;
+      g.C = A + k1, g.scm = n, g.scn = 1;
+      QCHECK((gemm_simt<float, float>(g, 1, st)));
+    }
+  }
+  return QUIP_OK;
+}
+
+quip_status quip_dequantize(const uint8_t* codes, const float* lo, const float* scale, int64_t m,
+                            int64_t n, float* W_hat_t, void* stream) {
+  if (!codes || !lo || !scale || !W_hat_t) return QUIP_ERR_ARG;
+  if (m <= 0 || n <= 0) return QUIP_ERR_SHAPE;
+  const int64_t total = m * n;
+  const unsigned grid = (unsigned)std::min<int64_t>((total / 4 + 255) / 256 + 1, 148 * 16);
+  k_dequant<<<grid, 256, 0, S(stream)>>>(codes, lo, scale, m, n, W_hat_t); count_launch();
+  QCHECK(cudaGetLastError());
+  return QUIP_OK;
+}
+
+quip_status quip_sync_status(void* stream) {
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return QUIP_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return QUIP_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return QUIP_ERR_CUDA;
+  return static_cast<quip_status>(v);
+}
+
+}  // extern "C"

@@ -1,0 +1,71 @@
+"""GPU parity at the full sizes of the Llama-shaped layers, in the launch
+configuration bench.py times (LayerQuantizer.run).  The FP64 oracle runs the
+same seeded layer on the host; where the whole oracle would take too long it
+runs on sampled rows (rows are independent once H~ and the transforms are
+fixed)."""
+import os
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import post_weight_quantization_09_b200 as Q
+from post_weight_quantization_09_b200 import _lib as L
+from quip_synth import CONFIGS, make_layer
+from parity_util import dev, host, ldlq_trajectory_check, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_device(cfg, d):
+    q = Q.LayerQuantizer(cfg.m, cfg.n, cfg.m_side, cfg.n_side, cfg.bits, cfg.block, cfg.damp, cfg.seed)
+    Wd = torch.from_numpy(d["W_bf16"].view(np.int16)).cuda().view(torch.bfloat16)
+    Xd = torch.from_numpy(d["X_bf16"].view(np.int16)).cuda().view(torch.bfloat16)
+    # H before LDL overwrites it: run the first stages separately to keep a copy
+    q.new_transform()
+    Q.quip_hessian_accumulate(Xd, q.H)
+    Q.quip_hessian_finalize(q.H, cfg.N, cfg.damp)
+    H_dev = host(q.H)
+    r = q.run(Wd, Xd)
+    assert Q.quip_sync_status() == L.QUIP_OK
+    return q, r, H_dev
+
+
+def test_attn7b_full_layer():
+    cfg = CONFIGS["attn7b"]
+    d = make_layer(cfg)
+    q, r, H_dev = _run_device(cfg, d)
+    t0 = time.time()
+    H = O.damp(O.hessian(d["X"]), cfg.damp)
+    h_err = rel_fro(H_dev, H)
+    assert h_err <= 1e-4, h_err
+    U = O.make_side(cfg.seed, "m", "hadamard", cfg.m)
+    V = O.make_side(cfg.seed, "n", "hadamard", cfg.n)
+    Wt, Ht = O.incoherence_forward(d["W"], H, U, V)
+    Uf, D = O.udu(Ht)
+    lo, s = O.row_grid(Wt, cfg.bits)
+    codes, Wt_hat, _ = O.ldlq(Wt, Uf, lo, s, cfg.bits)
+    loss = O.proxy_loss(Wt_hat, Wt, Ht)
+    C = host(r.codes)
+    lo_d, s_d = host(r.lo), host(r.scale)
+    agree = float((C == codes).mean())
+    Wt_hat_d = O.dequantize(C, lo_d, s_d)
+    loss_d = O.proxy_loss(Wt_hat_d, Wt, Ht)
+    same = C == codes
+    w_err = float(np.abs(Wt_hat_d - Wt_hat)[same].max() / s.max())
+    bad, not_near = ldlq_trajectory_check(C, Wt, Uf, lo_d, s_d, cfg.bits, tau=1e-3)
+    print(f"\nattn7b: H rel-Fro {h_err:.3e}  codes agree {agree:.6f}  loss {loss:.6g} vs {loss_d:.6g} "
+          f"(rel {abs(loss_d - loss) / loss:.2e})  W^ err/s {w_err:.2e}  trajectory mismatch {bad:.2e} "
+          f"(not near-tie {not_near:.2e})  oracle {time.time() - t0:.0f}s")
+    assert abs(loss_d - loss) / loss <= 1e-3
+    assert w_err <= 1e-4
+    assert agree >= 0.999
+    # sampled rows of the inverse transform: W^ = U^T W~^ V
+    rows = np.random.default_rng(0).choice(cfg.m, 16, replace=False)
+    Um, Vm = U.matrix(), V.matrix()
+    W_hat_d = host(r.W_hat)
+    for i in rows:
+        ref_row = (Um[:, i] @ Wt_hat_d) @ Vm          # row i of U^T W~^ V
+        assert np.abs(W_hat_d[i] - ref_row).max() <= 1e-4 * s_d.max()

@@ -1,0 +1,289 @@
+"""GPU parity, stage by stage: each CUDA stage, called through the C ABI on
+seeded inputs, against the FP64 oracle on the same inputs.  Sizes span
+several tiles with ragged tails; edge cases included."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import post_weight_quantization_09_b200 as Q
+from post_weight_quantization_09_b200 import _lib as L
+from quip_synth import CONFIGS, Side, make_layer, random_layer, round_to_bf16
+from parity_util import dev, host, ldlq_trajectory_check, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _status_clean():
+    Q.load()
+    Q.quip_sync_status()
+    yield
+    # no stage may leave a device-side error behind
+    assert Q.quip_sync_status() == L.QUIP_OK
+
+
+# ---------------------------------------------------------------- transforms
+
+
+@pytest.mark.parametrize("m,n,mk,nk", [
+    (64, 128, Side("hadamard"), Side("hadamard")),
+    (8, 2048, Side("hadamard"), Side("hadamard")),
+    (48, 86 * 3, Side("kronecker", 6, 8), Side("kronecker", 86, 3)),
+    (224, 32, Side("kronecker", 224, 1), Side("identity")),
+])
+def test_transform_factors_match_oracle(m, n, mk, nk):
+    tf = Q.Transform(1234, m, n, mk, nk)
+    for side, spec, dim in ((0, mk, m), (1, nk, n)):
+        f = tf.factors(side)
+        ref = O.make_side(1234, "m" if side == 0 else "n", spec.kind, dim, spec.p, spec.q)
+        if spec.kind == "hadamard":
+            np.testing.assert_array_equal(host(f["signs"]), ref.signs)
+        elif spec.kind == "kronecker":
+            np.testing.assert_allclose(host(f["A"]), ref.A, atol=2e-7)
+            np.testing.assert_allclose(host(f["B"]), ref.B, atol=2e-7)
+    tf.close()
+
+
+def test_transform_redraw_in_place():
+    tf = Q.Transform(1, 96, 64, Side("kronecker", 12, 8), Side("hadamard"))
+    tf.draw(99)
+    ref_m = O.make_side(99, "m", "kronecker", 96, 12, 8)
+    ref_n = O.make_side(99, "n", "hadamard", 64)
+    np.testing.assert_allclose(host(tf.factors(0)["A"]), ref_m.A, atol=2e-7)
+    np.testing.assert_array_equal(host(tf.factors(1)["signs"]), ref_n.signs)
+    tf.close()
+
+
+@pytest.mark.parametrize("m,n,mk,nk,dtype", [
+    (64, 128, Side("hadamard"), Side("hadamard"), "f32"),
+    (512, 1024, Side("hadamard"), Side("hadamard"), "bf16"),
+    (4096, 64, Side("hadamard"), Side("hadamard"), "bf16"),     # 2 column passes
+    (8, 8192, Side("hadamard"), Side("hadamard"), "f32"),       # largest row FWHT
+    (4, 8, Side("hadamard"), Side("hadamard"), "f32"),          # register-only paths
+    (96, 86 * 2, Side("kronecker", 12, 8), Side("kronecker", 86, 2), "bf16"),
+    (30, 64, Side("identity"), Side("hadamard"), "bf16"),
+])
+def test_incoherence_forward_inverse(m, n, mk, nk, dtype):
+    d = random_layer(m, n, min(4 * n, 2048), seed=m + n, dtype=dtype)
+    W, X = d["W"], d["X"]
+    H = O.damp(O.hessian(X), 0.01)
+    U = O.make_side(7, "m", mk.kind, m, mk.p, mk.q)
+    V = O.make_side(7, "n", nk.kind, n, nk.p, nk.q)
+    with_h = n <= 4096          # the explicit FP64 V H V^T is slow beyond that
+    Wt_ref, Ht_ref = O.incoherence_forward(W, H if with_h else np.eye(1), U, V) if with_h else \
+        (U.matrix() @ W @ V.matrix().T, None)
+    tf = Q.Transform(7, m, n, mk, nk)
+    Wd = dev(W, torch.bfloat16 if dtype == "bf16" else torch.float32)
+    Wt = torch.empty(m, n, device="cuda")
+    Hd = dev(H) if with_h else None
+    Q.quip_incoherence_forward(tf, Wd, Wt, Hd)
+    scale_w = np.abs(Wt_ref).max()
+    assert np.abs(host(Wt) - Wt_ref).max() <= 2e-6 * scale_w
+    if with_h:
+        assert rel_fro(host(Hd), Ht_ref) <= 2e-6
+    back = torch.empty_like(Wt)
+    Q.quip_incoherence_inverse(tf, Wt, back)
+    assert np.abs(host(back) - W).max() <= 4e-6 * np.abs(W).max()
+    Q.quip_incoherence_inverse(tf, Wt, Wt)                       # in place
+    assert np.abs(host(Wt) - W).max() <= 4e-6 * np.abs(W).max()
+    tf.close()
+
+
+# ---------------------------------------------------------------- Hessian
+
+
+@pytest.mark.parametrize("N,n,dtype", [
+    (1024, 128, "f32"), (1000, 320, "bf16"), (777, 576, "bf16"), (4096, 256, "bf16"),
+    (64, 64, "bf16"), (130, 40, "bf16"), (33, 7, "f32"),
+])
+def test_hessian_accumulate_and_finalize(N, n, dtype):
+    d = random_layer(4, n, N, seed=N + n, dtype=dtype, x_outlier_frac=0.05, lognormal=False)
+    X = d["X"]
+    ref = O.damp(O.hessian(X), 0.01)
+    Xd = dev(X, torch.bfloat16 if dtype == "bf16" else torch.float32)
+    H = torch.full((n, n), float("nan"), device="cuda")
+    Q.quip_hessian_accumulate(Xd, H)
+    # bf16 products are exact; the fp32 sums on the tensor cores lose up to
+    # about one ulp per 16-token MMA step, so the bound is the stated 1e-4
+    tol = 1e-4 if dtype == "bf16" else 1e-5
+    lower = np.tril(host(H))
+    assert rel_fro(lower, np.tril(X.astype(np.float64).T @ X)) <= tol
+    Q.quip_hessian_finalize(H, N, 0.01)
+    Hh = host(H)
+    np.testing.assert_array_equal(Hh, Hh.T)
+    assert rel_fro(Hh, ref) <= tol
+
+
+def test_hessian_streams_token_chunks():
+    d = random_layer(4, 320, 1500, seed=5, dtype="bf16", x_outlier_frac=0.02, lognormal=False)
+    X = d["X"]
+    Xd = dev(X, torch.bfloat16)
+    H = torch.empty(320, 320, device="cuda")
+    Q.quip_hessian_accumulate(Xd[:700], H, accumulate=False)
+    Q.quip_hessian_accumulate(Xd[700:1200], H, accumulate=True)
+    Q.quip_hessian_accumulate(Xd[1200:], H, accumulate=True)
+    Q.quip_hessian_finalize(H, 1500, 0.01)
+    assert rel_fro(host(H), O.damp(O.hessian(X), 0.01)) <= 1e-4
+
+
+def test_hessian_zero_tokens_and_strided_x():
+    H = torch.full((64, 64), 3.0, device="cuda")
+    Q.quip_hessian_accumulate(torch.empty(0, 64, dtype=torch.bfloat16, device="cuda"), H)
+    assert torch.all(torch.tril(H) == 0)
+    d = random_layer(4, 64, 256, seed=2, dtype="bf16")
+    big = torch.zeros(256, 128, dtype=torch.bfloat16, device="cuda")
+    big[:, :64] = dev(d["X"], torch.bfloat16)
+    Q.quip_hessian_accumulate(big[:, :64], H)                   # row stride 128
+    assert rel_fro(np.tril(host(H)), np.tril(d["X"].astype(np.float64).T @ d["X"])) <= 1e-4
+
+
+# ---------------------------------------------------------------- LDL
+
+
+@pytest.mark.parametrize("n", [16, 128, 200, 513])
+def test_ldl_matches_oracle(n):
+    rng = np.random.default_rng(n)
+    X = rng.standard_normal((3 * n, n)) * np.exp(rng.standard_normal(n))
+    H = O.damp(O.hessian(X), 0.01).astype(np.float32).astype(np.float64)
+    U_ref, D_ref = O.udu(H)
+    Hd = dev(H)
+    D = torch.empty(n, device="cuda")
+    Q.quip_ldl(Hd, D)
+    U = np.triu(host(Hd), 1)
+    # forward error within 10x of what an fp32 LAPACK factorisation reaches
+    J = np.arange(n)[::-1]
+    L32 = np.linalg.cholesky(H[np.ix_(J, J)].astype(np.float32)).astype(np.float64)
+    R32 = L32[np.ix_(J, J)]
+    U32 = np.triu(R32 / np.diag(R32)[None, :], 1)
+    err32 = np.abs(U32 - U_ref).max()
+    assert np.abs(U - U_ref).max() <= 10 * err32 + 1e-6
+    assert rel_fro(host(D), D_ref) <= 10 * rel_fro(np.diag(R32) ** 2, D_ref) + 1e-6
+    # backward error of the device factor, in FP64
+    R = (np.eye(n) + U) @ np.diag(host(D)) @ (np.eye(n) + U).T
+    assert rel_fro(R, H) <= 2e-6
+
+
+def test_ldl_diagonal_and_not_pd():
+    d = np.array([3.0, 1.0, 2.0, 5.0] * 20, dtype=np.float32)
+    Hd = dev(np.diag(d))
+    D = torch.empty(80, device="cuda")
+    Q.quip_ldl(Hd, D)
+    assert np.all(np.triu(host(Hd), 1) == 0)
+    np.testing.assert_allclose(host(D), d, rtol=1e-6)
+    bad = np.eye(70, dtype=np.float32)
+    bad[3, 5] = bad[5, 3] = 2.0                                  # indefinite
+    Q.quip_ldl(dev(bad), torch.empty(70, device="cuda"))
+    assert Q.quip_sync_status() == L.QUIP_ERR_NOT_PD
+
+
+# ---------------------------------------------------------------- LDLQ
+
+
+def _ldlq_inputs(m, n, seed, const_rows=()):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((2 * n, n))
+    X[:, rng.choice(n, max(1, n // 50), replace=False)] *= 20
+    H = O.damp(O.hessian(X), 0.01)
+    U, _ = O.udu(H)
+    W = rng.standard_normal((m, n)) * 0.02
+    for r in const_rows:
+        W[r] = 0.37
+    return W.astype(np.float32).astype(np.float64), U.astype(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("m,n,bits,block", [
+    (64, 128, 2, 32), (100, 256, 3, 64), (33, 256, 4, 128), (256, 128, 2, 128), (1, 64, 8, 64),
+    (70, 512, 2, 128),
+])
+def test_ldlq_stage_parity(m, n, bits, block):
+    W, U = _ldlq_inputs(m, n, seed=m * n + bits, const_rows=(0,) if m > 1 else ())
+    lo_ref, s_ref = O.row_grid(W, bits)
+    c_ref, _, _ = O.ldlq(W, U, lo_ref, s_ref, bits)
+    codes = torch.empty(m, n, dtype=torch.uint8, device="cuda")
+    lo = torch.empty(m, device="cuda")
+    sc = torch.empty(m, device="cuda")
+    Ud = dev(U)
+    Q.quip_ldlq_quantize(dev(W), Ud, bits, block, codes, lo, sc)
+    C = host(codes)
+    np.testing.assert_array_equal(host(lo), lo_ref)              # min is exact
+    np.testing.assert_allclose(host(sc), s_ref, rtol=3e-7)
+    agree = (C == c_ref).mean()
+    assert agree >= 0.999, agree
+    bad, not_near = ldlq_trajectory_check(C, W, U, host(lo), host(sc), bits, tau=1e-4)
+    assert not_near == 0.0, (bad, not_near)
+    if m > 1:
+        assert np.all(C[0] == 0)                                 # constant row: s = 1, codes 0
+
+
+def test_ldlq_identity_feedback_is_nearest():
+    rng = np.random.default_rng(3)
+    W = (rng.standard_normal((50, 128)) * 0.02).astype(np.float32)
+    codes = torch.empty(50, 128, dtype=torch.uint8, device="cuda")
+    lo = torch.empty(50, device="cuda")
+    sc = torch.empty(50, device="cuda")
+    Q.quip_ldlq_quantize(dev(W), torch.zeros(128, 128, device="cuda"), 3, 64, codes, lo, sc)
+    lo_h, s_h = host(lo), host(sc)
+    Wf = torch.tensor(W)
+    z = ((Wf - torch.tensor(lo_h, dtype=torch.float32)[:, None]) *
+         (1.0 / torch.tensor(s_h, dtype=torch.float32))[:, None])
+    want = torch.clamp(torch.round(z), 0, 7).numpy()
+    np.testing.assert_array_equal(host(codes), want)
+
+
+def test_ldlq_block_invariance_on_device():
+    W, U = _ldlq_inputs(128, 256, seed=11)
+    out = []
+    for block in (32, 64, 128):
+        codes = torch.empty(128, 256, dtype=torch.uint8, device="cuda")
+        lo, sc = torch.empty(128, device="cuda"), torch.empty(128, device="cuda")
+        Q.quip_ldlq_quantize(dev(W), dev(U), 2, block, codes, lo, sc)
+        out.append(host(codes))
+    assert (out[0] == out[1]).mean() >= 0.999 and (out[0] == out[2]).mean() >= 0.999
+
+
+def test_ldlq_nonfinite_weight_is_reported():
+    W = np.zeros((32, 64), dtype=np.float32)
+    W[5, 7] = np.nan
+    codes = torch.empty(32, 64, dtype=torch.uint8, device="cuda")
+    lo, sc = torch.empty(32, device="cuda"), torch.empty(32, device="cuda")
+    Q.quip_ldlq_quantize(dev(W), torch.zeros(64, 64, device="cuda"), 2, 32, codes, lo, sc)
+    assert Q.quip_sync_status() == L.QUIP_ERR_NONFINITE
+
+
+def test_dequantize_exact():
+    rng = np.random.default_rng(0)
+    C = rng.integers(0, 16, size=(37, 64)).astype(np.uint8)
+    lo = rng.standard_normal(37).astype(np.float32)
+    s = rng.uniform(0.01, 0.1, 37).astype(np.float32)
+    out = torch.empty(37, 64, device="cuda")
+    Q.quip_dequantize(dev(C, torch.uint8), dev(lo), dev(s), out)
+    want = O.dequantize(C, lo, s)
+    assert np.abs(host(out) - want).max() <= 1e-6 * np.abs(want).max()
+
+
+# ---------------------------------------------------------------- whole layer
+
+
+def test_tiny_config_pipeline():
+    cfg = CONFIGS["tiny"]
+    d = make_layer(cfg)
+    P = O.run_pipeline(d["W"], d["X"], cfg.seed, cfg.m_side, cfg.n_side, cfg.bits, cfg.damp)
+    q = Q.LayerQuantizer(cfg.m, cfg.n, cfg.m_side, cfg.n_side, cfg.bits, cfg.block, cfg.damp, cfg.seed)
+    r = q.run(dev(d["W"]), dev(d["X"]))
+    assert Q.quip_sync_status() == L.QUIP_OK
+    C = host(r.codes)
+    assert (C == P.codes).mean() >= 0.999
+    lo, s = host(r.lo), host(r.scale)
+    Wt_hat = O.dequantize(C, lo, s)
+    loss = O.proxy_loss(Wt_hat, P.Wt, P.Ht)
+    assert abs(loss - P.loss) / P.loss <= 1e-3
+    same = C == P.codes
+    assert np.abs(Wt_hat - P.Wt_hat)[same].max() <= 1e-4 * s.max()
+    # device inverse transform vs the oracle's inverse of the device codes
+    W_hat_ref = O.incoherence_inverse(Wt_hat, P.U, P.V)
+    assert np.abs(host(r.W_hat) - W_hat_ref).max() <= 1e-4 * s.max()
+    bad, not_near = ldlq_trajectory_check(C, P.Wt, P.Uf, lo, s, cfg.bits, tau=1e-3)
+    assert not_near == 0.0
