@@ -212,6 +212,38 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
                                uint8_t* codes, float* lo, float* scale, void* ws,
                                size_t ws_bytes, void* stream);
 
+/*
+ * Size of the device array quip_ldlq_quantize_static uses as its workspace.
+ */
+#define QUIP_LDLQ_STATIC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * quip_ldlq_quantize without a caller-supplied workspace and without any
+ * device allocation.  This entry point has no counterpart in the QuIP papers;
+ * it exists for callers that cannot call cudaMalloc: programs whose device
+ * memory is owned by a fixed pool or arena handed out by their own runtime,
+ * programs running under a hard memory cap, and latency-sensitive callers
+ * that must not trigger the device-wide synchronisation that cudaMalloc and
+ * cudaFree can cause.
+ *
+ * Same arguments, results and errors as quip_ldlq_quantize, minus (ws,
+ * ws_bytes).  The workspace is a fixed array of QUIP_LDLQ_STATIC_SCRATCH_BYTES
+ * in the library's own device memory, present on every GPU that loads the
+ * library until the process exits.  Layers whose workspace
+ * (quip_workspace_size(QUIP_OP_LDLQ, ...)) is larger are rejected with
+ * QUIP_ERR_WORKSPACE before anything is launched.
+ *  - The first call on each device looks up the array's device address for
+ *    that device (it must be the current device); make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one array and it keeps the last
+ *    call's contents; nothing in it needs to start at zero (every call
+ *    overwrites what it reads).  Calls whose work overlaps on the GPU
+ *    (different streams, or host threads) race on the array: order them.
+ */
+quip_status quip_ldlq_quantize_static(const float* W_t, const float* Uring, int64_t ldu,
+                                      int64_t m, int64_t n, int bits, int64_t block,
+                                      uint8_t* codes, float* lo, float* scale, void* stream);
+
 /* W_hat_t[i,j] = lo[i] + scale[i] * codes[i,j]  (device; m x n, row stride n). */
 quip_status quip_dequantize(const uint8_t* codes, const float* lo, const float* scale,
                             int64_t m, int64_t n, float* W_hat_t, void* stream);

@@ -36,6 +36,8 @@ SIGNATURES = {
     "quip_ldl": (c_int, [c_void_p, c_void_p, c_int64, c_void_p, c_size_t, c_void_p]),
     "quip_ldlq_quantize": (c_int, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int, c_int64,
                                    c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "quip_ldlq_quantize_static": (c_int, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int,
+                                          c_int64, c_void_p, c_void_p, c_void_p, c_void_p]),
     "quip_dequantize": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
     "quip_workspace_size": (c_int, [c_int, c_void_p, c_int64, c_int64, c_int64, POINTER(c_size_t)]),
     "quip_sync_status": (c_int, [c_void_p]),

@@ -626,6 +626,54 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
   return QUIP_OK;
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------- static scratch
+
+// Workspace of quip_ldlq_quantize_static: a fixed array in the library's own
+// device memory, so that entry point never allocates.  Host code may not use
+// the symbol as a pointer (on the host it is only a stand-in); its device
+// address is looked up once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_ldlq_scratch[QUIP_LDLQ_STATIC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+void* g_ldlq_scratch_ptr[kMaxDevices] = {};
+std::mutex g_ldlq_scratch_mu;
+
+// Device address of g_ldlq_scratch on the current device (looked up once).
+quip_status ldlq_static_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QUIP_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_ldlq_scratch_mu);
+  if (!g_ldlq_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_ldlq_scratch) != cudaSuccess || !p) return QUIP_ERR_CUDA;
+    g_ldlq_scratch_ptr[dev] = p;
+  }
+  *out = g_ldlq_scratch_ptr[dev];
+  return QUIP_OK;
+}
+}  // namespace
+
+extern "C" {
+
+quip_status quip_ldlq_quantize_static(const float* W_t, const float* Uring, int64_t ldu, int64_t m,
+                                      int64_t n, int bits, int64_t block, uint8_t* codes, float* lo,
+                                      float* scale, void* stream) {
+  size_t need = 0;
+  if (m > 0 && n > 0 && block > 0) {
+    quip_status s = quip_workspace_size(QUIP_OP_LDLQ, nullptr, m, n, block, &need);
+    if (s != QUIP_OK) return s;
+    if (need > (size_t)QUIP_LDLQ_STATIC_SCRATCH_BYTES) return QUIP_ERR_WORKSPACE;
+  }
+  void* ws = nullptr;
+  quip_status s = ldlq_static_scratch(&ws);
+  if (s != QUIP_OK) return s;
+  return quip_ldlq_quantize(W_t, Uring, ldu, m, n, bits, block, codes, lo, scale, ws,
+                            (size_t)QUIP_LDLQ_STATIC_SCRATCH_BYTES, stream);
+}
+
 quip_status quip_dequantize(const uint8_t* codes, const float* lo, const float* scale, int64_t m,
                             int64_t n, float* W_hat_t, void* stream) {
   if (!codes || !lo || !scale || !W_hat_t) return QUIP_ERR_ARG;
