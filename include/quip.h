@@ -181,7 +181,8 @@ quip_status quip_incoherence_inverse(const quip_transform* tf, const float* W_ha
  * LDL factorisation H_t = (I + Ů) diag(D) (I + Ů)^T with Ů strictly upper
  * triangular (the factorisation that defines LDLQ's feedback; QuIP,
  * adaptive-rounding section).  In place on H_t (n x n fp32, row stride n,
- * symmetric positive definite; only the upper triangle is read):
+ * symmetric positive definite; only the upper triangle is read; n % 4 == 0
+ * and H_t 16-byte aligned):
  * on return the strict upper triangle holds Ů, D (device, n fp32) the
  * pivots; the diagonal and lower triangle of H_t are unspecified.
  * A pivot <= 0 or non-finite sets QUIP_ERR_NOT_PD in the status word
@@ -201,9 +202,12 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
  * Evaluated in fp32, blocked over `block` columns (the result does not
  * depend on block in exact arithmetic).
  *   W_t   : device m x n fp32 (row stride n), not modified.
- *   Uring : device n x n fp32, row stride ldu >= n; only the strict upper
- *           triangle is read (the H_t buffer quip_ldl returned).
- *   bits  : 1..8.  block: 32, 64 or 128, with n % block == 0.
+ *   Uring : device n x n fp32, row stride ldu >= n (ldu % 4 == 0); only the
+ *           strict upper triangle is read (the H_t buffer quip_ldl returned).
+ *           W_t and Uring 16-byte aligned.
+ *   bits  : 1..8.  block: 32, 64 or 128, with n % block == 0; a performance
+ *           parameter (the result does not depend on it): 32 is processed in
+ *           64-column blocks and then also needs n % 64 == 0.
  *   codes : device m x n uint8 (row stride n).  lo, scale: device m fp32.
  * ws: QUIP_OP_LDLQ.
  */

@@ -1,0 +1,253 @@
+// fp32-accurate GEMM on the tcgen05 tensor cores from operands split into
+// three bf16 pieces:  x = x0 + x1 + x2 (x0 = bf16(x), x1 = bf16(x - x0),
+// x2 = bf16(x - x0 - x1)), so x is carried to ~24 significant bits.  The
+// product sum_k a_k b_k is formed from the six piece products whose order is
+// at most 2 (x_i y_j, i + j <= 2); the three dropped ones are below 2^-27
+// relative.  bf16 x bf16 products are exact in the fp32 accumulator.  The
+// terms run smallest first, (2,0) (1,1) (0,2) (1,0) (0,1) (0,0), so the
+// accumulator's own rounding acts on small partial sums for as long as
+// possible.
+//
+//   C[i][j] += alpha * sum_t sum_k A_pa(t)[i][k] * B_pb(t)[j][k]
+//
+// Both operands K-major (row-major [rows][K] bf16, piece p at row offset
+// p * piece_rows), loaded by TMA as 64-wide K boxes with the 128-byte swizzle.
+// Tile 128 x 256, one M=128 N=256 K=16 tcgen05.mma per 16 k, accumulators in
+// two 256-column TMEM buffers; 4-stage smem ring (48 KB per stage).
+// Bounded mbarrier waits as in the SYRK.
+#pragma once
+
+#include "common.cuh"
+
+namespace quip {
+namespace sgemm {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;              // 16 KB
+constexpr int B_BYTES = BN * BK * 2;              // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 48 KB
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr uint32_t IDESC = make_idesc_bf16(BM, BN, 0, 0);
+constexpr int NTERMS = 6;
+
+struct Params {
+  float* C;
+  int64_t ldc;
+  int M, N;                // output extent
+  int K;                   // K per piece (multiple of 64)
+  int a_piece_rows, b_piece_rows;   // row offset between pieces in the maps
+  int a_row0, b_row0;      // first row of the operand views in the maps
+  int a_k0, b_k0;          // first K column of the operand views
+  float alpha;
+  int upper_only;          // 1: skip tiles with no element i <= j (C square views)
+  int tiles_n;             // number of tile columns
+};
+
+struct Shared {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];       // accumulator buffer b ready (MMA -> epilogue)
+  uint64_t tempty[2];      // accumulator buffer b drained (epilogue -> MMA)
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ void term_pieces(int t, int& pa, int& pb) {
+  // (2,0) (1,1) (0,2) (1,0) (0,1) (0,0), one nibble per term
+  pa = (int)((0x001012u >> (4 * t)) & 0xFu);
+  pb = (int)((0x010210u >> (4 * t)) & 0xFu);
+}
+
+// Tile t of the grid (row-major over tiles_m x tiles_n); false if skipped.
+__device__ __forceinline__ bool tile_coords(const Params& p, int t, int& i0, int& j0) {
+  const int ti = t / p.tiles_n, tj = t % p.tiles_n;
+  i0 = ti * BM;
+  j0 = tj * BN;
+  return !(p.upper_only && i0 > j0 + BN - 1);
+}
+
+// Persistent: CTA b handles tiles b, b + gridDim.x, ...  Two accumulator
+// buffers of 256 TMEM columns let the epilogue of one tile run while the
+// tensor cores work on the next.  Warp 0 lane 0: TMA producer; warp 1
+// lane 0: MMA issuer; warps 4..7: epilogue (warp w reads TMEM lanes
+// 32 (w - 4).., one output row per thread, 256 columns in 8 chunks with the
+// result added to C with vector reductions).
+__global__ void __launch_bounds__(256, 1)
+    k_gemm_split_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    Params p, int ntiles) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Shared* sh = reinterpret_cast<Shared*>(smem + STAGES * STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kpp = p.K / BK;                         // K-steps per term
+  const int nkb = NTERMS * kpp;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&sh->full[s], 1);
+      mbar_init(&sh->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sh->tfull[b], 1);
+      mbar_init(&sh->tempty[b], 4);               // one arrival per epilogue warp
+    }
+    sh->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&sh->tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    int it = 0;                                   // global K-step counter (stage ring)
+    for (int t = blockIdx.x; t < ntiles && !sh->abort; t += gridDim.x) {
+      int i0, j0;
+      if (!tile_coords(p, t, i0, j0)) continue;
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
+        const int s = it % STAGES;
+        if (!mbar_wait(&sh->empty[s], (uint32_t)(((it / STAGES) & 1) ^ 1))) {
+          sh->abort = 1;
+          break;
+        }
+        int pa, pb;
+        term_pieces(kb / kpp, pa, pb);
+        const int kk = (kb % kpp) * BK;
+        uint8_t* a = smem + s * STAGE_BYTES;
+        mbar_arrive_expect_tx(&sh->full[s], STAGE_BYTES);
+        tma_load_2d(a, &tmA, &sh->full[s], p.a_k0 + kk, pa * p.a_piece_rows + p.a_row0 + i0);
+        tma_load_2d(a + A_BYTES, &tmB, &sh->full[s], p.b_k0 + kk, pb * p.b_piece_rows + p.b_row0 + j0);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    int it = 0, lt = 0;
+    for (int t = blockIdx.x; t < ntiles && !sh->abort; t += gridDim.x) {
+      int i0, j0;
+      if (!tile_coords(p, t, i0, j0)) continue;
+      const int b = lt & 1, use = lt >> 1;
+      if (!mbar_wait(&sh->tempty[b], (uint32_t)((use & 1) ^ 1))) {
+        sh->abort = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t acc = tmem + b * 256;
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
+        const int s = it % STAGES;
+        if (!mbar_wait(&sh->full[s], (uint32_t)((it / STAGES) & 1))) {
+          sh->abort = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
+        const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k) {
+          // K-major SW128: 8-row groups 1024 B apart; K advances 32 B per 16 elements
+          const uint64_t adesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
+          const uint64_t bdesc = make_sw128_desc(b_addr + k * 32, 16, 1024);
+          tc_mma_f16(acc, adesc, bdesc, IDESC, (kb | k) != 0);
+        }
+        tc_commit(&sh->empty[s]);
+      }
+      tc_commit(&sh->tfull[b]);
+      ++lt;
+    }
+  } else if (warp >= 4) {
+    const int quarter = warp - 4;
+    int lt = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      int i0, j0;
+      if (!tile_coords(p, t, i0, j0)) continue;
+      const int b = lt & 1, use = lt >> 1;
+      bool ok = mbar_wait(&sh->tfull[b], (uint32_t)(use & 1));
+      ok = __all_sync(0xffffffffu, ok) && !sh->abort;
+      if (!ok) break;
+      tc_fence_after();
+      const int row = i0 + quarter * 32 + lane;
+      const bool rok = row < p.M;
+      float* crow = p.C + (int64_t)(rok ? row : 0) * p.ldc;
+      const uint32_t tb = tmem + b * 256 + ((uint32_t)(quarter * 32) << 16);
+      const bool vec = (p.ldc & 3) == 0;
+      // C += alpha * acc through fire-and-forget vector reductions in L2: no
+      // read round trip; one addition per element per launch, so the result
+      // equals the plain read-add-write.
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        float v[32];
+        tmem_ld32(tb + c * 32, v);
+        const int jc = j0 + c * 32;
+        if (rok && jc < p.N) {
+          if (vec && jc + 32 <= p.N) {
+            float4* dst = reinterpret_cast<float4*>(crow + jc);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              atomicAdd(dst + q, make_float4(p.alpha * v[4 * q], p.alpha * v[4 * q + 1],
+                                             p.alpha * v[4 * q + 2], p.alpha * v[4 * q + 3]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (jc + e < p.N) atomicAdd(crow + jc + e, p.alpha * v[e]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->tempty[b]);
+      ++lt;
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace sgemm
+
+// fp32 -> three bf16 pieces, row-major copy: out[p][i][k] for p = 0..2.
+// Rows `rows`, K `cols` of the source (row stride lds); output row stride
+// ldo, piece stride piece_elems.
+__device__ __forceinline__ void split3(float x, __nv_bfloat16& p0, __nv_bfloat16& p1,
+                                       __nv_bfloat16& p2) {
+  p0 = __float2bfloat16_rn(x);
+  const float r1 = x - __bfloat162float(p0);
+  p1 = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(p1);
+  p2 = __float2bfloat16_rn(r2);
+}
+
+// out[p][j][i] = piece_p(U[i][j]) for i < j (strict upper), 0 otherwise:
+// the transposed, split copy of the LDL factor that LDLQ's trailing GEMM
+// reads as its K-major B operand.  32 x 32 tiles through shared memory.
+__global__ void __launch_bounds__(256) k_split_upper_transposed(const float* __restrict__ U,
+                                                                int64_t ldu, int64_t n,
+                                                                __nv_bfloat16* __restrict__ out) {
+  __shared__ float t[32][33];
+  const int64_t bi = blockIdx.y, bj = blockIdx.x;   // source tile (rows bi, cols bj)
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int r = ty; r < 32; r += 8) {
+    const int64_t i = bi * 32 + r, j = bj * 32 + tx;
+    t[r][tx] = (i < n && j < n && i < j) ? U[i * ldu + j] : 0.f;
+  }
+  __syncthreads();
+  const int64_t pn = n * n;
+  for (int r = ty; r < 32; r += 8) {
+    const int64_t j = bj * 32 + r, i = bi * 32 + tx;  // out row j, col i
+    if (i < n && j < n) {
+      __nv_bfloat16 p0, p1, p2;
+      split3(t[tx][r], p0, p1, p2);
+      out[j * n + i] = p0;
+      out[pn + j * n + i] = p1;
+      out[2 * pn + j * n + i] = p2;
+    }
+  }
+}
+
+}  // namespace quip

@@ -17,6 +17,7 @@
 #include "ldlq.cuh"
 #include "rng.cuh"
 #include "syrk_tc.cuh"
+#include "gemm_tc.cuh"
 
 using namespace quip;
 
@@ -81,6 +82,40 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint6
              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  return sms;
+}
+
+// C (+)= alpha * (3-piece A) (3-piece B)^T on the tensor cores; see gemm_tc.cuh.
+cudaError_t split_gemm(const CUtensorMap& ta, const CUtensorMap& tb, sgemm::Params p,
+                       cudaStream_t st) {
+  if (p.M <= 0 || p.N <= 0) return cudaSuccess;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(sgemm::k_gemm_split_tc,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         sgemm::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int tm = (p.M + sgemm::BM - 1) / sgemm::BM, tn = (p.N + sgemm::BN - 1) / sgemm::BN;
+  p.tiles_n = tn;
+  int valid = 0;                      // tiles that survive the upper-only filter
+  for (int ti = 0; ti < tm; ++ti)
+    for (int tj = 0; tj < tn; ++tj)
+      if (!(p.upper_only && ti * sgemm::BM > tj * sgemm::BN + sgemm::BN - 1)) ++valid;
+  const int grid = std::max(1, std::min(valid, num_sms()));
+  sgemm::k_gemm_split_tc<<<grid, 256, sgemm::SMEM_BYTES, st>>>(ta, tb, p, tm * tn); count_launch();
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- Hadamard plans
@@ -448,6 +483,18 @@ quip_status quip_hessian_finalize(float* H, int64_t n, int64_t N_total, float da
   return QUIP_OK;
 }
 
+// LDL workspace: Rinv (128 x 128 fp32), then the panel's three bf16 pieces (3 x n x 128).
+static size_t ldl_ws_bytes(int64_t n) {
+  return round256((size_t)LDL_PB * LDL_PB * 4) + round256((size_t)3 * n * LDL_PB * 2);
+}
+// LDLQ workspace: accumulator A (m x n fp32), the error of every column as
+// three bf16 pieces (3 x m x n), the split transposed factor (3 x n x n bf16).
+static size_t ldlq_ws_bytes(int64_t m, int64_t n, int64_t block) {
+  (void)block;
+  return round256((size_t)m * n * 4) + round256((size_t)3 * m * n * 2) +
+         round256((size_t)3 * n * n * 2);
+}
+
 quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int64_t n,
                                 int64_t block, size_t* bytes) {
   if (!bytes) return QUIP_ERR_ARG;
@@ -465,10 +512,12 @@ quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int
       return QUIP_OK;
     }
     case QUIP_OP_LDL:
+      if (n <= 0) return QUIP_ERR_SHAPE;
+      *bytes = ldl_ws_bytes(n);
       return QUIP_OK;
     case QUIP_OP_LDLQ:
       if (m <= 0 || n <= 0 || block <= 0) return QUIP_ERR_SHAPE;
-      *bytes = round256((size_t)m * n * sizeof(float)) + round256((size_t)m * block * sizeof(float));
+      *bytes = ldlq_ws_bytes(m, n, block);
       return QUIP_OK;
     default:
       return QUIP_ERR_ARG;
@@ -543,24 +592,39 @@ __global__ void k_square(float* D, int64_t n) {
 }  // namespace
 
 quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes, void* stream) {
-  (void)ws;
-  (void)ws_bytes;
   if (!H_t || !D) return QUIP_ERR_ARG;
   if (n <= 0 || n > ((int64_t)1 << 16)) return QUIP_ERR_SHAPE;
+  if ((n & 3) || (reinterpret_cast<uintptr_t>(H_t) & 15)) return QUIP_ERR_SHAPE;
+  quip_status s = check_ws(ws, ws_bytes, ldl_ws_bytes(n));
+  if (s != QUIP_OK) return s;
   cudaStream_t st = S(stream);
+  __nv_bfloat16* Rs = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) +
+                                                       round256((size_t)LDL_PB * LDL_PB * 4));
+  const size_t smem_panel = ((size_t)(LDL_PB + 64) * LDL_LD + 4 * 32 * 33) * sizeof(float);
+  static bool attr = false;
+  if (!attr) {
+    QCHECK(cudaFuncSetAttribute(k_ldl_panel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem_panel));
+    attr = true;
+  }
+  CUtensorMap ta, tb;
+  if (n > LDL_PB) {
+    if (!make_tmap_bf16_2d(&ta, Rs, LDL_PB, 3 * (uint64_t)n, LDL_PB * 2, 64, sgemm::BM) ||
+        !make_tmap_bf16_2d(&tb, Rs, LDL_PB, 3 * (uint64_t)n, LDL_PB * 2, 64, sgemm::BN))
+      return QUIP_ERR_CUDA;
+  }
   const int64_t P = (n + LDL_PB - 1) / LDL_PB;
   for (int64_t p = P - 1; p >= 0; --p) {
     const int64_t c0 = p * LDL_PB;
     const int w = (int)std::min<int64_t>(LDL_PB, n - c0);
-    k_ldl_diag<<<1, 256, 0, st>>>(H_t, n, c0, w); count_launch();
+    const unsigned grid = (unsigned)std::max<int64_t>(1, (c0 + 63) / 64);
+    k_ldl_panel<<<grid, 256, smem_panel, st>>>(H_t, n, c0, w, Rs); count_launch();
     if (c0 > 0) {
-      k_ldl_trsm<<<(unsigned)((c0 + 63) / 64), 64, 0, st>>>(H_t, n, c0, w); count_launch();
-      GemmArgs g{};
-      g.M = c0, g.N = c0, g.K = w, g.alpha = -1.f, g.beta = 1.f, g.tri = 2;
-      g.A = H_t + c0, g.sam = n, g.sak = 1;          // R[i][c0 + k]
-      g.B = H_t + c0, g.sbk = 1, g.sbn = n;          // R[j][c0 + k]
-      g.C = H_t, g.scm = n, g.scn = 1;
-      QCHECK((gemm_simt<float, float>(g, 1, st)));
+      // H[:c0, :c0] -= R12 R12^T on the upper tiles
+      sgemm::Params gp{};
+      gp.C = H_t, gp.ldc = n, gp.M = (int)c0, gp.N = (int)c0, gp.K = LDL_PB;
+      gp.a_piece_rows = (int)n, gp.b_piece_rows = (int)n, gp.alpha = -1.f, gp.upper_only = 1;
+      QCHECK(split_gemm(ta, tb, gp, st));
     }
   }
   k_diag_to<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(H_t, n, D); count_launch();
@@ -570,6 +634,54 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
   return QUIP_OK;
 }
 
+namespace {
+struct LdlqRun {
+  const float* Wt;
+  float* A;
+  const float* U;
+  int64_t ldu, m, n, B;
+  const float* lo;
+  const float* sc;
+  float qmax;
+  uint8_t* codes;
+  __nv_bfloat16* Es;
+  CUtensorMap ta, tb;
+  size_t smem;
+  cudaStream_t st;
+};
+
+cudaError_t ldlq_block(const LdlqRun& r, int64_t k0) {
+  const unsigned grid = (unsigned)((r.m + 15) / 16);
+  if (r.B == 64)
+    k_ldlq_chunk8<64><<<grid, 128, r.smem, r.st>>>(r.Wt, r.A, r.m, r.n, k0, r.U, r.ldu, r.lo, r.sc,
+                                                   r.qmax, r.codes, r.Es, r.n);
+  else
+    k_ldlq_chunk8<128><<<grid, 128, r.smem, r.st>>>(r.Wt, r.A, r.m, r.n, k0, r.U, r.ldu, r.lo, r.sc,
+                                                    r.qmax, r.codes, r.Es, r.n);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// Columns [a, b): left half, then A[:, mid:b] += Err[:, a:mid] Ů[a:mid, mid:b]
+// in one split GEMM, then the right half.  Every column's feedback is the
+// same sum as in the column-by-column definition, grouped differently.
+cudaError_t ldlq_range(const LdlqRun& r, int64_t a, int64_t b) {
+  const int64_t nb = (b - a) / r.B;
+  if (nb <= 1) return ldlq_block(r, a);
+  const int64_t mid = a + ((nb + 1) / 2) * r.B;
+  cudaError_t e = ldlq_range(r, a, mid);
+  if (e != cudaSuccess) return e;
+  sgemm::Params gp{};
+  gp.C = r.A + mid, gp.ldc = r.n, gp.M = (int)r.m, gp.N = (int)(b - mid), gp.K = (int)(mid - a);
+  gp.a_piece_rows = (int)r.m, gp.a_k0 = (int)a;
+  gp.b_piece_rows = (int)r.n, gp.b_row0 = (int)mid, gp.b_k0 = (int)a;
+  gp.alpha = 1.f;
+  e = split_gemm(r.ta, r.tb, gp, r.st);
+  if (e != cudaSuccess) return e;
+  return ldlq_range(r, mid, b);
+}
+}  // namespace
+
 quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu, int64_t m,
                                int64_t n, int bits, int64_t block, uint8_t* codes, float* lo,
                                float* scale, void* ws, size_t ws_bytes, void* stream) {
@@ -577,52 +689,47 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
   if (bits < 1 || bits > 8) return QUIP_ERR_ARG;
   if (m <= 0 || n <= 0 || ldu < n) return QUIP_ERR_SHAPE;
   if (!(block == 32 || block == 64 || block == 128) || n % block) return QUIP_ERR_SHAPE;
-  size_t need = 0;
-  quip_status s = quip_workspace_size(QUIP_OP_LDLQ, nullptr, m, n, block, &need);
+  // 32-column blocks are processed as 64-column blocks (same result)
+  const int64_t B = block < 64 ? 64 : block;
+  if (n % B) return QUIP_ERR_SHAPE;
+  if (m > ((int64_t)1 << 20) || n > ((int64_t)1 << 16)) return QUIP_ERR_SHAPE;
+  if ((ldu & 3) || (reinterpret_cast<uintptr_t>(Uring) & 15) || (reinterpret_cast<uintptr_t>(W_t) & 15))
+    return QUIP_ERR_ARG;
+  quip_status s = check_ws(ws, ws_bytes, ldlq_ws_bytes(m, n, block));
   if (s != QUIP_OK) return s;
-  if ((s = check_ws(ws, ws_bytes, need)) != QUIP_OK) return s;
-  cudaStream_t st = S(stream);
-  float* A = static_cast<float*>(ws);
-  float* E = reinterpret_cast<float*>(static_cast<char*>(ws) + round256((size_t)m * n * sizeof(float)));
-  const int qmax = (1 << bits) - 1;
-  k_row_grid<<<(unsigned)((m + 7) / 8), 256, 0, st>>>(W_t, m, n, qmax, lo, scale); count_launch();
-  QCHECK(cudaMemcpyAsync(A, W_t, (size_t)m * n * sizeof(float), cudaMemcpyDeviceToDevice, st));
-  const size_t smem = (size_t)block * block * 4 + 32 * (block + 4) * 4 + 32 * block;
-  static bool attr[3] = {false, false, false};
-  auto launch = [&](int64_t k0) -> cudaError_t {
-    const unsigned grid = (unsigned)((m + 31) / 32);
-    switch (block) {
-      case 32:
-        k_ldlq_block<32><<<grid, 128, smem, st>>>(W_t, A, m, n, k0, Uring, ldu, lo, scale,
-                                                  (float)qmax, codes, E); count_launch();
-        break;
-      case 64:
-        k_ldlq_block<64><<<grid, 128, smem, st>>>(W_t, A, m, n, k0, Uring, ldu, lo, scale,
-                                                  (float)qmax, codes, E); count_launch();
-        break;
-      default:
-        if (!attr[2]) {
-          cudaFuncSetAttribute(k_ldlq_block<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem);
-          attr[2] = true;
-        }
-        k_ldlq_block<128><<<grid, 128, smem, st>>>(W_t, A, m, n, k0, Uring, ldu, lo, scale,
-                                                   (float)qmax, codes, E); count_launch();
-    }
-    return cudaGetLastError();
-  };
-  for (int64_t k0 = 0; k0 < n; k0 += block) {
-    QCHECK(launch(k0));
-    const int64_t k1 = k0 + block;
-    if (k1 < n) {
-      GemmArgs g{};
-      g.M = m, g.N = n - k1, g.K = block, g.alpha = 1.f, g.beta = 1.f, g.tri = 0;
-      g.A = E, g.sam = block, g.sak = 1;
-      g.B = Uring + k0 * ldu + k1, g.sbk = ldu, g.sbn = 1;
-      g.C = A + k1, g.scm = n, g.scn = 1;
-      QCHECK((gemm_simt<float, float>(g, 1, st)));
-    }
+  LdlqRun r{};
+  r.st = S(stream);
+  char* w8 = static_cast<char*>(ws);
+  r.A = reinterpret_cast<float*>(w8);
+  w8 += round256((size_t)m * n * 4);
+  r.Es = reinterpret_cast<__nv_bfloat16*>(w8);
+  w8 += round256((size_t)3 * m * n * 2);
+  __nv_bfloat16* UTs = reinterpret_cast<__nv_bfloat16*>(w8);
+  r.Wt = W_t, r.U = Uring, r.ldu = ldu, r.m = m, r.n = n, r.B = B, r.lo = lo, r.sc = scale;
+  r.qmax = (float)((1 << bits) - 1), r.codes = codes;
+  k_row_grid<<<(unsigned)((m + 7) / 8), 256, 0, r.st>>>(W_t, m, n, (1 << bits) - 1, lo, scale);
+  count_launch();
+  QCHECK(cudaMemcpyAsync(r.A, W_t, (size_t)m * n * sizeof(float), cudaMemcpyDeviceToDevice, r.st));
+  if (n > B) {
+    const unsigned T = (unsigned)((n + 31) / 32);
+    k_split_upper_transposed<<<dim3(T, T), 256, 0, r.st>>>(Uring, ldu, n, UTs); count_launch();
+    if (!make_tmap_bf16_2d(&r.ta, r.Es, (uint64_t)n, 3 * (uint64_t)m, (uint64_t)n * 2, 64, sgemm::BM) ||
+        !make_tmap_bf16_2d(&r.tb, UTs, (uint64_t)n, 3 * (uint64_t)n, (uint64_t)n * 2, 64, sgemm::BN))
+      return QUIP_ERR_CUDA;
   }
+  auto smem_for = [](int64_t b) {
+    return ((size_t)b * 8 * (b / 8 + 4) + 16 * (b + 4)) * 4 + 16 * b;
+  };
+  r.smem = smem_for(B);
+  static bool attr = false;
+  if (!attr) {
+    QCHECK(cudaFuncSetAttribute(k_ldlq_chunk8<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem_for(64)));
+    QCHECK(cudaFuncSetAttribute(k_ldlq_chunk8<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem_for(128)));
+    attr = true;
+  }
+  QCHECK(ldlq_range(r, 0, n));
   return QUIP_OK;
 }
 

@@ -157,6 +157,7 @@ __global__ void __launch_bounds__(256, 1)
             dst[q] = f;
           }
         } else {
+#pragma unroll
           for (int e = 0; e < 32; ++e)
             if (jc + e < n) hrow[jc + e] = accumulate ? hrow[jc + e] + v[e] : v[e];
         }

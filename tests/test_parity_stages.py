@@ -143,7 +143,7 @@ def test_hessian_zero_tokens_and_strided_x():
 # ---------------------------------------------------------------- LDL
 
 
-@pytest.mark.parametrize("n", [16, 128, 200, 513])
+@pytest.mark.parametrize("n", [16, 128, 200, 516])
 def test_ldl_matches_oracle(n):
     rng = np.random.default_rng(n)
     X = rng.standard_normal((3 * n, n)) * np.exp(rng.standard_normal(n))
@@ -166,6 +166,12 @@ def test_ldl_matches_oracle(n):
     assert rel_fro(R, H) <= 2e-6
 
 
+def test_ldl_rejects_unaligned_order():
+    with pytest.raises(Q.QuipError) as e:
+        Q.quip_ldl(torch.eye(513, device="cuda"), torch.empty(513, device="cuda"))
+    assert e.value.status == L.QUIP_ERR_SHAPE
+
+
 def test_ldl_diagonal_and_not_pd():
     d = np.array([3.0, 1.0, 2.0, 5.0] * 20, dtype=np.float32)
     Hd = dev(np.diag(d))
@@ -173,9 +179,9 @@ def test_ldl_diagonal_and_not_pd():
     Q.quip_ldl(Hd, D)
     assert np.all(np.triu(host(Hd), 1) == 0)
     np.testing.assert_allclose(host(D), d, rtol=1e-6)
-    bad = np.eye(70, dtype=np.float32)
+    bad = np.eye(72, dtype=np.float32)
     bad[3, 5] = bad[5, 3] = 2.0                                  # indefinite
-    Q.quip_ldl(dev(bad), torch.empty(70, device="cuda"))
+    Q.quip_ldl(dev(bad), torch.empty(72, device="cuda"))
     assert Q.quip_sync_status() == L.QUIP_ERR_NOT_PD
 
 
