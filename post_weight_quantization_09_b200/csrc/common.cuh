@@ -9,6 +9,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 

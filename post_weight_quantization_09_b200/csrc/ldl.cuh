@@ -24,15 +24,16 @@ constexpr int LDL_LD = LDL_PB + 1;     // padded shared-memory row
 
 // ---------------------------------------------------------------- warp-level 32 x 32 blocks
 
-// Backward Cholesky and inverse of a 32 x 32 block in one sweep, one warp.
-// Lane i keeps row i of A (a[]) and column i of X = R^-1 (x[]).  At step k
-// (31 .. 0) row k of R is complete; lane k publishes it, every lane j then
-// forms x_kj = (delta_kj - sum_{m>k} R_km x_mj) / R_kk, and the leading
-// block is updated with the new column k of R (published as rb).
+// Backward Cholesky and inverse of a 32 x 32 block in one sweep, one warp,
+// everything in registers: lane i keeps row i of A (a[]) and column i of
+// X = R^-1 (x[]).  Step k (31 .. 0): the pivot comes from lane k by shuffle;
+// 1 / sqrt(A_kk) is one rsqrt (a few ulp, far inside the fp32 factorisation
+// error); lane i forms R[i][k]; row k of R is read from lane k by shuffles to
+// form x_kj = (delta_kj - sum_{m>k} R_km x_mj) / R_kk; the leading block is
+// updated with the new column, the entry the next pivot needs first.
 // S: block (upper triangle read, R written back); Xo: X (32 x 32, full).
 // Returns false (warp-uniform) if a pivot is not positive.
-__device__ __forceinline__ bool warp_chol_inv32(float* S, int lds, float* Xo, int ldx,
-                                                float* rb, float* rk) {
+__device__ __forceinline__ bool warp_chol_inv32(float* S, int lds, float* Xo, int ldx) {
   const int lane = threadIdx.x & 31;
   float a[32], x[32];
 #pragma unroll
@@ -45,26 +46,18 @@ __device__ __forceinline__ bool warp_chol_inv32(float* S, int lds, float* Xo, in
   for (int k = 31; k >= 0; --k) {
     const float d = __shfl_sync(0xffffffffu, a[k], k);
     ok = ok && (d > 0.f) && isfinite(d);
-    const float r = sqrtf(d);
-    const float ir = 1.0f / r;
-    const float l = (lane == k) ? r : a[k] * ir;
+    const float ir = rsqrtf(d);
+    const float l = (lane == k) ? d * ir : a[k] * ir;
     a[k] = l;
-    rb[lane] = l;                                  // column k of R (rows < k)
-    if (lane == k) {
 #pragma unroll
-      for (int m = k + 1; m < 32; ++m) rk[m] = a[m];   // row k of R (columns > k)
-    }
-    __syncwarp();
+    for (int j = k - 1; j >= 0; --j) a[j] = fmaf(-l, __shfl_sync(0xffffffffu, l, j), a[j]);
     float s0 = (lane == k) ? 1.f : 0.f, s1 = 0.f;
 #pragma unroll
     for (int m = k + 1; m < 32; m += 2) {
-      s0 = fmaf(-rk[m], x[m], s0);
-      if (m + 1 < 32) s1 = fmaf(-rk[m + 1], x[m + 1], s1);
+      s0 = fmaf(-__shfl_sync(0xffffffffu, a[m], k), x[m], s0);
+      if (m + 1 < 32) s1 = fmaf(-__shfl_sync(0xffffffffu, a[m + 1], k), x[m + 1], s1);
     }
     x[k] = (lane >= k) ? (s0 + s1) * ir : 0.f;
-#pragma unroll
-    for (int j = 0; j < k; ++j) a[j] = fmaf(-l, rb[j], a[j]);
-    __syncwarp();
   }
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
@@ -87,12 +80,13 @@ __device__ __forceinline__ bool warp_chol_inv32(float* S, int lds, float* Xo, in
 // Returns false if a pivot was not positive.
 __device__ bool ldl_factor_diag(float* A, float* X, float* rb, float* rk, int* bad) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  (void)rk;
   if (tid == 0) *bad = 0;
   __syncthreads();
   for (int J = 3; J >= 0; --J) {
     float* XJ = X + J * 32 * 33;
     if (warp == 0) {
-      const bool ok = warp_chol_inv32(A + (32 * J) * LDL_LD + 32 * J, LDL_LD, XJ, 33, rb, rk);
+      const bool ok = warp_chol_inv32(A + (32 * J) * LDL_LD + 32 * J, LDL_LD, XJ, 33);
       if (!ok && lane == 0) *bad = 1;
     }
     __syncthreads();                              // also orders the rest-update of J + 1
@@ -185,7 +179,8 @@ __global__ void __launch_bounds__(256) k_ldl_panel(float* __restrict__ H, int64_
   float* R = sm;                                  // 128 x LDL_LD
   float* T = R + LDL_PB * LDL_LD;                 // 64 x LDL_LD
   float* X = T + 64 * LDL_LD;                     // 4 x 32 x 33
-  __shared__ float rb[32], rk[32];
+  __shared__ __align__(16) float rb[32];
+  __shared__ float rk[32];
   __shared__ int bad;
   const int tid = threadIdx.x;
   const int64_t r0 = (int64_t)blockIdx.x * 64;
