@@ -52,7 +52,7 @@ import numpy as np
 __all__ = [
     "hessian", "damp", "splitmix64", "uniform53", "random_signs", "gaussian_matrix",
     "haar_orthogonal", "sylvester_hadamard", "hadamard_row", "SideTransform", "make_side",
-    "incoherence_forward", "incoherence_inverse", "udu", "row_grid", "quantize",
+    "incoherence_forward", "incoherence_inverse", "incoherence_rows", "incoherence_hessian", "udu", "row_grid", "quantize",
     "ldlq", "ldlq_blocked", "nearest", "optq", "dequantize", "proxy_loss", "Pipeline",
     "run_pipeline", "STREAM_M_SIGNS", "STREAM_N_SIGNS", "STREAM_M_A", "STREAM_M_B",
     "STREAM_N_A", "STREAM_N_B",
@@ -226,6 +226,22 @@ def incoherence_forward(W: np.ndarray, H: np.ndarray, U: SideTransform, V: SideT
     Wt = Um @ np.asarray(W, dtype=np.float64) @ Vn.T
     Ht = Vn @ np.asarray(H, dtype=np.float64) @ Vn.T
     return Wt, 0.5 * (Ht + Ht.T)
+
+
+def incoherence_rows(W: np.ndarray, U: SideTransform, V: SideTransform, rows) -> np.ndarray:
+    """Rows `rows` of W~ = U W V^T, row i being U[i, :] W V^T (same definition
+    as incoherence_forward, restricted to some output rows; rows of W~ are
+    what the row-independent LDLQ consumes)."""
+    Vn = V.matrix()
+    Ur = np.stack([U.row(int(i)) for i in rows])
+    return (Ur @ np.asarray(W, dtype=np.float64)) @ Vn.T
+
+
+def incoherence_hessian(H: np.ndarray, V: SideTransform) -> np.ndarray:
+    """H~ = V H V^T (symmetrised), the Hessian half of incoherence_forward."""
+    Vn = V.matrix()
+    Ht = Vn @ np.asarray(H, dtype=np.float64) @ Vn.T
+    return 0.5 * (Ht + Ht.T)
 
 
 def incoherence_inverse(Wt_hat: np.ndarray, U: SideTransform, V: SideTransform) -> np.ndarray:

@@ -12,8 +12,13 @@
 //
 // Both operands K-major (row-major [rows][K] bf16, piece p at row offset
 // p * piece_rows), loaded by TMA as 64-wide K boxes with the 128-byte swizzle.
-// Tile 128 x 256, one M=128 N=256 K=16 tcgen05.mma per 16 k, accumulators in
-// two 256-column TMEM buffers; 4-stage smem ring (48 KB per stage).
+// Tile 128 x 256, one M=128 N=256 K=16 tcgen05.mma per 16 k; 4-stage smem
+// ring (48 KB per stage).  The tensor core's fp32 accumulation drops low bits
+// (about one ulp of the running sum per MMA), so K is cut into chunks of
+// KCP = 512 per piece: each chunk (all six terms) accumulates into a fresh
+// TMEM buffer (columns [0, 256)), and the epilogue folds it into an fp32
+// running sum kept in a second TMEM buffer (columns [256, 512)) with
+// round-to-nearest adds; the tile's sum is added to C once, at its last chunk.
 // Bounded mbarrier waits as in the SYRK.
 #pragma once
 
@@ -43,11 +48,13 @@ struct Params {
   int tiles_n;             // number of tile columns
 };
 
+constexpr int KCP = 512;                           // K per piece per accumulation chunk
+
 struct Shared {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
-  uint64_t tfull[2];       // accumulator buffer b ready (MMA -> epilogue)
-  uint64_t tempty[2];      // accumulator buffer b drained (epilogue -> MMA)
+  uint64_t tfull;          // chunk accumulated (MMA -> epilogue)
+  uint64_t tempty;         // chunk buffer drained (epilogue -> MMA)
   uint32_t tmem_base;
   int abort;
 };
@@ -66,12 +73,16 @@ __device__ __forceinline__ bool tile_coords(const Params& p, int t, int& i0, int
   return !(p.upper_only && i0 > j0 + BN - 1);
 }
 
-// Persistent: CTA b handles tiles b, b + gridDim.x, ...  Two accumulator
-// buffers of 256 TMEM columns let the epilogue of one tile run while the
-// tensor cores work on the next.  Warp 0 lane 0: TMA producer; warp 1
-// lane 0: MMA issuer; warps 4..7: epilogue (warp w reads TMEM lanes
-// 32 (w - 4).., one output row per thread, 256 columns in 8 chunks with the
-// result added to C with vector reductions).
+// K-step `st` of a chunk covering piece columns [kc0, kc0 + kcl): term and offset.
+__device__ __forceinline__ void chunk_step(int st, int kcl, int& term, int& kk) {
+  const int per = kcl / BK;
+  term = st / per;
+  kk = (st % per) * BK;
+}
+
+// Persistent: CTA b handles tiles b, b + gridDim.x, ...  Warp 0 lane 0: TMA
+// producer; warp 1 lane 0: MMA issuer; warps 4..7: epilogue (warp w reads
+// TMEM lanes 32 (w - 4)..; one output row per thread, 256 columns).
 __global__ void __launch_bounds__(256, 1)
     k_gemm_split_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     Params p, int ntiles) {
@@ -80,18 +91,15 @@ __global__ void __launch_bounds__(256, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Shared* sh = reinterpret_cast<Shared*>(smem + STAGES * STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kpp = p.K / BK;                         // K-steps per term
-  const int nkb = NTERMS * kpp;
+  const int nchunk = (p.K + KCP - 1) / KCP;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&sh->full[s], 1);
       mbar_init(&sh->empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sh->tfull[b], 1);
-      mbar_init(&sh->tempty[b], 4);               // one arrival per epilogue warp
-    }
+    mbar_init(&sh->tfull, 1);
+    mbar_init(&sh->tempty, 4);                      // one arrival per epilogue warp
     sh->abort = 0;
     fence_mbar_init();
   }
@@ -104,100 +112,119 @@ __global__ void __launch_bounds__(256, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    int it = 0;                                   // global K-step counter (stage ring)
+    int it = 0;                                     // global K-step counter (stage ring)
     for (int t = blockIdx.x; t < ntiles && !sh->abort; t += gridDim.x) {
       int i0, j0;
       if (!tile_coords(p, t, i0, j0)) continue;
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int s = it % STAGES;
-        if (!mbar_wait(&sh->empty[s], (uint32_t)(((it / STAGES) & 1) ^ 1))) {
-          sh->abort = 1;
-          break;
+      for (int c = 0; c < nchunk && !sh->abort; ++c) {
+        const int kc0 = c * KCP, kcl = min(KCP, p.K - kc0);
+        const int steps = NTERMS * (kcl / BK);
+        for (int st = 0; st < steps; ++st, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&sh->empty[s], (uint32_t)(((it / STAGES) & 1) ^ 1))) {
+            sh->abort = 1;
+            break;
+          }
+          int term, kk, pa, pb;
+          chunk_step(st, kcl, term, kk);
+          term_pieces(term, pa, pb);
+          uint8_t* a = smem + s * STAGE_BYTES;
+          mbar_arrive_expect_tx(&sh->full[s], STAGE_BYTES);
+          tma_load_2d(a, &tmA, &sh->full[s], p.a_k0 + kc0 + kk, pa * p.a_piece_rows + p.a_row0 + i0);
+          tma_load_2d(a + A_BYTES, &tmB, &sh->full[s], p.b_k0 + kc0 + kk,
+                      pb * p.b_piece_rows + p.b_row0 + j0);
         }
-        int pa, pb;
-        term_pieces(kb / kpp, pa, pb);
-        const int kk = (kb % kpp) * BK;
-        uint8_t* a = smem + s * STAGE_BYTES;
-        mbar_arrive_expect_tx(&sh->full[s], STAGE_BYTES);
-        tma_load_2d(a, &tmA, &sh->full[s], p.a_k0 + kk, pa * p.a_piece_rows + p.a_row0 + i0);
-        tma_load_2d(a + A_BYTES, &tmB, &sh->full[s], p.b_k0 + kk, pb * p.b_piece_rows + p.b_row0 + j0);
       }
     }
   } else if (warp == 1 && lane == 0) {
-    int it = 0, lt = 0;
+    int it = 0, gc = 0;                             // gc: global chunk counter
     for (int t = blockIdx.x; t < ntiles && !sh->abort; t += gridDim.x) {
       int i0, j0;
       if (!tile_coords(p, t, i0, j0)) continue;
-      const int b = lt & 1, use = lt >> 1;
-      if (!mbar_wait(&sh->tempty[b], (uint32_t)((use & 1) ^ 1))) {
-        sh->abort = 1;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t acc = tmem + b * 256;
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int s = it % STAGES;
-        if (!mbar_wait(&sh->full[s], (uint32_t)((it / STAGES) & 1))) {
+      for (int c = 0; c < nchunk && !sh->abort; ++c, ++gc) {
+        if (!mbar_wait(&sh->tempty, (uint32_t)((gc & 1) ^ 1))) {   // chunk buffer free
           sh->abort = 1;
           break;
         }
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
-        const uint32_t b_addr = a_addr + A_BYTES;
+        const int kcl = min(KCP, p.K - c * KCP);
+        const int steps = NTERMS * (kcl / BK);
+        for (int st = 0; st < steps; ++st, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&sh->full[s], (uint32_t)((it / STAGES) & 1))) {
+            sh->abort = 1;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
-        for (int k = 0; k < BK / 16; ++k) {
-          // K-major SW128: 8-row groups 1024 B apart; K advances 32 B per 16 elements
-          const uint64_t adesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
-          const uint64_t bdesc = make_sw128_desc(b_addr + k * 32, 16, 1024);
-          tc_mma_f16(acc, adesc, bdesc, IDESC, (kb | k) != 0);
+          for (int k = 0; k < BK / 16; ++k) {
+            // K-major SW128: 8-row groups 1024 B apart; K advances 32 B per 16 elements
+            const uint64_t adesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
+            const uint64_t bdesc = make_sw128_desc(b_addr + k * 32, 16, 1024);
+            tc_mma_f16(tmem, adesc, bdesc, IDESC, (st | k) != 0);
+          }
+          tc_commit(&sh->empty[s]);
         }
-        tc_commit(&sh->empty[s]);
+        tc_commit(&sh->tfull);
       }
-      tc_commit(&sh->tfull[b]);
-      ++lt;
     }
   } else if (warp >= 4) {
     const int quarter = warp - 4;
-    int lt = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    int gc = 0;
+    bool stop = false;
+    for (int t = blockIdx.x; t < ntiles && !stop; t += gridDim.x) {
       int i0, j0;
       if (!tile_coords(p, t, i0, j0)) continue;
-      const int b = lt & 1, use = lt >> 1;
-      bool ok = mbar_wait(&sh->tfull[b], (uint32_t)(use & 1));
-      ok = __all_sync(0xffffffffu, ok) && !sh->abort;
-      if (!ok) break;
-      tc_fence_after();
       const int row = i0 + quarter * 32 + lane;
       const bool rok = row < p.M;
       float* crow = p.C + (int64_t)(rok ? row : 0) * p.ldc;
-      const uint32_t tb = tmem + b * 256 + ((uint32_t)(quarter * 32) << 16);
+      const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
       const bool vec = (p.ldc & 3) == 0;
-      // C += alpha * acc through fire-and-forget vector reductions in L2: no
-      // read round trip; one addition per element per launch, so the result
-      // equals the plain read-add-write.
+      for (int c = 0; c < nchunk; ++c, ++gc) {
+        bool ok = mbar_wait(&sh->tfull, (uint32_t)(gc & 1));
+        ok = __all_sync(0xffffffffu, ok) && !sh->abort;
+        if (!ok) {
+          stop = true;
+          break;
+        }
+        tc_fence_after();
+        const bool first = c == 0, last = c == nchunk - 1;
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        float v[32];
-        tmem_ld32(tb + c * 32, v);
-        const int jc = j0 + c * 32;
-        if (rok && jc < p.N) {
-          if (vec && jc + 32 <= p.N) {
-            float4* dst = reinterpret_cast<float4*>(crow + jc);
+        for (int c8 = 0; c8 < 8; ++c8) {
+          float v[32];
+          tmem_ld32(tmem + lanes + c8 * 32, v);
+          if (!first) {
+            float su[32];
+            tmem_ld32(tmem + lanes + 256 + c8 * 32, su);
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              atomicAdd(dst + q, make_float4(p.alpha * v[4 * q], p.alpha * v[4 * q + 1],
-                                             p.alpha * v[4 * q + 2], p.alpha * v[4 * q + 3]));
+            for (int e = 0; e < 32; ++e) v[e] += su[e];
+          }
+          if (!last) {
+            tmem_st32(tmem + lanes + 256 + c8 * 32, v);
           } else {
+            // C += alpha * sum through fire-and-forget vector reductions in L2
+            const int jc = j0 + c8 * 32;
+            if (rok && jc < p.N) {
+              if (vec && jc + 32 <= p.N) {
+                float4* dst = reinterpret_cast<float4*>(crow + jc);
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (jc + e < p.N) atomicAdd(crow + jc + e, p.alpha * v[e]);
+                for (int q = 0; q < 8; ++q)
+                  atomicAdd(dst + q, make_float4(p.alpha * v[4 * q], p.alpha * v[4 * q + 1],
+                                                 p.alpha * v[4 * q + 2], p.alpha * v[4 * q + 3]));
+              } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                  if (jc + e < p.N) atomicAdd(crow + jc + e, p.alpha * v[e]);
+              }
+            }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->tempty);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->tempty[b]);
-      ++lt;
     }
   }
   __syncwarp();

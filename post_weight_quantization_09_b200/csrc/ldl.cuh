@@ -164,7 +164,9 @@ __device__ bool ldl_factor_diag(float* A, float* X, float* rb, float* rk, int* b
 
 // One panel of the backward blocked factorisation, columns [c0, c0 + w), w <= 128:
 // every CTA loads and factors the diagonal block (the same deterministic
-// computation in each, so all agree), CTA 0 writes R_pp back to H, and each
+// computation in each, so all agree), CTA 0 writes R_pp to Rd (a 128 x 128
+// slot of the workspace: H's own diagonal block must stay intact until every
+// CTA of the launch, possibly in a later wave, has read it), and each
 // CTA solves 64 rows of R12 = H12 R_pp^-T by block back substitution over the
 // four 32-column blocks (J = 3 .. 0):
 //   t_J = h_J - sum_{K > J} r_K R_JK^T,   r_J = t_J X_JJ^T,
@@ -174,7 +176,8 @@ __device__ bool ldl_factor_diag(float* A, float* X, float* rb, float* rk, int* b
 // Grid: max(1, ceil(c0 / 64)) CTAs of 256 threads.
 // Dynamic smem: 128 x 129 (R_pp) + 64 x 129 (row tile) + 4 x 32 x 33 floats.
 __global__ void __launch_bounds__(256) k_ldl_panel(float* __restrict__ H, int64_t n, int64_t c0,
-                                                   int w, __nv_bfloat16* __restrict__ Rs) {
+                                                   int w, __nv_bfloat16* __restrict__ Rs,
+                                                   float* __restrict__ Rd) {
   extern __shared__ __align__(16) float sm[];
   float* R = sm;                                  // 128 x LDL_LD
   float* T = R + LDL_PB * LDL_LD;                 // 64 x LDL_LD
@@ -214,10 +217,7 @@ __global__ void __launch_bounds__(256) k_ldl_panel(float* __restrict__ H, int64_
   if (blockIdx.x == 0) {
     if (!ok && tid == 0) record_status(QUIP_ERR_NOT_PD);
 #pragma unroll 4
-    for (int e = tid; e < LDL_PB * LDL_PB; e += 256) {
-      const int i = e >> 7, j = e & 127;
-      if (i < w && j < w && j >= i) H[(c0 + i) * n + c0 + j] = R[i * LDL_LD + j];
-    }
+    for (int e = tid; e < LDL_PB * LDL_PB; e += 256) Rd[e] = R[(e >> 7) * LDL_LD + (e & 127)];
   }
   if (c0 == 0) return;
   const int ty = tid >> 3, tx = tid & 7;
@@ -277,6 +277,19 @@ __global__ void __launch_bounds__(256) k_ldl_panel(float* __restrict__ H, int64_
     Rs[gi * LDL_PB + k] = p0;
     Rs[pstride + gi * LDL_PB + k] = p1;
     Rs[2 * pstride + gi * LDL_PB + k] = p2;
+  }
+}
+
+// Copy every panel's diagonal factor block from Rd[p] (128 x 128) into H's
+// upper triangle: block p covers rows / columns [128 p, 128 p + w).
+__global__ void k_ldl_scatter_diag(float* __restrict__ H, int64_t n, const float* __restrict__ Rd) {
+  const int64_t p = blockIdx.x;
+  const int64_t c0 = p * LDL_PB;
+  const int w = (int)((n - c0) < LDL_PB ? (n - c0) : LDL_PB);
+  const float* src = Rd + p * LDL_PB * LDL_PB;
+  for (int e = threadIdx.x; e < LDL_PB * LDL_PB; e += blockDim.x) {
+    const int i = e >> 7, j = e & 127;
+    if (i < w && j < w && j >= i) H[(c0 + i) * n + c0 + j] = src[e];
   }
 }
 

@@ -483,9 +483,11 @@ quip_status quip_hessian_finalize(float* H, int64_t n, int64_t N_total, float da
   return QUIP_OK;
 }
 
-// LDL workspace: Rinv (128 x 128 fp32), then the panel's three bf16 pieces (3 x n x 128).
+// LDL workspace: the panels' diagonal factor blocks (P x 128 x 128 fp32), then
+// the current panel's three bf16 pieces (3 x n x 128).
+static int64_t ldl_panels(int64_t n) { return (n + LDL_PB - 1) / LDL_PB; }
 static size_t ldl_ws_bytes(int64_t n) {
-  return round256((size_t)LDL_PB * LDL_PB * 4) + round256((size_t)3 * n * LDL_PB * 2);
+  return round256((size_t)ldl_panels(n) * LDL_PB * LDL_PB * 4) + round256((size_t)3 * n * LDL_PB * 2);
 }
 // LDLQ workspace: accumulator A (m x n fp32), the error of every column as
 // three bf16 pieces (3 x m x n), the split transposed factor (3 x n x n bf16).
@@ -598,8 +600,9 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
   quip_status s = check_ws(ws, ws_bytes, ldl_ws_bytes(n));
   if (s != QUIP_OK) return s;
   cudaStream_t st = S(stream);
-  __nv_bfloat16* Rs = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) +
-                                                       round256((size_t)LDL_PB * LDL_PB * 4));
+  float* Rd = static_cast<float*>(ws);
+  __nv_bfloat16* Rs = reinterpret_cast<__nv_bfloat16*>(
+      static_cast<char*>(ws) + round256((size_t)ldl_panels(n) * LDL_PB * LDL_PB * 4));
   const size_t smem_panel = ((size_t)(LDL_PB + 64) * LDL_LD + 4 * 32 * 33) * sizeof(float);
   static bool attr = false;
   if (!attr) {
@@ -618,7 +621,8 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
     const int64_t c0 = p * LDL_PB;
     const int w = (int)std::min<int64_t>(LDL_PB, n - c0);
     const unsigned grid = (unsigned)std::max<int64_t>(1, (c0 + 63) / 64);
-    k_ldl_panel<<<grid, 256, smem_panel, st>>>(H_t, n, c0, w, Rs); count_launch();
+    k_ldl_panel<<<grid, 256, smem_panel, st>>>(H_t, n, c0, w, Rs, Rd + p * LDL_PB * LDL_PB);
+    count_launch();
     if (c0 > 0) {
       // H[:c0, :c0] -= R12 R12^T on the upper tiles
       sgemm::Params gp{};
@@ -627,6 +631,7 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
       QCHECK(split_gemm(ta, tb, gp, st));
     }
   }
+  k_ldl_scatter_diag<<<(unsigned)P, 256, 0, st>>>(H_t, n, Rd); count_launch();
   k_diag_to<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(H_t, n, D); count_launch();
   k_scale_upper<<<(unsigned)n, 256, 0, st>>>(H_t, n, D); count_launch();
   k_square<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(D, n); count_launch();

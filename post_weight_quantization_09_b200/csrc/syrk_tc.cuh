@@ -16,8 +16,13 @@
 //    columns [0, 256) and [256, 512).
 //  * 3-stage smem ring (64 KB per stage) with full / empty mbarriers; the
 //    MMA thread frees a stage with tcgen05.commit.
-//  * epilogue: all 8 warps read the accumulators with tcgen05.ld (warp w
-//    reads TMEM lanes 32 (w % 4) .. of accumulator w / 4) and store fp32 rows.
+//  * The tensor core's fp32 accumulation drops low bits (about one ulp of
+//    the running sum per MMA step), so the token range is cut into chunks of
+//    2048: each chunk starts a fresh TMEM accumulator, and warps 4..7 add the
+//    chunk's sums into H in fp32 (the first chunk stores, later chunks add by
+//    vector reductions issued by the same thread to the same addresses, so
+//    the order, and the result, are fixed) while the producer already loads
+//    the next chunk.  Warp w reads TMEM lanes 32 (w - 4) of both accumulators.
 // Every mbarrier wait is bounded (common.cuh); on a timeout the CTA records
 // QUIP_ERR_TIMEOUT, skips the stores, waits for its own MMAs and frees TMEM.
 #pragma once
@@ -36,10 +41,13 @@ constexpr int STAGE_BYTES = 2 * SLAB_BYTES;   // A + B = 64 KB
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr uint32_t IDESC = make_idesc_bf16(128, 256, /*a_mn=*/1, /*b_mn=*/1);
 
+constexpr int KCHUNK = 2048 / BK;              // K-steps per accumulation chunk
+
 struct Shared {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
-  uint64_t accum;
+  uint64_t tfull;          // chunk accumulated (MMA -> epilogue)
+  uint64_t tempty;         // chunk drained (epilogue -> MMA)
   uint32_t tmem_base;
   int abort;
 };
@@ -66,13 +74,15 @@ __global__ void __launch_bounds__(256, 1)
   const bool diag = (ti == tj);
   const int i0 = ti * BT, j0 = tj * BT;
   const int nkb = (N + BK - 1) / BK;
+  const int nch = (nkb + KCHUNK - 1) / KCHUNK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&sh->full[s], 1);
       mbar_init(&sh->empty[s], 1);
     }
-    mbar_init(&sh->accum, 1);
+    mbar_init(&sh->tfull, 1);
+    mbar_init(&sh->tempty, 4);                  // one arrival per epilogue warp
     sh->abort = 0;
     fence_mbar_init();
   }
@@ -103,6 +113,14 @@ __global__ void __launch_bounds__(256, 1)
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
     for (int kb = 0; kb < nkb; ++kb) {
+      const int kc = kb % KCHUNK, ch = kb / KCHUNK;
+      if (kc == 0 && ch > 0) {                   // wait until chunk ch - 1 is drained
+        if (!mbar_wait(&sh->tempty, (uint32_t)((ch - 1) & 1))) {
+          sh->abort = 1;
+          break;
+        }
+        tc_fence_after();
+      }
       const int s = kb % STAGES;
       const uint32_t par = (uint32_t)((kb / STAGES) & 1);
       if (!mbar_wait(&sh->full[s], par)) {
@@ -120,50 +138,57 @@ __global__ void __launch_bounds__(256, 1)
         for (int h = 0; h < 2; ++h) {
           const uint64_t adesc =
               make_sw128_desc(a_addr + h * 2 * BOX_BYTES + kk * 2048, BOX_BYTES, 1024);
-          tc_mma_f16(tmem + h * 256, adesc, bdesc, IDESC, (kb | kk) != 0);
+          tc_mma_f16(tmem + h * 256, adesc, bdesc, IDESC, (kc | kk) != 0);
         }
       }
       tc_commit(&sh->empty[s]);
+      if (kc == KCHUNK - 1 || kb == nkb - 1) tc_commit(&sh->tfull);
     }
-    tc_commit(&sh->accum);   // always: tracks every MMA issued above
-  }
-  __syncwarp();
-  __syncthreads();
-
-  // ---------------- epilogue (all warps)
-  bool ok = mbar_wait(&sh->accum, 0);
-  ok = __all_sync(0xffffffffu, ok) && (sh->abort == 0) && nkb > 0;
-  tc_fence_after();
-  if (ok) {
-    const int quarter = warp & 3, half = warp >> 2;
-    const int row = i0 + half * 128 + quarter * 32 + lane;
-    const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + half * 256;
-    float* hrow = H + (int64_t)row * n;
+  } else if (warp >= 4) {
+    // ---------------- epilogue: H (+)= chunk sums, lower triangle only
+    const int quarter = warp - 4;
+    for (int ch = 0; ch < nch; ++ch) {
+      bool ok = mbar_wait(&sh->tfull, (uint32_t)(ch & 1));
+      ok = __all_sync(0xffffffffu, ok) && !sh->abort;
+      if (!ok) break;
+      tc_fence_after();
+      const bool add = accumulate || ch > 0;
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
-      float v[32];
-      tmem_ld32(tbase + c * 32, v);
-      const int jc = j0 + c * 32;
-      if (row < n && jc <= row) {
-        if (jc + 32 <= n && (n & 3) == 0) {
-          float4* dst = reinterpret_cast<float4*>(hrow + jc);
+      for (int h = 0; h < 2; ++h) {
+        const int row = i0 + h * 128 + quarter * 32 + lane;
+        const uint32_t tb = tmem + ((uint32_t)(quarter * 32) << 16) + h * 256;
+        float* hrow = H + (int64_t)(row < n ? row : 0) * n;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          float v[32];
+          tmem_ld32(tb + c * 32, v);
+          const int jc = j0 + c * 32;
+          if (row < n && jc <= row) {
+            if (jc + 32 <= n && (n & 3) == 0) {
+              float4* dst = reinterpret_cast<float4*>(hrow + jc);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float4 f = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-            if (accumulate) {
-              const float4 o = dst[q];
-              f.x += o.x, f.y += o.y, f.z += o.z, f.w += o.w;
+              for (int q = 0; q < 8; ++q) {
+                const float4 f = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                if (add) atomicAdd(dst + q, f);
+                else dst[q] = f;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (jc + e < n) {
+                  if (add) atomicAdd(hrow + jc + e, v[e]);
+                  else hrow[jc + e] = v[e];
+                }
             }
-            dst[q] = f;
           }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (jc + e < n) hrow[jc + e] = accumulate ? hrow[jc + e] + v[e] : v[e];
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->tempty);
     }
   }
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

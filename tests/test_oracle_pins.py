@@ -146,6 +146,18 @@ def test_incoherence_preserves_proxy_and_inverts():
     assert np.abs(Wt2).max() < 0.5
 
 
+def test_incoherence_rows_and_hessian_match_full_forward():
+    rng = np.random.default_rng(12)
+    W = rng.standard_normal((24, 16))
+    H = _spd(16, 5)
+    U = O.make_side(4, "m", "kronecker", 24, 6, 4)
+    V = O.make_side(4, "n", "hadamard", 16)
+    Wt, Ht = O.incoherence_forward(W, H, U, V)
+    rows = [0, 7, 23]
+    np.testing.assert_allclose(O.incoherence_rows(W, U, V, rows), Wt[rows], atol=1e-14)
+    np.testing.assert_allclose(O.incoherence_hessian(H, V), Ht, atol=1e-13)
+
+
 def test_hadamard_sign_placement_hand_example():
     # V = H_4 diag(s) / 2 with s = (1, -1, 1, 1): V e_1 = s_1 * H_4[:, 1] / 2
     S = O.SideTransform("hadamard", 4, signs=np.array([1.0, -1.0, 1.0, 1.0]))

@@ -69,3 +69,51 @@ def test_attn7b_full_layer():
     for i in rows:
         ref_row = (Um[:, i] @ Wt_hat_d) @ Vm          # row i of U^T W~^ V
         assert np.abs(W_hat_d[i] - ref_row).max() <= 1e-4 * s_d.max()
+
+
+def _sampled_layer_check(name, nrows=256):
+    """Whole layer on the device vs the FP64 oracle on `nrows` sampled rows
+    (the oracle forms H, H~ and its LDL in full; W~ and LDLQ only for the
+    sampled rows, which is exact because rows are independent)."""
+    cfg = CONFIGS[name]
+    d = make_layer(cfg)
+    q, r, H_dev = _run_device(cfg, d)
+    Wt_dev = host(q.W_t)
+    t0 = time.time()
+    H = O.damp(O.hessian(d["X"]), cfg.damp)
+    h_err = rel_fro(H_dev, H)
+    U = O.make_side(cfg.seed, "m", cfg.m_side.kind, cfg.m, cfg.m_side.p, cfg.m_side.q)
+    V = O.make_side(cfg.seed, "n", cfg.n_side.kind, cfg.n, cfg.n_side.p, cfg.n_side.q)
+    Ht = O.incoherence_hessian(H, V)
+    del H
+    Uf, D = O.udu(Ht)
+    rows = np.sort(np.random.default_rng(1).choice(cfg.m, nrows, replace=False))
+    Wt = O.incoherence_rows(d["W"], U, V, rows)
+    w_scale = np.abs(Wt).max()
+    wt_err = np.abs(Wt_dev[rows] - Wt).max() / w_scale
+    lo, s = O.row_grid(Wt, cfg.bits)
+    codes, Wt_hat, _ = O.ldlq(Wt, Uf, lo, s, cfg.bits)
+    C = host(r.codes)[rows]
+    lo_d, s_d = host(r.lo)[rows], host(r.scale)[rows]
+    agree = float((C == codes).mean())
+    Wt_hat_d = O.dequantize(C, lo_d, s_d)
+    loss = O.proxy_loss(Wt_hat, Wt, Ht)
+    loss_d = O.proxy_loss(Wt_hat_d, Wt, Ht)
+    same = C == codes
+    w_err = float(np.abs(Wt_hat_d - Wt_hat)[same].max() / s.max())
+    bad, not_near = ldlq_trajectory_check(C, Wt, Uf, lo_d, s_d, cfg.bits, tau=1e-3)
+    print(f"\n{name}: H rel-Fro {h_err:.3e}  W~ err {wt_err:.2e}  codes agree {agree:.6f} on {nrows} rows  "
+          f"loss {loss:.6g} vs {loss_d:.6g} (rel {abs(loss_d - loss) / loss:.2e})  W^ err/s {w_err:.2e}  "
+          f"trajectory mismatch {bad:.2e} (not near-tie {not_near:.2e})  oracle {time.time() - t0:.0f}s")
+    assert h_err <= 1e-4
+    assert wt_err <= 1e-5
+    assert abs(loss_d - loss) / loss <= 1e-3
+    assert w_err <= 1e-4
+    assert not_near == 0.0
+    assert agree >= 0.999
+    return q, r
+
+
+@pytest.mark.parametrize("name", ["up7b", "down7b", "gate70b"])
+def test_llama_layers_sampled_rows(name):
+    _sampled_layer_check(name)

@@ -106,9 +106,9 @@ def test_hessian_accumulate_and_finalize(N, n, dtype):
     Xd = dev(X, torch.bfloat16 if dtype == "bf16" else torch.float32)
     H = torch.full((n, n), float("nan"), device="cuda")
     Q.quip_hessian_accumulate(Xd, H)
-    # bf16 products are exact; the fp32 sums on the tensor cores lose up to
-    # about one ulp per 16-token MMA step, so the bound is the stated 1e-4
-    tol = 1e-4 if dtype == "bf16" else 1e-5
+    # bf16 products are exact; the tensor cores' fp32 sums lose about one ulp
+    # per 16-token MMA step, bounded by the kernel's 2048-token chunks
+    tol = 2e-5 if dtype == "bf16" else 1e-5
     lower = np.tril(host(H))
     assert rel_fro(lower, np.tril(X.astype(np.float64).T @ X)) <= tol
     Q.quip_hessian_finalize(H, N, 0.01)
@@ -164,6 +164,25 @@ def test_ldl_matches_oracle(n):
     # backward error of the device factor, in FP64
     R = (np.eye(n) + U) @ np.diag(host(D)) @ (np.eye(n) + U).T
     assert rel_fro(R, H) <= 2e-6
+
+
+def test_ldl_panel_grid_beyond_one_wave():
+    # n = 9728: the first panel's solve runs on 150 CTAs (more than one per SM),
+    # so CTAs of a later wave must still see the unfactored diagonal block.
+    n = 9728
+    rng = np.random.default_rng(5)
+    G = rng.standard_normal((n, 64))
+    H = (np.eye(n) * 0.5 + G @ G.T / 64).astype(np.float32).astype(np.float64)
+    U_ref, D_ref = O.udu(H)
+    Hd = dev(H)
+    D = torch.empty(n, device="cuda")
+    Q.quip_ldl(Hd, D)
+    assert Q.quip_sync_status() == L.QUIP_OK
+    U = host(Hd)
+    rows = rng.choice(n, 64, replace=False)
+    for i in rows:
+        np.testing.assert_allclose(U[i, i + 1:], U_ref[i, i + 1:], atol=5e-4)
+    np.testing.assert_allclose(host(D), D_ref, rtol=5e-4)
 
 
 def test_ldl_rejects_unaligned_order():
