@@ -319,7 +319,7 @@ def run_ours(args, cfg: LayerConfig):
     lo_h = torch.empty(cfg.m, dtype=torch.float32).pin_memory()
     sc_h = torch.empty(cfg.m, dtype=torch.float32).pin_memory()
     e2e_ms = []
-    for i in range(args.e2e_steps + 1):
+    for i in range(max(1, args.e2e_steps) + 1):
         flush.zero_()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -2,9 +2,15 @@
 //   C_b[i][j] = alpha * sum_k A_b[i][k] * B_b[k][j] + beta * C_b[i][j]
 // with arbitrary element strides for every operand (so transposes are free).
 // Used where the contraction is small or must stay in fp32: the Kronecker
-// factors of the incoherence transform, the fp32-input Hessian, and the
-// trailing updates of the LDL and LDLQ steps.
+// factors of the incoherence transform and the fp32-input Hessian.  With
+// Acc = double the products and sums are taken in fp64 (inputs converted on
+// the way into shared memory, the result rounded to fp32 once): the Hessian's
+// Kronecker transform uses it, because an fp32 sum over a Haar factor's row
+// carries an error proportional to the largest entries of H into every entry
+// of the transformed H, including its small-eigenvalue directions.
 #pragma once
+
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -25,20 +31,26 @@ struct GemmArgs {
 constexpr int SG_BM = 64, SG_BN = 64, SG_BK = 16;
 
 // 256 threads; each computes a 4 x 4 block of the 64 x 64 tile.
-template <typename TA, typename TB>
+template <typename Acc, typename T>
+__device__ __forceinline__ Acc to_acc(T x) {
+  if constexpr (std::is_same<T, double>::value) return (Acc)x;
+  else return (Acc)to_f32<T>(x);
+}
+
+template <typename TA, typename TB, typename Acc = float>
 __global__ void __launch_bounds__(256) k_gemm_simt(GemmArgs g) {
   const int64_t ti = blockIdx.y, tj = blockIdx.x, b = blockIdx.z;
   if (g.tri == 1 && ti < tj) return;
   if (g.tri == 2 && ti > tj) return;
-  __shared__ float sA[SG_BK][SG_BM + 4];
-  __shared__ float sB[SG_BK][SG_BN + 4];
+  __shared__ Acc sA[SG_BK][SG_BM + 4];
+  __shared__ Acc sB[SG_BK][SG_BN + 4];
   const TA* A = reinterpret_cast<const TA*>(g.A) + b * g.sab;
   const TB* B = reinterpret_cast<const TB*>(g.B) + b * g.sbb;
   float* C = g.C + b * g.scb;
   const int tid = threadIdx.x;
   const int tx = tid % 16, ty = tid / 16;
   const int64_t i0 = ti * SG_BM, j0 = tj * SG_BN;
-  float acc[4][4] = {};
+  Acc acc[4][4] = {};
   for (int64_t k0 = 0; k0 < g.K; k0 += SG_BK) {
     // A tile 64 x 16 and B tile 16 x 64: 1024 elements each, 4 per thread.
 #pragma unroll
@@ -48,19 +60,19 @@ __global__ void __launch_bounds__(256) k_gemm_simt(GemmArgs g) {
         const int kk = (g.sak == 1) ? (idx % SG_BK) : (idx / SG_BM);
         const int ii = (g.sak == 1) ? (idx / SG_BK) : (idx % SG_BM);
         const int64_t gi = i0 + ii, gk = k0 + kk;
-        sA[kk][ii] = (gi < g.M && gk < g.K) ? to_f32<TA>(A[gi * g.sam + gk * g.sak]) : 0.f;
+        sA[kk][ii] = (gi < g.M && gk < g.K) ? to_acc<Acc, TA>(A[gi * g.sam + gk * g.sak]) : Acc(0);
       }
       {
         const int jj = (g.sbn == 1) ? (idx % SG_BN) : (idx / SG_BK);
         const int kk = (g.sbn == 1) ? (idx / SG_BN) : (idx % SG_BK);
         const int64_t gj = j0 + jj, gk = k0 + kk;
-        sB[kk][jj] = (gj < g.N && gk < g.K) ? to_f32<TB>(B[gk * g.sbk + gj * g.sbn]) : 0.f;
+        sB[kk][jj] = (gj < g.N && gk < g.K) ? to_acc<Acc, TB>(B[gk * g.sbk + gj * g.sbn]) : Acc(0);
       }
     }
     __syncthreads();
 #pragma unroll
     for (int kk = 0; kk < SG_BK; ++kk) {
-      float a[4], bb[4];
+      Acc a[4], bb[4];
 #pragma unroll
       for (int r = 0; r < 4; ++r) a[r] = sA[kk][ty + 16 * r];
 #pragma unroll
@@ -68,7 +80,7 @@ __global__ void __launch_bounds__(256) k_gemm_simt(GemmArgs g) {
 #pragma unroll
       for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(a[r], bb[c], acc[r][c]);
+        for (int c = 0; c < 4; ++c) acc[r][c] = fma(a[r], bb[c], acc[r][c]);
     }
     __syncthreads();
   }
@@ -81,18 +93,18 @@ __global__ void __launch_bounds__(256) k_gemm_simt(GemmArgs g) {
       const int64_t gj = j0 + tx + 16 * c;
       if (gj >= g.N) continue;
       float* p = C + gi * g.scm + gj * g.scn;
-      const float v = g.alpha * acc[r][c];
+      const float v = (float)((Acc)g.alpha * acc[r][c]);
       *p = (g.beta == 0.f) ? v : fmaf(g.beta, *p, v);
     }
   }
 }
 
-template <typename TA, typename TB>
+template <typename TA, typename TB, typename Acc = float>
 inline cudaError_t gemm_simt(const GemmArgs& g, int64_t batch, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || batch <= 0) return cudaSuccess;
   dim3 grid((unsigned)((g.N + SG_BN - 1) / SG_BN), (unsigned)((g.M + SG_BM - 1) / SG_BM),
             (unsigned)batch);
-  k_gemm_simt<TA, TB><<<grid, 256, 0, st>>>(g); count_launch();
+  k_gemm_simt<TA, TB, Acc><<<grid, 256, 0, st>>>(g); count_launch();
   return cudaGetLastError();
 }
 

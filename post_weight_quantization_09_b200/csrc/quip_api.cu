@@ -35,6 +35,8 @@ struct SideData {
   float* signs = nullptr;   // HADAMARD
   float* A = nullptr;       // KRONECKER p x p
   float* B = nullptr;       // KRONECKER q x q
+  double* A64 = nullptr;    // KRONECKER: the same factors in fp64 (Hessian transform)
+  double* B64 = nullptr;
   double* G = nullptr;      // KRONECKER: Gaussian draw scratch, max(p,q)^2
   double* Qc = nullptr;     // KRONECKER: CGS2 scratch, max(p,q)^2
 };
@@ -203,57 +205,76 @@ cudaError_t fwht_cols(float* A, int64_t ld, int64_t ncols, int64_t R, const floa
 
 // Rows: dst[i, :] = vec(A' Xr_i B'^T) for each row Xr_i (p x q view) of src,
 // with A' = A or A^T, B' = B or B^T (transpose = inverse transform).
-template <typename TIn>
+// Acc = double: fp64 factors and fp64 sums (the Hessian's transform).
+template <typename Acc>
+struct KronFactors {
+  using F = typename std::conditional<std::is_same<Acc, double>::value, double, float>::type;
+  static const F* A(const SideData& sd) {
+    if constexpr (std::is_same<Acc, double>::value) return sd.A64;
+    else return sd.A;
+  }
+  static const F* B(const SideData& sd) {
+    if constexpr (std::is_same<Acc, double>::value) return sd.B64;
+    else return sd.B;
+  }
+};
+
+template <typename TIn, typename Acc = float>
 cudaError_t kron_rows(const TIn* src, int64_t ldsrc, float* dst, int64_t rows,
                       const SideData& sd, bool transpose, float* tmp, cudaStream_t st) {
+  using KF = KronFactors<Acc>;
+  using F = typename KF::F;
   const int64_t p = sd.p, q = sd.q, n = p * q;
   GemmArgs g{};
   // tmp_i = Xr_i B'^T : M = p, N = q, K = q, batched over rows
   g.M = p, g.N = q, g.K = q, g.alpha = 1.f, g.beta = 0.f, g.tri = 0;
   g.A = src, g.sam = q, g.sak = 1, g.sab = ldsrc;
-  g.B = sd.B;
+  g.B = KF::B(sd);
   if (!transpose) g.sbk = 1, g.sbn = q;   // B'^T[k][j] = B[j][k]
   else g.sbk = q, g.sbn = 1;              // (B^T)^T = B
   g.sbb = 0;
   g.C = tmp, g.scm = q, g.scn = 1, g.scb = n;
-  cudaError_t e = gemm_simt<TIn, float>(g, rows, st);
+  cudaError_t e = gemm_simt<TIn, F, Acc>(g, rows, st);
   if (e != cudaSuccess) return e;
   // dst_i = A' tmp_i : M = p, N = q, K = p
   GemmArgs h{};
   h.M = p, h.N = q, h.K = p, h.alpha = 1.f, h.beta = 0.f, h.tri = 0;
-  h.A = sd.A;
+  h.A = KF::A(sd);
   if (!transpose) h.sam = p, h.sak = 1;
   else h.sam = 1, h.sak = p;
   h.sab = 0;
   h.B = tmp, h.sbk = q, h.sbn = 1, h.sbb = n;
   h.C = dst, h.scm = q, h.scn = 1, h.scb = n;
-  return gemm_simt<float, float>(h, rows, st);
+  return gemm_simt<F, float, Acc>(h, rows, st);
 }
 
 // Columns: X (R x ncols, R = p q) <- (A' (x) B') X, through tmp.
+template <typename Acc = float>
 cudaError_t kron_cols(float* X, int64_t ncols, const SideData& sd, bool transpose, float* tmp,
                       cudaStream_t st) {
+  using KF = KronFactors<Acc>;
+  using F = typename KF::F;
   const int64_t p = sd.p, q = sd.q;
   GemmArgs g{};
   // tmp[a'] = B' X[a'] : batch p, M = q, N = ncols, K = q
   g.M = q, g.N = ncols, g.K = q, g.alpha = 1.f, g.beta = 0.f, g.tri = 0;
-  g.A = sd.B;
+  g.A = KF::B(sd);
   if (!transpose) g.sam = q, g.sak = 1;
   else g.sam = 1, g.sak = q;
   g.sab = 0;
   g.B = X, g.sbk = ncols, g.sbn = 1, g.sbb = q * ncols;
   g.C = tmp, g.scm = ncols, g.scn = 1, g.scb = q * ncols;
-  cudaError_t e = gemm_simt<float, float>(g, p, st);
+  cudaError_t e = gemm_simt<F, float, Acc>(g, p, st);
   if (e != cudaSuccess) return e;
   // X = A' tmp (tmp as p x (q ncols))
   GemmArgs h{};
   h.M = p, h.N = q * ncols, h.K = p, h.alpha = 1.f, h.beta = 0.f, h.tri = 0;
-  h.A = sd.A;
+  h.A = KF::A(sd);
   if (!transpose) h.sam = p, h.sak = 1;
   else h.sam = 1, h.sak = p;
   h.B = tmp, h.sbk = q * ncols, h.sbn = 1;
   h.C = X, h.scm = q * ncols, h.scn = 1;
-  return gemm_simt<float, float>(h, 1, st);
+  return gemm_simt<F, float, Acc>(h, 1, st);
 }
 
 __global__ void k_convert_rows_bf16(const __nv_bfloat16* in, int64_t ld, float* out, int64_t m,
@@ -350,6 +371,8 @@ static quip_status alloc_side(SideData& sd, int kind, int64_t dim, int64_t p, in
     const int64_t mx = std::max(p, q);
     QCHECK(cudaMalloc(&sd.A, p * p * sizeof(float)));
     QCHECK(cudaMalloc(&sd.B, q * q * sizeof(float)));
+    QCHECK(cudaMalloc(&sd.A64, p * p * sizeof(double)));
+    QCHECK(cudaMalloc(&sd.B64, q * q * sizeof(double)));
     QCHECK(cudaMalloc(&sd.G, mx * mx * sizeof(double)));
     QCHECK(cudaMalloc(&sd.Qc, mx * mx * sizeof(double)));
   }
@@ -368,7 +391,8 @@ static quip_status draw_side(const SideData& sd, uint64_t seed, int which, cudaS
       const int64_t d = f == 0 ? sd.p : sd.q;
       k_gaussian<<<(unsigned)((d * d + 255) / 256), 256, 0, st>>>(sd.G, d * d, seed, f == 0 ? sa : sb);
       count_launch();
-      k_haar_cgs2<<<1, 256, 0, st>>>(sd.G, sd.Qc, f == 0 ? sd.A : sd.B, (int)d);
+      k_haar_cgs2<<<1, 256, 0, st>>>(sd.G, sd.Qc, f == 0 ? sd.A : sd.B, f == 0 ? sd.A64 : sd.B64,
+                                       (int)d);
       count_launch();
     }
   }
@@ -411,6 +435,8 @@ quip_status quip_transform_destroy(quip_transform* tf) {
     cudaFree(sd.signs);
     cudaFree(sd.A);
     cudaFree(sd.B);
+    cudaFree(sd.A64);
+    cudaFree(sd.B64);
     cudaFree(sd.G);
     cudaFree(sd.Qc);
   }
@@ -556,8 +582,13 @@ quip_status quip_incoherence_forward(const quip_transform* tf, const void* W, in
     QCHECK(side_rows<float>(V, false, static_cast<const float*>(W), ldw, W_t, m, tmp, st));
   QCHECK(side_cols(U, false, W_t, n, tmp, st));
   if (H) {
-    QCHECK(side_rows<float>(V, false, H, n, H, n, tmp, st));   // H V^T
-    QCHECK(side_cols(V, false, H, n, tmp, st));                // V (H V^T)
+    if (V.kind == QUIP_T_KRONECKER) {                           // fp64 sums, see gemm_simt.cuh
+      QCHECK((kron_rows<float, double>(H, n, H, n, V, false, tmp, st)));   // H V^T
+      QCHECK((kron_cols<double>(H, n, V, false, tmp, st)));                // V (H V^T)
+    } else {
+      QCHECK(side_rows<float>(V, false, H, n, H, n, tmp, st));   // H V^T
+      QCHECK(side_cols(V, false, H, n, tmp, st));                // V (H V^T)
+    }
   }
   return QUIP_OK;
 }

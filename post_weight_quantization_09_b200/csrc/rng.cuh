@@ -49,10 +49,12 @@ __global__ void k_gaussian(double* G, int64_t count, uint64_t seed, uint32_t str
 // Q of G = QR with diag(R) > 0 (the Haar-distributed orthogonal factor), by
 // classical Gram-Schmidt with one re-orthogonalisation pass (CGS2) in fp64.
 // One CTA of 256 threads; p <= 256.  Qc: p x p fp64 workspace (column j of Q
-// stored contiguously at Qc + j*p).  Q: p x p fp32 output, row-major.
+// stored contiguously at Qc + j*p).  Q: p x p fp32 output, row-major; Q64
+// the same in fp64.
 __global__ void __launch_bounds__(256) k_haar_cgs2(const double* __restrict__ G,
                                                     double* __restrict__ Qc,
-                                                    float* __restrict__ Q, int p) {
+                                                    float* __restrict__ Q,
+                                                    double* __restrict__ Q64, int p) {
   __shared__ double v[256];
   __shared__ double r[256];
   __shared__ double red[8];
@@ -92,7 +94,9 @@ __global__ void __launch_bounds__(256) k_haar_cgs2(const double* __restrict__ G,
   }
   for (int64_t e = tid; e < (int64_t)p * p; e += blockDim.x) {
     const int row = (int)(e / p), col = (int)(e % p);
-    Q[e] = (float)Qc[(int64_t)col * p + row];
+    const double x = Qc[(int64_t)col * p + row];
+    Q[e] = (float)x;
+    Q64[e] = x;
   }
 }
 
