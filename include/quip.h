@@ -187,6 +187,9 @@ quip_status quip_incoherence_inverse(const quip_transform* tf, const float* W_ha
  * pivots; the diagonal and lower triangle of H_t are unspecified.
  * A pivot <= 0 or non-finite sets QUIP_ERR_NOT_PD in the status word
  * (quip_sync_status).  ws: QUIP_OP_LDL.
+ * Part of the trailing update runs on a second stream of the current device
+ * (created on first use, kept for the process); it forks from and joins back
+ * into `stream` by events, so the call is ordered on `stream` like any other.
  */
 quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
                      void* stream);

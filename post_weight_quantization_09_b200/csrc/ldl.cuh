@@ -11,6 +11,9 @@
 //     R_pp        = backward Cholesky of the updated diagonal block  (1 CTA)
 //     R[:p, p]    = H[:p, p] R_pp^-T                      (row-parallel solve)
 //     H[:p, :p]  -= R[:p, p] R[:p, p]^T   (upper triangle; trailing update)
+// The trailing update is split in two (look-ahead): the columns of panel
+// p - 1 first, on the critical path, then the rest on a second stream, where
+// it overlaps the next panel's diagonal factor and row solve.
 // Everything in place in the upper triangle of H (row-major, stride n).
 #pragma once
 
@@ -162,31 +165,23 @@ __device__ bool ldl_factor_diag(float* A, float* X, float* rb, float* rk, int* b
   return *bad == 0;
 }
 
-// One panel of the backward blocked factorisation, columns [c0, c0 + w), w <= 128:
-// every CTA loads and factors the diagonal block (the same deterministic
-// computation in each, so all agree), CTA 0 writes R_pp to Rd (a 128 x 128
-// slot of the workspace: H's own diagonal block must stay intact until every
-// CTA of the launch, possibly in a later wave, has read it), and each
-// CTA solves 64 rows of R12 = H12 R_pp^-T by block back substitution over the
-// four 32-column blocks (J = 3 .. 0):
-//   t_J = h_J - sum_{K > J} r_K R_JK^T,   r_J = t_J X_JJ^T,
-// with a 2 x 4 register tile per thread (rows 2 ty, 2 ty + 1; columns tx + 8 c).
-// R12 goes back into H's columns [c0, c0 + 128) and, as three bf16 pieces,
-// into Rs[p][i][k] (piece stride n * 128, row stride 128; columns >= w zero).
-// Grid: max(1, ceil(c0 / 64)) CTAs of 256 threads.
-// Dynamic smem: 128 x 129 (R_pp) + 64 x 129 (row tile) + 4 x 32 x 33 floats.
-__global__ void __launch_bounds__(256) k_ldl_panel(float* __restrict__ H, int64_t n, int64_t c0,
-                                                   int w, __nv_bfloat16* __restrict__ Rs,
-                                                   float* __restrict__ Rd) {
+// Diagonal block of one panel, columns [c0, c0 + w), w <= 128, by one CTA:
+// load the updated block (identity-padded past w), factor it
+// (ldl_factor_diag), write R_pp to Rd (128 x 128, upper triangle valid) and
+// the inverses X_JJ of its 32 x 32 diagonal blocks to Xw (4 x 32 x 33).
+// R_pp goes to the workspace, not into H: H's own diagonal blocks are copied
+// in by k_ldl_scatter_diag after the last panel.
+// Dynamic smem: 128 x 129 + 4 x 32 x 33 floats.
+__global__ void __launch_bounds__(256) k_ldl_diag(const float* __restrict__ H, int64_t n,
+                                                  int64_t c0, int w, float* __restrict__ Rd,
+                                                  float* __restrict__ Xw) {
   extern __shared__ __align__(16) float sm[];
   float* R = sm;                                  // 128 x LDL_LD
-  float* T = R + LDL_PB * LDL_LD;                 // 64 x LDL_LD
-  float* X = T + 64 * LDL_LD;                     // 4 x 32 x 33
+  float* X = R + LDL_PB * LDL_LD;                 // 4 x 32 x 33
   __shared__ __align__(16) float rb[32];
   __shared__ float rk[32];
   __shared__ int bad;
   const int tid = threadIdx.x;
-  const int64_t r0 = (int64_t)blockIdx.x * 64;
 #pragma unroll 4
   for (int e = tid; e < LDL_PB * 32; e += 256) {
     const int i = e >> 5, j4 = (e & 31) * 4;
@@ -200,6 +195,43 @@ __global__ void __launch_bounds__(256) k_ldl_panel(float* __restrict__ H, int64_
       d[c] = (i < w && j < w) ? (j >= i ? vv[c] : 0.f) : (i == j ? 1.f : 0.f);
     }
   }
+  __syncthreads();
+  const bool ok = ldl_factor_diag(R, X, rb, rk, &bad);
+  if (!ok && tid == 0) record_status(QUIP_ERR_NOT_PD);
+#pragma unroll 4
+  for (int e = tid; e < LDL_PB * LDL_PB; e += 256) Rd[e] = R[(e >> 7) * LDL_LD + (e & 127)];
+  for (int e = tid; e < 4 * 32 * 33; e += 256) Xw[e] = X[e];
+}
+
+// Rows [64 b, 64 b + 64) of R12 = H12 R_pp^-T for one panel (H12 = H[:c0,
+// c0:c0+w]), from the panel's R_pp (Rd) and X_JJ (Xw), by block back
+// substitution over the four 32-column blocks (J = 3 .. 0):
+//   t_J = h_J - sum_{K > J} r_K R_JK^T,   r_J = t_J X_JJ^T,
+// with a 2 x 4 register tile per thread (rows 2 ty, 2 ty + 1; columns tx + 8 c).
+// R12 goes back into H's columns [c0, c0 + w) and, as three bf16 pieces,
+// into Rs[q][i][k] (piece stride n * 128, row stride 128; columns >= w zero).
+// Grid: ceil(c0 / 64) CTAs of 256 threads.
+// Dynamic smem: 96 x 129 (the rows of R_pp that hold blocks R_JK, J < K)
+// + 64 x 129 (row tile) + 4 x 32 x 33 floats.
+constexpr int LDL_RROWS = 96;
+__global__ void __launch_bounds__(256) k_ldl_rows(float* __restrict__ H, int64_t n, int64_t c0,
+                                                  int w, const float* __restrict__ Rd,
+                                                  const float* __restrict__ Xw,
+                                                  __nv_bfloat16* __restrict__ Rs) {
+  extern __shared__ __align__(16) float sm[];
+  float* R = sm;                                  // 96 x LDL_LD
+  float* T = R + LDL_RROWS * LDL_LD;              // 64 x LDL_LD
+  float* X = T + 64 * LDL_LD;                     // 4 x 32 x 33
+  const int tid = threadIdx.x;
+  const int64_t r0 = (int64_t)blockIdx.x * 64;
+#pragma unroll 4
+  for (int e = tid; e < LDL_RROWS * 32; e += 256) {
+    const int i = e >> 5, j4 = (e & 31) * 4;
+    const float4 v = *reinterpret_cast<const float4*>(Rd + i * LDL_PB + j4);
+    float* d = R + i * LDL_LD + j4;
+    d[0] = v.x, d[1] = v.y, d[2] = v.z, d[3] = v.w;
+  }
+  for (int e = tid; e < 4 * 32 * 33; e += 256) X[e] = Xw[e];
 #pragma unroll 4
   for (int e = tid; e < 64 * 32; e += 256) {
     const int i = e >> 5, j4 = (e & 31) * 4;
@@ -213,13 +245,6 @@ __global__ void __launch_bounds__(256) k_ldl_panel(float* __restrict__ H, int64_
     d[3] = (j4 + 3 < w) ? v.w : 0.f;
   }
   __syncthreads();
-  const bool ok = ldl_factor_diag(R, X, rb, rk, &bad);
-  if (blockIdx.x == 0) {
-    if (!ok && tid == 0) record_status(QUIP_ERR_NOT_PD);
-#pragma unroll 4
-    for (int e = tid; e < LDL_PB * LDL_PB; e += 256) Rd[e] = R[(e >> 7) * LDL_LD + (e & 127)];
-  }
-  if (c0 == 0) return;
   const int ty = tid >> 3, tx = tid & 7;
   const int i0 = 2 * ty;
   for (int J = 3; J >= 0; --J) {

@@ -86,6 +86,30 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint6
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A second stream and two events per device for the LDL look-ahead, created
+// on first use and kept for the life of the process.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+cudaError_t side_stream(SideStream& out) {
+  static std::mutex mu;
+  static SideStream per_dev[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  SideStream& ss = per_dev[dev];
+  if (!ss.s) {
+    if ((e = cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+  }
+  out = ss;
+  return cudaSuccess;
+}
+
 int num_sms() {
   static int sms = 0;
   if (!sms) {
@@ -98,8 +122,9 @@ int num_sms() {
 }
 
 // C (+)= alpha * (3-piece A) (3-piece B)^T on the tensor cores; see gemm_tc.cuh.
+// max_ctas > 0 caps the persistent grid (leaves SMs to a concurrent stream).
 cudaError_t split_gemm(const CUtensorMap& ta, const CUtensorMap& tb, sgemm::Params p,
-                       cudaStream_t st) {
+                       cudaStream_t st, int max_ctas = 0) {
   if (p.M <= 0 || p.N <= 0) return cudaSuccess;
   static bool attr = false;
   if (!attr) {
@@ -115,7 +140,8 @@ cudaError_t split_gemm(const CUtensorMap& ta, const CUtensorMap& tb, sgemm::Para
   for (int ti = 0; ti < tm; ++ti)
     for (int tj = 0; tj < tn; ++tj)
       if (!(p.upper_only && ti * sgemm::BM > tj * sgemm::BN + sgemm::BN - 1)) ++valid;
-  const int grid = std::max(1, std::min(valid, num_sms()));
+  const int cap = max_ctas > 0 ? std::min(max_ctas, num_sms()) : num_sms();
+  const int grid = std::max(1, std::min(valid, cap));
   sgemm::k_gemm_split_tc<<<grid, 256, sgemm::SMEM_BYTES, st>>>(ta, tb, p, tm * tn); count_launch();
   return cudaGetLastError();
 }
@@ -512,8 +538,12 @@ quip_status quip_hessian_finalize(float* H, int64_t n, int64_t N_total, float da
 // LDL workspace: the panels' diagonal factor blocks (P x 128 x 128 fp32), then
 // the current panel's three bf16 pieces (3 x n x 128).
 static int64_t ldl_panels(int64_t n) { return (n + LDL_PB - 1) / LDL_PB; }
+// LDL workspace: every panel's R_pp (128 x 128 fp32) and X_JJ blocks
+// (4 x 32 x 33 fp32), and two buffers of a panel's R12 as 3 bf16 pieces.
+constexpr size_t LDL_XW = 4 * 32 * 33;
 static size_t ldl_ws_bytes(int64_t n) {
-  return round256((size_t)ldl_panels(n) * LDL_PB * LDL_PB * 4) + round256((size_t)3 * n * LDL_PB * 2);
+  return round256((size_t)ldl_panels(n) * LDL_PB * LDL_PB * 4) +
+         round256((size_t)ldl_panels(n) * LDL_XW * 4) + round256((size_t)6 * n * LDL_PB * 2);
 }
 // LDLQ workspace: accumulator A (m x n fp32), the error of every column as
 // three bf16 pieces (3 x m x n), the split transposed factor (3 x n x n bf16).
@@ -631,37 +661,70 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
   quip_status s = check_ws(ws, ws_bytes, ldl_ws_bytes(n));
   if (s != QUIP_OK) return s;
   cudaStream_t st = S(stream);
+  const int64_t P = ldl_panels(n);
   float* Rd = static_cast<float*>(ws);
+  float* Xw = reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                       round256((size_t)P * LDL_PB * LDL_PB * 4));
   __nv_bfloat16* Rs = reinterpret_cast<__nv_bfloat16*>(
-      static_cast<char*>(ws) + round256((size_t)ldl_panels(n) * LDL_PB * LDL_PB * 4));
-  const size_t smem_panel = ((size_t)(LDL_PB + 64) * LDL_LD + 4 * 32 * 33) * sizeof(float);
+      reinterpret_cast<char*>(Xw) + round256((size_t)P * LDL_XW * 4));
+  const size_t smem_diag = ((size_t)LDL_PB * LDL_LD + LDL_XW) * sizeof(float);
+  const size_t smem_rows = ((size_t)(LDL_RROWS + 64) * LDL_LD + LDL_XW) * sizeof(float);
   static bool attr = false;
   if (!attr) {
-    QCHECK(cudaFuncSetAttribute(k_ldl_panel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem_panel));
+    QCHECK(cudaFuncSetAttribute(k_ldl_diag, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem_diag));
+    QCHECK(cudaFuncSetAttribute(k_ldl_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem_rows));
     attr = true;
   }
+  // Rs holds two panels' R12 (buffer p & 1), pieces at rows (3 buf + q) n.
   CUtensorMap ta, tb;
   if (n > LDL_PB) {
-    if (!make_tmap_bf16_2d(&ta, Rs, LDL_PB, 3 * (uint64_t)n, LDL_PB * 2, 64, sgemm::BM) ||
-        !make_tmap_bf16_2d(&tb, Rs, LDL_PB, 3 * (uint64_t)n, LDL_PB * 2, 64, sgemm::BN))
+    if (!make_tmap_bf16_2d(&ta, Rs, LDL_PB, 6 * (uint64_t)n, LDL_PB * 2, 64, sgemm::BM) ||
+        !make_tmap_bf16_2d(&tb, Rs, LDL_PB, 6 * (uint64_t)n, LDL_PB * 2, 64, sgemm::BN))
       return QUIP_ERR_CUDA;
   }
-  const int64_t P = (n + LDL_PB - 1) / LDL_PB;
+  SideStream side;
+  if (P > 2) QCHECK(side_stream(side));
+  bool bulk_pending = false;
   for (int64_t p = P - 1; p >= 0; --p) {
     const int64_t c0 = p * LDL_PB;
     const int w = (int)std::min<int64_t>(LDL_PB, n - c0);
-    const unsigned grid = (unsigned)std::max<int64_t>(1, (c0 + 63) / 64);
-    k_ldl_panel<<<grid, 256, smem_panel, st>>>(H_t, n, c0, w, Rs, Rd + p * LDL_PB * LDL_PB);
+    const int buf = (int)(p & 1);
+    float* Rdp = Rd + p * LDL_PB * LDL_PB;
+    float* Xwp = Xw + p * LDL_XW;
+    k_ldl_diag<<<1, 256, smem_diag, st>>>(H_t, n, c0, w, Rdp, Xwp);
     count_launch();
-    if (c0 > 0) {
-      // H[:c0, :c0] -= R12 R12^T on the upper tiles
+    if (c0 == 0) break;
+    k_ldl_rows<<<(unsigned)((c0 + 63) / 64), 256, smem_rows, st>>>(H_t, n, c0, w, Rdp, Xwp,
+                                                                   Rs + (size_t)buf * 3 * n * LDL_PB);
+    count_launch();
+    // Look-ahead: H[:c0, panel p - 1] -= R12 R12[panel p - 1]^T.  It adds into
+    // the region the previous bulk update also adds into, so it waits for
+    // that update (a fixed order of the two additions per element).
+    if (bulk_pending) QCHECK(cudaStreamWaitEvent(st, side.join, 0));
+    sgemm::Params la{};
+    la.C = H_t + (c0 - LDL_PB), la.ldc = n, la.M = (int)c0, la.N = LDL_PB, la.K = LDL_PB;
+    la.a_piece_rows = (int)n, la.b_piece_rows = (int)n;
+    la.a_row0 = 3 * (int)n * buf, la.b_row0 = 3 * (int)n * buf + (int)(c0 - LDL_PB);
+    la.alpha = -1.f, la.upper_only = 0;
+    QCHECK(split_gemm(ta, tb, la, st));
+    if (c0 > LDL_PB) {
+      // The rest, H[:c0-128, :c0-128] -= R12 R12^T on the upper tiles, on the
+      // side stream; a few SMs stay free for the next diagonal factor.
+      QCHECK(cudaEventRecord(side.fork, st));
+      QCHECK(cudaStreamWaitEvent(side.s, side.fork, 0));
       sgemm::Params gp{};
-      gp.C = H_t, gp.ldc = n, gp.M = (int)c0, gp.N = (int)c0, gp.K = LDL_PB;
-      gp.a_piece_rows = (int)n, gp.b_piece_rows = (int)n, gp.alpha = -1.f, gp.upper_only = 1;
-      QCHECK(split_gemm(ta, tb, gp, st));
+      gp.C = H_t, gp.ldc = n, gp.M = (int)(c0 - LDL_PB), gp.N = (int)(c0 - LDL_PB), gp.K = LDL_PB;
+      gp.a_piece_rows = (int)n, gp.b_piece_rows = (int)n;
+      gp.a_row0 = gp.b_row0 = 3 * (int)n * buf;
+      gp.alpha = -1.f, gp.upper_only = 1;
+      QCHECK(split_gemm(ta, tb, gp, side.s, num_sms() - 2));
+      QCHECK(cudaEventRecord(side.join, side.s));
+      bulk_pending = true;
     }
   }
+  if (bulk_pending) QCHECK(cudaStreamWaitEvent(st, side.join, 0));
   k_ldl_scatter_diag<<<(unsigned)P, 256, 0, st>>>(H_t, n, Rd); count_launch();
   k_diag_to<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(H_t, n, D); count_launch();
   k_scale_upper<<<(unsigned)n, 256, 0, st>>>(H_t, n, D); count_launch();
