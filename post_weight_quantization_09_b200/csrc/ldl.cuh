@@ -6,14 +6,25 @@
 //
 // Computed as H = R R^T with R upper triangular ("backward" Cholesky), then
 // D_k = R_kk^2 and Ů_jk = R_jk / R_kk.  Blocked right-looking from the
-// bottom-right, panel width PB:
-//   for p = P-1 .. 0 (columns [p*PB, (p+1)*PB)):
-//     R_pp        = backward Cholesky of the updated diagonal block  (1 CTA)
-//     R[:p, p]    = H[:p, p] R_pp^-T                      (row-parallel solve)
-//     H[:p, :p]  -= R[:p, p] R[:p, p]^T   (upper triangle; trailing update)
-// The trailing update is split in two (look-ahead): the columns of panel
-// p - 1 first, on the critical path, then the rest on a second stream, where
-// it overlaps the next panel's diagonal factor and row solve.
+// bottom-right in panels of PB = 128 columns; panel p covers columns
+// [c0, c0 + w), c0 = 128 p, and R12(p) = R[:c0, panel p]:
+//
+//   k_ldl_factor(p)  R_pp = backward Cholesky of the updated diagonal block,
+//                    with the inverses X_J of its four 32 x 32 diagonal
+//                    blocks, and the 128 "next" rows R12(p)[c0-128 : c0]
+//                    (4 CTAs, each factors the block redundantly and solves
+//                    32 of those rows);
+//   k_ldl_rows(p)    R12(p) = H[:c0, panel p] R_pp^-T (16 rows per CTA) and
+//                    the look-ahead product L(p) = R12(p) R12(p)[c0-128:c0]^T,
+//                    i.e. panel p's update of panel p - 1, into a side buffer;
+//   bulk(p)          H[:c0-128, :c0-128] -= R12 R12^T (upper tiles; tensor-
+//                    core split GEMM on a second stream, quip_api.cu).
+//
+// Panel p - 1 is read as H - L(p): every element of a column panel receives
+// its updates in panel order (the bulk updates in stream order, then L(p)),
+// as in the unblocked factorisation, so the result does not depend on how
+// the two streams interleave.  The bulk update of panel p + 1 overlaps the
+// factor and row kernels of panel p.
 // Everything in place in the upper triangle of H (row-major, stride n).
 #pragma once
 
@@ -23,298 +34,470 @@
 namespace quip {
 
 constexpr int LDL_PB = 128;
-constexpr int LDL_LD = LDL_PB + 1;     // padded shared-memory row
+constexpr int LDL_LDA = 132;    // smem row stride of 128-wide tiles (16-B rows)
+constexpr int LDL_LDX = 36;     // smem row stride of 32-wide tiles (16-B rows)
+constexpr int LDL_FT = 512;     // threads of k_ldl_factor
+constexpr int LDL_FCTAS = 4;    // CTAs of k_ldl_factor when c0 > 0 (32 next rows each)
+constexpr int LDL_RT = 256;     // threads of k_ldl_rows
+constexpr int LDL_RR = 16;      // rows per k_ldl_rows CTA
+constexpr int LDL_HT = 384;     // helper threads of k_ldl_factor (warps w % 4 != 0)
 
-// ---------------------------------------------------------------- warp-level 32 x 32 blocks
+// ---------------------------------------------------------------- helpers
 
-// Backward Cholesky and inverse of a 32 x 32 block in one sweep, one warp,
-// everything in registers: lane i keeps row i of A (a[]) and column i of
-// X = R^-1 (x[]).  Step k (31 .. 0): the pivot comes from lane k by shuffle;
-// 1 / sqrt(A_kk) is one rsqrt (a few ulp, far inside the fp32 factorisation
-// error); lane i forms R[i][k]; row k of R is read from lane k by shuffles to
-// form x_kj = (delta_kj - sum_{m>k} R_km x_mj) / R_kk; the leading block is
-// updated with the new column, the entry the next pivot needs first.
-// S: block (upper triangle read, R written back); Xo: X (32 x 32, full).
-// Returns false (warp-uniform) if a pivot is not positive.
-__device__ __forceinline__ bool warp_chol_inv32(float* S, int lds, float* Xo, int ldx) {
-  const int lane = threadIdx.x & 31;
-  float a[32], x[32];
+// acc[a][b] += sum_{t < len} P[a * ps + t] * Q[b * qs + t]; len % 4 == 0,
+// every row 16-byte aligned.  Sums run in t order.
+template <int NA, int NB>
+__device__ __forceinline__ void dot_rows(float (&acc)[NA][NB], const float* P, int ps,
+                                         const float* Q, int qs, int len) {
+#pragma unroll 2
+  for (int t = 0; t < len; t += 4) {
+    float4 pv[NA], qv[NB];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    a[j] = (j >= lane) ? S[lane * lds + j] : S[j * lds + lane];
-    x[j] = 0.f;
+    for (int a = 0; a < NA; ++a) pv[a] = *reinterpret_cast<const float4*>(P + a * ps + t);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) qv[b] = *reinterpret_cast<const float4*>(Q + b * qs + t);
+#pragma unroll
+    for (int a = 0; a < NA; ++a)
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        acc[a][b] = fmaf(pv[a].x, qv[b].x, acc[a][b]);
+        acc[a][b] = fmaf(pv[a].y, qv[b].y, acc[a][b]);
+        acc[a][b] = fmaf(pv[a].z, qv[b].z, acc[a][b]);
+        acc[a][b] = fmaf(pv[a].w, qv[b].w, acc[a][b]);
+      }
+  }
+}
+
+__device__ __forceinline__ void helpers_sync() {      // the helper warps of k_ldl_factor
+  asm volatile("bar.sync 1, %0;" ::"n"(LDL_HT) : "memory");
+}
+
+// Backward Cholesky of a 32 x 32 block S (upper triangle read, row stride
+// lds, 16-byte rows) and the inverse of its factor, by one warp.  Lane i
+// keeps row i of the block in registers (only j >= i is ever used).  Step k
+// (31 .. 0): the pivot comes by shuffle from lane k, which formed it from its
+// own previous column entry (so the chain from pivot to pivot is one
+// shuffle, one rsqrtf, one multiply and one fma); lane i forms
+// R[i][k] = l_i, publishes it in a double-buffered shared column and
+// updates its row with the column's entries l_j, j < k (broadcast 16-byte
+// loads).  1 / R_kk is the rsqrtf of the pivot.  Then X = R^-1 column by
+// column (lane j: column j), right-looking back substitution over the
+// columns of R, read as broadcast rows of a transposed copy.
+// scratch: 32 x LDL_LDX + 64 floats.  On return S's upper triangle holds R
+// (its lower triangle zero) and X (row stride ldx, lower part zero) holds
+// R^-1.  Returns false (warp-uniform) if a pivot was not positive and finite.
+__device__ __forceinline__ bool warp_chol_inv32(float* S, int lds, float* X, int ldx,
+                                                float* scratch) {
+  const int lane = threadIdx.x & 31;
+  float a[32], rin[32];
+  float* col = scratch + 32 * LDL_LDX;            // 2 x 32
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 v = *reinterpret_cast<const float4*>(S + lane * lds + 4 * q);
+    a[4 * q + 0] = (4 * q + 0 >= lane) ? v.x : 0.f;
+    a[4 * q + 1] = (4 * q + 1 >= lane) ? v.y : 0.f;
+    a[4 * q + 2] = (4 * q + 2 >= lane) ? v.z : 0.f;
+    a[4 * q + 3] = (4 * q + 3 >= lane) ? v.w : 0.f;
   }
   bool ok = true;
+  float self = a[31];
 #pragma unroll
   for (int k = 31; k >= 0; --k) {
-    const float d = __shfl_sync(0xffffffffu, a[k], k);
-    ok = ok && (d > 0.f) && isfinite(d);
-    const float ir = rsqrtf(d);
-    const float l = (lane == k) ? d * ir : a[k] * ir;
+    const float piv = __shfl_sync(0xffffffffu, self, k);
+    ok = ok && (piv > 0.f) && (piv < INFINITY);
+    const float r = rsqrtf(piv);
+    rin[k] = r;
+    const float l = (lane == k) ? piv * r : a[k] * r;
     a[k] = l;
+    if (k > 0) {
+      self = fmaf(-l, l, a[k - 1]);        // lane k - 1: its next pivot
+      float* cb = col + (k & 1) * 32;
+      cb[lane] = l;
+      __syncwarp();
 #pragma unroll
-    for (int j = k - 1; j >= 0; --j) a[j] = fmaf(-l, __shfl_sync(0xffffffffu, l, j), a[j]);
-    float s0 = (lane == k) ? 1.f : 0.f, s1 = 0.f;
-#pragma unroll
-    for (int m = k + 1; m < 32; m += 2) {
-      s0 = fmaf(-__shfl_sync(0xffffffffu, a[m], k), x[m], s0);
-      if (m + 1 < 32) s1 = fmaf(-__shfl_sync(0xffffffffu, a[m + 1], k), x[m + 1], s1);
+      for (int j4 = 0; j4 < k; j4 += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(cb + j4);
+        if (j4 + 0 < k) a[j4 + 0] = fmaf(-l, v.x, a[j4 + 0]);
+        if (j4 + 1 < k) a[j4 + 1] = fmaf(-l, v.y, a[j4 + 1]);
+        if (j4 + 2 < k) a[j4 + 2] = fmaf(-l, v.z, a[j4 + 2]);
+        if (j4 + 3 < k) a[j4 + 3] = fmaf(-l, v.w, a[j4 + 3]);
+      }
     }
-    x[k] = (lane >= k) ? (s0 + s1) * ir : 0.f;
   }
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    if (j >= lane) S[lane * lds + j] = a[j];
-    Xo[j * ldx + lane] = x[j];
+  for (int q = 0; q < 8; ++q) {
+    const float4 v = make_float4(4 * q + 0 >= lane ? a[4 * q + 0] : 0.f, 4 * q + 1 >= lane ? a[4 * q + 1] : 0.f,
+                                 4 * q + 2 >= lane ? a[4 * q + 2] : 0.f, 4 * q + 3 >= lane ? a[4 * q + 3] : 0.f);
+    *reinterpret_cast<float4*>(S + lane * lds + 4 * q) = v;
   }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) scratch[j * LDL_LDX + lane] = (j >= lane) ? a[j] : 0.f;   // row j = column j of R
+  __syncwarp();
+  float x[32];
+#pragma unroll
+  for (int m = 0; m < 32; ++m) x[m] = (m == lane) ? 1.f : 0.f;
+#pragma unroll
+  for (int k = 31; k >= 0; --k) {
+    x[k] *= rin[k];
+    const float* rc = scratch + k * LDL_LDX;
+#pragma unroll
+    for (int m4 = 0; m4 < k; m4 += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(rc + m4);
+      if (m4 + 0 < k) x[m4 + 0] = fmaf(-v.x, x[k], x[m4 + 0]);
+      if (m4 + 1 < k) x[m4 + 1] = fmaf(-v.y, x[k], x[m4 + 1]);
+      if (m4 + 2 < k) x[m4 + 2] = fmaf(-v.z, x[k], x[m4 + 2]);
+      if (m4 + 3 < k) x[m4 + 3] = fmaf(-v.w, x[k], x[m4 + 3]);
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < 32; ++m) X[m * ldx + lane] = x[m];
   __syncwarp();
   return ok;
 }
 
-// Factor the panel's 128 x 128 diagonal block held in shared memory A
-// (rows of LDL_LD floats, upper triangle valid, identity-padded past w) as
-// 4 x 4 blocks of 32, by the whole CTA (256 threads).  For J = 3 .. 0:
-//   warp 0:  A_JJ = R_JJ R_JJ^T and X_JJ = R_JJ^-1 (warp_chol_inv32);
-//   all:     R_IJ = A_IJ X_JJ^T for the rows above (I < J);
-//   all:     the next diagonal block A_{J-1,J-1} -= R_{J-1,J} R_{J-1,J}^T;
-//   warps 1-7 (while warp 0 factors block J-1): the rest of
-//            A[0:32J, 0:32J] -= R[0:32J, J] R[0:32J, J]^T (upper part).
-// On return A's upper triangle holds R and X[J] (32 x 33 each) the inverses.
-// Returns false if a pivot was not positive.
-__device__ bool ldl_factor_diag(float* A, float* X, float* rb, float* rk, int* bad) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  (void)rk;
-  if (tid == 0) *bad = 0;
-  __syncthreads();
-  for (int J = 3; J >= 0; --J) {
-    float* XJ = X + J * 32 * 33;
-    if (warp == 0) {
-      const bool ok = warp_chol_inv32(A + (32 * J) * LDL_LD + 32 * J, LDL_LD, XJ, 33);
-      if (!ok && lane == 0) *bad = 1;
-    }
-    __syncthreads();                              // also orders the rest-update of J + 1
-    if (J == 0) break;
-    const int rows = 32 * J;
-    {
-      float out[3][4];
-      const int k0 = tid & 7, ib = tid >> 3;
+// ---------------------------------------------------------------- block steps on shared tiles
+// Tiles are row-major 128-wide (stride LDL_LDA) or 32-wide (stride
+// LDL_LDX).  Each step maps tasks of 2 x 2 outputs onto threads
+// [t0, t0 + nt): rows (ti, ti + h) and columns (tk, tk + 16), consecutive
+// threads on consecutive columns (conflict-free 16-byte loads).
+
+// R_IJ = A_IJ X_J^T for rows [i0, i0 + nr) of column block J, in place
+// (nr even, <= 2 * 16 * 2 tasks per thread: nr * 8 <= 2 nt).  `bar` syncs the
+// participating threads between the reads and the writes.
+template <typename Bar>
+__device__ __forceinline__ void blk_trsm(float* A, const float* XJ, int J, int i0, int nr, int t,
+                                         int nt, Bar bar) {
+  const int h = nr / 2, ntask = h * 16;
+  float out[2][2][2];
+  int tasks[2];
 #pragma unroll
-      for (int rg = 0; rg < 3; ++rg) {
-        const int i = ib + 32 * rg;
+  for (int u = 0; u < 2; ++u) {
+    const int e = t + u * nt;
+    tasks[u] = e;
+    if (e < ntask) {
+      const int ti = e >> 4, tk = e & 15;
+      float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+      dot_rows<2, 2>(acc, A + (i0 + ti) * LDL_LDA + 32 * J, h * LDL_LDA, XJ + tk * LDL_LDX,
+                     16 * LDL_LDX, 32);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) out[rg][c] = 0.f;
-        if (i < rows) {
-          const float* ar = A + i * LDL_LD + 32 * J;
-#pragma unroll 8
-          for (int t = 0; t < 32; ++t) {
-            const float av = ar[t];
+      for (int a = 0; a < 2; ++a)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) out[rg][c] = fmaf(av, XJ[(k0 + 8 * c) * 33 + t], out[rg][c]);
-          }
-        }
-      }
-      __syncthreads();
-#pragma unroll
-      for (int rg = 0; rg < 3; ++rg) {
-        const int i = ib + 32 * rg;
-        if (i < rows)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) A[i * LDL_LD + 32 * J + k0 + 8 * c] = out[rg][c];
-      }
-      __syncthreads();
-    }
-    {
-      const int i = 32 * (J - 1) + (tid >> 3);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int k = 32 * (J - 1) + (tid & 7) + 8 * c;
-        if (k < i) continue;
-        const float* ri = A + i * LDL_LD + 32 * J;
-        const float* rr = A + k * LDL_LD + 32 * J;
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int t = 0; t < 32; t += 2) {
-          s0 = fmaf(ri[t], rr[t], s0);
-          s1 = fmaf(ri[t + 1], rr[t + 1], s1);
-        }
-        A[i * LDL_LD + k] -= s0 + s1;
-      }
-    }
-    __syncthreads();
-    if (warp > 0) {
-      const int nr = 32 * (J - 1);
-      const int t0 = tid - 32, nt = 224;
-      for (int e = t0; e < nr * rows; e += nt) {
-        const int i = e / rows, k = e % rows;
-        if (k < i) continue;
-        const float* ri = A + i * LDL_LD + 32 * J;
-        const float* rr = A + k * LDL_LD + 32 * J;
-        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-        for (int t = 0; t < 32; t += 4) {
-          s0 = fmaf(ri[t], rr[t], s0);
-          s1 = fmaf(ri[t + 1], rr[t + 1], s1);
-          s2 = fmaf(ri[t + 2], rr[t + 2], s2);
-          s3 = fmaf(ri[t + 3], rr[t + 3], s3);
-        }
-        A[i * LDL_LD + k] -= (s0 + s1) + (s2 + s3);
-      }
+        for (int b = 0; b < 2; ++b) out[u][a][b] = acc[a][b];
     }
   }
-  __syncthreads();
-  return *bad == 0;
+  bar();
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int e = tasks[u];
+    if (e < ntask) {
+      const int ti = e >> 4, tk = e & 15;
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b = 0; b < 2; ++b) A[(i0 + ti + a * h) * LDL_LDA + 32 * J + tk + 16 * b] = out[u][a][b];
+    }
+  }
+  bar();
 }
 
-// Diagonal block of one panel, columns [c0, c0 + w), w <= 128, by one CTA:
-// load the updated block (identity-padded past w), factor it
-// (ldl_factor_diag), write R_pp to Rd (128 x 128, upper triangle valid) and
-// the inverses X_JJ of its 32 x 32 diagonal blocks to Xw (4 x 32 x 33).
-// R_pp goes to the workspace, not into H: H's own diagonal blocks are copied
-// in by k_ldl_scatter_diag after the last panel.
-// Dynamic smem: 128 x 129 + 4 x 32 x 33 floats.
-__global__ void __launch_bounds__(256) k_ldl_diag(const float* __restrict__ H, int64_t n,
-                                                  int64_t c0, int w, float* __restrict__ Rd,
-                                                  float* __restrict__ Xw) {
+// A[i][j] -= sum_t R[i][32J + t] R[j][32J + t] (R = A's column block J) for
+// the upper elements (j >= i) of rows [i0, i0 + nr) x columns [j0, j0 + nc)
+// (nr, nc even).  Tasks: rows (ti, ti + nr/2), columns (tj, tj + nc/2).
+__device__ __forceinline__ void blk_update(float* A, int J, int i0, int nr, int j0, int nc, int t,
+                                           int nt) {
+  const int hr = nr / 2, hc = nc / 2, ntask = hr * hc;
+  for (int e = t; e < ntask; e += nt) {
+    const int ti = e / hc, tj = e % hc;
+    const int ia = i0 + ti, ja = j0 + tj;
+    if (ia > ja + hc) continue;                       // all four below the diagonal
+    float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    dot_rows<2, 2>(acc, A + ia * LDL_LDA + 32 * J, hr * LDL_LDA, A + ja * LDL_LDA + 32 * J,
+                   hc * LDL_LDA, 32);
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const int i = ia + a * hr, j = ja + b * hc;
+        if (j >= i) A[i * LDL_LDA + j] -= acc[a][b];
+      }
+  }
+}
+
+// One column block J of the back substitution R12 = T R_pp^-T for an
+// NR-row tile T (stride LDL_LDA; columns of blocks K > J already solved):
+//   T[:, J] -= sum_{K > J} T[:, K] R_JK^T,   T[:, J] = T[:, J] X_J^T.
+// Rp: rows of R_pp (stride LDL_LDA), XJ: X_J (stride LDL_LDX).
+// NR * 8 tasks of 2 x 2: rows (ti, ti + NR/2), columns (tk, tk + 16); at
+// most two per thread.
+template <int NR, typename Bar>
+__device__ __forceinline__ void blk_solve(float* T, const float* Rp, const float* XJ, int J,
+                                          int t, int nt, Bar bar) {
+  constexpr int NTASK = NR * 8, HR = NR / 2;
+  float out[2][2][2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int e = t + u * nt;
+    if (e < NTASK && J < 3) {
+      const int ti = e >> 4, tk = e & 15;
+      float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+      const int c1 = 32 * (J + 1);
+      dot_rows<2, 2>(acc, T + ti * LDL_LDA + c1, HR * LDL_LDA, Rp + (32 * J + tk) * LDL_LDA + c1,
+                     16 * LDL_LDA, LDL_PB - c1);
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b = 0; b < 2; ++b) T[(ti + HR * a) * LDL_LDA + 32 * J + tk + 16 * b] -= acc[a][b];
+    }
+  }
+  bar();
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int e = t + u * nt;
+    if (e < NTASK) {
+      const int ti = e >> 4, tk = e & 15;
+      float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+      dot_rows<2, 2>(acc, T + ti * LDL_LDA + 32 * J, HR * LDL_LDA, XJ + tk * LDL_LDX,
+                     16 * LDL_LDX, 32);
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b = 0; b < 2; ++b) out[u][a][b] = acc[a][b];
+    }
+  }
+  bar();
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int e = t + u * nt;
+    if (e < NTASK) {
+      const int ti = e >> 4, tk = e & 15;
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b = 0; b < 2; ++b) T[(ti + HR * a) * LDL_LDA + 32 * J + tk + 16 * b] = out[u][a][b];
+    }
+  }
+  bar();
+}
+
+// ---------------------------------------------------------------- kernels
+
+// Factor of panel p, columns [c0, c0 + w), w <= 128.  Every CTA loads the
+// updated diagonal block (H - Lin, identity-padded past w) and factors it
+// (the same deterministic computation in each), as 4 x 4 blocks of 32:
+//   for J = 3 .. 0:
+//     warp 0:      R_JJ, X_J = R_JJ^-1                         (warp_chol_inv32)
+//     all:         R_{J-1,J} = A_{J-1,J} X_J^T;  A_{J-1,J-1} -= R_{J-1,J} R_{J-1,J}^T
+//     helpers (warps w % 4 != 0), while warp 0 factors block J - 1: the other rows of block
+//                  column J (R_IJ, I < J - 1), the rest of the trailing
+//                  update, and column block J of this CTA's 32 next rows
+//                  (blk_solve).
+// CTA c (when c0 > 0) solves next rows c0 - 128 + 32 c .. + 31 of R12(p)
+// into Nx (128 x 128, row i = global row c0 - 128 + i).  CTA 0 writes R_pp
+// (Rd, 128 x 128, upper; lower zero), X_J (Xw, 4 x 32 x 32) and D (Dv[c0 +
+// k] = R_kk^2); with c0 == 0 (the last panel, one CTA) it also writes the
+// block's Ů into H.  Lin: the look-ahead buffer of panel p + 1 (rows
+// [0, c0 + 128) x 128), or NULL.
+// Dynamic smem: (128 + 32) x LDL_LDA + 5 x 32 x LDL_LDX + 96 floats.
+__global__ void __launch_bounds__(LDL_FT, 1)
+    k_ldl_factor(float* __restrict__ H, int64_t n, int64_t c0, int w, const float* __restrict__ Lin,
+                 float* __restrict__ Rd, float* __restrict__ Xw, float* __restrict__ Nx,
+                 float* __restrict__ Dv) {
   extern __shared__ __align__(16) float sm[];
-  float* R = sm;                                  // 128 x LDL_LD
-  float* X = R + LDL_PB * LDL_LD;                 // 4 x 32 x 33
-  __shared__ __align__(16) float rb[32];
-  __shared__ float rk[32];
+  float* A = sm;                                     // 128 x LDL_LDA
+  float* T = A + LDL_PB * LDL_LDA;                   // 32 x LDL_LDA (next rows)
+  float* X = T + 32 * LDL_LDA;                       // 4 x 32 x LDL_LDX
+  float* scr = X + 4 * 32 * LDL_LDX;                 // 32 x LDL_LDX + 96
   __shared__ int bad;
-  const int tid = threadIdx.x;
-#pragma unroll 4
-  for (int e = tid; e < LDL_PB * 32; e += 256) {
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const bool has_next = c0 > 0;
+  if (tid == 0) bad = 0;
+#pragma unroll
+  for (int e = tid; e < LDL_PB * 32; e += LDL_FT) {
     const int i = e >> 5, j4 = (e & 31) * 4;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i < w && j4 < w) v = *reinterpret_cast<const float4*>(H + (c0 + i) * n + c0 + j4);
-    float* d = R + i * LDL_LD + j4;
-    const float vv[4] = {v.x, v.y, v.z, v.w};
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (i < w && j4 < w) {
+      const float4 h = *reinterpret_cast<const float4*>(H + (c0 + i) * n + c0 + j4);
+      v[0] = h.x, v[1] = h.y, v[2] = h.z, v[3] = h.w;
+      if (Lin) {
+        const float4 l = *reinterpret_cast<const float4*>(Lin + (c0 + i) * LDL_PB + j4);
+        v[0] -= l.x, v[1] -= l.y, v[2] -= l.z, v[3] -= l.w;
+      }
+    }
+    float o[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const int j = j4 + c;
-      d[c] = (i < w && j < w) ? (j >= i ? vv[c] : 0.f) : (i == j ? 1.f : 0.f);
+      o[c] = (i < w && j < w) ? (j >= i ? v[c] : 0.f) : (i == j ? 1.f : 0.f);
     }
+    *reinterpret_cast<float4*>(A + i * LDL_LDA + j4) = make_float4(o[0], o[1], o[2], o[3]);
   }
-  __syncthreads();
-  const bool ok = ldl_factor_diag(R, X, rb, rk, &bad);
-  if (!ok && tid == 0) record_status(QUIP_ERR_NOT_PD);
-#pragma unroll 4
-  for (int e = tid; e < LDL_PB * LDL_PB; e += 256) Rd[e] = R[(e >> 7) * LDL_LD + (e & 127)];
-  for (int e = tid; e < 4 * 32 * 33; e += 256) Xw[e] = X[e];
-}
-
-// Rows [64 b, 64 b + 64) of R12 = H12 R_pp^-T for one panel (H12 = H[:c0,
-// c0:c0+w]), from the panel's R_pp (Rd) and X_JJ (Xw), by block back
-// substitution over the four 32-column blocks (J = 3 .. 0):
-//   t_J = h_J - sum_{K > J} r_K R_JK^T,   r_J = t_J X_JJ^T,
-// with a 2 x 4 register tile per thread (rows 2 ty, 2 ty + 1; columns tx + 8 c).
-// R12 goes back into H's columns [c0, c0 + w) and, as three bf16 pieces,
-// into Rs[q][i][k] (piece stride n * 128, row stride 128; columns >= w zero).
-// Grid: ceil(c0 / 64) CTAs of 256 threads.
-// Dynamic smem: 96 x 129 (the rows of R_pp that hold blocks R_JK, J < K)
-// + 64 x 129 (row tile) + 4 x 32 x 33 floats.
-constexpr int LDL_RROWS = 96;
-__global__ void __launch_bounds__(256) k_ldl_rows(float* __restrict__ H, int64_t n, int64_t c0,
-                                                  int w, const float* __restrict__ Rd,
-                                                  const float* __restrict__ Xw,
-                                                  __nv_bfloat16* __restrict__ Rs) {
-  extern __shared__ __align__(16) float sm[];
-  float* R = sm;                                  // 96 x LDL_LD
-  float* T = R + LDL_RROWS * LDL_LD;              // 64 x LDL_LD
-  float* X = T + 64 * LDL_LD;                     // 4 x 32 x 33
-  const int tid = threadIdx.x;
-  const int64_t r0 = (int64_t)blockIdx.x * 64;
-#pragma unroll 4
-  for (int e = tid; e < LDL_RROWS * 32; e += 256) {
-    const int i = e >> 5, j4 = (e & 31) * 4;
-    const float4 v = *reinterpret_cast<const float4*>(Rd + i * LDL_PB + j4);
-    float* d = R + i * LDL_LD + j4;
-    d[0] = v.x, d[1] = v.y, d[2] = v.z, d[3] = v.w;
-  }
-  for (int e = tid; e < 4 * 32 * 33; e += 256) X[e] = Xw[e];
-#pragma unroll 4
-  for (int e = tid; e < 64 * 32; e += 256) {
-    const int i = e >> 5, j4 = (e & 31) * 4;
-    const int64_t gi = r0 + i;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (gi < c0 && j4 < w) v = *reinterpret_cast<const float4*>(H + gi * n + c0 + j4);
-    float* d = T + i * LDL_LD + j4;
-    d[0] = (j4 < w) ? v.x : 0.f;
-    d[1] = (j4 + 1 < w) ? v.y : 0.f;
-    d[2] = (j4 + 2 < w) ? v.z : 0.f;
-    d[3] = (j4 + 3 < w) ? v.w : 0.f;
-  }
-  __syncthreads();
-  const int ty = tid >> 3, tx = tid & 7;
-  const int i0 = 2 * ty;
-  for (int J = 3; J >= 0; --J) {
-    float acc[2][4];
+  if (has_next) {
+    const int64_t g0 = c0 - LDL_PB + 32 * (int64_t)blockIdx.x;
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[a][c] = T[(i0 + a) * LDL_LD + 32 * J + tx + 8 * c];
-    for (int K = J + 1; K < 4; ++K) {
-#pragma unroll 8
-      for (int t = 0; t < 32; ++t) {
-        const float h0 = T[i0 * LDL_LD + 32 * K + t], h1 = T[(i0 + 1) * LDL_LD + 32 * K + t];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const float rv = R[(32 * J + tx + 8 * c) * LDL_LD + 32 * K + t];
-          acc[0][c] = fmaf(-h0, rv, acc[0][c]);
-          acc[1][c] = fmaf(-h1, rv, acc[1][c]);
+    for (int e = tid; e < 32 * 32; e += LDL_FT) {
+      const int i = e >> 5, j4 = (e & 31) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j4 < w) {
+        v = *reinterpret_cast<const float4*>(H + (g0 + i) * n + c0 + j4);
+        if (Lin) {
+          const float4 l = *reinterpret_cast<const float4*>(Lin + (g0 + i) * LDL_PB + j4);
+          v.x -= l.x, v.y -= l.y, v.z -= l.z, v.w -= l.w;
         }
       }
+      *reinterpret_cast<float4*>(T + i * LDL_LDA + j4) = v;   // w % 4 == 0
     }
-    __syncthreads();
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) T[(i0 + a) * LDL_LD + 32 * J + tx + 8 * c] = acc[a][c];
-    __syncthreads();
-    const float* XJ = X + J * 32 * 33;
-    float out[2][4] = {};
-#pragma unroll 8
-    for (int t = 0; t < 32; ++t) {
-      const float h0 = T[i0 * LDL_LD + 32 * J + t], h1 = T[(i0 + 1) * LDL_LD + 32 * J + t];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float xv = XJ[(tx + 8 * c) * 33 + t];
-        out[0][c] = fmaf(h0, xv, out[0][c]);
-        out[1][c] = fmaf(h1, xv, out[1][c]);
+  }
+  __syncthreads();
+
+  auto all_sync = [] { __syncthreads(); };
+  for (int J = 3; J >= 0; --J) {
+    if (warp == 0) {
+      const bool ok = warp_chol_inv32(A + 32 * J * LDL_LDA + 32 * J, LDL_LDA, X + J * 32 * LDL_LDX,
+                                      LDL_LDX, scr);
+      if (!ok && (tid & 31) == 0) bad = 1;
+    } else if (J < 3 && (warp & 3)) {
+      // deferred work of block column JJ = J + 1, on the warps that do not
+      // share warp 0's scheduler (warp w runs on sub-partition w % 4)
+      const int JJ = J + 1, th = (warp - 1 - (warp >> 2)) * 32 + (tid & 31), nth = LDL_HT;
+      if (JJ >= 2) {
+        blk_trsm(A, X + JJ * 32 * LDL_LDX, JJ, 0, 32 * (JJ - 1), th, nth, helpers_sync);
+        blk_update(A, JJ, 0, 32 * (JJ - 1), 0, 32 * JJ, th, nth);
       }
+      if (has_next) blk_solve<32>(T, A, X + JJ * 32 * LDL_LDX, JJ, th, nth, helpers_sync);
     }
     __syncthreads();
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) T[(i0 + a) * LDL_LD + 32 * J + tx + 8 * c] = out[a][c];
+    if (J == 0) break;
+    blk_trsm(A, X + J * 32 * LDL_LDX, J, 32 * (J - 1), 32, tid, LDL_FT, all_sync);
+    blk_update(A, J, 32 * (J - 1), 32, 32 * (J - 1), 32, tid, LDL_FT);
     __syncthreads();
   }
-  const int64_t pstride = n * LDL_PB;
-  for (int e = tid; e < 64 * LDL_PB; e += 256) {
-    const int ii = e >> 7, k = e & 127;
-    const int64_t gi = r0 + ii;
-    if (gi >= c0) continue;
-    const float v = (k < w) ? T[ii * LDL_LD + k] : 0.f;
-    if (k < w) H[gi * n + c0 + k] = v;
-    __nv_bfloat16 p0, p1, p2;
-    split3(v, p0, p1, p2);
-    Rs[gi * LDL_PB + k] = p0;
-    Rs[pstride + gi * LDL_PB + k] = p1;
-    Rs[2 * pstride + gi * LDL_PB + k] = p2;
+  if (has_next) blk_solve<32>(T, A, X, 0, tid, LDL_FT, all_sync);
+
+  if (blockIdx.x == 0) {
+    if (tid == 0 && bad) record_status(QUIP_ERR_NOT_PD);
+#pragma unroll
+    for (int e = tid; e < LDL_PB * 32; e += LDL_FT) {
+      const int i = e >> 5, j4 = (e & 31) * 4;
+      const float4 v = *reinterpret_cast<const float4*>(A + i * LDL_LDA + j4);
+      *reinterpret_cast<float4*>(Rd + i * LDL_PB + j4) =
+          make_float4(j4 >= i ? v.x : 0.f, j4 + 1 >= i ? v.y : 0.f, j4 + 2 >= i ? v.z : 0.f,
+                      j4 + 3 >= i ? v.w : 0.f);
+    }
+    for (int e = tid; e < 4 * 32 * 32; e += LDL_FT)
+      Xw[e] = X[(e >> 10) * 32 * LDL_LDX + ((e >> 5) & 31) * LDL_LDX + (e & 31)];
+    for (int k = tid; k < w; k += LDL_FT) {
+      const float r = A[k * LDL_LDA + k];
+      Dv[c0 + k] = r * r;
+    }
+    if (!has_next) {
+      for (int e = tid; e < LDL_PB * LDL_PB; e += LDL_FT) {
+        const int i = e >> 7, j = e & 127;
+        if (i < j && j < w) H[(c0 + i) * n + c0 + j] = A[i * LDL_LDA + j] / A[j * LDL_LDA + j];
+      }
+    }
+  }
+  if (has_next) {
+    for (int e = tid; e < 32 * 32; e += LDL_FT) {
+      const int i = e >> 5, j4 = (e & 31) * 4;
+      *reinterpret_cast<float4*>(Nx + (32 * blockIdx.x + i) * LDL_PB + j4) =
+          *reinterpret_cast<const float4*>(T + i * LDL_LDA + j4);
+    }
   }
 }
 
-// Copy every panel's diagonal factor block from Rd[p] (128 x 128) into H's
-// upper triangle: block p covers rows / columns [128 p, 128 p + w).
-__global__ void k_ldl_scatter_diag(float* __restrict__ H, int64_t n, const float* __restrict__ Rd) {
-  const int64_t p = blockIdx.x;
-  const int64_t c0 = p * LDL_PB;
-  const int w = (int)((n - c0) < LDL_PB ? (n - c0) : LDL_PB);
-  const float* src = Rd + p * LDL_PB * LDL_PB;
-  for (int e = threadIdx.x; e < LDL_PB * LDL_PB; e += blockDim.x) {
-    const int i = e >> 7, j = e & 127;
-    if (i < w && j < w && j >= i) H[(c0 + i) * n + c0 + j] = src[e];
+// Rows [r0, r0 + LDL_RR) of R12(p) = (H - Lin)[:c0, panel p] R_pp^-T by block
+// back substitution with R_pp (Rd) and X_J (Xw), then
+//   Ů:   H[r, c0 + k] = R12[r][k] / R_kk          (k < w)
+//   Rs:  R12 as three bf16 pieces Rs[q][r][k]     (piece stride n * 128; zero for k >= w)
+//   Lout[r][j] = sum_k R12[r][k] Nx[j][k]         (panel p's update of panel p - 1)
+// CTA 0 also writes the Ů of the diagonal block.
+// Grid: ceil(c0 / LDL_RR) CTAs of 256 threads.
+// Dynamic smem: LDL_RR x LDL_LDA (T) + 128 x LDL_LDA (R_pp, later Nx) + 4 x 32 x LDL_LDX
+// + 128 floats.
+__global__ void __launch_bounds__(LDL_RT, 2)
+    k_ldl_rows(float* __restrict__ H, int64_t n, int64_t c0, int w, const float* __restrict__ Lin,
+               const float* __restrict__ Rd, const float* __restrict__ Xw,
+               const float* __restrict__ Nx, __nv_bfloat16* __restrict__ Rs,
+               float* __restrict__ Lout) {
+  extern __shared__ __align__(16) float sm[];
+  float* T = sm;                                     // LDL_RR x LDL_LDA
+  float* Rp = T + LDL_RR * LDL_LDA;                      // 128 x LDL_LDA: R_pp, then Nx
+  float* X = Rp + LDL_PB * LDL_LDA;                  // 4 x 32 x LDL_LDX
+  float* Rkk = X + 4 * 32 * LDL_LDX;                 // 128
+  const int tid = threadIdx.x;
+  const int64_t r0 = (int64_t)blockIdx.x * LDL_RR;
+  for (int e = tid; e < LDL_RR * 32; e += LDL_RT) {
+    const int i = e >> 5, j4 = (e & 31) * 4;
+    const int64_t g = r0 + i;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (g < c0 && j4 < w) {
+      v = *reinterpret_cast<const float4*>(H + g * n + c0 + j4);
+      if (Lin) {
+        const float4 l = *reinterpret_cast<const float4*>(Lin + g * LDL_PB + j4);
+        v.x -= l.x, v.y -= l.y, v.z -= l.z, v.w -= l.w;
+      }
+    }
+    *reinterpret_cast<float4*>(T + i * LDL_LDA + j4) = v;
+  }
+#pragma unroll 4
+  for (int e = tid; e < LDL_PB * 32; e += LDL_RT) {
+    const int i = e >> 5, j4 = (e & 31) * 4;
+    *reinterpret_cast<float4*>(Rp + i * LDL_LDA + j4) =
+        *reinterpret_cast<const float4*>(Rd + i * LDL_PB + j4);
+  }
+  for (int e = tid; e < 4 * 32 * 8; e += LDL_RT) {
+    const int jb = e >> 8, r = (e >> 3) & 31, c4 = (e & 7) * 4;
+    *reinterpret_cast<float4*>(X + jb * 32 * LDL_LDX + r * LDL_LDX + c4) =
+        *reinterpret_cast<const float4*>(Xw + jb * 1024 + r * 32 + c4);
+  }
+  __syncthreads();
+  if (tid < LDL_PB) Rkk[tid] = Rp[tid * LDL_LDA + tid];
+  auto all_sync = [] { __syncthreads(); };
+  for (int J = 3; J >= 0; --J) blk_solve<LDL_RR>(T, Rp, X + J * 32 * LDL_LDX, J, tid, LDL_RT, all_sync);
+
+  const int64_t pstride = n * LDL_PB;
+  for (int e = tid; e < LDL_RR * LDL_PB; e += LDL_RT) {
+    const int i = e >> 7, k = e & 127;
+    const int64_t g = r0 + i;
+    if (g >= c0) continue;
+    const float v = T[i * LDL_LDA + k];
+    if (k < w) H[g * n + c0 + k] = v / Rkk[k];
+    __nv_bfloat16 p0, p1, p2;
+    split3(v, p0, p1, p2);
+    Rs[g * LDL_PB + k] = p0;
+    Rs[pstride + g * LDL_PB + k] = p1;
+    Rs[2 * pstride + g * LDL_PB + k] = p2;
+  }
+  if (blockIdx.x == 0) {
+    for (int e = tid; e < LDL_PB * LDL_PB; e += LDL_RT) {
+      const int i = e >> 7, j = e & 127;
+      if (i < j && j < w) H[(c0 + i) * n + c0 + j] = Rp[i * LDL_LDA + j] / Rkk[j];
+    }
+  }
+  __syncthreads();
+#pragma unroll 4
+  for (int e = tid; e < LDL_PB * 32; e += LDL_RT) {
+    const int i = e >> 5, j4 = (e & 31) * 4;
+    *reinterpret_cast<float4*>(Rp + i * LDL_LDA + j4) =
+        *reinterpret_cast<const float4*>(Nx + i * LDL_PB + j4);
+  }
+  __syncthreads();
+  // warp w: columns [16 w, 16 w + 16); lane: rows rg + 8 a, columns 16 w + cg + 4 b
+  constexpr int RA = LDL_RR / 8;
+  const int warp = tid >> 5, lane = tid & 31, rg = lane & 7, cg = lane >> 3;
+  float acc[RA][4];
+#pragma unroll
+  for (int a = 0; a < RA; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+  dot_rows<RA, 4>(acc, T + rg * LDL_LDA, 8 * LDL_LDA, Rp + (16 * warp + cg) * LDL_LDA, 4 * LDL_LDA,
+                  LDL_PB);
+#pragma unroll
+  for (int a = 0; a < RA; ++a) {
+    const int64_t g = r0 + rg + 8 * a;
+    if (g < c0)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) Lout[g * LDL_PB + 16 * warp + cg + 4 * b] = acc[a][b];
   }
 }
 

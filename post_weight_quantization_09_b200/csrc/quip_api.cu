@@ -86,11 +86,13 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint6
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// A second stream and two events per device for the LDL look-ahead, created
-// on first use and kept for the life of the process.
+// A second stream per device for the LDL bulk updates, with a fork event and
+// a ring of join events, created on first use and kept for the process.
+constexpr int kJoinRing = 4;
 struct SideStream {
   cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t join[kJoinRing] = {};
 };
 cudaError_t side_stream(SideStream& out) {
   static std::mutex mu;
@@ -102,9 +104,12 @@ cudaError_t side_stream(SideStream& out) {
   std::lock_guard<std::mutex> lk(mu);
   SideStream& ss = per_dev[dev];
   if (!ss.s) {
-    if ((e = cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+    SideStream t;
+    if ((e = cudaStreamCreateWithFlags(&t.s, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&t.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+    for (int i = 0; i < kJoinRing; ++i)
+      if ((e = cudaEventCreateWithFlags(&t.join[i], cudaEventDisableTiming)) != cudaSuccess) return e;
+    ss = t;
   }
   out = ss;
   return cudaSuccess;
@@ -535,15 +540,13 @@ quip_status quip_hessian_finalize(float* H, int64_t n, int64_t N_total, float da
   return QUIP_OK;
 }
 
-// LDL workspace: the panels' diagonal factor blocks (P x 128 x 128 fp32), then
-// the current panel's three bf16 pieces (3 x n x 128).
 static int64_t ldl_panels(int64_t n) { return (n + LDL_PB - 1) / LDL_PB; }
-// LDL workspace: every panel's R_pp (128 x 128 fp32) and X_JJ blocks
-// (4 x 32 x 33 fp32), and two buffers of a panel's R12 as 3 bf16 pieces.
-constexpr size_t LDL_XW = 4 * 32 * 33;
+// LDL workspace: the current panel's R_pp (128 x 128 fp32), X_J blocks
+// (4 x 32 x 32 fp32) and next rows (128 x 128 fp32); two look-ahead buffers
+// (n x 128 fp32) and two panels' R12 as three bf16 pieces (3 x n x 128).
 static size_t ldl_ws_bytes(int64_t n) {
-  return round256((size_t)ldl_panels(n) * LDL_PB * LDL_PB * 4) +
-         round256((size_t)ldl_panels(n) * LDL_XW * 4) + round256((size_t)6 * n * LDL_PB * 2);
+  return 2 * round256((size_t)LDL_PB * LDL_PB * 4) + round256((size_t)4 * 32 * 32 * 4) +
+         round256((size_t)2 * n * LDL_PB * 4) + round256((size_t)6 * n * LDL_PB * 2);
 }
 // LDLQ workspace: accumulator A (m x n fp32), the error of every column as
 // three bf16 pieces (3 x m x n), the split transposed factor (3 x n x n bf16).
@@ -638,22 +641,6 @@ quip_status quip_incoherence_inverse(const quip_transform* tf, const float* W_ha
   return QUIP_OK;
 }
 
-namespace {
-__global__ void k_diag_to(const float* H, int64_t n, float* D) {
-  const int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (k < n) D[k] = H[k * n + k];
-}
-// Ů[j][k] = R[j][k] / R[k][k] for k > j (row j per CTA); D holds R_kk.
-__global__ void k_scale_upper(float* H, int64_t n, const float* D) {
-  const int64_t j = blockIdx.x;
-  for (int64_t k = j + 1 + threadIdx.x; k < n; k += blockDim.x) H[j * n + k] /= D[k];
-}
-__global__ void k_square(float* D, int64_t n) {
-  const int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (k < n) D[k] = D[k] * D[k];
-}
-}  // namespace
-
 quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes, void* stream) {
   if (!H_t || !D) return QUIP_ERR_ARG;
   if (n <= 0 || n > ((int64_t)1 << 16)) return QUIP_ERR_SHAPE;
@@ -662,56 +649,53 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
   if (s != QUIP_OK) return s;
   cudaStream_t st = S(stream);
   const int64_t P = ldl_panels(n);
-  float* Rd = static_cast<float*>(ws);
-  float* Xw = reinterpret_cast<float*>(static_cast<char*>(ws) +
-                                       round256((size_t)P * LDL_PB * LDL_PB * 4));
-  __nv_bfloat16* Rs = reinterpret_cast<__nv_bfloat16*>(
-      reinterpret_cast<char*>(Xw) + round256((size_t)P * LDL_XW * 4));
-  const size_t smem_diag = ((size_t)LDL_PB * LDL_LD + LDL_XW) * sizeof(float);
-  const size_t smem_rows = ((size_t)(LDL_RROWS + 64) * LDL_LD + LDL_XW) * sizeof(float);
+  char* w8 = static_cast<char*>(ws);
+  float* Rd = reinterpret_cast<float*>(w8);
+  w8 += round256((size_t)LDL_PB * LDL_PB * 4);
+  float* Nx = reinterpret_cast<float*>(w8);
+  w8 += round256((size_t)LDL_PB * LDL_PB * 4);
+  float* Xw = reinterpret_cast<float*>(w8);
+  w8 += round256((size_t)4 * 32 * 32 * 4);
+  float* Lb = reinterpret_cast<float*>(w8);
+  w8 += round256((size_t)2 * n * LDL_PB * 4);
+  __nv_bfloat16* Rs = reinterpret_cast<__nv_bfloat16*>(w8);
+  const size_t smem_f = ((size_t)(LDL_PB + 32) * LDL_LDA + 5 * 32 * LDL_LDX + 96) * sizeof(float);
+  const size_t smem_r =
+      ((size_t)(LDL_RR + LDL_PB) * LDL_LDA + 4 * 32 * LDL_LDX + LDL_PB) * sizeof(float);
   static bool attr = false;
   if (!attr) {
-    QCHECK(cudaFuncSetAttribute(k_ldl_diag, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem_diag));
-    QCHECK(cudaFuncSetAttribute(k_ldl_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem_rows));
+    QCHECK(cudaFuncSetAttribute(k_ldl_factor, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_f));
+    QCHECK(cudaFuncSetAttribute(k_ldl_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_r));
     attr = true;
   }
   // Rs holds two panels' R12 (buffer p & 1), pieces at rows (3 buf + q) n.
   CUtensorMap ta, tb;
-  if (n > LDL_PB) {
+  SideStream side;
+  if (P > 2) {
     if (!make_tmap_bf16_2d(&ta, Rs, LDL_PB, 6 * (uint64_t)n, LDL_PB * 2, 64, sgemm::BM) ||
         !make_tmap_bf16_2d(&tb, Rs, LDL_PB, 6 * (uint64_t)n, LDL_PB * 2, 64, sgemm::BN))
       return QUIP_ERR_CUDA;
+    QCHECK(side_stream(side));
   }
-  SideStream side;
-  if (P > 2) QCHECK(side_stream(side));
-  bool bulk_pending = false;
+  const float* Lin = nullptr;
   for (int64_t p = P - 1; p >= 0; --p) {
     const int64_t c0 = p * LDL_PB;
     const int w = (int)std::min<int64_t>(LDL_PB, n - c0);
     const int buf = (int)(p & 1);
-    float* Rdp = Rd + p * LDL_PB * LDL_PB;
-    float* Xwp = Xw + p * LDL_XW;
-    k_ldl_diag<<<1, 256, smem_diag, st>>>(H_t, n, c0, w, Rdp, Xwp);
+    // panel p has had every update except panel p + 1's once the bulk update
+    // of panel p + 2 is done (panel p + 1's arrives through Lin)
+    if (p + 2 <= P - 1) QCHECK(cudaStreamWaitEvent(st, side.join[(p + 2) % kJoinRing], 0));
+    k_ldl_factor<<<c0 > 0 ? LDL_FCTAS : 1, LDL_FT, smem_f, st>>>(H_t, n, c0, w, Lin, Rd, Xw, Nx, D);
     count_launch();
     if (c0 == 0) break;
-    k_ldl_rows<<<(unsigned)((c0 + 63) / 64), 256, smem_rows, st>>>(H_t, n, c0, w, Rdp, Xwp,
-                                                                   Rs + (size_t)buf * 3 * n * LDL_PB);
+    float* Lout = Lb + (size_t)buf * n * LDL_PB;
+    k_ldl_rows<<<(unsigned)((c0 + LDL_RR - 1) / LDL_RR), LDL_RT, smem_r, st>>>(
+        H_t, n, c0, w, Lin, Rd, Xw, Nx, Rs + (size_t)buf * 3 * n * LDL_PB, Lout);
     count_launch();
-    // Look-ahead: H[:c0, panel p - 1] -= R12 R12[panel p - 1]^T.  It adds into
-    // the region the previous bulk update also adds into, so it waits for
-    // that update (a fixed order of the two additions per element).
-    if (bulk_pending) QCHECK(cudaStreamWaitEvent(st, side.join, 0));
-    sgemm::Params la{};
-    la.C = H_t + (c0 - LDL_PB), la.ldc = n, la.M = (int)c0, la.N = LDL_PB, la.K = LDL_PB;
-    la.a_piece_rows = (int)n, la.b_piece_rows = (int)n;
-    la.a_row0 = 3 * (int)n * buf, la.b_row0 = 3 * (int)n * buf + (int)(c0 - LDL_PB);
-    la.alpha = -1.f, la.upper_only = 0;
-    QCHECK(split_gemm(ta, tb, la, st));
     if (c0 > LDL_PB) {
-      // The rest, H[:c0-128, :c0-128] -= R12 R12^T on the upper tiles, on the
-      // side stream; a few SMs stay free for the next diagonal factor.
+      // H[:c0-128, :c0-128] -= R12 R12^T on the upper tiles, on the side
+      // stream; the SMs that the next panel's factor and row kernels need
+      // stay free.
       QCHECK(cudaEventRecord(side.fork, st));
       QCHECK(cudaStreamWaitEvent(side.s, side.fork, 0));
       sgemm::Params gp{};
@@ -719,16 +703,13 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
       gp.a_piece_rows = (int)n, gp.b_piece_rows = (int)n;
       gp.a_row0 = gp.b_row0 = 3 * (int)n * buf;
       gp.alpha = -1.f, gp.upper_only = 1;
-      QCHECK(split_gemm(ta, tb, gp, side.s, num_sms() - 2));
-      QCHECK(cudaEventRecord(side.join, side.s));
-      bulk_pending = true;
+      const int next_rows_sms = (int)(((c0 - LDL_PB) / LDL_RR + 1) / 2);
+      const int cap = std::max(num_sms() / 2, num_sms() - LDL_FCTAS - next_rows_sms);
+      QCHECK(split_gemm(ta, tb, gp, side.s, cap));
+      QCHECK(cudaEventRecord(side.join[p % kJoinRing], side.s));
     }
+    Lin = Lout;
   }
-  if (bulk_pending) QCHECK(cudaStreamWaitEvent(st, side.join, 0));
-  k_ldl_scatter_diag<<<(unsigned)P, 256, 0, st>>>(H_t, n, Rd); count_launch();
-  k_diag_to<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(H_t, n, D); count_launch();
-  k_scale_upper<<<(unsigned)n, 256, 0, st>>>(H_t, n, D); count_launch();
-  k_square<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(D, n); count_launch();
   QCHECK(cudaGetLastError());
   return QUIP_OK;
 }
