@@ -68,6 +68,96 @@ def stage_work(cfg: LayerConfig):
     }
 
 
+def _ldlq_gemm_flops(m: int, n: int, b: int) -> float:
+    """Algorithmic flops of LDLQ's trailing GEMMs: the recursive split of the
+    columns into halves, 2 m (right width) (left width) per split."""
+    def rec(a, c):
+        nb = (c - a) // b
+        if nb <= 1:
+            return 0.0
+        mid = a + ((nb + 1) // 2) * b
+        return rec(a, mid) + 2.0 * m * (c - mid) * (mid - a) + rec(mid, c)
+    return rec(0, n)
+
+
+def kernel_work(cfg: LayerConfig):
+    """Algorithmic work per step of the library's kernels, by kernel name:
+    (kind, amount, bound).  Flops count multiply-adds as 2; bytes are the
+    minimum reads + writes of the kernel's operands.  The tensor-core split
+    GEMMs are counted at their fp32 algorithmic flops (2 M N K) although they
+    run six bf16 products per multiply-add (the three-piece split)."""
+    m, n, N, B = cfg.m, cfg.n, cfg.N, max(cfg.block, 64)
+    xb = 2 if cfg.dtype == "bf16" else 4
+    PB = 128
+    P = (n + PB - 1) // PB
+    fac = rows = bulk = 0.0
+    for p in range(P - 1, -1, -1):
+        c0 = p * PB
+        w = min(PB, n - c0)
+        fac += w ** 3 / 3.0 + (128.0 * w * w if c0 > 0 else 0.0)
+        if c0 > 0:
+            rows += c0 * (w * w + 2.0 * w * 128)
+        if c0 > PB:
+            M = c0 - PB
+            bulk += M * (M + 1) * PB            # upper triangle, 2 flops per multiply-add
+    kw = {
+        "k_syrk_tc": ("flops", float(N) * n * (n + 1), "tensor"),
+        "k_ldl_factor": ("flops", fac, "alu"),
+        "k_ldl_rows": ("flops", rows, "alu"),
+        "k_gemm_split_tc[ldl]": ("flops", bulk, "tensor"),
+        "k_gemm_split_tc[ldlq]": ("flops", _ldlq_gemm_flops(m, n, B), "tensor"),
+        "k_ldlq_chunk8": ("flops", float(m) * n * (B - 1), "alu"),
+        "k_row_grid": ("bytes", 4.0 * m * n + 8.0 * m, "hbm"),
+        "k_dequant": ("bytes", 5.0 * m * n + 8.0 * m, "hbm"),
+        "k_split_upper_transposed": ("bytes", 4.0 * n * n / 2 + 6.0 * n * n, "hbm"),
+        "k_mirror_scale": ("bytes", 8.0 * n * n, "hbm"),
+    }
+    # Hadamard passes: rows read their input (W once as bf16/f32, H and W^
+    # in fp32) and write fp32; column passes read and write fp32.
+    had = lambda s: s.kind == "hadamard"
+    fr = fc = 0.0
+    if had(cfg.n_side):
+        fr += (xb + 4.0) * m * n + 8.0 * n * n + 8.0 * m * n    # W, H (fwd), W^ (inv)
+        fc += 8.0 * n * n                                       # H columns (fwd)
+    if had(cfg.m_side):
+        fc += 2 * 8.0 * m * n                                   # W~ (fwd), W^ (inv)
+    if fr:
+        kw["k_fwht_rows"] = ("bytes", fr, "hbm")
+    if fc:
+        kw["k_fwht_cols"] = ("bytes", fc, "hbm")
+    return kw
+
+
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# one `ncu --set full` capture of each kernel on the attn7b workload (see
+# profiles/), with the first 12 hex digits of the SHA-1 of the source file
+# the kernel was built from: the figure is reported only while that file is
+# unchanged and only for the workload it was captured on.
+KERNEL_TRAFFIC = {
+    "k_syrk_tc": ("syrk_tc.cuh", "260ad4eebdfc", 71597824),
+    "k_ldl_factor": ("ldl.cuh", "fbc7579dcf4b", 335360),
+    "k_ldl_rows": ("ldl.cuh", "fbc7579dcf4b", 3834112),
+    "k_ldlq_chunk8": ("ldlq.cuh", "6bffcb01b1c3", 4312064),
+    "k_fwht_cols": ("fwht.cuh", "dbbc29ed00b7", 79775232),
+    "k_fwht_rows": ("fwht.cuh", "dbbc29ed00b7", 45301760),
+    "k_dequant": ("ldlq.cuh", "6bffcb01b1c3", 26946304),
+}
+TRAFFIC_WORKLOAD = "attn7b"
+
+
+def kernel_traffic(name: str, workload: str):
+    import hashlib
+    ent = KERNEL_TRAFFIC.get(name)
+    if ent is None or workload != TRAFFIC_WORKLOAD:
+        return None
+    src = os.path.join(ROOT, "post_weight_quantization_09_b200", "csrc", ent[0])
+    try:
+        h = hashlib.sha1(open(src, "rb").read()).hexdigest()[:12]
+    except OSError:
+        return None
+    return ent[2] if h == ent[1] else None
+
+
 def roofline_entry(kind, amount, bound, ms, pk):
     if kind == "bytes":
         achieved = amount / (ms * 1e-3) / 1e9
@@ -306,6 +396,16 @@ def run_ours(args, cfg: LayerConfig):
     if st != L.QUIP_OK:
         raise RuntimeError(f"device status after timing: {L.status_string(st)}")
 
+    # ---- per-kernel device time: the same steps again, each launch bracketed
+    # by CUDA events on its own stream (kept out of the timed region above)
+    Q.quip_timing_begin()
+    for _ in range(args.steps):
+        flush.zero_()
+        torch.cuda.synchronize()
+        step()
+    torch.cuda.synchronize()
+    per_kernel = Q.quip_timing_end()
+
     total_ms = float(sum(step_ms))
     if world > 1:
         t = torch.tensor([total_ms], device="cuda")
@@ -350,10 +450,23 @@ def run_ours(args, cfg: LayerConfig):
         ms = statistics.mean(stage_ms[i])
         kind, amount, bound = work[name]
         stages[name] = {"ms": round(ms, 4), **roofline_entry(kind, amount, bound, ms, pk)}
-    dominant = max(stages, key=lambda k: stages[k]["ms"])
-    roof = {k: v for k, v in stages[dominant].items() if k != "ms"}
-    roof["stage"] = dominant
-    roof["peak_source"] = pk["source"]
+    kwork = kernel_work(cfg)
+    kernels = {}
+    for name, (cnt, tot_ms) in per_kernel.items():
+        ent = {"launches_per_step": cnt / args.steps, "ms_per_step": round(tot_ms / args.steps, 4)}
+        if name in kwork:
+            kind, amount, bound = kwork[name]
+            ent.update(roofline_entry(kind, amount, bound, tot_ms / args.steps, pk))
+            ent["traffic"] = kernel_traffic(name, cfg.name)
+        kernels[name] = ent
+    ranked = sorted((k for k in kernels if "frac" in kernels[k]), key=lambda k: -kernels[k]["ms_per_step"])
+    dominant = ranked[0]
+    dk = kernels[dominant]
+    roof = {"bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"], "unit": dk["unit"],
+            "frac": dk["frac"], "traffic": kernel_traffic(dominant, cfg.name), "kernel": dominant,
+            "launches_per_step": dk["launches_per_step"],
+            "avg_launch_ms": round(dk["ms_per_step"] / max(dk["launches_per_step"], 1e-9), 5),
+            "peak_source": pk["source"]}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -363,6 +476,7 @@ def run_ours(args, cfg: LayerConfig):
         "config": config_desc(cfg, args),
         "roofline": roof,
         "stages": stages,
+        "kernels": kernels,
         "e2e": {"value": world * cfg.m * cfg.n / (e2e * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
         "gpu_launches": int(launches),
@@ -381,7 +495,7 @@ def run_ours(args, cfg: LayerConfig):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="attn7b", choices=sorted(CONFIGS))

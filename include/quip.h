@@ -264,6 +264,23 @@ quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int
                                  int64_t block, size_t* bytes);
 
 /*
+ * Per-kernel device timing, for measurement (the QuIP papers have no
+ * counterpart).  quip_timing_begin() discards earlier records and turns
+ * timing on: from then on every kernel the library launches, on any stream,
+ * is bracketed by two CUDA events recorded on its own stream and filed under
+ * the kernel's name.  quip_timing_end() turns timing off, waits for the
+ * recorded events, and writes up to max_entries aggregates, largest total
+ * first: names[i] (static string owned by the library), launches[i] and
+ * total_ms[i] (sum of the launches' event-measured durations).
+ * *n_entries receives the number of distinct kernels recorded.  The events
+ * add a few microseconds of host work per launch; time a run without them
+ * for throughput.  Not meant for concurrent use from several host threads.
+ */
+quip_status quip_timing_begin(void);
+quip_status quip_timing_end(const char** names, uint64_t* launches, double* total_ms,
+                            int max_entries, int* n_entries);
+
+/*
  * Synchronise `stream`, then return and clear the device status word
  * (QUIP_OK if no device-side error was recorded since the last call), or
  * QUIP_ERR_CUDA if a CUDA error is pending.  The status word is shared by all

@@ -21,7 +21,7 @@ from ._lib import QuipError, load, status_string  # noqa: F401
 __all__ = [
     "Transform", "quip_hessian_accumulate", "quip_hessian_finalize", "quip_incoherence_forward",
     "quip_incoherence_inverse", "quip_ldl", "quip_ldlq_quantize", "quip_dequantize",
-    "quip_workspace_size", "quip_sync_status", "LayerQuantizer", "quantize_layer", "QuipError",
+    "quip_workspace_size", "quip_sync_status", "quip_timing_begin", "quip_timing_end", "LayerQuantizer", "quantize_layer", "QuipError",
     "KIND",
 ]
 
@@ -196,6 +196,21 @@ def quip_dequantize(codes: torch.Tensor, lo: torch.Tensor, scale: torch.Tensor, 
 
 def quip_sync_status(stream=None) -> int:
     return load().quip_sync_status(_s(stream))
+
+
+def quip_timing_begin() -> None:
+    L.check(load().quip_timing_begin(), "quip_timing_begin")
+
+
+def quip_timing_end(max_entries: int = 64) -> dict:
+    """{kernel name: (launches, total ms)} of the launches since quip_timing_begin()."""
+    lib = load()
+    names = (ctypes.c_char_p * max_entries)()
+    counts = (ctypes.c_uint64 * max_entries)()
+    ms = (ctypes.c_double * max_entries)()
+    n = ctypes.c_int(0)
+    L.check(lib.quip_timing_end(names, counts, ms, max_entries, ctypes.byref(n)), "quip_timing_end")
+    return {names[i].decode(): (int(counts[i]), float(ms[i])) for i in range(min(n.value, max_entries))}
 
 
 @dataclass

@@ -41,6 +41,9 @@ SIGNATURES = {
     "quip_dequantize": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
     "quip_workspace_size": (c_int, [c_int, c_void_p, c_int64, c_int64, c_int64, POINTER(c_size_t)]),
     "quip_sync_status": (c_int, [c_void_p]),
+    "quip_timing_begin": (c_int, []),
+    "quip_timing_end": (c_int, [POINTER(c_char_p), POINTER(c_uint64), POINTER(ctypes.c_double), c_int,
+                                POINTER(c_int)]),
 }
 
 _lib = None

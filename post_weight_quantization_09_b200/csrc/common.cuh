@@ -9,6 +9,9 @@
 
 #include <atomic>
 #include <cstdint>
+#include <mutex>
+#include <utility>
+#include <vector>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -24,6 +27,47 @@ namespace quip {
 // Host-side count of kernels this library has enqueued since it was loaded.
 inline std::atomic<unsigned long long> g_launch_count{0};
 inline void count_launch() { g_launch_count.fetch_add(1, std::memory_order_relaxed); }
+
+// Optional per-kernel device timing (quip_timing_begin / quip_timing_end):
+// while it is on, every launch is bracketed by a pair of CUDA events
+// recorded on the launching stream, filed under the kernel's name.
+struct TimingRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+inline std::atomic<bool> g_timing_on{false};
+inline std::mutex g_timing_mu;
+inline std::vector<TimingRec> g_timing_recs;
+inline std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_timing_pool;
+
+// One kernel launch: construct right before the launch, on the same stream.
+struct LaunchScope {
+  cudaStream_t st;
+  cudaEvent_t b = nullptr;
+  LaunchScope(const char* name, cudaStream_t s) : st(s) {
+    if (!g_timing_on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    std::pair<cudaEvent_t, cudaEvent_t> ev{nullptr, nullptr};
+    if (!g_timing_pool.empty()) {
+      ev = g_timing_pool.back();
+      g_timing_pool.pop_back();
+    } else if (cudaEventCreate(&ev.first) != cudaSuccess || cudaEventCreate(&ev.second) != cudaSuccess) {
+      return;
+    }
+    if (cudaEventRecord(ev.first, st) != cudaSuccess) {
+      g_timing_pool.push_back(ev);
+      return;
+    }
+    g_timing_recs.push_back({name, ev.first, ev.second});
+    b = ev.second;
+  }
+  ~LaunchScope() {
+    count_launch();
+    if (b) cudaEventRecord(b, st);
+  }
+  LaunchScope(const LaunchScope&) = delete;
+  LaunchScope& operator=(const LaunchScope&) = delete;
+};
 
 // Library status word (one per device that loads the library).  Kernels
 // record the first error with atomicCAS; quip_sync_status() reads and clears.

@@ -104,7 +104,10 @@ inline cudaError_t gemm_simt(const GemmArgs& g, int64_t batch, cudaStream_t st) 
   if (g.M <= 0 || g.N <= 0 || batch <= 0) return cudaSuccess;
   dim3 grid((unsigned)((g.N + SG_BN - 1) / SG_BN), (unsigned)((g.M + SG_BM - 1) / SG_BM),
             (unsigned)batch);
-  k_gemm_simt<TA, TB, Acc><<<grid, 256, 0, st>>>(g); count_launch();
+  {
+    LaunchScope ls("k_gemm_simt", st);
+    k_gemm_simt<TA, TB, Acc><<<grid, 256, 0, st>>>(g);
+  }
   return cudaGetLastError();
 }
 

@@ -6,6 +6,7 @@
 
 #include <cmath>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -129,7 +130,7 @@ int num_sms() {
 // C (+)= alpha * (3-piece A) (3-piece B)^T on the tensor cores; see gemm_tc.cuh.
 // max_ctas > 0 caps the persistent grid (leaves SMs to a concurrent stream).
 cudaError_t split_gemm(const CUtensorMap& ta, const CUtensorMap& tb, sgemm::Params p,
-                       cudaStream_t st, int max_ctas = 0) {
+                       cudaStream_t st, const char* name, int max_ctas = 0) {
   if (p.M <= 0 || p.N <= 0) return cudaSuccess;
   static bool attr = false;
   if (!attr) {
@@ -147,7 +148,8 @@ cudaError_t split_gemm(const CUtensorMap& ta, const CUtensorMap& tb, sgemm::Para
       if (!(p.upper_only && ti * sgemm::BM > tj * sgemm::BN + sgemm::BN - 1)) ++valid;
   const int cap = max_ctas > 0 ? std::min(max_ctas, num_sms()) : num_sms();
   const int grid = std::max(1, std::min(valid, cap));
-  sgemm::k_gemm_split_tc<<<grid, 256, sgemm::SMEM_BYTES, st>>>(ta, tb, p, tm * tn); count_launch();
+  LaunchScope ls(name, st);
+  sgemm::k_gemm_split_tc<<<grid, 256, sgemm::SMEM_BYTES, st>>>(ta, tb, p, tm * tn);
   return cudaGetLastError();
 }
 
@@ -160,8 +162,9 @@ cudaError_t fwht_rows(const TIn* in, int64_t ldin, float* out, int64_t ldout, in
   if (rows <= 0) return cudaSuccess;
   const int L = ilog2(d);
   if (L < 4) {
+    LaunchScope ls("k_fwht_rows", st);
     k_fwht_rows_small<TIn><<<(unsigned)((rows + 127) / 128), 128, 0, st>>>(
-        in, ldin, out, ldout, rows, (int)d, pre, post, row_sign, scale); count_launch();
+        in, ldin, out, ldout, rows, (int)d, pre, post, row_sign, scale);
     return cudaGetLastError();
   }
   const int T = (int)(d / 16);
@@ -171,8 +174,11 @@ cudaError_t fwht_rows(const TIn* in, int64_t ldin, float* out, int64_t ldout, in
   const unsigned grid = (unsigned)((rows + RPC - 1) / RPC);
 #define QUIP_ROWS_CASE(LL)                                                                    \
   case LL:                                                                                    \
-    k_fwht_rows<LL, TIn><<<grid, NT, smem, st>>>(in, ldin, out, ldout, rows, pre, post,       \
-                                                 row_sign, scale); count_launch();                           \
+    {                                                                                         \
+      LaunchScope ls("k_fwht_rows", st);                                                      \
+      k_fwht_rows<LL, TIn><<<grid, NT, smem, st>>>(in, ldin, out, ldout, rows, pre, post,     \
+                                                   row_sign, scale);                          \
+    }                                                                                         \
     break;
   switch (L) {
     QUIP_ROWS_CASE(4)
@@ -198,7 +204,10 @@ cudaError_t fwht_cols_pass(float* A, int64_t ld, int64_t ncols, int64_t R, int L
   const int threads = 32 * ((1 << LG) / 16);
 #define QUIP_COLS_CASE(LL)                                                                 \
   case LL:                                                                                 \
-    k_fwht_cols<LL><<<grid, threads, 0, st>>>(A, ld, ncols, gs, pre, post, scale); count_launch();         \
+    {                                                                                      \
+      LaunchScope ls("k_fwht_cols", st);                                                   \
+      k_fwht_cols<LL><<<grid, threads, 0, st>>>(A, ld, ncols, gs, pre, post, scale);       \
+    }                                                                                      \
     break;
   switch (LG) {
     QUIP_COLS_CASE(4)
@@ -221,8 +230,9 @@ cudaError_t fwht_cols(float* A, int64_t ld, int64_t ncols, int64_t R, const floa
   const int L = ilog2(R);
   const float scale = (float)(1.0 / std::sqrt((double)R));
   if (L < 4) {
+    LaunchScope ls("k_fwht_cols", st);
     k_fwht_cols_small<<<(unsigned)((ncols + 127) / 128), 128, 0, st>>>(A, ld, ncols, (int)R,
-                                                                        pre, post, scale); count_launch();
+                                                                        pre, post, scale);
     return cudaGetLastError();
   }
   if (L <= 8) return fwht_cols_pass(A, ld, ncols, R, L, 1, pre, post, scale, st);
@@ -338,9 +348,11 @@ cudaError_t side_rows(const SideData& sd, bool inverse, const TIn* src, int64_t 
   const unsigned grid = (unsigned)std::min<int64_t>((rows * n + 255) / 256, 65535 * 8);
   if constexpr (std::is_same<TIn, float>::value) {
     if ((const void*)src == (const void*)dst && ldsrc == n) return cudaSuccess;
-    k_copy_rows_f32<<<grid, 256, 0, st>>>(src, ldsrc, dst, rows, n); count_launch();
+    LaunchScope ls("k_copy_rows", st);
+    k_copy_rows_f32<<<grid, 256, 0, st>>>(src, ldsrc, dst, rows, n);
   } else {
-    k_convert_rows_bf16<<<grid, 256, 0, st>>>(src, ldsrc, dst, rows, n); count_launch();
+    LaunchScope ls("k_copy_rows", st);
+    k_convert_rows_bf16<<<grid, 256, 0, st>>>(src, ldsrc, dst, rows, n);
   }
   return cudaGetLastError();
 }
@@ -413,18 +425,20 @@ static quip_status alloc_side(SideData& sd, int kind, int64_t dim, int64_t p, in
 // Draw one side's random data from `seed` into its existing buffers.
 static quip_status draw_side(const SideData& sd, uint64_t seed, int which, cudaStream_t st) {
   if (sd.kind == QUIP_T_HADAMARD) {
+    LaunchScope ls("k_random_signs", st);
     k_random_signs<<<(unsigned)((sd.dim + 255) / 256), 256, 0, st>>>(sd.signs, sd.dim, seed,
                                                                       which == 0 ? 0u : 1u);
-    count_launch();
   } else if (sd.kind == QUIP_T_KRONECKER) {
     const uint32_t sa = which == 0 ? 2u : 4u, sb = which == 0 ? 3u : 5u;
     for (int f = 0; f < 2; ++f) {
       const int64_t d = f == 0 ? sd.p : sd.q;
-      k_gaussian<<<(unsigned)((d * d + 255) / 256), 256, 0, st>>>(sd.G, d * d, seed, f == 0 ? sa : sb);
-      count_launch();
+      {
+        LaunchScope ls("k_gaussian", st);
+        k_gaussian<<<(unsigned)((d * d + 255) / 256), 256, 0, st>>>(sd.G, d * d, seed, f == 0 ? sa : sb);
+      }
+      LaunchScope ls("k_haar_cgs2", st);
       k_haar_cgs2<<<1, 256, 0, st>>>(sd.G, sd.Qc, f == 0 ? sd.A : sd.B, f == 0 ? sd.A64 : sd.B64,
                                        (int)d);
-      count_launch();
     }
   }
   QCHECK(cudaGetLastError());
@@ -513,8 +527,11 @@ quip_status quip_hessian_accumulate(const void* X, int dtype, int64_t N, int64_t
       attr = true;
     }
     const int T = (int)((n + syrk::BT - 1) / syrk::BT);
-    syrk::k_syrk_tc<<<T * (T + 1) / 2, 256, syrk::SMEM_BYTES, st>>>(map, H_acc, (int)n, (int)N,
-                                                                     accumulate ? 1 : 0); count_launch();
+    {
+      LaunchScope ls("k_syrk_tc", st);
+      syrk::k_syrk_tc<<<T * (T + 1) / 2, 256, syrk::SMEM_BYTES, st>>>(map, H_acc, (int)n, (int)N,
+                                                                       accumulate ? 1 : 0);
+    }
     QCHECK(cudaGetLastError());
     return QUIP_OK;
   }
@@ -533,9 +550,15 @@ quip_status quip_hessian_finalize(float* H, int64_t n, int64_t N_total, float da
   if (n <= 0 || N_total < 1) return QUIP_ERR_SHAPE;
   if (!(damp >= 0.f) || !std::isfinite(damp)) return QUIP_ERR_ARG;
   cudaStream_t st = S(stream);
-  k_finalize_diag<<<1, 1024, 0, st>>>(H, n, 1.0 / (double)N_total, (double)damp); count_launch();
+  {
+    LaunchScope ls("k_finalize_diag", st);
+    k_finalize_diag<<<1, 1024, 0, st>>>(H, n, 1.0 / (double)N_total, (double)damp);
+  }
   const unsigned T = (unsigned)((n + 31) / 32);
-  k_mirror_scale<<<dim3(T, T), 256, 0, st>>>(H, n, (float)(1.0 / (double)N_total)); count_launch();
+  {
+    LaunchScope ls("k_mirror_scale", st);
+    k_mirror_scale<<<dim3(T, T), 256, 0, st>>>(H, n, (float)(1.0 / (double)N_total));
+  }
   QCHECK(cudaGetLastError());
   return QUIP_OK;
 }
@@ -685,13 +708,17 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
     // panel p has had every update except panel p + 1's once the bulk update
     // of panel p + 2 is done (panel p + 1's arrives through Lin)
     if (p + 2 <= P - 1) QCHECK(cudaStreamWaitEvent(st, side.join[(p + 2) % kJoinRing], 0));
-    k_ldl_factor<<<c0 > 0 ? LDL_FCTAS : 1, LDL_FT, smem_f, st>>>(H_t, n, c0, w, Lin, Rd, Xw, Nx, D);
-    count_launch();
+    {
+      LaunchScope ls("k_ldl_factor", st);
+      k_ldl_factor<<<c0 > 0 ? LDL_FCTAS : 1, LDL_FT, smem_f, st>>>(H_t, n, c0, w, Lin, Rd, Xw, Nx, D);
+    }
     if (c0 == 0) break;
     float* Lout = Lb + (size_t)buf * n * LDL_PB;
-    k_ldl_rows<<<(unsigned)((c0 + LDL_RR - 1) / LDL_RR), LDL_RT, smem_r, st>>>(
-        H_t, n, c0, w, Lin, Rd, Xw, Nx, Rs + (size_t)buf * 3 * n * LDL_PB, Lout);
-    count_launch();
+    {
+      LaunchScope ls("k_ldl_rows", st);
+      k_ldl_rows<<<(unsigned)((c0 + LDL_RR - 1) / LDL_RR), LDL_RT, smem_r, st>>>(
+          H_t, n, c0, w, Lin, Rd, Xw, Nx, Rs + (size_t)buf * 3 * n * LDL_PB, Lout);
+    }
     if (c0 > LDL_PB) {
       // H[:c0-128, :c0-128] -= R12 R12^T on the upper tiles, on the side
       // stream; the SMs that the next panel's factor and row kernels need
@@ -705,7 +732,7 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
       gp.alpha = -1.f, gp.upper_only = 1;
       const int next_rows_sms = (int)(((c0 - LDL_PB) / LDL_RR + 1) / 2);
       const int cap = std::max(num_sms() / 2, num_sms() - LDL_FCTAS - next_rows_sms);
-      QCHECK(split_gemm(ta, tb, gp, side.s, cap));
+      QCHECK(split_gemm(ta, tb, gp, side.s, "k_gemm_split_tc[ldl]", cap));
       QCHECK(cudaEventRecord(side.join[p % kJoinRing], side.s));
     }
     Lin = Lout;
@@ -732,13 +759,13 @@ struct LdlqRun {
 
 cudaError_t ldlq_block(const LdlqRun& r, int64_t k0) {
   const unsigned grid = (unsigned)((r.m + 15) / 16);
+  LaunchScope ls("k_ldlq_chunk8", r.st);
   if (r.B == 64)
     k_ldlq_chunk8<64><<<grid, 128, r.smem, r.st>>>(r.Wt, r.A, r.m, r.n, k0, r.U, r.ldu, r.lo, r.sc,
                                                    r.qmax, r.codes, r.Es, r.n);
   else
     k_ldlq_chunk8<128><<<grid, 128, r.smem, r.st>>>(r.Wt, r.A, r.m, r.n, k0, r.U, r.ldu, r.lo, r.sc,
                                                     r.qmax, r.codes, r.Es, r.n);
-  count_launch();
   return cudaGetLastError();
 }
 
@@ -756,7 +783,7 @@ cudaError_t ldlq_range(const LdlqRun& r, int64_t a, int64_t b) {
   gp.a_piece_rows = (int)r.m, gp.a_k0 = (int)a;
   gp.b_piece_rows = (int)r.n, gp.b_row0 = (int)mid, gp.b_k0 = (int)a;
   gp.alpha = 1.f;
-  e = split_gemm(r.ta, r.tb, gp, r.st);
+  e = split_gemm(r.ta, r.tb, gp, r.st, "k_gemm_split_tc[ldlq]");
   if (e != cudaSuccess) return e;
   return ldlq_range(r, mid, b);
 }
@@ -787,12 +814,17 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
   __nv_bfloat16* UTs = reinterpret_cast<__nv_bfloat16*>(w8);
   r.Wt = W_t, r.U = Uring, r.ldu = ldu, r.m = m, r.n = n, r.B = B, r.lo = lo, r.sc = scale;
   r.qmax = (float)((1 << bits) - 1), r.codes = codes;
-  k_row_grid<<<(unsigned)((m + 7) / 8), 256, 0, r.st>>>(W_t, m, n, (1 << bits) - 1, lo, scale);
-  count_launch();
+  {
+    LaunchScope ls("k_row_grid", r.st);
+    k_row_grid<<<(unsigned)((m + 7) / 8), 256, 0, r.st>>>(W_t, m, n, (1 << bits) - 1, lo, scale);
+  }
   QCHECK(cudaMemcpyAsync(r.A, W_t, (size_t)m * n * sizeof(float), cudaMemcpyDeviceToDevice, r.st));
   if (n > B) {
     const unsigned T = (unsigned)((n + 31) / 32);
-    k_split_upper_transposed<<<dim3(T, T), 256, 0, r.st>>>(Uring, ldu, n, UTs); count_launch();
+    {
+      LaunchScope ls("k_split_upper_transposed", r.st);
+      k_split_upper_transposed<<<dim3(T, T), 256, 0, r.st>>>(Uring, ldu, n, UTs);
+    }
     if (!make_tmap_bf16_2d(&r.ta, r.Es, (uint64_t)n, 3 * (uint64_t)m, (uint64_t)n * 2, 64, sgemm::BM) ||
         !make_tmap_bf16_2d(&r.tb, UTs, (uint64_t)n, 3 * (uint64_t)n, (uint64_t)n * 2, 64, sgemm::BN))
       return QUIP_ERR_CUDA;
@@ -867,9 +899,55 @@ quip_status quip_dequantize(const uint8_t* codes, const float* lo, const float* 
   if (m <= 0 || n <= 0) return QUIP_ERR_SHAPE;
   const int64_t total = m * n;
   const unsigned grid = (unsigned)std::min<int64_t>((total / 4 + 255) / 256 + 1, 148 * 16);
-  k_dequant<<<grid, 256, 0, S(stream)>>>(codes, lo, scale, m, n, W_hat_t); count_launch();
+  {
+    LaunchScope ls("k_dequant", S(stream));
+    k_dequant<<<grid, 256, 0, S(stream)>>>(codes, lo, scale, m, n, W_hat_t);
+  }
   QCHECK(cudaGetLastError());
   return QUIP_OK;
+}
+
+quip_status quip_timing_begin(void) {
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  for (const TimingRec& r : g_timing_recs) g_timing_pool.push_back({r.a, r.b});
+  g_timing_recs.clear();
+  g_timing_on.store(true);
+  return QUIP_OK;
+}
+
+quip_status quip_timing_end(const char** names, uint64_t* launches, double* total_ms,
+                            int max_entries, int* n_entries) {
+  g_timing_on.store(false);
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  struct Agg {
+    const char* name;
+    uint64_t count;
+    double ms;
+  };
+  std::vector<Agg> agg;
+  quip_status st = QUIP_OK;
+  for (const TimingRec& r : g_timing_recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) {
+      st = QUIP_ERR_CUDA;
+      continue;
+    }
+    size_t i = 0;
+    while (i < agg.size() && std::strcmp(agg[i].name, r.name) != 0) ++i;
+    if (i == agg.size()) agg.push_back({r.name, 0, 0.0});
+    agg[i].count += 1;
+    agg[i].ms += ms;
+  }
+  for (const TimingRec& r : g_timing_recs) g_timing_pool.push_back({r.a, r.b});
+  g_timing_recs.clear();
+  std::sort(agg.begin(), agg.end(), [](const Agg& x, const Agg& y) { return x.ms > y.ms; });
+  if (n_entries) *n_entries = (int)agg.size();
+  for (int i = 0; i < max_entries && i < (int)agg.size(); ++i) {
+    if (names) names[i] = agg[i].name;
+    if (launches) launches[i] = agg[i].count;
+    if (total_ms) total_ms[i] = agg[i].ms;
+  }
+  return st;
 }
 
 quip_status quip_sync_status(void* stream) {
