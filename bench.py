@@ -80,13 +80,19 @@ def _ldlq_gemm_flops(m: int, n: int, b: int) -> float:
     return rec(0, n)
 
 
+def _ldlq_block_flops(m: int, n: int, b: int = 128) -> float:
+    """In-block feedback of LDLQ: each b-column block feeds every column's
+    error to the block's later columns, m w (w - 1) flops for a w-wide block."""
+    return float(sum(m * min(b, n - k0) * (min(b, n - k0) - 1) for k0 in range(0, n, b)))
+
+
 def kernel_work(cfg: LayerConfig):
     """Algorithmic work per step of the library's kernels, by kernel name:
     (kind, amount, bound).  Flops count multiply-adds as 2; bytes are the
     minimum reads + writes of the kernel's operands.  The tensor-core split
     GEMMs are counted at their fp32 algorithmic flops (2 M N K) although they
     run six bf16 products per multiply-add (the three-piece split)."""
-    m, n, N, B = cfg.m, cfg.n, cfg.N, max(cfg.block, 64)
+    m, n, N = cfg.m, cfg.n, cfg.N
     xb = 2 if cfg.dtype == "bf16" else 4
     PB = 128
     P = (n + PB - 1) // PB
@@ -105,8 +111,8 @@ def kernel_work(cfg: LayerConfig):
         "k_ldl_factor": ("flops", fac, "alu"),
         "k_ldl_rows": ("flops", rows, "alu"),
         "k_gemm_split_tc[ldl]": ("flops", bulk, "tensor"),
-        "k_gemm_split_tc[ldlq]": ("flops", _ldlq_gemm_flops(m, n, B), "tensor"),
-        "k_ldlq_chunk8": ("flops", float(m) * n * (B - 1), "alu"),
+        "k_gemm_split_tc[ldlq]": ("flops", _ldlq_gemm_flops(m, n, 128), "tensor"),
+        "k_ldlq_tc": ("flops", _ldlq_block_flops(m, n), "alu"),
         "k_row_grid": ("bytes", 4.0 * m * n + 8.0 * m, "hbm"),
         "k_dequant": ("bytes", 5.0 * m * n + 8.0 * m, "hbm"),
         "k_split_upper_transposed": ("bytes", 4.0 * n * n / 2 + 6.0 * n * n, "hbm"),
@@ -137,7 +143,6 @@ KERNEL_TRAFFIC = {
     "k_syrk_tc": ("syrk_tc.cuh", "260ad4eebdfc", 71597824),
     "k_ldl_factor": ("ldl.cuh", "fbc7579dcf4b", 335360),
     "k_ldl_rows": ("ldl.cuh", "fbc7579dcf4b", 3834112),
-    "k_ldlq_chunk8": ("ldlq.cuh", "6bffcb01b1c3", 4312064),
     "k_fwht_cols": ("fwht.cuh", "dbbc29ed00b7", 79775232),
     "k_fwht_rows": ("fwht.cuh", "dbbc29ed00b7", 45301760),
     "k_dequant": ("ldlq.cuh", "6bffcb01b1c3", 26946304),

@@ -208,9 +208,10 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
  *   Uring : device n x n fp32, row stride ldu >= n (ldu % 4 == 0); only the
  *           strict upper triangle is read (the H_t buffer quip_ldl returned).
  *           W_t and Uring 16-byte aligned.
- *   bits  : 1..8.  block: 32, 64 or 128, with n % block == 0; a performance
- *           parameter (the result does not depend on it): 32 is processed in
- *           64-column blocks and then also needs n % 64 == 0.
+ *   bits  : 1..8.  block: 32, 64 or 128, with n % block == 0 and n % 64 == 0;
+ *           a performance hint only (the result does not depend on it in
+ *           exact arithmetic): this build always processes 128-column
+ *           blocks (the last one 64 wide when n % 128 == 64).
  *   codes : device m x n uint8 (row stride n).  lo, scale: device m fp32.
  * ws: QUIP_OP_LDLQ.
  */

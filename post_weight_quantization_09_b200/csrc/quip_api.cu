@@ -746,26 +746,23 @@ struct LdlqRun {
   const float* Wt;
   float* A;
   const float* U;
-  int64_t ldu, m, n, B;
+  int64_t ldu, m, n;
   const float* lo;
   const float* sc;
   float qmax;
   uint8_t* codes;
   __nv_bfloat16* Es;
-  CUtensorMap ta, tb;
-  size_t smem;
+  CUtensorMap ta, tb, tu;
   cudaStream_t st;
 };
 
-cudaError_t ldlq_block(const LdlqRun& r, int64_t k0) {
-  const unsigned grid = (unsigned)((r.m + 15) / 16);
-  LaunchScope ls("k_ldlq_chunk8", r.st);
-  if (r.B == 64)
-    k_ldlq_chunk8<64><<<grid, 128, r.smem, r.st>>>(r.Wt, r.A, r.m, r.n, k0, r.U, r.ldu, r.lo, r.sc,
-                                                   r.qmax, r.codes, r.Es, r.n);
-  else
-    k_ldlq_chunk8<128><<<grid, 128, r.smem, r.st>>>(r.Wt, r.A, r.m, r.n, k0, r.U, r.ldu, r.lo, r.sc,
-                                                    r.qmax, r.codes, r.Es, r.n);
+constexpr int LDQ_BLK = 128;               // LDLQ block width (columns)
+
+cudaError_t ldlq_block(const LdlqRun& r, int64_t k0, int w) {
+  const unsigned grid = (unsigned)((r.m + 127) / 128);
+  LaunchScope ls("k_ldlq_tc", r.st);
+  k_ldlq_tc<<<grid, 256, LQT_SMEM, r.st>>>(r.tu, r.Wt, r.A, r.m, r.n, k0, w, r.U, r.ldu, r.lo, r.sc,
+                                          r.qmax, r.codes, r.Es, r.n);
   return cudaGetLastError();
 }
 
@@ -773,9 +770,9 @@ cudaError_t ldlq_block(const LdlqRun& r, int64_t k0) {
 // in one split GEMM, then the right half.  Every column's feedback is the
 // same sum as in the column-by-column definition, grouped differently.
 cudaError_t ldlq_range(const LdlqRun& r, int64_t a, int64_t b) {
-  const int64_t nb = (b - a) / r.B;
-  if (nb <= 1) return ldlq_block(r, a);
-  const int64_t mid = a + ((nb + 1) / 2) * r.B;
+  const int64_t nb = (b - a + LDQ_BLK - 1) / LDQ_BLK;
+  if (nb <= 1) return ldlq_block(r, a, (int)(b - a));
+  const int64_t mid = a + ((nb + 1) / 2) * LDQ_BLK;
   cudaError_t e = ldlq_range(r, a, mid);
   if (e != cudaSuccess) return e;
   sgemm::Params gp{};
@@ -796,9 +793,9 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
   if (bits < 1 || bits > 8) return QUIP_ERR_ARG;
   if (m <= 0 || n <= 0 || ldu < n) return QUIP_ERR_SHAPE;
   if (!(block == 32 || block == 64 || block == 128) || n % block) return QUIP_ERR_SHAPE;
-  // 32-column blocks are processed as 64-column blocks (same result)
-  const int64_t B = block < 64 ? 64 : block;
-  if (n % B) return QUIP_ERR_SHAPE;
+  // every block size is processed in 128-column blocks (the last one may be
+  // 64 wide; same result), so n must be a multiple of 64
+  if (n % 64) return QUIP_ERR_SHAPE;
   if (m > ((int64_t)1 << 20) || n > ((int64_t)1 << 16)) return QUIP_ERR_SHAPE;
   if ((ldu & 3) || (reinterpret_cast<uintptr_t>(Uring) & 15) || (reinterpret_cast<uintptr_t>(W_t) & 15))
     return QUIP_ERR_ARG;
@@ -812,33 +809,28 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
   r.Es = reinterpret_cast<__nv_bfloat16*>(w8);
   w8 += round256((size_t)3 * m * n * 2);
   __nv_bfloat16* UTs = reinterpret_cast<__nv_bfloat16*>(w8);
-  r.Wt = W_t, r.U = Uring, r.ldu = ldu, r.m = m, r.n = n, r.B = B, r.lo = lo, r.sc = scale;
+  r.Wt = W_t, r.U = Uring, r.ldu = ldu, r.m = m, r.n = n, r.lo = lo, r.sc = scale;
   r.qmax = (float)((1 << bits) - 1), r.codes = codes;
   {
     LaunchScope ls("k_row_grid", r.st);
     k_row_grid<<<(unsigned)((m + 7) / 8), 256, 0, r.st>>>(W_t, m, n, (1 << bits) - 1, lo, scale);
   }
   QCHECK(cudaMemcpyAsync(r.A, W_t, (size_t)m * n * sizeof(float), cudaMemcpyDeviceToDevice, r.st));
-  if (n > B) {
+  {
     const unsigned T = (unsigned)((n + 31) / 32);
-    {
-      LaunchScope ls("k_split_upper_transposed", r.st);
-      k_split_upper_transposed<<<dim3(T, T), 256, 0, r.st>>>(Uring, ldu, n, UTs);
-    }
+    LaunchScope ls("k_split_upper_transposed", r.st);
+    k_split_upper_transposed<<<dim3(T, T), 256, 0, r.st>>>(Uring, ldu, n, UTs);
+  }
+  if (!make_tmap_bf16_2d(&r.tu, UTs, (uint64_t)n, 3 * (uint64_t)n, (uint64_t)n * 2, 64, 128))
+    return QUIP_ERR_CUDA;
+  if (n > LDQ_BLK) {
     if (!make_tmap_bf16_2d(&r.ta, r.Es, (uint64_t)n, 3 * (uint64_t)m, (uint64_t)n * 2, 64, sgemm::BM) ||
         !make_tmap_bf16_2d(&r.tb, UTs, (uint64_t)n, 3 * (uint64_t)n, (uint64_t)n * 2, 64, sgemm::BN))
       return QUIP_ERR_CUDA;
   }
-  auto smem_for = [](int64_t b) {
-    return ((size_t)b * 8 * (b / 8 + 4) + 16 * (b + 4)) * 4 + 16 * b;
-  };
-  r.smem = smem_for(B);
   static bool attr = false;
   if (!attr) {
-    QCHECK(cudaFuncSetAttribute(k_ldlq_chunk8<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem_for(64)));
-    QCHECK(cudaFuncSetAttribute(k_ldlq_chunk8<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem_for(128)));
+    QCHECK(cudaFuncSetAttribute(k_ldlq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, LQT_SMEM));
     attr = true;
   }
   QCHECK(ldlq_range(r, 0, n));
