@@ -62,10 +62,10 @@ __global__ void __launch_bounds__(256) k_row_grid(const float* __restrict__ Wt, 
 //   3. forms, along the way, the group's feedback to the next group
 //      (`carry`, fp32) and hands the 16 errors and codes to its helper
 //      through shared memory.
-// The helper writes the codes and the errors' three bf16 pieces to global
-// memory and the pieces into a shared A operand (128-byte swizzled,
-// K-major); once all 128 rows are there, one helper issues the group's
-// feedback to every column from two groups on as six tcgen05.mma kind::f16
+// The helper writes the errors' three bf16 pieces into a shared A operand
+// (128-byte swizzled, K-major) and then the codes and pieces to global
+// memory; once all 128 rows are there, warp 8 issues the group's feedback
+// to every column from two groups on as six tcgen05.mma kind::f16
 // (M = 128, N = w - 16 (g + 2), K = 16; the three-piece product terms of
 // order <= 2, as in the split GEMM) accumulating in TMEM.  The B operand is
 // the block of the split transposed factor (Ů^T pieces), loaded once by TMA.
@@ -90,8 +90,24 @@ struct LqtShared {
 };
 
 // Named barriers (id 0 is __syncthreads): FULL + slot (rows -> helpers),
-// EMPTY + slot (helpers -> rows), HELP (the 128 helper threads).
-constexpr int LQT_FULL = 1, LQT_EMPTY = 3, LQT_HELP = 5;
+// EMPTY + slot (helpers -> rows), AREADY + slot (helpers -> MMA warp).
+constexpr int LQT_FULL = 1, LQT_EMPTY = 3, LQT_AREADY = 5;
+constexpr int LQT_THREADS = 288;                       // 4 row, 4 helper, 1 MMA warp
+
+// Three bf16 pieces of two values at once (the same pieces as split3 on each):
+// returns the packed bf16 pairs (low half = a) of piece 0, 1, 2.
+__device__ __forceinline__ void split3x2(float a, float b, uint32_t& q0, uint32_t& q1,
+                                         uint32_t& q2) {
+  const __nv_bfloat162 p0 = __floats2bfloat162_rn(a, b);
+  const float2 f0 = __bfloat1622float2(p0);
+  const float a1 = a - f0.x, b1 = b - f0.y;
+  const __nv_bfloat162 p1 = __floats2bfloat162_rn(a1, b1);
+  const float2 f1 = __bfloat1622float2(p1);
+  const __nv_bfloat162 p2 = __floats2bfloat162_rn(a1 - f1.x, b1 - f1.y);
+  q0 = *reinterpret_cast<const uint32_t*>(&p0);
+  q1 = *reinterpret_cast<const uint32_t*>(&p1);
+  q2 = *reinterpret_cast<const uint32_t*>(&p2);
+}
 __device__ __forceinline__ void nb_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
@@ -99,7 +115,7 @@ __device__ __forceinline__ void nb_arrive(int id, int count) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(LQT_THREADS, 1)
     k_ldlq_tc(const __grid_constant__ CUtensorMap tmU, const float* __restrict__ Wt,
               const float* __restrict__ A, int64_t m, int64_t n, int64_t k0, int w,
               const float* __restrict__ U, int64_t ldu, const float* __restrict__ lo,
@@ -111,7 +127,8 @@ __global__ void __launch_bounds__(256, 1)
   LqtShared* sh = reinterpret_cast<LqtShared*>(smem + LQT_BAR_OFF);
   float* band = reinterpret_cast<float*>(smem + LQT_BAND_OFF);
   const int tid = threadIdx.x, warp = tid >> 5;
-  const bool helper = warp >= 4;
+  const bool helper = warp >= 4 && warp < 8;
+  const bool mma_warp = warp == 8;
   const int r = tid & 127;                              // row within the CTA
   const int64_t row = (int64_t)blockIdx.x * 128 + r;
   const bool valid = row < m;
@@ -131,7 +148,7 @@ __global__ void __launch_bounds__(256, 1)
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
   const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
-  if (tid == 128) {
+  if (tid == 256) {
     // Ů^T pieces: map rows p n + j (j in [k0, k0 + 128)), columns k in [k0 + 64 h, + 64)
     tma_prefetch_desc(&tmU);
     mbar_arrive_expect_tx(&sh->tma_bar, (uint32_t)(3 * nh * LQT_TILE));
@@ -148,7 +165,7 @@ __global__ void __launch_bounds__(256, 1)
       const int k = e >> 5, jj = e & 31, j = 16 * (k >> 4) + jj;
       band[e] = (k < w && j < w && j > k) ? U[(k0 + k) * ldu + k0 + j] : 0.f;
     }
-  } else {
+  } else if (!mma_warp) {
     // the row's accumulated values into TMEM columns [0, w)
     for (int c64 = 0; c64 < w / 64; ++c64) {
       float v[2][32];
@@ -167,7 +184,7 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   tc_fence_after();
 
-  if (!helper) {
+  if (!helper && !mma_warp) {
     // ------------------------------------------------------------ row warps
     const float l = valid ? lo[row] : 0.f;
     const float s = valid ? sc[row] : 1.f;
@@ -243,10 +260,9 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
       for (int t = 0; t < 16; ++t) wv[t] = wn[t];
     }
-  } else {
+  } else if (helper) {
     // ------------------------------------------------------------ helper warps
     const int64_t pst = m * lde;
-    bool tma_done = false;
 #pragma unroll 1
     for (int g = 0; g < ngroups; ++g) {
       const int slot = g & 1;
@@ -262,14 +278,8 @@ __global__ void __launch_bounds__(256, 1)
       if (g + 2 < ngroups) nb_arrive(LQT_EMPTY + slot, 256);
       uint32_t pk[3][8];
 #pragma unroll
-      for (int t = 0; t < 16; t += 2) {
-        __nv_bfloat16 a0, a1, a2, b0, b1, b2;
-        split3(e[t], a0, a1, a2);
-        split3(e[t + 1], b0, b1, b2);
-        pk[0][t >> 1] = (uint32_t)__bfloat16_as_ushort(a0) | ((uint32_t)__bfloat16_as_ushort(b0) << 16);
-        pk[1][t >> 1] = (uint32_t)__bfloat16_as_ushort(a1) | ((uint32_t)__bfloat16_as_ushort(b1) << 16);
-        pk[2][t >> 1] = (uint32_t)__bfloat16_as_ushort(a2) | ((uint32_t)__bfloat16_as_ushort(b2) << 16);
-      }
+      for (int t = 0; t < 16; t += 2)
+        split3x2(e[t], e[t + 1], pk[0][t >> 1], pk[1][t >> 1], pk[2][t >> 1]);
       const int nN = w - 16 * (g + 2);
       if (nN > 0) {
         // K-slice sl = g % 4 of the A operand: 16-byte chunks 2 sl, 2 sl + 1
@@ -287,31 +297,7 @@ __global__ void __launch_bounds__(256, 1)
               make_uint4(pk[p][4], pk[p][5], pk[p][6], pk[p][7]);
         }
         fence_proxy_async_smem();
-        nb_sync(LQT_HELP, 128);
-        if (r == 0 && !sh->fail) {
-          if (!tma_done) {
-            if (!mbar_wait(&sh->tma_bar, 0)) sh->fail = 1;
-            tma_done = true;
-          }
-          if (!sh->fail) {
-            tc_fence_after();
-            const uint32_t idesc = make_idesc_bf16(128, nN, 0, 0);
-            const int h = g >> 2;
-            const uint32_t a_base = smem_u32(smem + LQT_A_OFF) + sl * 32;
-            const uint32_t b_base =
-                smem_u32(smem + LQT_B_OFF + h * 3 * LQT_TILE) + sl * 32 + 16 * (g + 2) * 128;
-#pragma unroll
-            for (int term = 0; term < sgemm::NTERMS; ++term) {
-              int pa, pb;
-              sgemm::term_pieces(term, pa, pb);
-              const uint64_t adesc = make_sw128_desc(a_base + pa * LQT_TILE, 16, 1024);
-              const uint64_t bdesc = make_sw128_desc(b_base + pb * LQT_TILE, 16, 1024);
-              tc_mma_f16(tmem + 16 * (g + 2), adesc, bdesc, idesc, 1u);
-            }
-          }
-          // always signal, so the row warps' bounded waits see the phase
-          tc_commit(&sh->mma_bar[slot]);
-        }
+        nb_arrive(LQT_AREADY + slot, 160);
       }
       if (valid) {
         *reinterpret_cast<uint4*>(codes + row * n + k0 + 16 * g) = cw;
@@ -323,9 +309,53 @@ __global__ void __launch_bounds__(256, 1)
         }
       }
     }
+  } else {
+    // ------------------------------------------------------------ MMA warp
+    bool tma_done = false;
+    // descriptor bases; a K-slice and a row offset add (bytes >> 4) to the
+    // start-address field (all shared addresses here are below 256 KB)
+    uint64_t adesc0[3], bdesc0[2][3];
+#pragma unroll
+    for (int p = 0; p < 3; ++p) {
+      adesc0[p] = make_sw128_desc(smem_u32(smem + LQT_A_OFF + p * LQT_TILE), 16, 1024);
+      bdesc0[0][p] = make_sw128_desc(smem_u32(smem + LQT_B_OFF + p * LQT_TILE), 16, 1024);
+      bdesc0[1][p] = make_sw128_desc(smem_u32(smem + LQT_B_OFF + (3 + p) * LQT_TILE), 16, 1024);
+    }
+#pragma unroll 1
+    for (int g = 0; g + 2 < ngroups; ++g) {
+      const int slot = g & 1, sl = g & 3, nN = w - 16 * (g + 2);
+      nb_sync(LQT_AREADY + slot, 160);
+      if ((tid & 31) == 0) {
+        if (!tma_done && !sh->fail) {
+          if (!mbar_wait(&sh->tma_bar, 0)) sh->fail = 1;
+          tma_done = true;
+        }
+        if (!sh->fail) {
+          tc_fence_after();
+          const uint32_t idesc = make_idesc_bf16(128, nN, 0, 0);
+          const int h = g >> 2;
+          const uint64_t aoff = (uint64_t)((sl * 32) >> 4);
+          const uint64_t boff = (uint64_t)((sl * 32 + 16 * (g + 2) * 128) >> 4);
+          const uint32_t dcol = tmem + 16 * (g + 2);
+          const uint64_t b0 = (h ? bdesc0[1][0] : bdesc0[0][0]) + boff;
+          const uint64_t b1 = (h ? bdesc0[1][1] : bdesc0[0][1]) + boff;
+          const uint64_t b2 = (h ? bdesc0[1][2] : bdesc0[0][2]) + boff;
+          // (2,0) (1,1) (0,2) (1,0) (0,1) (0,0): smallest terms first
+          tc_mma_f16(dcol, adesc0[2] + aoff, b0, idesc, 1u);
+          tc_mma_f16(dcol, adesc0[1] + aoff, b1, idesc, 1u);
+          tc_mma_f16(dcol, adesc0[0] + aoff, b2, idesc, 1u);
+          tc_mma_f16(dcol, adesc0[1] + aoff, b0, idesc, 1u);
+          tc_mma_f16(dcol, adesc0[0] + aoff, b1, idesc, 1u);
+          tc_mma_f16(dcol, adesc0[0] + aoff, b0, idesc, 1u);
+        }
+        // always signal, so the row warps' bounded waits see the phase
+        tc_commit(&sh->mma_bar[slot]);
+      }
+      __syncwarp();
+    }
     // every MMA done before TMEM is freed: the last group that issued any
     const int last = ngroups - 3;
-    if (r == 0 && last >= 0) {
+    if ((tid & 31) == 0 && last >= 0) {
       if (!mbar_wait(&sh->mma_bar[last & 1], (uint32_t)((last >> 1) & 1))) sh->fail = 1;
     }
   }

@@ -761,7 +761,7 @@ constexpr int LDQ_BLK = 128;               // LDLQ block width (columns)
 cudaError_t ldlq_block(const LdlqRun& r, int64_t k0, int w) {
   const unsigned grid = (unsigned)((r.m + 127) / 128);
   LaunchScope ls("k_ldlq_tc", r.st);
-  k_ldlq_tc<<<grid, 256, LQT_SMEM, r.st>>>(r.tu, r.Wt, r.A, r.m, r.n, k0, w, r.U, r.ldu, r.lo, r.sc,
+  k_ldlq_tc<<<grid, LQT_THREADS, LQT_SMEM, r.st>>>(r.tu, r.Wt, r.A, r.m, r.n, k0, w, r.U, r.ldu, r.lo, r.sc,
                                           r.qmax, r.codes, r.Es, r.n);
   return cudaGetLastError();
 }
