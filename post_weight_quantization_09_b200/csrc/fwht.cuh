@@ -12,6 +12,9 @@
 //  * k_fwht_cols: mixes groups of g = 2^G rows (16 <= g <= 256) at a row
 //    stride, 32 columns per CTA; H_R = H_a (x) H_b lets a column transform of
 //    length R = a*b run as two such passes (inner rows then strided rows).
+//  * d = 4096 (rows) and R = 4096 (columns) have dedicated one-pass kernels,
+//    k_fwht_row4096 and k_fwht_col4096 (radix 16 in registers, shared-memory
+//    transpositions in between).
 // Optional sign vectors: pre (applied to the input index), post (applied to
 // the output index), and a per-row sign for the orthogonal direction.
 #pragma once
@@ -220,6 +223,119 @@ __global__ void __launch_bounds__(32 * ((1 << LOGG) / 16))
     float x = v[r] * scale;
     if (post) x *= post[grow];
     if (cok) A[grow * ld + col] = x;
+  }
+}
+
+// ---------------------------------------------------------------- 4096-point transforms
+// Radix-16 in three register stages (index bits 0-3, 4-7, 8-11) with two
+// transpositions through shared memory between them; the shared index of
+// element k is k + k/16 (one pad word per 16), which makes every stage's
+// accesses conflict-free.
+
+__device__ __forceinline__ int pad16(int k) { return k + (k >> 4); }
+
+// One row of 4096 per CTA (256 threads).  Thread t: stage A on elements
+// 16 t + j (16-byte loads), stage B on 256 (t / 16) + 16 j + t % 16, stage C
+// on 256 j + t, stored straight from registers (coalesced across threads).
+template <typename TIn>
+__global__ void __launch_bounds__(256)
+    k_fwht_row4096(const TIn* __restrict__ in, int64_t ldin, float* out, int64_t ldout,
+                   const float* __restrict__ pre, const float* __restrict__ post,
+                   const float* __restrict__ row_sign, float scale) {
+  __shared__ float sr[4096 + 256];
+  const int t = threadIdx.x;
+  const int64_t row = blockIdx.x;
+  float v[16];
+  load16(in + row * ldin + 16 * t, v);
+  if (pre) {
+    const float4* pp = reinterpret_cast<const float4*>(pre + 16 * t);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 f = pp[q];
+      v[4 * q] *= f.x, v[4 * q + 1] *= f.y, v[4 * q + 2] *= f.z, v[4 * q + 3] *= f.w;
+    }
+  }
+  reg_fwht<4>(v);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) sr[pad16(16 * t + j)] = v[j];
+  __syncthreads();
+  const int hi = t >> 4, lo = t & 15;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] = sr[pad16(256 * hi + 16 * j + lo)];
+  reg_fwht<4>(v);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) sr[pad16(256 * hi + 16 * j + lo)] = v[j];
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] = sr[pad16(256 * j + t)];
+  reg_fwht<4>(v);
+  const float rs = row_sign ? row_sign[row] * scale : scale;
+  float* o = out + row * ldout;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int k = 256 * j + t;
+    o[k] = v[j] * rs * (post ? post[k] : 1.f);
+  }
+}
+
+// 4096-point column transform of 8 columns per CTA (1024 threads), in place.
+// Thread unit u (two per thread) handles column c = u % 8: stage A on rows
+// 16 o + j (o = u / 8; loaded straight from global memory), stage B on rows
+// 256 (u / 128) + 16 j + (u / 8) % 16, stage C on rows 256 j + u / 8 (stored
+// straight to global memory).  Shared index of (row k, column c):
+// pad16(k) 8 + c, conflict-free.  pre / post are indexed by the row; scale
+// multiplies the output.  Dynamic smem: (4096 + 256) x 8 floats.
+constexpr int FWHT_C4K_NC = 8, FWHT_C4K_THREADS = 1024;
+__global__ void __launch_bounds__(FWHT_C4K_THREADS, 1)
+    k_fwht_col4096(float* A, int64_t ld, int64_t ncols, const float* __restrict__ pre,
+                   const float* __restrict__ post, float scale) {
+  constexpr int NC = FWHT_C4K_NC, NTH = FWHT_C4K_THREADS;
+  extern __shared__ float sc[];
+  const int tid = threadIdx.x;
+  const int64_t c0 = (int64_t)blockIdx.x * NC;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int u = tid + NTH * h, c = u % NC, o = u / NC;
+    const bool cok = c0 + c < ncols;
+    float v[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int k = 16 * o + j;
+      float x = cok ? A[k * ld + c0 + c] : 0.f;
+      if (pre) x *= pre[k];
+      v[j] = x;
+    }
+    reg_fwht<4>(v);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) sc[pad16(16 * o + j) * NC + c] = v[j];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int u = tid + NTH * h, c = u % NC, lo = (u / NC) & 15, hi = u / (16 * NC);
+    float v[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = sc[pad16(256 * hi + 16 * j + lo) * NC + c];
+    reg_fwht<4>(v);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) sc[pad16(256 * hi + 16 * j + lo) * NC + c] = v[j];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int u = tid + NTH * h, c = u % NC, low = u / NC;
+    const bool cok = c0 + c < ncols;
+    float v[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = sc[pad16(256 * j + low) * NC + c];
+    reg_fwht<4>(v);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int k = 256 * j + low;
+      float x = v[j] * scale;
+      if (post) x *= post[k];
+      if (cok) A[k * ld + c0 + c] = x;
+    }
   }
 }
 

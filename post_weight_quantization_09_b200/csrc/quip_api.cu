@@ -167,6 +167,12 @@ cudaError_t fwht_rows(const TIn* in, int64_t ldin, float* out, int64_t ldout, in
         in, ldin, out, ldout, rows, (int)d, pre, post, row_sign, scale);
     return cudaGetLastError();
   }
+  if (L == 12) {
+    LaunchScope ls("k_fwht_rows", st);
+    k_fwht_row4096<TIn><<<(unsigned)rows, 256, 0, st>>>(in, ldin, out, ldout, pre, post, row_sign,
+                                                         scale);
+    return cudaGetLastError();
+  }
   const int T = (int)(d / 16);
   const int NT = T > 256 ? T : 256;
   const int RPC = NT / T;
@@ -236,6 +242,20 @@ cudaError_t fwht_cols(float* A, int64_t ld, int64_t ncols, int64_t R, const floa
     return cudaGetLastError();
   }
   if (L <= 8) return fwht_cols_pass(A, ld, ncols, R, L, 1, pre, post, scale, st);
+  if (L == 12) {
+    constexpr int kSmem = (4096 + 256) * FWHT_C4K_NC * (int)sizeof(float);
+    static bool attr = false;
+    if (!attr) {
+      cudaError_t e = cudaFuncSetAttribute(k_fwht_col4096, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    const int64_t ntiles = (ncols + FWHT_C4K_NC - 1) / FWHT_C4K_NC;
+    LaunchScope ls("k_fwht_cols", st);
+    k_fwht_col4096<<<(unsigned)ntiles, FWHT_C4K_THREADS, kSmem, st>>>(A, ld, ncols,
+                                                                                       pre, post, scale);
+    return cudaGetLastError();
+  }
   const int Li = (L + 1) / 2, Lo = L - Li;
   cudaError_t e = fwht_cols_pass(A, ld, ncols, R, Li, 1, pre, nullptr, 1.0f, st);
   if (e != cudaSuccess) return e;
