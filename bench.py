@@ -288,6 +288,28 @@ def dist_setup():
     return world, rank, local
 
 
+def rank_config(cfg: LayerConfig, rank: int) -> LayerConfig:
+    """Each rank quantises its own layer of the same shape (seed + rank)."""
+    return LayerConfig(**{**cfg.__dict__, "seed": cfg.seed + rank})
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Largest value of x over the ranks (the job's step time); no-op at N = 1."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(cfg: LayerConfig, world: int, ms_per_step: float) -> float:
+    """Whole-job quantized weights per second: every rank's layer over the
+    slowest rank's step time (weak scaling)."""
+    return world * cfg.m * cfg.n / (ms_per_step * 1e-3)
+
+
 def run_reference(args, cfg: LayerConfig):
     world, rank, _ = dist_setup()
     if rank != 0:
@@ -339,7 +361,7 @@ def run_ours(args, cfg: LayerConfig):
     import post_weight_quantization_09_b200 as Q
     from post_weight_quantization_09_b200 import _lib as L
     lib = Q.load()
-    rcfg = LayerConfig(**{**cfg.__dict__, "seed": cfg.seed + rank})
+    rcfg = rank_config(cfg, rank)
     d = make_layer(rcfg)
     as_t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 \
         else torch.from_numpy(a)
@@ -411,13 +433,9 @@ def run_ours(args, cfg: LayerConfig):
     torch.cuda.synchronize()
     per_kernel = Q.quip_timing_end()
 
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(sum(step_ms)), world, "cuda")
     ms_per_step = total_ms / args.steps
-    value = world * cfg.m * cfg.n / (ms_per_step * 1e-3)
+    value = job_throughput(cfg, world, ms_per_step)
 
     # ---- end to end through the public API: pinned host inputs in, codes + grid out
     codes_h = torch.empty(cfg.m, cfg.n, dtype=torch.uint8).pin_memory()
@@ -434,11 +452,7 @@ def run_ours(args, cfg: LayerConfig):
         torch.cuda.synchronize()
         if i > 0:                      # the first one is a warm-up
             e2e_ms.append(e0.elapsed_time(e1))
-    e2e = statistics.mean(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e = float(t.item())
+    e2e = max_over_ranks(statistics.mean(e2e_ms), world, "cuda")
     h2d = W_h.numel() * W_h.element_size() + X_h.numel() * X_h.element_size()
     d2h = codes_h.numel() + 4 * (lo_h.numel() + sc_h.numel())
 
@@ -482,7 +496,7 @@ def run_ours(args, cfg: LayerConfig):
         "roofline": roof,
         "stages": stages,
         "kernels": kernels,
-        "e2e": {"value": world * cfg.m * cfg.n / (e2e * 1e-3), "unit": UNIT,
+        "e2e": {"value": job_throughput(cfg, world, e2e), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
