@@ -87,6 +87,7 @@ __global__ void __launch_bounds__(256, 1)
     k_gemm_split_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     Params p, int ntiles) {
   extern __shared__ uint8_t smem_raw[];
+  pdl_wait_then_release();
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Shared* sh = reinterpret_cast<Shared*>(smem + STAGES * STAGE_BYTES);

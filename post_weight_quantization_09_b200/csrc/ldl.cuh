@@ -303,6 +303,7 @@ __global__ void __launch_bounds__(LDL_FT, 1)
                  float* __restrict__ Rd, float* __restrict__ Xw, float* __restrict__ Nx,
                  float* __restrict__ Dv) {
   extern __shared__ __align__(16) float sm[];
+  pdl_wait_then_release();
   float* A = sm;                                     // 128 x LDL_LDA
   float* T = A + LDL_PB * LDL_LDA;                   // 32 x LDL_LDA (next rows)
   float* X = T + 32 * LDL_LDA;                       // 4 x 32 x LDL_LDX
@@ -420,6 +421,7 @@ __global__ void __launch_bounds__(LDL_RT, 2)
                const float* __restrict__ Nx, __nv_bfloat16* __restrict__ Rs,
                float* __restrict__ Lout) {
   extern __shared__ __align__(16) float sm[];
+  pdl_wait_then_release();
   float* T = sm;                                     // LDL_RR x LDL_LDA
   float* Rp = T + LDL_RR * LDL_LDA;                      // 128 x LDL_LDA: R_pp, then Nx
   float* X = Rp + LDL_PB * LDL_LDA;                  // 4 x 32 x LDL_LDX

@@ -122,6 +122,7 @@ __global__ void __launch_bounds__(LQT_THREADS, 1)
               const float* __restrict__ sc, float qmax, uint8_t* __restrict__ codes,
               __nv_bfloat16* __restrict__ Es, int64_t lde) {
   extern __shared__ uint8_t smem_raw[];
+  pdl_wait_then_release();
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   LqtShared* sh = reinterpret_cast<LqtShared*>(smem + LQT_BAR_OFF);

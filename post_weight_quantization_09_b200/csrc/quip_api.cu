@@ -116,6 +116,25 @@ cudaError_t side_stream(SideStream& out) {
   return cudaSuccess;
 }
 
+// Launch with programmatic stream serialization (the kernel starts with
+// pdl_wait_then_release, so it may be scheduled while its predecessor on
+// the stream finishes).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 int num_sms() {
   static int sms = 0;
   if (!sms) {
@@ -149,8 +168,8 @@ cudaError_t split_gemm(const CUtensorMap& ta, const CUtensorMap& tb, sgemm::Para
   const int cap = max_ctas > 0 ? std::min(max_ctas, num_sms()) : num_sms();
   const int grid = std::max(1, std::min(valid, cap));
   LaunchScope ls(name, st);
-  sgemm::k_gemm_split_tc<<<grid, 256, sgemm::SMEM_BYTES, st>>>(ta, tb, p, tm * tn);
-  return cudaGetLastError();
+  return launch_pdl(sgemm::k_gemm_split_tc, dim3(grid), dim3(256), sgemm::SMEM_BYTES, st, ta, tb, p,
+                    tm * tn);
 }
 
 // ---------------------------------------------------------------- Hadamard plans
@@ -730,14 +749,16 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
     if (p + 2 <= P - 1) QCHECK(cudaStreamWaitEvent(st, side.join[(p + 2) % kJoinRing], 0));
     {
       LaunchScope ls("k_ldl_factor", st);
-      k_ldl_factor<<<c0 > 0 ? LDL_FCTAS : 1, LDL_FT, smem_f, st>>>(H_t, n, c0, w, Lin, Rd, Xw, Nx, D);
+      QCHECK(launch_pdl(k_ldl_factor, dim3(c0 > 0 ? LDL_FCTAS : 1), dim3(LDL_FT), smem_f, st, H_t, n,
+                        c0, w, Lin, Rd, Xw, Nx, D));
     }
     if (c0 == 0) break;
     float* Lout = Lb + (size_t)buf * n * LDL_PB;
     {
       LaunchScope ls("k_ldl_rows", st);
-      k_ldl_rows<<<(unsigned)((c0 + LDL_RR - 1) / LDL_RR), LDL_RT, smem_r, st>>>(
-          H_t, n, c0, w, Lin, Rd, Xw, Nx, Rs + (size_t)buf * 3 * n * LDL_PB, Lout);
+      QCHECK(launch_pdl(k_ldl_rows, dim3((unsigned)((c0 + LDL_RR - 1) / LDL_RR)), dim3(LDL_RT),
+                        smem_r, st, H_t, n, c0, w, Lin, (const float*)Rd, (const float*)Xw,
+                        (const float*)Nx, Rs + (size_t)buf * 3 * n * LDL_PB, Lout));
     }
     if (c0 > LDL_PB) {
       // H[:c0-128, :c0-128] -= R12 R12^T on the upper tiles, on the side
@@ -781,9 +802,9 @@ constexpr int LDQ_BLK = 128;               // LDLQ block width (columns)
 cudaError_t ldlq_block(const LdlqRun& r, int64_t k0, int w) {
   const unsigned grid = (unsigned)((r.m + 127) / 128);
   LaunchScope ls("k_ldlq_tc", r.st);
-  k_ldlq_tc<<<grid, LQT_THREADS, LQT_SMEM, r.st>>>(r.tu, r.Wt, r.A, r.m, r.n, k0, w, r.U, r.ldu, r.lo, r.sc,
-                                          r.qmax, r.codes, r.Es, r.n);
-  return cudaGetLastError();
+  return launch_pdl(k_ldlq_tc, dim3(grid), dim3(LQT_THREADS), (size_t)LQT_SMEM, r.st, r.tu, r.Wt,
+                    (const float*)r.A, r.m, r.n, k0, w, r.U, r.ldu, r.lo, r.sc, r.qmax, r.codes, r.Es,
+                    r.n);
 }
 
 // Columns [a, b): left half, then A[:, mid:b] += Err[:, a:mid] Ů[a:mid, mid:b]
