@@ -12,13 +12,14 @@
 //
 // Both operands K-major (row-major [rows][K] bf16, piece p at row offset
 // p * piece_rows), loaded by TMA as 64-wide K boxes with the 128-byte swizzle.
-// Tile 128 x 256, one M=128 N=256 K=16 tcgen05.mma per 16 k; 4-stage smem
-// ring (48 KB per stage).  The tensor core's fp32 accumulation drops low bits
-// (about one ulp of the running sum per MMA), so K is cut into chunks of
-// KCP = 512 per piece: each chunk (all six terms) accumulates into a fresh
-// TMEM buffer (columns [0, 256)), and the epilogue folds it into an fp32
-// running sum kept in a second TMEM buffer (columns [256, 512)) with
-// round-to-nearest adds; the tile's sum is added to C once, at its last chunk.
+// Tile 128 x TN (TN = 256, or 64 for narrow outputs), one M=128 N=TN K=16
+// tcgen05.mma per 16 k; 4-stage smem ring (16 KB + TN x 128 B per stage).
+// The tensor core's fp32 accumulation drops low bits (about one ulp of the
+// running sum per MMA), so K is cut into chunks of KCP = 512 per piece: each
+// chunk (all six terms) accumulates into a fresh TMEM buffer (columns
+// [0, TN)), and the epilogue folds it into an fp32 running sum kept in a
+// second TMEM buffer (columns [TN, 2 TN)) with round-to-nearest adds; the
+// tile's sum is added to C once, at its last chunk.
 // Bounded mbarrier waits as in the SYRK.
 #pragma once
 
@@ -27,12 +28,13 @@
 namespace quip {
 namespace sgemm {
 
+// Tile N width BN: 256, or 64 for narrow outputs (more tiles, more CTAs).
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;              // 16 KB
-constexpr int B_BYTES = BN * BK * 2;              // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 48 KB
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
-constexpr uint32_t IDESC = make_idesc_bf16(BM, BN, 0, 0);
+template <int TN> __host__ __device__ constexpr int b_bytes() { return TN * BK * 2; }
+template <int TN> __host__ __device__ constexpr int stage_bytes() { return A_BYTES + b_bytes<TN>(); }
+template <int TN> __host__ __device__ constexpr int smem_bytes() { return STAGES * stage_bytes<TN>() + 1024 + 256; }
+constexpr int SMEM_BYTES = smem_bytes<BN>();
 constexpr int NTERMS = 6;
 
 struct Params {
@@ -66,11 +68,12 @@ __device__ __forceinline__ void term_pieces(int t, int& pa, int& pb) {
 }
 
 // Tile t of the grid (row-major over tiles_m x tiles_n); false if skipped.
+template <int TN>
 __device__ __forceinline__ bool tile_coords(const Params& p, int t, int& i0, int& j0) {
   const int ti = t / p.tiles_n, tj = t % p.tiles_n;
   i0 = ti * BM;
-  j0 = tj * BN;
-  return !(p.upper_only && i0 > j0 + BN - 1);
+  j0 = tj * TN;
+  return !(p.upper_only && i0 > j0 + TN - 1);
 }
 
 // K-step `st` of a chunk covering piece columns [kc0, kc0 + kcl): term and offset.
@@ -82,10 +85,14 @@ __device__ __forceinline__ void chunk_step(int st, int kcl, int& term, int& kk) 
 
 // Persistent: CTA b handles tiles b, b + gridDim.x, ...  Warp 0 lane 0: TMA
 // producer; warp 1 lane 0: MMA issuer; warps 4..7: epilogue (warp w reads
-// TMEM lanes 32 (w - 4)..; one output row per thread, 256 columns).
+// TMEM lanes 32 (w - 4)..; one output row per thread, TN columns).
+template <int TN>
 __global__ void __launch_bounds__(256, 1)
     k_gemm_split_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     Params p, int ntiles) {
+  constexpr int STAGE_BYTES = stage_bytes<TN>();
+  constexpr uint32_t IDESC = make_idesc_bf16(BM, TN, 0, 0);
+  constexpr uint32_t TCOLS = 2 * TN;               // chunk buffer + running sum
   extern __shared__ uint8_t smem_raw[];
   pdl_wait_then_release();
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -104,7 +111,7 @@ __global__ void __launch_bounds__(256, 1)
     sh->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(&sh->tmem_base, 512);
+  if (warp == 0) tmem_alloc(&sh->tmem_base, TCOLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -116,7 +123,7 @@ __global__ void __launch_bounds__(256, 1)
     int it = 0;                                     // global K-step counter (stage ring)
     for (int t = blockIdx.x; t < ntiles && !sh->abort; t += gridDim.x) {
       int i0, j0;
-      if (!tile_coords(p, t, i0, j0)) continue;
+      if (!tile_coords<TN>(p, t, i0, j0)) continue;
       for (int c = 0; c < nchunk && !sh->abort; ++c) {
         const int kc0 = c * KCP, kcl = min(KCP, p.K - kc0);
         const int steps = NTERMS * (kcl / BK);
@@ -141,7 +148,7 @@ __global__ void __launch_bounds__(256, 1)
     int it = 0, gc = 0;                             // gc: global chunk counter
     for (int t = blockIdx.x; t < ntiles && !sh->abort; t += gridDim.x) {
       int i0, j0;
-      if (!tile_coords(p, t, i0, j0)) continue;
+      if (!tile_coords<TN>(p, t, i0, j0)) continue;
       for (int c = 0; c < nchunk && !sh->abort; ++c, ++gc) {
         if (!mbar_wait(&sh->tempty, (uint32_t)((gc & 1) ^ 1))) {   // chunk buffer free
           sh->abort = 1;
@@ -177,7 +184,7 @@ __global__ void __launch_bounds__(256, 1)
     bool stop = false;
     for (int t = blockIdx.x; t < ntiles && !stop; t += gridDim.x) {
       int i0, j0;
-      if (!tile_coords(p, t, i0, j0)) continue;
+      if (!tile_coords<TN>(p, t, i0, j0)) continue;
       const int row = i0 + quarter * 32 + lane;
       const bool rok = row < p.M;
       float* crow = p.C + (int64_t)(rok ? row : 0) * p.ldc;
@@ -193,17 +200,17 @@ __global__ void __launch_bounds__(256, 1)
         tc_fence_after();
         const bool first = c == 0, last = c == nchunk - 1;
 #pragma unroll 1
-        for (int c8 = 0; c8 < 8; ++c8) {
+        for (int c8 = 0; c8 < TN / 32; ++c8) {
           float v[32];
           tmem_ld32(tmem + lanes + c8 * 32, v);
           if (!first) {
             float su[32];
-            tmem_ld32(tmem + lanes + 256 + c8 * 32, su);
+            tmem_ld32(tmem + lanes + TN + c8 * 32, su);
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] += su[e];
           }
           if (!last) {
-            tmem_st32(tmem + lanes + 256 + c8 * 32, v);
+            tmem_st32(tmem + lanes + TN + c8 * 32, v);
           } else {
             // C += alpha * sum through fire-and-forget vector reductions in L2
             const int jc = j0 + c8 * 32;
@@ -233,7 +240,7 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, TCOLS);
   }
 }
 

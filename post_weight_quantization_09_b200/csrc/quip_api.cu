@@ -148,28 +148,40 @@ int num_sms() {
 
 // C (+)= alpha * (3-piece A) (3-piece B)^T on the tensor cores; see gemm_tc.cuh.
 // max_ctas > 0 caps the persistent grid (leaves SMs to a concurrent stream).
-cudaError_t split_gemm(const CUtensorMap& ta, const CUtensorMap& tb, sgemm::Params p,
-                       cudaStream_t st, const char* name, int max_ctas = 0) {
-  if (p.M <= 0 || p.N <= 0) return cudaSuccess;
+// tb64, when given, is B's map with 64-row boxes: outputs too narrow to fill
+// the GPU with 256-wide tiles then use 64-wide ones.
+template <int TN>
+cudaError_t split_gemm_tn(const CUtensorMap& ta, const CUtensorMap& tb, sgemm::Params p,
+                          cudaStream_t st, const char* name, int max_ctas) {
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(sgemm::k_gemm_split_tc,
+    cudaError_t e = cudaFuncSetAttribute(sgemm::k_gemm_split_tc<TN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         sgemm::SMEM_BYTES);
+                                         sgemm::smem_bytes<TN>());
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  const int tm = (p.M + sgemm::BM - 1) / sgemm::BM, tn = (p.N + sgemm::BN - 1) / sgemm::BN;
+  const int tm = (p.M + sgemm::BM - 1) / sgemm::BM, tn = (p.N + TN - 1) / TN;
   p.tiles_n = tn;
   int valid = 0;                      // tiles that survive the upper-only filter
   for (int ti = 0; ti < tm; ++ti)
     for (int tj = 0; tj < tn; ++tj)
-      if (!(p.upper_only && ti * sgemm::BM > tj * sgemm::BN + sgemm::BN - 1)) ++valid;
+      if (!(p.upper_only && ti * sgemm::BM > tj * TN + TN - 1)) ++valid;
   const int cap = max_ctas > 0 ? std::min(max_ctas, num_sms()) : num_sms();
   const int grid = std::max(1, std::min(valid, cap));
   LaunchScope ls(name, st);
-  return launch_pdl(sgemm::k_gemm_split_tc, dim3(grid), dim3(256), sgemm::SMEM_BYTES, st, ta, tb, p,
-                    tm * tn);
+  return launch_pdl(sgemm::k_gemm_split_tc<TN>, dim3(grid), dim3(256), (size_t)sgemm::smem_bytes<TN>(),
+                    st, ta, tb, p, tm * tn);
+}
+
+cudaError_t split_gemm(const CUtensorMap& ta, const CUtensorMap& tb, sgemm::Params p,
+                       cudaStream_t st, const char* name, int max_ctas = 0,
+                       const CUtensorMap* tb64 = nullptr) {
+  if (p.M <= 0 || p.N <= 0) return cudaSuccess;
+  const int tiles256 = ((p.M + sgemm::BM - 1) / sgemm::BM) * ((p.N + sgemm::BN - 1) / sgemm::BN);
+  if (tb64 && !p.upper_only && 2 * tiles256 < num_sms())
+    return split_gemm_tn<64>(ta, *tb64, p, st, name, max_ctas);
+  return split_gemm_tn<sgemm::BN>(ta, tb, p, st, name, max_ctas);
 }
 
 // ---------------------------------------------------------------- Hadamard plans
@@ -793,7 +805,7 @@ struct LdlqRun {
   float qmax;
   uint8_t* codes;
   __nv_bfloat16* Es;
-  CUtensorMap ta, tb, tu;
+  CUtensorMap ta, tb, tb64, tu;
   cudaStream_t st;
 };
 
@@ -821,7 +833,7 @@ cudaError_t ldlq_range(const LdlqRun& r, int64_t a, int64_t b) {
   gp.a_piece_rows = (int)r.m, gp.a_k0 = (int)a;
   gp.b_piece_rows = (int)r.n, gp.b_row0 = (int)mid, gp.b_k0 = (int)a;
   gp.alpha = 1.f;
-  e = split_gemm(r.ta, r.tb, gp, r.st, "k_gemm_split_tc[ldlq]");
+  e = split_gemm(r.ta, r.tb, gp, r.st, "k_gemm_split_tc[ldlq]", 0, &r.tb64);
   if (e != cudaSuccess) return e;
   return ldlq_range(r, mid, b);
 }
@@ -866,7 +878,8 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
     return QUIP_ERR_CUDA;
   if (n > LDQ_BLK) {
     if (!make_tmap_bf16_2d(&r.ta, r.Es, (uint64_t)n, 3 * (uint64_t)m, (uint64_t)n * 2, 64, sgemm::BM) ||
-        !make_tmap_bf16_2d(&r.tb, UTs, (uint64_t)n, 3 * (uint64_t)n, (uint64_t)n * 2, 64, sgemm::BN))
+        !make_tmap_bf16_2d(&r.tb, UTs, (uint64_t)n, 3 * (uint64_t)n, (uint64_t)n * 2, 64, sgemm::BN) ||
+        !make_tmap_bf16_2d(&r.tb64, UTs, (uint64_t)n, 3 * (uint64_t)n, (uint64_t)n * 2, 64, 64))
       return QUIP_ERR_CUDA;
   }
   static bool attr = false;
