@@ -11,11 +11,12 @@
 //
 //   k_ldl_factor(p)  R_pp = backward Cholesky of the updated diagonal block,
 //                    with the inverses X_J of its four 32 x 32 diagonal
-//                    blocks, and the 128 "next" rows R12(p)[c0-128 : c0]
-//                    (4 CTAs, each factors the block redundantly and solves
-//                    32 of those rows);
-//   k_ldl_rows(p)    R12(p) = H[:c0, panel p] R_pp^-T (16 rows per CTA) and
-//                    the look-ahead product L(p) = R12(p) R12(p)[c0-128:c0]^T,
+//                    blocks, the block's Ů and D, and the 128 "next" rows
+//                    Nx = R12(p)[c0-128 : c0] (4 CTAs, each factors the block
+//                    redundantly and solves 32 of those rows);
+//   k_ldl_rows(p)    R12(p) = H[:c0, panel p] R_pp^-T (32 rows per block;
+//                    the rows of Nx are taken from there), its Ů and bf16
+//                    pieces, and the look-ahead product L(p) = R12(p) Nx^T,
 //                    i.e. panel p's update of panel p - 1, into a side buffer;
 //   bulk(p)          H[:c0-128, :c0-128] -= R12 R12^T (upper tiles; tensor-
 //                    core split GEMM on a second stream, quip_api.cu).
@@ -37,9 +38,10 @@ constexpr int LDL_PB = 128;
 constexpr int LDL_LDA = 132;    // smem row stride of 128-wide tiles (16-B rows)
 constexpr int LDL_LDX = 36;     // smem row stride of 32-wide tiles (16-B rows)
 constexpr int LDL_FT = 512;     // threads of k_ldl_factor
-constexpr int LDL_FCTAS = 4;    // CTAs of k_ldl_factor when c0 > 0 (32 next rows each)
+constexpr int LDL_NX = 128;     // next rows solved by k_ldl_factor (32 per CTA)
+constexpr int LDL_FCTAS = LDL_NX / 32;
 constexpr int LDL_RT = 256;     // threads of k_ldl_rows
-constexpr int LDL_RR = 16;      // rows per k_ldl_rows CTA
+constexpr int LDL_RR = 32;      // rows per k_ldl_rows block
 constexpr int LDL_HT = 384;     // helper threads of k_ldl_factor (warps w % 4 != 0)
 
 // ---------------------------------------------------------------- helpers
@@ -294,8 +296,7 @@ __device__ __forceinline__ void blk_solve(float* T, const float* Rp, const float
 // CTA c (when c0 > 0) solves next rows c0 - 128 + 32 c .. + 31 of R12(p)
 // into Nx (128 x 128, row i = global row c0 - 128 + i).  CTA 0 writes R_pp
 // (Rd, 128 x 128, upper; lower zero), X_J (Xw, 4 x 32 x 32) and D (Dv[c0 +
-// k] = R_kk^2); with c0 == 0 (the last panel, one CTA) it also writes the
-// block's Ů into H.  Lin: the look-ahead buffer of panel p + 1 (rows
+// k] = R_kk^2); the CTAs split the block's rows for its Ů in H.  Lin: the look-ahead buffer of panel p + 1 (rows
 // [0, c0 + 128) x 128), or NULL.
 // Dynamic smem: (128 + 32) x LDL_LDA + 5 x 32 x LDL_LDX + 96 floats.
 __global__ void __launch_bounds__(LDL_FT, 1)
@@ -390,11 +391,13 @@ __global__ void __launch_bounds__(LDL_FT, 1)
       const float r = A[k * LDL_LDA + k];
       Dv[c0 + k] = r * r;
     }
-    if (!has_next) {
-      for (int e = tid; e < LDL_PB * LDL_PB; e += LDL_FT) {
-        const int i = e >> 7, j = e & 127;
-        if (i < j && j < w) H[(c0 + i) * n + c0 + j] = A[i * LDL_LDA + j] / A[j * LDL_LDA + j];
-      }
+  }
+  {
+    // this CTA's share of the block's Ů
+    const int rows = LDL_PB / gridDim.x, i0 = rows * blockIdx.x;
+    for (int e = tid; e < rows * LDL_PB; e += LDL_FT) {
+      const int i = i0 + (e >> 7), j = e & 127;
+      if (i < j && j < w) H[(c0 + i) * n + c0 + j] = A[i * LDL_LDA + j] / A[j * LDL_LDA + j];
     }
   }
   if (has_next) {
@@ -406,100 +409,150 @@ __global__ void __launch_bounds__(LDL_FT, 1)
   }
 }
 
-// Rows [r0, r0 + LDL_RR) of R12(p) = (H - Lin)[:c0, panel p] R_pp^-T by block
-// back substitution with R_pp (Rd) and X_J (Xw), then
-//   Ů:   H[r, c0 + k] = R12[r][k] / R_kk          (k < w)
-//   Rs:  R12 as three bf16 pieces Rs[q][r][k]     (piece stride n * 128; zero for k >= w)
-//   Lout[r][j] = sum_k R12[r][k] Nx[j][k]         (panel p's update of panel p - 1)
-// CTA 0 also writes the Ů of the diagonal block.
-// Grid: ceil(c0 / LDL_RR) CTAs of 256 threads.
-// Dynamic smem: LDL_RR x LDL_LDA (T) + 128 x LDL_LDA (R_pp, later Nx) + 4 x 32 x LDL_LDX
-// + 128 floats.
-__global__ void __launch_bounds__(LDL_RT, 2)
-    k_ldl_rows(float* __restrict__ H, int64_t n, int64_t c0, int w, const float* __restrict__ Lin,
-               const float* __restrict__ Rd, const float* __restrict__ Xw,
-               const float* __restrict__ Nx, __nv_bfloat16* __restrict__ Rs,
-               float* __restrict__ Lout) {
-  extern __shared__ __align__(16) float sm[];
+// Tiles come in by TMA from fp32 2-D maps without swizzle whose boxes are
+// LDL_LDA (or LDL_LDX) columns wide, so that they land with the padded smem
+// row stride; rows and columns past a tensor's extent arrive as zeros.
+
+// One thread waits for the CTA's tile copies (bounded; after a timeout it
+// waits once more for the copies still in flight) and tells the CTA.
+__device__ __forceinline__ bool tiles_arrived(uint64_t* bar, int* flag) {
+  if (threadIdx.x == 0) {
+    const bool ok = mbar_wait(bar, 0);
+    if (!ok) mbar_wait(bar, 0);
+    *flag = ok ? 1 : 0;
+  }
+  __syncthreads();
+  return *flag != 0;
+}
+
+__device__ __forceinline__ float* align128(uint8_t* p) {
+  return reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(p) + 127) & ~uintptr_t(127));
+}
+
+// Row blocks r0 = row0 + 32 b .. + 31 (b = blockIdx.x, blockIdx.x +
+// gridDim.x, ... < nblk) of panel p:
+//   R12 = (H - Lin)[rows, panel p] R_pp^-T by block back substitution with
+//         R_pp (Rd) and X_J (Xw); rows in [c0 - 128, c0) are taken from Nx;
+//   Ů:    H[r, c0 + k] = R12[r][k] / R_kk          (k < w)
+//   Rs:   R12 as three bf16 pieces Rs[q][r][k]     (piece stride n * 128; zero for k >= w)
+//   Lout[r][j] = sum_k R12[r][k] Nx[j][k]          (panel p's update of panel p - 1)
+// 256 threads; Lout's product: warp v columns [16 v, 16 v + 16), lane
+// (rg, cg) rows rg + 8 a and columns 16 v + cg + 4 b.  R_pp, X_J and Nx are
+// loaded once per CTA; the row tiles of each block on the mbarrier's next
+// phase.
+// Maps: mH32 / mL32 as for k_ldl_factor; mR: Rd (128 x 128, 128-row box);
+// mX: Xw as 128 x 32 (box LDL_LDX wide); mN32 / mN128: Nx (32 / 128-row
+// boxes).
+// Dynamic smem: 128 + (2 x 32 + 2 x 128) x LDL_LDA x 4 + 128 x LDL_LDX x 4 bytes.
+__global__ void __launch_bounds__(LDL_RT, 1)
+    k_ldl_rows(const __grid_constant__ CUtensorMap mH32, const __grid_constant__ CUtensorMap mL32,
+               const __grid_constant__ CUtensorMap mR, const __grid_constant__ CUtensorMap mX,
+               const __grid_constant__ CUtensorMap mN32, const __grid_constant__ CUtensorMap mN128,
+               float* __restrict__ H, int64_t n, int64_t c0, int w, int lin0, int64_t row0,
+               int nblk, __nv_bfloat16* __restrict__ Rs, float* __restrict__ Lout) {
+  extern __shared__ __align__(16) uint8_t ldl_smem_raw[];
   pdl_wait_then_release();
-  float* T = sm;                                     // LDL_RR x LDL_LDA
-  float* Rp = T + LDL_RR * LDL_LDA;                      // 128 x LDL_LDA: R_pp, then Nx
-  float* X = Rp + LDL_PB * LDL_LDA;                  // 4 x 32 x LDL_LDX
-  float* Rkk = X + 4 * 32 * LDL_LDX;                 // 128
-  const int tid = threadIdx.x;
-  const int64_t r0 = (int64_t)blockIdx.x * LDL_RR;
-  for (int e = tid; e < LDL_RR * 32; e += LDL_RT) {
-    const int i = e >> 5, j4 = (e & 31) * 4;
-    const int64_t g = r0 + i;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (g < c0 && j4 < w) {
-      v = *reinterpret_cast<const float4*>(H + g * n + c0 + j4);
-      if (Lin) {
-        const float4 l = *reinterpret_cast<const float4*>(Lin + g * LDL_PB + j4);
-        v.x -= l.x, v.y -= l.y, v.z -= l.z, v.w -= l.w;
+  float* T = align128(ldl_smem_raw);                 // 32 x LDL_LDA: H - Lin, then R12
+  float* Lt = T + LDL_RR * LDL_LDA;                  // 32 x LDL_LDA: Lin rows, then Lout
+  float* Rp = Lt + LDL_RR * LDL_LDA;                 // 128 x LDL_LDA: R_pp
+  float* N = Rp + LDL_PB * LDL_LDA;                  // 128 x LDL_LDA: Nx
+  float* X = N + LDL_PB * LDL_LDA;                   // 4 x 32 x LDL_LDX
+  __shared__ float rkk[LDL_PB];
+  __shared__ int ld_ok;
+  __shared__ __align__(8) uint64_t ld_bar;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    mbar_init(&ld_bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto all_sync = [] { __syncthreads(); };
+  const int64_t pstride = n * LDL_PB;
+  constexpr int RA = LDL_RR / 8;
+  const int rg = lane & 7, cg = lane >> 3, cw = 16 * warp;
+  int it = 0;
+  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x, ++it) {
+    const int64_t r0 = row0 + (int64_t)blk * LDL_RR;
+    const bool from_nx = r0 >= c0 - LDL_NX, lin = lin0 >= 0 && !from_nx;
+    if (tid == 0) {
+      constexpr uint32_t B128 = LDL_PB * LDL_LDA * 4, B32 = LDL_RR * LDL_LDA * 4,
+                         BX = LDL_PB * LDL_LDX * 4;
+      mbar_arrive_expect_tx(&ld_bar, B32 * (lin ? 2u : 1u) + (it == 0 ? 2u * B128 + BX : 0u));
+      if (from_nx) {
+        tma_load_2d(T, &mN32, &ld_bar, 0, (int)(r0 - c0 + LDL_NX));
+      } else {
+        tma_load_2d(T, &mH32, &ld_bar, (int)c0, (int)r0);
+        if (lin) tma_load_2d(Lt, &mL32, &ld_bar, 0, lin0 + (int)r0);
+      }
+      if (it == 0) {
+        tma_load_2d(X, &mX, &ld_bar, 0, 0);
+        tma_load_2d(Rp, &mR, &ld_bar, 0, 0);
+        tma_load_2d(N, &mN128, &ld_bar, 0, 0);
+      }
+      const bool ok = mbar_wait(&ld_bar, (uint32_t)(it & 1));
+      if (!ok) mbar_wait(&ld_bar, (uint32_t)(it & 1));   // copies in flight: bounded again
+      ld_ok = ok ? 1 : 0;
+    }
+    __syncthreads();
+    if (!ld_ok) return;
+    if (!from_nx) {
+      // T = H - Lin on columns < w, zero past w
+      for (int e = tid; e < LDL_RR * 32; e += LDL_RT) {
+        const int i = e >> 5, j4 = (e & 31) * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (j4 < w) {
+          v = *reinterpret_cast<const float4*>(T + i * LDL_LDA + j4);
+          if (lin) {
+            const float4 l = *reinterpret_cast<const float4*>(Lt + i * LDL_LDA + j4);
+            v.x -= l.x, v.y -= l.y, v.z -= l.z, v.w -= l.w;
+          }
+        }
+        *reinterpret_cast<float4*>(T + i * LDL_LDA + j4) = v;
       }
     }
-    *reinterpret_cast<float4*>(T + i * LDL_LDA + j4) = v;
-  }
-#pragma unroll 4
-  for (int e = tid; e < LDL_PB * 32; e += LDL_RT) {
-    const int i = e >> 5, j4 = (e & 31) * 4;
-    *reinterpret_cast<float4*>(Rp + i * LDL_LDA + j4) =
-        *reinterpret_cast<const float4*>(Rd + i * LDL_PB + j4);
-  }
-  for (int e = tid; e < 4 * 32 * 8; e += LDL_RT) {
-    const int jb = e >> 8, r = (e >> 3) & 31, c4 = (e & 7) * 4;
-    *reinterpret_cast<float4*>(X + jb * 32 * LDL_LDX + r * LDL_LDX + c4) =
-        *reinterpret_cast<const float4*>(Xw + jb * 1024 + r * 32 + c4);
-  }
-  __syncthreads();
-  if (tid < LDL_PB) Rkk[tid] = Rp[tid * LDL_LDA + tid];
-  auto all_sync = [] { __syncthreads(); };
-  for (int J = 3; J >= 0; --J) blk_solve<LDL_RR>(T, Rp, X + J * 32 * LDL_LDX, J, tid, LDL_RT, all_sync);
+    if (it == 0 && tid < LDL_PB) rkk[tid] = Rp[tid * LDL_LDA + tid];
+    __syncthreads();
+    if (!from_nx)
+      for (int J = 3; J >= 0; --J) blk_solve<LDL_RR>(T, Rp, X + J * 32 * LDL_LDX, J, tid, LDL_RT, all_sync);
 
-  const int64_t pstride = n * LDL_PB;
-  for (int e = tid; e < LDL_RR * LDL_PB; e += LDL_RT) {
-    const int i = e >> 7, k = e & 127;
-    const int64_t g = r0 + i;
-    if (g >= c0) continue;
-    const float v = T[i * LDL_LDA + k];
-    if (k < w) H[g * n + c0 + k] = v / Rkk[k];
-    __nv_bfloat16 p0, p1, p2;
-    split3(v, p0, p1, p2);
-    Rs[g * LDL_PB + k] = p0;
-    Rs[pstride + g * LDL_PB + k] = p1;
-    Rs[2 * pstride + g * LDL_PB + k] = p2;
-  }
-  if (blockIdx.x == 0) {
-    for (int e = tid; e < LDL_PB * LDL_PB; e += LDL_RT) {
-      const int i = e >> 7, j = e & 127;
-      if (i < j && j < w) H[(c0 + i) * n + c0 + j] = Rp[i * LDL_LDA + j] / Rkk[j];
+    // Ů and the bf16 pieces, 4 columns per task
+    for (int e = tid; e < LDL_RR * 32; e += LDL_RT) {
+      const int i = e >> 5, k4 = (e & 31) * 4;
+      const int64_t g = r0 + i;
+      const float4 v = *reinterpret_cast<const float4*>(T + i * LDL_LDA + k4);
+      if (k4 < w)
+        *reinterpret_cast<float4*>(H + g * n + c0 + k4) =
+            make_float4(v.x / rkk[k4], v.y / rkk[k4 + 1], v.z / rkk[k4 + 2], v.w / rkk[k4 + 3]);
+      __nv_bfloat16 pc[3][4];
+      split3(v.x, pc[0][0], pc[1][0], pc[2][0]);
+      split3(v.y, pc[0][1], pc[1][1], pc[2][1]);
+      split3(v.z, pc[0][2], pc[1][2], pc[2][2]);
+      split3(v.w, pc[0][3], pc[1][3], pc[2][3]);
+#pragma unroll
+      for (int q = 0; q < 3; ++q)
+        *reinterpret_cast<uint2*>(Rs + q * pstride + g * LDL_PB + k4) =
+            *reinterpret_cast<const uint2*>(pc[q]);
     }
-  }
-  __syncthreads();
-#pragma unroll 4
-  for (int e = tid; e < LDL_PB * 32; e += LDL_RT) {
-    const int i = e >> 5, j4 = (e & 31) * 4;
-    *reinterpret_cast<float4*>(Rp + i * LDL_LDA + j4) =
-        *reinterpret_cast<const float4*>(Nx + i * LDL_PB + j4);
-  }
-  __syncthreads();
-  // warp w: columns [16 w, 16 w + 16); lane: rows rg + 8 a, columns 16 w + cg + 4 b
-  constexpr int RA = LDL_RR / 8;
-  const int warp = tid >> 5, lane = tid & 31, rg = lane & 7, cg = lane >> 3;
-  float acc[RA][4];
+
+    // Lout = R12 Nx^T, staged in Lt for row-contiguous stores
+    float acc[RA][4];
 #pragma unroll
-  for (int a = 0; a < RA; ++a)
+    for (int a = 0; a < RA; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-  dot_rows<RA, 4>(acc, T + rg * LDL_LDA, 8 * LDL_LDA, Rp + (16 * warp + cg) * LDL_LDA, 4 * LDL_LDA,
-                  LDL_PB);
+      for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+    dot_rows<RA, 4>(acc, T + rg * LDL_LDA, 8 * LDL_LDA, N + (cw + cg) * LDL_LDA, 4 * LDL_LDA, LDL_PB);
 #pragma unroll
-  for (int a = 0; a < RA; ++a) {
-    const int64_t g = r0 + rg + 8 * a;
-    if (g < c0)
+    for (int a = 0; a < RA; ++a)
 #pragma unroll
-      for (int b = 0; b < 4; ++b) Lout[g * LDL_PB + 16 * warp + cg + 4 * b] = acc[a][b];
+      for (int b = 0; b < 4; ++b) Lt[(rg + 8 * a) * LDL_LDA + cw + cg + 4 * b] = acc[a][b];
+    __syncthreads();
+    for (int e = tid; e < LDL_RR * 32; e += LDL_RT) {
+      const int i = e >> 5, j4 = (e & 31) * 4;
+      *reinterpret_cast<float4*>(Lout + (r0 + i) * LDL_PB + j4) =
+          *reinterpret_cast<const float4*>(Lt + i * LDL_LDA + j4);
+    }
+    fence_proxy_async_smem();                         // T and Lt free for the next block's copies
+    __syncthreads();
   }
 }
 

@@ -87,6 +87,21 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint6
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 2-D map without swizzle (boxes may be wider than the tensor: the
+// columns past it arrive as zeros).
+bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                      uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // A second stream per device for the LDL bulk updates, with a fork event and
 // a ring of join events, created on first use and kept for the process.
 constexpr int kJoinRing = 4;
@@ -735,13 +750,22 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
   __nv_bfloat16* Rs = reinterpret_cast<__nv_bfloat16*>(w8);
   const size_t smem_f = ((size_t)(LDL_PB + 32) * LDL_LDA + 5 * 32 * LDL_LDX + 96) * sizeof(float);
   const size_t smem_r =
-      ((size_t)(LDL_RR + LDL_PB) * LDL_LDA + 4 * 32 * LDL_LDX + LDL_PB) * sizeof(float);
+      128 + ((size_t)(2 * LDL_RR + 2 * LDL_PB) * LDL_LDA + LDL_PB * LDL_LDX) * sizeof(float);
   static bool attr = false;
   if (!attr) {
     QCHECK(cudaFuncSetAttribute(k_ldl_factor, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_f));
     QCHECK(cudaFuncSetAttribute(k_ldl_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_r));
     attr = true;
   }
+  // fp32 tiles for the row kernel, landing with the padded smem row stride
+  CUtensorMap mH32, mL32, mR, mX, mN32, mN128;
+  if (!make_tmap_f32_2d(&mH32, H_t, n, n, n * 4, LDL_LDA, LDL_RR) ||
+      !make_tmap_f32_2d(&mL32, Lb, LDL_PB, 2 * n, LDL_PB * 4, LDL_LDA, LDL_RR) ||
+      !make_tmap_f32_2d(&mR, Rd, LDL_PB, LDL_PB, LDL_PB * 4, LDL_LDA, LDL_PB) ||
+      !make_tmap_f32_2d(&mX, Xw, 32, LDL_PB, 32 * 4, LDL_LDX, LDL_PB) ||
+      !make_tmap_f32_2d(&mN32, Nx, LDL_PB, LDL_PB, LDL_PB * 4, LDL_LDA, LDL_RR) ||
+      !make_tmap_f32_2d(&mN128, Nx, LDL_PB, LDL_PB, LDL_PB * 4, LDL_LDA, LDL_PB))
+    return QUIP_ERR_CUDA;
   // Rs holds two panels' R12 (buffer p & 1), pieces at rows (3 buf + q) n.
   CUtensorMap ta, tb;
   SideStream side;
@@ -752,6 +776,7 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
     QCHECK(side_stream(side));
   }
   const float* Lin = nullptr;
+  int lin0 = -1;                 // Lin's first row in mL32
   for (int64_t p = P - 1; p >= 0; --p) {
     const int64_t c0 = p * LDL_PB;
     const int w = (int)std::min<int64_t>(LDL_PB, n - c0);
@@ -767,10 +792,11 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
     if (c0 == 0) break;
     float* Lout = Lb + (size_t)buf * n * LDL_PB;
     {
+      const int nblk = (int)(c0 / LDL_RR);
       LaunchScope ls("k_ldl_rows", st);
-      QCHECK(launch_pdl(k_ldl_rows, dim3((unsigned)((c0 + LDL_RR - 1) / LDL_RR)), dim3(LDL_RT),
-                        smem_r, st, H_t, n, c0, w, Lin, (const float*)Rd, (const float*)Xw,
-                        (const float*)Nx, Rs + (size_t)buf * 3 * n * LDL_PB, Lout));
+      QCHECK(launch_pdl(k_ldl_rows, dim3((unsigned)nblk), dim3(LDL_RT), smem_r, st, mH32, mL32, mR, mX,
+                        mN32, mN128, H_t, n, c0, w, lin0, (int64_t)0, nblk,
+                        Rs + (size_t)buf * 3 * n * LDL_PB, Lout));
     }
     if (c0 > LDL_PB) {
       // H[:c0-128, :c0-128] -= R12 R12^T on the upper tiles, on the side
@@ -783,12 +809,13 @@ quip_status quip_ldl(float* H_t, float* D, int64_t n, void* ws, size_t ws_bytes,
       gp.a_piece_rows = (int)n, gp.b_piece_rows = (int)n;
       gp.a_row0 = gp.b_row0 = 3 * (int)n * buf;
       gp.alpha = -1.f, gp.upper_only = 1;
-      const int next_rows_sms = (int)(((c0 - LDL_PB) / LDL_RR + 1) / 2);
+      const int next_rows_sms = (int)((c0 - LDL_PB) / LDL_RR);
       const int cap = std::max(num_sms() / 2, num_sms() - LDL_FCTAS - next_rows_sms);
       QCHECK(split_gemm(ta, tb, gp, side.s, "k_gemm_split_tc[ldl]", cap));
       QCHECK(cudaEventRecord(side.join[p % kJoinRing], side.s));
     }
     Lin = Lout;
+    lin0 = buf * (int)n;
   }
   QCHECK(cudaGetLastError());
   return QUIP_OK;
