@@ -112,7 +112,7 @@ def kernel_work(cfg: LayerConfig):
         "k_ldl_rows": ("flops", rows, "alu"),
         "k_gemm_split_tc[ldl]": ("flops", bulk, "tensor"),
         "k_gemm_split_tc[ldlq]": ("flops", _ldlq_gemm_flops(m, n, 128), "tensor"),
-        "k_ldlq_tc": ("flops", _ldlq_block_flops(m, n), "alu"),
+        "k_ldlq_block": ("flops", _ldlq_block_flops(m, n), "alu"),
         "k_row_grid": ("bytes", 4.0 * m * n + 8.0 * m, "hbm"),
         "k_dequant": ("bytes", 5.0 * m * n + 8.0 * m, "hbm"),
         "k_split_upper_transposed": ("bytes", 4.0 * n * n / 2 + 6.0 * n * n, "hbm"),

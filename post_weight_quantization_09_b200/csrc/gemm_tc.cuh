@@ -260,10 +260,13 @@ __device__ __forceinline__ void split3(float x, __nv_bfloat16& p0, __nv_bfloat16
 
 // out[p][j][i] = piece_p(U[i][j]) for i < j (strict upper), 0 otherwise:
 // the transposed, split copy of the LDL factor that LDLQ's trailing GEMM
-// reads as its K-major B operand.  32 x 32 tiles through shared memory.
+// reads as its K-major B operand; outf[j][i] = U[i][j] (same zeros), the
+// fp32 transposed copy the LDLQ block kernel reads.  32 x 32 tiles through
+// shared memory.
 __global__ void __launch_bounds__(256) k_split_upper_transposed(const float* __restrict__ U,
                                                                 int64_t ldu, int64_t n,
-                                                                __nv_bfloat16* __restrict__ out) {
+                                                                __nv_bfloat16* __restrict__ out,
+                                                                float* __restrict__ outf) {
   __shared__ float t[32][33];
   const int64_t bi = blockIdx.y, bj = blockIdx.x;   // source tile (rows bi, cols bj)
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -281,6 +284,7 @@ __global__ void __launch_bounds__(256) k_split_upper_transposed(const float* __r
       out[j * n + i] = p0;
       out[pn + j * n + i] = p1;
       out[2 * pn + j * n + i] = p2;
+      outf[j * n + i] = t[tx][r];
     }
   }
 }

@@ -638,11 +638,12 @@ static size_t ldl_ws_bytes(int64_t n) {
          round256((size_t)2 * n * LDL_PB * 4) + round256((size_t)6 * n * LDL_PB * 2);
 }
 // LDLQ workspace: accumulator A (m x n fp32), the error of every column as
-// three bf16 pieces (3 x m x n), the split transposed factor (3 x n x n bf16).
+// three bf16 pieces (3 x m x n), the split transposed factor (3 x n x n
+// bf16) and the transposed factor (n x n fp32).
 static size_t ldlq_ws_bytes(int64_t m, int64_t n, int64_t block) {
   (void)block;
   return round256((size_t)m * n * 4) + round256((size_t)3 * m * n * 2) +
-         round256((size_t)3 * n * n * 2);
+         round256((size_t)3 * n * n * 2) + round256((size_t)n * n * 4);
 }
 
 quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int64_t n,
@@ -832,18 +833,17 @@ struct LdlqRun {
   float qmax;
   uint8_t* codes;
   __nv_bfloat16* Es;
-  CUtensorMap ta, tb, tb64, tu;
+  CUtensorMap ta, tb, tb64, tacc, tut, tband;
   cudaStream_t st;
 };
 
 constexpr int LDQ_BLK = 128;               // LDLQ block width (columns)
 
 cudaError_t ldlq_block(const LdlqRun& r, int64_t k0, int w) {
-  const unsigned grid = (unsigned)((r.m + 127) / 128);
-  LaunchScope ls("k_ldlq_tc", r.st);
-  return launch_pdl(k_ldlq_tc, dim3(grid), dim3(LQT_THREADS), (size_t)LQT_SMEM, r.st, r.tu, r.Wt,
-                    (const float*)r.A, r.m, r.n, k0, w, r.U, r.ldu, r.lo, r.sc, r.qmax, r.codes, r.Es,
-                    r.n);
+  const unsigned grid = (unsigned)((r.m + LQB_ROWS - 1) / LQB_ROWS);
+  LaunchScope ls("k_ldlq_block", r.st);
+  return launch_pdl(k_ldlq_block, dim3(grid), dim3(LQB_THREADS), (size_t)LQB_SMEM, r.st, r.tacc, r.tut,
+                    r.tband, r.Wt, r.m, r.n, k0, w, r.lo, r.sc, r.qmax, r.codes, r.Es, r.n);
 }
 
 // Columns [a, b): left half, then A[:, mid:b] += Err[:, a:mid] Ů[a:mid, mid:b]
@@ -889,6 +889,8 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
   r.Es = reinterpret_cast<__nv_bfloat16*>(w8);
   w8 += round256((size_t)3 * m * n * 2);
   __nv_bfloat16* UTs = reinterpret_cast<__nv_bfloat16*>(w8);
+  w8 += round256((size_t)3 * n * n * 2);
+  float* UTf = reinterpret_cast<float*>(w8);
   r.Wt = W_t, r.U = Uring, r.ldu = ldu, r.m = m, r.n = n, r.lo = lo, r.sc = scale;
   r.qmax = (float)((1 << bits) - 1), r.codes = codes;
   {
@@ -899,9 +901,11 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
   {
     const unsigned T = (unsigned)((n + 31) / 32);
     LaunchScope ls("k_split_upper_transposed", r.st);
-    k_split_upper_transposed<<<dim3(T, T), 256, 0, r.st>>>(Uring, ldu, n, UTs);
+    k_split_upper_transposed<<<dim3(T, T), 256, 0, r.st>>>(Uring, ldu, n, UTs, UTf);
   }
-  if (!make_tmap_bf16_2d(&r.tu, UTs, (uint64_t)n, 3 * (uint64_t)n, (uint64_t)n * 2, 64, 128))
+  if (!make_tmap_f32_2d(&r.tacc, r.A, (uint64_t)n, (uint64_t)m, (uint64_t)n * 4, LQB_S, LQB_ROWS) ||
+      !make_tmap_f32_2d(&r.tut, UTf, (uint64_t)n, (uint64_t)n, (uint64_t)n * 4, LQB_S, 128) ||
+      !make_tmap_f32_2d(&r.tband, Uring, (uint64_t)n, (uint64_t)n, (uint64_t)ldu * 4, 32, 16))
     return QUIP_ERR_CUDA;
   if (n > LDQ_BLK) {
     if (!make_tmap_bf16_2d(&r.ta, r.Es, (uint64_t)n, 3 * (uint64_t)m, (uint64_t)n * 2, 64, sgemm::BM) ||
@@ -911,7 +915,7 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
   }
   static bool attr = false;
   if (!attr) {
-    QCHECK(cudaFuncSetAttribute(k_ldlq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, LQT_SMEM));
+    QCHECK(cudaFuncSetAttribute(k_ldlq_block, cudaFuncAttributeMaxDynamicSharedMemorySize, LQB_SMEM));
     attr = true;
   }
   QCHECK(ldlq_range(r, 0, n));
