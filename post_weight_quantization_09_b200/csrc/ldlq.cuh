@@ -73,8 +73,9 @@ __device__ __forceinline__ void nb_arrive(int id, int count) {
 
 // Block step over the w columns [k0, k0 + w) (w = 128, or 64 for a last,
 // partial block) for 32 rows per CTA, on the FP32 pipes: warp 0 rounds
-// (lane r = row r), warps 1-3 apply the feedback that can wait.  TMA brings
-// the rows' accumulated values of the block (acc, row r at stride LQB_S:
+// (lane r = row r), warps 1-3 apply the feedback that can wait.  Global
+// memory is touched only by the copies in and the stores out: TMA brings
+// the rows' W~ and accumulated values of the block (wt, acc; row r at stride LQB_S:
 // 16-byte accesses of a warp are conflict-free), the transposed Ů block
 // (UT[j][k] = Ů[k0 + k][k0 + j], zero for k >= j) and the band of Ů next to
 // the diagonal (band[k][jj] = Ů[k0 + k][k0 + 16 (k / 16) + jj], as eight
@@ -85,36 +86,41 @@ __device__ __forceinline__ void nb_arrive(int id, int count) {
 //      group's feedback, in registers);
 //   2. rounds column by column, feeding each error to the group's later
 //      columns and, into carry, to the next group;
-//   3. hands the 16 errors to the helpers (shared slot g % 2) and stores
-//      the codes and the errors' three bf16 pieces (the trailing GEMMs'
-//      A operand).
-// Helper thread (h, r) adds group g's feedback to row r's columns from two
-// groups on that it owns (4-column chunks c with c % 3 == h - 1),
-// acc[r][j] += sum_t e_t Ů[16 g + t][j], with broadcast 16-byte loads of UT
-// rows, while warp 0 rounds group g + 1.  Named barriers pass the hand-off
+//   3. hands the 16 errors and codes to the helpers (shared slot g % 2).
+// The helpers stage the codes and the errors' three bf16 pieces (the
+// trailing GEMMs' A operand; written out with coalesced stores after the
+// last group) and add group g's feedback to the columns from
+// two groups on, acc[r][j] += sum_t e_t Ů[16 g + t][j] (each thread: four
+// rows and every twelfth 4-column chunk, so one broadcast 16-byte load of a
+// UT row serves 16 fmas), while warp 0 rounds group g + 1.  Named barriers
+// pass the hand-off
 // slots: READY + slot (warp 0 -> helpers, every group) and DONE + slot
 // (helpers -> warp 0, only for groups that warp 0 will wait on).
 // Rounding: clamp to [0, qmax] first, then add and subtract 1.5 * 2^23,
 // which rounds half to even exactly like rintf on that range (and leaves
 // the integer, the code, in the low mantissa bits).
-// Maps: tmA over the accumulator (m x n fp32, LQB_S x 32 boxes), tmUT over
+// Maps: tmA over the accumulator and tmW over W~ (m x n fp32, LQB_S x 32 boxes), tmUT over
 // the transposed factor (n x n fp32, LQB_S x 128 boxes), tmU over the
 // factor Ů (the LDL's output, row stride ldu; 32 x 16 boxes).
 constexpr int LQB_ROWS = 32;                           // rows per CTA
 constexpr int LQB_THREADS = 128;                       // warp 0 rounds, warps 1-3 help
 constexpr int LQB_S = 132;                             // smem row stride of acc and UT
-constexpr int LQB_ES = 20;                             // smem row stride of the error slots
+constexpr int LQB_ES = 20;                             // smem row stride of the slots: 16 errors, 4 code words
 constexpr int LQB_ACC = LQB_ROWS * LQB_S * 4;          // bytes of the acc tile
 constexpr int LQB_UT = 128 * LQB_S * 4;                // bytes of the UT tile
 constexpr int LQB_BAND = 128 * 32 * 4;                 // bytes of the band
-constexpr int LQB_E = 2 * LQB_ROWS * LQB_ES * 4;       // bytes of the two error slots
-constexpr int LQB_SMEM = 128 + LQB_ACC + LQB_UT + LQB_BAND + LQB_E;
+constexpr int LQB_E = 2 * LQB_ROWS * LQB_ES * 4;       // bytes of the two error slots (+ codes)
+constexpr int LQB_PS = 136;                            // row stride (bf16) of the staged pieces
+constexpr int LQB_CS = 144;                            // row stride (bytes) of the staged codes
+constexpr int LQB_P = 3 * LQB_ROWS * LQB_PS * 2;       // bytes of the staged pieces
+constexpr int LQB_C = LQB_ROWS * LQB_CS;               // bytes of the staged codes
+constexpr int LQB_SMEM = 128 + 2 * LQB_ACC + LQB_UT + LQB_BAND + LQB_E + LQB_P + LQB_C;
 constexpr int LQB_READY = 1, LQB_DONE = 3;             // named barrier ids (+ slot)
 
 __global__ void __launch_bounds__(LQB_THREADS, 1)
     k_ldlq_block(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmUT,
-                 const __grid_constant__ CUtensorMap tmU, const float* __restrict__ Wt, int64_t m,
-                 int64_t n, int64_t k0, int w, const float* __restrict__ lo,
+                 const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmW,
+                 int64_t m, int64_t n, int64_t k0, int w, const float* __restrict__ lo,
                  const float* __restrict__ sc, float qmax, uint8_t* __restrict__ codes,
                  __nv_bfloat16* __restrict__ Es, int64_t lde) {
   extern __shared__ __align__(16) uint8_t lqb_raw[];
@@ -122,6 +128,9 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
   float* UT = acc + LQB_ROWS * LQB_S;
   float* band = UT + 128 * LQB_S;
   float* eslot = band + 128 * 32;                      // [2][32][LQB_ES]
+  float* wt = eslot + 2 * LQB_ROWS * LQB_ES;           // [32][LQB_S]: the rows' W~ of the block
+  __nv_bfloat16* ps = reinterpret_cast<__nv_bfloat16*>(wt + LQB_ROWS * LQB_S);   // [3][32][LQB_PS]
+  uint8_t* cs = reinterpret_cast<uint8_t*>(ps + 3 * LQB_ROWS * LQB_PS);        // [32][LQB_CS]
   __shared__ __align__(8) uint64_t bar;
   __shared__ int ok_s;
   const int tid = threadIdx.x, warp = tid >> 5, r = tid & 31;
@@ -134,8 +143,9 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
   __syncthreads();
   pdl_wait_then_release();
   if (tid == 0) {
-    mbar_arrive_expect_tx(&bar, (uint32_t)(LQB_ACC + LQB_UT + LQB_BAND));
+    mbar_arrive_expect_tx(&bar, (uint32_t)(2 * LQB_ACC + LQB_UT + LQB_BAND));
     tma_load_2d(acc, &tmA, &bar, (int)k0, (int)(blockIdx.x * LQB_ROWS));
+    tma_load_2d(wt, &tmW, &bar, (int)k0, (int)(blockIdx.x * LQB_ROWS));
     tma_load_2d(UT, &tmUT, &bar, (int)k0, (int)k0);
     for (int i = 0; i < 8; ++i)
       tma_load_2d(band + 16 * 32 * i, &tmU, &bar, (int)(k0 + 16 * i), (int)(k0 + 16 * i));
@@ -156,59 +166,94 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
 
   if (warp > 0) {
     // ------------------------------------------------------------ helpers
-    float* myacc = acc + r * LQB_S;
-    const int h = warp - 1;
+    // thread (h, lane): rows lane % 8 + 8 i (i < 4) and the 4-column chunks
+    // c with c % 12 == 4 h + lane / 8 (every Ů^T load serves four rows);
+    // helper warp 0 also stores row `lane`'s codes and error pieces.
+    const int h = warp - 1, rb = r & 7, cls = 4 * h + (r >> 3);
 #pragma unroll 1
     for (int g = 0; g < ngroups; ++g) {
       const int slot = g & 1;
       nb_sync(LQB_READY + slot, LQB_THREADS);
-      const float* es = eslot + (slot * LQB_ROWS + r) * LQB_ES;
-      float e[16];
+      const float* eb = eslot + slot * LQB_ROWS * LQB_ES;
+      if (h == 0) {
+        // row r's codes and error pieces into the staging buffers
+        const float* es = eb + r * LQB_ES;
+        float e[16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 v = *reinterpret_cast<const float4*>(es + 4 * q);
-        e[4 * q] = v.x, e[4 * q + 1] = v.y, e[4 * q + 2] = v.z, e[4 * q + 3] = v.w;
+        for (int q = 0; q < 4; ++q) {
+          const float4 v = *reinterpret_cast<const float4*>(es + 4 * q);
+          e[4 * q] = v.x, e[4 * q + 1] = v.y, e[4 * q + 2] = v.z, e[4 * q + 3] = v.w;
+        }
+        *reinterpret_cast<uint4*>(cs + r * LQB_CS + 16 * g) = *reinterpret_cast<const uint4*>(es + 16);
+        uint32_t pk[3][8];
+#pragma unroll
+        for (int t = 0; t < 16; t += 2)
+          split3x2(e[t], e[t + 1], pk[0][t >> 1], pk[1][t >> 1], pk[2][t >> 1]);
+#pragma unroll
+        for (int p = 0; p < 3; ++p) {
+          uint4* dst = reinterpret_cast<uint4*>(ps + (p * LQB_ROWS + r) * LQB_PS + 16 * g);
+          dst[0] = make_uint4(pk[p][0], pk[p][1], pk[p][2], pk[p][3]);
+          dst[1] = make_uint4(pk[p][4], pk[p][5], pk[p][6], pk[p][7]);
+        }
       }
-      const float* ug = UT + 16 * g;
       const int c0 = 4 * (g + 2);                      // first chunk two groups on
-      int c = c0 + ((h - c0 % 3) + 3) % 3;             // first chunk this warp owns
-#pragma unroll 1
-      for (; 4 * c < w; c += 3) {
-        const int j = 4 * c;
-        const float4 a4 = *reinterpret_cast<const float4*>(myacc + j);
-        float a[4] = {a4.x, a4.y, a4.z, a4.w};
+      int c = c0 + ((cls - c0 % 12) + 12) % 12;        // first chunk of this class
+      if (4 * c < w) {
+        float e[4][16];
 #pragma unroll
-        for (int t4 = 0; t4 < 16; t4 += 4) {
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const float4 u = *reinterpret_cast<const float4*>(ug + (j + q) * LQB_S + t4);
-            a[q] = fmaf(e[t4 + 0], u.x, a[q]);
-            a[q] = fmaf(e[t4 + 1], u.y, a[q]);
-            a[q] = fmaf(e[t4 + 2], u.z, a[q]);
-            a[q] = fmaf(e[t4 + 3], u.w, a[q]);
+            const float4 v = *reinterpret_cast<const float4*>(eb + (rb + 8 * i) * LQB_ES + 4 * q);
+            e[i][4 * q] = v.x, e[i][4 * q + 1] = v.y, e[i][4 * q + 2] = v.z, e[i][4 * q + 3] = v.w;
           }
+        const float* ug = UT + 16 * g;
+#pragma unroll 1
+        for (; 4 * c < w; c += 12) {
+          const int j = 4 * c;
+          float a[4][4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 a4 = *reinterpret_cast<const float4*>(acc + (rb + 8 * i) * LQB_S + j);
+            a[i][0] = a4.x, a[i][1] = a4.y, a[i][2] = a4.z, a[i][3] = a4.w;
+          }
+#pragma unroll
+          for (int t4 = 0; t4 < 16; t4 += 4) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float4 u = *reinterpret_cast<const float4*>(ug + (j + q) * LQB_S + t4);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                a[i][q] = fmaf(e[i][t4 + 0], u.x, a[i][q]);
+                a[i][q] = fmaf(e[i][t4 + 1], u.y, a[i][q]);
+                a[i][q] = fmaf(e[i][t4 + 2], u.z, a[i][q]);
+                a[i][q] = fmaf(e[i][t4 + 3], u.w, a[i][q]);
+              }
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4*>(acc + (rb + 8 * i) * LQB_S + j) =
+                make_float4(a[i][0], a[i][1], a[i][2], a[i][3]);
         }
-        *reinterpret_cast<float4*>(myacc + j) = make_float4(a[0], a[1], a[2], a[3]);
       }
       if (g + 2 < ngroups) nb_arrive(LQB_DONE + slot, LQB_THREADS);
     }
-    return;
-  }
+  } else {
 
   // ------------------------------------------------------------ warp 0: rounding
   const float l = valid ? lo[row] : 0.f;
   const float s = valid ? sc[row] : 1.f;
   const float inv = 1.0f / s;
-  const int64_t pst = m * lde;
   constexpr float kRound = 12582912.0f;                // 1.5 * 2^23
   const float* myacc = acc + r * LQB_S;
+  const float* mywt = wt + r * LQB_S;
   float carry[16], wv[16];
 #pragma unroll
   for (int t = 0; t < 16; ++t) carry[t] = 0.f;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (valid) f = *reinterpret_cast<const float4*>(Wt + row * n + k0 + 4 * q);
+    const float4 f = *reinterpret_cast<const float4*>(mywt + 4 * q);
     wv[4 * q] = f.x, wv[4 * q + 1] = f.y, wv[4 * q + 2] = f.z, wv[4 * q + 3] = f.w;
   }
 #pragma unroll 1
@@ -228,13 +273,16 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
     float wn[16];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (valid && g + 1 < ngroups)
-        f = *reinterpret_cast<const float4*>(Wt + row * n + k0 + 16 * (g + 1) + 4 * q);
+      const float4 f = *reinterpret_cast<const float4*>(mywt + 16 * ((g + 1) & 7) + 4 * q);
       wn[4 * q] = f.x, wn[4 * q + 1] = f.y, wn[4 * q + 2] = f.z, wn[4 * q + 3] = f.w;
     }
     float e[16];
     uint32_t cw[4] = {0u, 0u, 0u, 0u};
+    // the group's super-diagonal Ů[t][t + 1] in registers: the rounding chain
+    // (column t's error into column t + 1) never waits for shared memory
+    float sd[15];
+#pragma unroll
+    for (int t = 0; t < 15; ++t) sd[t] = band[(16 * g + t) * 32 + t + 1];
 #pragma unroll
     for (int j = 0; j < 16; ++j) carry[j] = 0.f;
 #pragma unroll
@@ -244,16 +292,17 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
       const float cq = zr - kRound;
       const float err = wv[t] - fmaf(s, cq, l);
       e[t] = err;
+      if (t < 15) cur[t + 1] = fmaf(err, sd[t], cur[t + 1]);
       cw[t >> 2] |= (__float_as_uint(zr) & 0xffu) << (8 * (t & 3));
       // band row 16 g + t: this group's later columns, then the next group's
       const float* ur = band + (16 * g + t) * 32;
 #pragma unroll
-      for (int q4 = ((t + 1) >> 2) << 2; q4 < 16; q4 += 4) {
+      for (int q4 = ((t + 2) >> 2) << 2; q4 < 16; q4 += 4) {
         const float4 u = *reinterpret_cast<const float4*>(ur + q4);
-        if (q4 + 0 > t) cur[q4 + 0] = fmaf(err, u.x, cur[q4 + 0]);
-        if (q4 + 1 > t) cur[q4 + 1] = fmaf(err, u.y, cur[q4 + 1]);
-        if (q4 + 2 > t) cur[q4 + 2] = fmaf(err, u.z, cur[q4 + 2]);
-        if (q4 + 3 > t) cur[q4 + 3] = fmaf(err, u.w, cur[q4 + 3]);
+        if (q4 + 0 > t + 1) cur[q4 + 0] = fmaf(err, u.x, cur[q4 + 0]);
+        if (q4 + 1 > t + 1) cur[q4 + 1] = fmaf(err, u.y, cur[q4 + 1]);
+        if (q4 + 2 > t + 1) cur[q4 + 2] = fmaf(err, u.z, cur[q4 + 2]);
+        if (q4 + 3 > t + 1) cur[q4 + 3] = fmaf(err, u.w, cur[q4 + 3]);
       }
 #pragma unroll
       for (int q4 = 0; q4 < 16; q4 += 4) {
@@ -264,26 +313,35 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
         carry[q4 + 3] = fmaf(err, u.w, carry[q4 + 3]);
       }
     }
+    // hand the errors and codes to the helpers
     float* es = eslot + (slot * LQB_ROWS + r) * LQB_ES;
 #pragma unroll
     for (int q = 0; q < 4; ++q)
       *reinterpret_cast<float4*>(es + 4 * q) = make_float4(e[4 * q], e[4 * q + 1], e[4 * q + 2], e[4 * q + 3]);
+    *reinterpret_cast<uint4*>(es + 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
     nb_arrive(LQB_READY + slot, LQB_THREADS);
-    if (valid) {
-      *reinterpret_cast<uint4*>(codes + row * n + k0 + 16 * g) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-      uint32_t pk[3][8];
-#pragma unroll
-      for (int t = 0; t < 16; t += 2)
-        split3x2(e[t], e[t + 1], pk[0][t >> 1], pk[1][t >> 1], pk[2][t >> 1]);
-#pragma unroll
-      for (int p = 0; p < 3; ++p) {
-        uint4* dst = reinterpret_cast<uint4*>(Es + p * pst + row * lde + k0 + 16 * g);
-        dst[0] = make_uint4(pk[p][0], pk[p][1], pk[p][2], pk[p][3]);
-        dst[1] = make_uint4(pk[p][4], pk[p][5], pk[p][6], pk[p][7]);
-      }
-    }
 #pragma unroll
     for (int t = 0; t < 16; ++t) wv[t] = wn[t];
+  }
+  }
+  // every group staged: codes and pieces out with coalesced 16-byte stores
+  __syncthreads();
+  const int64_t pst = m * lde;
+  const int nv = w / 8;                                // 16-byte vectors per row and piece
+  for (int e = tid; e < 3 * LQB_ROWS * nv; e += LQB_THREADS) {
+    const int p = e / (LQB_ROWS * nv), rr = (e / nv) % LQB_ROWS, v = e % nv;
+    const int64_t gr = (int64_t)blockIdx.x * LQB_ROWS + rr;
+    if (gr < m)
+      *reinterpret_cast<uint4*>(Es + p * pst + gr * lde + k0 + 8 * v) =
+          *reinterpret_cast<const uint4*>(ps + (p * LQB_ROWS + rr) * LQB_PS + 8 * v);
+  }
+  const int nc = w / 16;                               // 16-byte vectors of codes per row
+  for (int e = tid; e < LQB_ROWS * nc; e += LQB_THREADS) {
+    const int rr = e / nc, v = e % nc;
+    const int64_t gr = (int64_t)blockIdx.x * LQB_ROWS + rr;
+    if (gr < m)
+      *reinterpret_cast<uint4*>(codes + gr * n + k0 + 16 * v) =
+          *reinterpret_cast<const uint4*>(cs + rr * LQB_CS + 16 * v);
   }
 }
 

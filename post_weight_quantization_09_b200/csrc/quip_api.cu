@@ -833,7 +833,7 @@ struct LdlqRun {
   float qmax;
   uint8_t* codes;
   __nv_bfloat16* Es;
-  CUtensorMap ta, tb, tb64, tacc, tut, tband;
+  CUtensorMap ta, tb, tb64, tacc, tut, tband, tw;
   cudaStream_t st;
 };
 
@@ -843,7 +843,7 @@ cudaError_t ldlq_block(const LdlqRun& r, int64_t k0, int w) {
   const unsigned grid = (unsigned)((r.m + LQB_ROWS - 1) / LQB_ROWS);
   LaunchScope ls("k_ldlq_block", r.st);
   return launch_pdl(k_ldlq_block, dim3(grid), dim3(LQB_THREADS), (size_t)LQB_SMEM, r.st, r.tacc, r.tut,
-                    r.tband, r.Wt, r.m, r.n, k0, w, r.lo, r.sc, r.qmax, r.codes, r.Es, r.n);
+                    r.tband, r.tw, r.m, r.n, k0, w, r.lo, r.sc, r.qmax, r.codes, r.Es, r.n);
 }
 
 // Columns [a, b): left half, then A[:, mid:b] += Err[:, a:mid] Ů[a:mid, mid:b]
@@ -904,6 +904,7 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
     k_split_upper_transposed<<<dim3(T, T), 256, 0, r.st>>>(Uring, ldu, n, UTs, UTf);
   }
   if (!make_tmap_f32_2d(&r.tacc, r.A, (uint64_t)n, (uint64_t)m, (uint64_t)n * 4, LQB_S, LQB_ROWS) ||
+      !make_tmap_f32_2d(&r.tw, W_t, (uint64_t)n, (uint64_t)m, (uint64_t)n * 4, LQB_S, LQB_ROWS) ||
       !make_tmap_f32_2d(&r.tut, UTf, (uint64_t)n, (uint64_t)n, (uint64_t)n * 4, LQB_S, 128) ||
       !make_tmap_f32_2d(&r.tband, Uring, (uint64_t)n, (uint64_t)n, (uint64_t)ldu * 4, 32, 16))
     return QUIP_ERR_CUDA;
