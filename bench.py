@@ -115,7 +115,7 @@ def kernel_work(cfg: LayerConfig):
         "k_ldlq_block": ("flops", _ldlq_block_flops(m, n), "alu"),
         "k_row_grid": ("bytes", 4.0 * m * n + 8.0 * m, "hbm"),
         "k_dequant": ("bytes", 5.0 * m * n + 8.0 * m, "hbm"),
-        "k_split_upper_transposed": ("bytes", 4.0 * n * n / 2 + 6.0 * n * n, "hbm"),
+        "k_split_upper_transposed": ("bytes", 4.0 * n * n / 2 + 10.0 * n * n, "hbm"),
         "k_mirror_scale": ("bytes", 8.0 * n * n, "hbm"),
     }
     # Hadamard passes: rows read their input (W once as bf16/f32, H and W^
@@ -141,11 +141,13 @@ def kernel_work(cfg: LayerConfig):
 # unchanged and only for the workload it was captured on.
 KERNEL_TRAFFIC = {
     "k_syrk_tc": ("syrk_tc.cuh", "260ad4eebdfc", 71597824),
-    "k_ldl_factor": ("ldl.cuh", "fbc7579dcf4b", 335360),
-    "k_ldl_rows": ("ldl.cuh", "fbc7579dcf4b", 3834112),
-    "k_fwht_cols": ("fwht.cuh", "dbbc29ed00b7", 79775232),
-    "k_fwht_rows": ("fwht.cuh", "dbbc29ed00b7", 45301760),
-    "k_dequant": ("ldlq.cuh", "6bffcb01b1c3", 26946304),
+    "k_ldlq_block": ("ldlq.cuh", "9204cd9090d5", 6490880),
+    "k_ldl_factor": ("ldl.cuh", "df9cc064a14e", 338944),
+    "k_ldl_rows": ("ldl.cuh", "df9cc064a14e", 4653824),
+    "k_dequant": ("ldlq.cuh", "9204cd9090d5", 27231744),
+    "k_row_grid": ("ldlq.cuh", "9204cd9090d5", 67338496),
+    "k_split_upper_transposed": ("gemm_tc.cuh", "bbd3187cebb4", 146050816),
+    "k_gemm_split_tc[ldl]": ("gemm_tc.cuh", "bbd3187cebb4", 28437248),
 }
 TRAFFIC_WORKLOAD = "attn7b"
 
