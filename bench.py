@@ -141,13 +141,14 @@ def kernel_work(cfg: LayerConfig):
 # unchanged and only for the workload it was captured on.
 KERNEL_TRAFFIC = {
     "k_syrk_tc": ("syrk_tc.cuh", "260ad4eebdfc", 71597824),
-    "k_ldlq_block": ("ldlq.cuh", "9204cd9090d5", 6490880),
+    "k_ldlq_block": ("ldlq.cuh", "449a391e49fc", 6490880),
     "k_ldl_factor": ("ldl.cuh", "df9cc064a14e", 338944),
     "k_ldl_rows": ("ldl.cuh", "df9cc064a14e", 4653824),
-    "k_dequant": ("ldlq.cuh", "9204cd9090d5", 27231744),
-    "k_row_grid": ("ldlq.cuh", "9204cd9090d5", 67338496),
-    "k_split_upper_transposed": ("gemm_tc.cuh", "bbd3187cebb4", 146050816),
-    "k_gemm_split_tc[ldl]": ("gemm_tc.cuh", "bbd3187cebb4", 28437248),
+    "k_dequant": ("ldlq.cuh", "449a391e49fc", 26102272),
+    "k_row_grid": ("ldlq.cuh", "449a391e49fc", 67615488),
+    "k_split_upper_transposed": ("gemm_tc.cuh", "92453856d596", 148098048),
+    "k_gemm_split_tc[ldl]": ("gemm_tc.cuh", "92453856d596", 28437248),
+    "k_fwht_cols": ("fwht.cuh", "94ad670265cc", 82387456),
 }
 TRAFFIC_WORKLOAD = "attn7b"
 

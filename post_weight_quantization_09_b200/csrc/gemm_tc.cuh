@@ -262,7 +262,8 @@ __device__ __forceinline__ void split3(float x, __nv_bfloat16& p0, __nv_bfloat16
 // the transposed, split copy of the LDL factor that LDLQ's trailing GEMM
 // reads as its K-major B operand; outf[j][i] = U[i][j] (same zeros), the
 // fp32 transposed copy the LDLQ block kernel reads.  32 x 32 tiles through
-// shared memory.
+// shared memory; source tiles below the diagonal are not read (all their
+// outputs are zero); each thread writes two adjacent outputs.  n even.
 __global__ void __launch_bounds__(256) k_split_upper_transposed(const float* __restrict__ U,
                                                                 int64_t ldu, int64_t n,
                                                                 __nv_bfloat16* __restrict__ out,
@@ -270,22 +271,30 @@ __global__ void __launch_bounds__(256) k_split_upper_transposed(const float* __r
   __shared__ float t[32][33];
   const int64_t bi = blockIdx.y, bj = blockIdx.x;   // source tile (rows bi, cols bj)
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (int r = ty; r < 32; r += 8) {
-    const int64_t i = bi * 32 + r, j = bj * 32 + tx;
-    t[r][tx] = (i < n && j < n && i < j) ? U[i * ldu + j] : 0.f;
+  const bool below = bi > bj;
+  if (!below) {
+    for (int r = ty; r < 32; r += 8) {
+      const int64_t i = bi * 32 + r, j = bj * 32 + tx;
+      t[r][tx] = (i < n && j < n && i < j) ? U[i * ldu + j] : 0.f;
+    }
   }
   __syncthreads();
   const int64_t pn = n * n;
-  for (int r = ty; r < 32; r += 8) {
-    const int64_t j = bj * 32 + r, i = bi * 32 + tx;  // out row j, col i
-    if (i < n && j < n) {
-      __nv_bfloat16 p0, p1, p2;
-      split3(t[tx][r], p0, p1, p2);
-      out[j * n + i] = p0;
-      out[pn + j * n + i] = p1;
-      out[2 * pn + j * n + i] = p2;
-      outf[j * n + i] = t[tx][r];
+  const int i2 = 2 * (tx & 15);
+  for (int rr = 2 * ty + (tx >> 4); rr < 32; rr += 16) {
+    const int64_t j = bj * 32 + rr, i = bi * 32 + i2;   // out row j, columns i, i + 1
+    if (j >= n || i >= n) continue;
+    const float a = below ? 0.f : t[i2][rr], b = below ? 0.f : t[i2 + 1][rr];
+    __nv_bfloat16 pa[3], pb[3];
+    split3(a, pa[0], pa[1], pa[2]);
+    split3(b, pb[0], pb[1], pb[2]);
+#pragma unroll
+    for (int p = 0; p < 3; ++p) {
+      __nv_bfloat162 v;
+      v.x = pa[p], v.y = pb[p];
+      *reinterpret_cast<__nv_bfloat162*>(out + p * pn + j * n + i) = v;
     }
+    *reinterpret_cast<float2*>(outf + j * n + i) = make_float2(a, b);
   }
 }
 

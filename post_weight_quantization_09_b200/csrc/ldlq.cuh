@@ -27,6 +27,7 @@ __global__ void __launch_bounds__(256) k_row_grid(const float* __restrict__ Wt, 
   float mn = INFINITY, mx = -INFINITY;
   bool fin = true;
   if ((n & 3) == 0) {
+#pragma unroll 8
     for (int64_t j = 4 * lane; j < n; j += 128) {
       const float4 v = *reinterpret_cast<const float4*>(w + j);
       mn = fminf(mn, fminf(fminf(v.x, v.y), fminf(v.z, v.w)));
@@ -345,25 +346,37 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
   }
 }
 
-// W~^[i][j] = lo[i] + s[i] * codes[i][j]
-__global__ void k_dequant(const uint8_t* __restrict__ codes, const float* __restrict__ lo,
-                          const float* __restrict__ sc, int64_t m, int64_t n, float* out) {
-  const int64_t total = m * n;
-  for (int64_t e = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) * 4; e < total;
-       e += (int64_t)gridDim.x * blockDim.x * 4) {
-    if (e + 3 < total && (n & 3) == 0) {
-      const int64_t i = e / n;
-      const uchar4 c = *reinterpret_cast<const uchar4*>(codes + e);
-      const float l = lo[i], s = sc[i];
-      float4 v;
-      v.x = fmaf(s, (float)c.x, l), v.y = fmaf(s, (float)c.y, l);
-      v.z = fmaf(s, (float)c.z, l), v.w = fmaf(s, (float)c.w, l);
-      *reinterpret_cast<float4*>(out + e) = v;
-    } else {
-      for (int64_t f = e; f < e + 4 && f < total; ++f) {
-        const int64_t i = f / n;
-        out[f] = fmaf(sc[i], (float)codes[f], lo[i]);
+// W~^[i][j] = lo[i] + s[i] * codes[i][j].  Rows i = blockIdx.y, + gridDim.y,
+// ...; with vec (n % 4 == 0, both arrays 16-byte aligned) thread t of CTA x
+// expands the 4-code groups 4 (1024 x + 256 q + t), q < 4 (coalesced 4-byte
+// loads and 16-byte stores across the CTA), else one code at a time.
+constexpr int DQ_THREADS = 256;
+__global__ void __launch_bounds__(DQ_THREADS) k_dequant(const uint8_t* __restrict__ codes,
+                                                        const float* __restrict__ lo,
+                                                        const float* __restrict__ sc, int64_t m,
+                                                        int64_t n, int vec, float* __restrict__ out) {
+  for (int64_t i = blockIdx.y; i < m; i += gridDim.y) {
+    const float l = lo[i], s = sc[i];
+    const uint8_t* c = codes + i * n;
+    float* o = out + i * n;
+    if (vec) {
+      for (int64_t j0 = 4 * (int64_t)blockIdx.x * 4 * DQ_THREADS; j0 < n;
+           j0 += 16 * (int64_t)gridDim.x * DQ_THREADS) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int64_t j = j0 + 4 * (q * DQ_THREADS + threadIdx.x);
+          if (j < n) {
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(c + j);
+            *reinterpret_cast<float4*>(o + j) =
+                make_float4(fmaf(s, (float)(w & 0xffu), l), fmaf(s, (float)((w >> 8) & 0xffu), l),
+                            fmaf(s, (float)((w >> 16) & 0xffu), l), fmaf(s, (float)(w >> 24), l));
+          }
+        }
       }
+    } else {
+      for (int64_t j = (int64_t)blockIdx.x * DQ_THREADS + threadIdx.x; j < n;
+           j += (int64_t)gridDim.x * DQ_THREADS)
+        o[j] = fmaf(s, (float)c[j], l);
     }
   }
 }

@@ -975,11 +975,14 @@ quip_status quip_dequantize(const uint8_t* codes, const float* lo, const float* 
                             int64_t n, float* W_hat_t, void* stream) {
   if (!codes || !lo || !scale || !W_hat_t) return QUIP_ERR_ARG;
   if (m <= 0 || n <= 0) return QUIP_ERR_SHAPE;
-  const int64_t total = m * n;
-  const unsigned grid = (unsigned)std::min<int64_t>((total / 4 + 255) / 256 + 1, 148 * 16);
+  const int vec = (n & 3) == 0 && (reinterpret_cast<uintptr_t>(codes) & 3) == 0 &&
+                  (reinterpret_cast<uintptr_t>(W_hat_t) & 15) == 0;
+  const int64_t per_cta = (vec ? 16 : 1) * (int64_t)DQ_THREADS;
+  const unsigned gx = (unsigned)std::min<int64_t>((n + per_cta - 1) / per_cta, 1024);
+  const unsigned gy = (unsigned)std::min<int64_t>(m, 65535);
   {
     LaunchScope ls("k_dequant", S(stream));
-    k_dequant<<<grid, 256, 0, S(stream)>>>(codes, lo, scale, m, n, W_hat_t);
+    k_dequant<<<dim3(gx, gy), DQ_THREADS, 0, S(stream)>>>(codes, lo, scale, m, n, vec, W_hat_t);
   }
   QCHECK(cudaGetLastError());
   return QUIP_OK;
