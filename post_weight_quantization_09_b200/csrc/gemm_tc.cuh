@@ -28,7 +28,7 @@
 namespace quip {
 namespace sgemm {
 
-// Tile N width BN: 256, or 64 for narrow outputs (more tiles, more CTAs).
+// Tile N width BN: 256, or 128 / 64 for narrow outputs (more tiles, more CTAs).
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;              // 16 KB
 template <int TN> __host__ __device__ constexpr int b_bytes() { return TN * BK * 2; }

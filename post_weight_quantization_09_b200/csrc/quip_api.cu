@@ -191,11 +191,25 @@ cudaError_t split_gemm_tn(const CUtensorMap& ta, const CUtensorMap& tb, sgemm::P
 
 cudaError_t split_gemm(const CUtensorMap& ta, const CUtensorMap& tb, sgemm::Params p,
                        cudaStream_t st, const char* name, int max_ctas = 0,
-                       const CUtensorMap* tb64 = nullptr) {
+                       const CUtensorMap* tb64 = nullptr, const CUtensorMap* tb128 = nullptr) {
   if (p.M <= 0 || p.N <= 0) return cudaSuccess;
-  const int tiles256 = ((p.M + sgemm::BM - 1) / sgemm::BM) * ((p.N + sgemm::BN - 1) / sgemm::BN);
-  if (tb64 && !p.upper_only && 2 * tiles256 < num_sms())
-    return split_gemm_tn<64>(ta, *tb64, p, st, name, max_ctas);
+  if (p.upper_only || (!tb64 && !tb128))
+    return split_gemm_tn<sgemm::BN>(ta, tb, p, st, name, max_ctas);
+  // Tile width by a cost model: waves of tiles x tile width (a tile's time
+  // grows with its width at a fixed K); 64-wide tiles count double, their
+  // MMAs being bound by the A operand's shared-memory reads.  Ties go to
+  // the wider tile.
+  const int cap = max_ctas > 0 ? std::min(max_ctas, num_sms()) : num_sms();
+  const int64_t tm = (p.M + sgemm::BM - 1) / sgemm::BM;
+  auto cost = [&](int tn) {
+    const int64_t tiles = tm * ((p.N + tn - 1) / tn);
+    return ((tiles + cap - 1) / cap) * tn * (tn == 64 ? 2 : 1);
+  };
+  int best = sgemm::BN;
+  if (tb128 && cost(128) < cost(best)) best = 128;
+  if (tb64 && cost(64) < cost(best)) best = 64;
+  if (best == 128) return split_gemm_tn<128>(ta, *tb128, p, st, name, max_ctas);
+  if (best == 64) return split_gemm_tn<64>(ta, *tb64, p, st, name, max_ctas);
   return split_gemm_tn<sgemm::BN>(ta, tb, p, st, name, max_ctas);
 }
 
@@ -833,7 +847,7 @@ struct LdlqRun {
   float qmax;
   uint8_t* codes;
   __nv_bfloat16* Es;
-  CUtensorMap ta, tb, tb64, tacc, tut, tband, tw;
+  CUtensorMap ta, tb, tb64, tb128, tacc, tut, tband, tw;
   cudaStream_t st;
 };
 
@@ -860,7 +874,7 @@ cudaError_t ldlq_range(const LdlqRun& r, int64_t a, int64_t b) {
   gp.a_piece_rows = (int)r.m, gp.a_k0 = (int)a;
   gp.b_piece_rows = (int)r.n, gp.b_row0 = (int)mid, gp.b_k0 = (int)a;
   gp.alpha = 1.f;
-  e = split_gemm(r.ta, r.tb, gp, r.st, "k_gemm_split_tc[ldlq]", 0, &r.tb64);
+  e = split_gemm(r.ta, r.tb, gp, r.st, "k_gemm_split_tc[ldlq]", 0, &r.tb64, &r.tb128);
   if (e != cudaSuccess) return e;
   return ldlq_range(r, mid, b);
 }
@@ -911,7 +925,8 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
   if (n > LDQ_BLK) {
     if (!make_tmap_bf16_2d(&r.ta, r.Es, (uint64_t)n, 3 * (uint64_t)m, (uint64_t)n * 2, 64, sgemm::BM) ||
         !make_tmap_bf16_2d(&r.tb, UTs, (uint64_t)n, 3 * (uint64_t)n, (uint64_t)n * 2, 64, sgemm::BN) ||
-        !make_tmap_bf16_2d(&r.tb64, UTs, (uint64_t)n, 3 * (uint64_t)n, (uint64_t)n * 2, 64, 64))
+        !make_tmap_bf16_2d(&r.tb64, UTs, (uint64_t)n, 3 * (uint64_t)n, (uint64_t)n * 2, 64, 64) ||
+        !make_tmap_bf16_2d(&r.tb128, UTs, (uint64_t)n, 3 * (uint64_t)n, (uint64_t)n * 2, 64, 128))
       return QUIP_ERR_CUDA;
   }
   static bool attr = false;
