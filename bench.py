@@ -514,6 +514,63 @@ def run_ours(args, cfg: LayerConfig):
         dist.destroy_process_group()
 
 
+def run_group(args, cfg: LayerConfig):
+    """G layers of cfg's shape reading the same input X (q / k / v of an
+    attention block, up / gate of an MLP): one Hessian, one transform of it
+    and one LDL for the group, LDLQ on the stacked rows.  value = G m n /
+    step time (quantized weights per second)."""
+    import torch
+    import post_weight_quantization_09_b200 as Q
+    from post_weight_quantization_09_b200 import _lib as L
+    world, rank, local = dist_setup()
+    if world > 1:
+        raise SystemExit("--group runs on one GPU")
+    torch.cuda.set_device(local)
+    lib = Q.load()
+    G = args.group
+    as_t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 \
+        else torch.from_numpy(a)
+    Ws, X = [], None
+    for g in range(G):
+        d = make_layer(rank_config(cfg, g))           # seed + g: G different weight matrices
+        Ws.append(as_t(d["W_bf16"] if cfg.dtype == "bf16" else d["W"]).cuda())
+        if X is None:
+            X = as_t(d["X_bf16"] if cfg.dtype == "bf16" else d["X"]).cuda()
+    q = Q.LayerGroupQuantizer(G, cfg.m, cfg.n, cfg.m_side, cfg.n_side, cfg.bits, cfg.block, cfg.damp,
+                              cfg.seed)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")   # 256 MB > L2
+    for _ in range(max(3, args.warmup)):
+        q.run(Ws, X)
+    torch.cuda.synchronize()
+    st = Q.quip_sync_status()
+    if st != L.QUIP_OK:
+        raise RuntimeError(f"device status after warm-up: {L.status_string(st)}")
+    step_ms = []
+    launches0 = lib.quip_kernel_launches()
+    with ClockSampler(local) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            q.run(Ws, X)
+            b.record(stream)
+            torch.cuda.synchronize()
+            step_ms.append(a.elapsed_time(b))
+    launches = (lib.quip_kernel_launches() - launches0) // max(1, args.steps)
+    ms = statistics.mean(step_ms)
+    desc = config_desc(cfg, args)
+    desc["workload"] = f"{G} layers sharing one input, each " + desc["workload"]
+    desc["group"] = G
+    line = {"metric": METRIC, "value": G * cfg.m * cfg.n / (ms * 1e-3), "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded Gaussian W / X with outliers, bf16; no weights or C4 in the box)",
+            "config": desc, "gpu_launches_per_step": launches, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -523,12 +580,17 @@ def main():
     ap.add_argument("--config", default="attn7b", choices=sorted(CONFIGS))
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--group", type=int, default=1,
+                    help="layers of the config's shape sharing one input (one Hessian and LDL)")
     args = ap.parse_args()
     cfg = CONFIGS[args.config]
     if args.impl == "reference":
         run_reference(args, cfg)
     else:
-        run_ours(args, cfg)
+        if args.group > 1:
+            run_group(args, cfg)
+        else:
+            run_ours(args, cfg)
 
 
 if __name__ == "__main__":

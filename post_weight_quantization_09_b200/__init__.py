@@ -21,7 +21,8 @@ from ._lib import QuipError, load, status_string  # noqa: F401
 __all__ = [
     "Transform", "quip_hessian_accumulate", "quip_hessian_finalize", "quip_incoherence_forward",
     "quip_incoherence_inverse", "quip_ldl", "quip_ldlq_quantize", "quip_dequantize",
-    "quip_workspace_size", "quip_sync_status", "quip_timing_begin", "quip_timing_end", "LayerQuantizer", "quantize_layer", "QuipError",
+    "quip_workspace_size", "quip_sync_status", "quip_timing_begin", "quip_timing_end", "LayerQuantizer",
+    "LayerGroupQuantizer", "quantize_layer", "QuipError",
     "KIND",
 ]
 
@@ -283,6 +284,66 @@ class LayerQuantizer:
         codes_out.copy_(r.codes, non_blocking=True)
         lo_out.copy_(r.lo, non_blocking=True)
         scale_out.copy_(r.scale, non_blocking=True)
+
+
+class LayerGroupQuantizer:
+    """Quantise G layers of the same shape that read the same input (the
+    q, k and v projections of an attention block; up and gate of an MLP):
+    the proxy Hessian H = X^T X / N, its incoherence transform and its LDL
+    are computed once, and LDLQ runs once on the G incoherent weight
+    matrices stacked by rows (rows are independent: each row's rounding
+    only involves its own entries and the shared factor).  All layers use
+    the same transform (U, V), as one seed draws it; ``run`` issues the whole
+    group on one stream through the C ABI.  Each layer's codes, grid and
+    dequantised weights are exactly those of ``LayerQuantizer`` on that layer
+    with the same X."""
+
+    def __init__(self, groups: int, m: int, n: int, m_side, n_side, bits: int, block: int,
+                 damp: float = 0.01, seed: int = 0, device: str = "cuda", stream=None):
+        if groups < 1:
+            raise ValueError("groups must be >= 1")
+        self.G, self.m, self.n = groups, m, n
+        self.bits, self.block, self.damp, self.seed = bits, block, damp, seed
+        self.stream = stream
+        dev = torch.device(device)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.H = torch.empty(n, n, **f32)
+        self.W_t = torch.empty(groups * m, n, **f32)
+        self.D = torch.empty(n, **f32)
+        self.codes = torch.empty(groups * m, n, dtype=torch.uint8, device=dev)
+        self.lo = torch.empty(groups * m, **f32)
+        self.scale = torch.empty(groups * m, **f32)
+        self.W_hat = torch.empty(groups * m, n, **f32)
+        self.tf = Transform(seed, m, n, m_side, n_side, stream)
+        ws = 0
+        for op, mm, blk in ((L.QUIP_OP_INCOHERENCE_FORWARD, m, 0), (L.QUIP_OP_INCOHERENCE_INVERSE, m, 0),
+                            (L.QUIP_OP_LDL, m, 0), (L.QUIP_OP_LDLQ, groups * m, block)):
+            ws = max(ws, quip_workspace_size(op, self.tf if op != L.QUIP_OP_LDLQ else None, mm, n, blk))
+        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+
+    def run(self, Ws, X: torch.Tensor, redraw_transform: bool = True) -> "LayerResult":
+        """Ws: G tensors m x n (or one G m x n tensor); X: N x n calibration
+        inputs shared by the layers.  Returns the stacked results (layer g in
+        rows [g m, (g + 1) m))."""
+        Ws = list(Ws.split(self.m, dim=0)) if isinstance(Ws, torch.Tensor) else list(Ws)
+        if len(Ws) != self.G:
+            raise ValueError(f"expected {self.G} weight matrices, got {len(Ws)}")
+        st, m = self.stream, self.m
+        if redraw_transform:
+            self.tf.draw(self.seed, st)
+        quip_hessian_accumulate(X, self.H, False, st)
+        quip_hessian_finalize(self.H, X.shape[0], self.damp, st)
+        for g, W in enumerate(Ws):
+            quip_incoherence_forward(self.tf, W, self.W_t[g * m:(g + 1) * m], self.H if g == 0 else None,
+                                     self.ws, st)
+        quip_ldl(self.H, self.D, self.ws, st)
+        quip_ldlq_quantize(self.W_t, self.H, self.bits, self.block, self.codes, self.lo, self.scale,
+                           self.ws, st)
+        quip_dequantize(self.codes, self.lo, self.scale, self.W_hat, st)
+        for g in range(self.G):
+            rows = self.W_hat[g * m:(g + 1) * m]
+            quip_incoherence_inverse(self.tf, rows, rows, self.ws, st)
+        return LayerResult(self.codes, self.lo, self.scale, self.W_hat)
 
 
 def quantize_layer(W: torch.Tensor, X: torch.Tensor, m_side, n_side, bits: int, block: int,

@@ -294,9 +294,10 @@ __device__ __forceinline__ void blk_solve(float* T, const float* Rp, const float
 //                  update, and column block J of this CTA's 32 next rows
 //                  (blk_solve).
 // CTA c (when c0 > 0) solves next rows c0 - 128 + 32 c .. + 31 of R12(p)
-// into Nx (128 x 128, row i = global row c0 - 128 + i).  CTA 0 writes R_pp
-// (Rd, 128 x 128, upper; lower zero), X_J (Xw, 4 x 32 x 32) and D (Dv[c0 +
-// k] = R_kk^2); the CTAs split the block's rows for its Ů in H.  Lin: the look-ahead buffer of panel p + 1 (rows
+// into Nx (128 x 128, row i = global row c0 - 128 + i).  The CTAs split the
+// stores of R_pp (Rd, 128 x 128, upper; lower zero) and X_J (Xw, 4 x 32 x
+// 32); CTA 0 writes D (Dv[c0 + k] = R_kk^2); the CTAs split the block's rows
+// for its Ů in H.  Lin: the look-ahead buffer of panel p + 1 (rows
 // [0, c0 + 128) x 128), or NULL.
 // Dynamic smem: (128 + 32) x LDL_LDA + 5 x 32 x LDL_LDX + 96 floats.
 __global__ void __launch_bounds__(LDL_FT, 1)
@@ -375,22 +376,25 @@ __global__ void __launch_bounds__(LDL_FT, 1)
   }
   if (has_next) blk_solve<32>(T, A, X, 0, tid, LDL_FT, all_sync);
 
-  if (blockIdx.x == 0) {
-    if (tid == 0 && bad) record_status(QUIP_ERR_NOT_PD);
-#pragma unroll
-    for (int e = tid; e < LDL_PB * 32; e += LDL_FT) {
+  {
+    // R_pp, X_J and D: every CTA holds the same factor, so the CTAs split
+    // the stores (CTA c: rows / blocks c, c + gridDim.x, ... of four)
+    if (blockIdx.x == 0 && tid == 0 && bad) record_status(QUIP_ERR_NOT_PD);
+    const int nc = gridDim.x;
+    for (int e = tid + LDL_FT * blockIdx.x; e < LDL_PB * 32; e += LDL_FT * nc) {
       const int i = e >> 5, j4 = (e & 31) * 4;
       const float4 v = *reinterpret_cast<const float4*>(A + i * LDL_LDA + j4);
       *reinterpret_cast<float4*>(Rd + i * LDL_PB + j4) =
           make_float4(j4 >= i ? v.x : 0.f, j4 + 1 >= i ? v.y : 0.f, j4 + 2 >= i ? v.z : 0.f,
                       j4 + 3 >= i ? v.w : 0.f);
     }
-    for (int e = tid; e < 4 * 32 * 32; e += LDL_FT)
+    for (int e = tid + LDL_FT * blockIdx.x; e < 4 * 32 * 32; e += LDL_FT * nc)
       Xw[e] = X[(e >> 10) * 32 * LDL_LDX + ((e >> 5) & 31) * LDL_LDX + (e & 31)];
-    for (int k = tid; k < w; k += LDL_FT) {
-      const float r = A[k * LDL_LDA + k];
-      Dv[c0 + k] = r * r;
-    }
+    if (blockIdx.x == 0)
+      for (int k = tid; k < w; k += LDL_FT) {
+        const float r = A[k * LDL_LDA + k];
+        Dv[c0 + k] = r * r;
+      }
   }
   {
     // this CTA's share of the block's Ů
