@@ -162,8 +162,11 @@ quip_status quip_hessian_finalize(float* H, int64_t n, int64_t N_total, float da
  * Incoherence pre-processing (QuIP, incoherence-processing section):
  *   W_t = U W V^T   (m x n fp32, row stride n), W: device m x n, row stride
  *                   ldw, dtype QUIP_BF16 or QUIP_F32; W and W_t must not overlap;
+ *                   skipped when W is NULL (then W_t, w_dtype and ldw are ignored);
  *   H   = V H V^T   in place (n x n fp32, full symmetric on entry and exit),
- *                   skipped when H is NULL.
+ *                   skipped when H is NULL.  W and H may not both be NULL.
+ * The two are independent: a caller may transform H first (the LDL needs
+ * only H~) and W later, e.g. while W is still being copied to the device.
  * ws: workspace for QUIP_OP_INCOHERENCE_FORWARD.
  */
 quip_status quip_incoherence_forward(const quip_transform* tf, const void* W, int w_dtype,

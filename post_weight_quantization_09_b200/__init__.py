@@ -144,14 +144,20 @@ def quip_hessian_finalize(H: torch.Tensor, N_total: int, damp: float, stream=Non
             "quip_hessian_finalize")
 
 
-def quip_incoherence_forward(tf: Transform, W: torch.Tensor, W_t: torch.Tensor,
+def quip_incoherence_forward(tf: Transform, W: Optional[torch.Tensor], W_t: Optional[torch.Tensor],
                              H: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
                              stream=None) -> None:
-    _cuda(W, "W"), _cuda(W_t, "W_t")
+    """W_t = U W V^T (skipped when W is None) and H = V H V^T in place
+    (skipped when H is None)."""
+    if W is not None:
+        _cuda(W, "W"), _cuda(W_t, "W_t")
+    ref = W if W is not None else H
     need = quip_workspace_size(L.QUIP_OP_INCOHERENCE_FORWARD, tf, tf.m, tf.n)
     if ws is None:
-        ws = _ws(need, W.device)
-    L.check(load().quip_incoherence_forward(tf.handle, _p(W), _dtype(W), W.stride(0), _p(W_t), _p(H),
+        ws = _ws(need, ref.device if ref is not None else torch.device("cuda"))
+    dt = _dtype(W) if W is not None else L.QUIP_F32
+    ldw = W.stride(0) if W is not None else tf.n
+    L.check(load().quip_incoherence_forward(tf.handle, _p(W), dt, ldw, _p(W_t), _p(H),
                                             _p(ws), 0 if ws is None else ws.numel(), _s(stream)),
             "quip_incoherence_forward")
 
@@ -253,16 +259,27 @@ class LayerQuantizer:
         """Draw (U, V) again from the seed on the device (part of a full pass)."""
         self.tf.draw(self.seed, self.stream)
 
-    def run(self, W: torch.Tensor, X: torch.Tensor, redraw_transform: bool = True) -> LayerResult:
+    def run(self, W: torch.Tensor, X: torch.Tensor, redraw_transform: bool = True,
+            w_ready: Optional[torch.cuda.Event] = None, after_ldlq=None) -> LayerResult:
+        """The whole layer on one stream.  H's transform and the LDL come
+        before W's transform (they do not need W): ``w_ready``, when given, is
+        waited for just before W is read, so a copy of W can overlap them.
+        ``after_ldlq`` (a callable) is invoked once codes and grid are final."""
         st = self.stream
+        stream = st if st is not None else torch.cuda.current_stream()
         if redraw_transform:
             self.new_transform()
         quip_hessian_accumulate(X, self.H, False, st)
         quip_hessian_finalize(self.H, X.shape[0], self.damp, st)
-        quip_incoherence_forward(self.tf, W, self.W_t, self.H, self.ws, st)
+        quip_incoherence_forward(self.tf, None, None, self.H, self.ws, st)
         quip_ldl(self.H, self.D, self.ws, st)
+        if w_ready is not None:
+            stream.wait_event(w_ready)
+        quip_incoherence_forward(self.tf, W, self.W_t, None, self.ws, st)
         quip_ldlq_quantize(self.W_t, self.H, self.bits, self.block, self.codes, self.lo, self.scale,
                            self.ws, st)
+        if after_ldlq is not None:
+            after_ldlq()
         quip_dequantize(self.codes, self.lo, self.scale, self.W_hat, st)
         quip_incoherence_inverse(self.tf, self.W_hat, self.W_hat, self.ws, st)
         return LayerResult(self.codes, self.lo, self.scale, self.W_hat)
@@ -271,19 +288,36 @@ class LayerQuantizer:
                  lo_out: torch.Tensor, scale_out: torch.Tensor) -> None:
         """Host in, host out: copy W and X (pinned host tensors) to the device,
         run the layer, copy codes / lo / scale back into the pinned outputs.
-        Everything is enqueued on the current stream; synchronise to read."""
+        X is copied on the layer's stream; W on a second stream, overlapping
+        the Hessian, its transform and the LDL; the results go back on that
+        second stream while the dequantisation and inverse transform run.
+        Everything is joined into the layer's stream; synchronise it to read."""
         if getattr(self, "_W_dev", None) is None or self._W_dev.shape != W_host.shape \
                 or self._W_dev.dtype != W_host.dtype:
             self._W_dev = torch.empty_like(W_host, device="cuda")
         if getattr(self, "_X_dev", None) is None or self._X_dev.shape != X_host.shape \
                 or self._X_dev.dtype != X_host.dtype:
             self._X_dev = torch.empty_like(X_host, device="cuda")
-        self._W_dev.copy_(W_host, non_blocking=True)
-        self._X_dev.copy_(X_host, non_blocking=True)
-        r = self.run(self._W_dev, self._X_dev)
-        codes_out.copy_(r.codes, non_blocking=True)
-        lo_out.copy_(r.lo, non_blocking=True)
-        scale_out.copy_(r.scale, non_blocking=True)
+        if getattr(self, "_copy", None) is None:
+            self._copy = torch.cuda.Stream()
+        main = self.stream if self.stream is not None else torch.cuda.current_stream()
+        cp = self._copy
+        cp.wait_stream(main)                       # the previous call is done with _W_dev
+        with torch.cuda.stream(cp):
+            self._W_dev.copy_(W_host, non_blocking=True)
+        w_ready = cp.record_event()
+        with torch.cuda.stream(main):
+            self._X_dev.copy_(X_host, non_blocking=True)
+
+        def results_out():
+            cp.wait_stream(main)
+            with torch.cuda.stream(cp):
+                codes_out.copy_(self.codes, non_blocking=True)
+                lo_out.copy_(self.lo, non_blocking=True)
+                scale_out.copy_(self.scale, non_blocking=True)
+
+        self.run(self._W_dev, self._X_dev, w_ready=w_ready, after_ldlq=results_out)
+        main.wait_stream(cp)
 
 
 class LayerGroupQuantizer:

@@ -86,7 +86,7 @@ __device__ __forceinline__ void nb_arrive(int id, int count) {
 //      takes cur = the group's accumulated values + carry (the previous
 //      group's feedback, in registers);
 //   2. rounds column by column, feeding each error to the group's later
-//      columns and, into carry, to the next group;
+//      columns, then forms the group's feedback to the next group (carry);
 //   3. hands the 16 errors and codes to the helpers (shared slot g % 2).
 // The helpers stage the codes and the errors' three bf16 pieces (the
 // trailing GEMMs' A operand; written out with coalesced stores after the
@@ -284,10 +284,19 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
     float sd[15];
 #pragma unroll
     for (int t = 0; t < 15; ++t) sd[t] = band[(16 * g + t) * 32 + t + 1];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) carry[j] = 0.f;
+    // Software-pipelined: column t's error reaches column t + 1 at once (the
+    // super-diagonal), and the group's later columns one step later, after
+    // column t + 1 has been rounded, from a band row loaded a step ahead.
+    float bprev[16], eprev = 0.f;
 #pragma unroll
     for (int t = 0; t < 16; ++t) {
+      float bcur[16];
+      const float* ur = band + (16 * g + t) * 32;      // band row 16 g + t
+#pragma unroll
+      for (int q4 = ((t + 2) >> 2) << 2; q4 < 16; q4 += 4) {
+        const float4 u = *reinterpret_cast<const float4*>(ur + q4);
+        bcur[q4] = u.x, bcur[q4 + 1] = u.y, bcur[q4 + 2] = u.z, bcur[q4 + 3] = u.w;
+      }
       const float z = (cur[t] - l) * inv;
       const float zr = fminf(fmaxf(z, 0.f), qmax) + kRound;
       const float cq = zr - kRound;
@@ -295,23 +304,28 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
       e[t] = err;
       if (t < 15) cur[t + 1] = fmaf(err, sd[t], cur[t + 1]);
       cw[t >> 2] |= (__float_as_uint(zr) & 0xffu) << (8 * (t & 3));
-      // band row 16 g + t: this group's later columns, then the next group's
-      const float* ur = band + (16 * g + t) * 32;
+      // column t - 1's error into columns t + 1 ..
 #pragma unroll
-      for (int q4 = ((t + 2) >> 2) << 2; q4 < 16; q4 += 4) {
-        const float4 u = *reinterpret_cast<const float4*>(ur + q4);
-        if (q4 + 0 > t + 1) cur[q4 + 0] = fmaf(err, u.x, cur[q4 + 0]);
-        if (q4 + 1 > t + 1) cur[q4 + 1] = fmaf(err, u.y, cur[q4 + 1]);
-        if (q4 + 2 > t + 1) cur[q4 + 2] = fmaf(err, u.z, cur[q4 + 2]);
-        if (q4 + 3 > t + 1) cur[q4 + 3] = fmaf(err, u.w, cur[q4 + 3]);
-      }
+      for (int j = t + 1; j < 16; ++j)
+        if (t >= 1) cur[j] = fmaf(eprev, bprev[j], cur[j]);
+      eprev = err;
+#pragma unroll
+      for (int j = t + 2; j < 16; ++j) bprev[j] = bcur[j];
+    }
+    // the group's feedback to the next group (off the rounding chain; every
+    // carry element sums its terms in column order, as the chain would)
+#pragma unroll
+    for (int j = 0; j < 16; ++j) carry[j] = 0.f;
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      const float* ur = band + (16 * g + t) * 32 + 16;
 #pragma unroll
       for (int q4 = 0; q4 < 16; q4 += 4) {
-        const float4 u = *reinterpret_cast<const float4*>(ur + 16 + q4);
-        carry[q4 + 0] = fmaf(err, u.x, carry[q4 + 0]);
-        carry[q4 + 1] = fmaf(err, u.y, carry[q4 + 1]);
-        carry[q4 + 2] = fmaf(err, u.z, carry[q4 + 2]);
-        carry[q4 + 3] = fmaf(err, u.w, carry[q4 + 3]);
+        const float4 u = *reinterpret_cast<const float4*>(ur + q4);
+        carry[q4 + 0] = fmaf(e[t], u.x, carry[q4 + 0]);
+        carry[q4 + 1] = fmaf(e[t], u.y, carry[q4 + 1]);
+        carry[q4 + 2] = fmaf(e[t], u.z, carry[q4 + 2]);
+        carry[q4 + 3] = fmaf(e[t], u.w, carry[q4 + 3]);
       }
     }
     // hand the errors and codes to the helpers

@@ -698,14 +698,16 @@ static quip_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 quip_status quip_incoherence_forward(const quip_transform* tf, const void* W, int w_dtype,
                                      int64_t ldw, float* W_t, float* H, void* ws, size_t ws_bytes,
                                      void* stream) {
-  if (!tf || !W || !W_t) return QUIP_ERR_ARG;
-  if (w_dtype != QUIP_F32 && w_dtype != QUIP_BF16) return QUIP_ERR_ARG;
+  if (!tf || (!W && !H) || (W && !W_t)) return QUIP_ERR_ARG;
   const int64_t m = tf->m, n = tf->n;
-  if (ldw < n) return QUIP_ERR_SHAPE;
   const SideData &U = tf->side[0], &V = tf->side[1];
-  if (V.kind == QUIP_T_HADAMARD && n >= 16) {   // vector loads in the row kernel
-    const size_t esz = w_dtype == QUIP_BF16 ? 2 : 4;
-    if ((reinterpret_cast<uintptr_t>(W) % 16) || ((ldw * esz) % 16)) return QUIP_ERR_ARG;
+  if (W) {
+    if (w_dtype != QUIP_F32 && w_dtype != QUIP_BF16) return QUIP_ERR_ARG;
+    if (ldw < n) return QUIP_ERR_SHAPE;
+    if (V.kind == QUIP_T_HADAMARD && n >= 16) {   // vector loads in the row kernel
+      const size_t esz = w_dtype == QUIP_BF16 ? 2 : 4;
+      if ((reinterpret_cast<uintptr_t>(W) % 16) || ((ldw * esz) % 16)) return QUIP_ERR_ARG;
+    }
   }
   size_t need = 0;
   quip_status s = quip_workspace_size(QUIP_OP_INCOHERENCE_FORWARD, tf, m, n, 0, &need);
@@ -713,11 +715,13 @@ quip_status quip_incoherence_forward(const quip_transform* tf, const void* W, in
   if ((s = check_ws(ws, ws_bytes, need)) != QUIP_OK) return s;
   cudaStream_t st = S(stream);
   float* tmp = static_cast<float*>(ws);
-  if (w_dtype == QUIP_BF16)
-    QCHECK(side_rows<__nv_bfloat16>(V, false, static_cast<const __nv_bfloat16*>(W), ldw, W_t, m, tmp, st));
-  else
-    QCHECK(side_rows<float>(V, false, static_cast<const float*>(W), ldw, W_t, m, tmp, st));
-  QCHECK(side_cols(U, false, W_t, n, tmp, st));
+  if (W) {
+    if (w_dtype == QUIP_BF16)
+      QCHECK(side_rows<__nv_bfloat16>(V, false, static_cast<const __nv_bfloat16*>(W), ldw, W_t, m, tmp, st));
+    else
+      QCHECK(side_rows<float>(V, false, static_cast<const float*>(W), ldw, W_t, m, tmp, st));
+    QCHECK(side_cols(U, false, W_t, n, tmp, st));
+  }
   if (H) {
     if (V.kind == QUIP_T_KRONECKER) {                           // fp64 sums, see gemm_simt.cuh
       QCHECK((kron_rows<float, double>(H, n, H, n, V, false, tmp, st)));   // H V^T

@@ -312,3 +312,38 @@ def test_tiny_config_pipeline():
     assert np.abs(host(r.W_hat) - W_hat_ref).max() <= 1e-4 * s.max()
     bad, not_near = ldlq_trajectory_check(C, P.Wt, P.Uf, lo, s, cfg.bits, tau=1e-3)
     assert not_near == 0.0
+
+
+def test_incoherence_forward_h_only_then_w_only_equals_joint():
+    m, n = 64, 256
+    tf = Q.Transform(77, m, n, Side("hadamard"), Side("kronecker", 16, 16))
+    d = random_layer(m, n, 512, seed=5)
+    W = dev(d["W"])
+    H0 = dev(d["X"].T.astype(np.float64) @ d["X"] / 512.0)
+    Wt1, H1 = torch.empty(m, n, device="cuda"), H0.clone()
+    Q.quip_incoherence_forward(tf, W, Wt1, H1)
+    Wt2, H2 = torch.empty(m, n, device="cuda"), H0.clone()
+    Q.quip_incoherence_forward(tf, None, None, H2)
+    Q.quip_incoherence_forward(tf, W, Wt2, None)
+    assert torch.equal(Wt1, Wt2) and torch.equal(H1, H2)
+    with pytest.raises(Q.QuipError):
+        Q.quip_incoherence_forward(tf, None, None, None)
+
+
+def test_run_host_equals_device_run():
+    cfg = CONFIGS["tiny"]
+    d = make_layer(cfg)
+    q = Q.LayerQuantizer(cfg.m, cfg.n, cfg.m_side, cfg.n_side, cfg.bits, cfg.block, cfg.damp, cfg.seed)
+    r = q.run(dev(d["W"]), dev(d["X"]))
+    codes, lo, sc = r.codes.cpu(), r.lo.cpu(), r.scale.cpu()
+    q2 = Q.LayerQuantizer(cfg.m, cfg.n, cfg.m_side, cfg.n_side, cfg.bits, cfg.block, cfg.damp, cfg.seed)
+    Wh = torch.from_numpy(d["W"]).pin_memory()
+    Xh = torch.from_numpy(d["X"]).pin_memory()
+    co = torch.empty(cfg.m, cfg.n, dtype=torch.uint8).pin_memory()
+    lo_h = torch.empty(cfg.m).pin_memory()
+    sc_h = torch.empty(cfg.m).pin_memory()
+    for _ in range(2):                                 # twice: the buffers are reused
+        co.zero_(), lo_h.zero_(), sc_h.zero_()
+        q2.run_host(Wh, Xh, co, lo_h, sc_h)
+        torch.cuda.current_stream().synchronize()
+        assert torch.equal(co, codes) and torch.equal(lo_h, lo) and torch.equal(sc_h, sc)
