@@ -232,6 +232,8 @@ class LayerQuantizer:
     """Buffers and transform for quantising one m x n layer; ``run`` issues the
     whole pipeline on one stream through the C ABI."""
 
+    X_CHUNKS = 4            # token chunks of X in run_host (copy / Hessian overlap)
+
     def __init__(self, m: int, n: int, m_side, n_side, bits: int, block: int, damp: float = 0.01,
                  seed: int = 0, device: str = "cuda", stream=None):
         self.m, self.n, self.bits, self.block, self.damp, self.seed = m, n, bits, block, damp, seed
@@ -260,16 +262,24 @@ class LayerQuantizer:
         self.tf.draw(self.seed, self.stream)
 
     def run(self, W: torch.Tensor, X: torch.Tensor, redraw_transform: bool = True,
-            w_ready: Optional[torch.cuda.Event] = None, after_ldlq=None) -> LayerResult:
+            w_ready: Optional[torch.cuda.Event] = None, after_ldlq=None,
+            x_ready=None) -> LayerResult:
         """The whole layer on one stream.  H's transform and the LDL come
         before W's transform (they do not need W): ``w_ready``, when given, is
         waited for just before W is read, so a copy of W can overlap them.
+        ``x_ready``, when given, is a list of (first row, end row, event): the
+        Hessian accumulates each token chunk of X once its event completes.
         ``after_ldlq`` (a callable) is invoked once codes and grid are final."""
         st = self.stream
         stream = st if st is not None else torch.cuda.current_stream()
         if redraw_transform:
             self.new_transform()
-        quip_hessian_accumulate(X, self.H, False, st)
+        if x_ready:
+            for i, (a, b, ev) in enumerate(x_ready):
+                stream.wait_event(ev)
+                quip_hessian_accumulate(X[a:b], self.H, i > 0, st)
+        else:
+            quip_hessian_accumulate(X, self.H, False, st)
         quip_hessian_finalize(self.H, X.shape[0], self.damp, st)
         quip_incoherence_forward(self.tf, None, None, self.H, self.ws, st)
         quip_ldl(self.H, self.D, self.ws, st)
@@ -288,9 +298,10 @@ class LayerQuantizer:
                  lo_out: torch.Tensor, scale_out: torch.Tensor) -> None:
         """Host in, host out: copy W and X (pinned host tensors) to the device,
         run the layer, copy codes / lo / scale back into the pinned outputs.
-        X is copied on the layer's stream; W on a second stream, overlapping
+        Copies run on a second stream: X in X_CHUNKS token chunks, each
+        accumulated into the Hessian as soon as it lands, then W, overlapping
         the Hessian, its transform and the LDL; the results go back on that
-        second stream while the dequantisation and inverse transform run.
+        stream while the dequantisation and inverse transform run.
         Everything is joined into the layer's stream; synchronise it to read."""
         if getattr(self, "_W_dev", None) is None or self._W_dev.shape != W_host.shape \
                 or self._W_dev.dtype != W_host.dtype:
@@ -302,12 +313,17 @@ class LayerQuantizer:
             self._copy = torch.cuda.Stream()
         main = self.stream if self.stream is not None else torch.cuda.current_stream()
         cp = self._copy
-        cp.wait_stream(main)                       # the previous call is done with _W_dev
+        cp.wait_stream(main)                       # the previous call is done with the buffers
+        N = X_host.shape[0]
+        step = max(1, -(-N // self.X_CHUNKS))
+        x_ready = []
         with torch.cuda.stream(cp):
+            for a in range(0, N, step):
+                b = min(N, a + step)
+                self._X_dev[a:b].copy_(X_host[a:b], non_blocking=True)
+                x_ready.append((a, b, cp.record_event()))
             self._W_dev.copy_(W_host, non_blocking=True)
         w_ready = cp.record_event()
-        with torch.cuda.stream(main):
-            self._X_dev.copy_(X_host, non_blocking=True)
 
         def results_out():
             cp.wait_stream(main)
@@ -316,7 +332,7 @@ class LayerQuantizer:
                 lo_out.copy_(self.lo, non_blocking=True)
                 scale_out.copy_(self.scale, non_blocking=True)
 
-        self.run(self._W_dev, self._X_dev, w_ready=w_ready, after_ldlq=results_out)
+        self.run(self._W_dev, self._X_dev, w_ready=w_ready, after_ldlq=results_out, x_ready=x_ready)
         main.wait_stream(cp)
 
 
