@@ -37,7 +37,12 @@ Readings where the pages are silent (each one is listed in the design doc):
     matrix with the sign of diag(R) folded into Q);
   * the random signs and Gaussians come from SplitMix64, counter-based (see
     ``splitmix64``); the CUDA library implements the same published
-    generator independently.
+    generator independently;
+  * the random permutation within the fast orthogonal multiplication (QuIP,
+    Experiments, "Further Ablation", Table 5; the algorithm box that placed
+    it was lost): optional per side, applied to the coordinates before the
+    structured factor, S = T P with (P x)_r = x_{pi[r]}; pi sorts the draws
+    of the side's permutation stream (``random_permutation``).
 
 Pinned by tests/test_oracle_*.py (CPU).  Functions with no pin: none.
 """
@@ -55,7 +60,7 @@ __all__ = [
     "incoherence_forward", "incoherence_inverse", "incoherence_rows", "incoherence_hessian", "udu", "row_grid", "quantize",
     "ldlq", "ldlq_blocked", "nearest", "optq", "dequantize", "proxy_loss", "Pipeline",
     "run_pipeline", "STREAM_M_SIGNS", "STREAM_N_SIGNS", "STREAM_M_A", "STREAM_M_B",
-    "STREAM_N_A", "STREAM_N_B",
+    "STREAM_N_A", "STREAM_N_B", "STREAM_M_PERM", "STREAM_N_PERM", "random_permutation",
 ]
 
 # ----------------------------------------------------------------------------
@@ -96,6 +101,7 @@ _M2 = np.uint64(0x94D049BB133111EB)
 
 STREAM_M_SIGNS, STREAM_N_SIGNS = 0, 1
 STREAM_M_A, STREAM_M_B, STREAM_N_A, STREAM_N_B = 2, 3, 4, 5
+STREAM_M_PERM, STREAM_N_PERM = 6, 7
 
 
 def splitmix64(seed: int, stream: int, index: np.ndarray) -> np.ndarray:
@@ -143,6 +149,17 @@ def haar_orthogonal(G: np.ndarray) -> np.ndarray:
     return Q * d[None, :]
 
 
+def random_permutation(seed: int, stream: int, n: int) -> np.ndarray:
+    """pi = the indices that sort the stream's first n draws (ascending).
+
+    A uniformly random permutation: the draws are distinct (the SplitMix64
+    finaliser is a bijection of 64-bit words), so every order is equally
+    likely.  (P x)_r = x_{pi[r]}.
+    """
+    keys = splitmix64(seed, stream, np.arange(n, dtype=np.uint64))
+    return np.argsort(keys, kind="stable")
+
+
 def sylvester_hadamard(n: int) -> np.ndarray:
     """H_1 = [1], H_2k = [[H_k, H_k], [H_k, -H_k]] (Sylvester, natural order)."""
     if n < 1 or n & (n - 1):
@@ -168,17 +185,21 @@ def hadamard_row(n: int, i: int) -> np.ndarray:
 class SideTransform:
     """One random orthogonal matrix S (m-side U or n-side V).
 
-    kind 'hadamard': S = H_d diag(s) / sqrt(d)          ([QuIP#] abstract)
-    kind 'kronecker': S = A (x) B, A p x p, B q x q     ([QuIP] Introduction)
-    kind 'identity':  S = I
+    kind 'hadamard': T = H_d diag(s) / sqrt(d)          ([QuIP#] abstract)
+    kind 'kronecker': T = A (x) B, A p x p, B q x q     ([QuIP] Introduction)
+    kind 'identity':  T = I
+    S = T P when perm is given ((P x)_r = x_{perm[r]}: the random permutation
+    within the fast orthogonal multiplication, [QuIP] Experiments, "Further
+    Ablation" / Table 5), else S = T.
     """
     kind: str
     dim: int
     signs: Optional[np.ndarray] = None
     A: Optional[np.ndarray] = None
     B: Optional[np.ndarray] = None
+    perm: Optional[np.ndarray] = None
 
-    def matrix(self) -> np.ndarray:
+    def _structured(self) -> np.ndarray:
         d = self.dim
         if self.kind == "identity":
             return np.eye(d)
@@ -186,32 +207,48 @@ class SideTransform:
             return sylvester_hadamard(d) * self.signs[None, :] / math.sqrt(d)
         return np.kron(self.A, self.B)
 
+    def perm_matrix(self) -> np.ndarray:
+        """P with P[r, perm[r]] = 1 (the identity without a permutation)."""
+        P = np.zeros((self.dim, self.dim))
+        p = self.perm if self.perm is not None else np.arange(self.dim)
+        P[np.arange(self.dim), p] = 1.0
+        return P
+
+    def matrix(self) -> np.ndarray:
+        T = self._structured()
+        return T if self.perm is None else T @ self.perm_matrix()
+
     def row(self, i: int) -> np.ndarray:
         d = self.dim
         if self.kind == "identity":
             r = np.zeros(d)
             r[i] = 1.0
-            return r
-        if self.kind == "hadamard":
-            return hadamard_row(d, i) * self.signs / math.sqrt(d)
-        q = self.B.shape[0]
-        return np.kron(self.A[i // q], self.B[i % q])
+        elif self.kind == "hadamard":
+            r = hadamard_row(d, i) * self.signs / math.sqrt(d)
+        else:
+            q = self.B.shape[0]
+            r = np.kron(self.A[i // q], self.B[i % q])
+        return r if self.perm is None else r @ self.perm_matrix()
 
 
-def make_side(seed: int, side: str, kind: str, dim: int, p: int = 0, q: int = 0) -> SideTransform:
+def make_side(seed: int, side: str, kind: str, dim: int, p: int = 0, q: int = 0,
+              permute: bool = False) -> SideTransform:
     """Draw the transform for side 'm' (rows of W) or 'n' (columns of W)."""
+    perm = None
+    if permute:
+        perm = random_permutation(seed, STREAM_M_PERM if side == "m" else STREAM_N_PERM, dim)
     if kind == "identity":
-        return SideTransform("identity", dim)
+        return SideTransform("identity", dim, perm=perm)
     if kind == "hadamard":
         st = STREAM_M_SIGNS if side == "m" else STREAM_N_SIGNS
-        return SideTransform("hadamard", dim, signs=random_signs(seed, st, dim))
+        return SideTransform("hadamard", dim, signs=random_signs(seed, st, dim), perm=perm)
     if kind == "kronecker":
         if p * q != dim:
             raise ValueError("Kronecker factors must multiply to the dimension")
         sa, sb = (STREAM_M_A, STREAM_M_B) if side == "m" else (STREAM_N_A, STREAM_N_B)
         A = haar_orthogonal(gaussian_matrix(seed, sa, p))
         B = haar_orthogonal(gaussian_matrix(seed, sb, q))
-        return SideTransform("kronecker", dim, A=A, B=B)
+        return SideTransform("kronecker", dim, A=A, B=B, perm=perm)
     raise ValueError(kind)
 
 
@@ -421,8 +458,8 @@ def run_pipeline(W: np.ndarray, X: np.ndarray, seed: int, m_side, n_side, bits: 
     W = np.asarray(W, dtype=np.float64)
     m, n = W.shape
     H = damp(hessian(X), alpha)
-    U = make_side(seed, "m", m_side.kind, m, m_side.p, m_side.q)
-    V = make_side(seed, "n", n_side.kind, n, n_side.p, n_side.q)
+    U = make_side(seed, "m", m_side.kind, m, m_side.p, m_side.q, getattr(m_side, "permute", False))
+    V = make_side(seed, "n", n_side.kind, n, n_side.p, n_side.q, getattr(n_side, "permute", False))
     Wt, Ht = incoherence_forward(W, H, U, V)
     Uf, D = udu(Ht)
     lo, s = row_grid(Wt, bits)

@@ -38,11 +38,13 @@ class Side:
     """Incoherence transform requested for one side of W.
 
     kind: 'hadamard' (dimension a power of two), 'kronecker' (p*q == dim) or
-    'identity'.
+    'identity'; permute: a random permutation of the coordinates is applied
+    before the structured transform.
     """
     kind: str
     p: int = 0
     q: int = 0
+    permute: bool = False
 
 
 @dataclass(frozen=True)

@@ -122,3 +122,24 @@ def test_planted_sign_placement_is_caught(monkeypatch):
     monkeypatch.setitem(Q.__dict__, "_matrix_orig", Q.SideTransform.matrix)
     monkeypatch.setattr(Q.SideTransform, "matrix", _signs_on_output)
     assert _fails([P.test_hadamard_sign_placement_hand_example])
+
+
+def _perm_matrix_transposed(self):
+    return Q.__dict__["_perm_matrix_orig"](self).T             # planted: P^T (pi^-1) for P
+
+
+def _permutation_descending(seed, stream, n):
+    keys = Q.splitmix64(seed, stream, np.arange(n, dtype=np.uint64))
+    return np.argsort(keys, kind="stable")[::-1]                # planted: descending order
+
+
+def test_planted_permutation_direction_is_caught(monkeypatch):
+    monkeypatch.setitem(Q.__dict__, "_perm_matrix_orig", Q.SideTransform.perm_matrix)
+    monkeypatch.setattr(Q.SideTransform, "perm_matrix", _perm_matrix_transposed)
+    assert _fails([P.test_permutation_only_side_is_indexing])
+
+
+def test_planted_permutation_order_is_caught(monkeypatch):
+    monkeypatch.setattr(Q, "random_permutation", _permutation_descending)
+    monkeypatch.setattr(O, "random_permutation", _permutation_descending)
+    assert _fails([P.test_random_permutation_sorts_its_draws_brute_force])

@@ -366,3 +366,55 @@ def test_synth_recipe():
     d2 = random_layer(5, 7, 11, seed=3, dtype="bf16")
     # bf16 storage: low 16 bits of every float32 are zero
     assert np.all((d2["W"].view(np.uint32) & 0xFFFF) == 0)
+
+
+# ---------------------------------------------------------------- random permutation (QuIP, Table 5)
+
+
+def test_random_permutation_sorts_its_draws_brute_force():
+    # tiny case by hand: pi must list the indices of the draws in increasing order
+    for seed, n in ((0, 5), (9, 8)):
+        keys = [int(k) for k in O.splitmix64(seed, O.STREAM_N_PERM, np.arange(n, dtype=np.uint64))]
+        pi = O.random_permutation(seed, O.STREAM_N_PERM, n)
+        assert sorted(pi.tolist()) == list(range(n))
+        assert all(keys[pi[r]] < keys[pi[r + 1]] for r in range(n - 1))
+        # brute force: the order of the draws, found by repeatedly taking the smallest
+        rest, order = list(range(n)), []
+        while rest:
+            i = min(rest, key=lambda j: keys[j])
+            order.append(i)
+            rest.remove(i)
+        assert pi.tolist() == order
+
+
+def test_permutation_only_side_is_indexing():
+    # identity structure with a permutation: W~ = P_m W P_n^T, i.e. W~[r, c] = W[pi_m[r], pi_n[c]],
+    # and H~[a, b] = H[pi_n[a], pi_n[b]]; the inverse indexes back
+    rng = np.random.default_rng(21)
+    W = rng.standard_normal((6, 8))
+    H = _spd(8, 4)
+    U = O.make_side(5, "m", "identity", 6, permute=True)
+    V = O.make_side(5, "n", "identity", 8, permute=True)
+    pm, pn = U.perm, V.perm
+    assert pm.tolist() != list(range(6)) and pn.tolist() != list(range(8))
+    Wt, Ht = O.incoherence_forward(W, H, U, V)
+    np.testing.assert_array_equal(Wt, W[pm][:, pn])
+    np.testing.assert_allclose(Ht, H[pn][:, pn], atol=0)
+    np.testing.assert_allclose(O.incoherence_inverse(Wt, U, V), W, atol=0)
+
+
+@pytest.mark.parametrize("kind,dim,p,q", [("hadamard", 32, 0, 0), ("kronecker", 12, 3, 4)])
+def test_permuted_side_orthogonal_rows_and_proxy(kind, dim, p, q):
+    S = O.make_side(3, "n", kind, dim, p, q, permute=True)
+    T = O.make_side(3, "n", kind, dim, p, q)
+    M = S.matrix()
+    np.testing.assert_allclose(M @ M.T, np.eye(dim), atol=1e-12)
+    # S = T P: column pi[r] of S is column r of T
+    np.testing.assert_allclose(M[:, S.perm], T.matrix(), atol=1e-15)
+    for i in (0, dim - 1):
+        np.testing.assert_allclose(S.row(i), M[i], atol=1e-15)
+    rng = np.random.default_rng(8)
+    W = rng.standard_normal((5, dim))
+    H = _spd(dim, 9)
+    Wt, Ht = O.incoherence_forward(W, H, O.make_side(0, "m", "identity", 5), S)
+    assert np.trace(Wt @ Ht @ Wt.T) == pytest.approx(np.trace(W @ H @ W.T), rel=1e-12)
