@@ -342,7 +342,8 @@ def run_reference(args, cfg: LayerConfig):
 
 
 def config_desc(cfg: LayerConfig, args):
-    side = lambda s: s.kind if s.kind != "kronecker" else f"kronecker {s.p}x{s.q}"
+    side = lambda s: (s.kind if s.kind != "kronecker" else f"kronecker {s.p}x{s.q}") + \
+        (" with random permutation" if getattr(s, "permute", False) else "")
     return {
         "workload": f"{cfg.name}: W {cfg.m}x{cfg.n} {cfg.dtype}, X {cfg.N}x{cfg.n} {cfg.dtype}, "
                     f"U {side(cfg.m_side)}, V {side(cfg.n_side)}, LDLQ block {cfg.block}, {cfg.bits}-bit",
@@ -582,8 +583,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--group", type=int, default=1,
                     help="layers of the config's shape sharing one input (one Hessian and LDL)")
+    ap.add_argument("--permute", action="store_true",
+                    help="random permutation within both sides' orthogonal transforms")
     args = ap.parse_args()
     cfg = CONFIGS[args.config]
+    if args.permute:
+        from dataclasses import replace
+        cfg = replace(cfg, m_side=replace(cfg.m_side, permute=True),
+                      n_side=replace(cfg.n_side, permute=True))
     if args.impl == "reference":
         run_reference(args, cfg)
     else:

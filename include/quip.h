@@ -70,6 +70,12 @@ typedef enum {
                             1 <= p, q <= 256                                     */
 } quip_tkind;
 
+/* Flag OR'ed into a side's kind: a random permutation of the coordinates
+ * before the structured factor T, S = T P with (P x)_r = x_{pi[r]} (QuIP,
+ * Experiments, "Further Ablation" / Table 5: the random permutation step
+ * within the fast orthogonal multiplication).  d <= 65536. */
+#define QUIP_T_PERMUTE 0x100
+
 /* Operations whose workspace quip_workspace_size() reports. */
 typedef enum {
   QUIP_OP_INCOHERENCE_FORWARD = 0,
@@ -96,12 +102,15 @@ uint64_t quip_kernel_launches(void);
  * randomized Hadamard).  Randomness: counter-based SplitMix64 (Steele, Lea &
  * Flood 2014); element i of stream t is output t*2^40 + i + 1 of the
  * sequence started at `seed`.  Streams: 0 = m-side signs, 1 = n-side signs,
- * 2 / 3 = m-side A / B Gaussians, 4 / 5 = n-side A / B Gaussians.  A sign is
+ * 2 / 3 = m-side A / B Gaussians, 4 / 5 = n-side A / B Gaussians, 6 / 7 =
+ * m-side / n-side permutation draws (pi lists the indices of the side's
+ * first d draws in increasing order of the draw).  A sign is
  * -1 when the draw's top bit is set.  A Gaussian matrix element e (row-major)
  * is sqrt(-2 ln u1) cos(2 pi u2) with u = ((draw >> 11) + 1) 2^-53 of draws
  * 2e and 2e+1; the factor is Q of G = QR with diag(R) > 0.
  * Signs, factors and the QR are computed on the device on `stream`.
- *   m_kind / n_kind : quip_tkind for each side; m_p*m_q == m for KRONECKER.
+ *   m_kind / n_kind : quip_tkind for each side, optionally | QUIP_T_PERMUTE;
+ *                     m_p*m_q == m for KRONECKER.
  *   out             : receives the new object (host pointer to a handle).
  * Allocates device memory owned by the object (freed by destroy).  The
  * object may be used on any stream after the creating stream has passed it.
@@ -131,6 +140,13 @@ quip_status quip_transform_destroy(quip_transform* tf);
 quip_status quip_transform_info(const quip_transform* tf, int side, int* kind,
                                 int64_t* p, int64_t* q, const float** signs,
                                 const float** A, const float** B);
+
+/*
+ * Device pointer (library-owned, read-only) of one side's permutation pi
+ * (d int32, (P x)_r = x_{pi[r]}), or NULL when the side has none
+ * (QUIP_T_PERMUTE not given).  side 0 = m side, 1 = n side.
+ */
+quip_status quip_transform_permutation(const quip_transform* tf, int side, const int32_t** perm);
 
 /*
  * Proxy Hessian accumulation (QuIP, adaptive-rounding section: H is the

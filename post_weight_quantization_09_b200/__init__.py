@@ -29,6 +29,11 @@ __all__ = [
 KIND = {"identity": L.QUIP_T_IDENTITY, "hadamard": L.QUIP_T_HADAMARD, "kronecker": L.QUIP_T_KRONECKER}
 
 
+def _kind(side) -> int:
+    """quip_tkind of a side spec (kind, p, q[, permute]), with QUIP_T_PERMUTE when asked."""
+    return KIND[side.kind] | (L.QUIP_T_PERMUTE if getattr(side, "permute", False) else 0)
+
+
 def _p(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -74,8 +79,8 @@ class Transform:
         self.m_side, self.n_side = m_side, n_side
         h = ctypes.c_void_p()
         L.check(lib.quip_transform_create(
-            ctypes.c_uint64(seed & 0xFFFFFFFFFFFFFFFF), m, n, KIND[m_side.kind], m_side.p, m_side.q,
-            KIND[n_side.kind], n_side.p, n_side.q, _s(stream), ctypes.byref(h)), "quip_transform_create")
+            ctypes.c_uint64(seed & 0xFFFFFFFFFFFFFFFF), m, n, _kind(m_side), m_side.p, m_side.q,
+            _kind(n_side), n_side.p, n_side.q, _s(stream), ctypes.byref(h)), "quip_transform_create")
         self.handle = h
 
     def draw(self, seed: int, stream=None) -> None:
@@ -95,7 +100,8 @@ class Transform:
             pass
 
     def factors(self, side: int) -> dict:
-        """Copies of one side's data: {'kind', 'signs'} or {'kind', 'A', 'B'} (fp32, cuda)."""
+        """Copies of one side's data: {'kind', 'signs'} or {'kind', 'A', 'B'} (fp32, cuda),
+        plus 'perm' (int32, cuda) when the side has a random permutation."""
         kind, p, q = ctypes.c_int(), ctypes.c_int64(), ctypes.c_int64()
         s, a, b = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_void_p()
         L.check(load().quip_transform_info(self.handle, side, ctypes.byref(kind), ctypes.byref(p),
@@ -114,6 +120,13 @@ class Transform:
             _memcpy_d2d(A.data_ptr(), a.value, A.numel() * 4)
             _memcpy_d2d(B.data_ptr(), b.value, B.numel() * 4)
             out["A"], out["B"] = A, B
+        pp = ctypes.c_void_p()
+        L.check(load().quip_transform_permutation(self.handle, side, ctypes.byref(pp)),
+                "quip_transform_permutation")
+        if pp.value:
+            P = torch.empty(dim, dtype=torch.int32, device="cuda")
+            _memcpy_d2d(P.data_ptr(), pp.value, dim * 4)
+            out["perm"] = P
         return out
 
 

@@ -13,6 +13,7 @@ QUIP_OK, QUIP_ERR_ARG, QUIP_ERR_SHAPE, QUIP_ERR_UNSUPPORTED = 0, 1, 2, 3
 QUIP_ERR_NOT_PD, QUIP_ERR_NONFINITE, QUIP_ERR_CUDA, QUIP_ERR_TIMEOUT, QUIP_ERR_WORKSPACE = 4, 5, 6, 7, 8
 QUIP_F32, QUIP_BF16 = 0, 1
 QUIP_T_IDENTITY, QUIP_T_HADAMARD, QUIP_T_KRONECKER = 0, 1, 2
+QUIP_T_PERMUTE = 0x100
 QUIP_OP_INCOHERENCE_FORWARD, QUIP_OP_INCOHERENCE_INVERSE, QUIP_OP_LDL, QUIP_OP_LDLQ = 0, 1, 2, 3
 
 # name -> (restype, argtypes); the list of every symbol include/quip.h declares
@@ -27,6 +28,7 @@ SIGNATURES = {
     "quip_transform_info": (c_int, [c_void_p, c_int, POINTER(c_int), POINTER(c_int64),
                                     POINTER(c_int64), POINTER(c_void_p), POINTER(c_void_p),
                                     POINTER(c_void_p)]),
+    "quip_transform_permutation": (c_int, [c_void_p, c_int, POINTER(c_void_p)]),
     "quip_hessian_accumulate": (c_int, [c_void_p, c_int, c_int64, c_int64, c_int64, c_void_p, c_int,
                                         c_void_p]),
     "quip_hessian_finalize": (c_int, [c_void_p, c_int64, c_int64, c_float, c_void_p]),

@@ -40,6 +40,10 @@ struct SideData {
   double* B64 = nullptr;
   double* G = nullptr;      // KRONECKER: Gaussian draw scratch, max(p,q)^2
   double* Qc = nullptr;     // KRONECKER: CGS2 scratch, max(p,q)^2
+  bool permute = false;     // S = T P, (P x)_r = x_{perm[r]}
+  int32_t* perm = nullptr;  // pi (dim)
+  int32_t* iperm = nullptr; // pi^-1 (dim)
+  uint64_t* keys = nullptr; // permutation draws (dim)
 };
 
 inline bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -447,6 +451,36 @@ cudaError_t side_cols(const SideData& sd, bool inverse, float* X, int64_t ncols,
   return cudaSuccess;
 }
 
+// out[r][c] = in[rp[r]][cp[c]] (a NULL permutation is the identity), fp32
+// out; rows by blockIdx.y (grid-stride), four output columns per thread.
+template <typename TIn>
+__global__ void __launch_bounds__(256) k_gather2d(const TIn* __restrict__ in, int64_t ldin,
+                                                  float* __restrict__ out, int64_t ldout,
+                                                  int64_t rows, int64_t cols,
+                                                  const int32_t* __restrict__ rp,
+                                                  const int32_t* __restrict__ cp) {
+  for (int64_t r = blockIdx.y; r < rows; r += gridDim.y) {
+    const TIn* src = in + (rp ? (int64_t)rp[r] : r) * ldin;
+    float* dst = out + r * ldout;
+    for (int64_t c = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); c < cols;
+         c += 4 * (int64_t)gridDim.x * blockDim.x) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (c + k < cols) dst[c + k] = to_f32(src[cp ? (int64_t)cp[c + k] : c + k]);
+    }
+  }
+}
+
+template <typename TIn>
+cudaError_t gather2d(const TIn* in, int64_t ldin, float* out, int64_t ldout, int64_t rows,
+                     int64_t cols, const int32_t* rp, const int32_t* cp, cudaStream_t st) {
+  const unsigned gx = (unsigned)std::min<int64_t>((cols + 1023) / 1024, 64);
+  const unsigned gy = (unsigned)std::min<int64_t>(rows, 65535);
+  LaunchScope ls("k_gather2d", st);
+  k_gather2d<TIn><<<dim3(gx, gy), 256, 0, st>>>(in, ldin, out, ldout, rows, cols, rp, cp);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 struct quip_transform {
@@ -477,8 +511,11 @@ const char* quip_version(void) { return "quip-b200 0.1.0 sm_100a"; }
 
 uint64_t quip_kernel_launches(void) { return g_launch_count.load(); }
 
-static quip_status check_side(int kind, int64_t dim, int64_t p, int64_t q) {
+static quip_status check_side(int kind_flags, int64_t dim, int64_t p, int64_t q) {
+  if (kind_flags & ~(0xFF | QUIP_T_PERMUTE)) return QUIP_ERR_ARG;
+  const int kind = kind_flags & 0xFF;
   if (dim <= 0) return QUIP_ERR_SHAPE;
+  if ((kind_flags & QUIP_T_PERMUTE) && dim > 65536) return QUIP_ERR_SHAPE;
   if (kind == QUIP_T_IDENTITY) return QUIP_OK;
   if (kind == QUIP_T_HADAMARD) return (is_pow2(dim) && dim >= 2 && dim <= 8192) ? QUIP_OK : QUIP_ERR_SHAPE;
   if (kind == QUIP_T_KRONECKER)
@@ -486,8 +523,15 @@ static quip_status check_side(int kind, int64_t dim, int64_t p, int64_t q) {
   return QUIP_ERR_ARG;
 }
 
-static quip_status alloc_side(SideData& sd, int kind, int64_t dim, int64_t p, int64_t q) {
+static quip_status alloc_side(SideData& sd, int kind_flags, int64_t dim, int64_t p, int64_t q) {
+  const int kind = kind_flags & 0xFF;
   sd.kind = kind, sd.dim = dim, sd.p = p, sd.q = q;
+  sd.permute = (kind_flags & QUIP_T_PERMUTE) != 0;
+  if (sd.permute) {
+    QCHECK(cudaMalloc(&sd.perm, dim * sizeof(int32_t)));
+    QCHECK(cudaMalloc(&sd.iperm, dim * sizeof(int32_t)));
+    QCHECK(cudaMalloc(&sd.keys, dim * sizeof(uint64_t)));
+  }
   if (kind == QUIP_T_HADAMARD) {
     QCHECK(cudaMalloc(&sd.signs, dim * sizeof(float)));
   } else if (kind == QUIP_T_KRONECKER) {
@@ -504,6 +548,15 @@ static quip_status alloc_side(SideData& sd, int kind, int64_t dim, int64_t p, in
 
 // Draw one side's random data from `seed` into its existing buffers.
 static quip_status draw_side(const SideData& sd, uint64_t seed, int which, cudaStream_t st) {
+  if (sd.permute) {
+    const unsigned g = (unsigned)((sd.dim + 255) / 256);
+    {
+      LaunchScope ls("k_perm_keys", st);
+      k_perm_keys<<<g, 256, 0, st>>>(sd.keys, sd.dim, seed, which == 0 ? 6u : 7u);
+    }
+    LaunchScope ls("k_perm_rank", st);
+    k_perm_rank<<<g, 256, 0, st>>>(sd.keys, sd.dim, sd.perm, sd.iperm);
+  }
   if (sd.kind == QUIP_T_HADAMARD) {
     LaunchScope ls("k_random_signs", st);
     k_random_signs<<<(unsigned)((sd.dim + 255) / 256), 256, 0, st>>>(sd.signs, sd.dim, seed,
@@ -564,6 +617,9 @@ quip_status quip_transform_destroy(quip_transform* tf) {
     cudaFree(sd.B64);
     cudaFree(sd.G);
     cudaFree(sd.Qc);
+    cudaFree(sd.perm);
+    cudaFree(sd.iperm);
+    cudaFree(sd.keys);
   }
   delete tf;
   return QUIP_OK;
@@ -580,6 +636,12 @@ quip_status quip_transform_info(const quip_transform* tf, int side, int* kind, i
   if (signs) *signs = sd.signs;
   if (A) *A = sd.A;
   if (B) *B = sd.B;
+  return QUIP_OK;
+}
+
+quip_status quip_transform_permutation(const quip_transform* tf, int side, const int32_t** perm) {
+  if (!tf || side < 0 || side > 1 || !perm) return QUIP_ERR_ARG;
+  *perm = tf->side[side].perm;
   return QUIP_OK;
 }
 
@@ -660,6 +722,22 @@ static size_t ldlq_ws_bytes(int64_t m, int64_t n, int64_t block) {
          round256((size_t)3 * n * n * 2) + round256((size_t)n * n * 4);
 }
 
+// Transform workspace: Kronecker temporaries, then the permutation scratch
+// (the forward pass gathers H into it, the inverse gathers W^).
+static size_t transform_kron_bytes(const quip_transform* tf, int op) {
+  const bool kron = tf->side[0].kind == QUIP_T_KRONECKER || tf->side[1].kind == QUIP_T_KRONECKER;
+  if (!kron) return 0;
+  size_t e = (size_t)tf->m * tf->n;
+  if (op == QUIP_OP_INCOHERENCE_FORWARD) e = std::max(e, (size_t)tf->n * tf->n);
+  return round256(e * sizeof(float));
+}
+static size_t transform_perm_bytes(const quip_transform* tf, int op) {
+  if (op == QUIP_OP_INCOHERENCE_FORWARD)
+    return tf->side[1].permute ? round256((size_t)tf->n * tf->n * sizeof(float)) : 0;
+  return (tf->side[0].permute || tf->side[1].permute) ? round256((size_t)tf->m * tf->n * sizeof(float))
+                                                      : 0;
+}
+
 quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int64_t n,
                                 int64_t block, size_t* bytes) {
   if (!bytes) return QUIP_ERR_ARG;
@@ -668,12 +746,7 @@ quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int
     case QUIP_OP_INCOHERENCE_FORWARD:
     case QUIP_OP_INCOHERENCE_INVERSE: {
       if (!tf) return QUIP_ERR_ARG;
-      const bool kron = tf->side[0].kind == QUIP_T_KRONECKER || tf->side[1].kind == QUIP_T_KRONECKER;
-      if (kron) {
-        size_t e = (size_t)tf->m * tf->n;
-        if (op == QUIP_OP_INCOHERENCE_FORWARD) e = std::max(e, (size_t)tf->n * tf->n);
-        *bytes = round256(e * sizeof(float));
-      }
+      *bytes = transform_kron_bytes(tf, op) + transform_perm_bytes(tf, op);
       return QUIP_OK;
     }
     case QUIP_OP_LDL:
@@ -715,12 +788,29 @@ quip_status quip_incoherence_forward(const quip_transform* tf, const void* W, in
   if ((s = check_ws(ws, ws_bytes, need)) != QUIP_OK) return s;
   cudaStream_t st = S(stream);
   float* tmp = static_cast<float*>(ws);
+  float* pscr = reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                         transform_kron_bytes(tf, QUIP_OP_INCOHERENCE_FORWARD));
   if (W) {
-    if (w_dtype == QUIP_BF16)
+    const int32_t* rp = U.permute ? U.perm : nullptr;
+    const int32_t* cp = V.permute ? V.perm : nullptr;
+    if (rp || cp) {
+      // W_t = P_m W P_n^T (W_t[r][c] = W[pi_m[r]][pi_n[c]]), then the structured factors in place
+      if (w_dtype == QUIP_BF16)
+        QCHECK(gather2d<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(W), ldw, W_t, n, m, n, rp, cp, st));
+      else
+        QCHECK(gather2d<float>(static_cast<const float*>(W), ldw, W_t, n, m, n, rp, cp, st));
+      QCHECK(side_rows<float>(V, false, W_t, n, W_t, m, tmp, st));
+    } else if (w_dtype == QUIP_BF16) {
       QCHECK(side_rows<__nv_bfloat16>(V, false, static_cast<const __nv_bfloat16*>(W), ldw, W_t, m, tmp, st));
-    else
+    } else {
       QCHECK(side_rows<float>(V, false, static_cast<const float*>(W), ldw, W_t, m, tmp, st));
+    }
     QCHECK(side_cols(U, false, W_t, n, tmp, st));
+  }
+  if (H && V.permute) {
+    // P_n H P_n^T, through the scratch
+    QCHECK(gather2d<float>(H, n, pscr, n, n, n, V.perm, V.perm, st));
+    QCHECK(cudaMemcpyAsync(H, pscr, (size_t)n * n * sizeof(float), cudaMemcpyDeviceToDevice, st));
   }
   if (H) {
     if (V.kind == QUIP_T_KRONECKER) {                           // fp64 sums, see gemm_simt.cuh
@@ -746,6 +836,15 @@ quip_status quip_incoherence_inverse(const quip_transform* tf, const float* W_ha
   float* tmp = static_cast<float*>(ws);
   QCHECK(side_rows<float>(tf->side[1], true, W_hat_t, n, W_hat, m, tmp, st));
   QCHECK(side_cols(tf->side[0], true, W_hat, n, tmp, st));
+  const SideData &U = tf->side[0], &V = tf->side[1];
+  if (U.permute || V.permute) {
+    // W^ = P_m^T (T_m^T W~^ T_n) P_n: W^[r][c] = M[pi_m^-1[r]][pi_n^-1[c]], through the scratch
+    float* pscr = reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                           transform_kron_bytes(tf, QUIP_OP_INCOHERENCE_INVERSE));
+    QCHECK(gather2d<float>(W_hat, n, pscr, n, m, n, U.permute ? U.iperm : nullptr,
+                           V.permute ? V.iperm : nullptr, st));
+    QCHECK(cudaMemcpyAsync(W_hat, pscr, (size_t)m * n * sizeof(float), cudaMemcpyDeviceToDevice, st));
+  }
   return QUIP_OK;
 }
 

@@ -33,6 +33,40 @@ __global__ void k_random_signs(float* s, int64_t n, uint64_t seed, uint32_t stre
   }
 }
 
+// Random permutation of n coordinates: key_i = draw i of `stream`; pi sorts
+// the keys in increasing order ((P x)_r = x_{pi[r]}).  The draws are
+// distinct (the SplitMix64 finaliser is a bijection), so the rank of key i,
+// #{j : key_j < key_i}, is pi^-1[i].
+__global__ void k_perm_keys(uint64_t* keys, int64_t n, uint64_t seed, uint32_t stream) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    keys[i] = splitmix64(seed, stream, (uint64_t)i);
+}
+
+// rank by counting (n <= 65536: n^2 comparisons, keys staged through shared
+// memory in tiles): iperm[i] = rank of key i, perm[rank] = i.
+constexpr int PERM_TILE = 2048;
+__global__ void __launch_bounds__(256) k_perm_rank(const uint64_t* __restrict__ keys, int64_t n,
+                                                   int32_t* __restrict__ perm,
+                                                   int32_t* __restrict__ iperm) {
+  __shared__ uint64_t tile[PERM_TILE];
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const uint64_t ki = i < n ? keys[i] : 0ull;
+  int32_t rank = 0;
+  for (int64_t j0 = 0; j0 < n; j0 += PERM_TILE) {
+    const int len = (int)min((int64_t)PERM_TILE, n - j0);
+    __syncthreads();
+    for (int t = threadIdx.x; t < len; t += blockDim.x) tile[t] = keys[j0 + t];
+    __syncthreads();
+#pragma unroll 8
+    for (int t = 0; t < len; ++t) rank += tile[t] < ki ? 1 : 0;
+  }
+  if (i < n) {
+    iperm[i] = rank;
+    perm[rank] = (int32_t)i;
+  }
+}
+
 // p x p Gaussian matrix, row-major element e from draws 2e, 2e+1:
 // u = ((draw >> 11) + 1) 2^-53 in (0, 1], g = sqrt(-2 ln u1) cos(2 pi u2).
 __global__ void k_gaussian(double* G, int64_t count, uint64_t seed, uint32_t stream) {

@@ -33,12 +33,19 @@ def _status_clean():
     (8, 2048, Side("hadamard"), Side("hadamard")),
     (48, 86 * 3, Side("kronecker", 6, 8), Side("kronecker", 86, 3)),
     (224, 32, Side("kronecker", 224, 1), Side("identity")),
+    (64, 128, Side("hadamard", permute=True), Side("hadamard", permute=True)),
+    (28672, 48, Side("kronecker", 224, 128, True), Side("identity", permute=True)),
 ])
 def test_transform_factors_match_oracle(m, n, mk, nk):
     tf = Q.Transform(1234, m, n, mk, nk)
     for side, spec, dim in ((0, mk, m), (1, nk, n)):
         f = tf.factors(side)
-        ref = O.make_side(1234, "m" if side == 0 else "n", spec.kind, dim, spec.p, spec.q)
+        ref = O.make_side(1234, "m" if side == 0 else "n", spec.kind, dim, spec.p, spec.q,
+                          spec.permute)
+        if spec.permute:
+            np.testing.assert_array_equal(f["perm"].cpu().numpy(), ref.perm)
+        else:
+            assert "perm" not in f
         if spec.kind == "hadamard":
             np.testing.assert_array_equal(host(f["signs"]), ref.signs)
         elif spec.kind == "kronecker":
@@ -65,13 +72,18 @@ def test_transform_redraw_in_place():
     (4, 8, Side("hadamard"), Side("hadamard"), "f32"),          # register-only paths
     (96, 86 * 2, Side("kronecker", 12, 8), Side("kronecker", 86, 2), "bf16"),
     (30, 64, Side("identity"), Side("hadamard"), "bf16"),
+    # random permutation within the fast orthogonal multiplication
+    (64, 128, Side("hadamard", permute=True), Side("hadamard", permute=True), "bf16"),
+    (512, 1024, Side("identity"), Side("hadamard", permute=True), "f32"),
+    (96, 86 * 2, Side("kronecker", 12, 8, True), Side("kronecker", 86, 2, True), "f32"),
+    (30, 64, Side("identity", permute=True), Side("identity", permute=True), "bf16"),
 ])
 def test_incoherence_forward_inverse(m, n, mk, nk, dtype):
     d = random_layer(m, n, min(4 * n, 2048), seed=m + n, dtype=dtype)
     W, X = d["W"], d["X"]
     H = O.damp(O.hessian(X), 0.01)
-    U = O.make_side(7, "m", mk.kind, m, mk.p, mk.q)
-    V = O.make_side(7, "n", nk.kind, n, nk.p, nk.q)
+    U = O.make_side(7, "m", mk.kind, m, mk.p, mk.q, mk.permute)
+    V = O.make_side(7, "n", nk.kind, n, nk.p, nk.q, nk.permute)
     with_h = n <= 4096          # the explicit FP64 V H V^T is slow beyond that
     Wt_ref, Ht_ref = O.incoherence_forward(W, H if with_h else np.eye(1), U, V) if with_h else \
         (U.matrix() @ W @ V.matrix().T, None)
@@ -347,3 +359,25 @@ def test_run_host_equals_device_run():
         q2.run_host(Wh, Xh, co, lo_h, sc_h)
         torch.cuda.current_stream().synchronize()
         assert torch.equal(co, codes) and torch.equal(lo_h, lo) and torch.equal(sc_h, sc)
+
+
+@pytest.mark.parametrize("mk,nk", [
+    (Side("hadamard", permute=True), Side("hadamard", permute=True)),
+    (Side("kronecker", 8, 8, True), Side("hadamard", permute=True)),
+])
+def test_pipeline_with_random_permutations(mk, nk):
+    m, n, bits, block, seed = 64, 256, 2, 128, 3
+    d = random_layer(m, n, 1024, seed=41)
+    P = O.run_pipeline(d["W"], d["X"], seed, mk, nk, bits, 0.01)
+    q = Q.LayerQuantizer(m, n, mk, nk, bits, block, 0.01, seed)
+    r = q.run(dev(d["W"]), dev(d["X"]))
+    assert Q.quip_sync_status() == L.QUIP_OK
+    C = host(r.codes)
+    assert (C == P.codes).mean() >= 0.999
+    lo, s = host(r.lo), host(r.scale)
+    Wt_hat = O.dequantize(C, lo, s)
+    assert abs(O.proxy_loss(Wt_hat, P.Wt, P.Ht) - P.loss) / P.loss <= 1e-3
+    W_hat_ref = O.incoherence_inverse(Wt_hat, P.U, P.V)
+    assert np.abs(host(r.W_hat) - W_hat_ref).max() <= 1e-4 * s.max()
+    bad, not_near = ldlq_trajectory_check(C, P.Wt, P.Uf, lo, s, bits, tau=1e-3)
+    assert not_near == 0.0
