@@ -17,7 +17,9 @@ Sources (page title, then the section / equation each step follows):
           - Incoherence-processing section: H~ <- V H V^T, W~ <- U W V^T and
             the trace identity tr(W~ H~ W~^T) = tr(W H W^T).
           - Experiments, "Methods.": damping H <- H + alpha*mean(diag(H)) I;
-            nearest rounding and LDLQ as rounding methods; LDLQ = OPTQ.
+            nearest rounding and LDLQ as rounding methods; LDLQ = OPTQ;
+            LDLQ-RG (re-order by diag(H), then greedy updates of the proxy)
+            and "Greedy" (the greedy updates alone).
 [QuIP#] "QuIP#: Even Better LLM Quantization with Hadamard Incoherence and
         Lattice Codebooks" (arXiv 2402.04396), abstract: incoherence by the
         randomized Hadamard transform.
@@ -42,7 +44,13 @@ Readings where the pages are silent (each one is listed in the design doc):
     Experiments, "Further Ablation", Table 5; the algorithm box that placed
     it was lost): optional per side, applied to the coordinates before the
     structured factor, S = T P with (P x)_r = x_{pi[r]}; pi sorts the draws
-    of the side's permutation stream (``random_permutation``).
+    of the side's permutation stream (``random_permutation``);
+  * LDLQ-RG and Greedy ("Methods." names them in one sentence each): the
+    re-ordering quantises columns by decreasing diag(H~) (ties by index);
+    a greedy update sets one column to its exact coordinate minimiser on
+    the grid, others held; a pass visits every column once, in the
+    quantisation order; Greedy starts from nearest rounding; the number of
+    passes is a parameter (the pages give none).
 
 Pinned by tests/test_oracle_*.py (CPU).  Functions with no pin: none.
 """
@@ -61,6 +69,7 @@ __all__ = [
     "ldlq", "ldlq_blocked", "nearest", "optq", "dequantize", "proxy_loss", "Pipeline",
     "run_pipeline", "STREAM_M_SIGNS", "STREAM_N_SIGNS", "STREAM_M_A", "STREAM_M_B",
     "STREAM_N_A", "STREAM_N_B", "STREAM_M_PERM", "STREAM_N_PERM", "random_permutation",
+    "diag_order", "greedy_pass", "quantize_layer",
 ]
 
 # ----------------------------------------------------------------------------
@@ -411,6 +420,77 @@ def optq(Wt: np.ndarray, H: np.ndarray, lo: np.ndarray, s: np.ndarray, bits: int
     return codes
 
 
+def diag_order(H: np.ndarray) -> np.ndarray:
+    """LDLQ-RG's quantisation order ([QuIP] Experiments, "Methods.": LDLQ-RG
+    re-orders the weights by diag(H)): the column indices sorted by
+    decreasing H_kk, equal diagonal entries by increasing index.
+    order[r] is the column quantised r-th."""
+    d = np.diag(np.asarray(H, dtype=np.float64))
+    return np.argsort(-d, kind="stable")
+
+
+def greedy_pass(Wt: np.ndarray, H: np.ndarray, lo: np.ndarray, s: np.ndarray, bits: int,
+                codes: np.ndarray, order=None) -> np.ndarray:
+    """One pass of greedy updates to the proxy ([QuIP] Experiments,
+    "Methods.": LDLQ-RG adds greedy updates to the proxy, "Greedy" performs
+    them alone).  The columns are visited in ``order`` (default 0..n-1); at
+    column k every other column is held at its current value and column k
+    takes, per row, the grid point that minimises
+    tr((W^ - W) H (W^ - W)^T) over that one column.  As a function of
+    W^_k the proxy is H_kk (W^_k - t_k)^2 + const with
+        t_k = W_k - sum_{j != k} (W^_j - W_j) H_jk / H_kk,
+    so the minimiser on the grid is the grid point nearest t_k: Q(t_k).
+    Returns the new codes."""
+    Wt = np.asarray(Wt, dtype=np.float64)
+    H = np.asarray(H, dtype=np.float64)
+    lo = np.asarray(lo, dtype=np.float64)
+    s = np.asarray(s, dtype=np.float64)
+    c = np.array(codes, dtype=np.int64, copy=True)
+    m, n = Wt.shape
+    E = (lo[:, None] + s[:, None] * c) - Wt     # W^ - W, kept current
+    for k in (range(n) if order is None else order):
+        others = E @ H[:, k] - E[:, k] * H[k, k]
+        t = Wt[:, k] - others / H[k, k]
+        c[:, k] = quantize(t, lo, s, bits)
+        E[:, k] = lo + s * c[:, k] - Wt[:, k]
+    return c
+
+
+def quantize_layer(method: str, Wt: np.ndarray, Ht: np.ndarray, lo: np.ndarray, s: np.ndarray,
+                   bits: int, passes: int = 1) -> np.ndarray:
+    """The rounding methods of [QuIP] Experiments, "Methods.", on the
+    incoherent weights and Hessian, one per-row grid (lo, s):
+      nearest : nearest rounding;
+      ldlq    : LDLQ with the LDL factor of Ht;
+      greedy  : nearest rounding, then ``passes`` greedy passes;
+      ldlq_rg : columns re-ordered by decreasing diag(Ht), LDLQ in that
+                order (the LDL factor of the re-ordered Ht), then ``passes``
+                greedy passes visiting the columns in the same order.
+    Returns the codes in the original column order."""
+    Wt = np.asarray(Wt, dtype=np.float64)
+    Ht = np.asarray(Ht, dtype=np.float64)
+    if method == "nearest":
+        return nearest(Wt, lo, s, bits)
+    if method == "ldlq":
+        return ldlq(Wt, udu(Ht)[0], lo, s, bits)[0]
+    if method == "greedy":
+        c = nearest(Wt, lo, s, bits)
+        for _ in range(passes):
+            c = greedy_pass(Wt, Ht, lo, s, bits, c)
+        return c
+    if method == "ldlq_rg":
+        order = diag_order(Ht)
+        Wp = Wt[:, order]
+        Hp = Ht[np.ix_(order, order)]
+        cp = ldlq(Wp, udu(Hp)[0], lo, s, bits)[0]
+        for _ in range(passes):
+            cp = greedy_pass(Wp, Hp, lo, s, bits, cp)
+        c = np.empty_like(cp)
+        c[:, order] = cp                        # column order[r] was quantised r-th
+        return c
+    raise ValueError(f"unknown rounding method {method!r}")
+
+
 # ----------------------------------------------------------------------------
 # O7/O8  Dequantisation, loss
 # ----------------------------------------------------------------------------
@@ -450,10 +530,13 @@ class Pipeline:
 
 
 def run_pipeline(W: np.ndarray, X: np.ndarray, seed: int, m_side, n_side, bits: int,
-                 alpha: float = 0.01, block: Optional[int] = None) -> Pipeline:
+                 alpha: float = 0.01, block: Optional[int] = None, method: str = "ldlq",
+                 passes: int = 1) -> Pipeline:
     """Hessian -> damping -> incoherence -> LDL -> grid -> LDLQ -> dequant -> inverse.
 
     ``m_side`` / ``n_side`` are objects with attributes kind, p, q.
+    ``method`` picks the rounding (``quantize_layer``); Uf and D stay the
+    LDL of Ht in its original order.
     """
     W = np.asarray(W, dtype=np.float64)
     m, n = W.shape
@@ -463,7 +546,10 @@ def run_pipeline(W: np.ndarray, X: np.ndarray, seed: int, m_side, n_side, bits: 
     Wt, Ht = incoherence_forward(W, H, U, V)
     Uf, D = udu(Ht)
     lo, s = row_grid(Wt, bits)
-    if block is None:
+    if method != "ldlq":
+        codes = quantize_layer(method, Wt, Ht, lo, s, bits, passes)
+        Wt_hat = dequantize(codes, lo, s)
+    elif block is None:
         codes, Wt_hat, _ = ldlq(Wt, Uf, lo, s, bits)
     else:
         codes, Wt_hat = ldlq_blocked(Wt, Uf, lo, s, bits, block)

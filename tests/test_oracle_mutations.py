@@ -143,3 +143,73 @@ def test_planted_permutation_order_is_caught(monkeypatch):
     monkeypatch.setattr(Q, "random_permutation", _permutation_descending)
     monkeypatch.setattr(O, "random_permutation", _permutation_descending)
     assert _fails([P.test_random_permutation_sorts_its_draws_brute_force])
+
+
+def _greedy_sign(Wt, H, lo, s, bits, codes, order=None):
+    c = np.array(codes, dtype=np.int64, copy=True)
+    E = (lo[:, None] + s[:, None] * c) - Wt
+    for k in (range(Wt.shape[1]) if order is None else order):
+        t = Wt[:, k] + (E @ H[:, k] - E[:, k] * H[k, k]) / H[k, k]      # planted: sign
+        c[:, k] = Q.quantize(t, lo, s, bits)
+        E[:, k] = lo + s * c[:, k] - Wt[:, k]
+    return c
+
+
+def _greedy_self_term(Wt, H, lo, s, bits, codes, order=None):
+    c = np.array(codes, dtype=np.int64, copy=True)
+    E = (lo[:, None] + s[:, None] * c) - Wt
+    for k in (range(Wt.shape[1]) if order is None else order):
+        t = Wt[:, k] - (E @ H[:, k]) / H[k, k]                          # planted: j = k kept
+        c[:, k] = Q.quantize(t, lo, s, bits)
+        E[:, k] = lo + s * c[:, k] - Wt[:, k]
+    return c
+
+
+def _greedy_unscaled(Wt, H, lo, s, bits, codes, order=None):
+    c = np.array(codes, dtype=np.int64, copy=True)
+    E = (lo[:, None] + s[:, None] * c) - Wt
+    for k in (range(Wt.shape[1]) if order is None else order):
+        t = Wt[:, k] - (E @ H[:, k] - E[:, k] * H[k, k])                 # planted: no 1/H_kk
+        c[:, k] = Q.quantize(t, lo, s, bits)
+        E[:, k] = lo + s * c[:, k] - Wt[:, k]
+    return c
+
+
+def _diag_order_ascending(H):
+    return np.argsort(np.diag(np.asarray(H, dtype=np.float64)), kind="stable")
+
+
+GREEDY_PINS = [P.test_rounding_methods_worked_example, P.test_greedy_update_is_the_coordinate_minimiser,
+               P.test_greedy_with_diagonal_h_is_nearest]
+
+
+@pytest.mark.parametrize("mutant", [_greedy_sign, _greedy_self_term, _greedy_unscaled])
+def test_planted_greedy_mistake_is_caught(monkeypatch, mutant):
+    monkeypatch.setattr(Q, "greedy_pass", mutant)
+    monkeypatch.setattr(O, "greedy_pass", mutant)
+    assert _fails(GREEDY_PINS)
+
+
+def test_planted_diag_order_direction_is_caught(monkeypatch):
+    monkeypatch.setattr(Q, "diag_order", _diag_order_ascending)
+    monkeypatch.setattr(O, "diag_order", _diag_order_ascending)
+    assert _fails([P.test_rounding_methods_worked_example, P.test_diag_order_brute_force])
+
+
+@pytest.mark.parametrize("twice", [False, True])
+def test_planted_rg_unpermute_mistake_is_caught(monkeypatch, twice):
+    # codes left in the quantisation order (c_p = c[:, pi]), or moved back the
+    # wrong way (c_p[:, pi] instead of c_p[:, pi^-1])
+    orig = Q.quantize_layer
+
+    def wrong(method, Wt, Ht, lo, s, bits, passes=1):
+        c = orig(method, Wt, Ht, lo, s, bits, passes)
+        if method != "ldlq_rg":
+            return c
+        order = Q.diag_order(Ht)
+        cp = c[:, order]
+        return cp[:, order] if twice else cp
+
+    monkeypatch.setattr(Q, "quantize_layer", wrong)
+    monkeypatch.setattr(O, "quantize_layer", wrong)
+    assert _fails([P.test_rounding_methods_worked_example, P.test_ldlq_rg_first_columns_and_equivariance])

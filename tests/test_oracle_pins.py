@@ -418,3 +418,135 @@ def test_permuted_side_orthogonal_rows_and_proxy(kind, dim, p, q):
     H = _spd(dim, 9)
     Wt, Ht = O.incoherence_forward(W, H, O.make_side(0, "m", "identity", 5), S)
     assert np.trace(Wt @ Ht @ Wt.T) == pytest.approx(np.trace(W @ H @ W.T), rel=1e-12)
+
+
+# ---------------------------------------------------------------- LDLQ-RG, Greedy
+
+
+def _proxy_codes(W, H, lo, s, c):
+    return O.proxy_loss(O.dequantize(c, lo, s), W, H)
+
+
+def test_rounding_methods_worked_example():
+    r = golden_rows("greedy_rg_n4_example.txt")
+    W = np.array([list(map(float, r[0].split()))])
+    H = np.array([list(map(float, r[i].split())) for i in range(1, 5)])
+    lo, s = O.row_grid(W, 2)
+    np.testing.assert_array_equal(O.diag_order(H), list(map(int, r[5].split())))
+    losses = list(map(float, r[10].split()))
+    for method, row, loss in zip(("nearest", "ldlq", "greedy", "ldlq_rg"), r[6:10], losses):
+        c = O.quantize_layer(method, W, H, lo, s, 2, passes=1)
+        np.testing.assert_array_equal(c[0], list(map(int, row.split())), err_msg=method)
+        assert _proxy_codes(W, H, lo, s, c) == pytest.approx(loss, rel=1e-12), method
+
+
+def test_diag_order_brute_force():
+    # exactly one ordering lists the diagonal non-increasing with equal entries
+    # by increasing index; find it among all n! orderings
+    rng = np.random.default_rng(31)
+    for n in (1, 2, 4, 5):
+        for _ in range(10):
+            d = rng.integers(0, 3, n).astype(float)
+            ok = [p for p in itertools.permutations(range(n))
+                  if all(d[p[r]] > d[p[r + 1]] or (d[p[r]] == d[p[r + 1]] and p[r] < p[r + 1])
+                         for r in range(n - 1))]
+            assert len(ok) == 1
+            np.testing.assert_array_equal(O.diag_order(np.diag(d) + 0.01), ok[0])
+
+
+def test_greedy_update_is_the_coordinate_minimiser():
+    # one greedy update of column k: per row, no other code of that column (the
+    # rest held) gives a lower proxy, found by trying all 2^b codes
+    rng = np.random.default_rng(41)
+    n, bits = 7, 2
+    H = _spd(n, 41, outliers=False)
+    W = rng.standard_normal((5, n))
+    lo, s = O.row_grid(W, bits)
+    c0 = rng.integers(0, 2 ** bits, W.shape)
+    for k in range(n):
+        c1 = O.greedy_pass(W, H, lo, s, bits, c0, order=[k])
+        np.testing.assert_array_equal(np.delete(c1, k, 1), np.delete(c0, k, 1))
+        for i in range(W.shape[0]):
+            vals = []
+            for v in range(2 ** bits):
+                c = c0[i].astype(np.float64)
+                c[k] = v
+                e = lo[i] + s[i] * c - W[i]
+                vals.append(float(e @ H @ e))
+            assert vals[c1[i, k]] <= min(vals) + 1e-12
+
+
+def test_greedy_with_diagonal_h_is_nearest():
+    # with H diagonal the columns decouple: from any codes, one pass rounds
+    # every column to nearest
+    rng = np.random.default_rng(42)
+    W = rng.standard_normal((9, 16))
+    lo, s = O.row_grid(W, 3)
+    c0 = rng.integers(0, 8, W.shape)
+    for H in (np.eye(16), np.diag(rng.uniform(0.5, 3, 16))):
+        np.testing.assert_array_equal(O.greedy_pass(W, H, lo, s, 3, c0), O.nearest(W, lo, s, 3))
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_greedy_passes_descend_to_a_coordinate_minimum(bits):
+    rng = np.random.default_rng(43 + bits)
+    n = 20
+    H = _spd(n, 43 + bits)
+    W = rng.standard_normal((6, n))
+    lo, s = O.row_grid(W, bits)
+    c = rng.integers(0, 2 ** bits, W.shape)
+    loss = _proxy_codes(W, H, lo, s, c)
+    for _ in range(100):
+        c2 = O.greedy_pass(W, H, lo, s, bits, c)
+        loss2 = _proxy_codes(W, H, lo, s, c2)
+        assert loss2 <= loss + 1e-12                   # coordinate descent never climbs
+        if np.array_equal(c2, c):
+            break
+        c, loss = c2, loss2
+    else:
+        pytest.fail("greedy passes did not settle")
+    # at the fixed point no single code change lowers a row's proxy
+    for i in range(W.shape[0]):
+        e0 = lo[i] + s[i] * c[i] - W[i]
+        l0 = float(e0 @ H @ e0)
+        for k in range(n):
+            for v in range(2 ** bits):
+                e = e0.copy()
+                e[k] = lo[i] + s[i] * v - W[i, k]
+                assert float(e @ H @ e) >= l0 - 1e-12
+
+
+def test_ldlq_rg_first_columns_and_equivariance():
+    rng = np.random.default_rng(44)
+    n, bits = 12, 2
+    H = _spd(n, 44, outliers=False)
+    W = rng.standard_normal((8, n))
+    lo, s = O.row_grid(W, bits)
+    order = O.diag_order(H)
+    c = O.quantize_layer("ldlq_rg", W, H, lo, s, bits, passes=0)
+    # the column quantised first (largest H_kk) has no feedback: nearest rounding
+    np.testing.assert_array_equal(c[:, order[0]], O.nearest(W[:, order[:1]], lo, s, bits)[:, 0])
+    # re-labelling the columns re-labels the codes (the order follows diag(H))
+    sig = rng.permutation(n)
+    c_sig = O.quantize_layer("ldlq_rg", W[:, sig], H[np.ix_(sig, sig)], lo, s, bits, passes=1)
+    np.testing.assert_array_equal(c_sig, O.quantize_layer("ldlq_rg", W, H, lo, s, bits, passes=1)[:, sig])
+    # with the diagonal already non-increasing, LDLQ-RG is LDLQ then greedy
+    Hs, Ws = H[np.ix_(order, order)], W[:, order]
+    want = O.greedy_pass(Ws, Hs, lo, s, bits, O.quantize_layer("ldlq", Ws, Hs, lo, s, bits))
+    np.testing.assert_array_equal(O.quantize_layer("ldlq_rg", Ws, Hs, lo, s, bits, passes=1), want)
+
+
+@pytest.mark.parametrize("n,bits", [(3, 2), (4, 2), (5, 2), (3, 3)])
+def test_rg_and_greedy_never_beat_brute_force(n, bits):
+    rng = np.random.default_rng(200 * n + bits)
+    H = _spd(n, 7 * n + bits, N=4 * n, outliers=False)
+    W = rng.standard_normal((5, n))
+    lo, s = O.row_grid(W, bits)
+    grid = np.array(list(itertools.product(range(2 ** bits), repeat=n)), dtype=np.float64)
+    for method in ("greedy", "ldlq_rg"):
+        c = O.quantize_layer(method, W, H, lo, s, bits, passes=2)
+        for i in range(W.shape[0]):
+            cand = lo[i] + s[i] * grid - W[i]
+            best = np.min(np.einsum("kj,jl,kl->k", cand, H, cand))
+            e = lo[i] + s[i] * c[i] - W[i]
+            assert float(e @ H @ e) >= best - 1e-12
