@@ -86,13 +86,19 @@ def _ldlq_block_flops(m: int, n: int, b: int = 128) -> float:
     return float(sum(m * min(b, n - k0) * (min(b, n - k0) - 1) for k0 in range(0, n, b)))
 
 
-def kernel_work(cfg: LayerConfig):
+def kernel_work(cfg: LayerConfig, method: str = "ldlq", passes: int = 1):
     """Algorithmic work per step of the library's kernels, by kernel name:
     (kind, amount, bound).  Flops count multiply-adds as 2; bytes are the
     minimum reads + writes of the kernel's operands.  The tensor-core split
     GEMMs are counted at their fp32 algorithmic flops (2 M N K) although they
-    run six bf16 products per multiply-add (the three-piece split)."""
+    run six bf16 products per multiply-add (the three-piece split).
+    ``method`` / ``passes``: the rounding method (LDLQ by default); a greedy
+    pass is one full GEMM (E H) plus LDLQ's recursion (block kernel and
+    trailing GEMMs)."""
     m, n, N = cfg.m, cfg.n, cfg.N
+    greedy = passes if method in ("greedy", "ldlq_rg") else 0
+    ldlq_runs = (1 if method in ("ldlq", "ldlq_rg") else 0) + greedy
+    has_ldl = method in ("ldlq", "ldlq_rg")
     xb = 2 if cfg.dtype == "bf16" else 4
     PB = 128
     P = (n + PB - 1) // PB
@@ -108,16 +114,31 @@ def kernel_work(cfg: LayerConfig):
             bulk += M * (M + 1) * PB            # upper triangle, 2 flops per multiply-add
     kw = {
         "k_syrk_tc": ("flops", float(N) * n * (n + 1), "tensor"),
-        "k_ldl_factor": ("flops", fac, "alu"),
-        "k_ldl_rows": ("flops", rows, "alu"),
-        "k_gemm_split_tc[ldl]": ("flops", bulk, "tensor"),
-        "k_gemm_split_tc[ldlq]": ("flops", _ldlq_gemm_flops(m, n, 128), "tensor"),
-        "k_ldlq_block": ("flops", _ldlq_block_flops(m, n), "alu"),
         "k_row_grid": ("bytes", 4.0 * m * n + 8.0 * m, "hbm"),
         "k_dequant": ("bytes", 5.0 * m * n + 8.0 * m, "hbm"),
-        "k_split_upper_transposed": ("bytes", 4.0 * n * n / 2 + 10.0 * n * n, "hbm"),
         "k_mirror_scale": ("bytes", 8.0 * n * n, "hbm"),
     }
+    if has_ldl:
+        kw.update({
+            "k_ldl_factor": ("flops", fac, "alu"),
+            "k_ldl_rows": ("flops", rows, "alu"),
+            "k_gemm_split_tc[ldl]": ("flops", bulk, "tensor"),
+            "k_split_upper_transposed": ("bytes", 4.0 * n * n / 2 + 10.0 * n * n, "hbm"),
+        })
+    if ldlq_runs:
+        kw["k_gemm_split_tc[ldlq]"] = ("flops", ldlq_runs * _ldlq_gemm_flops(m, n, 128), "tensor")
+        kw["k_ldlq_block"] = ("flops", ldlq_runs * _ldlq_block_flops(m, n), "alu")
+    if method in ("nearest", "greedy"):
+        kw["k_nearest"] = ("bytes", 5.0 * m * n + 8.0 * m, "hbm")
+    if greedy:
+        kw["k_gemm_split_tc[greedy]"] = ("flops", greedy * 2.0 * m * n * n, "tensor")
+        # codes + W in; W^, the accumulator and three bf16 error pieces out
+        kw["k_greedy_start"] = ("bytes", greedy * 19.0 * m * n, "hbm")
+        # H's upper triangle in; U'^T (fp32 and three pieces) and U' out
+        kw["k_greedy_factors"] = ("bytes", 16.0 * n * n, "hbm")
+    if method == "ldlq_rg":
+        # H~ gathered twice (8 n^2 each), W~ once (8 m n), the codes back (2 m n)
+        kw["k_permute"] = ("bytes", 16.0 * n * n + 10.0 * m * n, "hbm")
     # Hadamard passes: rows read their input (W once as bf16/f32, H and W^
     # in fp32) and write fp32; column passes read and write fp32.
     had = lambda s: s.kind == "hadamard"
@@ -141,14 +162,16 @@ def kernel_work(cfg: LayerConfig):
 # unchanged and only for the workload it was captured on.
 KERNEL_TRAFFIC = {
     "k_syrk_tc": ("syrk_tc.cuh", "260ad4eebdfc", 71597824),
-    "k_ldlq_block": ("ldlq.cuh", "449a391e49fc", 6490880),
-    "k_ldl_factor": ("ldl.cuh", "df9cc064a14e", 338944),
-    "k_ldl_rows": ("ldl.cuh", "df9cc064a14e", 4653824),
+    "k_ldlq_block": ("ldlq.cuh", "eb4bda779455", 6490368),
+    "k_ldl_factor": ("ldl.cuh", "6428de196929", 339200),
+    "k_ldl_rows": ("ldl.cuh", "6428de196929", 4653824),
     "k_dequant": ("ldlq.cuh", "449a391e49fc", 26102272),
     "k_row_grid": ("ldlq.cuh", "449a391e49fc", 67615488),
     "k_split_upper_transposed": ("gemm_tc.cuh", "92453856d596", 148098048),
-    "k_gemm_split_tc[ldl]": ("gemm_tc.cuh", "92453856d596", 28437248),
+    "k_gemm_split_tc[ldl]": ("gemm_tc.cuh", "4a73f99d9186", 28432128),
     "k_fwht_cols": ("fwht.cuh", "94ad670265cc", 82387456),
+    "k_greedy_start": ("rounding.cuh", "d4ef99d9fa8b", 263645696),
+    "k_greedy_factors": ("rounding.cuh", "d4ef99d9fa8b", 229122560),
 }
 TRAFFIC_WORKLOAD = "attn7b"
 
@@ -344,9 +367,14 @@ def run_reference(args, cfg: LayerConfig):
 def config_desc(cfg: LayerConfig, args):
     side = lambda s: (s.kind if s.kind != "kronecker" else f"kronecker {s.p}x{s.q}") + \
         (" with random permutation" if getattr(s, "permute", False) else "")
+    method = getattr(args, "method", "ldlq")
+    passes = getattr(args, "passes", 1)
+    rounding = {"ldlq": f"LDLQ block {cfg.block}", "nearest": "nearest rounding",
+                "greedy": f"Greedy ({passes} passes)",
+                "ldlq_rg": f"LDLQ-RG (block {cfg.block}, {passes} greedy passes)"}[method]
     return {
         "workload": f"{cfg.name}: W {cfg.m}x{cfg.n} {cfg.dtype}, X {cfg.N}x{cfg.n} {cfg.dtype}, "
-                    f"U {side(cfg.m_side)}, V {side(cfg.n_side)}, LDLQ block {cfg.block}, {cfg.bits}-bit",
+                    f"U {side(cfg.m_side)}, V {side(cfg.n_side)}, {rounding}, {cfg.bits}-bit",
         "m": cfg.m, "n": cfg.n, "tokens": cfg.N, "bits": cfg.bits, "block": cfg.block,
         "damp": cfg.damp, "l2": "flushed before every timed step (256 MB write)",
         "parallelism": f"replicas x{args.gpus} (one layer per GPU)",
@@ -374,7 +402,7 @@ def run_ours(args, cfg: LayerConfig):
     W = W_h.cuda()
     X = X_h.cuda()
     q = Q.LayerQuantizer(cfg.m, cfg.n, cfg.m_side, cfg.n_side, cfg.bits, cfg.block, cfg.damp,
-                         rcfg.seed)
+                         rcfg.seed, method=args.method, passes=args.passes)
     stream = torch.cuda.current_stream()
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")   # 256 MB > L2
 
@@ -389,9 +417,14 @@ def run_ours(args, cfg: LayerConfig):
         mark(3)
         Q.quip_incoherence_forward(q.tf, W, q.W_t, q.H, q.ws)
         mark(4)
-        Q.quip_ldl(q.H, q.D, q.ws)
-        mark(5)
-        Q.quip_ldlq_quantize(q.W_t, q.H, cfg.bits, cfg.block, q.codes, q.lo, q.scale, q.ws)
+        if args.method == "ldlq":
+            Q.quip_ldl(q.H, q.D, q.ws)
+            mark(5)
+            Q.quip_ldlq_quantize(q.W_t, q.H, cfg.bits, cfg.block, q.codes, q.lo, q.scale, q.ws)
+        else:
+            q.prepare_hessian()
+            mark(5)
+            q.round_weights()
         mark(6)
         Q.quip_dequantize(q.codes, q.lo, q.scale, q.W_hat)
         mark(7)
@@ -472,8 +505,11 @@ def run_ours(args, cfg: LayerConfig):
     for i, name in enumerate(STAGES):
         ms = statistics.mean(stage_ms[i])
         kind, amount, bound = work[name]
+        if args.method != "ldlq" and name in ("ldl", "ldlq"):
+            stages[name] = {"ms": round(ms, 4)}      # the method's own kernels: see "kernels"
+            continue
         stages[name] = {"ms": round(ms, 4), **roofline_entry(kind, amount, bound, ms, pk)}
-    kwork = kernel_work(cfg)
+    kwork = kernel_work(cfg, args.method, args.passes)
     kernels = {}
     for name, (cnt, tot_ms) in per_kernel.items():
         ent = {"launches_per_step": cnt / args.steps, "ms_per_step": round(tot_ms / args.steps, 4)}
@@ -585,6 +621,9 @@ def main():
                     help="layers of the config's shape sharing one input (one Hessian and LDL)")
     ap.add_argument("--permute", action="store_true",
                     help="random permutation within both sides' orthogonal transforms")
+    ap.add_argument("--method", default="ldlq", choices=["ldlq", "nearest", "greedy", "ldlq_rg"],
+                    help="rounding method (QuIP, Experiments, Methods)")
+    ap.add_argument("--passes", type=int, default=1, help="greedy passes of greedy / ldlq_rg")
     args = ap.parse_args()
     cfg = CONFIGS[args.config]
     if args.permute:
@@ -595,6 +634,8 @@ def main():
         run_reference(args, cfg)
     else:
         if args.group > 1:
+            if args.method != "ldlq":
+                raise SystemExit("--group runs LDLQ only")
             run_group(args, cfg)
         else:
             run_ours(args, cfg)

@@ -59,7 +59,7 @@ typedef enum {
   QUIP_ERR_WORKSPACE = 8     /* ws too small or misaligned                   */
 } quip_status;
 
-typedef enum { QUIP_F32 = 0, QUIP_BF16 = 1 } quip_dtype;
+typedef enum { QUIP_F32 = 0, QUIP_BF16 = 1, QUIP_U8 = 2 } quip_dtype;
 
 /* Kind of random orthogonal matrix on one side of W. */
 typedef enum {
@@ -81,7 +81,8 @@ typedef enum {
   QUIP_OP_INCOHERENCE_FORWARD = 0,
   QUIP_OP_INCOHERENCE_INVERSE = 1,
   QUIP_OP_LDL = 2,
-  QUIP_OP_LDLQ = 3
+  QUIP_OP_LDLQ = 3,
+  QUIP_OP_GREEDY = 4
 } quip_op;
 
 typedef struct quip_transform quip_transform;   /* opaque, library-owned */
@@ -271,13 +272,75 @@ quip_status quip_ldlq_quantize_static(const float* W_t, const float* Uring, int6
                                       int64_t m, int64_t n, int bits, int64_t block,
                                       uint8_t* codes, float* lo, float* scale, void* stream);
 
+/*
+ * Nearest rounding (QuIP, Experiments, "Methods.": the nearest-rounding
+ * baseline) on the per-row grid of quip_ldlq_quantize:
+ *   lo, scale as there; codes[i,j] = clamp(rint((W_t[i,j] - lo_i) / s_i), 0, 2^bits - 1)
+ * with the same fp32 steps as LDLQ's rounding (the quotient is formed as
+ * (W_t - lo) * (1 / s)).  W_t: device m x n fp32, row stride n; codes:
+ * device m x n uint8; lo, scale: device m fp32.  bits 1..8.
+ */
+quip_status quip_nearest_quantize(const float* W_t, int64_t m, int64_t n, int bits,
+                                  uint8_t* codes, float* lo, float* scale, void* stream);
+
+/*
+ * LDLQ-RG's quantisation order (QuIP, Experiments, "Methods.": LDLQ-RG
+ * re-orders the weights by diag(H)): perm[r] = the index k with the r-th
+ * largest H[k,k] (equal values by increasing k; -0 counts as +0; where a
+ * NaN goes is unspecified), iperm[perm[r]] = r.
+ *   H     : device, n x n fp32, row stride ldh; only the diagonal is read.
+ *   perm  : device n int32;  iperm: device n int32, or NULL.
+ * n <= 65536.
+ */
+quip_status quip_diag_order(const float* H, int64_t ldh, int64_t n, int32_t* perm, int32_t* iperm,
+                            void* stream);
+
+/*
+ * Gather out[r,c] = in[row_perm[r], col_perm[c]] (device; rows x cols,
+ * row strides ldin / ldout elements; a NULL list is the identity), for
+ * dtype QUIP_F32, QUIP_BF16 or QUIP_U8 (in and out of the same type, bits
+ * copied unchanged).  With perm from quip_diag_order, col_perm = perm puts
+ * a matrix's columns in the quantisation order and col_perm = iperm puts
+ * them back.  in and out must not overlap.  An index outside
+ * [0, rows) / [0, cols) writes 0 there and sets QUIP_ERR_ARG in the status
+ * word (quip_sync_status).
+ */
+quip_status quip_permute(const void* in, int dtype, int64_t rows, int64_t cols, int64_t ldin,
+                         const int32_t* row_perm, const int32_t* col_perm, void* out, int64_t ldout,
+                         void* stream);
+
+/*
+ * Greedy updates of the proxy tr((W^ - W_t) H (W^ - W_t)^T) (QuIP,
+ * Experiments, "Methods.": "Greedy" performs them alone, LDLQ-RG after
+ * LDLQ), `passes` passes.  A pass visits k = 0..n-1 and, every other column
+ * held at its current value, sets
+ *   codes[:,k] = clamp(rint((t_k - lo) / s), 0, 2^bits - 1),
+ *   t_k = W_t[:,k] - sum_{j != k} (W^[:,j] - W_t[:,j]) H[j,k] / H[k,k],
+ * W^ = lo + s codes: per row, the grid point that minimises the proxy over
+ * column k.  Evaluated in fp32 (tensor-core GEMMs on three bf16 pieces for
+ * the long sums, as LDLQ's); the grid (lo, scale) is not changed.
+ *   W_t   : device m x n fp32 (row stride n, 16-byte aligned), not modified.
+ *   H     : device n x n fp32, symmetric with a positive diagonal, row stride
+ *           ldh >= n; only the upper triangle (j <= k) is read.
+ *   lo, scale : device m fp32 (e.g. from quip_ldlq_quantize).
+ *   codes : device m x n uint8 (row stride n, 16-byte aligned), in: the
+ *           starting codes, out: the codes after the passes.
+ * n % 64 == 0, n <= 65536, m <= 2^20, bits 1..8, passes >= 0 (0: nothing
+ * is done).  To visit the columns in another order, permute W_t's columns
+ * and H's rows and columns first (quip_permute).  ws: QUIP_OP_GREEDY.
+ */
+quip_status quip_greedy_refine(const float* W_t, const float* H, int64_t ldh, int64_t m, int64_t n,
+                               int bits, const float* lo, const float* scale, uint8_t* codes,
+                               int passes, void* ws, size_t ws_bytes, void* stream);
+
 /* W_hat_t[i,j] = lo[i] + scale[i] * codes[i,j]  (device; m x n, row stride n). */
 quip_status quip_dequantize(const uint8_t* codes, const float* lo, const float* scale,
                             int64_t m, int64_t n, float* W_hat_t, void* stream);
 
 /*
  * Bytes of workspace `op` needs (quip_op).  tf is required for the
- * incoherence ops and ignored otherwise; block is used by QUIP_OP_LDLQ.
+ * incoherence ops and ignored otherwise; block is used by QUIP_OP_LDLQ;
+ * QUIP_OP_GREEDY takes m and n.
  * *bytes may be 0.
  */
 quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int64_t n,

@@ -21,12 +21,18 @@ from ._lib import QuipError, load, status_string  # noqa: F401
 __all__ = [
     "Transform", "quip_hessian_accumulate", "quip_hessian_finalize", "quip_incoherence_forward",
     "quip_incoherence_inverse", "quip_ldl", "quip_ldlq_quantize", "quip_dequantize",
+    "quip_nearest_quantize", "quip_diag_order", "quip_permute", "quip_greedy_refine", "METHODS",
     "quip_workspace_size", "quip_sync_status", "quip_timing_begin", "quip_timing_end", "LayerQuantizer",
     "LayerGroupQuantizer", "quantize_layer", "QuipError",
     "KIND",
 ]
 
 KIND = {"identity": L.QUIP_T_IDENTITY, "hadamard": L.QUIP_T_HADAMARD, "kronecker": L.QUIP_T_KRONECKER}
+
+# Rounding methods of the QuIP paper, Experiments, "Methods.": nearest
+# rounding; LDLQ; "Greedy" (nearest, then greedy passes over the proxy);
+# LDLQ-RG (columns by decreasing diag(H~), LDLQ in that order, greedy passes).
+METHODS = ("ldlq", "nearest", "greedy", "ldlq_rg")
 
 
 def _kind(side) -> int:
@@ -207,6 +213,45 @@ def quip_ldlq_quantize(W_t: torch.Tensor, Uring: torch.Tensor, bits: int, block:
                                       _s(stream)), "quip_ldlq_quantize")
 
 
+def quip_nearest_quantize(W_t: torch.Tensor, bits: int, codes: torch.Tensor, lo: torch.Tensor,
+                          scale: torch.Tensor, stream=None) -> None:
+    m, n = W_t.shape
+    L.check(load().quip_nearest_quantize(_p(W_t), m, n, bits, _p(codes), _p(lo), _p(scale), _s(stream)),
+            "quip_nearest_quantize")
+
+
+def quip_diag_order(H: torch.Tensor, perm: torch.Tensor, iperm: Optional[torch.Tensor] = None,
+                    stream=None) -> None:
+    _cuda(H, "H")
+    L.check(load().quip_diag_order(_p(H), H.stride(0), H.shape[0], _p(perm), _p(iperm), _s(stream)),
+            "quip_diag_order")
+
+
+_PERM_DTYPE = {torch.float32: L.QUIP_F32, torch.bfloat16: L.QUIP_BF16, torch.uint8: L.QUIP_U8}
+
+
+def quip_permute(inp: torch.Tensor, out: torch.Tensor, row_perm: Optional[torch.Tensor] = None,
+                 col_perm: Optional[torch.Tensor] = None, stream=None) -> None:
+    """out[r, c] = inp[row_perm[r], col_perm[c]] (None: identity)."""
+    if inp.dtype != out.dtype or inp.dtype not in _PERM_DTYPE:
+        raise TypeError(f"unsupported dtypes {inp.dtype} -> {out.dtype}")
+    rows, cols = inp.shape
+    L.check(load().quip_permute(_p(inp), _PERM_DTYPE[inp.dtype], rows, cols, inp.stride(0), _p(row_perm),
+                                _p(col_perm), _p(out), out.stride(0), _s(stream)), "quip_permute")
+
+
+def quip_greedy_refine(W_t: torch.Tensor, H: torch.Tensor, bits: int, lo: torch.Tensor,
+                       scale: torch.Tensor, codes: torch.Tensor, passes: int = 1,
+                       ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    m, n = W_t.shape
+    need = quip_workspace_size(L.QUIP_OP_GREEDY, None, m, n)
+    if ws is None:
+        ws = _ws(need, W_t.device)
+    L.check(load().quip_greedy_refine(_p(W_t), _p(H), H.stride(0), m, n, bits, _p(lo), _p(scale),
+                                      _p(codes), passes, _p(ws), 0 if ws is None else ws.numel(),
+                                      _s(stream)), "quip_greedy_refine")
+
+
 def quip_dequantize(codes: torch.Tensor, lo: torch.Tensor, scale: torch.Tensor, W_hat_t: torch.Tensor,
                     stream=None) -> None:
     m, n = codes.shape
@@ -243,14 +288,20 @@ class LayerResult:
 
 class LayerQuantizer:
     """Buffers and transform for quantising one m x n layer; ``run`` issues the
-    whole pipeline on one stream through the C ABI."""
+    whole pipeline on one stream through the C ABI.  ``method`` is one of
+    METHODS; ``passes`` is the number of greedy passes of "greedy" and
+    "ldlq_rg"."""
 
     X_CHUNKS = 4            # token chunks of X in run_host (copy / Hessian overlap)
 
     def __init__(self, m: int, n: int, m_side, n_side, bits: int, block: int, damp: float = 0.01,
-                 seed: int = 0, device: str = "cuda", stream=None):
+                 seed: int = 0, device: str = "cuda", stream=None, method: str = "ldlq",
+                 passes: int = 1):
+        if method not in METHODS:
+            raise ValueError(f"method must be one of {METHODS}")
         self.m, self.n, self.bits, self.block, self.damp, self.seed = m, n, bits, block, damp, seed
         self.m_side, self.n_side = m_side, n_side
+        self.method, self.passes = method, passes
         self.stream = stream
         dev = torch.device(device)
         f32 = dict(dtype=torch.float32, device=dev)
@@ -262,10 +313,20 @@ class LayerQuantizer:
         self.scale = torch.empty(m, **f32)
         self.W_hat = torch.empty(m, n, **f32)
         self.tf: Optional[Transform] = None
+        if method == "ldlq_rg":
+            # the re-ordered problem: H~ and W~ with columns (and H~'s rows) in
+            # the quantisation order, the codes in that order, the order itself
+            self.Hp = torch.empty(n, n, **f32)
+            self.Wp = torch.empty(m, n, **f32)
+            self.codes_p = torch.empty(m, n, dtype=torch.uint8, device=dev)
+            self.perm = torch.empty(n, dtype=torch.int32, device=dev)
+            self.iperm = torch.empty(n, dtype=torch.int32, device=dev)
         ws = 0
         probe = Transform(seed, m, n, m_side, n_side, stream)
         for op, blk in ((L.QUIP_OP_INCOHERENCE_FORWARD, 0), (L.QUIP_OP_INCOHERENCE_INVERSE, 0),
-                        (L.QUIP_OP_LDL, 0), (L.QUIP_OP_LDLQ, block)):
+                        (L.QUIP_OP_LDL, 0), (L.QUIP_OP_LDLQ, block), (L.QUIP_OP_GREEDY, 0)):
+            if op == L.QUIP_OP_GREEDY and method not in ("greedy", "ldlq_rg"):
+                continue
             ws = max(ws, quip_workspace_size(op, probe, m, n, blk))
         self.tf = probe
         self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
@@ -295,17 +356,50 @@ class LayerQuantizer:
             quip_hessian_accumulate(X, self.H, False, st)
         quip_hessian_finalize(self.H, X.shape[0], self.damp, st)
         quip_incoherence_forward(self.tf, None, None, self.H, self.ws, st)
-        quip_ldl(self.H, self.D, self.ws, st)
+        self.prepare_hessian()
         if w_ready is not None:
             stream.wait_event(w_ready)
         quip_incoherence_forward(self.tf, W, self.W_t, None, self.ws, st)
-        quip_ldlq_quantize(self.W_t, self.H, self.bits, self.block, self.codes, self.lo, self.scale,
-                           self.ws, st)
+        self.round_weights()
         if after_ldlq is not None:
             after_ldlq()
         quip_dequantize(self.codes, self.lo, self.scale, self.W_hat, st)
         quip_incoherence_inverse(self.tf, self.W_hat, self.W_hat, self.ws, st)
         return LayerResult(self.codes, self.lo, self.scale, self.W_hat)
+
+    def prepare_hessian(self) -> None:
+        """What the method needs from H~ (in self.H) before W~ exists: the LDL
+        for "ldlq"; for "ldlq_rg" the order by diag(H~) and the LDL of the
+        re-ordered H~ (in self.Hp; self.H is left as it is)."""
+        st = self.stream
+        if self.method == "ldlq_rg":
+            quip_diag_order(self.H, self.perm, self.iperm, st)
+            quip_permute(self.H, self.Hp, self.perm, self.perm, st)
+            quip_ldl(self.Hp, self.D, self.ws, st)
+        elif self.method == "ldlq":
+            quip_ldl(self.H, self.D, self.ws, st)
+
+    def round_weights(self) -> None:
+        """Codes and grid of W~ (in self.W_t) by the layer's method."""
+        st, method = self.stream, self.method
+        if method == "ldlq":
+            quip_ldlq_quantize(self.W_t, self.H, self.bits, self.block, self.codes, self.lo,
+                               self.scale, self.ws, st)
+        elif method in ("nearest", "greedy"):
+            quip_nearest_quantize(self.W_t, self.bits, self.codes, self.lo, self.scale, st)
+            if method == "greedy":
+                quip_greedy_refine(self.W_t, self.H, self.bits, self.lo, self.scale, self.codes,
+                                   self.passes, self.ws, st)
+        else:
+            quip_permute(self.W_t, self.Wp, None, self.perm, st)
+            quip_ldlq_quantize(self.Wp, self.Hp, self.bits, self.block, self.codes_p, self.lo,
+                               self.scale, self.ws, st)
+            if self.passes > 0:
+                # the LDL overwrote Hp: gather the re-ordered H~ again
+                quip_permute(self.H, self.Hp, self.perm, self.perm, st)
+                quip_greedy_refine(self.Wp, self.Hp, self.bits, self.lo, self.scale, self.codes_p,
+                                   self.passes, self.ws, st)
+            quip_permute(self.codes_p, self.codes, None, self.iperm, st)
 
     def run_host(self, W_host: torch.Tensor, X_host: torch.Tensor, codes_out: torch.Tensor,
                  lo_out: torch.Tensor, scale_out: torch.Tensor) -> None:
@@ -410,9 +504,10 @@ class LayerGroupQuantizer:
 
 
 def quantize_layer(W: torch.Tensor, X: torch.Tensor, m_side, n_side, bits: int, block: int,
-                   damp: float = 0.01, seed: int = 0) -> LayerResult:
+                   damp: float = 0.01, seed: int = 0, method: str = "ldlq", passes: int = 1) -> LayerResult:
     """Quantise one layer from host (or device) tensors; results come back to the host."""
-    q = LayerQuantizer(W.shape[0], W.shape[1], m_side, n_side, bits, block, damp, seed)
+    q = LayerQuantizer(W.shape[0], W.shape[1], m_side, n_side, bits, block, damp, seed,
+                       method=method, passes=passes)
     Wd = W.to("cuda", non_blocking=True)
     Xd = X.to("cuda", non_blocking=True)
     r = q.run(Wd, Xd)

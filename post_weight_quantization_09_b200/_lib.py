@@ -11,10 +11,11 @@ LIB_PATH = os.path.join(HERE, "libquip.so")
 
 QUIP_OK, QUIP_ERR_ARG, QUIP_ERR_SHAPE, QUIP_ERR_UNSUPPORTED = 0, 1, 2, 3
 QUIP_ERR_NOT_PD, QUIP_ERR_NONFINITE, QUIP_ERR_CUDA, QUIP_ERR_TIMEOUT, QUIP_ERR_WORKSPACE = 4, 5, 6, 7, 8
-QUIP_F32, QUIP_BF16 = 0, 1
+QUIP_F32, QUIP_BF16, QUIP_U8 = 0, 1, 2
 QUIP_T_IDENTITY, QUIP_T_HADAMARD, QUIP_T_KRONECKER = 0, 1, 2
 QUIP_T_PERMUTE = 0x100
 QUIP_OP_INCOHERENCE_FORWARD, QUIP_OP_INCOHERENCE_INVERSE, QUIP_OP_LDL, QUIP_OP_LDLQ = 0, 1, 2, 3
+QUIP_OP_GREEDY = 4
 
 # name -> (restype, argtypes); the list of every symbol include/quip.h declares
 SIGNATURES = {
@@ -40,6 +41,13 @@ SIGNATURES = {
                                    c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "quip_ldlq_quantize_static": (c_int, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int,
                                           c_int64, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "quip_nearest_quantize": (c_int, [c_void_p, c_int64, c_int64, c_int, c_void_p, c_void_p, c_void_p,
+                                      c_void_p]),
+    "quip_diag_order": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p]),
+    "quip_permute": (c_int, [c_void_p, c_int, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
+                             c_int64, c_void_p]),
+    "quip_greedy_refine": (c_int, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int, c_void_p,
+                                   c_void_p, c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
     "quip_dequantize": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
     "quip_workspace_size": (c_int, [c_int, c_void_p, c_int64, c_int64, c_int64, POINTER(c_size_t)]),
     "quip_sync_status": (c_int, [c_void_p]),

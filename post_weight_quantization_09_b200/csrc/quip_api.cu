@@ -17,6 +17,7 @@
 #include "ldl.cuh"
 #include "ldlq.cuh"
 #include "rng.cuh"
+#include "rounding.cuh"
 #include "syrk_tc.cuh"
 #include "gemm_tc.cuh"
 
@@ -471,9 +472,35 @@ __global__ void __launch_bounds__(256) k_gather2d(const TIn* __restrict__ in, in
   }
 }
 
+// Row gather with the source row staged in shared memory (k_permute_staged),
+// for rows of at most PERMUTE_STAGE_MAX bytes.
+template <typename TIn, typename TOut>
+cudaError_t permute_staged(const TIn* in, int64_t ldin, TOut* out, int64_t ldout, int64_t rows,
+                           int64_t cols, const int32_t* rp, const int32_t* cp, cudaStream_t st,
+                           const char* name) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_permute_staged<TIn, TOut>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)PERMUTE_STAGE_MAX);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int64_t row_bytes = cols * (int64_t)sizeof(TIn);
+  const size_t smem = (size_t)((row_bytes + 15) / 16 * 16);
+  const int vec = (row_bytes % 16 == 0) && ((ldin * (int64_t)sizeof(TIn)) % 16 == 0) &&
+                  (reinterpret_cast<uintptr_t>(in) & 15) == 0;
+  const unsigned grid = (unsigned)std::min<int64_t>(rows, (int64_t)num_sms() * 8);
+  LaunchScope ls(name, st);
+  k_permute_staged<TIn, TOut><<<grid, 256, smem, st>>>(in, ldin, out, ldout, rows, cols, vec, rp, cp);
+  return cudaGetLastError();
+}
+
 template <typename TIn>
 cudaError_t gather2d(const TIn* in, int64_t ldin, float* out, int64_t ldout, int64_t rows,
                      int64_t cols, const int32_t* rp, const int32_t* cp, cudaStream_t st) {
+  if (cols * (int64_t)sizeof(TIn) <= PERMUTE_STAGE_MAX)
+    return permute_staged<TIn, float>(in, ldin, out, ldout, rows, cols, rp, cp, st, "k_gather2d");
   const unsigned gx = (unsigned)std::min<int64_t>((cols + 1023) / 1024, 64);
   const unsigned gy = (unsigned)std::min<int64_t>(rows, 65535);
   LaunchScope ls("k_gather2d", st);
@@ -722,6 +749,13 @@ static size_t ldlq_ws_bytes(int64_t m, int64_t n, int64_t block) {
          round256((size_t)3 * n * n * 2) + round256((size_t)n * n * 4);
 }
 
+// Greedy workspace: the LDLQ run's buffers (accumulator, error pieces, the
+// transposed factor in pieces and in fp32) plus the factor U' (n x n fp32)
+// and the pass's starting W^ (m x n fp32).
+static size_t greedy_ws_bytes(int64_t m, int64_t n) {
+  return ldlq_ws_bytes(m, n, 128) + round256((size_t)n * n * 4) + round256((size_t)m * n * 4);
+}
+
 // Transform workspace: Kronecker temporaries, then the permutation scratch
 // (the forward pass gathers H into it, the inverse gathers W^).
 static size_t transform_kron_bytes(const quip_transform* tf, int op) {
@@ -756,6 +790,10 @@ quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int
     case QUIP_OP_LDLQ:
       if (m <= 0 || n <= 0 || block <= 0) return QUIP_ERR_SHAPE;
       *bytes = ldlq_ws_bytes(m, n, block);
+      return QUIP_OK;
+    case QUIP_OP_GREEDY:
+      if (m <= 0 || n <= 0) return QUIP_ERR_SHAPE;
+      *bytes = greedy_ws_bytes(m, n);
       return QUIP_OK;
     default:
       return QUIP_ERR_ARG;
@@ -963,6 +1001,32 @@ cudaError_t ldlq_block(const LdlqRun& r, int64_t k0, int w) {
                     r.tband, r.tw, r.m, r.n, k0, w, r.lo, r.sc, r.qmax, r.codes, r.Es, r.n);
 }
 
+// Tensor maps of a run: the block kernel's (accumulator, weights, the
+// transposed factor UTf, the factor's band) and, with gemm, the split
+// GEMMs' (errors Es as A; UTs, the transposed factor's bf16 pieces, as B in
+// 256-, 128- and 64-row boxes).
+bool ldlq_maps(LdlqRun& r, const float* UTf, const __nv_bfloat16* UTs, bool gemm) {
+  const uint64_t m = (uint64_t)r.m, n = (uint64_t)r.n;
+  if (!make_tmap_f32_2d(&r.tacc, r.A, n, m, n * 4, LQB_S, LQB_ROWS) ||
+      !make_tmap_f32_2d(&r.tw, r.Wt, n, m, n * 4, LQB_S, LQB_ROWS) ||
+      !make_tmap_f32_2d(&r.tut, UTf, n, n, n * 4, LQB_S, 128) ||
+      !make_tmap_f32_2d(&r.tband, r.U, n, n, (uint64_t)r.ldu * 4, 32, 16))
+    return false;
+  if (!gemm) return true;
+  return make_tmap_bf16_2d(&r.ta, r.Es, n, 3 * m, n * 2, 64, sgemm::BM) &&
+         make_tmap_bf16_2d(&r.tb, UTs, n, 3 * n, n * 2, 64, sgemm::BN) &&
+         make_tmap_bf16_2d(&r.tb64, UTs, n, 3 * n, n * 2, 64, 64) &&
+         make_tmap_bf16_2d(&r.tb128, UTs, n, 3 * n, n * 2, 64, 128);
+}
+
+void ldlq_block_attr() {
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(k_ldlq_block, cudaFuncAttributeMaxDynamicSharedMemorySize, LQB_SMEM);
+    attr = true;
+  }
+}
+
 // Columns [a, b): left half, then A[:, mid:b] += Err[:, a:mid] Ů[a:mid, mid:b]
 // in one split GEMM, then the right half.  Every column's feedback is the
 // same sum as in the column-by-column definition, grouped differently.
@@ -1020,24 +1084,152 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
     LaunchScope ls("k_split_upper_transposed", r.st);
     k_split_upper_transposed<<<dim3(T, T), 256, 0, r.st>>>(Uring, ldu, n, UTs, UTf);
   }
-  if (!make_tmap_f32_2d(&r.tacc, r.A, (uint64_t)n, (uint64_t)m, (uint64_t)n * 4, LQB_S, LQB_ROWS) ||
-      !make_tmap_f32_2d(&r.tw, W_t, (uint64_t)n, (uint64_t)m, (uint64_t)n * 4, LQB_S, LQB_ROWS) ||
-      !make_tmap_f32_2d(&r.tut, UTf, (uint64_t)n, (uint64_t)n, (uint64_t)n * 4, LQB_S, 128) ||
-      !make_tmap_f32_2d(&r.tband, Uring, (uint64_t)n, (uint64_t)n, (uint64_t)ldu * 4, 32, 16))
-    return QUIP_ERR_CUDA;
-  if (n > LDQ_BLK) {
-    if (!make_tmap_bf16_2d(&r.ta, r.Es, (uint64_t)n, 3 * (uint64_t)m, (uint64_t)n * 2, 64, sgemm::BM) ||
-        !make_tmap_bf16_2d(&r.tb, UTs, (uint64_t)n, 3 * (uint64_t)n, (uint64_t)n * 2, 64, sgemm::BN) ||
-        !make_tmap_bf16_2d(&r.tb64, UTs, (uint64_t)n, 3 * (uint64_t)n, (uint64_t)n * 2, 64, 64) ||
-        !make_tmap_bf16_2d(&r.tb128, UTs, (uint64_t)n, 3 * (uint64_t)n, (uint64_t)n * 2, 64, 128))
-      return QUIP_ERR_CUDA;
-  }
-  static bool attr = false;
-  if (!attr) {
-    QCHECK(cudaFuncSetAttribute(k_ldlq_block, cudaFuncAttributeMaxDynamicSharedMemorySize, LQB_SMEM));
-    attr = true;
-  }
+  if (!ldlq_maps(r, UTf, UTs, n > LDQ_BLK)) return QUIP_ERR_CUDA;
+  ldlq_block_attr();
   QCHECK(ldlq_range(r, 0, n));
+  return QUIP_OK;
+}
+
+quip_status quip_nearest_quantize(const float* W_t, int64_t m, int64_t n, int bits, uint8_t* codes,
+                                  float* lo, float* scale, void* stream) {
+  if (!W_t || !codes || !lo || !scale) return QUIP_ERR_ARG;
+  if (bits < 1 || bits > 8) return QUIP_ERR_ARG;
+  if (m <= 0 || n <= 0) return QUIP_ERR_SHAPE;
+  cudaStream_t st = S(stream);
+  {
+    LaunchScope ls("k_row_grid", st);
+    k_row_grid<<<(unsigned)((m + 7) / 8), 256, 0, st>>>(W_t, m, n, (1 << bits) - 1, lo, scale);
+  }
+  const int vec = (n & 3) == 0 && (reinterpret_cast<uintptr_t>(codes) & 3) == 0 &&
+                  (reinterpret_cast<uintptr_t>(W_t) & 15) == 0;
+  const int64_t per_cta = (vec ? 4 : 1) * (int64_t)NR_THREADS;
+  const unsigned gx = (unsigned)std::min<int64_t>((n + per_cta - 1) / per_cta, 1024);
+  const unsigned gy = (unsigned)std::min<int64_t>(m, 65535);
+  {
+    LaunchScope ls("k_nearest", st);
+    k_nearest<<<dim3(gx, gy), NR_THREADS, 0, st>>>(W_t, lo, scale, m, n, vec,
+                                                    (float)((1 << bits) - 1), codes);
+  }
+  QCHECK(cudaGetLastError());
+  return QUIP_OK;
+}
+
+quip_status quip_diag_order(const float* H, int64_t ldh, int64_t n, int32_t* perm, int32_t* iperm,
+                            void* stream) {
+  if (!H || !perm) return QUIP_ERR_ARG;
+  if (n <= 0 || n > 65536 || ldh < n) return QUIP_ERR_SHAPE;
+  cudaStream_t st = S(stream);
+  {
+    LaunchScope ls("k_diag_rank", st);
+    k_diag_rank<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(H, ldh, n, perm, iperm);
+  }
+  QCHECK(cudaGetLastError());
+  return QUIP_OK;
+}
+
+quip_status quip_permute(const void* in, int dtype, int64_t rows, int64_t cols, int64_t ldin,
+                         const int32_t* row_perm, const int32_t* col_perm, void* out, int64_t ldout,
+                         void* stream) {
+  if (!in || !out) return QUIP_ERR_ARG;
+  if (rows <= 0 || cols <= 0 || ldin < cols || ldout < cols) return QUIP_ERR_SHAPE;
+  if (rows > INT32_MAX || cols > INT32_MAX) return QUIP_ERR_SHAPE;
+  size_t es = 0;
+  if (dtype == QUIP_F32) es = 4;
+  else if (dtype == QUIP_BF16) es = 2;
+  else if (dtype == QUIP_U8) es = 1;
+  else return QUIP_ERR_ARG;
+  // the two arrays may not overlap
+  const char* a = static_cast<const char*>(in);
+  const char* b = static_cast<const char*>(out);
+  const size_t ea = es * (size_t)((rows - 1) * ldin + cols), eb = es * (size_t)((rows - 1) * ldout + cols);
+  if (a < b + eb && b < a + ea) return QUIP_ERR_ARG;
+  cudaStream_t st = S(stream);
+  if (cols * (int64_t)es <= PERMUTE_STAGE_MAX) {
+    cudaError_t e;
+    if (es == 4)
+      e = permute_staged(static_cast<const uint32_t*>(in), ldin, static_cast<uint32_t*>(out), ldout, rows,
+                         cols, row_perm, col_perm, st, "k_permute");
+    else if (es == 2)
+      e = permute_staged(static_cast<const uint16_t*>(in), ldin, static_cast<uint16_t*>(out), ldout, rows,
+                         cols, row_perm, col_perm, st, "k_permute");
+    else
+      e = permute_staged(static_cast<const uint8_t*>(in), ldin, static_cast<uint8_t*>(out), ldout, rows,
+                         cols, row_perm, col_perm, st, "k_permute");
+    QCHECK(e);
+    return QUIP_OK;
+  }
+  const unsigned gx = (unsigned)std::min<int64_t>((cols + 255) / 256, 64);
+  const unsigned gy = (unsigned)std::min<int64_t>(rows, 65535);
+  LaunchScope ls("k_permute", st);
+  if (es == 4)
+    k_permute<uint32_t><<<dim3(gx, gy), 256, 0, st>>>(static_cast<const uint32_t*>(in), ldin,
+                                                       static_cast<uint32_t*>(out), ldout, rows, cols,
+                                                       row_perm, col_perm);
+  else if (es == 2)
+    k_permute<uint16_t><<<dim3(gx, gy), 256, 0, st>>>(static_cast<const uint16_t*>(in), ldin,
+                                                       static_cast<uint16_t*>(out), ldout, rows, cols,
+                                                       row_perm, col_perm);
+  else
+    k_permute<uint8_t><<<dim3(gx, gy), 256, 0, st>>>(static_cast<const uint8_t*>(in), ldin,
+                                                      static_cast<uint8_t*>(out), ldout, rows, cols,
+                                                      row_perm, col_perm);
+  QCHECK(cudaGetLastError());
+  return QUIP_OK;
+}
+
+quip_status quip_greedy_refine(const float* W_t, const float* H, int64_t ldh, int64_t m, int64_t n,
+                               int bits, const float* lo, const float* scale, uint8_t* codes,
+                               int passes, void* ws, size_t ws_bytes, void* stream) {
+  if (!W_t || !H || !lo || !scale || !codes) return QUIP_ERR_ARG;
+  if (bits < 1 || bits > 8 || passes < 0) return QUIP_ERR_ARG;
+  if (m <= 0 || n <= 0 || ldh < n) return QUIP_ERR_SHAPE;
+  if (n % 64) return QUIP_ERR_SHAPE;
+  if (m > ((int64_t)1 << 20) || n > ((int64_t)1 << 16)) return QUIP_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(W_t) & 15) || (reinterpret_cast<uintptr_t>(codes) & 15))
+    return QUIP_ERR_ARG;
+  quip_status s = check_ws(ws, ws_bytes, greedy_ws_bytes(m, n));
+  if (s != QUIP_OK) return s;
+  if (passes == 0) return QUIP_OK;
+  cudaStream_t st = S(stream);
+  char* w8 = static_cast<char*>(ws);
+  LdlqRun r{};
+  r.st = st;
+  r.A = reinterpret_cast<float*>(w8);
+  w8 += round256((size_t)m * n * 4);
+  r.Es = reinterpret_cast<__nv_bfloat16*>(w8);
+  w8 += round256((size_t)3 * m * n * 2);
+  __nv_bfloat16* UTs = reinterpret_cast<__nv_bfloat16*>(w8);
+  w8 += round256((size_t)3 * n * n * 2);
+  float* UTf = reinterpret_cast<float*>(w8);
+  w8 += round256((size_t)n * n * 4);
+  float* Ur = reinterpret_cast<float*>(w8);
+  w8 += round256((size_t)n * n * 4);
+  float* What = reinterpret_cast<float*>(w8);
+  r.Wt = What, r.U = Ur, r.ldu = n, r.m = m, r.n = n, r.lo = lo, r.sc = scale;
+  r.qmax = (float)((1 << bits) - 1), r.codes = codes;
+  {
+    const unsigned T = (unsigned)(n / 32);
+    LaunchScope ls("k_greedy_factors", st);
+    k_greedy_factors<<<dim3(T, T), 256, 0, st>>>(H, ldh, n, UTf, UTs, Ur);
+  }
+  if (!ldlq_maps(r, UTf, UTs, true)) return QUIP_ERR_CUDA;
+  ldlq_block_attr();
+  const unsigned gx = (unsigned)std::min<int64_t>((n + 1023) / 1024, 1024);
+  const unsigned gy = (unsigned)std::min<int64_t>(m, 65535);
+  for (int p = 0; p < passes; ++p) {
+    {
+      LaunchScope ls("k_greedy_start", st);
+      k_greedy_start<<<dim3(gx, gy), 256, 0, st>>>(codes, lo, scale, W_t, m, n, What, r.A, r.Es);
+    }
+    // A = W^old - (E H) D^-1: every column's feedback from the pass's start
+    sgemm::Params gp{};
+    gp.C = r.A, gp.ldc = n, gp.M = (int)m, gp.N = (int)n, gp.K = (int)n;
+    gp.a_piece_rows = (int)m, gp.b_piece_rows = (int)n;
+    gp.alpha = -1.f;
+    QCHECK(split_gemm(r.ta, r.tb, gp, st, "k_gemm_split_tc[greedy]", 0, &r.tb64, &r.tb128));
+    // then LDLQ's recursion with weights W^old and factor U'_jk = H_jk / H_kk
+    QCHECK(ldlq_range(r, 0, n));
+  }
   return QUIP_OK;
 }
 

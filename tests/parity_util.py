@@ -45,3 +45,29 @@ def ldlq_trajectory_check(codes, Wt, U, lo, s, bits, tau):
 def oracle_layer(cfg, d):
     """Full FP64 pipeline for a config's synthetic layer (small configs)."""
     return O.run_pipeline(d["W"], d["X"], cfg.seed, cfg.m_side, cfg.n_side, cfg.bits, cfg.damp)
+
+
+def greedy_trajectory_check(C0, C1, Wt, H, lo, s, bits, tau):
+    """Every code of C1 must be the greedy decision of one pass from C0.
+
+    Column k is visited with columns j < k already updated (C1) and j > k
+    not yet (C0): in FP64,
+      t_k = W~_k - (sum_{j<k} E1_j H_jk + sum_{j>k} E0_j H_jk) / H_kk,
+      z_k = (t_k - lo)/s, E = lo + s c - W~.
+    Returns (mismatch fraction, fraction of mismatches that are NOT
+    near-ties), a near-tie having z_k within tau of a rounding boundary.
+    """
+    lo = np.asarray(lo, dtype=np.float64)[:, None]
+    s = np.asarray(s, dtype=np.float64)[:, None]
+    Wt = np.asarray(Wt, dtype=np.float64)
+    H = np.asarray(H, dtype=np.float64)
+    E0 = lo + s * np.asarray(C0, dtype=np.float64) - Wt
+    E1 = lo + s * np.asarray(C1, dtype=np.float64) - Wt
+    others = E1 @ np.triu(H, 1) + E0 @ np.tril(H, -1)
+    T = Wt - others / np.diag(H)[None, :]
+    z = (T - lo) / s
+    want = np.clip(np.rint(z), 0, 2 ** bits - 1)
+    bad = want != np.asarray(C1, dtype=np.float64)
+    frac = np.abs(z - np.floor(z) - 0.5)
+    near = frac < tau
+    return float(bad.mean()), float((bad & ~near).mean())

@@ -68,6 +68,25 @@ def test_host_argument_errors(lib):
     assert args(2, 64, 32, fake, 16) == L.QUIP_ERR_WORKSPACE
     assert args(2, 64, 32, ctypes.c_void_p(0x1004), 1 << 20) == L.QUIP_ERR_WORKSPACE
     assert lib.quip_dequantize(None, fake, fake, 2, 2, fake, None) == L.QUIP_ERR_ARG
+    # the other rounding methods
+    assert lib.quip_nearest_quantize(fake, 4, 8, 0, fake, fake, fake, None) == L.QUIP_ERR_ARG
+    assert lib.quip_nearest_quantize(None, 4, 8, 2, fake, fake, fake, None) == L.QUIP_ERR_ARG
+    assert lib.quip_nearest_quantize(fake, 0, 8, 2, fake, fake, fake, None) == L.QUIP_ERR_SHAPE
+    assert lib.quip_diag_order(fake, 8, 8, None, None, None) == L.QUIP_ERR_ARG
+    assert lib.quip_diag_order(fake, 4, 8, fake, None, None) == L.QUIP_ERR_SHAPE
+    assert lib.quip_diag_order(fake, 70000, 70000, fake, None, None) == L.QUIP_ERR_SHAPE
+    other = ctypes.c_void_p(0x100000)
+    assert lib.quip_permute(fake, 7, 4, 4, 4, None, None, other, 4, None) == L.QUIP_ERR_ARG
+    assert lib.quip_permute(fake, L.QUIP_F32, 4, 4, 4, None, None, fake, 4, None) == L.QUIP_ERR_ARG  # overlap
+    assert lib.quip_permute(fake, L.QUIP_U8, 4, 4, 3, None, None, other, 4, None) == L.QUIP_ERR_SHAPE
+    g = lambda W, m, n, bits, passes, ws, wsb: lib.quip_greedy_refine(
+        W, fake, n, m, n, bits, fake, fake, fake, passes, ws, wsb, None)
+    assert g(fake, 4, 64, 0, 1, fake, 1 << 30) == L.QUIP_ERR_ARG
+    assert g(fake, 4, 64, 2, -1, fake, 1 << 30) == L.QUIP_ERR_ARG
+    assert g(fake, 4, 96, 2, 1, fake, 1 << 30) == L.QUIP_ERR_SHAPE
+    assert g(ctypes.c_void_p(0x1004), 4, 64, 2, 1, fake, 1 << 30) == L.QUIP_ERR_ARG
+    assert g(fake, 4, 64, 2, 1, fake, 16) == L.QUIP_ERR_WORKSPACE
+    assert g(fake, 4, 64, 2, 0, fake, 1 << 30) == L.QUIP_OK          # no pass: nothing launched
 
 
 def test_workspace_sizes(lib):
@@ -75,6 +94,10 @@ def test_workspace_sizes(lib):
     assert lib.quip_workspace_size(L.QUIP_OP_LDLQ, None, 64, 128, 32, ctypes.byref(nb)) == 0
     assert nb.value >= (64 * 128 + 64 * 32) * 4 and nb.value % 256 == 0
     assert lib.quip_workspace_size(L.QUIP_OP_LDL, None, 64, 128, 0, ctypes.byref(nb)) == 0
+    ldlq = ctypes.c_size_t()
+    lib.quip_workspace_size(L.QUIP_OP_LDLQ, None, 64, 128, 128, ctypes.byref(ldlq))
+    assert lib.quip_workspace_size(L.QUIP_OP_GREEDY, None, 64, 128, 0, ctypes.byref(nb)) == 0
+    assert nb.value >= ldlq.value + (128 * 128 + 64 * 128) * 4 and nb.value % 256 == 0
     assert lib.quip_workspace_size(99, None, 1, 1, 1, ctypes.byref(nb)) == L.QUIP_ERR_ARG
     assert lib.quip_workspace_size(L.QUIP_OP_INCOHERENCE_FORWARD, None, 1, 1, 1,
                                    ctypes.byref(nb)) == L.QUIP_ERR_ARG
