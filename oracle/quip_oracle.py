@@ -50,7 +50,10 @@ Readings where the pages are silent (each one is listed in the design doc):
     a greedy update sets one column to its exact coordinate minimiser on
     the grid, others held; a pass visits every column once, in the
     quantisation order; Greedy starts from nearest rounding; the number of
-    passes is a parameter (the pages give none).
+    passes is a parameter (the pages give none);
+  * quantized inference: the pages give no storage format for the codes;
+    ``pack_codes`` defines the library's (a column-strided layout, so that
+    consecutive words hold consecutive columns).
 
 Pinned by tests/test_oracle_*.py (CPU).  Functions with no pin: none.
 """
@@ -69,7 +72,8 @@ __all__ = [
     "ldlq", "ldlq_blocked", "nearest", "optq", "dequantize", "proxy_loss", "Pipeline",
     "run_pipeline", "STREAM_M_SIGNS", "STREAM_N_SIGNS", "STREAM_M_A", "STREAM_M_B",
     "STREAM_N_A", "STREAM_N_B", "STREAM_M_PERM", "STREAM_N_PERM", "random_permutation",
-    "diag_order", "greedy_pass", "quantize_layer",
+    "diag_order", "greedy_pass", "quantize_layer", "code_slot_bits", "packed_words", "pack_codes",
+    "unpack_codes", "quantized_matvec",
 ]
 
 # ----------------------------------------------------------------------------
@@ -505,6 +509,70 @@ def proxy_loss(What: np.ndarray, W: np.ndarray, H: np.ndarray) -> float:
     """l(W^) = tr((W^ - W) H (W^ - W)^T)  ([QuIP] Introduction)."""
     E = np.asarray(What, dtype=np.float64) - np.asarray(W, dtype=np.float64)
     return float(np.einsum("ij,ij->", E @ np.asarray(H, dtype=np.float64), E))
+
+
+# ----------------------------------------------------------------------------
+# Quantized inference: the layer's product with a full-precision vector
+# ----------------------------------------------------------------------------
+
+
+def code_slot_bits(bits: int) -> int:
+    """Width of a code's slot in a packed 32-bit word: the code width when it
+    divides 32 (1, 2, 4, 8), else the next of 4 and 8 (3 -> 4; 5, 6, 7 -> 8)."""
+    if bits in (1, 2, 4, 8):
+        return bits
+    if 1 <= bits <= 8:
+        return 4 if bits < 4 else 8
+    raise ValueError("bits must be 1..8")
+
+
+def packed_words(n: int, bits: int) -> int:
+    """32-bit words per packed row: ceil(n / (32 / slot)), rounded up to a
+    multiple of 4 (16 bytes)."""
+    per = 32 // code_slot_bits(bits)
+    w = -(-n // per)
+    return -(-w // 4) * 4
+
+
+def pack_codes(codes: np.ndarray, bits: int) -> np.ndarray:
+    """Packed codes for the quantized matrix-vector product.  The pages print
+    no storage format (QuIP, Experiments, "Throughput Comparison." speaks of
+    a quantized-matrix full-precision-vector product kernel); this one is the
+    library's: row i has Wd = packed_words(n, bits) words, and code j of the
+    row sits in word j mod Wd at bit (j div Wd) * slot.  Unused slots are 0.
+    Returns (m, Wd) uint32."""
+    codes = np.asarray(codes, dtype=np.int64)
+    m, n = codes.shape
+    slot = code_slot_bits(bits)
+    Wd = packed_words(n, bits)
+    out = np.zeros((m, Wd), dtype=np.uint64)
+    for j in range(n):
+        out[:, j % Wd] |= (codes[:, j].astype(np.uint64) << np.uint64((j // Wd) * slot))
+    return out.astype(np.uint32)
+
+
+def unpack_codes(packed: np.ndarray, n: int, bits: int) -> np.ndarray:
+    """Inverse of pack_codes: (m, n) int64 codes."""
+    packed = np.asarray(packed, dtype=np.uint64)
+    slot = code_slot_bits(bits)
+    Wd = packed.shape[1]
+    mask = np.uint64((1 << slot) - 1)
+    out = np.zeros((packed.shape[0], n), dtype=np.int64)
+    for j in range(n):
+        out[:, j] = ((packed[:, j % Wd] >> np.uint64((j // Wd) * slot)) & mask).astype(np.int64)
+    return out
+
+
+def quantized_matvec(codes: np.ndarray, lo: np.ndarray, s: np.ndarray, U: SideTransform,
+                     V: SideTransform, x: np.ndarray) -> np.ndarray:
+    """y = W^ x for the quantized layer W^ = U^T (lo + s codes) V (QuIP,
+    incoherence-processing section: the post-processing that undoes the
+    transforms; Experiments, "Throughput Comparison.": the quantized matrix
+    times a full-precision vector at inference).  x: (B, n) vectors as rows;
+    returns (B, m).  Written as the plain definition: the dequantised
+    original-domain matrix times each vector."""
+    W_hat = incoherence_inverse(dequantize(codes, lo, s), U, V)
+    return np.asarray(x, dtype=np.float64) @ W_hat.T
 
 
 # ----------------------------------------------------------------------------

@@ -213,3 +213,33 @@ def test_planted_rg_unpermute_mistake_is_caught(monkeypatch, twice):
     monkeypatch.setattr(Q, "quantize_layer", wrong)
     monkeypatch.setattr(O, "quantize_layer", wrong)
     assert _fails([P.test_rounding_methods_worked_example, P.test_ldlq_rg_first_columns_and_equivariance])
+
+
+def _pack_contiguous(codes, bits):
+    # planted: consecutive codes in one word (word j div per, slot j mod per)
+    codes = np.asarray(codes, dtype=np.int64)
+    m, n = codes.shape
+    slot = Q.code_slot_bits(bits)
+    per = 32 // slot
+    out = np.zeros((m, Q.packed_words(n, bits)), dtype=np.uint64)
+    for j in range(n):
+        out[:, j // per] |= codes[:, j].astype(np.uint64) << np.uint64((j % per) * slot)
+    return out.astype(np.uint32)
+
+
+def _matvec_untransposed(codes, lo, s, U, V, x):
+    W_hat = U.matrix() @ Q.dequantize(codes, lo, s) @ V.matrix()     # planted: U for U^T
+    return np.asarray(x, dtype=np.float64) @ W_hat.T
+
+
+def test_planted_pack_layout_is_caught(monkeypatch):
+    monkeypatch.setattr(Q, "pack_codes", _pack_contiguous)
+    monkeypatch.setattr(O, "pack_codes", _pack_contiguous)
+    assert _fails([P.test_pack_codes_worked_example_and_roundtrip])
+
+
+def test_planted_matvec_transpose_is_caught(monkeypatch):
+    monkeypatch.setattr(Q, "quantized_matvec", _matvec_untransposed)
+    monkeypatch.setattr(O, "quantized_matvec", _matvec_untransposed)
+    assert _fails([P.test_quantized_matvec_worked_example,
+                   P.test_quantized_matvec_is_the_layer_applied_to_the_vector])

@@ -550,3 +550,58 @@ def test_rg_and_greedy_never_beat_brute_force(n, bits):
             best = np.min(np.einsum("kj,jl,kl->k", cand, H, cand))
             e = lo[i] + s[i] * c[i] - W[i]
             assert float(e @ H @ e) >= best - 1e-12
+
+
+# ---------------------------------------------------------------- quantized inference
+
+
+def test_pack_codes_worked_example_and_roundtrip():
+    r = golden_rows("qmatvec_example.txt")
+    for line, bits in ((r[0], 2), (r[1], 3)):
+        c, w = line.split("|")
+        codes = np.array([list(map(int, c.split()))])
+        np.testing.assert_array_equal(O.pack_codes(codes, bits)[0], list(map(int, w.split())))
+    rng = np.random.default_rng(50)
+    for bits in range(1, 9):
+        for n in (1, 5, 64, 129, 300):
+            c = rng.integers(0, 2 ** bits, (3, n))
+            p = O.pack_codes(c, bits)
+            assert p.shape == (3, O.packed_words(n, bits)) and p.shape[1] % 4 == 0
+            assert p.shape[1] * (32 // O.code_slot_bits(bits)) >= n
+            np.testing.assert_array_equal(O.unpack_codes(p, n, bits), c)
+            # the packed words hold exactly the codes' bits: popcounts agree
+            assert sum(bin(int(v)).count("1") for v in p.ravel()) == \
+                sum(bin(int(v)).count("1") for v in c.ravel())
+
+
+def test_quantized_matvec_worked_example():
+    r = golden_rows("qmatvec_example.txt")
+    codes = np.array(list(map(int, r[2].split()))).reshape(2, 2)
+    lo = np.array(list(map(float, r[3].split())))
+    s = np.array(list(map(float, r[4].split())))
+    x = np.array([list(map(float, r[5].split()))])
+    I = O.SideTransform("identity", 2)
+    np.testing.assert_allclose(O.quantized_matvec(codes, lo, s, I, I, x)[0],
+                               list(map(float, r[6].split())), atol=1e-15)
+    U = O.SideTransform("hadamard", 2, signs=np.array([1.0, 1.0]))
+    V = O.SideTransform("hadamard", 2, signs=np.array([1.0, -1.0]))
+    np.testing.assert_allclose(O.quantized_matvec(codes, lo, s, U, V, x)[0],
+                               list(map(float, r[7].split())), atol=1e-14)
+
+
+def test_quantized_matvec_is_the_layer_applied_to_the_vector():
+    # the product of the quantized layer with x equals quantising, then
+    # running the original-domain layer: y = W^ x, with W^ from the pipeline;
+    # and it is linear in x
+    cfg = CONFIGS["tiny"]
+    d = make_layer(cfg)
+    P = O.run_pipeline(d["W"], d["X"], cfg.seed, cfg.m_side, cfg.n_side, cfg.bits, cfg.damp)
+    rng = np.random.default_rng(51)
+    x = rng.standard_normal((3, cfg.n))
+    y = O.quantized_matvec(P.codes, P.lo, P.s, P.U, P.V, x)
+    np.testing.assert_allclose(y, x @ P.W_hat.T, rtol=1e-12, atol=1e-12)
+    y2 = O.quantized_matvec(P.codes, P.lo, P.s, P.U, P.V, 2 * x[:1] - x[1:2])
+    np.testing.assert_allclose(y2[0], 2 * y[0] - y[1], atol=1e-12)
+    # in the incoherent domain: U y = W~^ (V x)
+    np.testing.assert_allclose(y @ P.U.matrix().T,
+                               (x @ P.V.matrix().T) @ O.dequantize(P.codes, P.lo, P.s).T, atol=1e-12)
