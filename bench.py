@@ -551,6 +551,131 @@ def run_ours(args, cfg: LayerConfig):
         dist.destroy_process_group()
 
 
+def run_decode(args):
+    """Inference: one decode step of a batch of B tokens through every linear
+    layer of a Llama-2-7B decoder stack (32 blocks x q, k, v, o 4096x4096,
+    gate, up 11008x4096, down 4096x11008), each a QuantizedLinear on packed
+    b-bit codes with its incoherence transform applied around the product
+    (Hadamard on 4096-wide sides, Kronecker 86x128 on 11008-wide ones).
+    Codes, grids and transforms are seeded and synthetic (the product's time
+    does not depend on the code values).  The 224 products of a step are
+    captured in one CUDA graph; the packed codes (1.6 GB at 2 bits) exceed
+    L2, so every step streams them from HBM.  Attention and the activations
+    between layers are not part of the step: each product takes the previous
+    product's output when the widths match, else the step's input."""
+    import torch
+    import post_weight_quantization_09_b200 as Q
+    from post_weight_quantization_09_b200 import _lib as L
+    from quip_synth import Side
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    lib = Q.load()
+    bits, B, blocks = args.bits, args.decode_batch, args.decode_blocks
+    had, kron = Side("hadamard"), Side("kronecker", 86, 128)
+    shapes = [("q", 4096, 4096, had, had), ("k", 4096, 4096, had, had), ("v", 4096, 4096, had, had),
+              ("o", 4096, 4096, had, had), ("gate", 11008, 4096, kron, had),
+              ("up", 11008, 4096, kron, had), ("down", 4096, 11008, had, kron)]
+    g = torch.Generator(device="cuda").manual_seed(1234 + rank)
+    layers = []
+    for blk in range(blocks):
+        for i, (name, m, n, ms, ns) in enumerate(shapes):
+            seed = 1000 * blk + i + 7919 * rank
+            tf = Q.Transform(seed, m, n, ms, ns)
+            codes = torch.randint(0, 2 ** bits, (m, n), generator=g, device="cuda", dtype=torch.uint8)
+            lo = torch.rand(m, generator=g, device="cuda") * -0.05
+            sc = torch.rand(m, generator=g, device="cuda") * 0.01 + 0.001
+            layers.append(Q.QuantizedLinear(tf, codes, lo, sc, bits, max_batch=B))
+            del codes
+    torch.cuda.synchronize()
+    x0 = {4096: torch.randn(B, 4096, device="cuda", generator=g),
+          11008: torch.randn(B, 11008, device="cuda", generator=g)}
+    bufs = {d: [torch.empty(B, d, device="cuda") for _ in range(2)] for d in (4096, 11008)}
+
+    def step():
+        last = dict(x0)
+        for i, ql in enumerate(layers):
+            inp = last[ql.n]
+            out = bufs[ql.m][i % 2]
+            if out is inp:
+                out = bufs[ql.m][1 - i % 2]
+            ql(inp, out)
+            last[ql.m] = out
+
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+    torch.cuda.synchronize()
+    st = Q.quip_sync_status()
+    if st != L.QUIP_OK:
+        raise RuntimeError(f"device status after warm-up: {L.status_string(st)}")
+    graph = torch.cuda.CUDAGraph()
+    launches0 = lib.quip_kernel_launches()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    per_step_launches = lib.quip_kernel_launches() - launches0
+    torch.cuda.synchronize()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    ms = []
+    main = torch.cuda.current_stream()
+    with ClockSampler(local) as clk:
+        for _ in range(args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(main)
+            graph.replay()
+            e1.record(main)
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+    # per-kernel device time of the same step, eager, each launch bracketed by events
+    Q.quip_timing_begin()
+    with torch.cuda.stream(stream):
+        for _ in range(min(args.steps, 20)):
+            step()
+    torch.cuda.synchronize()
+    per_kernel = Q.quip_timing_end()
+    nrep = min(args.steps, 20)
+    st = Q.quip_sync_status()
+    if st != L.QUIP_OK:
+        raise RuntimeError(f"device status after timing: {L.status_string(st)}")
+    ms_step = max_over_ranks(statistics.mean(ms), world, "cuda")
+    code_bytes = sum(ql.packed.numel() * 4 for ql in layers)
+    grid_bytes = sum(8 * ql.m for ql in layers)
+    weights = sum(ql.m * ql.n for ql in layers)
+    pk = peaks()
+    qk = per_kernel.get("k_qmatvec", (0, 0.0))
+    qms = qk[1] / nrep
+    # algorithmic bytes of the products: packed codes, grids, x' in and z out
+    qbytes = code_bytes + grid_bytes + 4.0 * B * sum(ql.m + ql.n for ql in layers)
+    kernels = {k: {"launches_per_step": c / nrep, "ms_per_step": round(t / nrep, 4)}
+               for k, (c, t) in per_kernel.items()}
+    ach = qbytes / (qms * 1e-3) / 1e9 if qms > 0 else None
+    line = {
+        "metric": f"decode tokens/s through the quantized linear layers of a Llama-2-7B stack "
+                  f"({bits}-bit, batch {B})",
+        "value": world * B * 1e3 / ms_step, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded random codes, grids, transforms)",
+        "config": {"workload": f"{blocks} blocks x (q, k, v, o 4096x4096; gate, up 11008x4096; down "
+                               f"4096x11008), {bits}-bit packed codes ({code_bytes / 1e9:.2f} GB), "
+                               f"batch {B}, one CUDA graph per step",
+                   "weights": weights, "l2": "not flushed: the packed codes exceed L2 (126 MB)"},
+        "roofline": {"bound": "hbm", "achieved": round(ach, 1) if ach else None, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(ach / pk["hbm_gbs"], 4) if ach else None,
+                     "traffic": None, "kernel": "k_qmatvec",
+                     "step_gbs": round(qbytes / (ms_step * 1e-3) / 1e9, 1),
+                     "peak_source": pk["source"]},
+        "kernels": kernels,
+        "gpu_launches": int(per_step_launches * args.steps),
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+
+
 def run_group(args, cfg: LayerConfig):
     """G layers of cfg's shape reading the same input X (q / k / v of an
     attention block, up / gate of an MLP): one Hessian, one transform of it
@@ -624,12 +749,20 @@ def main():
     ap.add_argument("--method", default="ldlq", choices=["ldlq", "nearest", "greedy", "ldlq_rg"],
                     help="rounding method (QuIP, Experiments, Methods)")
     ap.add_argument("--passes", type=int, default=1, help="greedy passes of greedy / ldlq_rg")
+    ap.add_argument("--decode", action="store_true",
+                    help="inference: quantized products of a Llama-2-7B linear stack per decode step")
+    ap.add_argument("--decode-batch", type=int, default=1)
+    ap.add_argument("--decode-blocks", type=int, default=32)
+    ap.add_argument("--bits", type=int, default=2, help="code width of --decode")
     args = ap.parse_args()
     cfg = CONFIGS[args.config]
     if args.permute:
         from dataclasses import replace
         cfg = replace(cfg, m_side=replace(cfg.m_side, permute=True),
                       n_side=replace(cfg.n_side, permute=True))
+    if args.decode:
+        run_decode(args)
+        return
     if args.impl == "reference":
         run_reference(args, cfg)
     else:

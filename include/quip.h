@@ -82,7 +82,8 @@ typedef enum {
   QUIP_OP_INCOHERENCE_INVERSE = 1,
   QUIP_OP_LDL = 2,
   QUIP_OP_LDLQ = 3,
-  QUIP_OP_GREEDY = 4
+  QUIP_OP_GREEDY = 4,
+  QUIP_OP_QMATVEC = 5
 } quip_op;
 
 typedef struct quip_transform quip_transform;   /* opaque, library-owned */
@@ -333,14 +334,57 @@ quip_status quip_greedy_refine(const float* W_t, const float* H, int64_t ldh, in
                                int bits, const float* lo, const float* scale, uint8_t* codes,
                                int passes, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * 32-bit words per row of packed codes (the smallest valid ldp of
+ * quip_pack_codes / quip_qmatvec): ceil(n / (32 / slot)) rounded up to a
+ * multiple of 4, slot = bits for bits in {1, 2, 4, 8}, 4 for bits 3, 8 for
+ * bits 5..7.  Host only; 0 for invalid arguments.
+ */
+int64_t quip_packed_words(int64_t n, int bits);
+
+/*
+ * Pack b-bit codes for the quantized product (the pages print no storage
+ * format; this is the library's): code j of row i goes to word
+ * j mod Wd of row i at bit (j div Wd) * slot, Wd = quip_packed_words(n,
+ * bits); unused slots are 0.
+ *   codes  : device m x n uint8 (row stride n), values < 2^bits (higher
+ *            bits are dropped).
+ *   packed : device m x ldp uint32, ldp >= Wd, ldp % 4 == 0, 16-byte aligned.
+ */
+quip_status quip_pack_codes(const uint8_t* codes, int64_t m, int64_t n, int bits, uint32_t* packed,
+                            int64_t ldp, void* stream);
+
+/*
+ * The quantized layer times B full-precision vectors (QuIP, Experiments,
+ * "Throughput Comparison.": quantized matrix times full-precision vector,
+ * with the incoherence processing around it):
+ *   y_b = U^T (lo + s codes) V x_b     for b < B  (W^ = U^T W~^ V, the layer
+ *   the pipeline's inverse transform returns),
+ * computed as x' = V x (the transform's row kernels), z_i = lo_i sum(x') +
+ * s_i sum_j c_ij x'_j (one kernel over the packed codes, fp32 sums), y = U^T z.
+ *   tf     : the layer's transform (m x n).
+ *   packed : from quip_pack_codes with the same bits; row stride ldp words.
+ *   lo, scale : device m fp32 (the grid of the codes).
+ *   x      : device B x n, row stride ldx elements, QUIP_F32 or QUIP_BF16
+ *            (16-byte aligned rows when V is a Hadamard side without
+ *            permutation and n >= 16).
+ *   y      : device B x m fp32, row stride ldy.
+ * n % 4 == 0.  The product kernel takes the vectors 8 at a time (4 for
+ * 1-bit codes).  ws: QUIP_OP_QMATVEC with block = B.
+ */
+quip_status quip_qmatvec(const quip_transform* tf, const uint32_t* packed, int64_t ldp, const float* lo,
+                         const float* scale, int bits, const void* x, int x_dtype, int64_t ldx, int64_t B,
+                         float* y, int64_t ldy, void* ws, size_t ws_bytes, void* stream);
+
 /* W_hat_t[i,j] = lo[i] + scale[i] * codes[i,j]  (device; m x n, row stride n). */
 quip_status quip_dequantize(const uint8_t* codes, const float* lo, const float* scale,
                             int64_t m, int64_t n, float* W_hat_t, void* stream);
 
 /*
  * Bytes of workspace `op` needs (quip_op).  tf is required for the
- * incoherence ops and ignored otherwise; block is used by QUIP_OP_LDLQ;
- * QUIP_OP_GREEDY takes m and n.
+ * incoherence ops and QUIP_OP_QMATVEC and ignored otherwise; block is used
+ * by QUIP_OP_LDLQ, and is the number of vectors B for QUIP_OP_QMATVEC
+ * (whose m and n come from tf); QUIP_OP_GREEDY takes m and n.
  * *bytes may be 0.
  */
 quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int64_t n,

@@ -22,6 +22,7 @@ __all__ = [
     "Transform", "quip_hessian_accumulate", "quip_hessian_finalize", "quip_incoherence_forward",
     "quip_incoherence_inverse", "quip_ldl", "quip_ldlq_quantize", "quip_dequantize",
     "quip_nearest_quantize", "quip_diag_order", "quip_permute", "quip_greedy_refine", "METHODS",
+    "quip_packed_words", "quip_pack_codes", "quip_qmatvec", "QuantizedLinear",
     "quip_workspace_size", "quip_sync_status", "quip_timing_begin", "quip_timing_end", "LayerQuantizer",
     "LayerGroupQuantizer", "quantize_layer", "QuipError",
     "KIND",
@@ -250,6 +251,57 @@ def quip_greedy_refine(W_t: torch.Tensor, H: torch.Tensor, bits: int, lo: torch.
     L.check(load().quip_greedy_refine(_p(W_t), _p(H), H.stride(0), m, n, bits, _p(lo), _p(scale),
                                       _p(codes), passes, _p(ws), 0 if ws is None else ws.numel(),
                                       _s(stream)), "quip_greedy_refine")
+
+
+def quip_packed_words(n: int, bits: int) -> int:
+    return int(load().quip_packed_words(n, bits))
+
+
+def quip_pack_codes(codes: torch.Tensor, bits: int, packed: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """Packed codes (m x packed_words int32 words; see quip.h for the layout)."""
+    m, n = codes.shape
+    if packed is None:
+        packed = torch.empty(m, quip_packed_words(n, bits), dtype=torch.int32, device=codes.device)
+    L.check(load().quip_pack_codes(_p(codes), m, n, bits, _p(packed), packed.stride(0), _s(stream)),
+            "quip_pack_codes")
+    return packed
+
+
+def quip_qmatvec(tf: Transform, packed: torch.Tensor, lo: torch.Tensor, scale: torch.Tensor, bits: int,
+                 x: torch.Tensor, y: torch.Tensor, ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    """y[b] = U^T (lo + s codes) V x[b] for the rows b of x (B x n) into y (B x m)."""
+    B = x.shape[0]
+    if ws is None:
+        ws = _ws(quip_workspace_size(L.QUIP_OP_QMATVEC, tf, tf.m, tf.n, B), x.device)
+    L.check(load().quip_qmatvec(tf.handle, _p(packed), packed.stride(0), _p(lo), _p(scale), bits, _p(x),
+                                _dtype(x), x.stride(0), B, _p(y), y.stride(0), _p(ws),
+                                0 if ws is None else ws.numel(), _s(stream)), "quip_qmatvec")
+
+
+class QuantizedLinear:
+    """A quantized layer for inference: y = W^ x with W^ = U^T (lo + s codes) V
+    kept as packed codes, the per-row grid and the layer's transform (QuIP,
+    Experiments, "Throughput Comparison.").  ``max_batch`` sizes the
+    workspace; ``__call__`` takes x (B x n, fp32 or bf16, B <= max_batch)."""
+
+    def __init__(self, tf: Transform, codes: torch.Tensor, lo: torch.Tensor, scale: torch.Tensor,
+                 bits: int, max_batch: int = 8, stream=None):
+        self.tf, self.bits, self.stream = tf, bits, stream
+        self.m, self.n = tf.m, tf.n
+        self.packed = quip_pack_codes(codes, bits, stream=stream)
+        self.lo, self.scale = lo, scale
+        self.max_batch = max_batch
+        self.ws = torch.empty(max(quip_workspace_size(L.QUIP_OP_QMATVEC, tf, tf.m, tf.n, max_batch), 256),
+                              dtype=torch.uint8, device=codes.device)
+
+    def __call__(self, x: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        if x.shape[0] > self.max_batch:
+            raise ValueError(f"batch {x.shape[0]} > max_batch {self.max_batch}")
+        if out is None:
+            out = torch.empty(x.shape[0], self.m, dtype=torch.float32, device=x.device)
+        quip_qmatvec(self.tf, self.packed, self.lo, self.scale, self.bits, x, out, self.ws, self.stream)
+        return out
 
 
 def quip_dequantize(codes: torch.Tensor, lo: torch.Tensor, scale: torch.Tensor, W_hat_t: torch.Tensor,

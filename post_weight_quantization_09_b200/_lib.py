@@ -15,7 +15,7 @@ QUIP_F32, QUIP_BF16, QUIP_U8 = 0, 1, 2
 QUIP_T_IDENTITY, QUIP_T_HADAMARD, QUIP_T_KRONECKER = 0, 1, 2
 QUIP_T_PERMUTE = 0x100
 QUIP_OP_INCOHERENCE_FORWARD, QUIP_OP_INCOHERENCE_INVERSE, QUIP_OP_LDL, QUIP_OP_LDLQ = 0, 1, 2, 3
-QUIP_OP_GREEDY = 4
+QUIP_OP_GREEDY, QUIP_OP_QMATVEC = 4, 5
 
 # name -> (restype, argtypes); the list of every symbol include/quip.h declares
 SIGNATURES = {
@@ -48,6 +48,10 @@ SIGNATURES = {
                              c_int64, c_void_p]),
     "quip_greedy_refine": (c_int, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int, c_void_p,
                                    c_void_p, c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
+    "quip_packed_words": (c_int64, [c_int64, c_int]),
+    "quip_pack_codes": (c_int, [c_void_p, c_int64, c_int64, c_int, c_void_p, c_int64, c_void_p]),
+    "quip_qmatvec": (c_int, [c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_int, c_void_p, c_int,
+                             c_int64, c_int64, c_void_p, c_int64, c_void_p, c_size_t, c_void_p]),
     "quip_dequantize": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
     "quip_workspace_size": (c_int, [c_int, c_void_p, c_int64, c_int64, c_int64, POINTER(c_size_t)]),
     "quip_sync_status": (c_int, [c_void_p]),

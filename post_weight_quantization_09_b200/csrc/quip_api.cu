@@ -18,6 +18,7 @@
 #include "ldlq.cuh"
 #include "rng.cuh"
 #include "rounding.cuh"
+#include "qmatvec.cuh"
 #include "syrk_tc.cuh"
 #include "gemm_tc.cuh"
 
@@ -756,6 +757,21 @@ static size_t greedy_ws_bytes(int64_t m, int64_t n) {
   return ldlq_ws_bytes(m, n, 128) + round256((size_t)n * n * 4) + round256((size_t)m * n * 4);
 }
 
+// Quantized product: the transformed vectors x' (B x n), the products z
+// (B x m) and the Kronecker temporaries of the row transforms (B x max(m, n)),
+// all fp32.
+static size_t qmatvec_ws_bytes(int64_t m, int64_t n, int64_t B) {
+  return round256((size_t)B * n * 4) + round256((size_t)B * m * 4) +
+         round256((size_t)B * std::max(m, n) * 4) + 256;
+}
+
+// Slot width of a code in a packed word and the words of a packed row.
+static int code_slot(int bits) { return (bits == 1 || bits == 2 || bits == 4 || bits == 8) ? bits : (bits < 4 ? 4 : 8); }
+static int64_t packed_row_words(int64_t n, int bits) {
+  const int64_t per = 32 / code_slot(bits);
+  return ((n + per - 1) / per + 3) / 4 * 4;
+}
+
 // Transform workspace: Kronecker temporaries, then the permutation scratch
 // (the forward pass gathers H into it, the inverse gathers W^).
 static size_t transform_kron_bytes(const quip_transform* tf, int op) {
@@ -794,6 +810,11 @@ quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int
     case QUIP_OP_GREEDY:
       if (m <= 0 || n <= 0) return QUIP_ERR_SHAPE;
       *bytes = greedy_ws_bytes(m, n);
+      return QUIP_OK;
+    case QUIP_OP_QMATVEC:
+      if (!tf) return QUIP_ERR_ARG;
+      if (block <= 0) return QUIP_ERR_SHAPE;
+      *bytes = qmatvec_ws_bytes(tf->m, tf->n, block);
       return QUIP_OK;
     default:
       return QUIP_ERR_ARG;
@@ -1279,6 +1300,241 @@ quip_status quip_ldlq_quantize_static(const float* W_t, const float* Uring, int6
   if (s != QUIP_OK) return s;
   return quip_ldlq_quantize(W_t, Uring, ldu, m, n, bits, block, codes, lo, scale, ws,
                             (size_t)QUIP_LDLQ_STATIC_SCRATCH_BYTES, stream);
+}
+
+int64_t quip_packed_words(int64_t n, int bits) {
+  if (n <= 0 || bits < 1 || bits > 8) return 0;
+  return packed_row_words(n, bits);
+}
+
+quip_status quip_pack_codes(const uint8_t* codes, int64_t m, int64_t n, int bits, uint32_t* packed,
+                            int64_t ldp, void* stream) {
+  if (!codes || !packed) return QUIP_ERR_ARG;
+  if (bits < 1 || bits > 8) return QUIP_ERR_ARG;
+  if (m <= 0 || n <= 0) return QUIP_ERR_SHAPE;
+  const int64_t Wd = packed_row_words(n, bits);
+  if (ldp < Wd || (ldp & 3) || (reinterpret_cast<uintptr_t>(packed) & 15)) return QUIP_ERR_SHAPE;
+  cudaStream_t st = S(stream);
+  const unsigned grid = (unsigned)std::min<int64_t>((m * Wd + 255) / 256, (int64_t)num_sms() * 16);
+  LaunchScope ls("k_pack_codes", st);
+  switch (code_slot(bits)) {
+    case 1: k_pack_codes<1><<<grid, 256, 0, st>>>(codes, m, n, Wd, packed, ldp); break;
+    case 2: k_pack_codes<2><<<grid, 256, 0, st>>>(codes, m, n, Wd, packed, ldp); break;
+    case 4: k_pack_codes<4><<<grid, 256, 0, st>>>(codes, m, n, Wd, packed, ldp); break;
+    default: k_pack_codes<8><<<grid, 256, 0, st>>>(codes, m, n, Wd, packed, ldp); break;
+  }
+  QCHECK(cudaGetLastError());
+  return QUIP_OK;
+}
+
+}  // extern "C"
+
+namespace {
+template <int SLOT, int BC>
+cudaError_t qmatvec_launch(const uint32_t* packed, int64_t ldp, int64_t Wd, const float* lo,
+                           const float* sc, int64_t m, int64_t n, const float* xs, int nb, float* z,
+                           cudaStream_t st) {
+  const int64_t tasks = (m + qmv_rows<BC>() - 1) / qmv_rows<BC>();
+  const unsigned grid = (unsigned)std::max<int64_t>(
+      1, std::min<int64_t>((tasks + QMV_WARPS - 1) / QMV_WARPS, (int64_t)num_sms() * 8));
+  LaunchScope ls("k_qmatvec", st);
+  k_qmatvec<SLOT, BC><<<grid, QMV_WARPS * 32, 0, st>>>(packed, ldp, Wd, lo, sc, m, n, xs, n, nb, z, m);
+  return cudaGetLastError();
+}
+
+// The vectors in chunks of up to 8 (4 for 1-bit slots, whose 32 slots per
+// word would need more registers).
+template <int SLOT>
+cudaError_t qmatvec_slot(const uint32_t* packed, int64_t ldp, int64_t Wd, const float* lo, const float* sc,
+                         int64_t m, int64_t n, const float* xs, int64_t B, float* z, cudaStream_t st) {
+  const int bc = SLOT == 1 ? 4 : 8;
+  for (int64_t b0 = 0; b0 < B; b0 += bc) {
+    const int nb = (int)std::min<int64_t>(bc, B - b0);
+    const float* x = xs + b0 * n;
+    float* zz = z + b0 * m;
+    cudaError_t e;
+    if (nb > 4) e = qmatvec_launch<SLOT, (SLOT == 1 ? 4 : 8)>(packed, ldp, Wd, lo, sc, m, n, x, nb, zz, st);
+    else if (nb > 2) e = qmatvec_launch<SLOT, 4>(packed, ldp, Wd, lo, sc, m, n, x, nb, zz, st);
+    else if (nb == 2) e = qmatvec_launch<SLOT, 2>(packed, ldp, Wd, lo, sc, m, n, x, nb, zz, st);
+    else e = qmatvec_launch<SLOT, 1>(packed, ldp, Wd, lo, sc, m, n, x, nb, zz, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+// A Kronecker side on a few fp32 vectors in one launch (k_kron_vec).
+bool kron_vec_fits(const SideData& sd) {
+  return sd.kind == QUIP_T_KRONECKER && sd.p <= 65535 && sd.q <= 1024;
+}
+cudaError_t kron_vec(const SideData& sd, bool inverse, const float* x, int64_t ldx, float* y, int64_t ldy,
+                     int64_t B, cudaStream_t st) {
+  LaunchScope ls("k_kron_vec", st);
+  k_kron_vec<<<dim3((unsigned)sd.p, (unsigned)B), 256, 0, st>>>(sd.A, sd.B, (int)sd.p, (int)sd.q,
+                                                                inverse ? 1 : 0, x, ldx, y, ldy);
+  return cudaGetLastError();
+}
+
+// The one-launch product (k_qlinear) for Hadamard / identity sides without
+// permutation: the vectors in chunks of BC (8, 4, 2 or 1, as many as fit
+// BC x max(n, m) fp32 in shared memory).
+constexpr int64_t QL_SMEM_MAX = 200 * 1024;
+
+template <int SLOT, int BC, typename TX>
+cudaError_t qlinear_launch(const uint32_t* packed, int64_t ldp, int64_t Wd, const float* lo, const float* sc,
+                           int64_t m, int64_t n, const TX* x, int64_t ldx, int nb, const float* vs, float vscale,
+                           const float* us, float uscale, float* z, unsigned* counter, float* y, int64_t ldy,
+                           cudaStream_t st) {
+  const size_t smem = (size_t)BC * ((std::max(m, n) + 3) / 4 * 4) * sizeof(float);
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_qlinear<SLOT, BC, TX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)QL_SMEM_MAX);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  // one CTA per SM at most: every CTA transforms the
+  // vectors itself, so fewer, larger CTAs repeat that less
+  const int64_t tasks = (m + qmv_rows<BC>() - 1) / qmv_rows<BC>();
+  const unsigned grid = (unsigned)std::max<int64_t>(
+      1, std::min<int64_t>((tasks + ql_warps<BC>() - 1) / ql_warps<BC>(), (int64_t)num_sms()));
+  cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(unsigned), st);
+  if (e != cudaSuccess) return e;
+  LaunchScope ls("k_qlinear", st);
+  k_qlinear<SLOT, BC, TX><<<grid, ql_warps<BC>() * 32, smem, st>>>(packed, ldp, Wd, lo, sc, (int)m, (int)n, x, ldx,
+                                                             nb, vs, vscale, us, uscale, z, counter, y, ldy);
+  return cudaGetLastError();
+}
+
+template <int SLOT, typename TX>
+cudaError_t qlinear_slot(const uint32_t* packed, int64_t ldp, int64_t Wd, const float* lo, const float* sc,
+                         int64_t m, int64_t n, const TX* x, int64_t ldx, int64_t B, const float* vs,
+                         float vscale, const float* us, float uscale, float* z, unsigned* counter, float* y,
+                         int64_t ldy, int bc, cudaStream_t st) {
+  for (int64_t b0 = 0; b0 < B; b0 += bc) {
+    const int nb = (int)std::min<int64_t>(bc, B - b0);
+    const TX* xx = x + b0 * ldx;
+    float* yy = y + b0 * ldy;
+    cudaError_t e;
+#define QL_ARGS packed, ldp, Wd, lo, sc, m, n, xx, ldx, nb, vs, vscale, us, uscale, z, counter, yy, ldy, st
+    if (bc == 8) e = qlinear_launch<SLOT, 8, TX>(QL_ARGS);
+    else if (bc == 4) e = qlinear_launch<SLOT, 4, TX>(QL_ARGS);
+    else if (bc == 2) e = qlinear_launch<SLOT, 2, TX>(QL_ARGS);
+    else e = qlinear_launch<SLOT, 1, TX>(QL_ARGS);
+#undef QL_ARGS
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+template <typename TX>
+cudaError_t qlinear(int slot, const uint32_t* packed, int64_t ldp, int64_t Wd, const float* lo, const float* sc,
+                    int64_t m, int64_t n, const TX* x, int64_t ldx, int64_t B, const float* vs, float vscale,
+                    const float* us, float uscale, float* z, unsigned* counter, float* y, int64_t ldy, int bc,
+                    cudaStream_t st) {
+#define QL_ARGS packed, ldp, Wd, lo, sc, m, n, x, ldx, B, vs, vscale, us, uscale, z, counter, y, ldy, bc, st
+  switch (slot) {
+    case 1: return qlinear_slot<1, TX>(QL_ARGS);
+    case 2: return qlinear_slot<2, TX>(QL_ARGS);
+    case 4: return qlinear_slot<4, TX>(QL_ARGS);
+    default: return qlinear_slot<8, TX>(QL_ARGS);
+  }
+#undef QL_ARGS
+}
+}  // namespace
+
+extern "C" {
+
+quip_status quip_qmatvec(const quip_transform* tf, const uint32_t* packed, int64_t ldp, const float* lo,
+                         const float* scale, int bits, const void* x, int x_dtype, int64_t ldx, int64_t B,
+                         float* y, int64_t ldy, void* ws, size_t ws_bytes, void* stream) {
+  if (!tf || !packed || !lo || !scale || !x || !y) return QUIP_ERR_ARG;
+  if (bits < 1 || bits > 8) return QUIP_ERR_ARG;
+  if (x_dtype != QUIP_F32 && x_dtype != QUIP_BF16) return QUIP_ERR_ARG;
+  const int64_t m = tf->m, n = tf->n;
+  if (B <= 0 || ldx < n || ldy < m) return QUIP_ERR_SHAPE;
+  const int slot = code_slot(bits);
+  const int64_t Wd = packed_row_words(n, bits);
+  if (ldp < Wd || (ldp & 3) || (reinterpret_cast<uintptr_t>(packed) & 15)) return QUIP_ERR_SHAPE;
+  if (n % 4) return QUIP_ERR_SHAPE;
+  const SideData &U = tf->side[0], &V = tf->side[1];
+  if (V.kind == QUIP_T_HADAMARD && n >= 16 && !V.permute) {   // vector loads in the row kernel
+    const size_t esz = x_dtype == QUIP_BF16 ? 2 : 4;
+    if ((reinterpret_cast<uintptr_t>(x) % 16) || ((ldx * esz) % 16)) return QUIP_ERR_ARG;
+  }
+  quip_status s = check_ws(ws, ws_bytes, qmatvec_ws_bytes(m, n, B));
+  if (s != QUIP_OK) return s;
+  cudaStream_t st = S(stream);
+  char* w8 = static_cast<char*>(ws);
+  float* xs = reinterpret_cast<float*>(w8);
+  w8 += round256((size_t)B * n * 4);
+  float* z = reinterpret_cast<float*>(w8);
+  w8 += round256((size_t)B * m * 4);
+  float* tmp = reinterpret_cast<float*>(w8);
+  unsigned* counter = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(tmp) +
+                                                 round256((size_t)B * std::max(m, n) * 4));
+  // one launch per vector chunk (k_qlinear) when neither side permutes and a
+  // chunk's vectors fit in shared memory: Hadamard / identity sides inside
+  // the launch, a Kronecker side (k_kron_vec) as one more launch before
+  // (V x into xs) or after (U^T z from tmp)
+  const bool kin = V.kind == QUIP_T_KRONECKER, kout = U.kind == QUIP_T_KRONECKER;
+  const bool simple = !U.permute && !V.permute && (!kin || (kron_vec_fits(V) && x_dtype == QUIP_F32)) &&
+                      (!kout || kron_vec_fits(U));
+  const int64_t dmax = (std::max(m, n) + 3) / 4 * 4;
+  const int bc = std::min<int64_t>(B, 8) > 4 && 8 * dmax * 4 <= QL_SMEM_MAX ? 8
+               : std::min<int64_t>(B, 8) > 2 && 4 * dmax * 4 <= QL_SMEM_MAX ? 4
+               : std::min<int64_t>(B, 8) > 1 && 2 * dmax * 4 <= QL_SMEM_MAX ? 2
+               : dmax * 4 <= QL_SMEM_MAX ? 1 : 0;
+  if (simple && bc > 0 && m <= INT32_MAX && n <= INT32_MAX) {
+    const float* vs = V.kind == QUIP_T_HADAMARD ? V.signs : nullptr;
+    const float* us = U.kind == QUIP_T_HADAMARD ? U.signs : nullptr;
+    const float vscale = vs ? (float)(1.0 / std::sqrt((double)n)) : 1.f;
+    const float uscale = us ? (float)(1.0 / std::sqrt((double)m)) : 1.f;
+    const void* xin = x;
+    int64_t ldin = ldx;
+    if (kin) {
+      QCHECK(kron_vec(V, false, static_cast<const float*>(x), ldx, xs, n, B, st));
+      xin = xs, ldin = n;
+    }
+    float* yout = kout ? tmp : y;
+    const int64_t ldout = kout ? m : ldy;
+    cudaError_t e;
+    if (x_dtype == QUIP_BF16)
+      e = qlinear<__nv_bfloat16>(slot, packed, ldp, Wd, lo, scale, m, n, static_cast<const __nv_bfloat16*>(xin),
+                                 ldin, B, vs, vscale, us, uscale, z, counter, yout, ldout, bc, st);
+    else
+      e = qlinear<float>(slot, packed, ldp, Wd, lo, scale, m, n, static_cast<const float*>(xin), ldin, B, vs,
+                         vscale, us, uscale, z, counter, yout, ldout, bc, st);
+    QCHECK(e);
+    if (kout) QCHECK(kron_vec(U, true, tmp, m, y, ldy, B, st));
+    return QUIP_OK;
+  }
+  // x' = V x = T_n (P_n x), the vectors as rows
+  if (V.permute) {
+    if (x_dtype == QUIP_BF16)
+      QCHECK(gather2d<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x), ldx, xs, n, B, n, nullptr, V.perm, st));
+    else
+      QCHECK(gather2d<float>(static_cast<const float*>(x), ldx, xs, n, B, n, nullptr, V.perm, st));
+    QCHECK(side_rows<float>(V, false, xs, n, xs, B, tmp, st));
+  } else if (x_dtype == QUIP_BF16) {
+    QCHECK(side_rows<__nv_bfloat16>(V, false, static_cast<const __nv_bfloat16*>(x), ldx, xs, B, tmp, st));
+  } else {
+    QCHECK(side_rows<float>(V, false, static_cast<const float*>(x), ldx, xs, B, tmp, st));
+  }
+  // z = W~^ x'
+  switch (slot) {
+    case 1: QCHECK(qmatvec_slot<1>(packed, ldp, Wd, lo, scale, m, n, xs, B, z, st)); break;
+    case 2: QCHECK(qmatvec_slot<2>(packed, ldp, Wd, lo, scale, m, n, xs, B, z, st)); break;
+    case 4: QCHECK(qmatvec_slot<4>(packed, ldp, Wd, lo, scale, m, n, xs, B, z, st)); break;
+    default: QCHECK(qmatvec_slot<8>(packed, ldp, Wd, lo, scale, m, n, xs, B, z, st)); break;
+  }
+  // y = U^T z = P_m^T (T_m^T z)
+  if (U.permute || ldy != m) {
+    QCHECK(side_rows<float>(U, true, z, m, z, B, tmp, st));
+    QCHECK(gather2d<float>(z, m, y, ldy, B, m, nullptr, U.permute ? U.iperm : nullptr, st));
+  } else {
+    QCHECK(side_rows<float>(U, true, z, m, y, B, tmp, st));
+  }
+  return QUIP_OK;
 }
 
 quip_status quip_dequantize(const uint8_t* codes, const float* lo, const float* scale, int64_t m,

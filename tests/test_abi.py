@@ -87,6 +87,14 @@ def test_host_argument_errors(lib):
     assert g(ctypes.c_void_p(0x1004), 4, 64, 2, 1, fake, 1 << 30) == L.QUIP_ERR_ARG
     assert g(fake, 4, 64, 2, 1, fake, 16) == L.QUIP_ERR_WORKSPACE
     assert g(fake, 4, 64, 2, 0, fake, 1 << 30) == L.QUIP_OK          # no pass: nothing launched
+    # packing and the quantized product
+    assert lib.quip_packed_words(4096, 2) == 256 and lib.quip_packed_words(5, 3) == 4
+    assert lib.quip_packed_words(0, 2) == 0 and lib.quip_packed_words(8, 9) == 0
+    assert lib.quip_pack_codes(fake, 4, 8, 9, fake, 4, None) == L.QUIP_ERR_ARG
+    assert lib.quip_pack_codes(fake, 4, 64, 2, fake, 2, None) == L.QUIP_ERR_SHAPE      # ldp < 4
+    assert lib.quip_pack_codes(fake, 4, 64, 2, ctypes.c_void_p(0x1004), 4, None) == L.QUIP_ERR_SHAPE
+    assert lib.quip_qmatvec(None, fake, 4, fake, fake, 2, fake, L.QUIP_F32, 8, 1, fake, 8, fake, 1 << 20,
+                            None) == L.QUIP_ERR_ARG
 
 
 def test_workspace_sizes(lib):
