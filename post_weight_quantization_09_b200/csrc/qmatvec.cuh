@@ -4,8 +4,11 @@
 //   y = W^ x = U^T (W~^ (V x)),   W~^[i][j] = lo_i + s_i c_ij,
 // so the product in the incoherent domain is
 //   z_i = lo_i sum_j x'_j + s_i sum_j c_ij x'_j,   x' = V x,
-// and y = U^T z.  The transforms run as the library's row transforms; this
-// file holds the packing of the codes and the product kernel.
+// and y = U^T z.  This file holds the packing of the codes, the product
+// with the two transforms in the same launch (k_qlinear: Hadamard or
+// identity sides), a Kronecker side on a few vectors (k_kron_vec), and the
+// bare product (k_qmatvec) that the library's row transforms and gathers
+// surround when a side permutes.
 //
 // Packed layout (see quip.h): code j of row i sits in word j mod Wd of the
 // row at bit (j div Wd) * slot, Wd a multiple of 4.  A lane that loads the
