@@ -200,6 +200,43 @@ def roofline_entry(kind, amount, bound, ms, pk):
             "frac": round(achieved / peak, 4), "traffic": None}
 
 
+# Stages whose flops the library runs on the tensor cores as split-bf16
+# products (six bf16 products per fp32-accurate multiply-add), so their
+# fp32-algorithmic floor uses the bf16 peak / 6; the rest of their work (the
+# LDL's diagonal chain, LDLQ's in-block rounding) runs on the FP32 pipes.
+SPLIT_PRODUCTS = 6
+
+
+def pipeline_floor(cfg: LayerConfig, pk) -> dict:
+    """Speed-of-light time per stage: its work over the engine it runs on:
+    the bf16 Hessian at the bf16 tensor peak (an fp32 one at the FP32 FFMA
+    peak), the LDL and LDLQ flops at the fp32-accurate split-bf16 rate (bf16
+    peak / 6), every byte-counted stage at the measured HBM bandwidth.
+    Returns {stage: floor ms}."""
+    floors = {}
+    for name, (kind, amount, bound) in stage_work(cfg).items():
+        if kind == "bytes":
+            floors[name] = amount / (pk["hbm_gbs"] * 1e9) * 1e3
+        elif bound == "tensor":
+            floors[name] = amount / (pk["bf16_tflops"] * 1e12) * 1e3
+        elif name in ("ldl", "ldlq"):
+            floors[name] = amount / (pk["bf16_tflops"] / SPLIT_PRODUCTS * 1e12) * 1e3
+        else:                                           # fp32 inputs: FP32 pipes
+            floors[name] = amount / (FFMA_TFLOPS * 1e12) * 1e3
+    return floors
+
+
+def pipeline_entry(cfg: LayerConfig, pk, ms_per_step: float) -> dict:
+    """The pipeline fraction: the sum of the stages' floors / the measured step."""
+    floors = pipeline_floor(cfg, pk)
+    total = sum(floors.values())
+    return {"floor_ms": round(total, 4), "frac": round(total / ms_per_step, 4),
+            "stage_floor_ms": {k: round(v, 4) for k, v in floors.items()},
+            "denominators": f"HBM {pk['hbm_gbs']} GB/s; bf16 {pk['bf16_tflops']} TFLOP/s for the Hessian; "
+                            f"bf16 / {SPLIT_PRODUCTS} for the LDL and LDLQ flops (split-bf16 fp32-accurate "
+                            f"products); {pk['source']} peaks"}
+
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
 
@@ -535,6 +572,8 @@ def run_ours(args, cfg: LayerConfig):
         "config": config_desc(cfg, args),
         "roofline": roof,
         "stages": stages,
+        # speed of light of the LDLQ pipeline's stages over the measured step
+        **({"pipeline": pipeline_entry(cfg, pk, ms_per_step)} if args.method == "ldlq" else {}),
         "kernels": kernels,
         "e2e": {"value": job_throughput(cfg, world, e2e), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
