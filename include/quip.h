@@ -261,9 +261,12 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
  * library until the process exits.  Layers whose workspace
  * (quip_workspace_size(QUIP_OP_LDLQ, ...)) is larger are rejected with
  * QUIP_ERR_WORKSPACE before anything is launched.
- *  - The first call on each device looks up the array's device address for
- *    that device (it must be the current device); make that first call
- *    before any stream capture.
+ *  - Every call outside stream capture looks up the array's device address
+ *    on the current device (so a cudaDeviceReset in between is harmless); a
+ *    call whose stream is capturing reuses the address of the last call
+ *    outside capture on that device, so make one call on each device before
+ *    capturing (a device never called outside capture returns
+ *    QUIP_ERR_CUDA), and none between a cudaDeviceReset and a capture.
  *  - Every call on a device shares the one array and it keeps the last
  *    call's contents; nothing in it needs to start at zero (every call
  *    overwrites what it reads).  Calls whose work overlaps on the GPU

@@ -29,7 +29,7 @@ reading used here (and by the CUDA path) is the one the rest of the text
 supports: H = (I + U)(D)(I + U)^T with U strictly upper triangular, and
 W^_k = Q(W_k + (W - W^) U_k), column k using only columns j < k.
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings where the pages are silent (the CUDA path takes the same ones):
   * grid: per-row asymmetric min/max grid of 2^b levels over the whole
     incoherent row, fixed before rounding; s = (hi - lo) / (2^b - 1); a
     constant row uses s = 1;
@@ -68,7 +68,8 @@ import numpy as np
 __all__ = [
     "hessian", "damp", "splitmix64", "uniform53", "random_signs", "gaussian_matrix",
     "haar_orthogonal", "sylvester_hadamard", "hadamard_row", "SideTransform", "make_side",
-    "incoherence_forward", "incoherence_inverse", "incoherence_rows", "incoherence_hessian", "udu", "row_grid", "quantize",
+    "incoherence_forward", "incoherence_inverse", "incoherence_rows", "incoherence_hessian", "incoherence_hessian_rows",
+    "incoherence_inverse_rows", "udu", "row_grid", "quantize",
     "ldlq", "ldlq_blocked", "nearest", "optq", "dequantize", "proxy_loss", "Pipeline",
     "run_pipeline", "STREAM_M_SIGNS", "STREAM_N_SIGNS", "STREAM_M_A", "STREAM_M_B",
     "STREAM_N_A", "STREAM_N_B", "STREAM_M_PERM", "STREAM_N_PERM", "random_permutation",
@@ -243,6 +244,20 @@ class SideTransform:
             r = np.kron(self.A[i // q], self.B[i % q])
         return r if self.perm is None else r @ self.perm_matrix()
 
+    def col(self, i: int) -> np.ndarray:
+        """Column i of S (row i of S^T, what the inverse transform applies)."""
+        d = self.dim
+        j = i if self.perm is None else int(np.flatnonzero(self.perm == i)[0])
+        if self.kind == "identity":
+            c = np.zeros(d)
+            c[j] = 1.0
+        elif self.kind == "hadamard":
+            c = hadamard_row(d, j) * (self.signs[j] / math.sqrt(d))   # H_d is symmetric
+        else:
+            q = self.B.shape[0]
+            c = np.kron(self.A[:, j // q], self.B[:, j % q])
+        return c
+
 
 def make_side(seed: int, side: str, kind: str, dim: int, p: int = 0, q: int = 0,
               permute: bool = False) -> SideTransform:
@@ -292,6 +307,21 @@ def incoherence_hessian(H: np.ndarray, V: SideTransform) -> np.ndarray:
     Vn = V.matrix()
     Ht = Vn @ np.asarray(H, dtype=np.float64) @ Vn.T
     return 0.5 * (Ht + Ht.T)
+
+
+def incoherence_hessian_rows(H: np.ndarray, V: SideTransform, rows) -> np.ndarray:
+    """Rows `rows` of V H V^T (before symmetrisation), row i being
+    V[i, :] H V^T: the Hessian transform restricted to some rows."""
+    Vr = np.stack([V.row(int(i)) for i in rows])
+    return (Vr @ np.asarray(H, dtype=np.float64)) @ V.matrix().T
+
+
+def incoherence_inverse_rows(Wt_hat: np.ndarray, U: SideTransform, V: SideTransform, rows
+                             ) -> np.ndarray:
+    """Rows `rows` of W^ = U^T W~^ V, row i being U[:, i]^T W~^ V: the
+    inverse transform restricted to some output rows."""
+    Uc = np.stack([U.col(int(i)) for i in rows])
+    return (Uc @ np.asarray(Wt_hat, dtype=np.float64)) @ V.matrix()
 
 
 def incoherence_inverse(Wt_hat: np.ndarray, U: SideTransform, V: SideTransform) -> np.ndarray:

@@ -3,23 +3,25 @@
 // x2 = bf16(x - x0 - x1)), so x is carried to ~24 significant bits.  The
 // product sum_k a_k b_k is formed from the six piece products whose order is
 // at most 2 (x_i y_j, i + j <= 2); the three dropped ones are below 2^-27
-// relative.  bf16 x bf16 products are exact in the fp32 accumulator.  The
-// terms run smallest first, (2,0) (1,1) (0,2) (1,0) (0,1) (0,0), so the
-// accumulator's own rounding acts on small partial sums for as long as
-// possible.
+// relative.  bf16 x bf16 products are exact in the fp32 accumulator.
 //
 //   C[i][j] += alpha * sum_t sum_k A_pa(t)[i][k] * B_pb(t)[j][k]
 //
 // Both operands K-major (row-major [rows][K] bf16, piece p at row offset
 // p * piece_rows), loaded by TMA as 64-wide K boxes with the 128-byte swizzle.
-// Tile 128 x TN (TN = 256, or 64 for narrow outputs), one M=128 N=TN K=16
-// tcgen05.mma per 16 k; 4-stage smem ring (16 KB + TN x 128 B per stage).
+// Tile 128 x TN (TN = 256, or 128 / 64 for narrow outputs), one M=128 N=TN
+// K=16 tcgen05.mma per 16 k.  Every piece is loaded once per 64-wide K block:
+// the three A pieces together into one of two A slots (48 KB), the B pieces
+// one at a time into a ring of B slots, B2 first; the terms that need a B
+// piece run as soon as it lands: (0,2), then (1,1) (0,1), then (2,0) (1,0)
+// (0,0), so within a K block the small terms come first.
 // The tensor core's fp32 accumulation drops low bits (about one ulp of the
-// running sum per MMA), so K is cut into chunks of KCP = 512 per piece: each
-// chunk (all six terms) accumulates into a fresh TMEM buffer (columns
-// [0, TN)), and the epilogue folds it into an fp32 running sum kept in a
-// second TMEM buffer (columns [TN, 2 TN)) with round-to-nearest adds; the
-// tile's sum is added to C once, at its last chunk.
+// running sum per MMA), so K is cut into chunks of KCP = 512 per piece, each
+// accumulated in a fresh TMEM buffer.  With more than one chunk per tile the
+// epilogue folds each chunk into an fp32 running sum kept in a second TMEM
+// buffer (round-to-nearest adds) and adds the tile's sum to C once, at its
+// last chunk; with one chunk per tile the two TMEM buffers take alternate
+// tiles, so the next tile's products overlap this tile's epilogue.
 // Bounded mbarrier waits as in the SYRK.
 #pragma once
 
@@ -29,13 +31,16 @@ namespace quip {
 namespace sgemm {
 
 // Tile N width BN: 256, or 128 / 64 for narrow outputs (more tiles, more CTAs).
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;              // 16 KB
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int A_PIECE_BYTES = BM * BK * 2;        // 16 KB
+constexpr int A_BYTES = 3 * A_PIECE_BYTES;        // one A slot: the three pieces
+constexpr int A_SLOTS = 2;
 template <int TN> __host__ __device__ constexpr int b_bytes() { return TN * BK * 2; }
-template <int TN> __host__ __device__ constexpr int stage_bytes() { return A_BYTES + b_bytes<TN>(); }
-template <int TN> __host__ __device__ constexpr int smem_bytes() { return STAGES * stage_bytes<TN>() + 1024 + 256; }
+template <int TN> __host__ __device__ constexpr int b_slots() { return TN == 256 ? 4 : 8; }
+template <int TN> __host__ __device__ constexpr int smem_bytes() {
+  return A_SLOTS * A_BYTES + b_slots<TN>() * b_bytes<TN>() + 1024 + 256;
+}
 constexpr int SMEM_BYTES = smem_bytes<BN>();
-constexpr int NTERMS = 6;
 
 struct Params {
   float* C;
@@ -53,19 +58,15 @@ struct Params {
 constexpr int KCP = 512;                           // K per piece per accumulation chunk
 
 struct Shared {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
-  uint64_t tfull;          // chunk accumulated (MMA -> epilogue)
-  uint64_t tempty;         // chunk buffer drained (epilogue -> MMA)
+  uint64_t full_a[A_SLOTS];
+  uint64_t empty_a[A_SLOTS];
+  uint64_t full_b[8];
+  uint64_t empty_b[8];
+  uint64_t tfull[2];       // accumulator buffer complete (MMA -> epilogue)
+  uint64_t tempty[2];      // accumulator buffer drained (epilogue -> MMA)
   uint32_t tmem_base;
   int abort;
 };
-
-__device__ __forceinline__ void term_pieces(int t, int& pa, int& pb) {
-  // (2,0) (1,1) (0,2) (1,0) (0,1) (0,0), one nibble per term
-  pa = (int)((0x001012u >> (4 * t)) & 0xFu);
-  pb = (int)((0x010210u >> (4 * t)) & 0xFu);
-}
 
 // Tile t of the grid (row-major over tiles_m x tiles_n); false if skipped.
 template <int TN>
@@ -76,38 +77,44 @@ __device__ __forceinline__ bool tile_coords(const Params& p, int t, int& i0, int
   return !(p.upper_only && i0 > j0 + TN - 1);
 }
 
-// K-step `st` of a chunk covering piece columns [kc0, kc0 + kcl): term and offset.
-__device__ __forceinline__ void chunk_step(int st, int kcl, int& term, int& kk) {
-  const int per = kcl / BK;
-  term = st / per;
-  kk = (st % per) * BK;
-}
-
 // Persistent: CTA b handles tiles b, b + gridDim.x, ...  Warp 0 lane 0: TMA
 // producer; warp 1 lane 0: MMA issuer; warps 4..7: epilogue (warp w reads
 // TMEM lanes 32 (w - 4)..; one output row per thread, TN columns).
+// Accumulator buffers: with one chunk per tile (K <= KCP) buffer (local tile
+// index & 1); otherwise buffer 0 takes every chunk and buffer 1 holds the
+// running sum.
 template <int TN>
 __global__ void __launch_bounds__(256, 1)
     k_gemm_split_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     Params p, int ntiles) {
-  constexpr int STAGE_BYTES = stage_bytes<TN>();
+  constexpr int B_BYTES = b_bytes<TN>();
+  constexpr int NB = b_slots<TN>();
   constexpr uint32_t IDESC = make_idesc_bf16(BM, TN, 0, 0);
-  constexpr uint32_t TCOLS = 2 * TN;               // chunk buffer + running sum
+  constexpr uint32_t TCOLS = 2 * TN;
   extern __shared__ uint8_t smem_raw[];
   pdl_wait_then_release();
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Shared* sh = reinterpret_cast<Shared*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* sa = smem;                                // A slots
+  uint8_t* sb = smem + A_SLOTS * A_BYTES;            // B slots
+  Shared* sh = reinterpret_cast<Shared*>(sb + NB * B_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nchunk = (p.K + KCP - 1) / KCP;
+  const bool single = nchunk == 1;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&sh->full[s], 1);
-      mbar_init(&sh->empty[s], 1);
+    for (int s = 0; s < A_SLOTS; ++s) {
+      mbar_init(&sh->full_a[s], 1);
+      mbar_init(&sh->empty_a[s], 1);
     }
-    mbar_init(&sh->tfull, 1);
-    mbar_init(&sh->tempty, 4);                      // one arrival per epilogue warp
+    for (int s = 0; s < NB; ++s) {
+      mbar_init(&sh->full_b[s], 1);
+      mbar_init(&sh->empty_b[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sh->tfull[b], 1);
+      mbar_init(&sh->tempty[b], 4);                 // one arrival per epilogue warp
+    }
     sh->abort = 0;
     fence_mbar_init();
   }
@@ -120,67 +127,87 @@ __global__ void __launch_bounds__(256, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    int it = 0;                                     // global K-step counter (stage ring)
+    int ka = 0, kb = 0;                             // A-slot and B-slot counters
     for (int t = blockIdx.x; t < ntiles && !sh->abort; t += gridDim.x) {
       int i0, j0;
       if (!tile_coords<TN>(p, t, i0, j0)) continue;
-      for (int c = 0; c < nchunk && !sh->abort; ++c) {
-        const int kc0 = c * KCP, kcl = min(KCP, p.K - kc0);
-        const int steps = NTERMS * (kcl / BK);
-        for (int st = 0; st < steps; ++st, ++it) {
-          const int s = it % STAGES;
-          if (!mbar_wait(&sh->empty[s], (uint32_t)(((it / STAGES) & 1) ^ 1))) {
+      for (int k = 0; k < p.K && !sh->abort; k += BK, ++ka) {
+        const int s = ka % A_SLOTS;
+        if (!mbar_wait(&sh->empty_a[s], (uint32_t)(((ka / A_SLOTS) & 1) ^ 1))) {
+          sh->abort = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&sh->full_a[s], A_BYTES);
+#pragma unroll
+        for (int pa = 0; pa < 3; ++pa)
+          tma_load_2d(sa + s * A_BYTES + pa * A_PIECE_BYTES, &tmA, &sh->full_a[s], p.a_k0 + k,
+                      pa * p.a_piece_rows + p.a_row0 + i0);
+        for (int pb = 2; pb >= 0; --pb, ++kb) {
+          const int r = kb % NB;
+          if (!mbar_wait(&sh->empty_b[r], (uint32_t)(((kb / NB) & 1) ^ 1))) {
             sh->abort = 1;
             break;
           }
-          int term, kk, pa, pb;
-          chunk_step(st, kcl, term, kk);
-          term_pieces(term, pa, pb);
-          uint8_t* a = smem + s * STAGE_BYTES;
-          mbar_arrive_expect_tx(&sh->full[s], STAGE_BYTES);
-          tma_load_2d(a, &tmA, &sh->full[s], p.a_k0 + kc0 + kk, pa * p.a_piece_rows + p.a_row0 + i0);
-          tma_load_2d(a + A_BYTES, &tmB, &sh->full[s], p.b_k0 + kc0 + kk,
-                      pb * p.b_piece_rows + p.b_row0 + j0);
+          mbar_arrive_expect_tx(&sh->full_b[r], B_BYTES);
+          tma_load_2d(sb + r * B_BYTES, &tmB, &sh->full_b[r], p.b_k0 + k, pb * p.b_piece_rows + p.b_row0 + j0);
         }
       }
     }
   } else if (warp == 1 && lane == 0) {
-    int it = 0, gc = 0;                             // gc: global chunk counter
+    int ka = 0, kb = 0, gc = 0, lt = 0;             // gc: chunks, lt: tiles of this CTA
     for (int t = blockIdx.x; t < ntiles && !sh->abort; t += gridDim.x) {
       int i0, j0;
       if (!tile_coords<TN>(p, t, i0, j0)) continue;
       for (int c = 0; c < nchunk && !sh->abort; ++c, ++gc) {
-        if (!mbar_wait(&sh->tempty, (uint32_t)((gc & 1) ^ 1))) {   // chunk buffer free
+        // single chunk: buffer lt & 1, its use count lt >> 1; else buffer 0, use count gc
+        const int buf = single ? (lt & 1) : 0;
+        const int use = single ? (lt >> 1) : gc;
+        if (!mbar_wait(&sh->tempty[buf], (uint32_t)((use & 1) ^ 1))) {
           sh->abort = 1;
           break;
         }
         tc_fence_after();
-        const int kcl = min(KCP, p.K - c * KCP);
-        const int steps = NTERMS * (kcl / BK);
-        for (int st = 0; st < steps; ++st, ++it) {
-          const int s = it % STAGES;
-          if (!mbar_wait(&sh->full[s], (uint32_t)((it / STAGES) & 1))) {
+        const uint32_t acc = tmem + (uint32_t)(buf * TN);
+        const int kc0 = c * KCP, kc1 = min(p.K, kc0 + KCP);
+        bool first = true;
+        for (int k = kc0; k < kc1 && !sh->abort; k += BK, ++ka) {
+          const int s = ka % A_SLOTS;
+          if (!mbar_wait(&sh->full_a[s], (uint32_t)((ka / A_SLOTS) & 1))) {
             sh->abort = 1;
             break;
           }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
-          const uint32_t b_addr = a_addr + A_BYTES;
+          const uint32_t a_base = smem_u32(sa + s * A_BYTES);
+          for (int pb = 2; pb >= 0; --pb, ++kb) {
+            const int r = kb % NB;
+            if (!mbar_wait(&sh->full_b[r], (uint32_t)((kb / NB) & 1))) {
+              sh->abort = 1;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t b_addr = smem_u32(sb + r * B_BYTES);
+            // the A pieces pa with pa + pb <= 2, larger pa (smaller term) first
+            for (int pa = 2 - pb; pa >= 0; --pa) {
+              const uint32_t a_addr = a_base + pa * A_PIECE_BYTES;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            // K-major SW128: 8-row groups 1024 B apart; K advances 32 B per 16 elements
-            const uint64_t adesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
-            const uint64_t bdesc = make_sw128_desc(b_addr + k * 32, 16, 1024);
-            tc_mma_f16(tmem, adesc, bdesc, IDESC, (st | k) != 0);
+              for (int kk = 0; kk < BK / 16; ++kk) {
+                // K-major SW128: 8-row groups 1024 B apart; K advances 32 B per 16 elements
+                const uint64_t adesc = make_sw128_desc(a_addr + kk * 32, 16, 1024);
+                const uint64_t bdesc = make_sw128_desc(b_addr + kk * 32, 16, 1024);
+                tc_mma_f16(acc, adesc, bdesc, IDESC, first ? 0u : 1u);
+                first = false;
+              }
+            }
+            tc_commit(&sh->empty_b[r]);
           }
-          tc_commit(&sh->empty[s]);
+          tc_commit(&sh->empty_a[s]);
         }
-        tc_commit(&sh->tfull);
+        tc_commit(&sh->tfull[buf]);
       }
+      ++lt;
     }
   } else if (warp >= 4) {
     const int quarter = warp - 4;
-    int gc = 0;
+    int gc = 0, lt = 0;
     bool stop = false;
     for (int t = blockIdx.x; t < ntiles && !stop; t += gridDim.x) {
       int i0, j0;
@@ -191,7 +218,9 @@ __global__ void __launch_bounds__(256, 1)
       const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
       const bool vec = (p.ldc & 3) == 0;
       for (int c = 0; c < nchunk; ++c, ++gc) {
-        bool ok = mbar_wait(&sh->tfull, (uint32_t)(gc & 1));
+        const int buf = single ? (lt & 1) : 0;
+        const int use = single ? (lt >> 1) : gc;
+        bool ok = mbar_wait(&sh->tfull[buf], (uint32_t)(use & 1));
         ok = __all_sync(0xffffffffu, ok) && !sh->abort;
         if (!ok) {
           stop = true;
@@ -199,40 +228,44 @@ __global__ void __launch_bounds__(256, 1)
         }
         tc_fence_after();
         const bool first = c == 0, last = c == nchunk - 1;
+        const uint32_t tb = tmem + lanes + (uint32_t)(buf * TN);
 #pragma unroll 1
         for (int c8 = 0; c8 < TN / 32; ++c8) {
           float v[32];
-          tmem_ld32(tmem + lanes + c8 * 32, v);
-          if (!first) {
-            float su[32];
-            tmem_ld32(tmem + lanes + TN + c8 * 32, su);
+          tmem_ld32(tb + c8 * 32, v);
+          if (!single) {
+            if (!first) {
+              float su[32];
+              tmem_ld32(tmem + lanes + TN + c8 * 32, su);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] += su[e];
+              for (int e = 0; e < 32; ++e) v[e] += su[e];
+            }
+            if (!last) {
+              tmem_st32(tmem + lanes + TN + c8 * 32, v);
+              continue;
+            }
           }
-          if (!last) {
-            tmem_st32(tmem + lanes + TN + c8 * 32, v);
-          } else {
-            // C += alpha * sum through fire-and-forget vector reductions in L2
-            const int jc = j0 + c8 * 32;
-            if (rok && jc < p.N) {
-              if (vec && jc + 32 <= p.N) {
-                float4* dst = reinterpret_cast<float4*>(crow + jc);
+          // C += alpha * sum through fire-and-forget vector reductions in L2
+          const int jc = j0 + c8 * 32;
+          if (rok && jc < p.N) {
+            if (vec && jc + 32 <= p.N) {
+              float4* dst = reinterpret_cast<float4*>(crow + jc);
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
-                  atomicAdd(dst + q, make_float4(p.alpha * v[4 * q], p.alpha * v[4 * q + 1],
-                                                 p.alpha * v[4 * q + 2], p.alpha * v[4 * q + 3]));
-              } else {
+              for (int q = 0; q < 8; ++q)
+                atomicAdd(dst + q, make_float4(p.alpha * v[4 * q], p.alpha * v[4 * q + 1],
+                                               p.alpha * v[4 * q + 2], p.alpha * v[4 * q + 3]));
+            } else {
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                  if (jc + e < p.N) atomicAdd(crow + jc + e, p.alpha * v[e]);
-              }
+              for (int e = 0; e < 32; ++e)
+                if (jc + e < p.N) atomicAdd(crow + jc + e, p.alpha * v[e]);
             }
           }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sh->tempty);
+        if (lane == 0) mbar_arrive(&sh->tempty[buf]);
       }
+      ++lt;
     }
   }
   __syncwarp();

@@ -21,6 +21,7 @@
 #include "qmatvec.cuh"
 #include "syrk_tc.cuh"
 #include "gemm_tc.cuh"
+#include "kron_tc.cuh"
 
 using namespace quip;
 
@@ -41,12 +42,33 @@ struct SideData {
   double* A64 = nullptr;    // KRONECKER: the same factors in fp64 (Hessian transform)
   double* B64 = nullptr;
   double* G = nullptr;      // KRONECKER: Gaussian draw scratch, max(p,q)^2
-  double* Qc = nullptr;     // KRONECKER: CGS2 scratch, max(p,q)^2
+  double* Qc = nullptr;     // KRONECKER: QR scratch, max(p,q)^2
+  // KRONECKER: three bf16 pieces of A, A^T, B, B^T for the tensor-core
+  // products, each 3 x d x ld_piece(d) (rows padded to 16 bytes)
+  __nv_bfloat16* fpc = nullptr;
   bool permute = false;     // S = T P, (P x)_r = x_{perm[r]}
   int32_t* perm = nullptr;  // pi (dim)
   int32_t* iperm = nullptr; // pi^-1 (dim)
   uint64_t* keys = nullptr; // permutation draws (dim)
 };
+
+// Row stride (elements) of a d x d factor's bf16 pieces: rows padded to 16
+// bytes, as TMA requires.
+static int64_t factor_ld(int64_t d) { return (d + 7) / 8 * 8; }
+static int64_t factor_pieces_elems(int64_t p, int64_t q) {
+  return 6 * (p * factor_ld(p) + q * factor_ld(q));
+}
+// Pieces of factor v: 0 = A, 1 = A^T, 2 = B, 3 = B^T (each 3 x d x factor_ld(d)).
+static __nv_bfloat16* factor_pieces(const SideData& sd, int v) {
+  const int64_t a = 3 * sd.p * factor_ld(sd.p), b = 3 * sd.q * factor_ld(sd.q);
+  switch (v) {
+    case 0: return sd.fpc;
+    case 1: return sd.fpc + a;
+    case 2: return sd.fpc + 2 * a;
+    default: return sd.fpc + 2 * a + b;
+  }
+}
+
 
 inline bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
 inline int ilog2(int64_t x) {
@@ -404,6 +426,87 @@ cudaError_t kron_cols(float* X, int64_t ncols, const SideData& sd, bool transpos
   return gemm_simt<F, float, Acc>(h, 1, st);
 }
 
+// ---------------------------------------------------------------- Kronecker on the tensor cores
+
+// One batched factor product Y[z] = F X[z] (kron_tc.cuh).
+cudaError_t kron_tc_launch(const CUtensorMap& tf, const CUtensorMap& tx, kron::Params kp, int mode,
+                           cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(kron::k_kron_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kron::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  kp.tiles_m = (kp.M + kron::BM - 1) / kron::BM;
+  kp.tiles_n = (kp.N + kron::BN - 1) / kron::BN;
+  const int64_t tiles = (int64_t)kp.tiles_m * kp.tiles_n * kp.slabs;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, num_sms()));
+  LaunchScope ls("k_kron_tc", st);
+  return launch_pdl(kron::k_kron_tc, dim3(grid), dim3(256), (size_t)kron::SMEM_BYTES, st, tf, tx, kp, mode);
+}
+
+// Whether the m-side (column) Kronecker transform of an R x c matrix runs on
+// the tensor cores: TMA needs 16-byte row strides (c % 8 == 0), the products
+// index tiles with 32-bit coordinates.
+bool kron_cols_tc_ok(const SideData& sd, int64_t c) {
+  return sd.kind == QUIP_T_KRONECKER && c >= 8 && (c % 8) == 0 && sd.p * sd.q * 3 < ((int64_t)1 << 31) &&
+         sd.q * c < ((int64_t)1 << 31);
+}
+
+// Workspace of kron_cols_tc: two sets of three bf16 pieces of the R x c data.
+size_t kron_cols_tc_bytes(int64_t R, int64_t c) { return 2 * round256((size_t)3 * R * c * 2); }
+
+// dst (R x c fp32, row stride c) = (A' (x) B') src on the tensor cores, with
+// A' = A, B' = B (forward) or A^T, B^T (inverse).  src: bf16 (one piece) or
+// fp32 (split into three pieces first), row stride ld.  dst may alias an
+// fp32 src.  ws: kron_cols_tc_bytes(R, c).
+template <typename TIn>
+cudaError_t kron_cols_tc(const SideData& sd, bool transpose, const TIn* src, int64_t ld, float* dst,
+                         int64_t c, void* ws, cudaStream_t st) {
+  const int64_t p = sd.p, q = sd.q, R = p * q;
+  __nv_bfloat16* P1 = static_cast<__nv_bfloat16*>(ws);
+  __nv_bfloat16* P2 = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + round256((size_t)3 * R * c * 2));
+  const __nv_bfloat16* xsrc;
+  int xp;
+  int64_t xld;
+  if constexpr (std::is_same<TIn, __nv_bfloat16>::value) {
+    xsrc = src, xp = 1, xld = ld;
+  } else {
+    const int64_t total4 = R * c / 4;
+    const unsigned g = (unsigned)std::min<int64_t>((total4 + 255) / 256, 148 * 16);
+    {
+      LaunchScope ls("k_split_rows3", st);
+      k_split_rows3<<<g, 256, 0, st>>>(src, ld, R, c, P1);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    xsrc = P1, xp = 3, xld = c;
+  }
+  // stage 1: T_a' = B' X_a' for the p slabs of q rows, into P2 as pieces
+  CUtensorMap mf, mx;
+  const __nv_bfloat16* fb = factor_pieces(sd, transpose ? 3 : 2);
+  if (!make_tmap_bf16_2d(&mf, fb, (uint64_t)q, 3 * (uint64_t)q, (uint64_t)factor_ld(q) * 2, 64, kron::BM) ||
+      !make_tmap_bf16_2d(&mx, xsrc, (uint64_t)c, (uint64_t)(xp * R), (uint64_t)xld * 2, 64, 64))
+    return cudaErrorInvalidValue;
+  kron::Params kp{};
+  kp.M = (int)q, kp.K = (int)q, kp.N = (int)c, kp.slabs = (int)p;
+  kp.f_piece_rows = (int)q, kp.x_pieces = xp, kp.x_piece_rows = R, kp.x_slab_rows = q;
+  kp.Yp = P2, kp.ldy = c, kp.y_slab_rows = q, kp.y_piece_elems = R * c;
+  cudaError_t e = kron_tc_launch(mf, mx, kp, kron::OUT_PIECES, st);
+  if (e != cudaSuccess) return e;
+  // stage 2: Y = A' T with T as p x (q c), into dst (fp32)
+  const __nv_bfloat16* fa = factor_pieces(sd, transpose ? 1 : 0);
+  if (!make_tmap_bf16_2d(&mf, fa, (uint64_t)p, 3 * (uint64_t)p, (uint64_t)factor_ld(p) * 2, 64, kron::BM) ||
+      !make_tmap_bf16_2d(&mx, P2, (uint64_t)(q * c), 3 * (uint64_t)p, (uint64_t)(q * c) * 2, 64, 64))
+    return cudaErrorInvalidValue;
+  kron::Params k2{};
+  k2.M = (int)p, k2.K = (int)p, k2.N = (int)(q * c), k2.slabs = 1;
+  k2.f_piece_rows = (int)p, k2.x_pieces = 3, k2.x_piece_rows = p, k2.x_slab_rows = 0;
+  k2.Y = dst, k2.ldy = q * c, k2.y_slab_rows = 0;
+  return kron_tc_launch(mf, mx, k2, kron::OUT_F32, st);
+}
+
 __global__ void k_convert_rows_bf16(const __nv_bfloat16* in, int64_t ld, float* out, int64_t m,
                                     int64_t n) {
   const int64_t total = m * n;
@@ -419,9 +522,12 @@ __global__ void k_copy_rows_f32(const float* in, int64_t ld, float* out, int64_t
 }
 
 // n-side (row) transform of an m x n source into dst (row stride n).
+// wide: a Kronecker side takes fp64 factors and sums (the forward transform of
+// W: the rounding decisions of LDLQ are sensitive to the error of W~ itself,
+// and an fp32 sum over a factor row carries ~sqrt(q) u of it).
 template <typename TIn>
 cudaError_t side_rows(const SideData& sd, bool inverse, const TIn* src, int64_t ldsrc, float* dst,
-                      int64_t rows, float* tmp, cudaStream_t st) {
+                      int64_t rows, float* tmp, cudaStream_t st, bool wide = false) {
   const int64_t n = sd.dim;
   if (sd.kind == QUIP_T_HADAMARD) {
     const float scale = (float)(1.0 / std::sqrt((double)n));
@@ -429,7 +535,9 @@ cudaError_t side_rows(const SideData& sd, bool inverse, const TIn* src, int64_t 
     return fwht_rows<TIn>(src, ldsrc, dst, n, rows, n, inverse ? nullptr : sd.signs,
                           inverse ? sd.signs : nullptr, nullptr, scale, st);
   }
-  if (sd.kind == QUIP_T_KRONECKER) return kron_rows<TIn>(src, ldsrc, dst, rows, sd, inverse, tmp, st);
+  if (sd.kind == QUIP_T_KRONECKER)
+    return wide ? kron_rows<TIn, double>(src, ldsrc, dst, rows, sd, inverse, tmp, st)
+                : kron_rows<TIn>(src, ldsrc, dst, rows, sd, inverse, tmp, st);
   // identity
   const unsigned grid = (unsigned)std::min<int64_t>((rows * n + 255) / 256, 65535 * 8);
   if constexpr (std::is_same<TIn, float>::value) {
@@ -570,6 +678,7 @@ static quip_status alloc_side(SideData& sd, int kind_flags, int64_t dim, int64_t
     QCHECK(cudaMalloc(&sd.B64, q * q * sizeof(double)));
     QCHECK(cudaMalloc(&sd.G, mx * mx * sizeof(double)));
     QCHECK(cudaMalloc(&sd.Qc, mx * mx * sizeof(double)));
+    QCHECK(cudaMalloc(&sd.fpc, factor_pieces_elems(p, q) * sizeof(__nv_bfloat16)));
   }
   return QUIP_OK;
 }
@@ -597,9 +706,44 @@ static quip_status draw_side(const SideData& sd, uint64_t seed, int which, cudaS
         LaunchScope ls("k_gaussian", st);
         k_gaussian<<<(unsigned)((d * d + 255) / 256), 256, 0, st>>>(sd.G, d * d, seed, f == 0 ? sa : sb);
       }
-      LaunchScope ls("k_haar_cgs2", st);
-      k_haar_cgs2<<<1, 256, 0, st>>>(sd.G, sd.Qc, f == 0 ? sd.A : sd.B, f == 0 ? sd.A64 : sd.B64,
-                                       (int)d);
+      float* Q = f == 0 ? sd.A : sd.B;
+      double* Q64 = f == 0 ? sd.A64 : sd.B64;
+      if (d > HAAR_CHOL_MAX) {
+        LaunchScope ls("k_haar_cgs2", st);
+        k_haar_cgs2<<<1, 256, 0, st>>>(sd.G, sd.Qc, Q, Q64, (int)d);
+        continue;
+      }
+      // Cholesky-QR2: Y = G R1^-1 (into Qc, which first holds G^T G), then
+      // Q = Y R2^-1 (G, no longer needed, holds Y^T Y)
+      static bool attr = false;
+      if (!attr) {
+        QCHECK(cudaFuncSetAttribute(k_chol_solve64, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)chol_solve_smem(HAAR_CHOL_MAX)));
+        attr = true;
+      }
+      const unsigned t = (unsigned)((d + 31) / 32);
+      const size_t smem = chol_solve_smem((int)d);
+      {
+        LaunchScope ls("k_gram64", st);
+        k_gram64<<<dim3(t, t), 256, 0, st>>>(sd.G, sd.Qc, (int)d);
+      }
+      {
+        LaunchScope ls("k_chol_solve64", st);
+        k_chol_solve64<<<1, 1024, smem, st>>>(sd.Qc, sd.G, sd.Qc, nullptr, (int)d);
+      }
+      {
+        LaunchScope ls("k_gram64", st);
+        k_gram64<<<dim3(t, t), 256, 0, st>>>(sd.Qc, sd.G, (int)d);
+      }
+      LaunchScope ls("k_chol_solve64", st);
+      k_chol_solve64<<<1, 1024, smem, st>>>(sd.G, sd.Qc, Q64, Q, (int)d);
+    }
+    // bf16 pieces of A, A^T, B, B^T for the tensor-core products
+    for (int v = 0; v < 4; ++v) {
+      const int64_t d = v < 2 ? sd.p : sd.q;
+      LaunchScope ls("k_split_factor", st);
+      k_split_factor<<<(unsigned)((d * d + 255) / 256), 256, 0, st>>>(
+          v < 2 ? sd.A : sd.B, (int)d, (int)(v & 1), (int)factor_ld(d), factor_pieces(sd, v));
     }
   }
   QCHECK(cudaGetLastError());
@@ -645,6 +789,7 @@ quip_status quip_transform_destroy(quip_transform* tf) {
     cudaFree(sd.B64);
     cudaFree(sd.G);
     cudaFree(sd.Qc);
+    cudaFree(sd.fpc);
     cudaFree(sd.perm);
     cudaFree(sd.iperm);
     cudaFree(sd.keys);
@@ -775,11 +920,17 @@ static int64_t packed_row_words(int64_t n, int bits) {
 // Transform workspace: Kronecker temporaries, then the permutation scratch
 // (the forward pass gathers H into it, the inverse gathers W^).
 static size_t transform_kron_bytes(const quip_transform* tf, int op) {
-  const bool kron = tf->side[0].kind == QUIP_T_KRONECKER || tf->side[1].kind == QUIP_T_KRONECKER;
-  if (!kron) return 0;
-  size_t e = (size_t)tf->m * tf->n;
-  if (op == QUIP_OP_INCOHERENCE_FORWARD) e = std::max(e, (size_t)tf->n * tf->n);
-  return round256(e * sizeof(float));
+  const SideData &U = tf->side[0], &V = tf->side[1];
+  const bool u_tc = kron_cols_tc_ok(U, tf->n);
+  size_t b = 0;
+  if (V.kind == QUIP_T_KRONECKER || (U.kind == QUIP_T_KRONECKER && !u_tc)) {
+    // CUDA-core temporaries: one m x n (and, forward, n x n) fp32 matrix
+    size_t e = (size_t)tf->m * tf->n;
+    if (op == QUIP_OP_INCOHERENCE_FORWARD) e = std::max(e, (size_t)tf->n * tf->n);
+    b = round256(e * sizeof(float));
+  }
+  if (u_tc) b = std::max(b, kron_cols_tc_bytes(tf->m, tf->n));   // tensor-core pieces
+  return b;
 }
 static size_t transform_perm_bytes(const quip_transform* tf, int op) {
   if (op == QUIP_OP_INCOHERENCE_FORWARD)
@@ -849,22 +1000,31 @@ quip_status quip_incoherence_forward(const quip_transform* tf, const void* W, in
   float* tmp = static_cast<float*>(ws);
   float* pscr = reinterpret_cast<float*>(static_cast<char*>(ws) +
                                          transform_kron_bytes(tf, QUIP_OP_INCOHERENCE_FORWARD));
+  const bool u_tc = kron_cols_tc_ok(U, n);
   if (W) {
     const int32_t* rp = U.permute ? U.perm : nullptr;
     const int32_t* cp = V.permute ? V.perm : nullptr;
-    if (rp || cp) {
+    if (u_tc && !rp && !cp && w_dtype == QUIP_BF16 && (ldw % 8) == 0) {
+      // bf16 W is its own single piece: the m-side Kronecker factors first,
+      // straight from W (three products per term pair), then the n side in place
+      QCHECK(kron_cols_tc<__nv_bfloat16>(U, false, static_cast<const __nv_bfloat16*>(W), ldw, W_t, n, ws, st));
+      QCHECK(side_rows<float>(V, false, W_t, n, W_t, m, tmp, st, true));
+    } else if (rp || cp) {
       // W_t = P_m W P_n^T (W_t[r][c] = W[pi_m[r]][pi_n[c]]), then the structured factors in place
       if (w_dtype == QUIP_BF16)
         QCHECK(gather2d<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(W), ldw, W_t, n, m, n, rp, cp, st));
       else
         QCHECK(gather2d<float>(static_cast<const float*>(W), ldw, W_t, n, m, n, rp, cp, st));
-      QCHECK(side_rows<float>(V, false, W_t, n, W_t, m, tmp, st));
+      QCHECK(side_rows<float>(V, false, W_t, n, W_t, m, tmp, st, true));
     } else if (w_dtype == QUIP_BF16) {
-      QCHECK(side_rows<__nv_bfloat16>(V, false, static_cast<const __nv_bfloat16*>(W), ldw, W_t, m, tmp, st));
+      QCHECK(side_rows<__nv_bfloat16>(V, false, static_cast<const __nv_bfloat16*>(W), ldw, W_t, m, tmp, st, true));
     } else {
-      QCHECK(side_rows<float>(V, false, static_cast<const float*>(W), ldw, W_t, m, tmp, st));
+      QCHECK(side_rows<float>(V, false, static_cast<const float*>(W), ldw, W_t, m, tmp, st, true));
     }
-    QCHECK(side_cols(U, false, W_t, n, tmp, st));
+    if (!(u_tc && !rp && !cp && w_dtype == QUIP_BF16 && (ldw % 8) == 0)) {
+      if (u_tc) QCHECK(kron_cols_tc<float>(U, false, W_t, n, W_t, n, ws, st));
+      else QCHECK(side_cols(U, false, W_t, n, tmp, st));
+    }
   }
   if (H && V.permute) {
     // P_n H P_n^T, through the scratch
@@ -894,7 +1054,8 @@ quip_status quip_incoherence_inverse(const quip_transform* tf, const float* W_ha
   cudaStream_t st = S(stream);
   float* tmp = static_cast<float*>(ws);
   QCHECK(side_rows<float>(tf->side[1], true, W_hat_t, n, W_hat, m, tmp, st));
-  QCHECK(side_cols(tf->side[0], true, W_hat, n, tmp, st));
+  if (kron_cols_tc_ok(tf->side[0], n)) QCHECK(kron_cols_tc<float>(tf->side[0], true, W_hat, n, W_hat, n, ws, st));
+  else QCHECK(side_cols(tf->side[0], true, W_hat, n, tmp, st));
   const SideData &U = tf->side[0], &V = tf->side[1];
   if (U.permute || V.permute) {
     // W^ = P_m^T (T_m^T W~^ T_n) P_n: W^[r][c] = M[pi_m^-1[r]][pi_n^-1[c]], through the scratch
@@ -1269,15 +1430,24 @@ constexpr int kMaxDevices = 64;
 void* g_ldlq_scratch_ptr[kMaxDevices] = {};
 std::mutex g_ldlq_scratch_mu;
 
-// Device address of g_ldlq_scratch on the current device (looked up once).
-quip_status ldlq_static_scratch(void** out) {
+// Device address of g_ldlq_scratch on the current device.  Outside stream
+// capture it is looked up on every call (cheap once the module is loaded), so
+// a cudaDeviceReset, after which the module is loaded again and the array may
+// sit elsewhere, never leaves a stale address behind; while `stream` is
+// capturing, the address from the last call outside capture is used (and a
+// device never looked up outside capture is an error).
+quip_status ldlq_static_scratch(cudaStream_t stream, void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QUIP_ERR_CUDA;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return QUIP_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_ldlq_scratch_mu);
-  if (!g_ldlq_scratch_ptr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_ldlq_scratch) != cudaSuccess || !p) return QUIP_ERR_CUDA;
     g_ldlq_scratch_ptr[dev] = p;
+  } else if (!g_ldlq_scratch_ptr[dev]) {
+    return QUIP_ERR_CUDA;
   }
   *out = g_ldlq_scratch_ptr[dev];
   return QUIP_OK;
@@ -1296,7 +1466,7 @@ quip_status quip_ldlq_quantize_static(const float* W_t, const float* Uring, int6
     if (need > (size_t)QUIP_LDLQ_STATIC_SCRATCH_BYTES) return QUIP_ERR_WORKSPACE;
   }
   void* ws = nullptr;
-  quip_status s = ldlq_static_scratch(&ws);
+  quip_status s = ldlq_static_scratch(S(stream), &ws);
   if (s != QUIP_OK) return s;
   return quip_ldlq_quantize(W_t, Uring, ldu, m, n, bits, block, codes, lo, scale, ws,
                             (size_t)QUIP_LDLQ_STATIC_SCRATCH_BYTES, stream);

@@ -134,4 +134,151 @@ __global__ void __launch_bounds__(256) k_haar_cgs2(const double* __restrict__ G,
   }
 }
 
+// ---------------------------------------------------------------- Haar factor by Cholesky-QR2
+// Q of G = QR with diag(R) > 0 also equals Y R2^-1 with Y = G R1^-1, R1 the
+// upper Cholesky factor of G^T G and R2 that of Y^T Y (Cholesky-QR applied
+// twice): both factors have a positive diagonal, so R = R2 R1 does too and
+// Q is the same unique factor as any other QR with that sign convention,
+// up to rounding.  In fp64 one pass leaves Y orthogonal to about
+// cond(G)^2 u; the second pass brings it to u.  Square Gaussian factors up to
+// 224 x 224 (cond(G) of order p) are far inside that range.
+
+// Offset of (i, j), i <= j, in the column-major packed upper triangle
+// (column j holds rows 0 .. j).
+__host__ __device__ __forceinline__ int64_t packed_col(int64_t i, int64_t j) { return j * (j + 1) / 2 + i; }
+
+// Cp = Y^T Y (p x p, fp64), the upper triangle, packed by columns.  One
+// 32 x 32 output tile per CTA (tiles below the diagonal exit at once), 256
+// threads with four outputs each; 32-row slabs of both column blocks of Y
+// through shared memory; each sum runs over the rows in order.
+__global__ void __launch_bounds__(256) k_gram64(const double* __restrict__ Y,
+                                                double* __restrict__ Cp, int p) {
+  const int bi = blockIdx.y, bj = blockIdx.x;
+  if (bi > bj) return;
+  __shared__ double a[32][33], b[32][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int i0 = 32 * bi, j0 = 32 * bj;
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int r0 = 0; r0 < p; r0 += 32) {
+    for (int rr = ty; rr < 32; rr += 8) {
+      const int r = r0 + rr;
+      a[rr][tx] = (r < p && i0 + tx < p) ? Y[(int64_t)r * p + i0 + tx] : 0.0;
+      b[rr][tx] = (r < p && j0 + tx < p) ? Y[(int64_t)r * p + j0 + tx] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int rr = 0; rr < 32; ++rr) {
+      const double bv = b[rr][tx];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[u] = fma(a[rr][ty + 8 * u], bv, acc[u]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int i = i0 + ty + 8 * u, j = j0 + tx;
+    if (i < p && j < p && j >= i) Cp[packed_col(i, j)] = acc[u];
+  }
+}
+
+constexpr int HAAR_CHOL_MAX = 224;          // packed factor + two rows fit in shared memory
+constexpr int HAAR_CHOL_T = HAAR_CHOL_MAX / 32;
+__host__ __device__ constexpr size_t chol_solve_smem(int p) {
+  return ((size_t)p * (p + 1) / 2 + 2 * (size_t)p) * sizeof(double);
+}
+
+__device__ __forceinline__ double warp_allsum64(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// X = Y R^-1 with R the upper Cholesky factor of C (C = R^T R; Cp packed by
+// columns, fp64).  One CTA of 1024 threads (32 warps), p <= HAAR_CHOL_MAX.
+// Cp is copied to shared memory and factored in place, left-looking, one row
+// of R per step: R[k, j] = (C[k, j] - sum_{i<k} R[i, k] R[i, j]) / R[k, k],
+// R[k, k] = sqrt(C[k, k] - sum_{i<k} R[i, k]^2); warp w takes the columns
+// j = k + w, k + w + 32, ..., its lanes the terms i = lane, lane + 32, ...
+// (consecutive rows of a column are consecutive in shared memory), summed
+// by a butterfly.  Then the rows of X, one warp per row: for k = 0 .. p - 1,
+// X[r, k] = (Y[r, k] - sum_{i<k} X[r, i] R[i, k]) / R[k, k], lane l keeping
+// X[r, i] and Y[r, i] for i = l, l + 32, ... in registers.  X may alias Cp
+// (Cp is read in full before X is written); X must not alias Y.  out32, when
+// not NULL, gets X rounded to fp32 (row-major).  A pivot that is not
+// positive and finite is recorded as QUIP_ERR_NONFINITE.
+// Dynamic smem: chol_solve_smem(p).
+__global__ void __launch_bounds__(1024, 1) k_chol_solve64(const double* Cp, const double* __restrict__ Y,
+                                                          double* X, float* __restrict__ out32, int p) {
+  extern __shared__ double chs[];
+  double* R = chs;                                   // packed by columns, p (p + 1) / 2
+  double* row = R + (int64_t)p * (p + 1) / 2;        // p: row k before the scaling
+  double* rinv = row + p;                            // p: 1 / R[k][k]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t np = (int64_t)p * (p + 1) / 2;
+  for (int64_t e = tid; e < np; e += blockDim.x) R[e] = Cp[e];
+  __syncthreads();
+  bool ok = true;
+  for (int k = 0; k < p; ++k) {
+    double rk[HAAR_CHOL_T];
+#pragma unroll
+    for (int t = 0; t < HAAR_CHOL_T; ++t) {
+      const int i = lane + 32 * t;
+      rk[t] = i < k ? R[packed_col(i, k)] : 0.0;
+    }
+    for (int j = k + warp; j < p; j += 32) {
+      double s = 0.0;
+#pragma unroll
+      for (int t = 0; t < HAAR_CHOL_T; ++t) {
+        const int i = lane + 32 * t;
+        if (i < k) s = fma(rk[t], R[packed_col(i, j)], s);
+      }
+      s = warp_allsum64(s);
+      if (lane == 0) row[j] = R[packed_col(k, j)] - s;
+    }
+    __syncthreads();
+    const double d = row[k];
+    ok = ok && d > 0.0 && d < INFINITY;
+    const double rkk = sqrt(d);
+    for (int j = k + tid; j < p; j += blockDim.x) R[packed_col(k, j)] = (j == k) ? rkk : row[j] / rkk;
+    if (tid == 0) rinv[k] = 1.0 / rkk;
+    __syncthreads();
+  }
+  if (!ok) {
+    if (tid == 0) record_status(QUIP_ERR_NONFINITE);
+    return;
+  }
+  for (int r = warp; r < p; r += 32) {
+    double yv[HAAR_CHOL_T], xv[HAAR_CHOL_T];
+#pragma unroll
+    for (int t = 0; t < HAAR_CHOL_T; ++t) {
+      const int i = lane + 32 * t;
+      yv[t] = i < p ? Y[(int64_t)r * p + i] : 0.0;
+      xv[t] = 0.0;
+    }
+#pragma unroll
+    for (int kq = 0; kq < HAAR_CHOL_T; ++kq) {
+      for (int kl = 0; kl < 32; ++kl) {
+        const int k = 32 * kq + kl;
+        if (k >= p) break;
+        double s = 0.0;
+#pragma unroll
+        for (int t = 0; t <= kq; ++t) {
+          const int i = lane + 32 * t;
+          if (i < k) s = fma(xv[t], R[packed_col(i, k)], s);
+        }
+        s = warp_allsum64(s);
+        if (lane == kl) xv[kq] = (yv[kq] - s) * rinv[k];
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < HAAR_CHOL_T; ++t) {
+      const int i = lane + 32 * t;
+      if (i < p) {
+        X[(int64_t)r * p + i] = xv[t];
+        if (out32) out32[(int64_t)r * p + i] = (float)xv[t];
+      }
+    }
+  }
+}
+
 }  // namespace quip

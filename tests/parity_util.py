@@ -71,3 +71,13 @@ def greedy_trajectory_check(C0, C1, Wt, H, lo, s, bits, tau):
     frac = np.abs(z - np.floor(z) - 0.5)
     near = frac < tau
     return float(bad.mean()), float((bad & ~near).mean())
+
+
+def row_scaled_err(A, B, s, same):
+    """max |A - B| / s_i over the entries where the codes agree (mask
+    ``same``), each entry measured against its own row's grid step s_i: the
+    dequantised-weight tolerance is stated per row, so a row with a small
+    step is not judged against a larger row's step."""
+    s = np.asarray(s, dtype=np.float64)[:, None]
+    e = np.abs(np.asarray(A, dtype=np.float64) - np.asarray(B, dtype=np.float64)) / s
+    return float(e[np.asarray(same, dtype=bool)].max()) if np.any(same) else 0.0

@@ -156,6 +156,21 @@ def test_incoherence_rows_and_hessian_match_full_forward():
     rows = [0, 7, 23]
     np.testing.assert_allclose(O.incoherence_rows(W, U, V, rows), Wt[rows], atol=1e-14)
     np.testing.assert_allclose(O.incoherence_hessian(H, V), Ht, atol=1e-13)
+    np.testing.assert_allclose(O.incoherence_hessian_rows(H, V, [0, 9, 15]), Ht[[0, 9, 15]], atol=1e-13)
+    # the inverse restricted to rows: rows of U^T W~ V, and the round trip
+    Wi = O.incoherence_inverse(Wt, U, V)
+    np.testing.assert_allclose(O.incoherence_inverse_rows(Wt, U, V, rows), Wi[rows], atol=1e-14)
+    np.testing.assert_allclose(O.incoherence_inverse_rows(Wt, U, V, rows), W[rows], atol=1e-13)
+
+
+@pytest.mark.parametrize("kind,dim,p,q,perm", [("hadamard", 32, 0, 0, False), ("kronecker", 12, 3, 4, False),
+                                               ("hadamard", 16, 0, 0, True), ("kronecker", 12, 4, 3, True),
+                                               ("identity", 8, 0, 0, True)])
+def test_side_columns_are_the_matrix_columns(kind, dim, p, q, perm):
+    S = O.make_side(5, "n", kind, dim, p, q, permute=perm)
+    M = S.matrix()
+    for i in range(dim):
+        np.testing.assert_allclose(S.col(i), M[:, i], atol=1e-15)
 
 
 def test_hadamard_sign_placement_hand_example():

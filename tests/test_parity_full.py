@@ -14,7 +14,7 @@ import oracle as O
 import post_weight_quantization_09_b200 as Q
 from post_weight_quantization_09_b200 import _lib as L
 from quip_synth import CONFIGS, make_layer
-from parity_util import dev, host, ldlq_trajectory_check, rel_fro
+from parity_util import dev, host, ldlq_trajectory_check, rel_fro, row_scaled_err
 
 pytestmark = pytest.mark.gpu
 
@@ -53,14 +53,14 @@ def test_attn7b_full_layer():
     agree = float((C == codes).mean())
     Wt_hat_d = O.dequantize(C, lo_d, s_d)
     loss_d = O.proxy_loss(Wt_hat_d, Wt, Ht)
-    same = C == codes
-    w_err = float(np.abs(Wt_hat_d - Wt_hat)[same].max() / s.max())
+    w_err = row_scaled_err(Wt_hat_d, Wt_hat, s, C == codes)
     bad, not_near = ldlq_trajectory_check(C, Wt, Uf, lo_d, s_d, cfg.bits, tau=1e-3)
     print(f"\nattn7b: H rel-Fro {h_err:.3e}  codes agree {agree:.6f}  loss {loss:.6g} vs {loss_d:.6g} "
           f"(rel {abs(loss_d - loss) / loss:.2e})  W^ err/s {w_err:.2e}  trajectory mismatch {bad:.2e} "
           f"(not near-tie {not_near:.2e})  oracle {time.time() - t0:.0f}s")
     assert abs(loss_d - loss) / loss <= 1e-3
     assert w_err <= 1e-4
+    assert not_near == 0.0
     assert agree >= 0.999
     # sampled rows of the inverse transform: W^ = U^T W~^ V
     rows = np.random.default_rng(0).choice(cfg.m, 16, replace=False)
@@ -99,8 +99,7 @@ def _sampled_layer_check(name, nrows=256):
     Wt_hat_d = O.dequantize(C, lo_d, s_d)
     loss = O.proxy_loss(Wt_hat, Wt, Ht)
     loss_d = O.proxy_loss(Wt_hat_d, Wt, Ht)
-    same = C == codes
-    w_err = float(np.abs(Wt_hat_d - Wt_hat)[same].max() / s.max())
+    w_err = row_scaled_err(Wt_hat_d, Wt_hat, s, C == codes)
     bad, not_near = ldlq_trajectory_check(C, Wt, Uf, lo_d, s_d, cfg.bits, tau=1e-3)
     print(f"\n{name}: H rel-Fro {h_err:.3e}  W~ err {wt_err:.2e}  codes agree {agree:.6f} on {nrows} rows  "
           f"loss {loss:.6g} vs {loss_d:.6g} (rel {abs(loss_d - loss) / loss:.2e})  W^ err/s {w_err:.2e}  "

@@ -58,9 +58,12 @@ def test_static_workspace_matches_allocating_entry_point():
 
 def test_static_workspace_rejects_layers_that_do_not_fit():
     lib = Q.load()
-    fake = ctypes.c_void_p(0x1000)
-    # (m*n + m*block) * 4 bytes > 16 MiB: rejected before any launch
-    st = lib.quip_ldlq_quantize_static(fake, fake, 4096, 4096, 4096, 2, 128, fake, fake, fake, None)
+    # A 4096 x 4096 layer needs m*n*4 (accumulator) + 3*m*n*2 (error pieces)
+    # + 3*n*n*2 (factor pieces) + n*n*4 (fp32 factor) bytes, each rounded up
+    # to 256, far more than the 16 MiB array: rejected before any launch.
+    # The pointers are NULL, so should the size check ever regress, the call
+    # stops at the argument check (QUIP_ERR_ARG) instead of launching.
+    st = lib.quip_ldlq_quantize_static(None, None, 4096, 4096, 4096, 2, 128, None, None, None, None)
     assert st == L.QUIP_ERR_WORKSPACE
     need = Q.quip_workspace_size(L.QUIP_OP_LDLQ, None, 1024, 4096, 128)
     assert need > STATIC_BYTES
