@@ -6,7 +6,7 @@ draw (U, V) -> H = X^T X (tensor cores) -> finalise + damp -> W~ = U W V^T,
 H~ = V H V^T -> LDL of H~ -> LDLQ rounding -> dequantise -> inverse transform.
 Metric: quantized weights per second (m * n / step time), whole job.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config attn7b]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config gate70b] [--all-configs]
   python bench.py --impl reference ...    # the FP64 CPU oracle, bounded sample
 
 Multi-GPU (torchrun): each rank quantises its own layer of the same shape
@@ -136,6 +136,12 @@ def kernel_work(cfg: LayerConfig, method: str = "ldlq", passes: int = 1):
         kw["k_greedy_start"] = ("bytes", greedy * 19.0 * m * n, "hbm")
         # H's upper triangle in; U'^T (fp32 and three pieces) and U' out
         kw["k_greedy_factors"] = ("bytes", 16.0 * n * n, "hbm")
+    if cfg.m_side.kind == "kronecker":
+        # the m-side Kronecker factors on the tensor cores, forward and inverse:
+        # 2 (p + q) m n fp32-algorithmic flops each way (issued as 3 or 6
+        # bf16 piece products)
+        p_, q_ = cfg.m_side.p, cfg.m_side.q
+        kw["k_kron_tc"] = ("flops", 2 * 2.0 * (p_ + q_) * m * n, "tensor")
     if method == "ldlq_rg":
         # H~ gathered twice (8 n^2 each), W~ once (8 m n), the codes back (2 m n)
         kw["k_permute"] = ("bytes", 16.0 * n * n + 10.0 * m * n, "hbm")
@@ -547,6 +553,17 @@ def run_ours(args, cfg: LayerConfig):
     if st != L.QUIP_OK:
         raise RuntimeError(f"device status after warm-up: {L.status_string(st)}")
 
+    # the timed step: for LDLQ the library's whole-layer call on the
+    # device-resident W and X (quip_quantize_layer), else the method's calls
+    def whole_step():
+        if args.method == "ldlq":
+            q.run(W, X)
+        else:
+            step()
+
+    for _ in range(max(3, args.warmup)):
+        whole_step()
+    torch.cuda.synchronize()
     nev = len(STAGES) + 1
     step_ms, stage_ms = [], [[] for _ in STAGES]
     launches0 = lib.quip_kernel_launches()
@@ -556,18 +573,28 @@ def run_ours(args, cfg: LayerConfig):
             if world > 1:
                 dist.barrier()
             torch.cuda.synchronize()
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(nev)]
-            step(ev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            whole_step()
+            e1.record(stream)
             torch.cuda.synchronize()
-            step_ms.append(ev[0].elapsed_time(ev[-1]))
-            for i in range(len(STAGES)):
-                stage_ms[i].append(ev[i].elapsed_time(ev[i + 1]))
+            step_ms.append(e0.elapsed_time(e1))
             if world > 1:
                 dist.barrier()
     launches = lib.quip_kernel_launches() - launches0
     st = Q.quip_sync_status()
     if st != L.QUIP_OK:
         raise RuntimeError(f"device status after timing: {L.status_string(st)}")
+
+    # stage breakdown: the same path as one call per stage, events in between
+    for _ in range(args.steps):
+        flush.zero_()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(nev)]
+        step(ev)
+        torch.cuda.synchronize()
+        for i in range(len(STAGES)):
+            stage_ms[i].append(ev[i].elapsed_time(ev[i + 1]))
 
     # ---- per-kernel device time: the same steps again, each launch bracketed
     # by CUDA events on its own stream (kept out of the timed region above)
@@ -583,7 +610,8 @@ def run_ours(args, cfg: LayerConfig):
     ms_per_step = total_ms / args.steps
     value = job_throughput(cfg, world, ms_per_step)
 
-    # ---- end to end through the public API: pinned host inputs in, codes + grid out
+    # ---- end to end through the public API: pinned host inputs in, codes + grid
+    # out (LDLQ: one library call, quip_quantize_layer_host, copies included)
     codes_h = torch.empty(cfg.m, cfg.n, dtype=torch.uint8).pin_memory()
     lo_h = torch.empty(cfg.m, dtype=torch.float32).pin_memory()
     sc_h = torch.empty(cfg.m, dtype=torch.float32).pin_memory()
@@ -867,7 +895,10 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="attn7b", choices=sorted(CONFIGS))
+    ap.add_argument("--config", default="gate70b", choices=sorted(CONFIGS),
+                    help="workload (default: the largest single-GPU layer, the 70B-shaped MLP gate)")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="one JSON line per workload (tiny, attn7b, up7b, down7b, gate70b)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--group", type=int, default=1,
@@ -890,6 +921,14 @@ def main():
                       n_side=replace(cfg.n_side, permute=True))
     if args.decode:
         run_decode(args)
+        return
+    if args.all_configs:
+        from dataclasses import replace as _rep
+        for name in ("tiny", "attn7b", "up7b", "down7b", "gate70b"):
+            c = CONFIGS[name]
+            if args.permute:
+                c = _rep(c, m_side=_rep(c.m_side, permute=True), n_side=_rep(c.n_side, permute=True))
+            (run_reference if args.impl == "reference" else run_ours)(args, c)
         return
     if args.impl == "reference":
         run_reference(args, cfg)

@@ -394,6 +394,69 @@ quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int
                                  int64_t block, size_t* bytes);
 
 /*
+ * The whole path for one layer, from the problem statement of the QuIP page
+ * (W, calibration inputs X, bit width, damping, LDLQ block size, seed):
+ * draw (U, V) from `seed` into tf (quip_transform_draw), H = X^T X / N
+ * (quip_hessian_accumulate), damping (quip_hessian_finalize, alpha = damp),
+ * H~ = V H V^T and the LDL of H~ (quip_incoherence_forward, quip_ldl),
+ * W~ = U W V^T and LDLQ (quip_ldlq_quantize), then, when W_hat is not NULL,
+ * W^ = U^T (lo + s codes) V (quip_dequantize, quip_incoherence_inverse), in
+ * that order on `stream`; each step has the arguments, layout and errors of
+ * its own entry point.  The codes and grid are those of LDLQ in the
+ * incoherent basis (quip_ldlq_quantize); W^ is the dequantised layer in the
+ * original basis.
+ *   tf       : a transform made for this layer's m x n (quip_transform_create);
+ *              it is redrawn from `seed`.
+ *   W        : device, m x n, w_dtype QUIP_F32 or QUIP_BF16, row stride ldw.
+ *   X        : device, N x n (N >= 1 tokens), x_dtype QUIP_F32 or QUIP_BF16,
+ *              row stride ldx.
+ *   bits     : 1 .. 8.  block: 32, 64 or 128 with n % block == 0 and n % 64 == 0.
+ *   damp     : alpha >= 0.
+ *   codes    : device m x n uint8.  lo, scale: device m fp32.
+ *   W_hat    : device m x n fp32, or NULL to stop after the codes.
+ * ws: quip_layer_workspace_size(tf, N, w_dtype, x_dtype, block, 0, ...).
+ * On return ws holds, at offset 0, the n x n fp32 matrix whose strict upper
+ * triangle is Ů (as quip_ldl leaves it); at a = round256(4 n^2) the n pivots
+ * D (fp32); at a + round256(4 n) W~ (m x n fp32); round256(x) rounds x up to
+ * a multiple of 256.
+ * Device-side errors (non-PD H~, non-finite values) go to the status word.
+ */
+quip_status quip_quantize_layer(quip_transform* tf, uint64_t seed, const void* W, int w_dtype,
+                                int64_t ldw, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                                int bits, int64_t block, float damp, uint8_t* codes, float* lo,
+                                float* scale, float* W_hat, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * quip_quantize_layer from host memory to host memory.  W_host, X_host
+ * (same shapes, types and strides as above) are copied to the device on a
+ * library-owned copy stream, X in token chunks of at least 2048 so that the
+ * Hessian accumulates each chunk as it lands, W while the Hessian, H~ and the
+ * LDL run (they do not read W); codes_host (m x n uint8), lo_host and
+ * scale_host (m fp32) are copied back on that stream while W^ is formed on
+ * the device, and W^ (m x n fp32) into W_hat_host when it is not NULL (W^ is
+ * computed either way: it is the last step of the path).  One
+ * cudaMemcpy2DAsync / cudaMemcpyAsync per piece.  `stream` waits for every
+ * copy, so synchronising it makes all host outputs valid; host buffers
+ * should be page-locked for the copies to overlap the kernels.  All device
+ * buffers live in ws: quip_layer_workspace_size(tf, N, w_dtype, x_dtype,
+ * block, 1, ...).
+ */
+quip_status quip_quantize_layer_host(quip_transform* tf, uint64_t seed, const void* W_host,
+                                     int w_dtype, int64_t ldw, const void* X_host, int x_dtype,
+                                     int64_t N, int64_t ldx, int bits, int64_t block, float damp,
+                                     uint8_t* codes_host, float* lo_host, float* scale_host,
+                                     float* W_hat_host, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Device workspace of quip_quantize_layer (host = 0) or
+ * quip_quantize_layer_host (host = 1) for N tokens and the given types:
+ * H~ (n x n fp32), D, W~ (m x n fp32) and the largest stage workspace; the
+ * host variant adds device copies of W and X, the codes, the grid and W^.
+ */
+quip_status quip_layer_workspace_size(const quip_transform* tf, int64_t N, int w_dtype, int x_dtype,
+                                      int64_t block, int host, size_t* bytes);
+
+/*
  * Per-kernel device timing, for measurement (the QuIP papers have no
  * counterpart).  quip_timing_begin() discards earlier records and turns
  * timing on: from then on every kernel the library launches, on any stream,

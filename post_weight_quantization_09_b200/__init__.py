@@ -23,7 +23,8 @@ __all__ = [
     "quip_incoherence_inverse", "quip_ldl", "quip_ldlq_quantize", "quip_dequantize",
     "quip_nearest_quantize", "quip_diag_order", "quip_permute", "quip_greedy_refine", "METHODS",
     "quip_packed_words", "quip_pack_codes", "quip_qmatvec", "QuantizedLinear",
-    "quip_workspace_size", "quip_sync_status", "quip_timing_begin", "quip_timing_end", "LayerQuantizer",
+    "quip_workspace_size", "quip_layer_workspace_size", "quip_quantize_layer", "quip_quantize_layer_host",
+    "layer_views", "quip_sync_status", "quip_timing_begin", "quip_timing_end", "LayerQuantizer",
     "LayerGroupQuantizer", "quantize_layer", "QuipError",
     "KIND",
 ]
@@ -311,6 +312,54 @@ def quip_dequantize(codes: torch.Tensor, lo: torch.Tensor, scale: torch.Tensor, 
             "quip_dequantize")
 
 
+def quip_layer_workspace_size(tf: Transform, N: int, w_dtype: int, x_dtype: int, block: int,
+                              host: bool) -> int:
+    nb = ctypes.c_size_t()
+    L.check(load().quip_layer_workspace_size(tf.handle, N, w_dtype, x_dtype, block, int(host), ctypes.byref(nb)),
+            "quip_layer_workspace_size")
+    return nb.value
+
+
+def quip_quantize_layer(tf: Transform, seed: int, W: torch.Tensor, X: torch.Tensor, bits: int, block: int,
+                        damp: float, codes: torch.Tensor, lo: torch.Tensor, scale: torch.Tensor,
+                        W_hat: Optional[torch.Tensor], ws: torch.Tensor, stream=None) -> None:
+    """The whole layer on device tensors (include/quip.h)."""
+    _cuda(W, "W"), _cuda(X, "X")
+    L.check(load().quip_quantize_layer(
+        tf.handle, ctypes.c_uint64(seed & 0xFFFFFFFFFFFFFFFF), _p(W), _dtype(W), W.stride(0), _p(X), _dtype(X),
+        X.shape[0], X.stride(0), bits, block, damp, _p(codes), _p(lo), _p(scale), _p(W_hat), _p(ws), ws.numel(),
+        _s(stream)), "quip_quantize_layer")
+
+
+def quip_quantize_layer_host(tf: Transform, seed: int, W_host: torch.Tensor, X_host: torch.Tensor, bits: int,
+                             block: int, damp: float, codes_host: torch.Tensor, lo_host: torch.Tensor,
+                             scale_host: torch.Tensor, W_hat_host: Optional[torch.Tensor], ws: torch.Tensor,
+                             stream=None) -> None:
+    """The whole layer from host tensors to host tensors (include/quip.h);
+    synchronise `stream` before reading the outputs."""
+    for t, nm in ((W_host, "W_host"), (X_host, "X_host"), (codes_host, "codes_host")):
+        if t.is_cuda:
+            raise ValueError(f"{nm} must be a host tensor")
+    L.check(load().quip_quantize_layer_host(
+        tf.handle, ctypes.c_uint64(seed & 0xFFFFFFFFFFFFFFFF), _p(W_host), _dtype(W_host), W_host.stride(0),
+        _p(X_host), _dtype(X_host), X_host.shape[0], X_host.stride(0), bits, block, damp, _p(codes_host),
+        _p(lo_host), _p(scale_host), _p(W_hat_host), _p(ws), ws.numel(), _s(stream)), "quip_quantize_layer_host")
+
+
+def _round256(b: int) -> int:
+    return (b + 255) // 256 * 256
+
+
+def layer_views(ws: torch.Tensor, m: int, n: int):
+    """(H, D, W_t) inside a whole-layer workspace after the call: the n x n
+    matrix holding U in its strict upper triangle, D and W~ (the offsets
+    include/quip.h gives)."""
+    d0 = _round256(4 * n * n)
+    w0 = d0 + _round256(4 * n)
+    f32 = lambda a, cnt: ws[a:a + 4 * cnt].view(torch.float32)
+    return f32(0, n * n).view(n, n), f32(d0, n), f32(w0, m * n).view(m, n)
+
+
 def quip_sync_status(stream=None) -> int:
     return load().quip_sync_status(_s(stream))
 
@@ -387,6 +436,15 @@ class LayerQuantizer:
         """Draw (U, V) again from the seed on the device (part of a full pass)."""
         self.tf.draw(self.seed, self.stream)
 
+    def _layer_ws(self, N: int, w_dtype: int, x_dtype: int, host: bool) -> torch.Tensor:
+        """Workspace of the whole-layer calls for N tokens (kept per shape)."""
+        cache = self.__dict__.setdefault("_lws", {})
+        key = (N, w_dtype, x_dtype, host)
+        if key not in cache:
+            nb = quip_layer_workspace_size(self.tf, N, w_dtype, x_dtype, self.block, host)
+            cache[key] = torch.empty(max(nb, 256), dtype=torch.uint8, device=self.H.device)
+        return cache[key]
+
     def run(self, W: torch.Tensor, X: torch.Tensor, redraw_transform: bool = True,
             w_ready: Optional[torch.cuda.Event] = None, after_ldlq=None,
             x_ready=None) -> LayerResult:
@@ -398,6 +456,14 @@ class LayerQuantizer:
         ``after_ldlq`` (a callable) is invoked once codes and grid are final."""
         st = self.stream
         stream = st if st is not None else torch.cuda.current_stream()
+        if self.method == "ldlq" and redraw_transform and not x_ready and w_ready is None \
+                and after_ldlq is None:
+            # the whole layer in one library call
+            ws = self._layer_ws(X.shape[0], _dtype(W), _dtype(X), False)
+            quip_quantize_layer(self.tf, self.seed, W, X, self.bits, self.block, self.damp, self.codes, self.lo,
+                                self.scale, self.W_hat, ws, st)
+            self.H, self.D, self.W_t = layer_views(ws, self.m, self.n)
+            return LayerResult(self.codes, self.lo, self.scale, self.W_hat)
         if redraw_transform:
             self.new_transform()
         if x_ready:
@@ -461,7 +527,14 @@ class LayerQuantizer:
         accumulated into the Hessian as soon as it lands, then W, overlapping
         the Hessian, its transform and the LDL; the results go back on that
         stream while the dequantisation and inverse transform run.
-        Everything is joined into the layer's stream; synchronise it to read."""
+        Everything is joined into the layer's stream; synchronise it to read.
+        LDLQ runs as one library call (quip_quantize_layer_host), which does
+        these copies and their overlap itself."""
+        if self.method == "ldlq":
+            ws = self._layer_ws(X_host.shape[0], _dtype(W_host), _dtype(X_host), True)
+            quip_quantize_layer_host(self.tf, self.seed, W_host, X_host, self.bits, self.block, self.damp,
+                                     codes_out, lo_out, scale_out, None, ws, self.stream)
+            return
         if getattr(self, "_W_dev", None) is None or self._W_dev.shape != W_host.shape \
                 or self._W_dev.dtype != W_host.dtype:
             self._W_dev = torch.empty_like(W_host, device="cuda")

@@ -54,6 +54,13 @@ SIGNATURES = {
                              c_int64, c_int64, c_void_p, c_int64, c_void_p, c_size_t, c_void_p]),
     "quip_dequantize": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
     "quip_workspace_size": (c_int, [c_int, c_void_p, c_int64, c_int64, c_int64, POINTER(c_size_t)]),
+    "quip_quantize_layer": (c_int, [c_void_p, c_uint64, c_void_p, c_int, c_int64, c_void_p, c_int, c_int64,
+                                    c_int64, c_int, c_int64, c_float, c_void_p, c_void_p, c_void_p, c_void_p,
+                                    c_void_p, c_size_t, c_void_p]),
+    "quip_quantize_layer_host": (c_int, [c_void_p, c_uint64, c_void_p, c_int, c_int64, c_void_p, c_int,
+                                         c_int64, c_int64, c_int, c_int64, c_float, c_void_p, c_void_p,
+                                         c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "quip_layer_workspace_size": (c_int, [c_void_p, c_int64, c_int, c_int, c_int64, c_int, POINTER(c_size_t)]),
     "quip_sync_status": (c_int, [c_void_p]),
     "quip_timing_begin": (c_int, []),
     "quip_timing_end": (c_int, [POINTER(c_char_p), POINTER(c_uint64), POINTER(ctypes.c_double), c_int,

@@ -9,6 +9,7 @@
 #include <algorithm>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "fwht.cuh"
@@ -1723,6 +1724,214 @@ quip_status quip_dequantize(const uint8_t* codes, const float* lo, const float* 
   QCHECK(cudaGetLastError());
   return QUIP_OK;
 }
+
+// ---------------------------------------------------------------- whole layer
+
+namespace {
+// A per-device stream for host <-> device copies of quip_quantize_layer_host,
+// created on first use and kept for the process.
+cudaError_t copy_stream(cudaStream_t* out) {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev]) {
+    e = cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking);
+    if (e != cudaSuccess) return e;
+  }
+  *out = streams[dev];
+  return cudaSuccess;
+}
+
+// Device workspace of the whole-layer call: H (n x n), D (n), W~ (m x n),
+// then one region shared by the stages (the largest stage workspace); the
+// host variant adds device copies of W and X, and the device results: codes
+// (m x n), lo and scale (m each) and W^ (m x n fp32).
+struct LayerWs {
+  size_t H, D, Wt, stage, Wd, Xd, codes, lo, sc, What, total;
+};
+
+quip_status layer_ws(const quip_transform* tf, int64_t N, int w_dtype, int x_dtype, int64_t block, bool host,
+                     LayerWs* o) {
+  const int64_t m = tf->m, n = tf->n;
+  size_t st = 0, b = 0;
+  quip_status s;
+  const int ops[4] = {QUIP_OP_INCOHERENCE_FORWARD, QUIP_OP_INCOHERENCE_INVERSE, QUIP_OP_LDL, QUIP_OP_LDLQ};
+  for (int op : ops) {
+    if ((s = quip_workspace_size(op, tf, m, n, block, &b)) != QUIP_OK) return s;
+    st = std::max(st, b);
+  }
+  const size_t wes = w_dtype == QUIP_BF16 ? 2 : 4, xes = x_dtype == QUIP_BF16 ? 2 : 4;
+  *o = LayerWs{};
+  o->H = round256((size_t)n * n * 4);
+  o->D = round256((size_t)n * 4);
+  o->Wt = round256((size_t)m * n * 4);
+  o->stage = round256(std::max<size_t>(st, 256));
+  if (host) {
+    o->Wd = round256((size_t)m * n * wes);
+    o->Xd = round256((size_t)std::max<int64_t>(N, 1) * n * xes);
+    o->codes = round256((size_t)m * n);
+    o->lo = o->sc = round256((size_t)m * 4);
+    o->What = round256((size_t)m * n * 4);
+  }
+  o->total = o->H + o->D + o->Wt + o->stage + o->Wd + o->Xd + o->codes + o->lo + o->sc + o->What;
+  return QUIP_OK;
+}
+
+quip_status layer_args(const quip_transform* tf, int w_dtype, int64_t ldw, int x_dtype, int64_t N, int64_t ldx,
+                       int bits, int64_t block, float damp) {
+  if (!tf) return QUIP_ERR_ARG;
+  if ((w_dtype != QUIP_F32 && w_dtype != QUIP_BF16) || (x_dtype != QUIP_F32 && x_dtype != QUIP_BF16))
+    return QUIP_ERR_ARG;
+  if (bits < 1 || bits > 8 || !(damp >= 0.f) || !std::isfinite(damp)) return QUIP_ERR_ARG;
+  if (N < 1 || ldw < tf->n || ldx < tf->n) return QUIP_ERR_SHAPE;
+  if (!(block == 32 || block == 64 || block == 128) || tf->n % block || tf->n % 64) return QUIP_ERR_SHAPE;
+  return QUIP_OK;
+}
+
+// Token chunks of X in the host variant: X's copy lands in up to four
+// pieces, each accumulated into H as soon as it is on the device.
+int64_t layer_x_chunk(int64_t N) {
+  const int64_t c = (N + 3) / 4;
+  return std::max<int64_t>(2048, (c + 2047) / 2048 * 2048);
+}
+
+// The device part of the layer from W, X on the device: draw (U, V), H,
+// damping, H~, LDL, W~, LDLQ, and (W_hat non-NULL) W^.  x_ready, when given,
+// is one event per token chunk of layer_x_chunk(N), waited for before that
+// chunk is accumulated; w_ready is waited for before W is read; q_done is
+// recorded once codes and grid are final.
+quip_status layer_device(quip_transform* tf, uint64_t seed, const void* W, int w_dtype, int64_t ldw,
+                         const void* X, int x_dtype, int64_t N, int64_t ldx, int bits, int64_t block,
+                         float damp, uint8_t* codes, float* lo, float* scale, float* W_hat,
+                         const LayerWs& L, char* ws, cudaStream_t st, const cudaEvent_t* x_ready,
+                         cudaEvent_t w_ready, cudaEvent_t q_done) {
+  const int64_t m = tf->m, n = tf->n;
+  float* H = reinterpret_cast<float*>(ws);
+  float* D = reinterpret_cast<float*>(ws + L.H);
+  float* Wt = reinterpret_cast<float*>(ws + L.H + L.D);
+  void* sw = ws + L.H + L.D + L.Wt;
+  quip_status s;
+  if ((s = quip_transform_draw(tf, seed, st)) != QUIP_OK) return s;
+  const size_t xes = x_dtype == QUIP_BF16 ? 2 : 4;
+  if (x_ready) {
+    const int64_t step = layer_x_chunk(N);
+    int c = 0;
+    for (int64_t a = 0; a < N; a += step, ++c) {
+      QCHECK(cudaStreamWaitEvent(st, x_ready[c], 0));
+      const int64_t b = std::min(N, a + step);
+      if ((s = quip_hessian_accumulate(static_cast<const char*>(X) + (size_t)a * ldx * xes, x_dtype, b - a, n,
+                                       ldx, H, a > 0 ? 1 : 0, st)) != QUIP_OK)
+        return s;
+    }
+  } else if ((s = quip_hessian_accumulate(X, x_dtype, N, n, ldx, H, 0, st)) != QUIP_OK) {
+    return s;
+  }
+  if ((s = quip_hessian_finalize(H, n, N, damp, st)) != QUIP_OK) return s;
+  if ((s = quip_incoherence_forward(tf, nullptr, QUIP_F32, n, nullptr, H, sw, L.stage, st)) != QUIP_OK) return s;
+  if ((s = quip_ldl(H, D, n, sw, L.stage, st)) != QUIP_OK) return s;
+  if (w_ready) QCHECK(cudaStreamWaitEvent(st, w_ready, 0));
+  if ((s = quip_incoherence_forward(tf, W, w_dtype, ldw, Wt, nullptr, sw, L.stage, st)) != QUIP_OK) return s;
+  if ((s = quip_ldlq_quantize(Wt, H, n, m, n, bits, block, codes, lo, scale, sw, L.stage, st)) != QUIP_OK)
+    return s;
+  if (q_done) QCHECK(cudaEventRecord(q_done, st));
+  if (W_hat) {
+    if ((s = quip_dequantize(codes, lo, scale, m, n, W_hat, st)) != QUIP_OK) return s;
+    if ((s = quip_incoherence_inverse(tf, W_hat, W_hat, sw, L.stage, st)) != QUIP_OK) return s;
+  }
+  return QUIP_OK;
+}
+}  // namespace
+
+extern "C" {
+
+quip_status quip_layer_workspace_size(const quip_transform* tf, int64_t N, int w_dtype, int x_dtype,
+                                      int64_t block, int host, size_t* bytes) {
+  if (!tf || !bytes) return QUIP_ERR_ARG;
+  *bytes = 0;
+  LayerWs L;
+  quip_status s = layer_ws(tf, N, w_dtype, x_dtype, block, host != 0, &L);
+  if (s != QUIP_OK) return s;
+  *bytes = L.total;
+  return QUIP_OK;
+}
+
+quip_status quip_quantize_layer(quip_transform* tf, uint64_t seed, const void* W, int w_dtype, int64_t ldw,
+                                const void* X, int x_dtype, int64_t N, int64_t ldx, int bits, int64_t block,
+                                float damp, uint8_t* codes, float* lo, float* scale, float* W_hat, void* ws,
+                                size_t ws_bytes, void* stream) {
+  quip_status s = layer_args(tf, w_dtype, ldw, x_dtype, N, ldx, bits, block, damp);
+  if (s != QUIP_OK) return s;
+  if (!W || !X || !codes || !lo || !scale) return QUIP_ERR_ARG;
+  LayerWs L;
+  if ((s = layer_ws(tf, N, w_dtype, x_dtype, block, false, &L)) != QUIP_OK) return s;
+  if ((s = check_ws(ws, ws_bytes, L.total)) != QUIP_OK) return s;
+  return layer_device(tf, seed, W, w_dtype, ldw, X, x_dtype, N, ldx, bits, block, damp, codes, lo, scale, W_hat,
+                      L, static_cast<char*>(ws), S(stream), nullptr, nullptr, nullptr);
+}
+
+quip_status quip_quantize_layer_host(quip_transform* tf, uint64_t seed, const void* W_host, int w_dtype,
+                                     int64_t ldw, const void* X_host, int x_dtype, int64_t N, int64_t ldx,
+                                     int bits, int64_t block, float damp, uint8_t* codes_host, float* lo_host,
+                                     float* scale_host, float* W_hat_host, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  quip_status s = layer_args(tf, w_dtype, ldw, x_dtype, N, ldx, bits, block, damp);
+  if (s != QUIP_OK) return s;
+  if (!W_host || !X_host || !codes_host || !lo_host || !scale_host) return QUIP_ERR_ARG;
+  LayerWs L;
+  if ((s = layer_ws(tf, N, w_dtype, x_dtype, block, true, &L)) != QUIP_OK) return s;
+  if ((s = check_ws(ws, ws_bytes, L.total)) != QUIP_OK) return s;
+  const int64_t m = tf->m, n = tf->n;
+  const size_t wes = w_dtype == QUIP_BF16 ? 2 : 4, xes = x_dtype == QUIP_BF16 ? 2 : 4;
+  char* Wd = static_cast<char*>(ws) + L.H + L.D + L.Wt + L.stage;
+  char* Xd = Wd + L.Wd;
+  uint8_t* codes = reinterpret_cast<uint8_t*>(Xd + L.Xd);
+  float* lo = reinterpret_cast<float*>(reinterpret_cast<char*>(codes) + L.codes);
+  float* sc = reinterpret_cast<float*>(reinterpret_cast<char*>(lo) + L.lo);
+  float* What = reinterpret_cast<float*>(reinterpret_cast<char*>(sc) + L.sc);
+  cudaStream_t st = S(stream), cp = nullptr;
+  QCHECK(copy_stream(&cp));
+  const int64_t step = layer_x_chunk(N);
+  const int nch = (int)((N + step - 1) / step);
+  std::vector<cudaEvent_t> ev(nch + 4, nullptr);
+  for (auto& e : ev) QCHECK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+  cudaEvent_t fork = ev[nch], w_ready = ev[nch + 1], q_done = ev[nch + 2], out_done = ev[nch + 3];
+  // the copies start after earlier work on the caller's stream, which may
+  // still be reading this workspace
+  QCHECK(cudaEventRecord(fork, st));
+  QCHECK(cudaStreamWaitEvent(cp, fork, 0));
+  int c = 0;
+  for (int64_t a = 0; a < N; a += step, ++c) {
+    const int64_t b = std::min(N, a + step);
+    QCHECK(cudaMemcpy2DAsync(Xd + (size_t)a * n * xes, (size_t)n * xes,
+                             static_cast<const char*>(X_host) + (size_t)a * ldx * xes, (size_t)ldx * xes,
+                             (size_t)n * xes, (size_t)(b - a), cudaMemcpyHostToDevice, cp));
+    QCHECK(cudaEventRecord(ev[c], cp));
+  }
+  QCHECK(cudaMemcpy2DAsync(Wd, (size_t)n * wes, W_host, (size_t)ldw * wes, (size_t)n * wes, (size_t)m,
+                           cudaMemcpyHostToDevice, cp));
+  QCHECK(cudaEventRecord(w_ready, cp));
+  s = layer_device(tf, seed, Wd, w_dtype, n, Xd, x_dtype, N, n, bits, block, damp, codes, lo, sc, What, L,
+                   static_cast<char*>(ws), st, ev.data(), w_ready, q_done);
+  if (s == QUIP_OK) {
+    // codes and grid go back while W^ is formed; W^ after it
+    QCHECK(cudaStreamWaitEvent(cp, q_done, 0));
+    QCHECK(cudaMemcpyAsync(codes_host, codes, (size_t)m * n, cudaMemcpyDeviceToHost, cp));
+    QCHECK(cudaMemcpyAsync(lo_host, lo, (size_t)m * 4, cudaMemcpyDeviceToHost, cp));
+    QCHECK(cudaMemcpyAsync(scale_host, sc, (size_t)m * 4, cudaMemcpyDeviceToHost, cp));
+    if (W_hat_host) QCHECK(cudaMemcpyAsync(W_hat_host, What, (size_t)m * n * 4, cudaMemcpyDeviceToHost, st));
+  }
+  // the caller's stream covers every copy: it waits for the copy stream
+  QCHECK(cudaEventRecord(out_done, cp));
+  QCHECK(cudaStreamWaitEvent(st, out_done, 0));
+  for (auto& e : ev) cudaEventDestroy(e);
+  return s;
+}
+
+}  // extern "C"
 
 quip_status quip_timing_begin(void) {
   std::lock_guard<std::mutex> lk(g_timing_mu);
