@@ -103,8 +103,8 @@ __device__ __forceinline__ void nb_arrive(int id, int count) {
 // Maps: tmA over the accumulator and tmW over W~ (m x n fp32, LQB_S x 32 boxes), tmUT over
 // the transposed factor (n x n fp32, LQB_S x 128 boxes), tmU over the
 // factor Ů (the LDL's output, row stride ldu; 32 x 16 boxes).
-constexpr int LQB_ROWS = 32;                           // rows per CTA
-constexpr int LQB_THREADS = 128;                       // warp 0 rounds, warps 1-3 help
+constexpr int LQB_ROWS = 32;                           // rows per sub-group
+constexpr int LQB_THREADS = 128;                       // per sub-group: warp 0 rounds, warps 1-3 help
 constexpr int LQB_S = 132;                             // smem row stride of acc and UT
 constexpr int LQB_ES = 20;                             // smem row stride of the slots: 16 errors, 4 code words
 constexpr int LQB_ACC = LQB_ROWS * LQB_S * 4;          // bytes of the acc tile
@@ -115,28 +115,44 @@ constexpr int LQB_PS = 136;                            // row stride (bf16) of t
 constexpr int LQB_CS = 144;                            // row stride (bytes) of the staged codes
 constexpr int LQB_P = 3 * LQB_ROWS * LQB_PS * 2;       // bytes of the staged pieces
 constexpr int LQB_C = LQB_ROWS * LQB_CS;               // bytes of the staged codes
-constexpr int LQB_SMEM = 128 + 2 * LQB_ACC + LQB_UT + LQB_BAND + LQB_E + LQB_P + LQB_C;
-constexpr int LQB_READY = 1, LQB_DONE = 3;             // named barrier ids (+ slot)
+// Shared memory of a CTA of SUB sub-groups: per sub-group acc, wt, the slots
+// and the staging buffers; UT and the band once.
+__host__ __device__ constexpr int lqb_smem(int sub) {
+  return 128 + LQB_UT + LQB_BAND + sub * (2 * LQB_ACC + LQB_E + LQB_P + LQB_C);
+}
+constexpr int LQB_SMEM = lqb_smem(1);
+constexpr int LQB_READY = 1, LQB_DONE = 3;             // named barrier ids (+ slot, + 4 x sub-group)
 
-__global__ void __launch_bounds__(LQB_THREADS, 1)
+// SUB sub-groups of 32 rows per CTA (SUB x 128 threads): each sub-group is
+// the 32-row unit described above, with its own rounding warp, helpers,
+// slots and named barriers; the sub-groups share the UT and band tiles.
+template <int SUB>
+__global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
     k_ldlq_block(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmUT,
                  const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmW,
                  int64_t m, int64_t n, int64_t k0, int w, const float* __restrict__ lo,
                  const float* __restrict__ sc, float qmax, uint8_t* __restrict__ codes,
                  __nv_bfloat16* __restrict__ Es, int64_t lde) {
+  constexpr int CROWS = SUB * LQB_ROWS;                // rows per CTA
+  constexpr int CTHREADS = SUB * LQB_THREADS;
   extern __shared__ __align__(16) uint8_t lqb_raw[];
-  float* acc = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(lqb_raw) + 127) & ~uintptr_t(127));
-  float* UT = acc + LQB_ROWS * LQB_S;
+  float* UT = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(lqb_raw) + 127) & ~uintptr_t(127));
   float* band = UT + 128 * LQB_S;
-  float* eslot = band + 128 * 32;                      // [2][32][LQB_ES]
-  float* wt = eslot + 2 * LQB_ROWS * LQB_ES;           // [32][LQB_S]: the rows' W~ of the block
-  __nv_bfloat16* ps = reinterpret_cast<__nv_bfloat16*>(wt + LQB_ROWS * LQB_S);   // [3][32][LQB_PS]
-  uint8_t* cs = reinterpret_cast<uint8_t*>(ps + 3 * LQB_ROWS * LQB_PS);        // [32][LQB_CS]
+  float* acc0 = band + 128 * 32;                       // [CROWS][LQB_S]: accumulated values
+  float* wt0 = acc0 + CROWS * LQB_S;                   // [CROWS][LQB_S]: the rows' W~ of the block
+  float* eslot0 = wt0 + CROWS * LQB_S;                 // [SUB][2][32][LQB_ES]
+  __nv_bfloat16* ps = reinterpret_cast<__nv_bfloat16*>(eslot0 + SUB * 2 * LQB_ROWS * LQB_ES);  // [3][CROWS][LQB_PS]
+  uint8_t* cs = reinterpret_cast<uint8_t*>(ps + 3 * CROWS * LQB_PS);                          // [CROWS][LQB_CS]
   __shared__ __align__(8) uint64_t bar;
   __shared__ int ok_s;
-  const int tid = threadIdx.x, warp = tid >> 5, r = tid & 31;
-  const int64_t row = (int64_t)blockIdx.x * LQB_ROWS + r;
+  const int tid = threadIdx.x, sg = tid / LQB_THREADS, warp = (tid % LQB_THREADS) >> 5, r = tid & 31;
+  const int srow = sg * LQB_ROWS + r;                  // this thread's row within the CTA
+  const int64_t row = (int64_t)blockIdx.x * CROWS + srow;
   const bool valid = row < m;
+  float* acc = acc0 + sg * LQB_ROWS * LQB_S;           // this sub-group's tiles
+  float* wt = wt0 + sg * LQB_ROWS * LQB_S;
+  float* eslot = eslot0 + sg * 2 * LQB_ROWS * LQB_ES;
+  const int bar_ready = LQB_READY + 4 * sg, bar_done = LQB_DONE + 4 * sg;
   if (tid == 0) {
     mbar_init(&bar, 1);
     fence_mbar_init();
@@ -144,9 +160,11 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
   __syncthreads();
   pdl_wait_then_release();
   if (tid == 0) {
-    mbar_arrive_expect_tx(&bar, (uint32_t)(2 * LQB_ACC + LQB_UT + LQB_BAND));
-    tma_load_2d(acc, &tmA, &bar, (int)k0, (int)(blockIdx.x * LQB_ROWS));
-    tma_load_2d(wt, &tmW, &bar, (int)k0, (int)(blockIdx.x * LQB_ROWS));
+    mbar_arrive_expect_tx(&bar, (uint32_t)(SUB * 2 * LQB_ACC + LQB_UT + LQB_BAND));
+    for (int u = 0; u < SUB; ++u) {
+      tma_load_2d(acc0 + u * LQB_ROWS * LQB_S, &tmA, &bar, (int)k0, (int)(blockIdx.x * CROWS + u * LQB_ROWS));
+      tma_load_2d(wt0 + u * LQB_ROWS * LQB_S, &tmW, &bar, (int)k0, (int)(blockIdx.x * CROWS + u * LQB_ROWS));
+    }
     tma_load_2d(UT, &tmUT, &bar, (int)k0, (int)k0);
     for (int i = 0; i < 8; ++i)
       tma_load_2d(band + 16 * 32 * i, &tmU, &bar, (int)(k0 + 16 * i), (int)(k0 + 16 * i));
@@ -158,7 +176,7 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
   if (!ok_s) return;
   // band: keep Ů[k][j] for k < j < w only
 #pragma unroll 4
-  for (int e = tid; e < 128 * 32; e += LQB_THREADS) {
+  for (int e = tid; e < 128 * 32; e += CTHREADS) {
     const int k = e >> 5, j = 16 * (k >> 4) + (e & 31);
     if (j <= k || j >= w) band[e] = 0.f;
   }
@@ -174,7 +192,7 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
 #pragma unroll 1
     for (int g = 0; g < ngroups; ++g) {
       const int slot = g & 1;
-      nb_sync(LQB_READY + slot, LQB_THREADS);
+      nb_sync(bar_ready + slot, LQB_THREADS);
       const float* eb = eslot + slot * LQB_ROWS * LQB_ES;
       if (h == 0) {
         // row r's codes and error pieces into the staging buffers
@@ -185,14 +203,14 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
           const float4 v = *reinterpret_cast<const float4*>(es + 4 * q);
           e[4 * q] = v.x, e[4 * q + 1] = v.y, e[4 * q + 2] = v.z, e[4 * q + 3] = v.w;
         }
-        *reinterpret_cast<uint4*>(cs + r * LQB_CS + 16 * g) = *reinterpret_cast<const uint4*>(es + 16);
+        *reinterpret_cast<uint4*>(cs + srow * LQB_CS + 16 * g) = *reinterpret_cast<const uint4*>(es + 16);
         uint32_t pk[3][8];
 #pragma unroll
         for (int t = 0; t < 16; t += 2)
           split3x2(e[t], e[t + 1], pk[0][t >> 1], pk[1][t >> 1], pk[2][t >> 1]);
 #pragma unroll
         for (int p = 0; p < 3; ++p) {
-          uint4* dst = reinterpret_cast<uint4*>(ps + (p * LQB_ROWS + r) * LQB_PS + 16 * g);
+          uint4* dst = reinterpret_cast<uint4*>(ps + (p * CROWS + srow) * LQB_PS + 16 * g);
           dst[0] = make_uint4(pk[p][0], pk[p][1], pk[p][2], pk[p][3]);
           dst[1] = make_uint4(pk[p][4], pk[p][5], pk[p][6], pk[p][7]);
         }
@@ -238,7 +256,7 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
                 make_float4(a[i][0], a[i][1], a[i][2], a[i][3]);
         }
       }
-      if (g + 2 < ngroups) nb_arrive(LQB_DONE + slot, LQB_THREADS);
+      if (g + 2 < ngroups) nb_arrive(bar_done + slot, LQB_THREADS);
     }
   } else {
 
@@ -261,7 +279,7 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
   for (int g = 0; g < ngroups; ++g) {
     const int slot = g & 1;
     // group g - 2's feedback is in acc, and its slot is free again
-    if (g >= 2) nb_sync(LQB_DONE + slot, LQB_THREADS);
+    if (g >= 2) nb_sync(bar_done + slot, LQB_THREADS);
     float cur[16];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -334,7 +352,7 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
     for (int q = 0; q < 4; ++q)
       *reinterpret_cast<float4*>(es + 4 * q) = make_float4(e[4 * q], e[4 * q + 1], e[4 * q + 2], e[4 * q + 3]);
     *reinterpret_cast<uint4*>(es + 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-    nb_arrive(LQB_READY + slot, LQB_THREADS);
+    nb_arrive(bar_ready + slot, LQB_THREADS);
 #pragma unroll
     for (int t = 0; t < 16; ++t) wv[t] = wn[t];
   }
@@ -343,17 +361,17 @@ __global__ void __launch_bounds__(LQB_THREADS, 1)
   __syncthreads();
   const int64_t pst = m * lde;
   const int nv = w / 8;                                // 16-byte vectors per row and piece
-  for (int e = tid; e < 3 * LQB_ROWS * nv; e += LQB_THREADS) {
-    const int p = e / (LQB_ROWS * nv), rr = (e / nv) % LQB_ROWS, v = e % nv;
-    const int64_t gr = (int64_t)blockIdx.x * LQB_ROWS + rr;
+  for (int e = tid; e < 3 * CROWS * nv; e += CTHREADS) {
+    const int p = e / (CROWS * nv), rr = (e / nv) % CROWS, v = e % nv;
+    const int64_t gr = (int64_t)blockIdx.x * CROWS + rr;
     if (gr < m)
       *reinterpret_cast<uint4*>(Es + p * pst + gr * lde + k0 + 8 * v) =
-          *reinterpret_cast<const uint4*>(ps + (p * LQB_ROWS + rr) * LQB_PS + 8 * v);
+          *reinterpret_cast<const uint4*>(ps + (p * CROWS + rr) * LQB_PS + 8 * v);
   }
   const int nc = w / 16;                               // 16-byte vectors of codes per row
-  for (int e = tid; e < LQB_ROWS * nc; e += LQB_THREADS) {
+  for (int e = tid; e < CROWS * nc; e += CTHREADS) {
     const int rr = e / nc, v = e % nc;
-    const int64_t gr = (int64_t)blockIdx.x * LQB_ROWS + rr;
+    const int64_t gr = (int64_t)blockIdx.x * CROWS + rr;
     if (gr < m)
       *reinterpret_cast<uint4*>(codes + gr * n + k0 + 16 * v) =
           *reinterpret_cast<const uint4*>(cs + rr * LQB_CS + 16 * v);

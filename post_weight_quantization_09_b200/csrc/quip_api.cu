@@ -714,30 +714,49 @@ static quip_status draw_side(const SideData& sd, uint64_t seed, int which, cudaS
         k_haar_cgs2<<<1, 256, 0, st>>>(sd.G, sd.Qc, Q, Q64, (int)d);
         continue;
       }
-      // Cholesky-QR2: Y = G R1^-1 (into Qc, which first holds G^T G), then
-      // Q = Y R2^-1 (G, no longer needed, holds Y^T Y)
+      // Cholesky-QR2 (rng.cuh).  Pass 1: C1 = G^T G packed into Qc, R1 in
+      // place, Y = G R1^-1 into Q64 (free until the end).  Pass 2: C2 = Y^T Y
+      // into Qc, R2 in place, Q = Y R2^-1 into G (free by then) and, rounded,
+      // into Q; then G is copied to Q64.
       static bool attr = false;
       if (!attr) {
-        QCHECK(cudaFuncSetAttribute(k_chol_solve64, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        QCHECK(cudaFuncSetAttribute(k_chol64, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)chol_solve_smem(HAAR_CHOL_MAX)));
+        QCHECK(cudaFuncSetAttribute(k_trsm_rows64, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)chol_solve_smem(HAAR_CHOL_MAX)));
         attr = true;
       }
       const unsigned t = (unsigned)((d + 31) / 32);
       const size_t smem = chol_solve_smem((int)d);
+      const size_t smem_t = (size_t)d * (d + 1) / 2 * sizeof(double);
+      const unsigned rows = (unsigned)((d + HAAR_SOLVE_ROWS - 1) / HAAR_SOLVE_ROWS);
+      // pass 1: C1 = G^T G (Qc, packed), R1 in place, Y = G R1^-1 into Q64
       {
         LaunchScope ls("k_gram64", st);
         k_gram64<<<dim3(t, t), 256, 0, st>>>(sd.G, sd.Qc, (int)d);
       }
       {
-        LaunchScope ls("k_chol_solve64", st);
-        k_chol_solve64<<<1, 1024, smem, st>>>(sd.Qc, sd.G, sd.Qc, nullptr, (int)d);
+        LaunchScope ls("k_chol64", st);
+        k_chol64<<<1, 1024, smem, st>>>(sd.Qc, sd.Qc, (int)d);
       }
       {
-        LaunchScope ls("k_gram64", st);
-        k_gram64<<<dim3(t, t), 256, 0, st>>>(sd.Qc, sd.G, (int)d);
+        LaunchScope ls("k_trsm_rows64", st);
+        k_trsm_rows64<<<rows, 32 * HAAR_SOLVE_ROWS, smem_t, st>>>(sd.Qc, sd.G, Q64, nullptr, (int)d);
       }
-      LaunchScope ls("k_chol_solve64", st);
-      k_chol_solve64<<<1, 1024, smem, st>>>(sd.G, sd.Qc, Q64, Q, (int)d);
+      // pass 2: C2 = Y^T Y (Qc), R2 in place, Q = Y R2^-1 into G, then to Q64 / Q
+      {
+        LaunchScope ls("k_gram64", st);
+        k_gram64<<<dim3(t, t), 256, 0, st>>>(Q64, sd.Qc, (int)d);
+      }
+      {
+        LaunchScope ls("k_chol64", st);
+        k_chol64<<<1, 1024, smem, st>>>(sd.Qc, sd.Qc, (int)d);
+      }
+      {
+        LaunchScope ls("k_trsm_rows64", st);
+        k_trsm_rows64<<<rows, 32 * HAAR_SOLVE_ROWS, smem_t, st>>>(sd.Qc, Q64, sd.G, Q, (int)d);
+      }
+      QCHECK(cudaMemcpyAsync(Q64, sd.G, (size_t)d * d * sizeof(double), cudaMemcpyDeviceToDevice, st));
     }
     // bf16 pieces of A, A^T, B, B^T for the tensor-core products
     for (int v = 0; v < 4; ++v) {
@@ -1177,11 +1196,17 @@ struct LdlqRun {
 
 constexpr int LDQ_BLK = 128;               // LDLQ block width (columns)
 
+// One 32-row sub-group per CTA while that fits one wave of the GPU, else two
+// (fewer waves of the rows' rounding chains).
 cudaError_t ldlq_block(const LdlqRun& r, int64_t k0, int w) {
-  const unsigned grid = (unsigned)((r.m + LQB_ROWS - 1) / LQB_ROWS);
+  const int64_t units = (r.m + LQB_ROWS - 1) / LQB_ROWS;
   LaunchScope ls("k_ldlq_block", r.st);
-  return launch_pdl(k_ldlq_block, dim3(grid), dim3(LQB_THREADS), (size_t)LQB_SMEM, r.st, r.tacc, r.tut,
-                    r.tband, r.tw, r.m, r.n, k0, w, r.lo, r.sc, r.qmax, r.codes, r.Es, r.n);
+  if (units <= num_sms())
+    return launch_pdl(k_ldlq_block<1>, dim3((unsigned)units), dim3(LQB_THREADS), (size_t)lqb_smem(1), r.st,
+                      r.tacc, r.tut, r.tband, r.tw, r.m, r.n, k0, w, r.lo, r.sc, r.qmax, r.codes, r.Es, r.n);
+  return launch_pdl(k_ldlq_block<2>, dim3((unsigned)((units + 1) / 2)), dim3(2 * LQB_THREADS),
+                    (size_t)lqb_smem(2), r.st, r.tacc, r.tut, r.tband, r.tw, r.m, r.n, k0, w, r.lo, r.sc,
+                    r.qmax, r.codes, r.Es, r.n);
 }
 
 // Tensor maps of a run: the block kernel's (accumulator, weights, the
@@ -1205,7 +1230,8 @@ bool ldlq_maps(LdlqRun& r, const float* UTf, const __nv_bfloat16* UTs, bool gemm
 void ldlq_block_attr() {
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(k_ldlq_block, cudaFuncAttributeMaxDynamicSharedMemorySize, LQB_SMEM);
+    cudaFuncSetAttribute(k_ldlq_block<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, lqb_smem(1));
+    cudaFuncSetAttribute(k_ldlq_block<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, lqb_smem(2));
     attr = true;
   }
 }

@@ -193,26 +193,21 @@ __device__ __forceinline__ double warp_allsum64(double v) {
   return v;
 }
 
-// X = Y R^-1 with R the upper Cholesky factor of C (C = R^T R; Cp packed by
-// columns, fp64).  One CTA of 1024 threads (32 warps), p <= HAAR_CHOL_MAX.
-// Cp is copied to shared memory and factored in place, left-looking, one row
-// of R per step: R[k, j] = (C[k, j] - sum_{i<k} R[i, k] R[i, j]) / R[k, k],
+// R: the upper Cholesky factor of C (C = R^T R; Cp packed by columns,
+// fp64), written packed by columns to Rp (Rp may alias Cp).  One CTA of 1024
+// threads (32 warps), p <= HAAR_CHOL_MAX.  Cp is copied to shared memory and
+// factored in place, left-looking, one row of R per step:
+// R[k, j] = (C[k, j] - sum_{i<k} R[i, k] R[i, j]) / R[k, k],
 // R[k, k] = sqrt(C[k, k] - sum_{i<k} R[i, k]^2); warp w takes the columns
 // j = k + w, k + w + 32, ..., its lanes the terms i = lane, lane + 32, ...
 // (consecutive rows of a column are consecutive in shared memory), summed
-// by a butterfly.  Then the rows of X, one warp per row: for k = 0 .. p - 1,
-// X[r, k] = (Y[r, k] - sum_{i<k} X[r, i] R[i, k]) / R[k, k], lane l keeping
-// X[r, i] and Y[r, i] for i = l, l + 32, ... in registers.  X may alias Cp
-// (Cp is read in full before X is written); X must not alias Y.  out32, when
-// not NULL, gets X rounded to fp32 (row-major).  A pivot that is not
-// positive and finite is recorded as QUIP_ERR_NONFINITE.
+// by a butterfly.  A pivot that is not positive and finite is recorded as
+// QUIP_ERR_NONFINITE (and Rp is left as it is).
 // Dynamic smem: chol_solve_smem(p).
-__global__ void __launch_bounds__(1024, 1) k_chol_solve64(const double* Cp, const double* __restrict__ Y,
-                                                          double* X, float* __restrict__ out32, int p) {
+__global__ void __launch_bounds__(1024, 1) k_chol64(const double* Cp, double* Rp, int p) {
   extern __shared__ double chs[];
   double* R = chs;                                   // packed by columns, p (p + 1) / 2
   double* row = R + (int64_t)p * (p + 1) / 2;        // p: row k before the scaling
-  double* rinv = row + p;                            // p: 1 / R[k][k]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t np = (int64_t)p * (p + 1) / 2;
   for (int64_t e = tid; e < np; e += blockDim.x) R[e] = Cp[e];
@@ -240,43 +235,63 @@ __global__ void __launch_bounds__(1024, 1) k_chol_solve64(const double* Cp, cons
     ok = ok && d > 0.0 && d < INFINITY;
     const double rkk = sqrt(d);
     for (int j = k + tid; j < p; j += blockDim.x) R[packed_col(k, j)] = (j == k) ? rkk : row[j] / rkk;
-    if (tid == 0) rinv[k] = 1.0 / rkk;
     __syncthreads();
   }
   if (!ok) {
     if (tid == 0) record_status(QUIP_ERR_NONFINITE);
     return;
   }
-  for (int r = warp; r < p; r += 32) {
-    double yv[HAAR_CHOL_T], xv[HAAR_CHOL_T];
+  for (int64_t e = tid; e < np; e += blockDim.x) Rp[e] = R[e];
+}
+
+constexpr int HAAR_SOLVE_ROWS = 8;          // rows of X per CTA (one warp each)
+
+// X = Y R^-1, one warp per row of X (HAAR_SOLVE_ROWS rows per CTA), R (packed
+// by columns) copied to each CTA's shared memory: for k = 0 .. p - 1,
+// X[r, k] = (Y[r, k] - sum_{i<k} X[r, i] R[i, k]) / R[k, k], lane l keeping
+// X[r, i] and Y[r, i] for i = l, l + 32, ... in registers.  X must not alias
+// Y or Rp.  out32, when not NULL, gets X rounded to fp32 (row-major).
+// p <= HAAR_CHOL_MAX.  Dynamic smem: p (p + 1) / 2 doubles.
+__global__ void __launch_bounds__(32 * HAAR_SOLVE_ROWS) k_trsm_rows64(const double* __restrict__ Rp,
+                                                                    const double* __restrict__ Y,
+                                                                    double* __restrict__ X,
+                                                                    float* __restrict__ out32, int p) {
+  extern __shared__ double chs[];
+  double* R = chs;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t np = (int64_t)p * (p + 1) / 2;
+  for (int64_t e = tid; e < np; e += blockDim.x) R[e] = Rp[e];
+  __syncthreads();
+  const int r = blockIdx.x * HAAR_SOLVE_ROWS + warp;
+  if (r >= p) return;
+  double yv[HAAR_CHOL_T], xv[HAAR_CHOL_T];
 #pragma unroll
-    for (int t = 0; t < HAAR_CHOL_T; ++t) {
-      const int i = lane + 32 * t;
-      yv[t] = i < p ? Y[(int64_t)r * p + i] : 0.0;
-      xv[t] = 0.0;
-    }
+  for (int t = 0; t < HAAR_CHOL_T; ++t) {
+    const int i = lane + 32 * t;
+    yv[t] = i < p ? Y[(int64_t)r * p + i] : 0.0;
+    xv[t] = 0.0;
+  }
 #pragma unroll
-    for (int kq = 0; kq < HAAR_CHOL_T; ++kq) {
-      for (int kl = 0; kl < 32; ++kl) {
-        const int k = 32 * kq + kl;
-        if (k >= p) break;
-        double s = 0.0;
+  for (int kq = 0; kq < HAAR_CHOL_T; ++kq) {
+    for (int kl = 0; kl < 32; ++kl) {
+      const int k = 32 * kq + kl;
+      if (k >= p) break;
+      double s = 0.0;
 #pragma unroll
-        for (int t = 0; t <= kq; ++t) {
-          const int i = lane + 32 * t;
-          if (i < k) s = fma(xv[t], R[packed_col(i, k)], s);
-        }
-        s = warp_allsum64(s);
-        if (lane == kl) xv[kq] = (yv[kq] - s) * rinv[k];
+      for (int t = 0; t <= kq; ++t) {
+        const int i = lane + 32 * t;
+        if (i < k) s = fma(xv[t], R[packed_col(i, k)], s);
       }
+      s = warp_allsum64(s);
+      if (lane == kl) xv[kq] = (yv[kq] - s) / R[packed_col(k, k)];
     }
+  }
 #pragma unroll
-    for (int t = 0; t < HAAR_CHOL_T; ++t) {
-      const int i = lane + 32 * t;
-      if (i < p) {
-        X[(int64_t)r * p + i] = xv[t];
-        if (out32) out32[(int64_t)r * p + i] = (float)xv[t];
-      }
+  for (int t = 0; t < HAAR_CHOL_T; ++t) {
+    const int i = lane + 32 * t;
+    if (i < p) {
+      X[(int64_t)r * p + i] = xv[t];
+      if (out32) out32[(int64_t)r * p + i] = (float)xv[t];
     }
   }
 }

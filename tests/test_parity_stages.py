@@ -240,6 +240,9 @@ def _ldlq_inputs(m, n, seed, const_rows=()):
 @pytest.mark.parametrize("m,n,bits,block", [
     (64, 128, 2, 32), (100, 256, 3, 64), (33, 256, 4, 128), (256, 128, 2, 128), (1, 64, 8, 64),
     (70, 512, 2, 128), (40, 320, 3, 64), (129, 192, 2, 32),
+    # more 32-row units than SMs: two units per CTA, the last CTA's second
+    # unit partly past the last row
+    (4800 + 17, 192, 2, 64),
 ])
 def test_ldlq_stage_parity(m, n, bits, block):
     W, U = _ldlq_inputs(m, n, seed=m * n + bits, const_rows=(0,) if m > 1 else ())
