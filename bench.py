@@ -913,8 +913,24 @@ def main():
     ap.add_argument("--decode-batch", type=int, default=1)
     ap.add_argument("--decode-blocks", type=int, default=32)
     ap.add_argument("--bits", type=int, default=2, help="code width of --decode")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="a slice of the workload with this many rows of W (its n, sides and bits kept; "
+                         "a Kronecker m side keeps q and takes p = rows / q): for profiling at a size "
+                         "a capture can hold")
+    ap.add_argument("--tokens", type=int, default=0, help="calibration tokens of the slice (default: the workload's)")
     args = ap.parse_args()
     cfg = CONFIGS[args.config]
+    if args.rows or args.tokens:
+        from dataclasses import replace as _rep
+        ms = cfg.m_side
+        if args.rows:
+            if ms.kind == "kronecker":
+                if args.rows % ms.q:
+                    raise SystemExit(f"--rows must be a multiple of q = {ms.q}")
+                ms = _rep(ms, p=args.rows // ms.q)
+            elif ms.kind == "hadamard" and args.rows & (args.rows - 1):
+                raise SystemExit("--rows must be a power of two for a Hadamard m side")
+        cfg = _rep(cfg, name=f"{cfg.name}[slice]", m=args.rows or cfg.m, N=args.tokens or cfg.N, m_side=ms)
     if args.permute:
         from dataclasses import replace
         cfg = replace(cfg, m_side=replace(cfg.m_side, permute=True),

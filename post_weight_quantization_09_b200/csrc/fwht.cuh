@@ -278,6 +278,97 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// ---------------------------------------------------------------- 8192-point rows
+// Radix 32 x 16 x 16 ... as 32 x 32 x 8: index bits 0-4, 5-9 and 10-12 in
+// registers, 32 values per thread, two transpositions through shared memory
+// between them.  Shared index of element k: k + 4 (k / 32) (four pad words
+// per 32), so a thread's 32 consecutive elements start 16-byte aligned (the
+// first write is four-wide) and every other access of a warp covers 32
+// consecutive elements: conflict-free throughout, and no shuffles.
+__device__ __forceinline__ int pad32x4(int k) { return k + 4 * (k >> 5); }
+
+__device__ __forceinline__ void load32(const float* p, float (&v)[32]) {
+  const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 f = q[i];
+    v[4 * i] = f.x, v[4 * i + 1] = f.y, v[4 * i + 2] = f.z, v[4 * i + 3] = f.w;
+  }
+}
+__device__ __forceinline__ void load32(const __nv_bfloat16* p, float (&v)[32]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 u = q[i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
+      v[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+  }
+}
+
+// One row of 8192 per CTA (256 threads).  Thread t (warp w, lane l): stage A
+// on elements 32 t + r (r = bits 0-4); stage B on l + 32 r + 1024 w (bits
+// 5-9); stage C on t % 256 + 256 g + 1024 r (g < 4, r < 8: bits 10-12),
+// stored straight from registers, 32 consecutive floats per warp store.
+template <typename TIn>
+__global__ void __launch_bounds__(256)
+    k_fwht_row8192(const TIn* __restrict__ in, int64_t ldin, float* out, int64_t ldout,
+                   const float* __restrict__ pre, const float* __restrict__ post,
+                   const float* __restrict__ row_sign, float scale) {
+  __shared__ __align__(16) float sr[8192 + 1024];
+  const int t = threadIdx.x, w = t >> 5, l = t & 31;
+  const int64_t row = blockIdx.x;
+  float v[32];
+  load32(in + row * ldin + 32 * t, v);
+  if (pre) {
+    const float4* pp = reinterpret_cast<const float4*>(pre + 32 * t);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 f = pp[q];
+      v[4 * q] *= f.x, v[4 * q + 1] *= f.y, v[4 * q + 2] *= f.z, v[4 * q + 3] *= f.w;
+    }
+  }
+  reg_fwht<5>(v);
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<float4*>(sr + pad32x4(32 * t) + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < 32; ++r) v[r] = sr[pad32x4(l + 32 * r + 1024 * w)];
+  reg_fwht<5>(v);
+#pragma unroll
+  for (int r = 0; r < 32; ++r) sr[pad32x4(l + 32 * r + 1024 * w)] = v[r];
+  __syncthreads();
+  // stage C: four groups g of eight values each (register index 8 g + r)
+#pragma unroll
+  for (int g = 0; g < 4; ++g)
+#pragma unroll
+    for (int r = 0; r < 8; ++r) v[8 * g + r] = sr[pad32x4(t + 256 * g + 1024 * r)];
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      if ((e & h) == 0) {
+        const float a = v[e], b = v[e + h];
+        v[e] = a + b;
+        v[e + h] = a - b;
+      }
+    }
+  }
+  const float rs = row_sign ? row_sign[row] * scale : scale;
+  float* o = out + row * ldout;
+#pragma unroll
+  for (int g = 0; g < 4; ++g)
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int k = t + 256 * g + 1024 * r;
+      o[k] = v[8 * g + r] * rs * (post ? post[k] : 1.f);
+    }
+}
+
 // 4096-point column transform of 8 columns per CTA (1024 threads), in place.
 // Thread unit u (two per thread) handles column c = u % 8: stage A on rows
 // 16 o + j (o = u / 8; loaded straight from global memory), stage B on rows

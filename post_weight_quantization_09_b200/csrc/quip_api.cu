@@ -262,6 +262,12 @@ cudaError_t fwht_rows(const TIn* in, int64_t ldin, float* out, int64_t ldout, in
                                                          scale);
     return cudaGetLastError();
   }
+  if (L == 13) {
+    LaunchScope ls("k_fwht_rows", st);
+    k_fwht_row8192<TIn><<<(unsigned)rows, 256, 0, st>>>(in, ldin, out, ldout, pre, post, row_sign,
+                                                         scale);
+    return cudaGetLastError();
+  }
   const int T = (int)(d / 16);
   const int NT = T > 256 ? T : 256;
   const int RPC = NT / T;
@@ -435,16 +441,15 @@ cudaError_t kron_tc_launch(const CUtensorMap& tf, const CUtensorMap& tx, kron::P
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(kron::k_kron_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kron::SMEM_BYTES);
+                                         kron::SMEM_LIMIT);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  kp.tiles_m = (kp.M + kron::BM - 1) / kron::BM;
-  kp.tiles_n = (kp.N + kron::BN - 1) / kron::BN;
-  const int64_t tiles = (int64_t)kp.tiles_m * kp.tiles_n * kp.slabs;
+  kp.tiles_m = (kp.N + kron::BM - 1) / kron::BM;
+  const int64_t tiles = (int64_t)kp.tiles_m * kp.slabs;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, num_sms()));
   LaunchScope ls("k_kron_tc", st);
-  return launch_pdl(kron::k_kron_tc, dim3(grid), dim3(256), (size_t)kron::SMEM_BYTES, st, tf, tx, kp, mode);
+  return launch_pdl(kron::k_kron_tc, dim3(grid), dim3(256), (size_t)kron::smem_bytes(kp.nf), st, tf, tx, kp, mode);
 }
 
 // Whether the m-side (column) Kronecker transform of an R x c matrix runs on
@@ -486,23 +491,24 @@ cudaError_t kron_cols_tc(const SideData& sd, bool transpose, const TIn* src, int
   }
   // stage 1: T_a' = B' X_a' for the p slabs of q rows, into P2 as pieces
   CUtensorMap mf, mx;
+  const int nfq = (int)((q + 15) / 16 * 16), nfp = (int)((p + 15) / 16 * 16);
   const __nv_bfloat16* fb = factor_pieces(sd, transpose ? 3 : 2);
-  if (!make_tmap_bf16_2d(&mf, fb, (uint64_t)q, 3 * (uint64_t)q, (uint64_t)factor_ld(q) * 2, 64, kron::BM) ||
+  if (!make_tmap_bf16_2d(&mf, fb, (uint64_t)q, 3 * (uint64_t)q, (uint64_t)factor_ld(q) * 2, 64, (uint32_t)nfq) ||
       !make_tmap_bf16_2d(&mx, xsrc, (uint64_t)c, (uint64_t)(xp * R), (uint64_t)xld * 2, 64, 64))
     return cudaErrorInvalidValue;
   kron::Params kp{};
-  kp.M = (int)q, kp.K = (int)q, kp.N = (int)c, kp.slabs = (int)p;
+  kp.d = (int)q, kp.nf = nfq, kp.N = (int)c, kp.slabs = (int)p;
   kp.f_piece_rows = (int)q, kp.x_pieces = xp, kp.x_piece_rows = R, kp.x_slab_rows = q;
   kp.Yp = P2, kp.ldy = c, kp.y_slab_rows = q, kp.y_piece_elems = R * c;
   cudaError_t e = kron_tc_launch(mf, mx, kp, kron::OUT_PIECES, st);
   if (e != cudaSuccess) return e;
   // stage 2: Y = A' T with T as p x (q c), into dst (fp32)
   const __nv_bfloat16* fa = factor_pieces(sd, transpose ? 1 : 0);
-  if (!make_tmap_bf16_2d(&mf, fa, (uint64_t)p, 3 * (uint64_t)p, (uint64_t)factor_ld(p) * 2, 64, kron::BM) ||
+  if (!make_tmap_bf16_2d(&mf, fa, (uint64_t)p, 3 * (uint64_t)p, (uint64_t)factor_ld(p) * 2, 64, (uint32_t)nfp) ||
       !make_tmap_bf16_2d(&mx, P2, (uint64_t)(q * c), 3 * (uint64_t)p, (uint64_t)(q * c) * 2, 64, 64))
     return cudaErrorInvalidValue;
   kron::Params k2{};
-  k2.M = (int)p, k2.K = (int)p, k2.N = (int)(q * c), k2.slabs = 1;
+  k2.d = (int)p, k2.nf = nfp, k2.N = (int)(q * c), k2.slabs = 1;
   k2.f_piece_rows = (int)p, k2.x_pieces = 3, k2.x_piece_rows = p, k2.x_slab_rows = 0;
   k2.Y = dst, k2.ldy = q * c, k2.y_slab_rows = 0;
   return kron_tc_launch(mf, mx, k2, kron::OUT_F32, st);
@@ -721,13 +727,13 @@ static quip_status draw_side(const SideData& sd, uint64_t seed, int which, cudaS
       static bool attr = false;
       if (!attr) {
         QCHECK(cudaFuncSetAttribute(k_chol64, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)chol_solve_smem(HAAR_CHOL_MAX)));
+                                    (int)chol64_smem(HAAR_CHOL_MAX)));
         QCHECK(cudaFuncSetAttribute(k_trsm_rows64, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)chol_solve_smem(HAAR_CHOL_MAX)));
         attr = true;
       }
       const unsigned t = (unsigned)((d + 31) / 32);
-      const size_t smem = chol_solve_smem((int)d);
+      const size_t smem = chol64_smem((int)d);
       const size_t smem_t = (size_t)d * (d + 1) / 2 * sizeof(double);
       const unsigned rows = (unsigned)((d + HAAR_SOLVE_ROWS - 1) / HAAR_SOLVE_ROWS);
       // pass 1: C1 = G^T G (Qc, packed), R1 in place, Y = G R1^-1 into Q64

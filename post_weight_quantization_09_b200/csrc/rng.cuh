@@ -193,55 +193,67 @@ __device__ __forceinline__ double warp_allsum64(double v) {
   return v;
 }
 
+// Offset of (i, j), i <= j, in the row-major packed upper triangle (row i
+// holds columns i .. p - 1).
+__host__ __device__ __forceinline__ int64_t packed_row(int64_t i, int64_t j, int64_t p) {
+  return i * p - i * (i - 1) / 2 + (j - i);
+}
+
+constexpr int HAAR_CHOL_PARTS = 4;          // threads summing one entry of a row of R
+
 // R: the upper Cholesky factor of C (C = R^T R; Cp packed by columns,
 // fp64), written packed by columns to Rp (Rp may alias Cp).  One CTA of 1024
-// threads (32 warps), p <= HAAR_CHOL_MAX.  Cp is copied to shared memory and
-// factored in place, left-looking, one row of R per step:
+// threads, p <= HAAR_CHOL_MAX.  Cp is copied to shared memory packed by rows
+// and factored in place, left-looking, one row of R per step:
 // R[k, j] = (C[k, j] - sum_{i<k} R[i, k] R[i, j]) / R[k, k],
-// R[k, k] = sqrt(C[k, k] - sum_{i<k} R[i, k]^2); warp w takes the columns
-// j = k + w, k + w + 32, ..., its lanes the terms i = lane, lane + 32, ...
-// (consecutive rows of a column are consecutive in shared memory), summed
-// by a butterfly.  A pivot that is not positive and finite is recorded as
-// QUIP_ERR_NONFINITE (and Rp is left as it is).
-// Dynamic smem: chol_solve_smem(p).
+// R[k, k] = sqrt(C[k, k] - sum_{i<k} R[i, k]^2).  Thread (part, jj) forms the
+// part of the sum for column j = k + jj over i = part, part + 4, ... (a
+// warp reads 32 consecutive entries of a row of R and broadcasts R[i, k]);
+// the four parts meet in shared memory.  A pivot that is not positive and
+// finite is recorded as QUIP_ERR_NONFINITE (and Rp is left as it is).
+// Dynamic smem: chol_solve_smem(p) (the packed factor and 2 p doubles) plus
+// HAAR_CHOL_PARTS x 256 doubles.
+__host__ __device__ constexpr size_t chol64_smem(int p) {
+  return chol_solve_smem(p) + (size_t)HAAR_CHOL_PARTS * 256 * sizeof(double) + 256 * sizeof(int);
+}
 __global__ void __launch_bounds__(1024, 1) k_chol64(const double* Cp, double* Rp, int p) {
   extern __shared__ double chs[];
-  double* R = chs;                                   // packed by columns, p (p + 1) / 2
-  double* row = R + (int64_t)p * (p + 1) / 2;        // p: row k before the scaling
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t np = (int64_t)p * (p + 1) / 2;
-  for (int64_t e = tid; e < np; e += blockDim.x) R[e] = Cp[e];
+  double* R = chs;                                   // packed by rows, p (p + 1) / 2
+  double* part_s = R + (int64_t)p * (p + 1) / 2 + 2 * p;   // [HAAR_CHOL_PARTS][256]
+  int* rb = reinterpret_cast<int*>(part_s + HAAR_CHOL_PARTS * 256);   // R[i][j] = R[rb[i] + j]
+  const int tid = threadIdx.x, part = tid >> 8, jj = tid & 255;
+  for (int i = tid; i < p; i += blockDim.x) rb[i] = (int)(packed_row(i, i, p) - i);
+  for (int j = tid; j < p; j += blockDim.x)
+    for (int i = 0; i <= j; ++i) R[packed_row(i, j, p)] = Cp[packed_col(i, j)];
   __syncthreads();
   bool ok = true;
   for (int k = 0; k < p; ++k) {
-    double rk[HAAR_CHOL_T];
-#pragma unroll
-    for (int t = 0; t < HAAR_CHOL_T; ++t) {
-      const int i = lane + 32 * t;
-      rk[t] = i < k ? R[packed_col(i, k)] : 0.0;
-    }
-    for (int j = k + warp; j < p; j += 32) {
-      double s = 0.0;
-#pragma unroll
-      for (int t = 0; t < HAAR_CHOL_T; ++t) {
-        const int i = lane + 32 * t;
-        if (i < k) s = fma(rk[t], R[packed_col(i, j)], s);
+    const int j = k + jj;
+    // row k is rewritten below, after the barrier: read its diagonal first
+    const double ckk = R[rb[k] + k];
+    double s = 0.0;
+    if (j < p)
+      for (int i = part; i < k; i += HAAR_CHOL_PARTS) {
+        const double* ri = R + rb[i];
+        s = fma(ri[k], ri[j], s);
       }
-      s = warp_allsum64(s);
-      if (lane == 0) row[j] = R[packed_col(k, j)] - s;
-    }
+    part_s[part * 256 + jj] = s;
     __syncthreads();
-    const double d = row[k];
+    const double d = ckk - ((part_s[0] + part_s[256]) + (part_s[512] + part_s[768]));
     ok = ok && d > 0.0 && d < INFINITY;
-    const double rkk = sqrt(d);
-    for (int j = k + tid; j < p; j += blockDim.x) R[packed_col(k, j)] = (j == k) ? rkk : row[j] / rkk;
+    if (part == 0 && j < p) {
+      const double rkk = sqrt(d);
+      const double v = R[rb[k] + j] - ((part_s[jj] + part_s[256 + jj]) + (part_s[512 + jj] + part_s[768 + jj]));
+      R[rb[k] + j] = (jj == 0) ? rkk : v / rkk;
+    }
     __syncthreads();
   }
   if (!ok) {
     if (tid == 0) record_status(QUIP_ERR_NONFINITE);
     return;
   }
-  for (int64_t e = tid; e < np; e += blockDim.x) Rp[e] = R[e];
+  for (int j = tid; j < p; j += blockDim.x)
+    for (int i = 0; i <= j; ++i) Rp[packed_col(i, j)] = R[packed_row(i, j, p)];
 }
 
 constexpr int HAAR_SOLVE_ROWS = 8;          // rows of X per CTA (one warp each)
