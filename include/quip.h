@@ -400,9 +400,11 @@ quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int
  * (quip_hessian_accumulate), damping (quip_hessian_finalize, alpha = damp),
  * H~ = V H V^T and the LDL of H~ (quip_incoherence_forward, quip_ldl),
  * W~ = U W V^T and LDLQ (quip_ldlq_quantize), then, when W_hat is not NULL,
- * W^ = U^T (lo + s codes) V (quip_dequantize, quip_incoherence_inverse), in
- * that order on `stream`; each step has the arguments, layout and errors of
- * its own entry point.  The codes and grid are those of LDLQ in the
+ * W^ = U^T (lo + s codes) V (quip_dequantize, quip_incoherence_inverse);
+ * each step has the arguments, layout and errors of its own entry point.
+ * The Hessian path (V, H, H~, the LDL) runs on a library-owned stream of the
+ * highest priority, forked from and joined into `stream`; the weight path
+ * (U, W~) runs on `stream` beside it; LDLQ and W^ follow on `stream`.  The codes and grid are those of LDLQ in the
  * incoherent basis (quip_ldlq_quantize); W^ is the dequantised layer in the
  * original basis.
  *   tf       : a transform made for this layer's m x n (quip_transform_create);

@@ -225,14 +225,16 @@ cudaError_t split_gemm(const CUtensorMap& ta, const CUtensorMap& tb, sgemm::Para
   if (p.upper_only || (!tb64 && !tb128))
     return split_gemm_tn<sgemm::BN>(ta, tb, p, st, name, max_ctas);
   // Tile width by a cost model: waves of tiles x tile width (a tile's time
-  // grows with its width at a fixed K); 64-wide tiles count double, their
-  // MMAs being bound by the A operand's shared-memory reads.  Ties go to
-  // the wider tile.
+  // grows with its width at a fixed K); narrower tiles move more operand
+  // bytes per product from L2 (an A slot per K block serves TN columns), so
+  // 128-wide tiles count 1.25 times and 64-wide ones double (their MMAs are
+  // also bound by the A operand's shared-memory reads).  Ties go to the
+  // wider tile.
   const int cap = max_ctas > 0 ? std::min(max_ctas, num_sms()) : num_sms();
   const int64_t tm = (p.M + sgemm::BM - 1) / sgemm::BM;
   auto cost = [&](int tn) {
     const int64_t tiles = tm * ((p.N + tn - 1) / tn);
-    return ((tiles + cap - 1) / cap) * tn * (tn == 64 ? 2 : 1);
+    return ((tiles + cap - 1) / cap) * tn * (tn == 64 ? 8 : tn == 128 ? 5 : 4);
   };
   int best = sgemm::BN;
   if (tb128 && cost(128) < cost(best)) best = 128;
@@ -1778,12 +1780,33 @@ cudaError_t copy_stream(cudaStream_t* out) {
   return cudaSuccess;
 }
 
+// A per-device stream of the highest priority for the Hessian path of the
+// whole-layer call (H, H~, the LDL: a latency-bound chain that should get
+// SMs first), created on first use and kept for the process.
+cudaError_t hpath_stream(cudaStream_t* out) {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev]) {
+    int least = 0, greatest = 0;
+    if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
+    e = cudaStreamCreateWithPriority(&streams[dev], cudaStreamNonBlocking, greatest);
+    if (e != cudaSuccess) return e;
+  }
+  *out = streams[dev];
+  return cudaSuccess;
+}
+
 // Device workspace of the whole-layer call: H (n x n), D (n), W~ (m x n),
 // then one region shared by the stages (the largest stage workspace); the
 // host variant adds device copies of W and X, and the device results: codes
 // (m x n), lo and scale (m each) and W^ (m x n fp32).
 struct LayerWs {
-  size_t H, D, Wt, stage, Wd, Xd, codes, lo, sc, What, total;
+  size_t H, D, Wt, stage, wstage, Wd, Xd, codes, lo, sc, What, total;
 };
 
 quip_status layer_ws(const quip_transform* tf, int64_t N, int w_dtype, int x_dtype, int64_t block, bool host,
@@ -1802,6 +1825,9 @@ quip_status layer_ws(const quip_transform* tf, int64_t N, int w_dtype, int x_dty
   o->D = round256((size_t)n * 4);
   o->Wt = round256((size_t)m * n * 4);
   o->stage = round256(std::max<size_t>(st, 256));
+  // the W path's forward transform runs beside the Hessian path: its own region
+  if ((s = quip_workspace_size(QUIP_OP_INCOHERENCE_FORWARD, tf, m, n, block, &b)) != QUIP_OK) return s;
+  o->wstage = round256(std::max<size_t>(b, 256));
   if (host) {
     o->Wd = round256((size_t)m * n * wes);
     o->Xd = round256((size_t)std::max<int64_t>(N, 1) * n * xes);
@@ -1809,7 +1835,7 @@ quip_status layer_ws(const quip_transform* tf, int64_t N, int w_dtype, int x_dty
     o->lo = o->sc = round256((size_t)m * 4);
     o->What = round256((size_t)m * n * 4);
   }
-  o->total = o->H + o->D + o->Wt + o->stage + o->Wd + o->Xd + o->codes + o->lo + o->sc + o->What;
+  o->total = o->H + o->D + o->Wt + o->stage + o->wstage + o->Wd + o->Xd + o->codes + o->lo + o->sc + o->What;
   return QUIP_OK;
 }
 
@@ -1831,11 +1857,14 @@ int64_t layer_x_chunk(int64_t N) {
   return std::max<int64_t>(2048, (c + 2047) / 2048 * 2048);
 }
 
-// The device part of the layer from W, X on the device: draw (U, V), H,
-// damping, H~, LDL, W~, LDLQ, and (W_hat non-NULL) W^.  x_ready, when given,
-// is one event per token chunk of layer_x_chunk(N), waited for before that
-// chunk is accumulated; w_ready is waited for before W is read; q_done is
-// recorded once codes and grid are final.
+// The device part of the layer from W, X on the device.  Two paths that
+// meet before LDLQ: the Hessian path on the library's high-priority stream
+// (draw V, H = X^T X / N, damping, H~, the LDL of H~) and the weight path
+// on `st` (draw U, W~ = U W V^T, once V is drawn); then, on `st`, LDLQ and
+// (W_hat non-NULL) W^.  x_ready, when given, is one event per token chunk
+// of layer_x_chunk(N), waited for before that chunk is accumulated; w_ready
+// is waited for before W is read; q_done is recorded once codes and grid
+// are final.  Each path has its own workspace region.
 quip_status layer_device(quip_transform* tf, uint64_t seed, const void* W, int w_dtype, int64_t ldw,
                          const void* X, int x_dtype, int64_t N, int64_t ldx, int bits, int64_t block,
                          float damp, uint8_t* codes, float* lo, float* scale, float* W_hat,
@@ -1846,35 +1875,61 @@ quip_status layer_device(quip_transform* tf, uint64_t seed, const void* W, int w
   float* D = reinterpret_cast<float*>(ws + L.H);
   float* Wt = reinterpret_cast<float*>(ws + L.H + L.D);
   void* sw = ws + L.H + L.D + L.Wt;
-  quip_status s;
-  if ((s = quip_transform_draw(tf, seed, st)) != QUIP_OK) return s;
-  const size_t xes = x_dtype == QUIP_BF16 ? 2 : 4;
-  if (x_ready) {
-    const int64_t step = layer_x_chunk(N);
-    int c = 0;
-    for (int64_t a = 0; a < N; a += step, ++c) {
-      QCHECK(cudaStreamWaitEvent(st, x_ready[c], 0));
-      const int64_t b = std::min(N, a + step);
-      if ((s = quip_hessian_accumulate(static_cast<const char*>(X) + (size_t)a * ldx * xes, x_dtype, b - a, n,
-                                       ldx, H, a > 0 ? 1 : 0, st)) != QUIP_OK)
-        return s;
+  void* sw2 = ws + L.H + L.D + L.Wt + L.stage;
+  cudaStream_t hs = nullptr;
+  QCHECK(hpath_stream(&hs));
+  cudaEvent_t ev[3] = {};                             // fork, V drawn, Hessian path done
+  for (auto& e : ev) QCHECK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+  quip_status s = QUIP_OK;
+  auto run = [&]() -> quip_status {
+    quip_status r;
+    QCHECK(cudaEventRecord(ev[0], st));
+    QCHECK(cudaStreamWaitEvent(hs, ev[0], 0));
+    // ---- Hessian path (hs)
+    if ((r = draw_side(tf->side[1], seed, 1, hs)) != QUIP_OK) return r;
+    QCHECK(cudaEventRecord(ev[1], hs));
+    const size_t xes = x_dtype == QUIP_BF16 ? 2 : 4;
+    if (x_ready) {
+      const int64_t step = layer_x_chunk(N);
+      int c = 0;
+      for (int64_t a = 0; a < N; a += step, ++c) {
+        QCHECK(cudaStreamWaitEvent(hs, x_ready[c], 0));
+        const int64_t b = std::min(N, a + step);
+        if ((r = quip_hessian_accumulate(static_cast<const char*>(X) + (size_t)a * ldx * xes, x_dtype, b - a, n,
+                                         ldx, H, a > 0 ? 1 : 0, hs)) != QUIP_OK)
+          return r;
+      }
+    } else if ((r = quip_hessian_accumulate(X, x_dtype, N, n, ldx, H, 0, hs)) != QUIP_OK) {
+      return r;
     }
-  } else if ((s = quip_hessian_accumulate(X, x_dtype, N, n, ldx, H, 0, st)) != QUIP_OK) {
-    return s;
+    if ((r = quip_hessian_finalize(H, n, N, damp, hs)) != QUIP_OK) return r;
+    if ((r = quip_incoherence_forward(tf, nullptr, QUIP_F32, n, nullptr, H, sw, L.stage, hs)) != QUIP_OK) return r;
+    if ((r = quip_ldl(H, D, n, sw, L.stage, hs)) != QUIP_OK) return r;
+    QCHECK(cudaEventRecord(ev[2], hs));
+    // ---- weight path (st)
+    if ((r = draw_side(tf->side[0], seed, 0, st)) != QUIP_OK) return r;
+    if (w_ready) QCHECK(cudaStreamWaitEvent(st, w_ready, 0));
+    QCHECK(cudaStreamWaitEvent(st, ev[1], 0));
+    if ((r = quip_incoherence_forward(tf, W, w_dtype, ldw, Wt, nullptr, sw2, L.wstage, st)) != QUIP_OK) return r;
+    // ---- both
+    QCHECK(cudaStreamWaitEvent(st, ev[2], 0));
+    if ((r = quip_ldlq_quantize(Wt, H, n, m, n, bits, block, codes, lo, scale, sw, L.stage, st)) != QUIP_OK)
+      return r;
+    if (q_done) QCHECK(cudaEventRecord(q_done, st));
+    if (W_hat) {
+      if ((r = quip_dequantize(codes, lo, scale, m, n, W_hat, st)) != QUIP_OK) return r;
+      if ((r = quip_incoherence_inverse(tf, W_hat, W_hat, sw, L.stage, st)) != QUIP_OK) return r;
+    }
+    return QUIP_OK;
+  };
+  s = run();
+  if (s != QUIP_OK) {
+    // the caller's stream still waits for whatever was enqueued on hs
+    cudaEventRecord(ev[2], hs);
+    cudaStreamWaitEvent(st, ev[2], 0);
   }
-  if ((s = quip_hessian_finalize(H, n, N, damp, st)) != QUIP_OK) return s;
-  if ((s = quip_incoherence_forward(tf, nullptr, QUIP_F32, n, nullptr, H, sw, L.stage, st)) != QUIP_OK) return s;
-  if ((s = quip_ldl(H, D, n, sw, L.stage, st)) != QUIP_OK) return s;
-  if (w_ready) QCHECK(cudaStreamWaitEvent(st, w_ready, 0));
-  if ((s = quip_incoherence_forward(tf, W, w_dtype, ldw, Wt, nullptr, sw, L.stage, st)) != QUIP_OK) return s;
-  if ((s = quip_ldlq_quantize(Wt, H, n, m, n, bits, block, codes, lo, scale, sw, L.stage, st)) != QUIP_OK)
-    return s;
-  if (q_done) QCHECK(cudaEventRecord(q_done, st));
-  if (W_hat) {
-    if ((s = quip_dequantize(codes, lo, scale, m, n, W_hat, st)) != QUIP_OK) return s;
-    if ((s = quip_incoherence_inverse(tf, W_hat, W_hat, sw, L.stage, st)) != QUIP_OK) return s;
-  }
-  return QUIP_OK;
+  for (auto& e : ev) cudaEventDestroy(e);
+  return s;
 }
 }  // namespace
 
@@ -1918,7 +1973,7 @@ quip_status quip_quantize_layer_host(quip_transform* tf, uint64_t seed, const vo
   if ((s = check_ws(ws, ws_bytes, L.total)) != QUIP_OK) return s;
   const int64_t m = tf->m, n = tf->n;
   const size_t wes = w_dtype == QUIP_BF16 ? 2 : 4, xes = x_dtype == QUIP_BF16 ? 2 : 4;
-  char* Wd = static_cast<char*>(ws) + L.H + L.D + L.Wt + L.stage;
+  char* Wd = static_cast<char*>(ws) + L.H + L.D + L.Wt + L.stage + L.wstage;
   char* Xd = Wd + L.Wd;
   uint8_t* codes = reinterpret_cast<uint8_t*>(Xd + L.Xd);
   float* lo = reinterpret_cast<float*>(reinterpret_cast<char*>(codes) + L.codes);
