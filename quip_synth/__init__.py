@@ -30,7 +30,7 @@ from typing import Dict, Tuple
 import numpy as np
 
 __all__ = ["Side", "LayerConfig", "CONFIGS", "make_layer", "to_bf16_bits",
-           "bf16_bits_to_f32", "round_to_bf16"]
+           "bf16_bits_to_f32", "round_to_bf16", "calibration_chunks"]
 
 
 @dataclass(frozen=True)
@@ -149,3 +149,24 @@ def random_layer(m: int, n: int, N: int, seed: int, dtype: str = "f32", sigma: f
                       sigma=sigma, x_outlier_frac=x_outlier_frac, x_lognormal=lognormal,
                       dtype=dtype, seed=seed)
     return make_layer(cfg)
+
+
+def calibration_chunks(n: int, N: int, chunk: int, seed: int, x_outlier_frac: float = 0.01,
+                       x_outlier_mult: float = 20.0):
+    """Calibration activations streamed in token chunks, the recipe of the
+    Llama-shaped workloads (i.i.d. N(0, 1), a fraction of channels scaled by
+    ``x_outlier_mult``, rounded to bf16) at a token count too large to hold
+    at once: the QuIP paper calibrates on 128 segments of 2048 tokens
+    (Experiments, "Setup.").  The outlier channels are drawn once from
+    PCG64(seed); chunk c from PCG64(seed + 1 + c).  Yields (first token,
+    float32 values, bf16 bit patterns) per chunk of at most ``chunk`` tokens."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    k = int(round(x_outlier_frac * n))
+    ch = rng.choice(n, size=k, replace=False) if k > 0 else np.zeros(0, dtype=np.int64)
+    for c, a in enumerate(range(0, N, chunk)):
+        b = min(N, a + chunk)
+        r = np.random.Generator(np.random.PCG64(seed + 1 + c))
+        X = r.standard_normal((b - a, n), dtype=np.float32)
+        X[:, ch] *= np.float32(x_outlier_mult)
+        xb = to_bf16_bits(X)
+        yield a, bf16_bits_to_f32(xb), xb
