@@ -320,28 +320,34 @@ class ClockSampler:
 
 class OracleSample:
     """The FP64 oracle's own stage functions on a bounded sample of one layer,
-    each stage timed separately and scaled to the whole layer.
+    each stage timed on its own and extrapolated to the whole layer.
 
-    Row-separable stages run on ``rows`` sampled rows of W~ (the forward and
-    inverse transforms of those rows, their grid, LDLQ and dequantisation),
-    scaled by m / rows; the Hessian runs on the first ``tokens`` tokens,
-    scaled by N / tokens; the Hessian's transform on ``hrows`` rows of H~,
-    scaled by n / hrows; the transforms' draw, the damping and the LDL run at
-    full size.  Stages whose input would need a previous full-size stage take
-    a stand-in of the same shape (the LDL factors the damped token-sample
-    Hessian, LDLQ uses that factor; the inverse transform reads W in place of
-    the dequantised W~), which changes no stage's work.  ``stages`` lists
-    (name, scale); ``run(name)`` times one stage once and returns seconds."""
+    Row-separable stages (the forward and inverse transforms of W's rows,
+    grid and LDLQ, dequantisation) run on sampled rows, the Hessian on the
+    first tokens, the Hessian's transform on sampled rows of H~, each at two
+    sample sizes s1 < s2; a stage's whole-layer time is the straight line
+    through the two timings at the full size (a fixed part, e.g. building a
+    transform matrix or the per-column loop of LDLQ, plus a part per row),
+    t(S) = t1 + (t2 - t1) (S - s1) / (s2 - s1), neither part below zero.
+    The transforms' draw, the damping and the LDL run at full size.  Stages
+    whose input would need a previous full-size stage take a stand-in of the
+    same shape (the LDL factors the damped token-sample Hessian, LDLQ uses
+    that factor; the inverse transform reads W in place of the dequantised
+    W~), which changes no stage's work.  ``items`` lists (stage, size index);
+    ``run(item)`` times one stage once at one size and returns seconds."""
 
-    def __init__(self, cfg: LayerConfig, d, rows: int = 64, tokens: int = 1024, hrows: int = 256):
+    ROWS = (64, 256)
+    TOKENS = (512, 2048)
+    HROWS = (128, 512)
+
+    def __init__(self, cfg: LayerConfig, d):
         import oracle as O
         self.O, self.cfg = O, cfg
         m, n, N = cfg.m, cfg.n, cfg.N
-        self.r, self.t, self.hr = min(rows, m), min(tokens, N), min(hrows, n)
         rng = np.random.default_rng(7)
-        self.rows = np.sort(rng.choice(m, self.r, replace=False))
-        self.hrows_idx = np.sort(rng.choice(n, self.hr, replace=False))
-        self.X = d["X"][:self.t]
+        self.rows = np.sort(rng.choice(m, min(self.ROWS[1], m), replace=False))
+        self.hrows = np.sort(rng.choice(n, min(self.HROWS[1], n), replace=False))
+        self.X = d["X"][:min(self.TOKENS[1], N)]
         self.W = d["W"]
         # untimed set-up: the inputs each timed stage reads
         self.U = O.make_side(cfg.seed, "m", cfg.m_side.kind, m, cfg.m_side.p, cfg.m_side.q)
@@ -351,48 +357,76 @@ class OracleSample:
         self.Wt = O.incoherence_rows(self.W, self.U, self.V, self.rows)
         self.lo, self.s = O.row_grid(self.Wt, cfg.bits)
         self.codes, _, _ = O.ldlq(self.Wt, self.Uf, self.lo, self.s, cfg.bits)
-        self.stages = [("transform", 1.0), ("hessian", N / self.t), ("finalize", 1.0),
-                       ("incoherence_fwd_h", n / self.hr), ("incoherence_fwd_w", m / self.r),
-                       ("ldl", 1.0), ("ldlq", m / self.r), ("dequant", m / self.r),
-                       ("incoherence_inv", m / self.r)]
+        # stage -> (sample sizes, full size); None: full size only
+        self.scale = {"transform": None, "hessian": (self.TOKENS, N), "finalize": None,
+                      "incoherence_fwd_h": (self.HROWS, n), "incoherence_fwd_w": (self.ROWS, m),
+                      "ldl": None, "ldlq": (self.ROWS, m), "dequant": (self.ROWS, m),
+                      "incoherence_inv": (self.ROWS, m)}
+        self.items = []
+        for nm, sc in self.scale.items():
+            self.items += [(nm, 0)] if sc is None else [(nm, 0), (nm, 1)]
 
-    def run(self, name: str) -> float:
+    def size(self, name: str, k: int) -> int:
+        sc = self.scale[name]
+        return 0 if sc is None else min(sc[0][k], sc[1])
+
+    def run(self, item) -> float:
         O, cfg = self.O, self.cfg
+        name, k = item
+        sz = self.size(name, k)
         t0 = time.perf_counter()
         if name == "transform":
             O.make_side(cfg.seed, "m", cfg.m_side.kind, cfg.m, cfg.m_side.p, cfg.m_side.q)
             O.make_side(cfg.seed, "n", cfg.n_side.kind, cfg.n, cfg.n_side.p, cfg.n_side.q)
         elif name == "hessian":
-            O.hessian(self.X)
+            O.hessian(self.X[:sz])
         elif name == "finalize":
             O.damp(self.H, cfg.damp)
         elif name == "incoherence_fwd_h":
-            O.incoherence_hessian_rows(self.H, self.V, self.hrows_idx)
+            O.incoherence_hessian_rows(self.H, self.V, self.hrows[:sz])
         elif name == "incoherence_fwd_w":
-            O.incoherence_rows(self.W, self.U, self.V, self.rows)
+            O.incoherence_rows(self.W, self.U, self.V, self.rows[:sz])
         elif name == "ldl":
             O.udu(self.H)
         elif name == "ldlq":
-            lo, s = O.row_grid(self.Wt, cfg.bits)
-            O.ldlq(self.Wt, self.Uf, lo, s, cfg.bits)
+            lo, s = O.row_grid(self.Wt[:sz], cfg.bits)
+            O.ldlq(self.Wt[:sz], self.Uf, lo, s, cfg.bits)
         elif name == "dequant":
-            O.dequantize(self.codes, self.lo, self.s)
+            O.dequantize(self.codes[:sz], self.lo[:sz], self.s[:sz])
         elif name == "incoherence_inv":
-            O.incoherence_inverse_rows(self.W, self.U, self.V, self.rows)
+            O.incoherence_inverse_rows(self.W, self.U, self.V, self.rows[:sz])
         else:
             raise KeyError(name)
         return time.perf_counter() - t0
 
+    def stage_seconds(self, times) -> dict:
+        """Whole-layer seconds per stage from {item: [seconds, ...]} (means)."""
+        out = {}
+        for nm, sc in self.scale.items():
+            t1 = statistics.mean(times[(nm, 0)])
+            if sc is None:
+                out[nm] = t1
+                continue
+            t2 = statistics.mean(times[(nm, 1)])
+            s1, s2, full = self.size(nm, 0), self.size(nm, 1), sc[1]
+            if s2 <= s1:
+                out[nm] = t1 * full / max(s1, 1)
+                continue
+            per = max(0.0, (t2 - t1) / (s2 - s1))
+            fixed = max(0.0, t1 - per * s1)
+            out[nm] = fixed + per * full
+        return out
+
     def estimate(self, times) -> float:
-        """Whole-layer seconds from {stage: [seconds, ...]} (mean per stage)."""
-        return sum(statistics.mean(times[nm]) * sc for nm, sc in self.stages)
+        return sum(self.stage_seconds(times).values())
 
     def describe(self) -> str:
         c = self.cfg
-        return (f"FP64 oracle stage functions on {c.name}: Hessian on {self.t} of {c.N} tokens (x{c.N / self.t:g}), "
-                f"H~ on {self.hr} of {c.n} rows (x{c.n / self.hr:g}), W~, grid, LDLQ, dequantisation and "
-                f"inverse transform on {self.r} of {c.m} rows (x{c.m / self.r:g}); transform draw, damping and "
-                f"LDL at full size; each stage timed on its own and scaled linearly to the whole layer")
+        r, t, h = (self.size("ldlq", 0), self.size("ldlq", 1)), self.TOKENS, self.HROWS
+        return (f"FP64 oracle stage functions on {c.name}: Hessian on {t[0]} and {t[1]} of {c.N} tokens, H~ on "
+                f"{h[0]} and {h[1]} of {c.n} rows, W~, grid, LDLQ, dequantisation and inverse transform on "
+                f"{r[0]} and {r[1]} of {c.m} rows, each extrapolated to the whole layer along the line through "
+                f"its two timings (fixed + per-row part); transform draw, damping and LDL at full size")
 
 
 def blas_threads():
@@ -447,39 +481,38 @@ def stage_schedule(names, steps: int):
 
 
 def cpu_baseline_entry(cfg: LayerConfig, d) -> dict:
-    """The oracle on its bounded sample: every stage once untimed, then once
-    timed; the whole-layer estimate from the timed pass."""
+    """The oracle on its bounded sample: one untimed call to start the BLAS
+    threads, then every (stage, size) item twice, the faster timing kept (a
+    single short timing is noisy); the whole-layer estimate from those."""
     smp = OracleSample(cfg, d)
-    names = [nm for nm, _ in smp.stages]
-    for nm in names:
-        smp.run(nm)
-    times = {nm: [smp.run(nm)] for nm in names}
+    smp.run(("hessian", 0))
+    times = {it: [min(smp.run(it), smp.run(it))] for it in smp.items}
     sec = smp.estimate(times)
     return {"value": cfg.m * cfg.n / sec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": smp.describe() + f"; whole layer estimated at {sec:.1f} s",
-            "stage_seconds": {nm: round(statistics.mean(v), 4) for nm, v in times.items()}}
+            "stage_seconds": {nm: round(v, 4) for nm, v in smp.stage_seconds(times).items()}}
 
 
 def run_reference(args, cfg: LayerConfig):
     """The FP64 oracle (this problem's reference: the pages ship no code) on
     the host cores.  Each step times a bounded part of the oracle's sample of
-    the layer (stage functions in rotation, see OracleSample); value is the
-    layer's weights over the whole-layer time those samples give."""
+    the layer ((stage, size) items in rotation, see OracleSample); value is
+    the layer's weights over the whole-layer time those timings give."""
     world, rank, _ = dist_setup()
     if rank != 0:
         return
     d = make_layer(cfg)
     smp = OracleSample(cfg, d)
-    names = [nm for nm, _ in smp.stages]
-    for step in stage_schedule(names, max(args.warmup, 1)):
-        for nm in step:
-            smp.run(nm)
-    times = {nm: [] for nm in names}
+    items = smp.items
+    for step in stage_schedule(items, max(args.warmup, 1)):
+        for it in step:
+            smp.run(it)
+    times = {it: [] for it in items}
     step_s = []
-    for step in stage_schedule(names, args.steps):
+    for step in stage_schedule(items, args.steps):
         t0 = time.perf_counter()
-        for nm in step:
-            times[nm].append(smp.run(nm))
+        for it in step:
+            times[it].append(smp.run(it))
         step_s.append(time.perf_counter() - t0)
     sec = smp.estimate(times)
     value = cfg.m * cfg.n / sec
@@ -491,10 +524,9 @@ def run_reference(args, cfg: LayerConfig):
         "data": "synthetic", "config": config_desc(cfg, args),
         "layer_seconds_estimated": sec,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": smp.describe() + f"; step i times stage(s) {stage_schedule(names, args.steps)[0]}"
-                                   f"... in rotation over {len(names)} stages; ms_per_step is the measured wall "
-                                   f"time of one step, value the layer's weights over the {sec:.1f} s whole-layer "
-                                   f"estimate"},
+                         "sample": smp.describe() + f"; the {len(items)} (stage, size) timings in rotation, "
+                                   f"one or more per step; ms_per_step is the measured wall time of one step, "
+                                   f"value the layer's weights over the {sec:.1f} s whole-layer estimate"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

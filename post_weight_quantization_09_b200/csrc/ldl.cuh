@@ -91,8 +91,9 @@ __device__ __forceinline__ void helpers_sync() {      // the helper warps of k_l
 __device__ __forceinline__ bool warp_chol_inv32(float* S, int lds, float* X, int ldx,
                                                 float* scratch) {
   const int lane = threadIdx.x & 31;
-  float a[32], rin[32];
+  float a[32];
   float* col = scratch + 32 * LDL_LDX;            // 2 x 32
+  float* rin = col + 64;                          // 32: 1 / R_kk (kept in shared memory, not registers)
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     const float4 v = *reinterpret_cast<const float4*>(S + lane * lds + 4 * q);
@@ -108,7 +109,7 @@ __device__ __forceinline__ bool warp_chol_inv32(float* S, int lds, float* X, int
     const float piv = __shfl_sync(0xffffffffu, self, k);
     ok = ok && (piv > 0.f) && (piv < INFINITY);
     const float r = rsqrtf(piv);
-    rin[k] = r;
+    if (lane == 0) rin[k] = r;
     const float l = (lane == k) ? piv * r : a[k] * r;
     a[k] = l;
     if (k > 0) {
@@ -134,13 +135,13 @@ __device__ __forceinline__ bool warp_chol_inv32(float* S, int lds, float* X, int
   }
 #pragma unroll
   for (int j = 0; j < 32; ++j) scratch[j * LDL_LDX + lane] = (j >= lane) ? a[j] : 0.f;   // row j = column j of R
-  __syncwarp();
+  __syncwarp();                                   // also publishes rin
   float x[32];
 #pragma unroll
   for (int m = 0; m < 32; ++m) x[m] = (m == lane) ? 1.f : 0.f;
 #pragma unroll
   for (int k = 31; k >= 0; --k) {
-    x[k] *= rin[k];
+    x[k] *= rin[k];                               // broadcast read
     const float* rc = scratch + k * LDL_LDX;
 #pragma unroll
     for (int m4 = 0; m4 < k; m4 += 4) {
@@ -456,8 +457,8 @@ __global__ void __launch_bounds__(LDL_RT, 1)
                int nblk, __nv_bfloat16* __restrict__ Rs, float* __restrict__ Lout) {
   extern __shared__ __align__(16) uint8_t ldl_smem_raw[];
   pdl_wait_then_release();
-  float* T = align128(ldl_smem_raw);                 // 32 x LDL_LDA: H - Lin, then R12
-  float* Lt = T + LDL_RR * LDL_LDA;                  // 32 x LDL_LDA: Lin rows, then Lout
+  float* T = align128(ldl_smem_raw);                 // LDL_RR x LDL_LDA: H - Lin, then R12
+  float* Lt = T + LDL_RR * LDL_LDA;                  // LDL_RR x LDL_LDA: Lin rows, then Lout
   float* Rp = Lt + LDL_RR * LDL_LDA;                 // 128 x LDL_LDA: R_pp
   float* N = Rp + LDL_PB * LDL_LDA;                  // 128 x LDL_LDA: Nx
   float* X = N + LDL_PB * LDL_LDA;                   // 4 x 32 x LDL_LDX
