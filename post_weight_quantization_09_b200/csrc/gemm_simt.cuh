@@ -99,9 +99,126 @@ __global__ void __launch_bounds__(256) k_gemm_simt(GemmArgs g) {
   }
 }
 
+// fp64-accumulating GEMM with a larger register tile, for the products that
+// need fp64 sums (the n-side Kronecker factors): 128 x 128 output tile per
+// CTA of 256 threads, each thread 8 x 8 outputs as four 4 x 4 quadrants
+// (rows 4 ty + {0..3} and 64 + 4 ty + {0..3}, columns likewise with tx), so
+// a thread reads 16 doubles from shared memory per 64 FMAs and a warp's
+// reads are two 16-byte words per lane without bank conflicts.  K in slabs
+// of 8, the next slab loaded into registers while the current one is
+// used.  Inputs of any type are converted to fp64 on the way into shared
+// memory; the result is rounded to fp32 once.  Same GemmArgs as k_gemm_simt
+// (tri must be 0).
+constexpr int G64_BM = 128, G64_BN = 128, G64_BK = 8;
+
+template <typename TA, typename TB>
+__global__ void __launch_bounds__(256) k_gemm64(GemmArgs g) {
+  __shared__ __align__(16) double sA[2][G64_BK][G64_BM];
+  __shared__ __align__(16) double sB[2][G64_BK][G64_BN];
+  const int64_t ti = blockIdx.y, tj = blockIdx.x, b = blockIdx.z;
+  const TA* A = reinterpret_cast<const TA*>(g.A) + b * g.sab;
+  const TB* B = reinterpret_cast<const TB*>(g.B) + b * g.sbb;
+  float* C = g.C + b * g.scb;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int64_t i0 = ti * G64_BM, j0 = tj * G64_BN;
+  // staging: 128 x 8 elements of A and 8 x 128 of B per slab, 4 each per thread
+  double ra[4], rb[4];
+  auto load = [&](int64_t k0) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int idx = tid + e * 256;
+      {
+        const int kk = (g.sak == 1) ? (idx % G64_BK) : (idx / G64_BM);
+        const int ii = (g.sak == 1) ? (idx / G64_BK) : (idx % G64_BM);
+        const int64_t gi = i0 + ii, gk = k0 + kk;
+        ra[e] = (gi < g.M && gk < g.K) ? to_acc<double, TA>(A[gi * g.sam + gk * g.sak]) : 0.0;
+      }
+      {
+        const int jj = (g.sbn == 1) ? (idx % G64_BN) : (idx / G64_BK);
+        const int kk = (g.sbn == 1) ? (idx / G64_BN) : (idx % G64_BK);
+        const int64_t gj = j0 + jj, gk = k0 + kk;
+        rb[e] = (gj < g.N && gk < g.K) ? to_acc<double, TB>(B[gk * g.sbk + gj * g.sbn]) : 0.0;
+      }
+    }
+  };
+  auto store = [&](int buf) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int idx = tid + e * 256;
+      {
+        const int kk = (g.sak == 1) ? (idx % G64_BK) : (idx / G64_BM);
+        const int ii = (g.sak == 1) ? (idx / G64_BK) : (idx % G64_BM);
+        sA[buf][kk][ii] = ra[e];
+      }
+      {
+        const int jj = (g.sbn == 1) ? (idx % G64_BN) : (idx / G64_BK);
+        const int kk = (g.sbn == 1) ? (idx / G64_BN) : (idx % G64_BK);
+        sB[buf][kk][jj] = rb[e];
+      }
+    }
+  };
+  double acc[8][8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[r][c] = 0.0;
+  load(0);
+  store(0);
+  __syncthreads();
+  int buf = 0;
+  for (int64_t k0 = 0; k0 < g.K; k0 += G64_BK) {
+    const bool more = k0 + G64_BK < g.K;
+    if (more) load(k0 + G64_BK);
+#pragma unroll
+    for (int kk = 0; kk < G64_BK; ++kk) {
+      double a[8], bv[8];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const double2 a0 = *reinterpret_cast<const double2*>(&sA[buf][kk][64 * h + 4 * ty]);
+        const double2 a1 = *reinterpret_cast<const double2*>(&sA[buf][kk][64 * h + 4 * ty + 2]);
+        a[4 * h] = a0.x, a[4 * h + 1] = a0.y, a[4 * h + 2] = a1.x, a[4 * h + 3] = a1.y;
+        const double2 b0 = *reinterpret_cast<const double2*>(&sB[buf][kk][64 * h + 4 * tx]);
+        const double2 b1 = *reinterpret_cast<const double2*>(&sB[buf][kk][64 * h + 4 * tx + 2]);
+        bv[4 * h] = b0.x, bv[4 * h + 1] = b0.y, bv[4 * h + 2] = b1.x, bv[4 * h + 3] = b1.y;
+      }
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[r][c] = fma(a[r], bv[c], acc[r][c]);
+    }
+    if (more) {
+      store(buf ^ 1);
+      __syncthreads();
+      buf ^= 1;
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int64_t gi = i0 + 64 * (r >> 2) + 4 * ty + (r & 3);
+    if (gi >= g.M) continue;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int64_t gj = j0 + 64 * (c >> 2) + 4 * tx + (c & 3);
+      if (gj >= g.N) continue;
+      float* p = C + gi * g.scm + gj * g.scn;
+      const float v = (float)(g.alpha * acc[r][c]);
+      *p = (g.beta == 0.f) ? v : fmaf(g.beta, *p, v);
+    }
+  }
+}
+
 template <typename TA, typename TB, typename Acc = float>
 inline cudaError_t gemm_simt(const GemmArgs& g, int64_t batch, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || batch <= 0) return cudaSuccess;
+  if constexpr (std::is_same<Acc, double>::value) {
+    if (g.tri == 0) {
+      dim3 grid((unsigned)((g.N + G64_BN - 1) / G64_BN), (unsigned)((g.M + G64_BM - 1) / G64_BM),
+                (unsigned)batch);
+      LaunchScope ls("k_gemm64", st);
+      k_gemm64<TA, TB><<<grid, 256, 0, st>>>(g);
+      return cudaGetLastError();
+    }
+  }
   dim3 grid((unsigned)((g.N + SG_BN - 1) / SG_BN), (unsigned)((g.M + SG_BM - 1) / SG_BM),
             (unsigned)batch);
   {

@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(256, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nchunk = (p.K + KCP - 1) / KCP;
   const bool single = nchunk == 1;
+  constexpr int nbp = 3;                            // B pieces
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < A_SLOTS; ++s) {
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(256, 1)
         for (int pa = 0; pa < 3; ++pa)
           tma_load_2d(sa + s * A_BYTES + pa * A_PIECE_BYTES, &tmA, &sh->full_a[s], p.a_k0 + k,
                       pa * p.a_piece_rows + p.a_row0 + i0);
-        for (int pb = 2; pb >= 0; --pb, ++kb) {
+        for (int pb = nbp - 1; pb >= 0; --pb, ++kb) {
           const int r = kb % NB;
           if (!mbar_wait(&sh->empty_b[r], (uint32_t)(((kb / NB) & 1) ^ 1))) {
             sh->abort = 1;
@@ -177,7 +178,7 @@ __global__ void __launch_bounds__(256, 1)
             break;
           }
           const uint32_t a_base = smem_u32(sa + s * A_BYTES);
-          for (int pb = 2; pb >= 0; --pb, ++kb) {
+          for (int pb = nbp - 1; pb >= 0; --pb, ++kb) {
             const int r = kb % NB;
             if (!mbar_wait(&sh->full_b[r], (uint32_t)((kb / NB) & 1))) {
               sh->abort = 1;

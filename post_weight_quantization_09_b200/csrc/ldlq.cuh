@@ -158,16 +158,23 @@ __global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
     fence_mbar_init();
   }
   __syncthreads();
-  pdl_wait_then_release();
+  // W~, the transposed factor and the band come from kernels that finished
+  // before the one just ahead of this launch (a programmatic dependent launch
+  // starts only once its predecessor has passed its own wait): their copies
+  // start before the wait; the accumulated values, which that predecessor
+  // (a trailing GEMM) writes, after it
   if (tid == 0) {
     mbar_arrive_expect_tx(&bar, (uint32_t)(SUB * 2 * LQB_ACC + LQB_UT + LQB_BAND));
-    for (int u = 0; u < SUB; ++u) {
-      tma_load_2d(acc0 + u * LQB_ROWS * LQB_S, &tmA, &bar, (int)k0, (int)(blockIdx.x * CROWS + u * LQB_ROWS));
+    for (int u = 0; u < SUB; ++u)
       tma_load_2d(wt0 + u * LQB_ROWS * LQB_S, &tmW, &bar, (int)k0, (int)(blockIdx.x * CROWS + u * LQB_ROWS));
-    }
     tma_load_2d(UT, &tmUT, &bar, (int)k0, (int)k0);
     for (int i = 0; i < 8; ++i)
       tma_load_2d(band + 16 * 32 * i, &tmU, &bar, (int)(k0 + 16 * i), (int)(k0 + 16 * i));
+  }
+  pdl_wait_then_release();
+  if (tid == 0) {
+    for (int u = 0; u < SUB; ++u)
+      tma_load_2d(acc0 + u * LQB_ROWS * LQB_S, &tmA, &bar, (int)k0, (int)(blockIdx.x * CROWS + u * LQB_ROWS));
     const bool ok = mbar_wait(&bar, 0);
     if (!ok) mbar_wait(&bar, 0);                       // copies in flight: bounded again
     ok_s = ok ? 1 : 0;

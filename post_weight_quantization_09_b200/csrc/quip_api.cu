@@ -392,7 +392,14 @@ cudaError_t kron_rows(const TIn* src, int64_t ldsrc, float* dst, int64_t rows,
   else g.sbk = q, g.sbn = 1;              // (B^T)^T = B
   g.sbb = 0;
   g.C = tmp, g.scm = q, g.scn = 1, g.scb = n;
-  cudaError_t e = gemm_simt<TIn, F, Acc>(g, rows, st);
+  int64_t batches = rows;
+  if (ldsrc == n) {
+    // contiguous rows: the p x q views of all rows stack into one (rows p) x q
+    // matrix, one GEMM instead of `rows` small ones
+    g.M = rows * p, g.sab = 0, g.scb = 0;
+    batches = 1;
+  }
+  cudaError_t e = gemm_simt<TIn, F, Acc>(g, batches, st);
   if (e != cudaSuccess) return e;
   // dst_i = A' tmp_i : M = p, N = q, K = p
   GemmArgs h{};
