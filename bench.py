@@ -165,25 +165,24 @@ def kernel_work(cfg: LayerConfig, method: str = "ldlq", passes: int = 1):
     return kw
 
 
-# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# one `ncu --set full` capture of each kernel on the attn7b workload (see
-# profiles/), with the first 12 hex digits of the SHA-1 of the source file
-# the kernel was built from: the figure is reported only while that file is
-# unchanged and only for the workload it was captured on.
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
+# the gate70b layer, with the first 12 hex digits of the SHA-1 of the source
+# file the kernel was built from: a figure is reported only while that file
+# is unchanged and only for that workload.  The counters were taken on the
+# layer's first 7168 of 28672 rows and 8192 of 32768 tokens (one capture
+# stays a few GB): the LDL depends on n alone, so its split GEMMs' average is
+# the full layer's; the LDLQ GEMMs' A operand and accumulator and the
+# row-wise kernels' bytes grow with the rows, so their figures are the
+# slice's times 28672 / 7168 = 4.  Writes still in L2 when a kernel ends are
+# not counted (the LDLQ block kernel's codes and error pieces).
 KERNEL_TRAFFIC = {
-    "k_syrk_tc": ("syrk_tc.cuh", "260ad4eebdfc", 71597824),
-    "k_ldlq_block": ("ldlq.cuh", "eb4bda779455", 6490368),
-    "k_ldl_factor": ("ldl.cuh", "6428de196929", 339200),
-    "k_ldl_rows": ("ldl.cuh", "6428de196929", 4653824),
-    "k_dequant": ("ldlq.cuh", "449a391e49fc", 26102272),
-    "k_row_grid": ("ldlq.cuh", "449a391e49fc", 67615488),
-    "k_split_upper_transposed": ("gemm_tc.cuh", "92453856d596", 148098048),
-    "k_gemm_split_tc[ldl]": ("gemm_tc.cuh", "4a73f99d9186", 28432128),
-    "k_fwht_cols": ("fwht.cuh", "94ad670265cc", 82387456),
-    "k_greedy_start": ("rounding.cuh", "d4ef99d9fa8b", 263645696),
-    "k_greedy_factors": ("rounding.cuh", "d4ef99d9fa8b", 229122560),
+    "k_gemm_split_tc[ldlq]": ("gemm_tc.cuh", "1aabcc329733", 172766566),
+    "k_gemm_split_tc[ldl]": ("gemm_tc.cuh", "1aabcc329733", 61325242),
+    "k_ldlq_block": ("ldlq.cuh", "0bb6d47b4440", 44938240),
+    "k_dequant": ("ldlq.cuh", "0bb6d47b4440", 941438976),
+    "k_row_grid": ("ldlq.cuh", "0bb6d47b4440", 970614784),
 }
-TRAFFIC_WORKLOAD = "attn7b"
+TRAFFIC_WORKLOAD = "gate70b"
 
 
 def kernel_traffic(name: str, workload: str):
