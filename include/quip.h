@@ -185,6 +185,9 @@ quip_status quip_hessian_finalize(float* H, int64_t n, int64_t N_total, float da
  *                   skipped when H is NULL.  W and H may not both be NULL.
  * The two are independent: a caller may transform H first (the LDL needs
  * only H~) and W later, e.g. while W is still being copied to the device.
+ * When V is a Hadamard side with n >= 16, W (with ldw * element size a
+ * multiple of 16 bytes), W_t and H must be 16-byte aligned (the row kernels
+ * move 16-byte vectors), else QUIP_ERR_ARG.
  * ws: workspace for QUIP_OP_INCOHERENCE_FORWARD.
  */
 quip_status quip_incoherence_forward(const quip_transform* tf, const void* W, int w_dtype,
@@ -193,7 +196,9 @@ quip_status quip_incoherence_forward(const quip_transform* tf, const void* W, in
 
 /*
  * Incoherence post-processing: W_hat = U^T W_hat_t V (m x n fp32, row stride
- * n).  W_hat may equal W_hat_t (in place).  ws: QUIP_OP_INCOHERENCE_INVERSE.
+ * n).  W_hat may equal W_hat_t (in place).  When V is a Hadamard side with
+ * n >= 16 both must be 16-byte aligned, else QUIP_ERR_ARG.
+ * ws: QUIP_OP_INCOHERENCE_INVERSE.
  */
 quip_status quip_incoherence_inverse(const quip_transform* tf, const float* W_hat_t,
                                      float* W_hat, void* ws, size_t ws_bytes, void* stream);

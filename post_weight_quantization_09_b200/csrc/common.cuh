@@ -24,6 +24,18 @@
 
 namespace quip {
 
+// fp32 -> three bf16 pieces with x = p0 + p1 + p2 to fp32 precision (each
+// piece rounds the remainder of the ones before it to nearest even): the
+// operands of the split-bf16 tensor-core products.
+__device__ __forceinline__ void split3(float x, __nv_bfloat16& p0, __nv_bfloat16& p1,
+                                       __nv_bfloat16& p2) {
+  p0 = __float2bfloat16_rn(x);
+  const float r1 = x - __bfloat162float(p0);
+  p1 = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(p1);
+  p2 = __float2bfloat16_rn(r2);
+}
+
 // Host-side count of kernels this library has enqueued since it was loaded.
 inline std::atomic<unsigned long long> g_launch_count{0};
 inline void count_launch() { g_launch_count.fetch_add(1, std::memory_order_relaxed); }

@@ -19,6 +19,8 @@
 // the output index), and a per-row sign for the orthogonal direction.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace quip {
@@ -234,19 +236,50 @@ __global__ void __launch_bounds__(32 * ((1 << LOGG) / 16))
 
 __device__ __forceinline__ int pad16(int k) { return k + (k >> 4); }
 
+// Row sources and sinks of the two one-row-per-CTA kernels below.  A source
+// is fp32, bf16, or b-bit codes (uint8) dequantised on the way in as
+// lo[row] + s[row] * code (the product and sum of the dequantisation kernel,
+// one fused multiply-add).  The sink is fp32 (out, row stride ldout) or,
+// with PIECES, the three bf16 pieces of every output value (outp, row stride
+// ldout, piece stride pst; split3), the split the Kronecker kernel's inputs
+// take.
+struct RowDequant {
+  const float* lo;
+  const float* s;
+};
+
+__device__ __forceinline__ void load16(const uint8_t* p, float (&v)[16]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) v[4 * k + b] = (float)((w[k] >> (8 * b)) & 0xffu);
+}
+
+template <typename TIn, int N>
+__device__ __forceinline__ void dequant_in(const RowDequant& dq, int64_t row, float (&v)[N]) {
+  if constexpr (std::is_same<TIn, uint8_t>::value) {
+    const float l = dq.lo[row], sc = dq.s[row];
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = fmaf(sc, v[i], l);
+  }
+}
+
 // One row of 4096 per CTA (256 threads).  Thread t: stage A on elements
 // 16 t + j (16-byte loads), stage B on 256 (t / 16) + 16 j + t % 16, stage C
 // on 256 j + t, stored straight from registers (coalesced across threads).
-template <typename TIn>
+template <typename TIn, bool PIECES>
 __global__ void __launch_bounds__(256)
-    k_fwht_row4096(const TIn* __restrict__ in, int64_t ldin, float* out, int64_t ldout,
-                   const float* __restrict__ pre, const float* __restrict__ post,
-                   const float* __restrict__ row_sign, float scale) {
+    k_fwht_row4096(const TIn* __restrict__ in, int64_t ldin, RowDequant dq, float* out,
+                   __nv_bfloat16* outp, int64_t ldout, int64_t pst, const float* __restrict__ pre,
+                   const float* __restrict__ post, const float* __restrict__ row_sign, float scale) {
   __shared__ float sr[4096 + 256];
   const int t = threadIdx.x;
   const int64_t row = blockIdx.x;
   float v[16];
   load16(in + row * ldin + 16 * t, v);
+  dequant_in<TIn>(dq, row, v);
   if (pre) {
     const float4* pp = reinterpret_cast<const float4*>(pre + 16 * t);
 #pragma unroll
@@ -270,11 +303,16 @@ __global__ void __launch_bounds__(256)
   for (int j = 0; j < 16; ++j) v[j] = sr[pad16(256 * j + t)];
   reg_fwht<4>(v);
   const float rs = row_sign ? row_sign[row] * scale : scale;
-  float* o = out + row * ldout;
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const int k = 256 * j + t;
-    o[k] = v[j] * rs * (post ? post[k] : 1.f);
+    const float y = v[j] * rs * (post ? post[k] : 1.f);
+    if constexpr (PIECES) {
+      __nv_bfloat16* o = outp + row * ldout + k;
+      split3(y, o[0], o[pst], o[2 * pst]);
+    } else {
+      out[row * ldout + k] = y;
+    }
   }
 }
 
@@ -309,20 +347,35 @@ __device__ __forceinline__ void load32(const __nv_bfloat16* p, float (&v)[32]) {
   }
 }
 
+__device__ __forceinline__ void load32(const uint8_t* p, float (&v)[32]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint4 u = q[i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) v[16 * i + 4 * k + b] = (float)((w[k] >> (8 * b)) & 0xffu);
+  }
+}
+
 // One row of 8192 per CTA (256 threads).  Thread t (warp w, lane l): stage A
 // on elements 32 t + r (r = bits 0-4); stage B on l + 32 r + 1024 w (bits
-// 5-9); stage C on t % 256 + 256 g + 1024 r (g < 4, r < 8: bits 10-12),
-// stored straight from registers, 32 consecutive floats per warp store.
-template <typename TIn>
-__global__ void __launch_bounds__(256)
-    k_fwht_row8192(const TIn* __restrict__ in, int64_t ldin, float* out, int64_t ldout,
-                   const float* __restrict__ pre, const float* __restrict__ post,
-                   const float* __restrict__ row_sign, float scale) {
+// 5-9); stage C on 4 t + j + 1024 r (j < 4, r < 8: bits 10-12), read from
+// shared memory and stored four consecutive values at a time (16-byte
+// accesses; a warp's store covers 512 contiguous bytes).
+template <typename TIn, bool PIECES>
+__global__ void __launch_bounds__(256, 4)
+    k_fwht_row8192(const TIn* __restrict__ in, int64_t ldin, RowDequant dq, float* out,
+                   __nv_bfloat16* outp, int64_t ldout, int64_t pst, const float* __restrict__ pre,
+                   const float* __restrict__ post, const float* __restrict__ row_sign, float scale) {
   __shared__ __align__(16) float sr[8192 + 1024];
   const int t = threadIdx.x, w = t >> 5, l = t & 31;
   const int64_t row = blockIdx.x;
   float v[32];
   load32(in + row * ldin + 32 * t, v);
+  dequant_in<TIn>(dq, row, v);
   if (pre) {
     const float4* pp = reinterpret_cast<const float4*>(pre + 32 * t);
 #pragma unroll
@@ -342,31 +395,50 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
   for (int r = 0; r < 32; ++r) sr[pad32x4(l + 32 * r + 1024 * w)] = v[r];
   __syncthreads();
-  // stage C: four groups g of eight values each (register index 8 g + r)
+  // stage C: register index 4 r + j holds element 4 t + j + 1024 r
 #pragma unroll
-  for (int g = 0; g < 4; ++g)
-#pragma unroll
-    for (int r = 0; r < 8; ++r) v[8 * g + r] = sr[pad32x4(t + 256 * g + 1024 * r)];
+  for (int r = 0; r < 8; ++r) {
+    const float4 f = *reinterpret_cast<const float4*>(sr + pad32x4(4 * t + 1024 * r));
+    v[4 * r] = f.x, v[4 * r + 1] = f.y, v[4 * r + 2] = f.z, v[4 * r + 3] = f.w;
+  }
 #pragma unroll
   for (int h = 1; h < 8; h <<= 1) {
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      if ((e & h) == 0) {
-        const float a = v[e], b = v[e + h];
-        v[e] = a + b;
-        v[e + h] = a - b;
+    for (int r = 0; r < 8; ++r) {
+      if ((r & h) == 0) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float a = v[4 * r + j], b = v[4 * (r + h) + j];
+          v[4 * r + j] = a + b;
+          v[4 * (r + h) + j] = a - b;
+        }
       }
     }
   }
   const float rs = row_sign ? row_sign[row] * scale : scale;
-  float* o = out + row * ldout;
 #pragma unroll
-  for (int g = 0; g < 4; ++g)
+  for (int r = 0; r < 8; ++r) {
+    const int k = 4 * t + 1024 * r;
+    float y[4];
+    if (post) {
+      const float4 f = *reinterpret_cast<const float4*>(post + k);
+      y[0] = v[4 * r] * rs * f.x, y[1] = v[4 * r + 1] * rs * f.y;
+      y[2] = v[4 * r + 2] * rs * f.z, y[3] = v[4 * r + 3] * rs * f.w;
+    } else {
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int k = t + 256 * g + 1024 * r;
-      o[k] = v[8 * g + r] * rs * (post ? post[k] : 1.f);
+      for (int j = 0; j < 4; ++j) y[j] = v[4 * r + j] * rs;
     }
+    if constexpr (PIECES) {
+      __nv_bfloat16 pc[3][4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) split3(y[j], pc[0][j], pc[1][j], pc[2][j]);
+      __nv_bfloat16* o = outp + row * ldout + k;
+#pragma unroll
+      for (int f = 0; f < 3; ++f) *reinterpret_cast<uint2*>(o + f * pst) = *reinterpret_cast<const uint2*>(pc[f]);
+    } else {
+      *reinterpret_cast<float4*>(out + row * ldout + k) = make_float4(y[0], y[1], y[2], y[3]);
+    }
+  }
 }
 
 // 4096-point column transform of 8 columns per CTA (1024 threads), in place.

@@ -283,15 +283,6 @@ __global__ void __launch_bounds__(256, 1)
 // fp32 -> three bf16 pieces, row-major copy: out[p][i][k] for p = 0..2.
 // Rows `rows`, K `cols` of the source (row stride lds); output row stride
 // ldo, piece stride piece_elems.
-__device__ __forceinline__ void split3(float x, __nv_bfloat16& p0, __nv_bfloat16& p1,
-                                       __nv_bfloat16& p2) {
-  p0 = __float2bfloat16_rn(x);
-  const float r1 = x - __bfloat162float(p0);
-  p1 = __float2bfloat16_rn(r1);
-  const float r2 = r1 - __bfloat162float(p1);
-  p2 = __float2bfloat16_rn(r2);
-}
-
 // out[p][j][i] = piece_p(U[i][j]) for i < j (strict upper), 0 otherwise:
 // the transposed, split copy of the LDL factor that LDLQ's trailing GEMM
 // reads as its K-major B operand; outf[j][i] = U[i][j] (same zeros), the

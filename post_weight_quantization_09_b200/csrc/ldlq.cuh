@@ -73,30 +73,30 @@ __device__ __forceinline__ void nb_arrive(int id, int count) {
 }
 
 // Block step over the w columns [k0, k0 + w) (w = 128, or 64 for a last,
-// partial block) for 32 rows per CTA, on the FP32 pipes: warp 0 rounds
-// (lane r = row r), warps 1-3 apply the feedback that can wait.  Global
+// partial block) for 32 rows per sub-group, on the FP32 pipes: one warp
+// rounds (lane r = row r), the other three apply the feedback that can wait.  Global
 // memory is touched only by the copies in and the stores out: TMA brings
 // the rows' W~ and accumulated values of the block (wt, acc; row r at stride LQB_S:
 // 16-byte accesses of a warp are conflict-free), the transposed Ů block
 // (UT[j][k] = Ů[k0 + k][k0 + j], zero for k >= j) and the band of Ů next to
 // the diagonal (band[k][jj] = Ů[k0 + k][k0 + 16 (k / 16) + jj], as eight
 // 16 x 32 boxes; entries with j <= k or j >= w are zeroed after the copy).
-// Columns are taken in groups of 16.  For group g, warp 0
+// Columns are taken in groups of 16.  For group g, the rounding warp
 //   1. waits until the helpers have applied group g - 2's feedback, then
 //      takes cur = the group's accumulated values + carry (the previous
 //      group's feedback, in registers);
 //   2. rounds column by column, feeding each error to the group's later
-//      columns, then forms the group's feedback to the next group (carry);
+//      columns and into the group's feedback to the next group (carry);
 //   3. hands the 16 errors and codes to the helpers (shared slot g % 2).
 // The helpers stage the codes and the errors' three bf16 pieces (the
 // trailing GEMMs' A operand; written out with coalesced stores after the
 // last group) and add group g's feedback to the columns from
 // two groups on, acc[r][j] += sum_t e_t Ů[16 g + t][j] (each thread: four
 // rows and every twelfth 4-column chunk, so one broadcast 16-byte load of a
-// UT row serves 16 fmas), while warp 0 rounds group g + 1.  Named barriers
-// pass the hand-off
-// slots: READY + slot (warp 0 -> helpers, every group) and DONE + slot
-// (helpers -> warp 0, only for groups that warp 0 will wait on).
+// UT row serves 16 fmas), while the rounding warp takes group g + 1.  Named
+// barriers pass the hand-off slots: READY + slot (rounding warp -> helpers,
+// every group) and DONE + slot (helpers -> rounding warp, only for groups
+// it will wait on).
 // Rounding: clamp to [0, qmax] first, then add and subtract 1.5 * 2^23,
 // which rounds half to even exactly like rintf on that range (and leaves
 // the integer, the code, in the low mantissa bits).
@@ -104,7 +104,7 @@ __device__ __forceinline__ void nb_arrive(int id, int count) {
 // the transposed factor (n x n fp32, LQB_S x 128 boxes), tmU over the
 // factor Ů (the LDL's output, row stride ldu; 32 x 16 boxes).
 constexpr int LQB_ROWS = 32;                           // rows per sub-group
-constexpr int LQB_THREADS = 128;                       // per sub-group: warp 0 rounds, warps 1-3 help
+constexpr int LQB_THREADS = 128;                       // per sub-group: one warp rounds, three help
 constexpr int LQB_S = 132;                             // smem row stride of acc and UT
 constexpr int LQB_ES = 20;                             // smem row stride of the slots: 16 errors, 4 code words
 constexpr int LQB_ACC = LQB_ROWS * LQB_S * 4;          // bytes of the acc tile
@@ -146,6 +146,10 @@ __global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
   __shared__ __align__(8) uint64_t bar;
   __shared__ int ok_s;
   const int tid = threadIdx.x, sg = tid / LQB_THREADS, warp = (tid % LQB_THREADS) >> 5, r = tid & 31;
+  // the rounding warp of sub-group sg is its warp sg % 4: CTA warp 4 sg + sg,
+  // so the rounding warps sit on different SM sub-partitions (warp % 4) and
+  // do not share an issue slot
+  const int rw = sg & 3;
   const int srow = sg * LQB_ROWS + r;                  // this thread's row within the CTA
   const int64_t row = (int64_t)blockIdx.x * CROWS + srow;
   const bool valid = row < m;
@@ -190,12 +194,12 @@ __global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
   __syncthreads();
   const int ngroups = w / 16;
 
-  if (warp > 0) {
+  if (warp != rw) {
     // ------------------------------------------------------------ helpers
     // thread (h, lane): rows lane % 8 + 8 i (i < 4) and the 4-column chunks
     // c with c % 12 == 4 h + lane / 8 (every Ů^T load serves four rows);
     // helper warp 0 also stores row `lane`'s codes and error pieces.
-    const int h = warp - 1, rb = r & 7, cls = 4 * h + (r >> 3);
+    const int h = warp < rw ? warp : warp - 1, rb = r & 7, cls = 4 * h + (r >> 3);
 #pragma unroll 1
     for (int g = 0; g < ngroups; ++g) {
       const int slot = g & 1;
@@ -267,7 +271,7 @@ __global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
     }
   } else {
 
-  // ------------------------------------------------------------ warp 0: rounding
+  // ------------------------------------------------------------ the rounding warp
   const float l = valid ? lo[row] : 0.f;
   const float s = valid ? sc[row] : 1.f;
   const float inv = 1.0f / s;
@@ -296,6 +300,11 @@ __global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
       cur[4 * q + 2] = a.z + carry[4 * q + 2];
       cur[4 * q + 3] = a.w + carry[4 * q + 3];
     }
+    // carry now collects this group's feedback to the next group, one column
+    // at a time as the errors appear (the terms of every element summed in
+    // column order), in the issue slots the rounding chain leaves free
+#pragma unroll
+    for (int j = 0; j < 16; ++j) carry[j] = 0.f;
     float wn[16];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -328,6 +337,14 @@ __global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
       const float err = wv[t] - fmaf(s, cq, l);
       e[t] = err;
       if (t < 15) cur[t + 1] = fmaf(err, sd[t], cur[t + 1]);
+#pragma unroll
+      for (int q4 = 0; q4 < 16; q4 += 4) {
+        const float4 u = *reinterpret_cast<const float4*>(ur + 16 + q4);
+        carry[q4 + 0] = fmaf(err, u.x, carry[q4 + 0]);
+        carry[q4 + 1] = fmaf(err, u.y, carry[q4 + 1]);
+        carry[q4 + 2] = fmaf(err, u.z, carry[q4 + 2]);
+        carry[q4 + 3] = fmaf(err, u.w, carry[q4 + 3]);
+      }
       cw[t >> 2] |= (__float_as_uint(zr) & 0xffu) << (8 * (t & 3));
       // column t - 1's error into columns t + 1 ..
 #pragma unroll
@@ -336,22 +353,6 @@ __global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
       eprev = err;
 #pragma unroll
       for (int j = t + 2; j < 16; ++j) bprev[j] = bcur[j];
-    }
-    // the group's feedback to the next group (off the rounding chain; every
-    // carry element sums its terms in column order, as the chain would)
-#pragma unroll
-    for (int j = 0; j < 16; ++j) carry[j] = 0.f;
-#pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      const float* ur = band + (16 * g + t) * 32 + 16;
-#pragma unroll
-      for (int q4 = 0; q4 < 16; q4 += 4) {
-        const float4 u = *reinterpret_cast<const float4*>(ur + q4);
-        carry[q4 + 0] = fmaf(e[t], u.x, carry[q4 + 0]);
-        carry[q4 + 1] = fmaf(e[t], u.y, carry[q4 + 1]);
-        carry[q4 + 2] = fmaf(e[t], u.z, carry[q4 + 2]);
-        carry[q4 + 3] = fmaf(e[t], u.w, carry[q4 + 3]);
-      }
     }
     // hand the errors and codes to the helpers
     float* es = eslot + (slot * LQB_ROWS + r) * LQB_ES;

@@ -260,14 +260,14 @@ cudaError_t fwht_rows(const TIn* in, int64_t ldin, float* out, int64_t ldout, in
   }
   if (L == 12) {
     LaunchScope ls("k_fwht_rows", st);
-    k_fwht_row4096<TIn><<<(unsigned)rows, 256, 0, st>>>(in, ldin, out, ldout, pre, post, row_sign,
-                                                         scale);
+    k_fwht_row4096<TIn, false><<<(unsigned)rows, 256, 0, st>>>(in, ldin, RowDequant{}, out, nullptr, ldout, 0,
+                                                                pre, post, row_sign, scale);
     return cudaGetLastError();
   }
   if (L == 13) {
     LaunchScope ls("k_fwht_rows", st);
-    k_fwht_row8192<TIn><<<(unsigned)rows, 256, 0, st>>>(in, ldin, out, ldout, pre, post, row_sign,
-                                                         scale);
+    k_fwht_row8192<TIn, false><<<(unsigned)rows, 256, 0, st>>>(in, ldin, RowDequant{}, out, nullptr, ldout, 0,
+                                                                pre, post, row_sign, scale);
     return cudaGetLastError();
   }
   const int T = (int)(d / 16);
@@ -476,28 +476,14 @@ size_t kron_cols_tc_bytes(int64_t R, int64_t c) { return 2 * round256((size_t)3 
 // A' = A, B' = B (forward) or A^T, B^T (inverse).  src: bf16 (one piece) or
 // fp32 (split into three pieces first), row stride ld.  dst may alias an
 // fp32 src.  ws: kron_cols_tc_bytes(R, c).
-template <typename TIn>
-cudaError_t kron_cols_tc(const SideData& sd, bool transpose, const TIn* src, int64_t ld, float* dst,
-                         int64_t c, void* ws, cudaStream_t st) {
+// The two products of kron_cols_tc from data already in xp bf16 pieces
+// (xp = 1: bf16 data; xp = 3: the three pieces of fp32 data), piece f of row
+// r at xsrc + (f R + r) xld.  Stage 1 writes its pieces to the second half
+// of ws, so xsrc may be the first half.
+cudaError_t kron_cols_tc_x(const SideData& sd, bool transpose, const __nv_bfloat16* xsrc, int xp, int64_t xld,
+                           float* dst, int64_t c, void* ws, cudaStream_t st) {
   const int64_t p = sd.p, q = sd.q, R = p * q;
-  __nv_bfloat16* P1 = static_cast<__nv_bfloat16*>(ws);
   __nv_bfloat16* P2 = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + round256((size_t)3 * R * c * 2));
-  const __nv_bfloat16* xsrc;
-  int xp;
-  int64_t xld;
-  if constexpr (std::is_same<TIn, __nv_bfloat16>::value) {
-    xsrc = src, xp = 1, xld = ld;
-  } else {
-    const int64_t total4 = R * c / 4;
-    const unsigned g = (unsigned)std::min<int64_t>((total4 + 255) / 256, 148 * 16);
-    {
-      LaunchScope ls("k_split_rows3", st);
-      k_split_rows3<<<g, 256, 0, st>>>(src, ld, R, c, P1);
-    }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    xsrc = P1, xp = 3, xld = c;
-  }
   // stage 1: T_a' = B' X_a' for the p slabs of q rows, into P2 as pieces
   CUtensorMap mf, mx;
   const int nfq = (int)((q + 15) / 16 * 16), nfp = (int)((p + 15) / 16 * 16);
@@ -521,6 +507,26 @@ cudaError_t kron_cols_tc(const SideData& sd, bool transpose, const TIn* src, int
   k2.f_piece_rows = (int)p, k2.x_pieces = 3, k2.x_piece_rows = p, k2.x_slab_rows = 0;
   k2.Y = dst, k2.ldy = q * c, k2.y_slab_rows = 0;
   return kron_tc_launch(mf, mx, k2, kron::OUT_F32, st);
+}
+
+template <typename TIn>
+cudaError_t kron_cols_tc(const SideData& sd, bool transpose, const TIn* src, int64_t ld, float* dst,
+                         int64_t c, void* ws, cudaStream_t st) {
+  if constexpr (std::is_same<TIn, __nv_bfloat16>::value) {
+    return kron_cols_tc_x(sd, transpose, src, 1, ld, dst, c, ws, st);
+  } else {
+    const int64_t R = sd.p * sd.q;
+    __nv_bfloat16* P1 = static_cast<__nv_bfloat16*>(ws);
+    const int64_t total4 = R * c / 4;
+    const unsigned g = (unsigned)std::min<int64_t>((total4 + 255) / 256, 148 * 16);
+    {
+      LaunchScope ls("k_split_rows3", st);
+      k_split_rows3<<<g, 256, 0, st>>>(src, ld, R, c, P1);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return kron_cols_tc_x(sd, transpose, P1, 3, c, dst, c, ws, st);
+  }
 }
 
 __global__ void k_convert_rows_bf16(const __nv_bfloat16* in, int64_t ld, float* out, int64_t m,
@@ -1022,11 +1028,13 @@ quip_status quip_incoherence_forward(const quip_transform* tf, const void* W, in
   if (W) {
     if (w_dtype != QUIP_F32 && w_dtype != QUIP_BF16) return QUIP_ERR_ARG;
     if (ldw < n) return QUIP_ERR_SHAPE;
-    if (V.kind == QUIP_T_HADAMARD && n >= 16) {   // vector loads in the row kernel
+    if (V.kind == QUIP_T_HADAMARD && n >= 16) {   // vector loads and stores in the row kernels
       const size_t esz = w_dtype == QUIP_BF16 ? 2 : 4;
-      if ((reinterpret_cast<uintptr_t>(W) % 16) || ((ldw * esz) % 16)) return QUIP_ERR_ARG;
+      if ((reinterpret_cast<uintptr_t>(W) % 16) || ((ldw * esz) % 16) || (reinterpret_cast<uintptr_t>(W_t) % 16))
+        return QUIP_ERR_ARG;
     }
   }
+  if (H && V.kind == QUIP_T_HADAMARD && n >= 16 && (reinterpret_cast<uintptr_t>(H) % 16)) return QUIP_ERR_ARG;
   size_t need = 0;
   quip_status s = quip_workspace_size(QUIP_OP_INCOHERENCE_FORWARD, tf, m, n, 0, &need);
   if (s != QUIP_OK) return s;
@@ -1082,6 +1090,9 @@ quip_status quip_incoherence_inverse(const quip_transform* tf, const float* W_ha
                                      void* ws, size_t ws_bytes, void* stream) {
   if (!tf || !W_hat_t || !W_hat) return QUIP_ERR_ARG;
   const int64_t m = tf->m, n = tf->n;
+  if (tf->side[1].kind == QUIP_T_HADAMARD && n >= 16 &&
+      ((reinterpret_cast<uintptr_t>(W_hat_t) % 16) || (reinterpret_cast<uintptr_t>(W_hat) % 16)))
+    return QUIP_ERR_ARG;                               // vector loads and stores in the row kernels
   size_t need = 0;
   quip_status s = quip_workspace_size(QUIP_OP_INCOHERENCE_INVERSE, tf, m, n, 0, &need);
   if (s != QUIP_OK) return s;
@@ -1859,6 +1870,58 @@ quip_status layer_args(const quip_transform* tf, int w_dtype, int64_t ldw, int x
 
 // Token chunks of X in the host variant: X's copy lands in up to four
 // pieces, each accumulated into H as soon as it is on the device.
+// W_hat = U^T (lo + s . codes) V, the layer call's last step.  With an
+// n-side Hadamard of 4096 or 8192 points the dequantisation is folded into
+// the row kernel (it reads the codes), and with a tensor-core Kronecker m
+// side the row kernel writes the three bf16 pieces that the Kronecker
+// products read: no fp32 W~^ and no separate split pass in between.  The
+// arithmetic is that of quip_dequantize followed by quip_incoherence_inverse
+// (the same fused multiply-add per code, the same butterflies, the same
+// split), so W_hat is the same to the bit.  Other transforms take those two
+// calls.  ws: QUIP_OP_INCOHERENCE_INVERSE.
+quip_status inverse_from_codes(const quip_transform* tf, const uint8_t* codes, const float* lo,
+                               const float* scale, float* W_hat, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const int64_t m = tf->m, n = tf->n;
+  const SideData &U = tf->side[0], &V = tf->side[1];
+  const int L = n > 0 ? ilog2(n) : 0;
+  const bool fused = V.kind == QUIP_T_HADAMARD && !V.permute && !U.permute && (L == 12 || L == 13) &&
+                     (int64_t(1) << L) == n && (reinterpret_cast<uintptr_t>(codes) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(W_hat) & 15) == 0;
+  if (!fused) {
+    quip_status r = quip_dequantize(codes, lo, scale, m, n, W_hat, st);
+    if (r != QUIP_OK) return r;
+    return quip_incoherence_inverse(tf, W_hat, W_hat, ws, ws_bytes, st);
+  }
+  size_t need = 0;
+  quip_status s = quip_workspace_size(QUIP_OP_INCOHERENCE_INVERSE, tf, m, n, 0, &need);
+  if (s != QUIP_OK) return s;
+  if ((s = check_ws(ws, ws_bytes, need)) != QUIP_OK) return s;
+  const float sc = (float)(1.0 / std::sqrt((double)n));
+  const RowDequant dq{lo, scale};
+  const bool tc = kron_cols_tc_ok(U, n);
+  __nv_bfloat16* P1 = static_cast<__nv_bfloat16*>(ws);
+  const int64_t pst = m * n;
+  {
+    LaunchScope ls("k_fwht_rows", st);
+    if (L == 13 && tc)
+      k_fwht_row8192<uint8_t, true><<<(unsigned)m, 256, 0, st>>>(codes, n, dq, nullptr, P1, n, pst, nullptr,
+                                                                V.signs, nullptr, sc);
+    else if (L == 13)
+      k_fwht_row8192<uint8_t, false><<<(unsigned)m, 256, 0, st>>>(codes, n, dq, W_hat, nullptr, n, 0, nullptr,
+                                                                 V.signs, nullptr, sc);
+    else if (tc)
+      k_fwht_row4096<uint8_t, true><<<(unsigned)m, 256, 0, st>>>(codes, n, dq, nullptr, P1, n, pst, nullptr,
+                                                                V.signs, nullptr, sc);
+    else
+      k_fwht_row4096<uint8_t, false><<<(unsigned)m, 256, 0, st>>>(codes, n, dq, W_hat, nullptr, n, 0, nullptr,
+                                                                 V.signs, nullptr, sc);
+  }
+  QCHECK(cudaGetLastError());
+  if (tc) QCHECK(kron_cols_tc_x(U, true, P1, 3, n, W_hat, n, ws, st));
+  else QCHECK(side_cols(U, true, W_hat, n, static_cast<float*>(ws), st));
+  return QUIP_OK;
+}
+
 int64_t layer_x_chunk(int64_t N) {
   const int64_t c = (N + 3) / 4;
   return std::max<int64_t>(2048, (c + 2047) / 2048 * 2048);
@@ -1924,8 +1987,7 @@ quip_status layer_device(quip_transform* tf, uint64_t seed, const void* W, int w
       return r;
     if (q_done) QCHECK(cudaEventRecord(q_done, st));
     if (W_hat) {
-      if ((r = quip_dequantize(codes, lo, scale, m, n, W_hat, st)) != QUIP_OK) return r;
-      if ((r = quip_incoherence_inverse(tf, W_hat, W_hat, sw, L.stage, st)) != QUIP_OK) return r;
+      if ((r = inverse_from_codes(tf, codes, lo, scale, W_hat, sw, L.stage, st)) != QUIP_OK) return r;
     }
     return QUIP_OK;
   };

@@ -425,6 +425,35 @@ def test_layer_call_equals_the_stages_and_the_oracle():
         np.testing.assert_allclose(wh.numpy(), host(r.W_hat), atol=1e-4 * s.max())
 
 
+@pytest.mark.parametrize("n,mk", [
+    (8192, Side("kronecker", 8, 128)), (8192, Side("hadamard")),
+    (4096, Side("kronecker", 8, 128)), (4096, Side("identity")),
+])
+def test_layer_inverse_reads_the_codes(n, mk):
+    """In the layer call the n-side Hadamard row kernel (4096 or 8192 points)
+    reads the codes, the dequantisation folded in, and for a tensor-core
+    Kronecker m side writes the bf16 pieces the Kronecker products take.  W^
+    is the stage calls' quip_dequantize + quip_incoherence_inverse of the same
+    codes to the bit, and the oracle's U^T W~^ V of those codes within 1e-4 of
+    the row scale on sampled rows."""
+    m, N, bits, block, seed = 1024, 256, 2, 128, 21
+    nk = Side("hadamard")
+    d = random_layer(m, n, N, seed=31, dtype="bf16")
+    q = Q.LayerQuantizer(m, n, mk, nk, bits, block, 0.01, seed)
+    r = q.run(dev(d["W"], torch.bfloat16), dev(d["X"], torch.bfloat16))
+    assert Q.quip_sync_status() == L.QUIP_OK
+    Wh = torch.empty_like(r.W_hat)
+    Q.quip_dequantize(r.codes, r.lo, r.scale, Wh)
+    Q.quip_incoherence_inverse(q.tf, Wh, Wh, q.ws)
+    assert torch.equal(r.W_hat, Wh)
+    C, lo, s = host(r.codes), host(r.lo), host(r.scale)
+    U = O.make_side(seed, "m", mk.kind, m, mk.p, mk.q)
+    V = O.make_side(seed, "n", nk.kind, n)
+    rows = np.random.default_rng(3).choice(m, 12, replace=False)
+    ref = O.incoherence_inverse_rows(O.dequantize(C, lo, s), U, V, rows)
+    assert np.abs(host(r.W_hat)[rows] - ref).max() <= 1e-4 * s.max()
+
+
 @pytest.mark.parametrize("mk,nk", [
     (Side("hadamard", permute=True), Side("hadamard", permute=True)),
     (Side("kronecker", 8, 8, True), Side("hadamard", permute=True)),
