@@ -409,7 +409,8 @@ quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int
  * each step has the arguments, layout and errors of its own entry point.
  * The Hessian path (V, H, H~, the LDL) runs on a library-owned stream of the
  * highest priority, forked from and joined into `stream`; the weight path
- * (U, W~) runs on `stream` beside it; LDLQ and W^ follow on `stream`.  The codes and grid are those of LDLQ in the
+ * (U, W~, LDLQ's per-row grid and the start of its accumulator) runs on
+ * `stream` beside it; the rest of LDLQ and W^ follow on `stream`.  The codes and grid are those of LDLQ in the
  * incoherent basis (quip_ldlq_quantize); W^ is the dequantised layer in the
  * original basis.
  *   tf       : a transform made for this layer's m x n (quip_transform_create);
@@ -457,8 +458,10 @@ quip_status quip_quantize_layer_host(quip_transform* tf, uint64_t seed, const vo
 /*
  * Device workspace of quip_quantize_layer (host = 0) or
  * quip_quantize_layer_host (host = 1) for N tokens and the given types:
- * H~ (n x n fp32), D, W~ (m x n fp32) and the largest stage workspace; the
- * host variant adds device copies of W and X, the codes, the grid and W^.
+ * H~ (n x n fp32), D, W~ (m x n fp32), the largest stage workspace and the
+ * weight path's own region (its transform's workspace, then LDLQ's m x n
+ * fp32 accumulator); the host variant adds device copies of W and X, the
+ * codes, the grid and W^.
  */
 quip_status quip_layer_workspace_size(const quip_transform* tf, int64_t N, int w_dtype, int x_dtype,
                                       int64_t block, int host, size_t* bytes);
@@ -479,6 +482,19 @@ quip_status quip_layer_workspace_size(const quip_transform* tf, int64_t N, int w
 quip_status quip_timing_begin(void);
 quip_status quip_timing_end(const char** names, uint64_t* launches, double* total_ms,
                             int max_entries, int* n_entries);
+
+/*
+ * The launches recorded since quip_timing_begin() one by one, in the order
+ * they were enqueued (instead of quip_timing_end's aggregates; either call
+ * ends the recording and discards the records): names[i], start_ms[i] and
+ * end_ms[i] (the launch's two events, in ms after the first launch's start
+ * event) and stream_ids[i] (streams numbered in order of first appearance),
+ * for i < min(max_entries, *n_entries); *n_entries receives the number of
+ * launches recorded.  A timeline of the streams' overlap; the events between
+ * launches break programmatic dependent launch, so the gaps are upper bounds.
+ */
+quip_status quip_timing_trace(const char** names, double* start_ms, double* end_ms, int* stream_ids,
+                              int max_entries, int* n_entries);
 
 /*
  * Synchronise `stream`, then return and clear the device status word

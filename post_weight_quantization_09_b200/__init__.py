@@ -24,7 +24,7 @@ __all__ = [
     "quip_nearest_quantize", "quip_diag_order", "quip_permute", "quip_greedy_refine", "METHODS",
     "quip_packed_words", "quip_pack_codes", "quip_qmatvec", "QuantizedLinear",
     "quip_workspace_size", "quip_layer_workspace_size", "quip_quantize_layer", "quip_quantize_layer_host",
-    "layer_views", "quip_sync_status", "quip_timing_begin", "quip_timing_end", "LayerQuantizer",
+    "layer_views", "quip_sync_status", "quip_timing_begin", "quip_timing_end", "quip_timing_trace", "LayerQuantizer",
     "LayerGroupQuantizer", "quantize_layer", "QuipError",
     "KIND",
 ]
@@ -377,6 +377,19 @@ def quip_timing_end(max_entries: int = 64) -> dict:
     n = ctypes.c_int(0)
     L.check(lib.quip_timing_end(names, counts, ms, max_entries, ctypes.byref(n)), "quip_timing_end")
     return {names[i].decode(): (int(counts[i]), float(ms[i])) for i in range(min(n.value, max_entries))}
+
+
+def quip_timing_trace(max_entries: int = 8192) -> list:
+    """[(kernel name, start ms, end ms, stream id)] of the launches since
+    quip_timing_begin(), in enqueue order, times after the first launch's start."""
+    lib = load()
+    names = (ctypes.c_char_p * max_entries)()
+    t0 = (ctypes.c_double * max_entries)()
+    t1 = (ctypes.c_double * max_entries)()
+    sid = (ctypes.c_int * max_entries)()
+    n = ctypes.c_int(0)
+    L.check(lib.quip_timing_trace(names, t0, t1, sid, max_entries, ctypes.byref(n)), "quip_timing_trace")
+    return [(names[i].decode(), float(t0[i]), float(t1[i]), int(sid[i])) for i in range(min(n.value, max_entries))]
 
 
 @dataclass

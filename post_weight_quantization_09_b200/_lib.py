@@ -65,6 +65,8 @@ SIGNATURES = {
     "quip_timing_begin": (c_int, []),
     "quip_timing_end": (c_int, [POINTER(c_char_p), POINTER(c_uint64), POINTER(ctypes.c_double), c_int,
                                 POINTER(c_int)]),
+    "quip_timing_trace": (c_int, [POINTER(c_char_p), POINTER(ctypes.c_double), POINTER(ctypes.c_double),
+                                  POINTER(c_int), c_int, POINTER(c_int)]),
 }
 
 _lib = None

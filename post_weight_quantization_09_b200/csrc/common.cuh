@@ -46,6 +46,7 @@ inline void count_launch() { g_launch_count.fetch_add(1, std::memory_order_relax
 struct TimingRec {
   const char* name;
   cudaEvent_t a, b;
+  cudaStream_t st;
 };
 inline std::atomic<bool> g_timing_on{false};
 inline std::mutex g_timing_mu;
@@ -70,7 +71,7 @@ struct LaunchScope {
       g_timing_pool.push_back(ev);
       return;
     }
-    g_timing_recs.push_back({name, ev.first, ev.second});
+    g_timing_recs.push_back({name, ev.first, ev.second, st});
     b = ev.second;
   }
   ~LaunchScope() {

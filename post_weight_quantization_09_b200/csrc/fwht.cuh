@@ -239,14 +239,53 @@ __device__ __forceinline__ int pad16(int k) { return k + (k >> 4); }
 // Row sources and sinks of the two one-row-per-CTA kernels below.  A source
 // is fp32, bf16, or b-bit codes (uint8) dequantised on the way in as
 // lo[row] + s[row] * code (the product and sum of the dequantisation kernel,
-// one fused multiply-add).  The sink is fp32 (out, row stride ldout) or,
-// with PIECES, the three bf16 pieces of every output value (outp, row stride
-// ldout, piece stride pst; split3), the split the Kronecker kernel's inputs
-// take.
+// one fused multiply-add).  The sink (row stride ld) is
+//   ROW_F32     fp32 values y into out;
+//   ROW_PIECES  the three bf16 pieces of every y (split3) into outp, piece
+//               stride pst: the split the Kronecker kernel's inputs take;
+//   ROW_GRID    y into out and out2 (W~ and the start of LDLQ's
+//               accumulator), and the row's b-bit min / max grid lo[row] =
+//               min y, sc[row] = (max y - min y) / qmax (1 for a constant
+//               row), with QUIP_ERR_NONFINITE recorded for a non-finite y:
+//               the values of the row-grid kernel, taken while the row is
+//               still in registers.
 struct RowDequant {
   const float* lo;
   const float* s;
 };
+enum { ROW_F32 = 0, ROW_PIECES = 1, ROW_GRID = 2 };
+struct RowSink {
+  float* out;
+  float* out2;
+  __nv_bfloat16* outp;
+  int64_t ld, pst;
+  float* lo;
+  float* sc;
+  float qmax;
+};
+
+// Row grid of ROW_GRID from each thread's min / max / finiteness (the whole
+// CTA, NT threads, holds the row).  red: 3 * NT / 32 floats of shared memory.
+template <int NT>
+__device__ __forceinline__ void row_grid_store(float mn, float mx, bool fin, const RowSink& sk, int64_t row,
+                                               float* red) {
+  constexpr int NW = NT / 32;
+  mn = warp_min(mn);
+  mx = warp_max(mx);
+  fin = __all_sync(0xffffffffu, fin);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();                                   // red may alias smem the transform used
+  if (l == 0) red[w] = mn, red[NW + w] = mx, red[2 * NW + w] = fin ? 1.f : 0.f;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float a = red[0], b = red[NW];
+    bool f = red[2 * NW] != 0.f;
+    for (int i = 1; i < NW; ++i) a = fminf(a, red[i]), b = fmaxf(b, red[NW + i]), f = f && red[2 * NW + i] != 0.f;
+    if (!f) record_status(QUIP_ERR_NONFINITE);
+    sk.lo[row] = a;
+    sk.sc[row] = (b > a) ? (b - a) / sk.qmax : 1.0f;
+  }
+}
 
 __device__ __forceinline__ void load16(const uint8_t* p, float (&v)[16]) {
   const uint4 u = *reinterpret_cast<const uint4*>(p);
@@ -269,11 +308,11 @@ __device__ __forceinline__ void dequant_in(const RowDequant& dq, int64_t row, fl
 // One row of 4096 per CTA (256 threads).  Thread t: stage A on elements
 // 16 t + j (16-byte loads), stage B on 256 (t / 16) + 16 j + t % 16, stage C
 // on 256 j + t, stored straight from registers (coalesced across threads).
-template <typename TIn, bool PIECES>
+template <typename TIn, int SINK>
 __global__ void __launch_bounds__(256)
-    k_fwht_row4096(const TIn* __restrict__ in, int64_t ldin, RowDequant dq, float* out,
-                   __nv_bfloat16* outp, int64_t ldout, int64_t pst, const float* __restrict__ pre,
-                   const float* __restrict__ post, const float* __restrict__ row_sign, float scale) {
+    k_fwht_row4096(const TIn* __restrict__ in, int64_t ldin, RowDequant dq, RowSink sk,
+                   const float* __restrict__ pre, const float* __restrict__ post,
+                   const float* __restrict__ row_sign, float scale) {
   __shared__ float sr[4096 + 256];
   const int t = threadIdx.x;
   const int64_t row = blockIdx.x;
@@ -303,17 +342,24 @@ __global__ void __launch_bounds__(256)
   for (int j = 0; j < 16; ++j) v[j] = sr[pad16(256 * j + t)];
   reg_fwht<4>(v);
   const float rs = row_sign ? row_sign[row] * scale : scale;
+  float mn = INFINITY, mx = -INFINITY;
+  bool fin = true;
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const int k = 256 * j + t;
     const float y = v[j] * rs * (post ? post[k] : 1.f);
-    if constexpr (PIECES) {
-      __nv_bfloat16* o = outp + row * ldout + k;
-      split3(y, o[0], o[pst], o[2 * pst]);
+    if constexpr (SINK == ROW_PIECES) {
+      __nv_bfloat16* o = sk.outp + row * sk.ld + k;
+      split3(y, o[0], o[sk.pst], o[2 * sk.pst]);
     } else {
-      out[row * ldout + k] = y;
+      sk.out[row * sk.ld + k] = y;
+    }
+    if constexpr (SINK == ROW_GRID) {
+      sk.out2[row * sk.ld + k] = y;
+      mn = fminf(mn, y), mx = fmaxf(mx, y), fin = fin && isfinite(y);
     }
   }
+  if constexpr (SINK == ROW_GRID) row_grid_store<256>(mn, mx, fin, sk, row, sr);
 }
 
 // ---------------------------------------------------------------- 8192-point rows
@@ -365,11 +411,11 @@ __device__ __forceinline__ void load32(const uint8_t* p, float (&v)[32]) {
 // 5-9); stage C on 4 t + j + 1024 r (j < 4, r < 8: bits 10-12), read from
 // shared memory and stored four consecutive values at a time (16-byte
 // accesses; a warp's store covers 512 contiguous bytes).
-template <typename TIn, bool PIECES>
+template <typename TIn, int SINK>
 __global__ void __launch_bounds__(256, 4)
-    k_fwht_row8192(const TIn* __restrict__ in, int64_t ldin, RowDequant dq, float* out,
-                   __nv_bfloat16* outp, int64_t ldout, int64_t pst, const float* __restrict__ pre,
-                   const float* __restrict__ post, const float* __restrict__ row_sign, float scale) {
+    k_fwht_row8192(const TIn* __restrict__ in, int64_t ldin, RowDequant dq, RowSink sk,
+                   const float* __restrict__ pre, const float* __restrict__ post,
+                   const float* __restrict__ row_sign, float scale) {
   __shared__ __align__(16) float sr[8192 + 1024];
   const int t = threadIdx.x, w = t >> 5, l = t & 31;
   const int64_t row = blockIdx.x;
@@ -416,6 +462,8 @@ __global__ void __launch_bounds__(256, 4)
     }
   }
   const float rs = row_sign ? row_sign[row] * scale : scale;
+  float mn = INFINITY, mx = -INFINITY;
+  bool fin = true;
 #pragma unroll
   for (int r = 0; r < 8; ++r) {
     const int k = 4 * t + 1024 * r;
@@ -428,17 +476,23 @@ __global__ void __launch_bounds__(256, 4)
 #pragma unroll
       for (int j = 0; j < 4; ++j) y[j] = v[4 * r + j] * rs;
     }
-    if constexpr (PIECES) {
+    if constexpr (SINK == ROW_PIECES) {
       __nv_bfloat16 pc[3][4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) split3(y[j], pc[0][j], pc[1][j], pc[2][j]);
-      __nv_bfloat16* o = outp + row * ldout + k;
+      __nv_bfloat16* o = sk.outp + row * sk.ld + k;
 #pragma unroll
-      for (int f = 0; f < 3; ++f) *reinterpret_cast<uint2*>(o + f * pst) = *reinterpret_cast<const uint2*>(pc[f]);
+      for (int f = 0; f < 3; ++f) *reinterpret_cast<uint2*>(o + f * sk.pst) = *reinterpret_cast<const uint2*>(pc[f]);
     } else {
-      *reinterpret_cast<float4*>(out + row * ldout + k) = make_float4(y[0], y[1], y[2], y[3]);
+      *reinterpret_cast<float4*>(sk.out + row * sk.ld + k) = make_float4(y[0], y[1], y[2], y[3]);
+    }
+    if constexpr (SINK == ROW_GRID) {
+      *reinterpret_cast<float4*>(sk.out2 + row * sk.ld + k) = make_float4(y[0], y[1], y[2], y[3]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) mn = fminf(mn, y[j]), mx = fmaxf(mx, y[j]), fin = fin && isfinite(y[j]);
     }
   }
+  if constexpr (SINK == ROW_GRID) row_grid_store<256>(mn, mx, fin, sk, row, sr);
 }
 
 // 4096-point column transform of 8 columns per CTA (1024 threads), in place.

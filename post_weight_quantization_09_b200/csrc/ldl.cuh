@@ -80,9 +80,10 @@ __device__ __forceinline__ void helpers_sync() {      // the helper warps of k_l
 // (31 .. 0): the pivot comes by shuffle from lane k, which formed it from its
 // own previous column entry (so the chain from pivot to pivot is one
 // shuffle, one rsqrtf, one multiply and one fma); lane i forms
-// R[i][k] = l_i, publishes it in a double-buffered shared column and
-// updates its row with the column's entries l_j, j < k (broadcast 16-byte
-// loads).  1 / R_kk is the rsqrtf of the pivot.  Then X = R^-1 column by
+// R[i][k] = l_i and updates its entry of the next column with R[k-1][k]
+// from a second shuffle, then publishes l_i in a double-buffered shared
+// column and updates the older entries l_j, j < k - 1, from there
+// (broadcast 16-byte loads).  1 / R_kk is the rsqrtf of the pivot.  Then X = R^-1 column by
 // column (lane j: column j), right-looking back substitution over the
 // columns of R, read as broadcast rows of a transposed copy.
 // scratch: 32 x LDL_LDX + 64 floats.  On return S's upper triangle holds R
@@ -113,17 +114,23 @@ __device__ __forceinline__ bool warp_chol_inv32(float* S, int lds, float* X, int
     const float l = (lane == k) ? piv * r : a[k] * r;
     a[k] = l;
     if (k > 0) {
-      self = fmaf(-l, l, a[k - 1]);        // lane k - 1: its next pivot
+      // the next column first, with one shuffle (R[k-1][k] from lane k - 1):
+      // the next pivot (lane k - 1) and the next column wait for no
+      // shared-memory round trip
+      const float lk1 = __shfl_sync(0xffffffffu, l, k - 1);
+      a[k - 1] = fmaf(-l, lk1, a[k - 1]);
+      self = a[k - 1];                     // lane k - 1: its next pivot
+      // the older columns through the shared column (needed a step later)
       float* cb = col + (k & 1) * 32;
       cb[lane] = l;
       __syncwarp();
 #pragma unroll
-      for (int j4 = 0; j4 < k; j4 += 4) {
+      for (int j4 = 0; j4 < k - 1; j4 += 4) {
         const float4 v = *reinterpret_cast<const float4*>(cb + j4);
-        if (j4 + 0 < k) a[j4 + 0] = fmaf(-l, v.x, a[j4 + 0]);
-        if (j4 + 1 < k) a[j4 + 1] = fmaf(-l, v.y, a[j4 + 1]);
-        if (j4 + 2 < k) a[j4 + 2] = fmaf(-l, v.z, a[j4 + 2]);
-        if (j4 + 3 < k) a[j4 + 3] = fmaf(-l, v.w, a[j4 + 3]);
+        if (j4 + 0 < k - 1) a[j4 + 0] = fmaf(-l, v.x, a[j4 + 0]);
+        if (j4 + 1 < k - 1) a[j4 + 1] = fmaf(-l, v.y, a[j4 + 1]);
+        if (j4 + 2 < k - 1) a[j4 + 2] = fmaf(-l, v.z, a[j4 + 2]);
+        if (j4 + 3 < k - 1) a[j4 + 3] = fmaf(-l, v.w, a[j4 + 3]);
       }
     }
   }
@@ -284,6 +291,23 @@ __device__ __forceinline__ void blk_solve(float* T, const float* Rp, const float
 
 // ---------------------------------------------------------------- kernels
 
+// One thread waits for the CTA's tile copies (bounded; after a timeout it
+// waits once more for the copies still in flight) and tells the CTA.
+__device__ __forceinline__ bool tiles_arrived(uint64_t* bar, int* flag) {
+  if (threadIdx.x == 0) {
+    const bool ok = mbar_wait(bar, 0);
+    if (!ok) mbar_wait(bar, 0);
+    *flag = ok ? 1 : 0;
+  }
+  __syncthreads();
+  return *flag != 0;
+}
+
+__device__ __forceinline__ float* align128(uint8_t* p) {
+  return reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(p) + 127) & ~uintptr_t(127));
+}
+
+
 // Factor of panel p, columns [c0, c0 + w), w <= 128.  Every CTA loads the
 // updated diagonal block (H - Lin, identity-padded past w) and factors it
 // (the same deterministic computation in each), as 4 x 4 blocks of 32:
@@ -417,22 +441,6 @@ __global__ void __launch_bounds__(LDL_FT, 1)
 // Tiles come in by TMA from fp32 2-D maps without swizzle whose boxes are
 // LDL_LDA (or LDL_LDX) columns wide, so that they land with the padded smem
 // row stride; rows and columns past a tensor's extent arrive as zeros.
-
-// One thread waits for the CTA's tile copies (bounded; after a timeout it
-// waits once more for the copies still in flight) and tells the CTA.
-__device__ __forceinline__ bool tiles_arrived(uint64_t* bar, int* flag) {
-  if (threadIdx.x == 0) {
-    const bool ok = mbar_wait(bar, 0);
-    if (!ok) mbar_wait(bar, 0);
-    *flag = ok ? 1 : 0;
-  }
-  __syncthreads();
-  return *flag != 0;
-}
-
-__device__ __forceinline__ float* align128(uint8_t* p) {
-  return reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(p) + 127) & ~uintptr_t(127));
-}
 
 // Row blocks r0 = row0 + 32 b .. + 31 (b = blockIdx.x, blockIdx.x +
 // gridDim.x, ... < nblk) of panel p:

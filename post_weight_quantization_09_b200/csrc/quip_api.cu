@@ -160,6 +160,27 @@ cudaError_t side_stream(SideStream& out) {
   return cudaSuccess;
 }
 
+// A per-device stream of the highest priority for the Hessian path of the
+// whole-layer call (H, H~, the LDL: a latency-bound chain that should get
+// SMs first), created on first use and kept for the process.
+cudaError_t hpath_stream(cudaStream_t* out) {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev]) {
+    int least = 0, greatest = 0;
+    if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
+    e = cudaStreamCreateWithPriority(&streams[dev], cudaStreamNonBlocking, greatest);
+    if (e != cudaSuccess) return e;
+  }
+  *out = streams[dev];
+  return cudaSuccess;
+}
+
 // Launch with programmatic stream serialization (the kernel starts with
 // pdl_wait_then_release, so it may be scheduled while its predecessor on
 // the stream finishes).
@@ -246,6 +267,12 @@ cudaError_t split_gemm(const CUtensorMap& ta, const CUtensorMap& tb, sgemm::Para
 
 // ---------------------------------------------------------------- Hadamard plans
 
+inline RowSink f32_sink(float* out, int64_t ld) {
+  RowSink k{};
+  k.out = out, k.ld = ld;
+  return k;
+}
+
 template <typename TIn>
 cudaError_t fwht_rows(const TIn* in, int64_t ldin, float* out, int64_t ldout, int64_t rows,
                       int64_t d, const float* pre, const float* post, const float* row_sign,
@@ -260,14 +287,14 @@ cudaError_t fwht_rows(const TIn* in, int64_t ldin, float* out, int64_t ldout, in
   }
   if (L == 12) {
     LaunchScope ls("k_fwht_rows", st);
-    k_fwht_row4096<TIn, false><<<(unsigned)rows, 256, 0, st>>>(in, ldin, RowDequant{}, out, nullptr, ldout, 0,
-                                                                pre, post, row_sign, scale);
+    k_fwht_row4096<TIn, ROW_F32><<<(unsigned)rows, 256, 0, st>>>(in, ldin, RowDequant{}, f32_sink(out, ldout),
+                                                                  pre, post, row_sign, scale);
     return cudaGetLastError();
   }
   if (L == 13) {
     LaunchScope ls("k_fwht_rows", st);
-    k_fwht_row8192<TIn, false><<<(unsigned)rows, 256, 0, st>>>(in, ldin, RowDequant{}, out, nullptr, ldout, 0,
-                                                                pre, post, row_sign, scale);
+    k_fwht_row8192<TIn, ROW_F32><<<(unsigned)rows, 256, 0, st>>>(in, ldin, RowDequant{}, f32_sink(out, ldout),
+                                                                  pre, post, row_sign, scale);
     return cudaGetLastError();
   }
   const int T = (int)(d / 16);
@@ -1282,26 +1309,43 @@ cudaError_t ldlq_range(const LdlqRun& r, int64_t a, int64_t b) {
 }
 }  // namespace
 
-quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu, int64_t m,
-                               int64_t n, int bits, int64_t block, uint8_t* codes, float* lo,
-                               float* scale, void* ws, size_t ws_bytes, void* stream) {
-  if (!W_t || !Uring || !codes || !lo || !scale) return QUIP_ERR_ARG;
+}  // extern "C"
+
+namespace {
+// Argument checks of quip_ldlq_quantize that do not involve pointers.
+quip_status ldlq_shape_ok(int64_t m, int64_t n, int bits, int64_t block) {
   if (bits < 1 || bits > 8) return QUIP_ERR_ARG;
-  if (m <= 0 || n <= 0 || ldu < n) return QUIP_ERR_SHAPE;
+  if (m <= 0 || n <= 0) return QUIP_ERR_SHAPE;
   if (!(block == 32 || block == 64 || block == 128) || n % block) return QUIP_ERR_SHAPE;
   // every block size is processed in 128-column blocks (the last one may be
   // 64 wide; same result), so n must be a multiple of 64
   if (n % 64) return QUIP_ERR_SHAPE;
   if (m > ((int64_t)1 << 20) || n > ((int64_t)1 << 16)) return QUIP_ERR_SHAPE;
-  if ((ldu & 3) || (reinterpret_cast<uintptr_t>(Uring) & 15) || (reinterpret_cast<uintptr_t>(W_t) & 15))
-    return QUIP_ERR_ARG;
-  quip_status s = check_ws(ws, ws_bytes, ldlq_ws_bytes(m, n, block));
-  if (s != QUIP_OK) return s;
+  return QUIP_OK;
+}
+
+// The part of LDLQ that needs W~ only: the per-row grid and the accumulator's
+// start A = W~ (m x n fp32).
+cudaError_t ldlq_prepare(const float* W_t, int64_t m, int64_t n, int bits, float* lo, float* scale, float* A,
+                         cudaStream_t st) {
+  {
+    LaunchScope ls("k_row_grid", st);
+    k_row_grid<<<(unsigned)((m + 7) / 8), 256, 0, st>>>(W_t, m, n, (1 << bits) - 1, lo, scale);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyAsync(A, W_t, (size_t)m * n * sizeof(float), cudaMemcpyDeviceToDevice, st);
+}
+
+// The rest of LDLQ once ldlq_prepare has run: ws_rest holds the error pieces
+// and the transposed factor (ldlq_ws_bytes less the accumulator).
+quip_status ldlq_main(const float* W_t, const float* Uring, int64_t ldu, int64_t m, int64_t n, int bits,
+                      uint8_t* codes, const float* lo, const float* scale, float* A, void* ws_rest,
+                      cudaStream_t st) {
   LdlqRun r{};
-  r.st = S(stream);
-  char* w8 = static_cast<char*>(ws);
-  r.A = reinterpret_cast<float*>(w8);
-  w8 += round256((size_t)m * n * 4);
+  r.st = st;
+  char* w8 = static_cast<char*>(ws_rest);
+  r.A = A;
   r.Es = reinterpret_cast<__nv_bfloat16*>(w8);
   w8 += round256((size_t)3 * m * n * 2);
   __nv_bfloat16* UTs = reinterpret_cast<__nv_bfloat16*>(w8);
@@ -1309,11 +1353,6 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
   float* UTf = reinterpret_cast<float*>(w8);
   r.Wt = W_t, r.U = Uring, r.ldu = ldu, r.m = m, r.n = n, r.lo = lo, r.sc = scale;
   r.qmax = (float)((1 << bits) - 1), r.codes = codes;
-  {
-    LaunchScope ls("k_row_grid", r.st);
-    k_row_grid<<<(unsigned)((m + 7) / 8), 256, 0, r.st>>>(W_t, m, n, (1 << bits) - 1, lo, scale);
-  }
-  QCHECK(cudaMemcpyAsync(r.A, W_t, (size_t)m * n * sizeof(float), cudaMemcpyDeviceToDevice, r.st));
   {
     const unsigned T = (unsigned)((n + 31) / 32);
     LaunchScope ls("k_split_upper_transposed", r.st);
@@ -1323,6 +1362,26 @@ quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu
   ldlq_block_attr();
   QCHECK(ldlq_range(r, 0, n));
   return QUIP_OK;
+}
+}  // namespace
+
+extern "C" {
+
+quip_status quip_ldlq_quantize(const float* W_t, const float* Uring, int64_t ldu, int64_t m,
+                               int64_t n, int bits, int64_t block, uint8_t* codes, float* lo,
+                               float* scale, void* ws, size_t ws_bytes, void* stream) {
+  if (!W_t || !Uring || !codes || !lo || !scale) return QUIP_ERR_ARG;
+  quip_status s = ldlq_shape_ok(m, n, bits, block);
+  if (s != QUIP_OK) return s;
+  if (ldu < n) return QUIP_ERR_SHAPE;
+  if ((ldu & 3) || (reinterpret_cast<uintptr_t>(Uring) & 15) || (reinterpret_cast<uintptr_t>(W_t) & 15))
+    return QUIP_ERR_ARG;
+  if ((s = check_ws(ws, ws_bytes, ldlq_ws_bytes(m, n, block))) != QUIP_OK) return s;
+  cudaStream_t st = S(stream);
+  float* A = static_cast<float*>(ws);
+  QCHECK(ldlq_prepare(W_t, m, n, bits, lo, scale, A, st));
+  return ldlq_main(W_t, Uring, ldu, m, n, bits, codes, lo, scale, A,
+                   static_cast<char*>(ws) + round256((size_t)m * n * 4), st);
 }
 
 quip_status quip_nearest_quantize(const float* W_t, int64_t m, int64_t n, int bits, uint8_t* codes,
@@ -1798,26 +1857,6 @@ cudaError_t copy_stream(cudaStream_t* out) {
   return cudaSuccess;
 }
 
-// A per-device stream of the highest priority for the Hessian path of the
-// whole-layer call (H, H~, the LDL: a latency-bound chain that should get
-// SMs first), created on first use and kept for the process.
-cudaError_t hpath_stream(cudaStream_t* out) {
-  static std::mutex mu;
-  static cudaStream_t streams[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!streams[dev]) {
-    int least = 0, greatest = 0;
-    if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
-    e = cudaStreamCreateWithPriority(&streams[dev], cudaStreamNonBlocking, greatest);
-    if (e != cudaSuccess) return e;
-  }
-  *out = streams[dev];
-  return cudaSuccess;
-}
 
 // Device workspace of the whole-layer call: H (n x n), D (n), W~ (m x n),
 // then one region shared by the stages (the largest stage workspace); the
@@ -1843,9 +1882,10 @@ quip_status layer_ws(const quip_transform* tf, int64_t N, int w_dtype, int x_dty
   o->D = round256((size_t)n * 4);
   o->Wt = round256((size_t)m * n * 4);
   o->stage = round256(std::max<size_t>(st, 256));
-  // the W path's forward transform runs beside the Hessian path: its own region
+  // the W path's forward transform runs beside the Hessian path: its own
+  // region, which then holds LDLQ's accumulator (started on the W path)
   if ((s = quip_workspace_size(QUIP_OP_INCOHERENCE_FORWARD, tf, m, n, block, &b)) != QUIP_OK) return s;
-  o->wstage = round256(std::max<size_t>(b, 256));
+  o->wstage = round256(std::max<size_t>(std::max<size_t>(b, (size_t)m * n * 4), 256));
   if (host) {
     o->Wd = round256((size_t)m * n * wes);
     o->Xd = round256((size_t)std::max<int64_t>(N, 1) * n * xes);
@@ -1860,6 +1900,8 @@ quip_status layer_ws(const quip_transform* tf, int64_t N, int w_dtype, int x_dty
 quip_status layer_args(const quip_transform* tf, int w_dtype, int64_t ldw, int x_dtype, int64_t N, int64_t ldx,
                        int bits, int64_t block, float damp) {
   if (!tf) return QUIP_ERR_ARG;
+  quip_status s = ldlq_shape_ok(tf->m, tf->n, bits, block);
+  if (s != QUIP_OK) return s;
   if ((w_dtype != QUIP_F32 && w_dtype != QUIP_BF16) || (x_dtype != QUIP_F32 && x_dtype != QUIP_BF16))
     return QUIP_ERR_ARG;
   if (bits < 1 || bits > 8 || !(damp >= 0.f) || !std::isfinite(damp)) return QUIP_ERR_ARG;
@@ -1870,6 +1912,50 @@ quip_status layer_args(const quip_transform* tf, int w_dtype, int64_t ldw, int x
 
 // Token chunks of X in the host variant: X's copy lands in up to four
 // pieces, each accumulated into H as soon as it is on the device.
+// W~ = U W V^T and LDLQ's start (per-row grid, accumulator A = W~) for the
+// layer call.  With bf16 W, a tensor-core Kronecker m side and an n-side
+// Hadamard of 4096 or 8192 points, the Hadamard row kernel comes last and
+// writes W~ twice (W_t and A) and the row grid while each row is in
+// registers (no separate grid and copy passes); the values are those of
+// quip_incoherence_forward then ldlq_prepare (the same operations in the
+// same order; min and max are exact).  Otherwise those two calls.
+quip_status forward_w_ldlq_start(const quip_transform* tf, const void* W, int w_dtype, int64_t ldw, float* W_t,
+                                 int bits, float* lo, float* scale, float* A, void* ws, size_t ws_bytes,
+                                 cudaStream_t st) {
+  const int64_t m = tf->m, n = tf->n;
+  const SideData &U = tf->side[0], &V = tf->side[1];
+  const int L = n > 0 ? ilog2(n) : 0;
+  const bool fused = w_dtype == QUIP_BF16 && (ldw % 8) == 0 && (reinterpret_cast<uintptr_t>(W) & 15) == 0 &&
+                     V.kind == QUIP_T_HADAMARD && !V.permute && !U.permute && (L == 12 || L == 13) &&
+                     (int64_t(1) << L) == n && kron_cols_tc_ok(U, n) && (reinterpret_cast<uintptr_t>(W_t) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(A) & 15) == 0;
+  if (!fused) {
+    quip_status r = quip_incoherence_forward(tf, W, w_dtype, ldw, W_t, nullptr, ws, ws_bytes, st);
+    if (r != QUIP_OK) return r;
+    QCHECK(ldlq_prepare(W_t, m, n, bits, lo, scale, A, st));
+    return QUIP_OK;
+  }
+  size_t need = 0;
+  quip_status s = quip_workspace_size(QUIP_OP_INCOHERENCE_FORWARD, tf, m, n, 0, &need);
+  if (s != QUIP_OK) return s;
+  if ((s = check_ws(ws, ws_bytes, need)) != QUIP_OK) return s;
+  QCHECK(kron_cols_tc<__nv_bfloat16>(U, false, static_cast<const __nv_bfloat16*>(W), ldw, W_t, n, ws, st));
+  RowSink sk{};
+  sk.out = W_t, sk.out2 = A, sk.ld = n, sk.lo = lo, sk.sc = scale, sk.qmax = (float)((1 << bits) - 1);
+  const float sc = (float)(1.0 / std::sqrt((double)n));
+  {
+    LaunchScope ls("k_fwht_rows", st);
+    if (L == 13)
+      k_fwht_row8192<float, ROW_GRID><<<(unsigned)m, 256, 0, st>>>(W_t, n, RowDequant{}, sk, V.signs, nullptr,
+                                                                   nullptr, sc);
+    else
+      k_fwht_row4096<float, ROW_GRID><<<(unsigned)m, 256, 0, st>>>(W_t, n, RowDequant{}, sk, V.signs, nullptr,
+                                                                   nullptr, sc);
+  }
+  QCHECK(cudaGetLastError());
+  return QUIP_OK;
+}
+
 // W_hat = U^T (lo + s . codes) V, the layer call's last step.  With an
 // n-side Hadamard of 4096 or 8192 points the dequantisation is folded into
 // the row kernel (it reads the codes), and with a tensor-core Kronecker m
@@ -1901,20 +1987,20 @@ quip_status inverse_from_codes(const quip_transform* tf, const uint8_t* codes, c
   const bool tc = kron_cols_tc_ok(U, n);
   __nv_bfloat16* P1 = static_cast<__nv_bfloat16*>(ws);
   const int64_t pst = m * n;
+  RowSink sk{};
+  sk.ld = n;
+  if (tc) sk.outp = P1, sk.pst = pst;
+  else sk.out = W_hat;
   {
     LaunchScope ls("k_fwht_rows", st);
     if (L == 13 && tc)
-      k_fwht_row8192<uint8_t, true><<<(unsigned)m, 256, 0, st>>>(codes, n, dq, nullptr, P1, n, pst, nullptr,
-                                                                V.signs, nullptr, sc);
+      k_fwht_row8192<uint8_t, ROW_PIECES><<<(unsigned)m, 256, 0, st>>>(codes, n, dq, sk, nullptr, V.signs, nullptr, sc);
     else if (L == 13)
-      k_fwht_row8192<uint8_t, false><<<(unsigned)m, 256, 0, st>>>(codes, n, dq, W_hat, nullptr, n, 0, nullptr,
-                                                                 V.signs, nullptr, sc);
+      k_fwht_row8192<uint8_t, ROW_F32><<<(unsigned)m, 256, 0, st>>>(codes, n, dq, sk, nullptr, V.signs, nullptr, sc);
     else if (tc)
-      k_fwht_row4096<uint8_t, true><<<(unsigned)m, 256, 0, st>>>(codes, n, dq, nullptr, P1, n, pst, nullptr,
-                                                                V.signs, nullptr, sc);
+      k_fwht_row4096<uint8_t, ROW_PIECES><<<(unsigned)m, 256, 0, st>>>(codes, n, dq, sk, nullptr, V.signs, nullptr, sc);
     else
-      k_fwht_row4096<uint8_t, false><<<(unsigned)m, 256, 0, st>>>(codes, n, dq, W_hat, nullptr, n, 0, nullptr,
-                                                                 V.signs, nullptr, sc);
+      k_fwht_row4096<uint8_t, ROW_F32><<<(unsigned)m, 256, 0, st>>>(codes, n, dq, sk, nullptr, V.signs, nullptr, sc);
   }
   QCHECK(cudaGetLastError());
   if (tc) QCHECK(kron_cols_tc_x(U, true, P1, 3, n, W_hat, n, ws, st));
@@ -1980,11 +2066,14 @@ quip_status layer_device(quip_transform* tf, uint64_t seed, const void* W, int w
     if ((r = draw_side(tf->side[0], seed, 0, st)) != QUIP_OK) return r;
     if (w_ready) QCHECK(cudaStreamWaitEvent(st, w_ready, 0));
     QCHECK(cudaStreamWaitEvent(st, ev[1], 0));
-    if ((r = quip_incoherence_forward(tf, W, w_dtype, ldw, Wt, nullptr, sw2, L.wstage, st)) != QUIP_OK) return r;
+    // W~, and LDLQ's grid and accumulator (they need W~ only): still beside
+    // the LDL.  A lives in the W path's region, after the transform's use.
+    float* A = static_cast<float*>(sw2);
+    if ((r = forward_w_ldlq_start(tf, W, w_dtype, ldw, Wt, bits, lo, scale, A, sw2, L.wstage, st)) != QUIP_OK)
+      return r;
     // ---- both
     QCHECK(cudaStreamWaitEvent(st, ev[2], 0));
-    if ((r = quip_ldlq_quantize(Wt, H, n, m, n, bits, block, codes, lo, scale, sw, L.stage, st)) != QUIP_OK)
-      return r;
+    if ((r = ldlq_main(Wt, H, n, m, n, bits, codes, lo, scale, A, sw, st)) != QUIP_OK) return r;
     if (q_done) QCHECK(cudaEventRecord(q_done, st));
     if (W_hat) {
       if ((r = inverse_from_codes(tf, codes, lo, scale, W_hat, sw, L.stage, st)) != QUIP_OK) return r;
@@ -2129,6 +2218,36 @@ quip_status quip_timing_end(const char** names, uint64_t* launches, double* tota
     if (launches) launches[i] = agg[i].count;
     if (total_ms) total_ms[i] = agg[i].ms;
   }
+  return st;
+}
+
+quip_status quip_timing_trace(const char** names, double* start_ms, double* end_ms, int* stream_ids,
+                              int max_entries, int* n_entries) {
+  g_timing_on.store(false);
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  quip_status st = QUIP_OK;
+  std::vector<cudaStream_t> streams;
+  const int nrec = (int)g_timing_recs.size();
+  if (n_entries) *n_entries = nrec;
+  for (int i = 0; i < nrec && i < max_entries; ++i) {
+    const TimingRec& r = g_timing_recs[i];
+    float t0 = 0.f, t1 = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess ||
+        cudaEventElapsedTime(&t0, g_timing_recs[0].a, r.a) != cudaSuccess ||
+        cudaEventElapsedTime(&t1, g_timing_recs[0].a, r.b) != cudaSuccess) {
+      st = QUIP_ERR_CUDA;
+      continue;
+    }
+    size_t k = 0;
+    while (k < streams.size() && streams[k] != r.st) ++k;
+    if (k == streams.size()) streams.push_back(r.st);
+    if (names) names[i] = r.name;
+    if (start_ms) start_ms[i] = t0;
+    if (end_ms) end_ms[i] = t1;
+    if (stream_ids) stream_ids[i] = (int)k;
+  }
+  for (const TimingRec& r : g_timing_recs) g_timing_pool.push_back({r.a, r.b});
+  g_timing_recs.clear();
   return st;
 }
 

@@ -429,23 +429,35 @@ def test_layer_call_equals_the_stages_and_the_oracle():
     (8192, Side("kronecker", 8, 128)), (8192, Side("hadamard")),
     (4096, Side("kronecker", 8, 128)), (4096, Side("identity")),
 ])
-def test_layer_inverse_reads_the_codes(n, mk):
-    """In the layer call the n-side Hadamard row kernel (4096 or 8192 points)
-    reads the codes, the dequantisation folded in, and for a tensor-core
-    Kronecker m side writes the bf16 pieces the Kronecker products take.  W^
-    is the stage calls' quip_dequantize + quip_incoherence_inverse of the same
-    codes to the bit, and the oracle's U^T W~^ V of those codes within 1e-4 of
-    the row scale on sampled rows."""
+def test_layer_fused_row_kernels_equal_the_stages(n, mk):
+    """The layer call's fused row kernels on 4096- and 8192-point Hadamard n
+    sides: with a tensor-core Kronecker m side the forward row kernel also
+    writes LDLQ's accumulator and the per-row grid, and the inverse row
+    kernel reads the codes (the dequantisation folded in) and writes the
+    bf16 pieces the Kronecker products take.  Codes, grid, W~ and W^ equal the
+    stage calls' to the bit, and W^ the oracle's U^T W~^ V of those codes
+    within 1e-4 of the row scale on sampled rows."""
     m, N, bits, block, seed = 1024, 256, 2, 128, 21
     nk = Side("hadamard")
     d = random_layer(m, n, N, seed=31, dtype="bf16")
+    W, X = dev(d["W"], torch.bfloat16), dev(d["X"], torch.bfloat16)
+    st = Q.LayerQuantizer(m, n, mk, nk, bits, block, 0.01, seed)
+    st.new_transform()
+    Q.quip_hessian_accumulate(X, st.H)
+    Q.quip_hessian_finalize(st.H, N, 0.01)
+    Q.quip_incoherence_forward(st.tf, None, None, st.H, st.ws)
+    Q.quip_ldl(st.H, st.D, st.ws)
+    Q.quip_incoherence_forward(st.tf, W, st.W_t, None, st.ws)
+    Q.quip_ldlq_quantize(st.W_t, st.H, bits, block, st.codes, st.lo, st.scale, st.ws)
+    Q.quip_dequantize(st.codes, st.lo, st.scale, st.W_hat)
+    Q.quip_incoherence_inverse(st.tf, st.W_hat, st.W_hat, st.ws)
     q = Q.LayerQuantizer(m, n, mk, nk, bits, block, 0.01, seed)
-    r = q.run(dev(d["W"], torch.bfloat16), dev(d["X"], torch.bfloat16))
+    r = q.run(W, X)
     assert Q.quip_sync_status() == L.QUIP_OK
-    Wh = torch.empty_like(r.W_hat)
-    Q.quip_dequantize(r.codes, r.lo, r.scale, Wh)
-    Q.quip_incoherence_inverse(q.tf, Wh, Wh, q.ws)
-    assert torch.equal(r.W_hat, Wh)
+    assert torch.equal(q.W_t, st.W_t)
+    assert torch.equal(r.lo, st.lo) and torch.equal(r.scale, st.scale)
+    assert torch.equal(r.codes, st.codes)
+    assert torch.equal(r.W_hat, st.W_hat)
     C, lo, s = host(r.codes), host(r.lo), host(r.scale)
     U = O.make_side(seed, "m", mk.kind, m, mk.p, mk.q)
     V = O.make_side(seed, "n", nk.kind, n)
