@@ -82,8 +82,9 @@ __device__ __forceinline__ void helpers_sync() {      // the helper warps of k_l
 // shuffle, one rsqrtf, one multiply and one fma); lane i forms
 // R[i][k] = l_i and updates its entry of the next column with R[k-1][k]
 // from a second shuffle, then publishes l_i in a double-buffered shared
-// column and updates the older entries l_j, j < k - 1, from there
-// (broadcast 16-byte loads).  1 / R_kk is the rsqrtf of the pivot.  Then X = R^-1 column by
+// column (broadcast 16-byte loads) whose other entries, j < k - 1, it
+// applies in step k - 1 while that step's rsqrtf is in flight (warps issue
+// in order: the updates no longer hold up the next pivot).  1 / R_kk is the rsqrtf of the pivot.  Then X = R^-1 column by
 // column (lane j: column j), right-looking back substitution over the
 // columns of R, read as broadcast rows of a transposed copy.
 // scratch: 32 x LDL_LDX + 64 floats.  On return S's upper triangle holds R
@@ -105,33 +106,39 @@ __device__ __forceinline__ bool warp_chol_inv32(float* S, int lds, float* X, int
   }
   bool ok = true;
   float self = a[31];
+  float v[32];                                    // the previous step's column, from shared memory
+  float lp = 0.f;                                 // the previous step's l_i
 #pragma unroll
   for (int k = 31; k >= 0; --k) {
     const float piv = __shfl_sync(0xffffffffu, self, k);
     ok = ok && (piv > 0.f) && (piv < INFINITY);
     const float r = rsqrtf(piv);
+    // step k + 1's updates of the columns j < k, issued while rsqrtf is in
+    // flight (each entry still takes its updates in step order)
+    if (k < 31) {
+#pragma unroll
+      for (int j = 0; j < k; ++j) a[j] = fmaf(-lp, v[j], a[j]);
+    }
     if (lane == 0) rin[k] = r;
     const float l = (lane == k) ? piv * r : a[k] * r;
     a[k] = l;
     if (k > 0) {
-      // the next column first, with one shuffle (R[k-1][k] from lane k - 1):
+      // the next column at once, with one shuffle (R[k-1][k] from lane k - 1):
       // the next pivot (lane k - 1) and the next column wait for no
       // shared-memory round trip
       const float lk1 = __shfl_sync(0xffffffffu, l, k - 1);
       a[k - 1] = fmaf(-l, lk1, a[k - 1]);
       self = a[k - 1];                     // lane k - 1: its next pivot
-      // the older columns through the shared column (needed a step later)
+      // the older columns through the shared column, applied in the next step
       float* cb = col + (k & 1) * 32;
       cb[lane] = l;
       __syncwarp();
 #pragma unroll
       for (int j4 = 0; j4 < k - 1; j4 += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(cb + j4);
-        if (j4 + 0 < k - 1) a[j4 + 0] = fmaf(-l, v.x, a[j4 + 0]);
-        if (j4 + 1 < k - 1) a[j4 + 1] = fmaf(-l, v.y, a[j4 + 1]);
-        if (j4 + 2 < k - 1) a[j4 + 2] = fmaf(-l, v.z, a[j4 + 2]);
-        if (j4 + 3 < k - 1) a[j4 + 3] = fmaf(-l, v.w, a[j4 + 3]);
+        const float4 c = *reinterpret_cast<const float4*>(cb + j4);
+        v[j4] = c.x, v[j4 + 1] = c.y, v[j4 + 2] = c.z, v[j4 + 3] = c.w;
       }
+      lp = l;
     }
   }
 #pragma unroll

@@ -2060,17 +2060,19 @@ quip_status layer_device(quip_transform* tf, uint64_t seed, const void* W, int w
     }
     if ((r = quip_hessian_finalize(H, n, N, damp, hs)) != QUIP_OK) return r;
     if ((r = quip_incoherence_forward(tf, nullptr, QUIP_F32, n, nullptr, H, sw, L.stage, hs)) != QUIP_OK) return r;
-    if ((r = quip_ldl(H, D, n, sw, L.stage, hs)) != QUIP_OK) return r;
-    QCHECK(cudaEventRecord(ev[2], hs));
-    // ---- weight path (st)
+    // ---- weight path (st), enqueued before the LDL's many launches so that
+    // its kernels start while the Hessian is accumulated
     if ((r = draw_side(tf->side[0], seed, 0, st)) != QUIP_OK) return r;
     if (w_ready) QCHECK(cudaStreamWaitEvent(st, w_ready, 0));
     QCHECK(cudaStreamWaitEvent(st, ev[1], 0));
-    // W~, and LDLQ's grid and accumulator (they need W~ only): still beside
-    // the LDL.  A lives in the W path's region, after the transform's use.
+    // W~, and LDLQ's grid and accumulator (they need W~ only): beside the
+    // Hessian path.  A lives in the W path's region, after the transform's use.
     float* A = static_cast<float*>(sw2);
     if ((r = forward_w_ldlq_start(tf, W, w_dtype, ldw, Wt, bits, lo, scale, A, sw2, L.wstage, st)) != QUIP_OK)
       return r;
+    // ---- Hessian path: the LDL of H~
+    if ((r = quip_ldl(H, D, n, sw, L.stage, hs)) != QUIP_OK) return r;
+    QCHECK(cudaEventRecord(ev[2], hs));
     // ---- both
     QCHECK(cudaStreamWaitEvent(st, ev[2], 0));
     if ((r = ldlq_main(Wt, H, n, m, n, bits, codes, lo, scale, A, sw, st)) != QUIP_OK) return r;

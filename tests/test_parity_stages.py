@@ -486,3 +486,33 @@ def test_pipeline_with_random_permutations(mk, nk):
     assert np.abs(host(r.W_hat) - W_hat_ref).max() <= 1e-4 * s.max()
     bad, not_near = ldlq_trajectory_check(C, P.Wt, P.Uf, lo, s, bits, tau=1e-3)
     assert not_near == 0.0
+
+
+def test_timing_trace_lists_the_layer_launches():
+    """quip_timing_trace: one record per launch of the layer call, in enqueue
+    order, each with end >= start >= 0 on the stream it ran on; the Hessian
+    path (SYRK, LDL) and the weight path run on different streams.  The same
+    launches, aggregated, are what quip_timing_end reports."""
+    m, n, N, bits, block, seed = 256, 256, 512, 2, 128, 3
+    mk, nk = Side("kronecker", 2, 128), Side("hadamard")
+    d = random_layer(m, n, N, seed=2, dtype="bf16")
+    W, X = dev(d["W"], torch.bfloat16), dev(d["X"], torch.bfloat16)
+    q = Q.LayerQuantizer(m, n, mk, nk, bits, block, 0.01, seed)
+    q.run(W, X)
+    torch.cuda.synchronize()
+    Q.quip_timing_begin()
+    q.run(W, X)
+    torch.cuda.synchronize()
+    tr = Q.quip_timing_trace()
+    assert len(tr) > 10
+    assert all(b >= a >= 0.0 for _, a, b, _ in tr)
+    names = [k for k, _, _, _ in tr]
+    assert "k_syrk_tc" in names and "k_ldlq_block" in names and "k_ldl_factor" in names
+    sid = {k: s for k, _, _, s in tr}
+    assert sid["k_syrk_tc"] != sid["k_ldlq_block"]
+    Q.quip_timing_begin()
+    q.run(W, X)
+    torch.cuda.synchronize()
+    agg = Q.quip_timing_end()
+    assert sum(c for c, _ in agg.values()) == len(tr)
+    assert agg["k_syrk_tc"][0] == names.count("k_syrk_tc")
