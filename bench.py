@@ -174,13 +174,15 @@ def kernel_work(cfg: LayerConfig, method: str = "ldlq", passes: int = 1):
 # the full layer's; the LDLQ GEMMs' A operand and accumulator and the
 # row-wise kernels' bytes grow with the rows, so their figures are the
 # slice's times 28672 / 7168 = 4.  Writes still in L2 when a kernel ends are
-# not counted (the LDLQ block kernel's codes and error pieces).
+# not counted (the LDLQ block kernel's codes and error pieces).  The
+# dequantisation and row-grid figures were taken on a build of ldlq.cuh that
+# differs from this one only in the block kernel.
 KERNEL_TRAFFIC = {
-    "k_gemm_split_tc[ldlq]": ("gemm_tc.cuh", "1aabcc329733", 172766566),
-    "k_gemm_split_tc[ldl]": ("gemm_tc.cuh", "1aabcc329733", 61325242),
-    "k_ldlq_block": ("ldlq.cuh", "0bb6d47b4440", 44938240),
-    "k_dequant": ("ldlq.cuh", "0bb6d47b4440", 941438976),
-    "k_row_grid": ("ldlq.cuh", "0bb6d47b4440", 970614784),
+    "k_gemm_split_tc[ldlq]": ("gemm_tc.cuh", "07f39ed17af3", 172632584),
+    "k_gemm_split_tc[ldl]": ("gemm_tc.cuh", "07f39ed17af3", 61238127),
+    "k_ldlq_block": ("ldlq.cuh", "1b4f510b2a1b", 44941312),
+    "k_dequant": ("ldlq.cuh", "1b4f510b2a1b", 941438976),
+    "k_row_grid": ("ldlq.cuh", "1b4f510b2a1b", 970614784),
 }
 TRAFFIC_WORKLOAD = "gate70b"
 
