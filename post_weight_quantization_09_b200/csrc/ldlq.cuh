@@ -93,7 +93,10 @@ __device__ __forceinline__ void nb_arrive(int id, int count) {
 // last group) and add group g's feedback to the columns from
 // two groups on, acc[r][j] += sum_t e_t Ů[16 g + t][j] (each thread: four
 // rows and every twelfth 4-column chunk, so one broadcast 16-byte load of a
-// UT row serves 16 fmas), while the rounding warp takes group g + 1.  Named
+// UT row serves 16 fmas; the chunks' accumulated values stay in registers and
+// are stored to the shared tile once, after their last feedback, two groups
+// before the rounding warp reads them), while the rounding warp takes group
+// g + 1.  Named
 // barriers pass the hand-off slots: READY + slot (rounding warp -> helpers,
 // every group) and DONE + slot (helpers -> rounding warp, only for groups
 // it will wait on).
@@ -200,6 +203,23 @@ __global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
     // c with c % 12 == 4 h + lane / 8 (every Ů^T load serves four rows);
     // helper warp 0 also stores row `lane`'s codes and error pieces.
     const int h = warp < rw ? warp : warp - 1, rb = r & 7, cls = 4 * h + (r >> 3);
+    // this thread's chunks that take feedback (c >= 8, c < w / 4): at most two,
+    // cls + 12 k; their accumulated values stay in registers for the block
+    int cc[2];
+    bool has[2];
+    cc[0] = cls >= 8 ? cls : cls + 12;
+    cc[1] = cc[0] + 12;
+    float a[2][4][4];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      has[k] = 4 * cc[k] < w;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (has[k]) a4 = *reinterpret_cast<const float4*>(acc + (rb + 8 * i) * LQB_S + 4 * cc[k]);
+        a[k][i][0] = a4.x, a[k][i][1] = a4.y, a[k][i][2] = a4.z, a[k][i][3] = a4.w;
+      }
+    }
 #pragma unroll 1
     for (int g = 0; g < ngroups; ++g) {
       const int slot = g & 1;
@@ -226,9 +246,9 @@ __global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
           dst[1] = make_uint4(pk[p][4], pk[p][5], pk[p][6], pk[p][7]);
         }
       }
-      const int c0 = 4 * (g + 2);                      // first chunk two groups on
-      int c = c0 + ((cls - c0 % 12) + 12) % 12;        // first chunk of this class
-      if (4 * c < w) {
+      // group g's feedback into this thread's chunks from two groups on
+      const int c0 = 4 * (g + 2);
+      if ((has[0] && cc[0] >= c0) || (has[1] && cc[1] >= c0)) {
         float e[4][16];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
@@ -238,15 +258,10 @@ __global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
             e[i][4 * q] = v.x, e[i][4 * q + 1] = v.y, e[i][4 * q + 2] = v.z, e[i][4 * q + 3] = v.w;
           }
         const float* ug = UT + 16 * g;
-#pragma unroll 1
-        for (; 4 * c < w; c += 12) {
-          const int j = 4 * c;
-          float a[4][4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float4 a4 = *reinterpret_cast<const float4*>(acc + (rb + 8 * i) * LQB_S + j);
-            a[i][0] = a4.x, a[i][1] = a4.y, a[i][2] = a4.z, a[i][3] = a4.w;
-          }
+        for (int k = 0; k < 2; ++k) {
+          if (!has[k] || cc[k] < c0) continue;
+          const int j = 4 * cc[k];
 #pragma unroll
           for (int t4 = 0; t4 < 16; t4 += 4) {
 #pragma unroll
@@ -254,19 +269,24 @@ __global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
               const float4 u = *reinterpret_cast<const float4*>(ug + (j + q) * LQB_S + t4);
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
-                a[i][q] = fmaf(e[i][t4 + 0], u.x, a[i][q]);
-                a[i][q] = fmaf(e[i][t4 + 1], u.y, a[i][q]);
-                a[i][q] = fmaf(e[i][t4 + 2], u.z, a[i][q]);
-                a[i][q] = fmaf(e[i][t4 + 3], u.w, a[i][q]);
+                a[k][i][q] = fmaf(e[i][t4 + 0], u.x, a[k][i][q]);
+                a[k][i][q] = fmaf(e[i][t4 + 1], u.y, a[k][i][q]);
+                a[k][i][q] = fmaf(e[i][t4 + 2], u.z, a[k][i][q]);
+                a[k][i][q] = fmaf(e[i][t4 + 3], u.w, a[k][i][q]);
               }
             }
           }
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<float4*>(acc + (rb + 8 * i) * LQB_S + j) =
-                make_float4(a[i][0], a[i][1], a[i][2], a[i][3]);
         }
       }
+      // chunks the rounding warp takes two groups on have all their feedback:
+      // back to the shared tile (the only shared-memory traffic of acc)
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        if (has[k] && (cc[k] >> 2) == g + 2)
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4*>(acc + (rb + 8 * i) * LQB_S + 4 * cc[k]) =
+                make_float4(a[k][i][0], a[k][i][1], a[k][i][2], a[k][i][3]);
       if (g + 2 < ngroups) nb_arrive(bar_done + slot, LQB_THREADS);
     }
   } else {
