@@ -439,9 +439,10 @@ quip_status quip_quantize_layer(quip_transform* tf, uint64_t seed, const void* W
  * (same shapes, types and strides as above) are copied to the device on a
  * library-owned copy stream, X in token chunks of at least 2048 so that the
  * Hessian accumulates each chunk as it lands, W while the Hessian, H~ and the
- * LDL run (they do not read W); codes_host (m x n uint8), lo_host and
- * scale_host (m fp32) are copied back on that stream while W^ is formed on
- * the device, and W^ (m x n fp32) into W_hat_host when it is not NULL (W^ is
+ * LDL run (they do not read W); codes_host (m x n uint8) is copied back on
+ * that stream in column chunks (about eight, one cudaMemcpy2DAsync each) as
+ * LDLQ finishes their columns, lo_host and scale_host (m fp32) once LDLQ is
+ * done, and W^ (m x n fp32) into W_hat_host when it is not NULL (W^ is
  * computed either way: it is the last step of the path).  One
  * cudaMemcpy2DAsync / cudaMemcpyAsync per piece.  `stream` waits for every
  * copy, so synchronising it makes all host outputs valid; host buffers

@@ -1245,21 +1245,34 @@ struct LdlqRun {
   __nv_bfloat16* Es;
   CUtensorMap ta, tb, tb64, tb128, tacc, tut, tband, tw;
   cudaStream_t st;
+  // optional: code_ev[c] is recorded once the block kernels of column blocks
+  // [c code_every, (c + 1) code_every) have written their codes
+  const cudaEvent_t* code_ev;
+  int code_every;
 };
 
 constexpr int LDQ_BLK = 128;               // LDLQ block width (columns)
+constexpr int64_t LQB_BLOCK_COLS = LDQ_BLK;
 
 // One 32-row sub-group per CTA while that fits one wave of the GPU, else two
 // (fewer waves of the rows' rounding chains).
 cudaError_t ldlq_block(const LdlqRun& r, int64_t k0, int w) {
   const int64_t units = (r.m + LQB_ROWS - 1) / LQB_ROWS;
-  LaunchScope ls("k_ldlq_block", r.st);
-  if (units <= num_sms())
-    return launch_pdl(k_ldlq_block<1>, dim3((unsigned)units), dim3(LQB_THREADS), (size_t)lqb_smem(1), r.st,
-                      r.tacc, r.tut, r.tband, r.tw, r.m, r.n, k0, w, r.lo, r.sc, r.qmax, r.codes, r.Es, r.n);
-  return launch_pdl(k_ldlq_block<2>, dim3((unsigned)((units + 1) / 2)), dim3(2 * LQB_THREADS),
-                    (size_t)lqb_smem(2), r.st, r.tacc, r.tut, r.tband, r.tw, r.m, r.n, k0, w, r.lo, r.sc,
-                    r.qmax, r.codes, r.Es, r.n);
+  cudaError_t e;
+  {
+    LaunchScope ls("k_ldlq_block", r.st);
+    if (units <= num_sms())
+      e = launch_pdl(k_ldlq_block<1>, dim3((unsigned)units), dim3(LQB_THREADS), (size_t)lqb_smem(1), r.st,
+                     r.tacc, r.tut, r.tband, r.tw, r.m, r.n, k0, w, r.lo, r.sc, r.qmax, r.codes, r.Es, r.n);
+    else
+      e = launch_pdl(k_ldlq_block<2>, dim3((unsigned)((units + 1) / 2)), dim3(2 * LQB_THREADS),
+                     (size_t)lqb_smem(2), r.st, r.tacc, r.tut, r.tband, r.tw, r.m, r.n, k0, w, r.lo, r.sc,
+                     r.qmax, r.codes, r.Es, r.n);
+  }
+  if (e != cudaSuccess || !r.code_ev) return e;
+  const int64_t blk = k0 / LQB_BLOCK_COLS;
+  if ((blk + 1) % r.code_every == 0 || k0 + w >= r.n) e = cudaEventRecord(r.code_ev[blk / r.code_every], r.st);
+  return e;
 }
 
 // Tensor maps of a run: the block kernel's (accumulator, weights, the
@@ -1341,9 +1354,10 @@ cudaError_t ldlq_prepare(const float* W_t, int64_t m, int64_t n, int bits, float
 // and the transposed factor (ldlq_ws_bytes less the accumulator).
 quip_status ldlq_main(const float* W_t, const float* Uring, int64_t ldu, int64_t m, int64_t n, int bits,
                       uint8_t* codes, const float* lo, const float* scale, float* A, void* ws_rest,
-                      cudaStream_t st) {
+                      cudaStream_t st, const cudaEvent_t* code_ev = nullptr, int code_every = 1) {
   LdlqRun r{};
   r.st = st;
+  r.code_ev = code_ev, r.code_every = code_every;
   char* w8 = static_cast<char*>(ws_rest);
   r.A = A;
   r.Es = reinterpret_cast<__nv_bfloat16*>(w8);
@@ -2025,7 +2039,8 @@ quip_status layer_device(quip_transform* tf, uint64_t seed, const void* W, int w
                          const void* X, int x_dtype, int64_t N, int64_t ldx, int bits, int64_t block,
                          float damp, uint8_t* codes, float* lo, float* scale, float* W_hat,
                          const LayerWs& L, char* ws, cudaStream_t st, const cudaEvent_t* x_ready,
-                         cudaEvent_t w_ready, cudaEvent_t q_done) {
+                         cudaEvent_t w_ready, cudaEvent_t q_done, const cudaEvent_t* code_ev = nullptr,
+                         int code_every = 1) {
   const int64_t m = tf->m, n = tf->n;
   float* H = reinterpret_cast<float*>(ws);
   float* D = reinterpret_cast<float*>(ws + L.H);
@@ -2075,7 +2090,8 @@ quip_status layer_device(quip_transform* tf, uint64_t seed, const void* W, int w
     QCHECK(cudaEventRecord(ev[2], hs));
     // ---- both
     QCHECK(cudaStreamWaitEvent(st, ev[2], 0));
-    if ((r = ldlq_main(Wt, H, n, m, n, bits, codes, lo, scale, A, sw, st)) != QUIP_OK) return r;
+    if ((r = ldlq_main(Wt, H, n, m, n, bits, codes, lo, scale, A, sw, st, code_ev, code_every)) != QUIP_OK)
+      return r;
     if (q_done) QCHECK(cudaEventRecord(q_done, st));
     if (W_hat) {
       if ((r = inverse_from_codes(tf, codes, lo, scale, W_hat, sw, L.stage, st)) != QUIP_OK) return r;
@@ -2143,9 +2159,15 @@ quip_status quip_quantize_layer_host(quip_transform* tf, uint64_t seed, const vo
   QCHECK(copy_stream(&cp));
   const int64_t step = layer_x_chunk(N);
   const int nch = (int)((N + step - 1) / step);
-  std::vector<cudaEvent_t> ev(nch + 4, nullptr);
+  // the codes go back in about eight column chunks, each as soon as LDLQ's
+  // block kernels have finished its columns (they run in column order)
+  const int64_t nblk = (n + LQB_BLOCK_COLS - 1) / LQB_BLOCK_COLS;
+  const int every = (int)std::max<int64_t>(1, (nblk + 7) / 8);
+  const int ncc = (int)((nblk + every - 1) / every);
+  std::vector<cudaEvent_t> ev(nch + 4 + ncc, nullptr);
   for (auto& e : ev) QCHECK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
   cudaEvent_t fork = ev[nch], w_ready = ev[nch + 1], q_done = ev[nch + 2], out_done = ev[nch + 3];
+  const cudaEvent_t* code_ev = ev.data() + nch + 4;
   // the copies start after earlier work on the caller's stream, which may
   // still be reading this workspace
   QCHECK(cudaEventRecord(fork, st));
@@ -2162,11 +2184,17 @@ quip_status quip_quantize_layer_host(quip_transform* tf, uint64_t seed, const vo
                            cudaMemcpyHostToDevice, cp));
   QCHECK(cudaEventRecord(w_ready, cp));
   s = layer_device(tf, seed, Wd, w_dtype, n, Xd, x_dtype, N, n, bits, block, damp, codes, lo, sc, What, L,
-                   static_cast<char*>(ws), st, ev.data(), w_ready, q_done);
+                   static_cast<char*>(ws), st, ev.data(), w_ready, q_done, code_ev, every);
   if (s == QUIP_OK) {
-    // codes and grid go back while W^ is formed; W^ after it
+    // the codes go back while LDLQ runs, one column chunk (all rows, a 2-D
+    // copy) per event; the grid once LDLQ is done; W^ after it
+    for (int c = 0; c < ncc; ++c) {
+      const int64_t c0 = (int64_t)c * every * LQB_BLOCK_COLS, c1 = std::min(n, c0 + every * LQB_BLOCK_COLS);
+      QCHECK(cudaStreamWaitEvent(cp, code_ev[c], 0));
+      QCHECK(cudaMemcpy2DAsync(codes_host + c0, (size_t)n, codes + c0, (size_t)n, (size_t)(c1 - c0), (size_t)m,
+                               cudaMemcpyDeviceToHost, cp));
+    }
     QCHECK(cudaStreamWaitEvent(cp, q_done, 0));
-    QCHECK(cudaMemcpyAsync(codes_host, codes, (size_t)m * n, cudaMemcpyDeviceToHost, cp));
     QCHECK(cudaMemcpyAsync(lo_host, lo, (size_t)m * 4, cudaMemcpyDeviceToHost, cp));
     QCHECK(cudaMemcpyAsync(scale_host, sc, (size_t)m * 4, cudaMemcpyDeviceToHost, cp));
     if (W_hat_host) QCHECK(cudaMemcpyAsync(W_hat_host, What, (size_t)m * n * 4, cudaMemcpyDeviceToHost, st));
