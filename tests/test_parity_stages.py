@@ -373,6 +373,38 @@ def test_run_host_equals_device_run():
         assert torch.equal(co, codes) and torch.equal(lo_h, lo) and torch.equal(sc_h, sc)
 
 
+@pytest.mark.parametrize("n,nk,block", [
+    (1088, Side("kronecker", 17, 64), 64),     # 9 column blocks, the last 64 wide: 5 chunks of 2
+    (2048, Side("hadamard"), 128),             # 16 blocks: 8 chunks of 2
+])
+def test_host_call_streams_the_codes_back(n, nk, block):
+    """quip_quantize_layer_host copies the codes back in column chunks while
+    LDLQ runs (about eight, each after the block kernels that finish its
+    columns): with one token chunk (the same Hessian) the host codes, grid and
+    W^ are the device call's to the bit, including a last 64-wide block."""
+    m, N, bits, seed = 256, 1024, 3, 5
+    mk = Side("hadamard")
+    d = random_layer(m, n, N, seed=17, dtype="bf16")
+    q = Q.LayerQuantizer(m, n, mk, nk, bits, block, 0.01, seed)
+    r = q.run(dev(d["W"], torch.bfloat16), dev(d["X"], torch.bfloat16))
+    assert Q.quip_sync_status() == L.QUIP_OK
+    codes, lo, sc = r.codes.cpu(), r.lo.cpu(), r.scale.cpu()
+    W_hat = r.W_hat.cpu()
+    Wh = torch.from_numpy(d["W_bf16"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    Xh = torch.from_numpy(d["X_bf16"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    co = torch.full((m, n), 255, dtype=torch.uint8).pin_memory()
+    lo_h, sc_h = torch.empty(m).pin_memory(), torch.empty(m).pin_memory()
+    wh = torch.empty(m, n).pin_memory()
+    q2 = Q.LayerQuantizer(m, n, mk, nk, bits, block, 0.01, seed)
+    ws = torch.empty(Q.quip_layer_workspace_size(q2.tf, N, L.QUIP_BF16, L.QUIP_BF16, block, True),
+                     dtype=torch.uint8, device="cuda")
+    Q.quip_quantize_layer_host(q2.tf, seed, Wh, Xh, bits, block, 0.01, co, lo_h, sc_h, wh, ws)
+    torch.cuda.current_stream().synchronize()
+    assert Q.quip_sync_status() == L.QUIP_OK
+    assert torch.equal(co, codes) and torch.equal(lo_h, lo) and torch.equal(sc_h, sc)
+    assert torch.equal(wh, W_hat)
+
+
 def test_layer_call_equals_the_stages_and_the_oracle():
     """quip_quantize_layer (one library call) runs the same kernels in the
     same order as the stage-by-stage calls: identical codes, grid and W^;
