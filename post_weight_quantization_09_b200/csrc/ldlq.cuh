@@ -88,9 +88,10 @@ __device__ __forceinline__ void nb_arrive(int id, int count) {
 //   2. rounds column by column, feeding each error to the group's later
 //      columns and into the group's feedback to the next group (carry);
 //   3. hands the 16 errors and codes to the helpers (shared slot g % 2).
-// The helpers stage the codes and the errors' three bf16 pieces (the
-// trailing GEMMs' A operand; written out with coalesced stores after the
-// last group) and add group g's feedback to the columns from
+// The helpers write the codes and the errors' three bf16 pieces (the
+// trailing GEMMs' A operand) of each group to global memory as the group is
+// handed over (helper 0, lane r: row r; 16-byte stores spread over the
+// block instead of one burst at its end) and add group g's feedback to the columns from
 // two groups on, acc[r][j] += sum_t e_t Ů[16 g + t][j] (each thread: four
 // rows and every twelfth 4-column chunk, so one broadcast 16-byte load of a
 // UT row serves 16 fmas; the chunks' accumulated values stay in registers and
@@ -114,14 +115,10 @@ constexpr int LQB_ACC = LQB_ROWS * LQB_S * 4;          // bytes of the acc tile
 constexpr int LQB_UT = 128 * LQB_S * 4;                // bytes of the UT tile
 constexpr int LQB_BAND = 128 * 32 * 4;                 // bytes of the band
 constexpr int LQB_E = 2 * LQB_ROWS * LQB_ES * 4;       // bytes of the two error slots (+ codes)
-constexpr int LQB_PS = 136;                            // row stride (bf16) of the staged pieces
-constexpr int LQB_CS = 144;                            // row stride (bytes) of the staged codes
-constexpr int LQB_P = 3 * LQB_ROWS * LQB_PS * 2;       // bytes of the staged pieces
-constexpr int LQB_C = LQB_ROWS * LQB_CS;               // bytes of the staged codes
-// Shared memory of a CTA of SUB sub-groups: per sub-group acc, wt, the slots
-// and the staging buffers; UT and the band once.
+// Shared memory of a CTA of SUB sub-groups: per sub-group acc, wt and the
+// slots; UT and the band once.
 __host__ __device__ constexpr int lqb_smem(int sub) {
-  return 128 + LQB_UT + LQB_BAND + sub * (2 * LQB_ACC + LQB_E + LQB_P + LQB_C);
+  return 128 + LQB_UT + LQB_BAND + sub * (2 * LQB_ACC + LQB_E);
 }
 constexpr int LQB_SMEM = lqb_smem(1);
 constexpr int LQB_READY = 1, LQB_DONE = 3;             // named barrier ids (+ slot, + 4 x sub-group)
@@ -144,8 +141,6 @@ __global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
   float* acc0 = band + 128 * 32;                       // [CROWS][LQB_S]: accumulated values
   float* wt0 = acc0 + CROWS * LQB_S;                   // [CROWS][LQB_S]: the rows' W~ of the block
   float* eslot0 = wt0 + CROWS * LQB_S;                 // [SUB][2][32][LQB_ES]
-  __nv_bfloat16* ps = reinterpret_cast<__nv_bfloat16*>(eslot0 + SUB * 2 * LQB_ROWS * LQB_ES);  // [3][CROWS][LQB_PS]
-  uint8_t* cs = reinterpret_cast<uint8_t*>(ps + 3 * CROWS * LQB_PS);                          // [CROWS][LQB_CS]
   __shared__ __align__(8) uint64_t bar;
   __shared__ int ok_s;
   const int tid = threadIdx.x, sg = tid / LQB_THREADS, warp = (tid % LQB_THREADS) >> 5, r = tid & 31;
@@ -226,7 +221,8 @@ __global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
       nb_sync(bar_ready + slot, LQB_THREADS);
       const float* eb = eslot + slot * LQB_ROWS * LQB_ES;
       if (h == 0) {
-        // row r's codes and error pieces into the staging buffers
+        // row r's codes and error pieces of the group straight to global
+        // memory: 16-byte stores spread over the block's groups
         const float* es = eb + r * LQB_ES;
         float e[16];
 #pragma unroll
@@ -234,16 +230,19 @@ __global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
           const float4 v = *reinterpret_cast<const float4*>(es + 4 * q);
           e[4 * q] = v.x, e[4 * q + 1] = v.y, e[4 * q + 2] = v.z, e[4 * q + 3] = v.w;
         }
-        *reinterpret_cast<uint4*>(cs + srow * LQB_CS + 16 * g) = *reinterpret_cast<const uint4*>(es + 16);
         uint32_t pk[3][8];
 #pragma unroll
         for (int t = 0; t < 16; t += 2)
           split3x2(e[t], e[t + 1], pk[0][t >> 1], pk[1][t >> 1], pk[2][t >> 1]);
+        if (valid) {
+          *reinterpret_cast<uint4*>(codes + row * n + k0 + 16 * g) = *reinterpret_cast<const uint4*>(es + 16);
+          const int64_t pst = m * lde;
 #pragma unroll
-        for (int p = 0; p < 3; ++p) {
-          uint4* dst = reinterpret_cast<uint4*>(ps + (p * CROWS + srow) * LQB_PS + 16 * g);
-          dst[0] = make_uint4(pk[p][0], pk[p][1], pk[p][2], pk[p][3]);
-          dst[1] = make_uint4(pk[p][4], pk[p][5], pk[p][6], pk[p][7]);
+          for (int p = 0; p < 3; ++p) {
+            uint4* dst = reinterpret_cast<uint4*>(Es + p * pst + row * lde + k0 + 16 * g);
+            dst[0] = make_uint4(pk[p][0], pk[p][1], pk[p][2], pk[p][3]);
+            dst[1] = make_uint4(pk[p][4], pk[p][5], pk[p][6], pk[p][7]);
+          }
         }
       }
       // group g's feedback into this thread's chunks from two groups on
@@ -384,25 +383,6 @@ __global__ void __launch_bounds__(SUB * LQB_THREADS, 1)
 #pragma unroll
     for (int t = 0; t < 16; ++t) wv[t] = wn[t];
   }
-  }
-  // every group staged: codes and pieces out with coalesced 16-byte stores
-  __syncthreads();
-  const int64_t pst = m * lde;
-  const int nv = w / 8;                                // 16-byte vectors per row and piece
-  for (int e = tid; e < 3 * CROWS * nv; e += CTHREADS) {
-    const int p = e / (CROWS * nv), rr = (e / nv) % CROWS, v = e % nv;
-    const int64_t gr = (int64_t)blockIdx.x * CROWS + rr;
-    if (gr < m)
-      *reinterpret_cast<uint4*>(Es + p * pst + gr * lde + k0 + 8 * v) =
-          *reinterpret_cast<const uint4*>(ps + (p * CROWS + rr) * LQB_PS + 8 * v);
-  }
-  const int nc = w / 16;                               // 16-byte vectors of codes per row
-  for (int e = tid; e < CROWS * nc; e += CTHREADS) {
-    const int rr = e / nc, v = e % nc;
-    const int64_t gr = (int64_t)blockIdx.x * CROWS + rr;
-    if (gr < m)
-      *reinterpret_cast<uint4*>(codes + gr * n + k0 + 16 * v) =
-          *reinterpret_cast<const uint4*>(cs + rr * LQB_CS + 16 * v);
   }
 }
 
