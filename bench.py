@@ -180,9 +180,9 @@ def kernel_work(cfg: LayerConfig, method: str = "ldlq", passes: int = 1):
 KERNEL_TRAFFIC = {
     "k_gemm_split_tc[ldlq]": ("gemm_tc.cuh", "07f39ed17af3", 172632584),
     "k_gemm_split_tc[ldl]": ("gemm_tc.cuh", "07f39ed17af3", 61238127),
-    "k_ldlq_block": ("ldlq.cuh", "e00db76e6414", 44962816),
-    "k_dequant": ("ldlq.cuh", "e00db76e6414", 941438976),
-    "k_row_grid": ("ldlq.cuh", "e00db76e6414", 970614784),
+    "k_ldlq_block": ("ldlq.cuh", "294f51797099", 45038592),
+    "k_dequant": ("ldlq.cuh", "294f51797099", 941438976),
+    "k_row_grid": ("ldlq.cuh", "294f51797099", 970614784),
 }
 TRAFFIC_WORKLOAD = "gate70b"
 
