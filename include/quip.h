@@ -162,7 +162,10 @@ quip_status quip_transform_permutation(const quip_transform* tf, int side, const
  *                upper triangle is unspecified until quip_hessian_finalize.
  *   accumulate : 0 = overwrite, 1 = add to the lower triangle already there
  *                (stream X in token chunks; N may differ per call).
- * N == 0 with accumulate == 0 writes zeros.
+ * N == 0 with accumulate == 0 writes zeros.  Token shards add: GPUs that each
+ * accumulate their own tokens and sum H_acc (one all-reduce) before
+ * quip_hessian_finalize with the total token count all hold the Hessian of
+ * every token.
  */
 quip_status quip_hessian_accumulate(const void* X, int dtype, int64_t N, int64_t n,
                                     int64_t ldx, float* H_acc, int accumulate,

@@ -11,7 +11,7 @@ from __future__ import annotations
 
 import ctypes
 from dataclasses import dataclass
-from typing import Optional
+from typing import Optional, Tuple
 
 import torch
 
@@ -19,7 +19,8 @@ from . import _lib as L
 from ._lib import QuipError, load, status_string  # noqa: F401
 
 __all__ = [
-    "Transform", "quip_hessian_accumulate", "quip_hessian_finalize", "quip_incoherence_forward",
+    "Transform", "quip_hessian_accumulate", "quip_hessian_finalize", "quip_hessian_sharded",
+    "token_range", "allreduce_hessian", "quip_incoherence_forward",
     "quip_incoherence_inverse", "quip_ldl", "quip_ldlq_quantize", "quip_dequantize",
     "quip_nearest_quantize", "quip_diag_order", "quip_permute", "quip_greedy_refine", "METHODS",
     "quip_packed_words", "quip_pack_codes", "quip_qmatvec", "QuantizedLinear",
@@ -163,6 +164,48 @@ def quip_hessian_finalize(H: torch.Tensor, N_total: int, damp: float, stream=Non
     _cuda(H, "H")
     L.check(load().quip_hessian_finalize(_p(H), H.shape[0], N_total, damp, _s(stream)),
             "quip_hessian_finalize")
+
+
+def token_range(N_total: int, world: int, rank: int) -> Tuple[int, int]:
+    """Tokens [t0, t1) of N_total that rank ``rank`` of ``world`` accumulates
+    for a token-sharded Hessian: contiguous, sizes differ by at most one, the
+    ranks together cover each token once (a rank may get none)."""
+    if world < 1 or not 0 <= rank < world or N_total < 0:
+        raise ValueError(f"token_range: N_total={N_total}, world={world}, rank={rank}")
+    q, r = divmod(N_total, world)
+    t0 = rank * q + min(rank, r)
+    return t0, t0 + q + (1 if rank < r else 0)
+
+
+def allreduce_hessian(H_acc: torch.Tensor, group=None, stream=None) -> None:
+    """H_acc <- the sum of every rank's H_acc over ``group``: one all-reduce
+    of the n x n fp32 buffer, ordered on ``stream`` (default: the current
+    stream) for device buffers.  The strict upper triangle, which the
+    accumulation leaves unspecified, is summed too; quip_hessian_finalize
+    never reads it.  Without a process group of two or more ranks it does
+    nothing."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
+        return
+    if H_acc.is_cuda:
+        with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream()):
+            dist.all_reduce(H_acc, op=dist.ReduceOp.SUM, group=group)
+    else:
+        dist.all_reduce(H_acc, op=dist.ReduceOp.SUM, group=group)
+
+
+def quip_hessian_sharded(X_local: torch.Tensor, H: torch.Tensor, N_total: int, damp: float,
+                         group=None, stream=None) -> None:
+    """The proxy Hessian of calibration tokens spread over the ranks of
+    ``group`` (QuIP, adaptive-rounding section: H is the inputs' second
+    moment, a sum over tokens, so token shards add): each rank accumulates
+    X_local^T X_local over its own tokens, one all-reduce sums the partial
+    sums, and every rank finalizes the same H with the total count N_total
+    (the sum of the ranks' token counts) and damping ``damp``.  The LDL and
+    the rest of the layer then run on each rank from that H."""
+    quip_hessian_accumulate(X_local, H, stream=stream)
+    allreduce_hessian(H, group, stream)
+    quip_hessian_finalize(H, N_total, damp, stream=stream)
 
 
 def quip_incoherence_forward(tf: Transform, W: Optional[torch.Tensor], W_t: Optional[torch.Tensor],
