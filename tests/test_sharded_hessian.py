@@ -117,7 +117,10 @@ def test_sharded_hessian_on_the_device():
     Q.quip_hessian_accumulate(X, H0)
     Q.quip_hessian_finalize(H0, N, DAMP)
     assert torch.equal(H1, H0)
-    assert rel_fro(host(H1), ref) <= 1e-5
+    # bf16 products are exact; the tensor cores' fp32 sums lose about one ulp
+    # per 16-token MMA step (the bound of the plain Hessian tests)
+    tol = 2e-5
+    assert rel_fro(host(H1), ref) <= tol
     # two shards of token_range summed on one device (the all-reduce's sum)
     parts = []
     for r in range(2):
@@ -128,4 +131,4 @@ def test_sharded_hessian_on_the_device():
     H2 = parts[0] + parts[1]
     Q.quip_hessian_finalize(H2, N, DAMP)
     torch.cuda.synchronize()
-    assert rel_fro(host(H2), ref) <= 1e-5
+    assert rel_fro(host(H2), ref) <= tol
