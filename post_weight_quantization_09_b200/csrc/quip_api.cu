@@ -1880,6 +1880,26 @@ struct LayerWs {
   size_t H, D, Wt, stage, wstage, Wd, Xd, codes, lo, sc, What, total;
 };
 
+// The events of one layer call, destroyed on every way out of it, error
+// returns included (an event still pending is released once it completes).
+struct CallEvents {
+  std::vector<cudaEvent_t> e;
+  explicit CallEvents(size_t k) : e(k, nullptr) {}
+  ~CallEvents() {
+    for (cudaEvent_t x : e)
+      if (x) cudaEventDestroy(x);
+  }
+  CallEvents(const CallEvents&) = delete;
+  CallEvents& operator=(const CallEvents&) = delete;
+  cudaError_t create() {
+    for (auto& x : e) {
+      const cudaError_t r = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+      if (r != cudaSuccess) return r;
+    }
+    return cudaSuccess;
+  }
+};
+
 quip_status layer_ws(const quip_transform* tf, int64_t N, int w_dtype, int x_dtype, int64_t block, bool host,
                      LayerWs* o) {
   const int64_t m = tf->m, n = tf->n;
@@ -2049,8 +2069,9 @@ quip_status layer_device(quip_transform* tf, uint64_t seed, const void* W, int w
   void* sw2 = ws + L.H + L.D + L.Wt + L.stage;
   cudaStream_t hs = nullptr;
   QCHECK(hpath_stream(&hs));
-  cudaEvent_t ev[3] = {};                             // fork, V drawn, Hessian path done
-  for (auto& e : ev) QCHECK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+  CallEvents evs(3);                                  // fork, V drawn, Hessian path done
+  QCHECK(evs.create());
+  cudaEvent_t* ev = evs.e.data();
   quip_status s = QUIP_OK;
   auto run = [&]() -> quip_status {
     quip_status r;
@@ -2104,7 +2125,6 @@ quip_status layer_device(quip_transform* tf, uint64_t seed, const void* W, int w
     cudaEventRecord(ev[2], hs);
     cudaStreamWaitEvent(st, ev[2], 0);
   }
-  for (auto& e : ev) cudaEventDestroy(e);
   return s;
 }
 }  // namespace
@@ -2164,8 +2184,9 @@ quip_status quip_quantize_layer_host(quip_transform* tf, uint64_t seed, const vo
   const int64_t nblk = (n + LQB_BLOCK_COLS - 1) / LQB_BLOCK_COLS;
   const int every = (int)std::max<int64_t>(1, (nblk + 7) / 8);
   const int ncc = (int)((nblk + every - 1) / every);
-  std::vector<cudaEvent_t> ev(nch + 4 + ncc, nullptr);
-  for (auto& e : ev) QCHECK(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+  CallEvents evs((size_t)(nch + 4 + ncc));
+  QCHECK(evs.create());
+  std::vector<cudaEvent_t>& ev = evs.e;
   cudaEvent_t fork = ev[nch], w_ready = ev[nch + 1], q_done = ev[nch + 2], out_done = ev[nch + 3];
   const cudaEvent_t* code_ev = ev.data() + nch + 4;
   // the copies start after earlier work on the caller's stream, which may
@@ -2202,7 +2223,6 @@ quip_status quip_quantize_layer_host(quip_transform* tf, uint64_t seed, const vo
   // the caller's stream covers every copy: it waits for the copy stream
   QCHECK(cudaEventRecord(out_done, cp));
   QCHECK(cudaStreamWaitEvent(st, out_done, 0));
-  for (auto& e : ev) cudaEventDestroy(e);
   return s;
 }
 

@@ -97,6 +97,30 @@ def test_host_argument_errors(lib):
                             None) == L.QUIP_ERR_ARG
 
 
+def test_layer_calls_reject_a_missing_transform(lib):
+    # a transform cannot be made without a device; a null one is refused
+    # before any argument is read
+    fake = ctypes.c_void_p(0x1000)
+    nb = ctypes.c_size_t(7)
+    assert lib.quip_layer_workspace_size(None, 64, L.QUIP_BF16, L.QUIP_BF16, 32, 0,
+                                         ctypes.byref(nb)) == L.QUIP_ERR_ARG
+    rest = (0, fake, L.QUIP_BF16, 128, fake, L.QUIP_BF16, 64, 128, 2, 32, 0.01, fake, fake, fake,
+            None, fake, 1 << 20, None)
+    assert lib.quip_quantize_layer(None, *rest) == L.QUIP_ERR_ARG
+    assert lib.quip_quantize_layer_host(None, *rest) == L.QUIP_ERR_ARG
+
+
+def test_timing_calls_answer_on_the_host(lib):
+    # no launches recorded: begin, trace and end report nothing, on any host
+    assert lib.quip_timing_begin() == L.QUIP_OK
+    n = ctypes.c_int(-1)
+    assert lib.quip_timing_trace(None, None, None, None, 0, ctypes.byref(n)) == L.QUIP_OK
+    assert n.value == 0
+    n.value = -1
+    assert lib.quip_timing_end(None, None, None, 0, ctypes.byref(n)) == L.QUIP_OK
+    assert n.value == 0
+
+
 def test_workspace_sizes(lib):
     nb = ctypes.c_size_t()
     assert lib.quip_workspace_size(L.QUIP_OP_LDLQ, None, 64, 128, 32, ctypes.byref(nb)) == 0
