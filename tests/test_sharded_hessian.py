@@ -117,9 +117,9 @@ def test_sharded_hessian_on_the_device():
     Q.quip_hessian_accumulate(X, H0)
     Q.quip_hessian_finalize(H0, N, DAMP)
     assert torch.equal(H1, H0)
-    # bf16 products are exact; the tensor cores' fp32 sums lose about one ulp
-    # per 16-token MMA step (the bound of the plain Hessian tests)
-    tol = 2e-5
+    # the bound of the streamed Hessian tests; one token of 1001 left out or
+    # counted twice moves H by about 1e-3
+    tol = 1e-4
     assert rel_fro(host(H1), ref) <= tol
     # two shards of token_range summed on one device (the all-reduce's sum)
     parts = []
