@@ -421,7 +421,8 @@ quip_status quip_workspace_size(int op, const quip_transform* tf, int64_t m, int
  *   W        : device, m x n, w_dtype QUIP_F32 or QUIP_BF16, row stride ldw.
  *   X        : device, N x n (N >= 1 tokens), x_dtype QUIP_F32 or QUIP_BF16,
  *              row stride ldx.
- *   bits     : 1 .. 8.  block: 32, 64 or 128 with n % block == 0 and n % 64 == 0.
+ *   bits     : 1 .. 8.  block: 32, 64 or 128 with n % block == 0 and n % 64 == 0;
+ *              a performance hint, as for quip_ldlq_quantize.
  *   damp     : alpha >= 0.
  *   codes    : device m x n uint8.  lo, scale: device m fp32.
  *   W_hat    : device m x n fp32, or NULL to stop after the codes.
